@@ -1,0 +1,772 @@
+// CPU oracle for NVFP4 attention with ThriftAttention-style selective mixed
+// precision.  TEST INFRASTRUCTURE ONLY: tests, the smoke check and the CPU
+// baseline leg of the benchmark may load this library; the product path never
+// does.  It shares no code, header or table with the CUDA path.
+//
+// Plain, slow and sequential on purpose.  Every rounding is an IEEE-754
+// correctly rounded fp32/fp64 operation (built with -ffp-contract=off, no
+// fast-math); fused multiply-adds are written out explicitly with fmaf/fma
+// where the method's reading calls for them.
+//
+// Sources (the web pages this method is taken from):
+//  * "Attn-QAT: 4-Bit Attention With Quantization-Aware Training",
+//    Resumo tecnico section 1: the FP4 (E2M1) element has 15 distinct values.
+//  * "ThriftAttention" (Resumen Tecnico), Metodologia step 1 (block-mean
+//    importance S^_ij = qbar_i . kbar_j, top-k pairs) and step 2 (FP16 path for
+//    the selected pairs, NVFP4 path for the rest, FlashAttention-2 style online
+//    softmax merge, two-level quantisation of the probability blocks), and the
+//    kernel paragraph after it (FP4 blocks first, FP16 helper afterwards).
+//  * "Busca tus Escalas de Punto Flotante por Bloques" (ScaleSearch),
+//    Declaracion del Problema (NVFP4 block scale is E4M3 with mantissa bits),
+//    ScaleSearch "Mecanismo" (max scaling s = round(||x||_inf / 6) and the
+//    bit-offset candidate s(f)), "Estrategia de Busqueda" (f in [-2, 6],
+//    argmin of block MSE), and ScaleSearchAttention (Hadamard rotation of Q
+//    and K; QK^T and PV in NVFP4 with FP32 accumulation).
+//
+// Readings taken where the pages are silent (each is a choice, stated once):
+//  R1  block size 16, FP32 per-tensor scale g = amax/2688 (2688 = 6*448),
+//      g = 1 when the tensor is all zero.
+//  R2  E2M1 and UE4M3 conversions round to nearest, ties to even, saturating.
+//  R3  max scaling: S = UE4M3(amax_b / (6 g)); codes = E2M1(x * (1/(S g))).
+//  R4  ScaleSearch error of candidate f: fp32 sum, in element order, of
+//      (t - q)^2 with fmaf, times S_f^2 in fp64; candidates visited in the
+//      order 0,-2,-1,1,2,3,4,5,6; bytes outside 1..126 skipped; first strict
+//      minimum kept; a block whose max-scaling byte is 0 keeps byte 0.
+//  R5  Hadamard: unnormalised Sylvester transform, butterflies of stride
+//      1,2,4,...,d/2 in fp32, (a,b) -> (a+b, a-b); the 1/d is folded into the
+//      softmax scale.
+//  R6  16-blocks run along the contraction axis: Q,K along d; V along tokens;
+//      P along keys.
+//  R7  P: per row and key tile sigma = rowmax/2688, Phat = P * (2688/rowmax),
+//      NVFP4 with block scale UE4M3(amax/6) and no tensor scale.
+//  R8  block means in fp64 over the unrotated 16-bit inputs; scores by a
+//      sequential fp64 fma; k = ceil(frac * n_valid - 1e-9) per (batch, head)
+//      over the valid pairs; ties go to the lower linear index i*nB + j.
+//  R9  FP16 path: unrotated 16-bit Q, K, V; P rounded to the input dtype;
+//      l accumulates the fp32 probabilities before rounding.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cstdlib>
+#include <vector>
+#include <thread>
+#include <atomic>
+#include <algorithm>
+#include <limits>
+#include <functional>
+
+extern "C" {
+
+// ---------------------------------------------------------------- formats --
+
+// E2M1 magnitudes indexed by the 3-bit magnitude code (Attn-QAT, Resumo
+// tecnico 1: sixteen codes, +0 and -0 coincide, so 15 distinct values).
+static const float kE2M1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+// Nearest E2M1 magnitude by exhaustive comparison; ties go to the even code.
+// Values above 6 saturate to 6.  The sign bit copies the sign of t (so -0.0
+// and tiny negatives give 0x8).
+uint8_t orc_e2m1_encode(float t) {
+  uint8_t sign = std::signbit(t) ? 0x8 : 0x0;
+  double a = std::fabs((double)t);
+  if (std::isnan(t)) return sign | 0x7;  // not produced by the method
+  if (a >= 6.0) return sign | 0x7;       // saturation at the largest value
+  int best = 0;
+  double best_d = std::fabs(a - kE2M1Mag[0]);
+  for (int c = 1; c < 8; ++c) {
+    double dd = std::fabs(a - kE2M1Mag[c]);
+    if (dd < best_d || (dd == best_d && (c % 2) == 0 && (best % 2) == 1)) {
+      best = c;
+      best_d = dd;
+    }
+  }
+  return sign | (uint8_t)best;
+}
+
+float orc_e2m1_decode(uint8_t code) {
+  float m = kE2M1Mag[code & 0x7];
+  return (code & 0x8) ? -m : m;
+}
+
+// UE4M3 (unsigned E4M3FN: 4 exponent bits, bias 7, 3 mantissa bits,
+// subnormals m * 2^-9, 0x7F is NaN, largest finite 448).
+float orc_ue4m3_decode(uint8_t b) {
+  b &= 0x7F;
+  int e = b >> 3, m = b & 7;
+  if (b == 0x7F) return std::numeric_limits<float>::quiet_NaN();
+  if (e == 0) return std::ldexp((float)m, -9);
+  return std::ldexp(1.0f + (float)m / 8.0f, e - 7);
+}
+
+// Nearest of the 127 finite UE4M3 values by exhaustive search, ties to the
+// even byte, saturating at 448.  Negative inputs map to 0 (scales are >= 0).
+uint8_t orc_ue4m3_encode(float v) {
+  if (!(v > 0.0f)) return 0;
+  if (v >= 448.0f) return 0x7E;
+  int best = 0;
+  double best_d = std::fabs((double)v);
+  for (int b = 1; b <= 0x7E; ++b) {
+    double dd = std::fabs((double)v - (double)orc_ue4m3_decode((uint8_t)b));
+    if (dd < best_d || (dd == best_d && (b % 2) == 0 && (best % 2) == 1)) {
+      best = b;
+      best_d = dd;
+    }
+  }
+  return (uint8_t)best;
+}
+
+void orc_e2m1_encode_array(const float* x, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_encode(x[i]);
+}
+void orc_ue4m3_encode_array(const float* x, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_ue4m3_encode(x[i]);
+}
+
+// 16-bit storage types: 0 = IEEE fp16, 1 = bfloat16.  Both widen to fp32
+// exactly.
+float orc_half_to_float(uint16_t h, int dt) {
+  if (dt == 1) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+  }
+  int s = (h >> 15) & 1, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+  float v;
+  if (e == 0) v = std::ldexp((float)m, -24);
+  else if (e == 31) v = m ? std::numeric_limits<float>::quiet_NaN()
+                           : std::numeric_limits<float>::infinity();
+  else v = std::ldexp(1.0f + (float)m / 1024.0f, e - 15);
+  return s ? -v : v;
+}
+
+// Round a double to the 16-bit type (nearest, ties to even, overflow to inf).
+uint16_t orc_double_to_half(double x, int dt);
+
+}  // extern "C"
+
+extern "C" {
+
+// Round to nearest, ties to even, on a grid whose spacing is 2^(e-p) for a
+// value in [2^(e-1), 2^e), floored at the subnormal spacing 2^qmin; then
+// encode.  p = 11, qmin = -24 for fp16; p = 8, qmin = -133 for bfloat16.
+uint16_t orc_double_to_half(double x, int dt) {
+  const int p = dt == 1 ? 8 : 11;
+  const int qmin = dt == 1 ? -133 : -24;
+  const double maxv = dt == 1 ? std::ldexp(255.0 / 128.0, 127) : 65504.0;
+  uint16_t sign = std::signbit(x) ? 0x8000 : 0;
+  double a = std::fabs(x);
+  double r;
+  if (std::isnan(x)) return dt == 1 ? 0x7FC0 : 0x7E00;
+  if (a == 0.0) {
+    r = 0.0;
+  } else {
+    int e;
+    std::frexp(a, &e);  // a in [2^(e-1), 2^e)
+    int qe = std::max(e - p, qmin);
+    double scaled = std::ldexp(a, -qe);  // exact
+    r = std::ldexp(std::nearbyint(scaled), qe);
+  }
+  if (dt == 1) {
+    if (r > maxv) return sign | 0x7F80;
+    float f = (float)r;  // exact: r has at most 8 significant bits
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return sign | (uint16_t)((u >> 16) & 0x7FFF);
+  }
+  if (r > maxv) return sign | 0x7C00;
+  if (r == 0.0) return sign;
+  int e;
+  std::frexp(r, &e);
+  if (e - 1 < -14) {  // subnormal: r = m * 2^-24
+    return sign | (uint16_t)std::ldexp(r, 24);
+  }
+  int ef = e - 1;                              // r in [2^ef, 2^(ef+1))
+  double mant = std::ldexp(r, -ef) - 1.0;      // in [0, 1)
+  return sign | (uint16_t)(((ef + 15) << 10) | (int)std::ldexp(mant, 10));
+}
+
+// Unnormalised Sylvester-Hadamard transform of one row of length d (power of
+// two) in fp32 (ScaleSearchAttention, "Procesamiento de Incoherencia";
+// reading R5).  Butterfly stride h = 1, 2, ..., d/2; (a, b) -> (a+b, a-b) with
+// a at the lower index.
+void orc_fwht_row(float* x, int d) {
+  for (int h = 1; h < d; h *= 2) {
+    for (int i = 0; i < d; i += 2 * h) {
+      for (int j = i; j < i + h; ++j) {
+        float a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+    }
+  }
+}
+
+// Load a [rows, cols] 16-bit matrix as fp32, optionally rotating every row.
+static std::vector<float> load_rows(const uint16_t* x, int dt, int64_t rows,
+                                    int64_t cols, int hadamard) {
+  std::vector<float> v((size_t)(rows * cols));
+  for (int64_t i = 0; i < rows * cols; ++i) v[(size_t)i] = orc_half_to_float(x[i], dt);
+  if (hadamard)
+    for (int64_t r = 0; r < rows; ++r) orc_fwht_row(&v[(size_t)(r * cols)], (int)cols);
+  return v;
+}
+
+// Per-tensor FP32 scale g = amax / 2688 over all values (reading R1).
+static float tensor_scale_of(const std::vector<float>& v) {
+  float amax = 0.0f;
+  for (float f : v) amax = std::max(amax, std::fabs(f));
+  if (amax == 0.0f) return 1.0f;
+  return amax / 2688.0f;
+}
+
+float orc_tensor_scale(const uint16_t* x, int dt, int64_t rows, int64_t cols, int hadamard) {
+  return tensor_scale_of(load_rows(x, dt, rows, cols, hadamard));
+}
+
+// ScaleSearch error of one candidate scale byte for a block of 16 values x
+// under tensor scale g (reading R4): t = x * (1/(S g)), q = E2M1 grid value
+// of t, err = (sum over the block, in order, of (t-q)^2 with fmaf) * S^2.
+double orc_block_err(const float* x, float g, uint8_t S) {
+  float dec = orc_ue4m3_decode(S) * g;
+  float r = 1.0f / dec;
+  float acc = 0.0f;
+  for (int e = 0; e < 16; ++e) {
+    float t = x[e] * r;
+    float q = orc_e2m1_decode(orc_e2m1_encode(t));
+    float er = t - q;
+    acc = std::fmaf(er, er, acc);
+  }
+  double s = (double)orc_ue4m3_decode(S);
+  return (double)acc * (s * s);
+}
+
+// Quantise one 16-element block (readings R3, R4).  Writes 8 packed bytes
+// (element 2c in the low nibble, 2c+1 in the high nibble), the scale byte and
+// the chosen offset f.
+//
+// Max scaling (ScaleSearch "Mecanismo"): the block absmax is mapped to the
+// top FP4 value 6.  ScaleSearch ("Estrategia de Busqueda"): the candidate
+// bytes S0+f for f in [-2, 6], reinterpreted as UE4M3, and the one with the
+// smallest block error wins.
+void orc_quant_block(const float* x, float g, int use_ss, uint8_t* codes8,
+                     uint8_t* scale, int* f_out) {
+  float amax = 0.0f;
+  for (int e = 0; e < 16; ++e) amax = std::max(amax, std::fabs(x[e]));
+  float s_real = amax / (6.0f * g);
+  uint8_t S = orc_ue4m3_encode(s_real);
+  int best_f = 0;
+  if (use_ss && S != 0) {
+    static const int order[9] = {0, -2, -1, 1, 2, 3, 4, 5, 6};
+    double best = 0.0;
+    bool have = false;
+    for (int oi = 0; oi < 9; ++oi) {
+      int b = (int)S + order[oi];
+      if (b < 1 || b > 126) continue;
+      double err = orc_block_err(x, g, (uint8_t)b);
+      if (!have || err < best) {
+        best = err;
+        best_f = order[oi];
+        have = true;
+      }
+    }
+    S = (uint8_t)((int)S + best_f);
+  }
+  *scale = S;
+  if (f_out) *f_out = best_f;
+  uint8_t c[16];
+  if (S == 0) {
+    for (int e = 0; e < 16; ++e) c[e] = 0;
+  } else {
+    float dec = orc_ue4m3_decode(S) * g;
+    float r = 1.0f / dec;
+    for (int e = 0; e < 16; ++e) c[e] = orc_e2m1_encode(x[e] * r);
+  }
+  for (int i = 0; i < 8; ++i) codes8[i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+}
+
+// Quantise a [rows, cols] matrix with 16-blocks along cols.
+// codes [rows, cols/2], scales [rows, cols/16].  g is read when
+// tensor_scale_given != 0, else computed and written.  f_out (optional)
+// receives the chosen offsets [rows, cols/16].  Returns 0, or -1 on bad sizes.
+int orc_nvfp4_quantize(const uint16_t* x, int dt, int64_t rows, int64_t cols,
+                       int use_ss, int hadamard, int tensor_scale_given,
+                       uint8_t* codes, uint8_t* scales, float* g, int8_t* f_out) {
+  if (rows < 0 || cols <= 0 || cols % 16) return -1;
+  if (hadamard && (cols & (cols - 1))) return -1;
+  std::vector<float> v = load_rows(x, dt, rows, cols, hadamard);
+  if (!tensor_scale_given) *g = tensor_scale_of(v);
+  const float gg = *g;
+  const int64_t nb = cols / 16;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nb; ++b) {
+      int f;
+      orc_quant_block(&v[(size_t)(r * cols + b * 16)], gg, use_ss,
+                      &codes[r * (cols / 2) + b * 8], &scales[r * nb + b], &f);
+      if (f_out) f_out[r * nb + b] = (int8_t)f;
+    }
+  return 0;
+}
+
+// Same with 16-blocks along rows (the token axis of V): the matrix is read
+// transposed.  codes [cols, rows/2], scales [cols, rows/16].
+int orc_nvfp4_quantize_colblocks(const uint16_t* x, int dt, int64_t rows, int64_t cols,
+                                 int use_ss, int tensor_scale_given,
+                                 uint8_t* codes, uint8_t* scales, float* g, int8_t* f_out) {
+  if (rows <= 0 || cols <= 0 || rows % 16) return -1;
+  std::vector<float> v = load_rows(x, dt, rows, cols, 0);
+  if (!tensor_scale_given) *g = tensor_scale_of(v);
+  const float gg = *g;
+  const int64_t nb = rows / 16;
+  float blk[16];
+  for (int64_t c = 0; c < cols; ++c)
+    for (int64_t b = 0; b < nb; ++b) {
+      for (int e = 0; e < 16; ++e) blk[e] = v[(size_t)((b * 16 + e) * cols + c)];
+      int f;
+      orc_quant_block(blk, gg, use_ss, &codes[c * (rows / 2) + b * 8], &scales[c * nb + b], &f);
+      if (f_out) f_out[c * nb + b] = (int8_t)f;
+    }
+  return 0;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+// ------------------------------------------------------ block selection --
+//
+// ThriftAttention, Metodologia step 1: the sequence is cut into blocks, each
+// block pair (i, j) is scored by the dot product of the block-mean query and
+// key vectors, and the top-k pairs are computed in FP16 (reading R8).
+
+struct SeqView {
+  int64_t start;  // first token of the sequence in the packed token axis
+  int len;        // tokens
+};
+
+// Block means of one head of one sequence: x is [tokens, heads, d] packed,
+// blocks of blk tokens from the sequence start (the last may be partial).
+static void block_means(const uint16_t* x, int dt, int64_t tok_stride, int64_t head_off,
+                        const SeqView& s, int d, int blk, std::vector<double>& out) {
+  int nb = (s.len + blk - 1) / blk;
+  out.assign((size_t)nb * d, 0.0);
+  for (int b = 0; b < nb; ++b) {
+    int t0 = b * blk, t1 = std::min(s.len, t0 + blk);
+    for (int c = 0; c < d; ++c) {
+      double sum = 0.0;
+      for (int t = t0; t < t1; ++t)
+        sum += (double)orc_half_to_float(x[(s.start + t) * tok_stride + head_off + c], dt);
+      out[(size_t)b * d + c] = sum / (double)(t1 - t0);
+    }
+  }
+}
+
+static double pair_score(const double* qm, const double* km, int d) {
+  double acc = 0.0;
+  for (int c = 0; c < d; ++c) acc = std::fma(qm[c], km[c], acc);
+  return acc;
+}
+
+int64_t orc_topk_count(float frac, int64_t n_valid) {
+  double kk = std::ceil((double)frac * (double)n_valid - 1e-9);
+  if (kk < 0) kk = 0;
+  if (kk > (double)n_valid) kk = (double)n_valid;
+  return (int64_t)kk;
+}
+
+// Selection for one (sequence, head): mask [nB, nB] (1 = FP16 pair).
+static void select_one(const uint16_t* q, const uint16_t* k, int dt, int H, int Hkv,
+                       int h, const SeqView& s, int d, int blk, int causal, float frac,
+                       uint8_t* mask, double* scores) {
+  int nb = (s.len + blk - 1) / blk;
+  int hk = h / (H / Hkv);
+  std::vector<double> qm, km;
+  block_means(q, dt, (int64_t)H * d, (int64_t)h * d, s, d, blk, qm);
+  block_means(k, dt, (int64_t)Hkv * d, (int64_t)hk * d, s, d, blk, km);
+  std::vector<std::pair<double, int64_t>> cand;
+  for (int i = 0; i < nb; ++i)
+    for (int j = 0; j < nb; ++j) {
+      int64_t lin = (int64_t)i * nb + j;
+      mask[lin] = 0;
+      double sc = pair_score(&qm[(size_t)i * d], &km[(size_t)j * d], d);
+      if (scores) scores[lin] = sc;
+      if (causal && j > i) continue;
+      cand.push_back({sc, lin});
+    }
+  int64_t kk = orc_topk_count(frac, (int64_t)cand.size());
+  // Full sort: larger score first, then lower linear index.
+  std::sort(cand.begin(), cand.end(), [](const std::pair<double, int64_t>& a,
+                                         const std::pair<double, int64_t>& b) {
+    if (a.first != b.first) return a.first > b.first;
+    return a.second < b.second;
+  });
+  for (int64_t t = 0; t < kk; ++t) mask[cand[(size_t)t].second] = 1;
+}
+
+// q [B, N, H, d], k [B, N, Hkv, d] 16-bit; mask out uint8 [B, H, nB, nB];
+// scores (optional) fp64 [B, H, nB, nB] (every pair, valid or not).
+int orc_block_mean_topk(const uint16_t* q, const uint16_t* k, int dt, int B, int H, int Hkv,
+                        int N, int d, int blk, int causal, float frac, uint8_t* mask,
+                        double* scores) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || d <= 0 || blk <= 0) return -1;
+  int nb = (N + blk - 1) / blk;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      SeqView s{0, N};
+      int64_t off = ((int64_t)b * H + h) * nb * nb;
+      select_one(q + (int64_t)b * N * H * d, k + (int64_t)b * N * Hkv * d, dt, H, Hkv, h, s, d,
+                 blk, causal, frac, mask + off, scores ? scores + off : nullptr);
+    }
+  return 0;
+}
+
+// Varlen: q [total, H, d], k [total, Hkv, d]; cu_seqlens [nseq+1].  Masks of
+// sequence s are stored at mask_off(s) = H * sum_{s'<s} nB_{s'}^2, laid out
+// [H, nB_s, nB_s].
+int orc_block_mean_topk_varlen(const uint16_t* q, const uint16_t* k, int dt, int H, int Hkv,
+                               const int32_t* cu, int nseq, int d, int blk, int causal,
+                               float frac, uint8_t* mask) {
+  int64_t off = 0;
+  for (int sq = 0; sq < nseq; ++sq) {
+    SeqView s{cu[sq], cu[sq + 1] - cu[sq]};
+    int nb = (s.len + blk - 1) / blk;
+    for (int h = 0; h < H; ++h) {
+      select_one(q, k, dt, H, Hkv, h, s, d, blk, causal, frac, mask + off, nullptr);
+      off += (int64_t)nb * nb;
+    }
+  }
+  return 0;
+}
+
+// ------------------------------------------------------------ threading --
+
+static void parallel_for(int64_t n, int nthreads, const std::function<void(int64_t)>& fn) {
+  if (nthreads <= 1 || n <= 1) {
+    for (int64_t i = 0; i < n; ++i) fn(i);
+    return;
+  }
+  std::atomic<int64_t> next(0);
+  std::vector<std::thread> pool;
+  int nt = (int)std::min<int64_t>(nthreads, n);
+  for (int t = 0; t < nt; ++t)
+    pool.emplace_back([&]() {
+      for (;;) {
+        int64_t i = next.fetch_add(1);
+        if (i >= n) break;
+        fn(i);
+      }
+    });
+  for (auto& th : pool) th.join();
+}
+
+// Threaded quantiser of a [rows, cols] matrix (blocks along cols), writing
+// one unpacked 4-bit code per byte and one scale byte per block, for the
+// attention emulation below.  Same arithmetic as orc_nvfp4_quantize.
+static float quantize_rows_unpacked(const uint16_t* x, int dt, int64_t rows, int cols,
+                                    int use_ss, int hadamard, int nthreads,
+                                    std::vector<uint8_t>& codes, std::vector<uint8_t>& scales) {
+  const int64_t chunk = 4096;
+  const int64_t nchunks = (rows + chunk - 1) / chunk;
+  std::vector<float> part(nchunks, 0.0f);
+  parallel_for(nchunks, nthreads, [&](int64_t c) {
+    std::vector<float> row(cols);
+    float amax = 0.0f;
+    for (int64_t r = c * chunk; r < std::min(rows, (c + 1) * chunk); ++r) {
+      for (int e = 0; e < cols; ++e) row[e] = orc_half_to_float(x[r * cols + e], dt);
+      if (hadamard) orc_fwht_row(row.data(), cols);
+      for (int e = 0; e < cols; ++e) amax = std::max(amax, std::fabs(row[e]));
+    }
+    part[c] = amax;
+  });
+  float amax = 0.0f;
+  for (float a : part) amax = std::max(amax, a);
+  const float g = amax == 0.0f ? 1.0f : amax / 2688.0f;
+  codes.assign((size_t)(rows * cols), 0);
+  scales.assign((size_t)(rows * (cols / 16)), 0);
+  parallel_for(nchunks, nthreads, [&](int64_t c) {
+    std::vector<float> row(cols);
+    uint8_t packed[8];
+    for (int64_t r = c * chunk; r < std::min(rows, (c + 1) * chunk); ++r) {
+      for (int e = 0; e < cols; ++e) row[e] = orc_half_to_float(x[r * cols + e], dt);
+      if (hadamard) orc_fwht_row(row.data(), cols);
+      for (int b = 0; b < cols / 16; ++b) {
+        orc_quant_block(&row[b * 16], g, use_ss, packed, &scales[(size_t)(r * (cols / 16) + b)],
+                        nullptr);
+        for (int e = 0; e < 8; ++e) {
+          codes[(size_t)(r * cols + b * 16 + 2 * e)] = packed[e] & 0xF;
+          codes[(size_t)(r * cols + b * 16 + 2 * e + 1)] = packed[e] >> 4;
+        }
+      }
+    }
+  });
+  return g;
+}
+
+// ------------------------------------------------- attention emulation --
+//
+// ThriftAttention, Metodologia step 2 and the kernel paragraph after it:
+// for every query block, the key blocks that were not selected are visited
+// first on the NVFP4 path, then the selected ones on the FP16 path, all
+// merged by one FlashAttention-2 online softmax (base-2 exponent, running
+// max m, running sum l).  NVFP4 products follow ScaleSearchAttention
+// ("Ejecucion Nativa NVFP4": QK^T and PV on block-scaled FP4 values).
+// Arithmetic here is fp64 on exactly dequantised values; the probability
+// tile is rounded to fp32 before it is quantised (reading R7).
+
+struct AttnCtx {
+  int dt, H, Hkv, d, blk, causal, use_had;
+  const int32_t* cu;
+  int nseq;
+  int64_t total, ptot;
+  const uint16_t *q, *k, *v;
+  std::vector<uint8_t> qc, qs, kc, ks, vc, vs;  // unpacked codes, scale bytes
+  float gq, gk, gv;
+  std::vector<int64_t> pstart;   // padded token start of each sequence (V)
+  std::vector<int64_t> moff;     // mask offset of each sequence
+  const uint8_t* mask;
+};
+
+static inline double deq(uint8_t code, uint8_t sc, float g) {
+  return (double)orc_e2m1_decode(code) * (double)orc_ue4m3_decode(sc) * (double)g;
+}
+
+// One query block i of sequence s, head h.  Writes out rows and lse.
+static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, float* lse) {
+  const int d = C.d, blk = C.blk, H = C.H, Hkv = C.Hkv;
+  const int64_t st = C.cu[s];
+  const int len = C.cu[s + 1] - C.cu[s];
+  const int nb = (len + blk - 1) / blk;
+  const int hk = h / (H / Hkv);
+  const int r0 = i * blk, r1 = std::min(len, r0 + blk), nr = r1 - r0;
+  const double l2e = 1.4426950408889634;  // log2(e)
+  double s4 = l2e / std::sqrt((double)d);
+  if (C.use_had) s4 /= (double)d;
+  const double s16 = l2e / std::sqrt((double)d);
+  const uint8_t* mk = C.mask + C.moff[s] + (int64_t)h * nb * nb + (int64_t)i * nb;
+
+  std::vector<int> order;
+  for (int pass = 0; pass < 2; ++pass)
+    for (int j = 0; j < nb; ++j) {
+      if (C.causal && j > i) continue;
+      if ((mk[j] != 0) == (pass == 1)) order.push_back(pass == 0 ? j : -1 - j);
+    }
+
+  // Per-row query vectors: dequantised NVFP4 and the original 16-bit values.
+  std::vector<double> qh((size_t)nr * d), q16((size_t)nr * d);
+  for (int r = 0; r < nr; ++r)
+    for (int c = 0; c < d; ++c) {
+      int64_t e = ((st + r0 + r) * H + h) * d + c;
+      qh[(size_t)r * d + c] = deq(C.qc[(size_t)e], C.qs[(size_t)(e / 16)], C.gq);
+      q16[(size_t)r * d + c] = orc_half_to_float(C.q[e], C.dt);
+    }
+  std::vector<double> m(nr, -INFINITY), l(nr, 0.0), O((size_t)nr * d, 0.0);
+  std::vector<double> kt((size_t)blk * d), vt((size_t)blk * d), S(blk);
+  std::vector<float> Pt(blk), Ph(blk);
+  std::vector<double> Pq(blk);
+
+  for (int code : order) {
+    const bool fp4 = code >= 0;
+    const int j = fp4 ? code : -1 - code;
+    const int k0 = j * blk, k1 = std::min(len, k0 + blk), nk = k1 - k0;
+    for (int t = 0; t < nk; ++t)
+      for (int c = 0; c < d; ++c) {
+        int64_t e = ((st + k0 + t) * Hkv + hk) * d + c;
+        if (fp4) {
+          kt[(size_t)t * d + c] = deq(C.kc[(size_t)e], C.ks[(size_t)(e / 16)], C.gk);
+          int64_t ve = ((int64_t)hk * d + c) * C.ptot + C.pstart[s] + k0 + t;
+          vt[(size_t)t * d + c] = deq(C.vc[(size_t)ve], C.vs[(size_t)(ve / 16)], C.gv);
+        } else {
+          kt[(size_t)t * d + c] = orc_half_to_float(C.k[e], C.dt);
+          vt[(size_t)t * d + c] = orc_half_to_float(C.v[e], C.dt);
+        }
+      }
+    for (int r = 0; r < nr; ++r) {
+      const int row = r0 + r;
+      const double* qv = fp4 ? &qh[(size_t)r * d] : &q16[(size_t)r * d];
+      double mt = -INFINITY;
+      for (int t = 0; t < nk; ++t) {
+        if (C.causal && k0 + t > row) {
+          S[t] = -INFINITY;
+          continue;
+        }
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qv[c] * kt[(size_t)t * d + c];
+        S[t] = acc * (fp4 ? s4 : s16);
+        mt = std::max(mt, S[t]);
+      }
+      if (mt == -INFINITY) continue;
+      const double mn = std::max(m[r], mt);
+      const double alpha = std::exp2(m[r] - mn);  // 0 when m is still -inf
+      l[r] *= alpha;
+      for (int c = 0; c < d; ++c) O[(size_t)r * d + c] *= alpha;
+      float rowmax = 0.0f;
+      for (int t = 0; t < nk; ++t) {
+        Pt[t] = S[t] == -INFINITY ? 0.0f : (float)std::exp2(S[t] - mn);
+        l[r] += (double)Pt[t];
+        rowmax = std::max(rowmax, Pt[t]);
+      }
+      if (fp4) {
+        // Two-level quantisation of the probability row tile (reading R7).
+        if (rowmax == 0.0f) { m[r] = mn; continue; }
+        const float inv = 2688.0f / rowmax;
+        const float sigma = rowmax / 2688.0f;
+        for (int t = 0; t < blk; ++t) Ph[t] = t < nk ? Pt[t] * inv : 0.0f;
+        for (int b0 = 0; b0 < blk; b0 += 16) {
+          float amax = 0.0f;
+          for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
+          uint8_t sp = orc_ue4m3_encode(amax / 6.0f);
+          float dec = orc_ue4m3_decode(sp);
+          float rr = 1.0f / dec;
+          for (int e = 0; e < 16; ++e)
+            Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr)) *
+                                             (double)dec;
+        }
+        for (int c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int t = 0; t < nk; ++t) acc += Pq[t] * vt[(size_t)t * d + c];
+          O[(size_t)r * d + c] += (double)sigma * acc;
+        }
+      } else {
+        for (int c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int t = 0; t < nk; ++t)
+            acc += (double)orc_half_to_float(orc_double_to_half((double)Pt[t], C.dt), C.dt) *
+                   vt[(size_t)t * d + c];
+          O[(size_t)r * d + c] += acc;
+        }
+      }
+      m[r] = mn;
+    }
+  }
+  const double ln2 = 0.6931471805599453;
+  for (int r = 0; r < nr; ++r) {
+    const int64_t tok = st + r0 + r;
+    for (int c = 0; c < d; ++c) {
+      double o = l[r] > 0.0 ? O[(size_t)r * d + c] / l[r] : 0.0;
+      out[(tok * H + h) * d + c] = orc_double_to_half(o, C.dt);
+    }
+    lse[(int64_t)h * C.total + tok] = l[r] > 0.0 ? (float)(m[r] * ln2 + std::log(l[r])) : -INFINITY;
+  }
+}
+
+// Full emulation over packed sequences.  q [total, H, d], k/v [total, Hkv, d]
+// 16-bit; cu [nseq+1].  out 16-bit [total, H, d]; lse fp32 [H, total].
+// mask_io: if mask_given, the selection [per sequence: H, nB, nB] is read from
+// it, else it is computed (reading R8) and written there.  units: optional
+// list of (sequence, head, query block) triples to compute (n_units = 0 means
+// every unit); rows of other units are left untouched.  gs_out (optional)
+// receives g_Q, g_K, g_V.
+int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                    int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
+                    float frac, int use_ss, int use_had, uint8_t* mask_io, int mask_given,
+                    const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
+                    float* lse, float* gs_out) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
+  if (use_had && (d & (d - 1))) return -1;
+  AttnCtx C;
+  C.dt = dt; C.H = H; C.Hkv = Hkv; C.d = d; C.blk = blk; C.causal = causal; C.use_had = use_had;
+  C.cu = cu; C.nseq = nseq; C.q = q; C.k = k; C.v = v;
+  C.total = cu[nseq];
+  C.pstart.resize(nseq + 1);
+  C.moff.resize(nseq + 1);
+  C.pstart[0] = 0;
+  C.moff[0] = 0;
+  for (int s = 0; s < nseq; ++s) {
+    int len = cu[s + 1] - cu[s];
+    if (len <= 0) return -1;
+    int nb = (len + blk - 1) / blk;
+    C.pstart[s + 1] = C.pstart[s] + (int64_t)nb * blk;
+    C.moff[s + 1] = C.moff[s] + (int64_t)H * nb * nb;
+  }
+  C.ptot = C.pstart[nseq];
+  C.gq = quantize_rows_unpacked(q, dt, C.total * H, d, use_ss, use_had, nthreads, C.qc, C.qs);
+  C.gk = quantize_rows_unpacked(k, dt, C.total * Hkv, d, use_ss, use_had, nthreads, C.kc, C.ks);
+  // V: 16-blocks along tokens, every sequence zero-padded to a whole number of
+  // key blocks (reading R6).  The tensor scale covers the real tokens only.
+  {
+    float amax = 0.0f;
+    for (int64_t e = 0; e < C.total * Hkv * d; ++e) amax = std::max(amax, std::fabs(orc_half_to_float(v[e], dt)));
+    C.gv = amax == 0.0f ? 1.0f : amax / 2688.0f;
+    C.vc.assign((size_t)(Hkv * d * C.ptot), 0);
+    C.vs.assign((size_t)(Hkv * d * C.ptot / 16), 0);
+    parallel_for((int64_t)Hkv * d, nthreads, [&](int64_t hc) {
+      const int64_t hk = hc / d, c = hc % d;
+      float col[16];
+      uint8_t packed[8];
+      for (int s = 0; s < nseq; ++s) {
+        const int len = cu[s + 1] - cu[s];
+        for (int64_t t0 = 0; t0 < C.pstart[s + 1] - C.pstart[s]; t0 += 16) {
+          for (int e = 0; e < 16; ++e)
+            col[e] = t0 + e < len ? orc_half_to_float(v[((cu[s] + t0 + e) * Hkv + hk) * d + c], dt) : 0.0f;
+          const int64_t base = hc * C.ptot + C.pstart[s] + t0;
+          orc_quant_block(col, C.gv, use_ss, packed, &C.vs[(size_t)(base / 16)], nullptr);
+          for (int e = 0; e < 8; ++e) {
+            C.vc[(size_t)(base + 2 * e)] = packed[e] & 0xF;
+            C.vc[(size_t)(base + 2 * e + 1)] = packed[e] >> 4;
+          }
+        }
+      }
+    });
+  }
+  if (gs_out) { gs_out[0] = C.gq; gs_out[1] = C.gk; gs_out[2] = C.gv; }
+  if (!mask_given)
+    orc_block_mean_topk_varlen(q, k, dt, H, Hkv, cu, nseq, d, blk, causal, frac, mask_io);
+  C.mask = mask_io;
+  std::vector<int32_t> all;
+  if (n_units == 0) {
+    for (int s = 0; s < nseq; ++s) {
+      int nb = (cu[s + 1] - cu[s] + blk - 1) / blk;
+      for (int h = 0; h < H; ++h)
+        for (int i = 0; i < nb; ++i) { all.push_back(s); all.push_back(h); all.push_back(i); }
+    }
+    units = all.data();
+    n_units = (int64_t)all.size() / 3;
+  }
+  parallel_for(n_units, nthreads, [&](int64_t u) {
+    attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse);
+  });
+  return 0;
+}
+
+// Unquantised attention in fp64 (softmax(Q K^T / sqrt(d)) V) over packed
+// sequences; out fp64 [total, H, d], lse fp64 [H, total] (natural log).
+// rows (optional): list of (token, head) pairs to compute; n_rows = 0 = all.
+int orc_attn_fp64(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                  int Hkv, const int32_t* cu, int nseq, int d, int causal,
+                  const int64_t* rows, int64_t n_rows, int nthreads, double* out, double* lse) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv) return -1;
+  const int64_t total = cu[nseq];
+  std::vector<int32_t> seq_of((size_t)total);
+  for (int s = 0; s < nseq; ++s)
+    for (int64_t t = cu[s]; t < cu[s + 1]; ++t) seq_of[(size_t)t] = s;
+  const int64_t n = n_rows ? n_rows : total * H;
+  parallel_for(n, nthreads, [&](int64_t u) {
+    int64_t tok = n_rows ? rows[2 * u] : u / H;
+    int h = n_rows ? (int)rows[2 * u + 1] : (int)(u % H);
+    int s = seq_of[(size_t)tok];
+    int hk = h / (H / Hkv);
+    int64_t k0 = cu[s], k1 = causal ? tok + 1 : cu[s + 1];
+    std::vector<double> sc((size_t)(k1 - k0));
+    double mx = -INFINITY;
+    for (int64_t t = k0; t < k1; ++t) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c)
+        acc += (double)orc_half_to_float(q[(tok * H + h) * d + c], dt) *
+               (double)orc_half_to_float(k[(t * Hkv + hk) * d + c], dt);
+      sc[(size_t)(t - k0)] = acc / std::sqrt((double)d);
+      mx = std::max(mx, sc[(size_t)(t - k0)]);
+    }
+    double den = 0.0;
+    for (auto& x : sc) { x = std::exp(x - mx); den += x; }
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int64_t t = k0; t < k1; ++t)
+        acc += sc[(size_t)(t - k0)] * (double)orc_half_to_float(v[(t * Hkv + hk) * d + c], dt);
+      out[(tok * H + h) * d + c] = acc / den;
+    }
+    lse[(int64_t)h * total + tok] = mx + std::log(den);
+  });
+  return 0;
+}
+
+}  // extern "C"
