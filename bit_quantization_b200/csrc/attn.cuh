@@ -1,0 +1,465 @@
+// Mixed NVFP4 / FP16 attention forward (one CTA per 128 query rows of one
+// head of one sequence).
+//
+// ThriftAttention, Metodologia step 2 and the kernel paragraph after it:
+// the key tiles whose block pair was not selected are visited first on the
+// NVFP4 path, then the selected ones on the FP16 path; a CTA with no selected
+// pair never loads its 16-bit Q tile.  Both paths feed one online softmax
+// (FlashAttention-2 style, base-2, running max m and sum l).  The NVFP4 path
+// follows ScaleSearchAttention's native execution: QK^T and PV as
+// block-scaled E2M1 MMAs with UE4M3 scales and fp32 accumulation; P is
+// quantised in two levels (per row and key tile an fp32 factor rowmax/2688,
+// then NVFP4 16-key blocks).
+//
+// Roles (192 threads):
+//   warps 0-3  softmax + output: thread r owns query row r (TMEM lane r);
+//   warp 4     producer: bulk copies of the pre-quantised tile images;
+//   warp 5     tensor-memory owner and MMA issuer (one elected lane).
+// Tensor memory (512 columns): S double buffer [2][BLK], PV [D], then the
+// scale factors of Q, K (x2), P (x2) and V (x2).
+// Every wait is bounded; a wait that gives up sets the device status word
+// and the CTA drains and exits.
+#pragma once
+#include "quant_kernels.cuh"
+
+namespace thrift {
+
+struct AttnParams {
+  const uint8_t* q4;
+  const uint8_t* k4;
+  const uint8_t* v4;
+  const uint8_t* q16;
+  const uint8_t* k16;
+  const uint8_t* v16;
+  const uint8_t* mask;     // [nseq, H, nB, nB], 1 = FP16 pair
+  const uint32_t* amax;    // absmax bit patterns of (rotated) Q, K and of V
+  uint16_t* out;           // [total, H, D]
+  float* lse;
+  SeqInfo seqs;
+  int nseq, H, Hkv, nB, nTq, causal, lse_varlen;
+  int64_t total;
+  float scale4;            // log2(e)/sqrt(d), divided by d with the rotation
+  float scale16;           // log2(e)/sqrt(d)
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D, int BLK>
+struct AttnLayout {
+  static constexpr uint32_t align(uint32_t x) { return (x + 1023u) & ~1023u; }
+  static constexpr uint32_t QT4 = fp4_tile_bytes(128, D);
+  static constexpr uint32_t Q16B = f16_tile_bytes(128, D);
+  static constexpr uint32_t KT4 = fp4_tile_bytes(BLK, D);
+  static constexpr uint32_t VT4 = fp4_tile_bytes(D, BLK);
+  static constexpr uint32_t KT16 = f16_tile_bytes(BLK, D);
+  static constexpr uint32_t VT16 = f16_tile_bytes(D, BLK);
+  static constexpr uint32_t PT4 = fp4_tile_bytes(128, BLK);
+  static constexpr uint32_t P16B = f16_tile_bytes(128, BLK);
+  static constexpr uint32_t V4_OFF = align(KT4);
+  static constexpr uint32_t V16_OFF = align(KT16);
+  static constexpr uint32_t STG = align(V4_OFF + VT4) > align(V16_OFF + VT16)
+                                      ? align(V4_OFF + VT4)
+                                      : align(V16_OFF + VT16);
+  static constexpr uint32_t OFF_Q4 = 0;
+  static constexpr uint32_t OFF_Q16 = OFF_Q4 + align(QT4);
+  static constexpr uint32_t OFF_STG = OFF_Q16 + align(Q16B);
+  static constexpr uint32_t PT4A = align(PT4);  // one P slot
+  static constexpr uint32_t OFF_P4 = OFF_STG + 2 * STG;
+  static constexpr uint32_t OFF_P16 = OFF_P4 + 2 * PT4A;
+  static constexpr uint32_t OFF_LIST = OFF_P16 + align(P16B);
+  static constexpr uint32_t MAX_TILES = 1024;
+  static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
+  static constexpr uint32_t BYTES = OFF_BAR + 256;
+  static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
+  // tensor-memory columns
+  static constexpr uint32_t T_S = 0;
+  static constexpr uint32_t T_PV = 2 * BLK;
+  static constexpr uint32_t T_QSF = T_PV + D;
+  static constexpr uint32_t T_KSF = T_QSF + (D / 64) * 4;
+  static constexpr uint32_t T_PSF = T_KSF + 2 * (D / 64) * 4;
+  static constexpr uint32_t T_VSF = T_PSF + 2 * (BLK / 64) * 4;
+  static constexpr uint32_t T_END = T_VSF + 2 * (BLK / 64) * 4;
+  static_assert(T_END <= 512, "tensor memory budget");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+// Barrier slots inside the barrier area.
+enum : int {
+  B_Q4 = 0, B_Q16 = 1, B_KVF = 2 /* 2,3 */, B_KVE = 4 /* 4,5 */, B_SF = 6 /* 6,7 */,
+  B_SE = 8 /* 8,9 */, B_PF = 10 /* 10,11 */, B_OF = 12, B_OE = 13, B_DONE = 14, B_N = 15
+};
+
+// Waits with every lane of the warp; the result is uniform across the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int DT, int D, int BLK>
+__global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
+  using L = AttnLayout<D, BLK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint16_t* s_list = reinterpret_cast<uint16_t*>(sm + L::OFF_LIST);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::OFF_BAR + 8 * B_N);
+  int* s_n = reinterpret_cast<int*>(sm + L::OFF_BAR + 8 * B_N + 4);
+  int* s_n4 = s_n + 1;
+  volatile int* s_abort = s_n + 2;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+  int64_t start;
+  int len;
+  p.seqs.get(seq, start, len);
+  if (qt * 128 >= len) return;
+  const int hk = h / (p.H / p.Hkv);
+  const int nb = (int)ceil_div(len, BLK);
+  const int64_t nB2 = (int64_t)p.nB * p.nB;
+  const uint8_t* mrow = p.mask + ((int64_t)seq * p.H + h) * nB2;
+
+  if (tid == 0) {
+    for (int i = 0; i < B_N; ++i) {
+      const uint32_t cnt = (i == B_SE || i == B_SE + 1 || i == B_PF || i == B_PF + 1 || i == B_OE)
+                               ? 128u : 1u;
+      mbar_init(&bars[i], cnt);
+    }
+    *s_abort = 0;
+    // Tile list: NVFP4 tiles ascending, then FP16 tiles ascending.
+    const int qb0 = BLK == 128 ? qt : 2 * qt;
+    const int nqb = BLK == 128 ? 1 : min(2, nb - 2 * qt);
+    int n = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int j = 0; j < nb; ++j) {
+        bool need = false;
+        for (int b = qb0; b < qb0 + nqb; ++b) {
+          if (p.causal && j > b) continue;
+          if ((mrow[(int64_t)b * p.nB + j] != 0) == (pass == 1)) need = true;
+        }
+        if (need) s_list[n++] = (uint16_t)(j | (pass << 15));
+      }
+      if (pass == 0) *s_n4 = n;
+    }
+    *s_n = n;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const int n = *s_n, n4 = *s_n4;
+
+  uint8_t* q4s = sm + L::OFF_Q4;
+  uint8_t* q16s = sm + L::OFF_Q16;
+
+  if (warp == 4) {
+    // ------------------------------------------------------- producer --
+    if (lane == 0) {
+      const int64_t qtile = ((int64_t)seq * p.H + h) * p.nTq + qt;
+      bool q4_issued = false, q16_issued = false;
+      int issued[2] = {-1, -1};
+      if (n4 > 0) {
+        mbar_arrive_expect_tx(&bars[B_Q4], L::QT4);
+        bulk_g2s(q4s, p.q4 + qtile * L::QT4, L::QT4, &bars[B_Q4]);
+        q4_issued = true;
+      }
+      for (int t = 0; t < n && !*s_abort; ++t) {
+        const int st = t & 1;
+        const int j = s_list[t] & 0x7FFF;
+        const bool f16 = (s_list[t] >> 15) != 0;
+        if (t >= 2 && !mbar_wait(&bars[B_KVE + st], ((t >> 1) - 1) & 1, s_abort)) break;
+        if (f16 && !q16_issued) {
+          mbar_arrive_expect_tx(&bars[B_Q16], L::Q16B);
+          bulk_g2s(q16s, p.q16 + qtile * L::Q16B, L::Q16B, &bars[B_Q16]);
+          q16_issued = true;
+        }
+        uint8_t* stg = sm + L::OFF_STG + st * L::STG;
+        const int64_t ktile = ((int64_t)seq * p.Hkv + hk) * p.nB + j;
+        if (!f16) {
+          mbar_arrive_expect_tx(&bars[B_KVF + st], L::KT4 + L::VT4);
+          bulk_g2s(stg, p.k4 + ktile * L::KT4, L::KT4, &bars[B_KVF + st]);
+          bulk_g2s(stg + L::V4_OFF, p.v4 + ktile * L::VT4, L::VT4, &bars[B_KVF + st]);
+        } else {
+          mbar_arrive_expect_tx(&bars[B_KVF + st], L::KT16 + L::VT16);
+          bulk_g2s(stg, p.k16 + ktile * L::KT16, L::KT16, &bars[B_KVF + st]);
+          bulk_g2s(stg + L::V16_OFF, p.v16 + ktile * L::VT16, L::VT16, &bars[B_KVF + st]);
+        }
+        issued[st] = t;
+      }
+      // Drain: every copy this thread issued has landed before the CTA ends.
+      int dummy = 0;
+      volatile int* never = &dummy;
+      if (q4_issued) mbar_wait(&bars[B_Q4], 0, never, 200000000ull);
+      if (q16_issued) mbar_wait(&bars[B_Q16], 0, never, 200000000ull);
+      for (int st = 0; st < 2; ++st)
+        if (issued[st] >= 0) mbar_wait(&bars[B_KVF + st], (issued[st] >> 1) & 1, never, 200000000ull);
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      const uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
+      const uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
+      bool q4_ready = false, q16_ready = false;
+      const uint32_t q4a = smem_u32(q4s), q16a = smem_u32(q16s);
+      auto issue_qk = [&](int t) -> bool {
+        const int st = t & 1;
+        const bool f16 = (s_list[t] >> 15) != 0;
+        if (!mbar_wait(&bars[B_KVF + st], (t >> 1) & 1, s_abort)) return false;
+        if (!f16 && !q4_ready) {
+          if (!mbar_wait(&bars[B_Q4], 0, s_abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < D / 64; ++s)
+            tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
+                             make_sdesc(q4a + 128 * (D / 2) + 512 * s, 512, 128, SW_NONE));
+          q4_ready = true;
+        }
+        if (f16 && !q16_ready) {
+          if (!mbar_wait(&bars[B_Q16], 0, s_abort)) return false;
+          q16_ready = true;
+        }
+        if (t >= 2 && !mbar_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint32_t dS = tmem + L::T_S + st * BLK;
+        const uint32_t stg = smem_u32(sm + L::OFF_STG + st * L::STG);
+        if (!f16) {
+          const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
+#pragma unroll
+          for (int s = 0; s < D / 64; ++s)
+            tc_cp_32x128b_x4(ksf + 4 * s,
+                             make_sdesc(stg + BLK * (D / 2) + 512 * s, 512, 128, SW_NONE));
+#pragma unroll
+          for (int s = 0; s < D / 64; ++s)
+            mma_nvf4(dS, make_sdesc(q4a + 32 * s, 16, 8 * (D / 2), swz_mode_for_pitch(D / 2)),
+                     make_sdesc(stg + 32 * s, 16, 8 * (D / 2), swz_mode_for_pitch(D / 2)),
+                     id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s, s > 0);
+        } else {
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(dS, make_sdesc(q16a + (s / 4) * 128 * 128 + 32 * (s % 4), 16, 1024, SW_128B),
+                    make_sdesc(stg + (s / 4) * BLK * 128 + 32 * (s % 4), 16, 1024, SW_128B),
+                    id_qk16, s > 0);
+        }
+        tc_commit(&bars[B_SF + st]);
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int st = t & 1;
+        const bool f16 = (s_list[t] >> 15) != 0;
+        if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) return false;
+        if (t >= 1 && !mbar_wait(&bars[B_OE], (t - 1) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint32_t dO = tmem + L::T_PV;
+        const uint32_t stg = smem_u32(sm + L::OFF_STG + st * L::STG);
+        if (!f16) {
+          const uint32_t p4 = smem_u32(sm + L::OFF_P4 + st * L::PT4A);
+          const uint32_t v4 = stg + L::V4_OFF;
+          const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
+          const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
+#pragma unroll
+          for (int s = 0; s < BLK / 64; ++s) {
+            tc_cp_32x128b_x4(psf + 4 * s, make_sdesc(p4 + 128 * (BLK / 2) + 512 * s, 512, 128, SW_NONE));
+            tc_cp_32x128b_x4(vsf + 4 * s, make_sdesc(v4 + D * (BLK / 2) + 512 * s, 512, 128, SW_NONE));
+          }
+#pragma unroll
+          for (int s = 0; s < BLK / 64; ++s)
+            mma_nvf4(dO, make_sdesc(p4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
+                     make_sdesc(v4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
+                     id_pv4, psf + 4 * s, vsf + 4 * s, s > 0);
+        } else {
+          const uint32_t p16 = smem_u32(sm + L::OFF_P16);
+          const uint32_t v16 = stg + L::V16_OFF;
+#pragma unroll
+          for (int s = 0; s < BLK / 16; ++s)
+            mma_f16(dO, make_sdesc(p16 + (s / 4) * 128 * 128 + 32 * (s % 4), 16, 1024, SW_128B),
+                    make_sdesc(v16 + (s / 4) * D * 128 + 32 * (s % 4), 16, 1024, SW_128B),
+                    id_pv16, s > 0);
+        }
+        tc_commit(&bars[B_OF]);
+        tc_commit(&bars[B_KVE + st]);
+        return true;
+      };
+      bool ok = n > 0 ? issue_qk(0) : true;
+      for (int t = 0; t < n && ok; ++t) {
+        if (t + 1 < n) ok = issue_qk(t + 1);
+        if (ok) ok = issue_pv(t);
+      }
+      tc_commit(&bars[B_DONE]);
+      int dummy = 0;
+      volatile int* never = &dummy;
+      mbar_wait(&bars[B_DONE], 0, never, 200000000ull);
+    }
+  } else {
+    // -------------------------------------------------------- softmax --
+    const int r = tid;
+    const int row = qt * 128 + r;
+    const bool row_ok = row < len;
+    const int qb = BLK == 128 ? qt : 2 * qt + (r >= 64 ? 1 : 0);
+    const float gq = tensor_scale_from_amax(p.amax[0]);
+    const float gk = tensor_scale_from_amax(p.amax[1]);
+    const float gv = tensor_scale_from_amax(p.amax[2]);
+    const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float O[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) O[c] = 0.0f;
+    float m = -INFINITY, l = 0.0f;
+    float pend_alpha = 1.0f, pend_sigma = 0.0f;
+    int pending = -1;
+    bool prev16 = false;
+    bool ok = true;
+
+    auto accumulate = [&](int u) -> bool {
+      if (!warp_wait(&bars[B_OF], u & 1, s_abort)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        tmem_ld32(lane_base + L::T_PV + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          O[32 * c + i] = fmaf(O[32 * c + i], pend_alpha, pend_sigma * v[i]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_OE]);
+      return true;
+    };
+
+    for (int t = 0; t < n && ok; ++t) {
+      const int st = t & 1;
+      const int j = s_list[t] & 0x7FFF;
+      const bool f16 = (s_list[t] >> 15) != 0;
+      const bool pair_ok = row_ok && qb < nb && (!p.causal || j <= qb) &&
+                           ((mrow[(int64_t)qb * p.nB + j] != 0) == f16);
+      const int lim = pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1;
+      const float cs = f16 ? p.scale16 : cs4;
+      if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sb = lane_base + L::T_S + st * BLK;
+      // pass 1: tile row max of the scaled scores
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BLK / 32; ++c) {
+        float v[32];
+        tmem_ld32(sb + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * c + i <= lim) mt = fmaxf(mt, __fmul_rn(v[i], cs));
+      }
+      const float m_new = fmaxf(m, mt);
+      const float alpha = (m == -INFINITY) ? 1.0f : ex2_approx(__fsub_rn(m, m_new));
+      const float rowmax = (mt == -INFINITY) ? 0.0f : ex2_approx(__fsub_rn(mt, m_new));
+      l *= alpha;
+      // FP16 tiles share one P buffer: the previous FP16 PV must be done.
+      if (f16 && prev16 && pending >= 0) {
+        if (!accumulate(pending)) { ok = false; break; }
+        pending = -1;
+      }
+      const float inv = rowmax > 0.0f ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
+      const float sigma = f16 ? 1.0f : __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv);
+      float lsum = 0.0f;
+      uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+      uint8_t* p16 = sm + L::OFF_P16;
+#pragma unroll
+      for (int c = 0; c < BLK / 32; ++c) {
+        float v[32];
+        tmem_ld32(sb + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float a = __fmul_rn(v[i], cs);
+          v[i] = (32 * c + i <= lim) ? ex2_approx(__fsub_rn(a, m_new)) : 0.0f;
+          lsum += v[i];
+        }
+        if (!f16) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float ph[16];
+            float amax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              ph[e] = __fmul_rn(v[16 * b + e], inv);
+              amax = fmaxf(amax, ph[e]);
+            }
+            const uint32_t S = ue4m3(__fdiv_rn(amax, 6.0f));
+            const float rr = S ? __frcp_rn(ue4m3_decode(S)) : 0.0f;
+            uint32_t cb[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              cb[e] = e2m1x2(__fmul_rn(ph[2 * e], rr), __fmul_rn(ph[2 * e + 1], rr));
+            const uint32_t k16 = 2 * c + b;
+            *reinterpret_cast<uint2*>(p4 + swz_offset(r, k16 * 8, BLK / 2)) =
+                make_uint2(cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24),
+                           cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24));
+            p4[128 * (BLK / 2) + sf_offset(r, k16)] = (uint8_t)S;
+          }
+        } else {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = (uint32_t)f2h<DT>(v[8 * q8 + 2 * e]) |
+                     ((uint32_t)f2h<DT>(v[8 * q8 + 2 * e + 1]) << 16);
+            const uint32_t key0 = 32 * c + 8 * q8;
+            *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
+                                      swz_offset(r, (key0 % 64) * 2, 128)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      l += lsum;
+      m = m_new;
+      tc_fence_before();
+      mbar_arrive(&bars[B_SE + st]);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_PF + st]);
+      if (pending >= 0) {
+        if (!accumulate(pending)) { ok = false; break; }
+      }
+      pending = t;
+      pend_alpha = alpha;  // applied to O before PV(t) is added
+      pend_sigma = sigma;
+      prev16 = f16;
+    }
+    if (ok && pending >= 0) ok = accumulate(pending);
+    // epilogue
+    if (ok && row_ok) {
+      const float il = l > 0.0f ? 1.0f / l : 0.0f;
+      uint16_t* orow = p.out + ((start + row) * p.H + h) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 8) {
+        uint4 w;
+        w.x = (uint32_t)f2h<DT>(O[c] * il) | ((uint32_t)f2h<DT>(O[c + 1] * il) << 16);
+        w.y = (uint32_t)f2h<DT>(O[c + 2] * il) | ((uint32_t)f2h<DT>(O[c + 3] * il) << 16);
+        w.z = (uint32_t)f2h<DT>(O[c + 4] * il) | ((uint32_t)f2h<DT>(O[c + 5] * il) << 16);
+        w.w = (uint32_t)f2h<DT>(O[c + 6] * il) | ((uint32_t)f2h<DT>(O[c + 7] * il) << 16);
+        *reinterpret_cast<uint4*>(orow + c) = w;
+      }
+      const float lse = l > 0.0f ? m * 0.6931471805599453f + logf(l) : -INFINITY;
+      const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
+                                      : ((int64_t)seq * p.H + h) * len + row;
+      p.lse[li] = lse;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace thrift

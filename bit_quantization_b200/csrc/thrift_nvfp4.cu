@@ -1,0 +1,460 @@
+// C-ABI entry points of libthrift_nvfp4.so: argument checks, workspace
+// carving and kernel launches.  Declarations and the contract of every entry
+// point are in include/thrift_nvfp4.h.
+#include <cmath>
+#include <cstdio>
+#include <utility>
+#include <vector>
+
+#include "attn.cuh"
+#include "select.cuh"
+
+namespace thrift {
+namespace {
+
+constexpr int kThreads = 256;
+
+int grid_for(int64_t work_items, int per_block = kThreads) {
+  int64_t g = ceil_div(work_items, per_block);
+  if (g < 1) g = 1;
+  if (g > 148 * 16) g = 148 * 16;
+  return (int)g;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+thrift_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+// Bump allocator over the caller's workspace (1024-byte aligned slices).
+struct Carve {
+  uintptr_t base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(reinterpret_cast<uintptr_t>(b)) {}
+  template <class T>
+  T* take(size_t bytes) {
+    off = (off + 1023) & ~(size_t)1023;
+    T* p = reinterpret_cast<T*>(base + off);
+    off += bytes;
+    return p;
+  }
+};
+
+// ------------------------------------------------------- quantiser glue --
+
+template <int DT>
+void launch_amax(const void* x, int64_t n_blocks, int G, uint32_t* out, cudaStream_t st) {
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  const int grid = grid_for(n_blocks);
+  if (G == 8) amax_kernel<DT, 8><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
+  else if (G == 4) amax_kernel<DT, 4><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
+  else amax_kernel<DT, 0><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
+}
+
+template <int DT, int G, bool SS>
+void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, int given,
+                         uint8_t* codes, uint8_t* scales, cudaStream_t st) {
+  quant_rows_kernel<DT, G, SS><<<grid_for(nb), kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(x), nb, amax, ts, given, codes, scales);
+}
+
+template <int DT>
+void launch_quant_rows(const void* x, int64_t nb, int G, bool ss, uint32_t* amax, float* ts,
+                       int given, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
+  if (G == 8) {
+    if (ss) launch_quant_rows_t<DT, 8, true>(x, nb, amax, ts, given, codes, scales, st);
+    else launch_quant_rows_t<DT, 8, false>(x, nb, amax, ts, given, codes, scales, st);
+  } else if (G == 4) {
+    if (ss) launch_quant_rows_t<DT, 4, true>(x, nb, amax, ts, given, codes, scales, st);
+    else launch_quant_rows_t<DT, 4, false>(x, nb, amax, ts, given, codes, scales, st);
+  } else {
+    if (ss) launch_quant_rows_t<DT, 0, true>(x, nb, amax, ts, given, codes, scales, st);
+    else launch_quant_rows_t<DT, 0, false>(x, nb, amax, ts, given, codes, scales, st);
+  }
+}
+
+// ----------------------------------------------------- attention layout --
+
+struct AttnWs {
+  uint32_t* amax;
+  double* means_q;
+  double* means_k;
+  double* scores;
+  uint8_t* mask;
+  uint8_t *q4, *k4, *v4, *q16, *k16, *v16;
+  size_t bytes;
+};
+
+AttnWs carve_attn(void* ws, int nseq, int maxlen, int H, int Hkv, int d, int blk) {
+  Carve c(ws);
+  AttnWs w;
+  const int64_t nB = ceil_div(maxlen, blk), nTq = ceil_div(maxlen, 128);
+  w.amax = c.take<uint32_t>(256);
+  w.means_q = c.take<double>((size_t)nseq * H * nB * d * 8);
+  w.means_k = c.take<double>((size_t)nseq * Hkv * nB * d * 8);
+  w.scores = c.take<double>((size_t)nseq * H * nB * nB * 8);
+  w.mask = c.take<uint8_t>((size_t)nseq * H * nB * nB);
+  w.q4 = c.take<uint8_t>((size_t)nseq * H * nTq * fp4_tile_bytes(128, d));
+  w.k4 = c.take<uint8_t>((size_t)nseq * Hkv * nB * fp4_tile_bytes(blk, d));
+  w.v4 = c.take<uint8_t>((size_t)nseq * Hkv * nB * fp4_tile_bytes(d, blk));
+  w.q16 = c.take<uint8_t>((size_t)nseq * H * nTq * f16_tile_bytes(128, d));
+  w.k16 = c.take<uint8_t>((size_t)nseq * Hkv * nB * f16_tile_bytes(blk, d));
+  w.v16 = c.take<uint8_t>((size_t)nseq * Hkv * nB * f16_tile_bytes(d, blk));
+  w.bytes = c.off + 1024;
+  return w;
+}
+
+template <int DT, int G, bool HAD, bool SS>
+void launch_qk_image(const void* x, SeqInfo si, int nseq, int nh, int rows, int ntiles,
+                     const uint32_t* amax, uint8_t* i4, uint8_t* i16, cudaStream_t st) {
+  const int64_t nb = (int64_t)nseq * ntiles * rows * nh * G;
+  qk_image_kernel<DT, G, HAD, SS><<<grid_for(nb), kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(x), si, nseq, nh, rows, ntiles, amax, i4, i16);
+}
+
+template <int DT, int G>
+void dispatch_qk_image(bool had, bool ss, const void* x, SeqInfo si, int nseq, int nh, int rows,
+                       int ntiles, const uint32_t* amax, uint8_t* i4, uint8_t* i16,
+                       cudaStream_t st) {
+  if (had) {
+    if (ss) launch_qk_image<DT, G, true, true>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+    else launch_qk_image<DT, G, true, false>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+  } else {
+    if (ss) launch_qk_image<DT, G, false, true>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+    else launch_qk_image<DT, G, false, false>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+  }
+}
+
+// Optional event pairs around the attention kernel (thrift_kernel_timer_*).
+struct KernelTimer {
+  bool enabled = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;
+  size_t used = 0;
+  cudaEvent_t* next_pair() {
+    if (used == pool.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess) return nullptr;
+      if (cudaEventCreate(&b) != cudaSuccess) return nullptr;
+      pool.push_back({a, b});
+    }
+    return &pool[used++].first;
+  }
+};
+KernelTimer g_timer;
+
+template <int DT, int D, int BLK>
+thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) {
+  using L = AttnLayout<D, BLK>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<DT, D, BLK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)L::SMEM_ALLOC) != cudaSuccess)
+      return THRIFT_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid(nTq, p.H, p.nseq);
+  cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
+  if (ev) cudaEventRecord(ev[0], st);
+  attn_fwd_kernel<DT, D, BLK><<<grid, 192, L::SMEM_ALLOC, st>>>(p);
+  const thrift_status s = launch_status();
+  if (ev) cudaEventRecord(ev[1], st);
+  return s;
+}
+
+template <int DT>
+thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
+                        int64_t total, int maxlen, int H, int Hkv, int d, int blk, int causal,
+                        float frac, int ss, int had, void* out, float* lse, int lse_varlen,
+                        void* ws, cudaStream_t st) {
+  AttnWs w = carve_attn(ws, nseq, maxlen, H, Hkv, d, blk);
+  const int nB = (int)ceil_div(maxlen, blk), nTq = (int)ceil_div(maxlen, 128);
+  const int G = d / 16;
+  if (cudaMemsetAsync(w.amax, 0, 16, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+  launch_amax<DT>(q, total * H * d / 16, had ? G : 0, w.amax + 0, st);
+  launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, w.amax + 1, st);
+  launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
+  if (G == 8) {
+    dispatch_qk_image<DT, 8>(had, ss, q, si, nseq, H, 128, nTq, w.amax + 0, w.q4, w.q16, st);
+    dispatch_qk_image<DT, 8>(had, ss, k, si, nseq, Hkv, blk, nB, w.amax + 1, w.k4, w.k16, st);
+  } else {
+    dispatch_qk_image<DT, 4>(had, ss, q, si, nseq, H, 128, nTq, w.amax + 0, w.q4, w.q16, st);
+    dispatch_qk_image<DT, 4>(had, ss, k, si, nseq, Hkv, blk, nB, w.amax + 1, w.k4, w.k16, st);
+  }
+  {
+    const int64_t nv = (int64_t)nseq * Hkv * (nB * blk / 16) * d;
+    if (ss)
+      v_image_kernel<DT, true><<<grid_for(nv), kThreads, 0, st>>>(
+          static_cast<const uint16_t*>(v), si, nseq, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
+    else
+      v_image_kernel<DT, false><<<grid_for(nv), kThreads, 0, st>>>(
+          static_cast<const uint16_t*>(v), si, nseq, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
+  }
+  // selection
+  block_means_kernel<DT><<<grid_for((int64_t)nseq * H * nB * d), kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(q), si, nseq, H, d, blk, nB, w.means_q);
+  block_means_kernel<DT><<<grid_for((int64_t)nseq * Hkv * nB * d), kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(k), si, nseq, Hkv, d, blk, nB, w.means_k);
+  pair_scores_kernel<<<grid_for((int64_t)nseq * H * nB * nB), kThreads, 0, st>>>(
+      w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, w.scores);
+  topk_kernel<<<nseq * H, kTopkThreads, 0, st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
+  if (launch_status() != THRIFT_OK) return THRIFT_ERR_CUDA;
+
+  AttnParams p;
+  p.q4 = w.q4; p.k4 = w.k4; p.v4 = w.v4; p.q16 = w.q16; p.k16 = w.k16; p.v16 = w.v16;
+  p.mask = w.mask;
+  p.amax = w.amax;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.seqs = si;
+  p.nseq = nseq; p.H = H; p.Hkv = Hkv; p.nB = nB; p.nTq = nTq; p.causal = causal;
+  p.lse_varlen = lse_varlen;
+  p.total = total;
+  const double l2e = 1.4426950408889634;
+  p.scale16 = (float)(l2e / std::sqrt((double)d));
+  p.scale4 = (float)(l2e / std::sqrt((double)d) / (had ? (double)d : 1.0));
+  if (d == 128 && blk == 128) return launch_attn_kernel<DT, 128, 128>(p, nTq, st);
+  if (d == 128 && blk == 64) return launch_attn_kernel<DT, 128, 64>(p, nTq, st);
+  if (d == 64 && blk == 128) return launch_attn_kernel<DT, 64, 128>(p, nTq, st);
+  return launch_attn_kernel<DT, 64, 64>(p, nTq, st);
+}
+
+thrift_status check_attn_args(const void* q, const void* k, const void* v, int dt, int H, int Hkv,
+                              int maxlen, int d, int blk, float frac, const void* out,
+                              const float* lse) {
+  if (!q || !k || !v || !out || !lse) return THRIFT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (H <= 0 || Hkv <= 0 || H % Hkv || maxlen <= 0) return THRIFT_ERR_ARG;
+  if (!(frac >= 0.0f && frac <= 1.0f)) return THRIFT_ERR_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (ceil_div(maxlen, blk) > 1024) return THRIFT_ERR_UNSUPPORTED;
+  if (H > 65535) return THRIFT_ERR_UNSUPPORTED;
+  return THRIFT_OK;
+}
+
+}  // namespace
+}  // namespace thrift
+
+using namespace thrift;
+
+extern "C" {
+
+const char* thrift_status_string(int s) {
+  switch (s) {
+    case THRIFT_OK: return "ok";
+    case THRIFT_ERR_ARG: return "invalid argument";
+    case THRIFT_ERR_UNSUPPORTED: return "unsupported";
+    case THRIFT_ERR_CUDA: return "CUDA error";
+    case THRIFT_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+thrift_status thrift_device_status(int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return THRIFT_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (reset) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess)
+      return THRIFT_ERR_CUDA;
+  }
+  return (thrift_status)v;
+}
+
+thrift_status thrift_kernel_timer_enable(int enable) {
+  g_timer.enabled = enable != 0;
+  return THRIFT_OK;
+}
+
+thrift_status thrift_kernel_timer_read(double* total_ms, int* launches) {
+  if (!total_ms || !launches) return THRIFT_ERR_ARG;
+  double sum = 0.0;
+  for (size_t i = 0; i < g_timer.used; ++i) {
+    auto& pr = g_timer.pool[i];
+    if (cudaEventSynchronize(pr.second) != cudaSuccess) return THRIFT_ERR_CUDA;
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess) return THRIFT_ERR_CUDA;
+    sum += ms;
+  }
+  *total_ms = sum;
+  *launches = (int)g_timer.used;
+  g_timer.used = 0;
+  return THRIFT_OK;
+}
+
+size_t nvfp4_quantize_workspace_size(void) { return 256; }
+
+thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64_t cols,
+                             int use_scalesearch, int use_hadamard, int tensor_scale_given,
+                             uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 || cols > 4096) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (!tensor_scale || !workspace || ws_bytes < nvfp4_quantize_workspace_size())
+    return THRIFT_ERR_ARG;
+  if (use_hadamard && cols != 64 && cols != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (rows == 0) return THRIFT_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7))
+    return THRIFT_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  const int64_t nb = rows * cols / 16;
+  const int G = use_hadamard ? (int)(cols / 16) : 0;
+  if (!tensor_scale_given) {
+    if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+    if (dt == THRIFT_BF16) launch_amax<1>(x, nb, G, amax, st);
+    else launch_amax<0>(x, nb, G, amax, st);
+  }
+  if (dt == THRIFT_BF16)
+    launch_quant_rows<1>(x, nb, G, use_scalesearch != 0, amax, tensor_scale, tensor_scale_given,
+                         codes, scales, st);
+  else
+    launch_quant_rows<0>(x, nb, G, use_scalesearch != 0, amax, tensor_scale, tensor_scale_given,
+                         codes, scales, st);
+  return launch_status();
+}
+
+thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t rows,
+                                       int64_t cols, int use_scalesearch,
+                                       int tensor_scale_given, uint8_t* codes,
+                                       uint8_t* scales, float* tensor_scale, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  if (rows < 0 || cols <= 0 || rows % 16) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (!tensor_scale || !workspace || ws_bytes < nvfp4_quantize_workspace_size())
+    return THRIFT_ERR_ARG;
+  if (rows == 0) return THRIFT_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7) || ((rows / 2) % 8))
+    return THRIFT_ERR_ARG;
+  if ((rows * cols) % 16) return THRIFT_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  if (!tensor_scale_given) {
+    if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+    if (dt == THRIFT_BF16) launch_amax<1>(x, rows * cols / 16, 0, amax, st);
+    else launch_amax<0>(x, rows * cols / 16, 0, amax, st);
+  }
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  const int grid = grid_for((rows / 16) * cols);
+  if (dt == THRIFT_BF16) {
+    if (use_scalesearch)
+      quant_cols_kernel<1, true><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                                           tensor_scale_given, codes, scales);
+    else
+      quant_cols_kernel<1, false><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                                            tensor_scale_given, codes, scales);
+  } else {
+    if (use_scalesearch)
+      quant_cols_kernel<0, true><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                                           tensor_scale_given, codes, scales);
+    else
+      quant_cols_kernel<0, false><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                                            tensor_scale_given, codes, scales);
+  }
+  return launch_status();
+}
+
+size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int blk) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || blk <= 0) return 0;
+  const size_t nB = (size_t)ceil_div(N, blk);
+  return 3 * 1024 + (size_t)B * H * nB * d * 8 + (size_t)B * Hkv * nB * d * 8 +
+         (size_t)B * H * nB * nB * 8;
+}
+
+thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int B, int H,
+                              int Hkv, int N, int d, int blk, int causal, float topk_frac,
+                              uint8_t* mask, void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k || !mask || !workspace) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0) return THRIFT_ERR_ARG;
+  if (!(topk_frac >= 0.0f && topk_frac <= 1.0f)) return THRIFT_ERR_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (ceil_div(N, blk) > 1024) return THRIFT_ERR_UNSUPPORTED;
+  if (ws_bytes < block_mean_topk_workspace_size(B, H, Hkv, N, d, blk)) return THRIFT_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nB = (int)ceil_div(N, blk);
+  Carve c(workspace);
+  double* mq = c.take<double>((size_t)B * H * nB * d * 8);
+  double* mk = c.take<double>((size_t)B * Hkv * nB * d * 8);
+  double* sc = c.take<double>((size_t)B * H * nB * nB * 8);
+  SeqInfo si{nullptr, N};
+  const uint16_t* qp = static_cast<const uint16_t*>(q);
+  const uint16_t* kp = static_cast<const uint16_t*>(k);
+  if (dt == THRIFT_BF16) {
+    block_means_kernel<1><<<grid_for((int64_t)B * H * nB * d), kThreads, 0, st>>>(qp, si, B, H, d, blk, nB, mq);
+    block_means_kernel<1><<<grid_for((int64_t)B * Hkv * nB * d), kThreads, 0, st>>>(kp, si, B, Hkv, d, blk, nB, mk);
+  } else {
+    block_means_kernel<0><<<grid_for((int64_t)B * H * nB * d), kThreads, 0, st>>>(qp, si, B, H, d, blk, nB, mq);
+    block_means_kernel<0><<<grid_for((int64_t)B * Hkv * nB * d), kThreads, 0, st>>>(kp, si, B, Hkv, d, blk, nB, mk);
+  }
+  pair_scores_kernel<<<grid_for((int64_t)B * H * nB * nB), kThreads, 0, st>>>(mq, mk, si, B, H, Hkv, d, blk, nB, sc);
+  topk_kernel<<<B * H, kTopkThreads, 0, st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
+  return launch_status();
+}
+
+size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || (d != 64 && d != 128) ||
+      (blk != 64 && blk != 128))
+    return 0;
+  return carve_attn(nullptr, B, N, H, Hkv, d, blk).bytes;
+}
+
+thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
+                              int B, int H, int Hkv, int N, int d, int blk, int causal,
+                              float topk_frac, int use_scalesearch, int use_hadamard, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, N, d, blk, topk_frac, out, lse);
+  if (s != THRIFT_OK) return s;
+  if (B <= 0 || !workspace || !aligned16(workspace)) return THRIFT_ERR_ARG;
+  if (ws_bytes < thrift_attn_workspace_size(B, H, Hkv, N, d, blk)) return THRIFT_ERR_ARG;
+  if ((int64_t)B * ceil_div(N, 128) > 0x7FFFFFFF || B > 65535) return THRIFT_ERR_UNSUPPORTED;
+  SeqInfo si{nullptr, N};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t total = (int64_t)B * N;
+  if (dt == THRIFT_BF16)
+    return attn_impl<1>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
+                        use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
+  return attn_impl<0>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
+                      use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
+}
+
+size_t thrift_attn_varlen_workspace_size(int nseq, int64_t total, int max_seqlen, int H,
+                                         int Hkv, int d, int blk) {
+  (void)total;
+  if (nseq <= 0 || H <= 0 || Hkv <= 0 || max_seqlen <= 0 || (d != 64 && d != 128) ||
+      (blk != 64 && blk != 128))
+    return 0;
+  return carve_attn(nullptr, nseq, max_seqlen, H, Hkv, d, blk).bytes;
+}
+
+thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v,
+                                     thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                     int64_t total, int max_seqlen, int H, int Hkv, int d,
+                                     int blk, int causal, float topk_frac, int use_scalesearch,
+                                     int use_hadamard, void* out, float* lse, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, max_seqlen, d, blk, topk_frac, out, lse);
+  if (s != THRIFT_OK) return s;
+  if (!cu_seqlens || nseq <= 0 || nseq > 65535 || total <= 0 || !workspace ||
+      !aligned16(workspace))
+    return THRIFT_ERR_ARG;
+  if (ws_bytes < thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk))
+    return THRIFT_ERR_ARG;
+  SeqInfo si{cu_seqlens, 0};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == THRIFT_BF16)
+    return attn_impl<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal,
+                        topk_frac, use_scalesearch, use_hadamard, out, lse, 1, workspace, st);
+  return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
+                      use_scalesearch, use_hadamard, out, lse, 1, workspace, st);
+}
+
+}  // extern "C"

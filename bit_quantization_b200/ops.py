@@ -1,0 +1,256 @@
+"""ctypes binding of libthrift_nvfp4.so (C ABI in include/thrift_nvfp4.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and the current stream.  There is no
+fallback: a missing library, a missing CUDA device or a failing call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libthrift_nvfp4.so")
+
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
+F16, BF16 = 0, 1
+
+_lib = None
+
+# Exported names of the C ABI, in header order.
+EXPORTS = (
+    "thrift_status_string", "thrift_device_status", "nvfp4_quantize_workspace_size",
+    "nvfp4_quantize", "nvfp4_quantize_colblocks", "block_mean_topk_workspace_size",
+    "block_mean_topk", "thrift_attn_workspace_size", "thrift_attn_fwd",
+    "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
+    "thrift_kernel_timer_enable", "thrift_kernel_timer_read",
+)
+
+
+class ThriftError(RuntimeError):
+    pass
+
+
+def lib():
+    """Loads the library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ThriftError(
+                "libthrift_nvfp4.so is not built; run `python -m bit_quantization_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
+        L.thrift_status_string.restype = C.c_char_p
+        L.thrift_status_string.argtypes = [i32]
+        L.thrift_device_status.restype = i32
+        L.thrift_device_status.argtypes = [i32]
+        L.nvfp4_quantize_workspace_size.restype = sz
+        L.nvfp4_quantize_workspace_size.argtypes = []
+        L.nvfp4_quantize.restype = i32
+        L.nvfp4_quantize.argtypes = [P, i32, i64, i64, i32, i32, i32, P, P, P, P, sz, P]
+        L.nvfp4_quantize_colblocks.restype = i32
+        L.nvfp4_quantize_colblocks.argtypes = [P, i32, i64, i64, i32, i32, P, P, P, P, sz, P]
+        L.block_mean_topk_workspace_size.restype = sz
+        L.block_mean_topk_workspace_size.argtypes = [i32] * 6
+        L.block_mean_topk.restype = i32
+        L.block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P, sz, P]
+        L.thrift_attn_workspace_size.restype = sz
+        L.thrift_attn_workspace_size.argtypes = [i32] * 6
+        L.thrift_attn_fwd.restype = i32
+        L.thrift_attn_fwd.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                      i32, P, P, P, sz, P]
+        L.thrift_attn_varlen_workspace_size.restype = sz
+        L.thrift_attn_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+        L.thrift_attn_fwd_varlen.restype = i32
+        L.thrift_attn_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
+                                             i32, f32, i32, i32, P, P, P, sz, P]
+        L.thrift_kernel_timer_enable.restype = i32
+        L.thrift_kernel_timer_enable.argtypes = [i32]
+        L.thrift_kernel_timer_read.restype = i32
+        L.thrift_kernel_timer_read.argtypes = [P, P]
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().thrift_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise ThriftError(f"{what}: {status_string(code)} ({code})")
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return F16
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ThriftError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ThriftError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ThriftError("tensors must be contiguous")
+
+
+def _stream(t: torch.Tensor):
+    return C.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return C.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def device_status(reset: bool = False) -> int:
+    """Synchronises the device; returns OK or ERR_TIMEOUT (device wait gave up)."""
+    return lib().thrift_device_status(int(reset))
+
+
+def kernel_timer_enable(enable: bool):
+    _check(lib().thrift_kernel_timer_enable(int(enable)), "thrift_kernel_timer_enable")
+
+
+def kernel_timer_read():
+    """Returns (summed attention-kernel milliseconds, timed launches)."""
+    ms = C.c_double(0.0)
+    n = C.c_int(0)
+    _check(lib().thrift_kernel_timer_read(C.byref(ms), C.byref(n)), "thrift_kernel_timer_read")
+    return ms.value, n.value
+
+
+class Workspace:
+    """Grow-only device scratch buffer reused across calls on one device."""
+
+    def __init__(self):
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_ws = Workspace()
+
+
+# ------------------------------------------------------------------ quantiser
+
+def nvfp4_quantize(x: torch.Tensor, use_scalesearch=False, use_hadamard=False,
+                   tensor_scale: Optional[torch.Tensor] = None, codes=None, scales=None,
+                   workspace: Optional[torch.Tensor] = None):
+    """x [rows, cols] fp16/bf16 on CUDA -> (codes u8 [rows, cols/2],
+    scales u8 [rows, cols/16], tensor_scale f32 [1])."""
+    _need_cuda(x)
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    given = tensor_scale is not None
+    ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else _ws.get(lib().nvfp4_quantize_workspace_size(),
+                                                         x.device)
+    _check(lib().nvfp4_quantize(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
+                                int(use_hadamard), int(given), _ptr(codes), _ptr(scales),
+                                _ptr(ts), _ptr(ws), ws.numel(), _stream(x)), "nvfp4_quantize")
+    return codes, scales, ts
+
+
+def nvfp4_quantize_colblocks(x: torch.Tensor, use_scalesearch=False,
+                             tensor_scale: Optional[torch.Tensor] = None):
+    """x [rows, cols] -> (codes [cols, rows/2], scales [cols, rows/16], g)."""
+    _need_cuda(x)
+    rows, cols = x.shape
+    codes = torch.empty((cols, rows // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((cols, rows // 16), dtype=torch.uint8, device=x.device)
+    given = tensor_scale is not None
+    ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = _ws.get(lib().nvfp4_quantize_workspace_size(), x.device)
+    _check(lib().nvfp4_quantize_colblocks(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
+                                          int(given), _ptr(codes), _ptr(scales), _ptr(ts),
+                                          _ptr(ws), ws.numel(), _stream(x)),
+           "nvfp4_quantize_colblocks")
+    return codes, scales, ts
+
+
+# ------------------------------------------------------------------ selection
+
+def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, topk_frac: float):
+    """q [B,N,H,d], k [B,N,Hkv,d] -> mask u8 [B,H,nB,nB] (1 = FP16 pair)."""
+    _need_cuda(q, k)
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    nB = (N + blk - 1) // blk
+    mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
+    need = lib().block_mean_topk_workspace_size(B, H, Hkv, N, d, blk)
+    ws = _ws.get(need, q.device)
+    _check(lib().block_mean_topk(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk, int(causal),
+                                 float(topk_frac), _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
+           "block_mean_topk")
+    return mask
+
+
+# ------------------------------------------------------------------ attention
+
+def thrift_attn_workspace_size(B, H, Hkv, N, d, blk) -> int:
+    return int(lib().thrift_attn_workspace_size(B, H, Hkv, N, d, blk))
+
+
+def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesearch=False,
+                    use_hadamard=False, out=None, lse=None, workspace=None):
+    """q [B,N,H,d], k/v [B,N,Hkv,d] -> (out [B,N,H,d], lse f32 [B,H,N])."""
+    _need_cuda(q, k, v)
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    need = thrift_attn_workspace_size(B, H, Hkv, N, d, blk)
+    if need == 0:
+        raise ThriftError("thrift_attn_fwd: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    _check(lib().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, Hkv, N, d, blk,
+                                 int(causal), float(topk_frac), int(use_scalesearch),
+                                 int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                 _stream(q)), "thrift_attn_fwd")
+    return out, lse
+
+
+def thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk) -> int:
+    return int(lib().thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk))
+
+
+def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True,
+                           topk_frac=0.0, use_scalesearch=False, use_hadamard=False, out=None,
+                           lse=None, workspace=None):
+    """q [total,H,d], k/v [total,Hkv,d], cu_seqlens int32 [nseq+1] (CUDA) ->
+    (out [total,H,d], lse f32 [H,total])."""
+    _need_cuda(q, k, v, cu_seqlens)
+    if cu_seqlens.dtype != torch.int32:
+        raise ThriftError("cu_seqlens must be int32")
+    total, H, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    need = thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk)
+    if need == 0:
+        raise ThriftError("thrift_attn_fwd_varlen: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    _check(lib().thrift_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens),
+                                        nseq, total, int(max_seqlen), H, Hkv, d, blk,
+                                        int(causal), float(topk_frac), int(use_scalesearch),
+                                        int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws),
+                                        ws.numel(), _stream(q)), "thrift_attn_fwd_varlen")
+    return out, lse

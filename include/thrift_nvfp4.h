@@ -1,0 +1,164 @@
+/*
+ * thrift_nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 attention library.
+ *
+ * Block-scaled 4-bit (NVFP4) attention forward with selective FP16 block
+ * pairs.  Sources of the method (web pages):
+ *   [AQ] "Attn-QAT: 4-Bit Attention With Quantization-Aware Training",
+ *        Resumo tecnico 1 (E2M1: 15 distinct values).
+ *   [TA] "ThriftAttention", Metodologia: step 1 (block-mean scores
+ *        S^_ij = qbar_i . kbar_j, top-k pairs), step 2 (FP16 path for the
+ *        selected pairs, NVFP4 for the rest, FlashAttention-2 online softmax
+ *        merge, two-level quantisation of P), and the kernel paragraph that
+ *        follows (FP4 blocks first, then the FP16 helper; tiles with no
+ *        selected pair skip the FP16 path).
+ *   [SS] "Busca tus Escalas de Punto Flotante por Bloques": Declaracion del
+ *        Problema (NVFP4, E4M3 block scale), ScaleSearch Mecanismo and
+ *        Estrategia de Busqueda (s = round(||x||_inf/6); offsets f in [-2,6]
+ *        on the scale's bit pattern; least block MSE), ScaleSearchAttention
+ *        (Hadamard rotation of Q/K; QK^T and PV on FP4 tensor cores with FP32
+ *        accumulation).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory.  Scratch lives in the caller's
+ *     `workspace` (device memory of at least the size the matching
+ *     *_workspace_size function returns, 256-byte aligned).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are validated on the host before any
+ *     launch; a bad argument returns THRIFT_ERR_ARG / THRIFT_ERR_UNSUPPORTED
+ *     and launches nothing.  A failed launch returns THRIFT_ERR_CUDA.
+ *   - Device-side waits are bounded; a wait that gives up sets the device
+ *     status word read by thrift_device_status() and the kernel returns.
+ *   - 16-bit inputs: fp16 or bf16 (thrift_dtype).  Pointers must be 16-byte
+ *     aligned.
+ *   - FP4 codes are E2M1, two per byte: element 2c in the low nibble, 2c+1
+ *     in the high nibble.  Block scales are UE4M3 bytes (bias 7, max 0x7E =
+ *     448).  The per-tensor FP32 scale is g = amax/2688 (g = 1 for an all-zero
+ *     tensor); dequantised value = e2m1(code) * ue4m3(scale) * g.
+ */
+#ifndef THRIFT_NVFP4_H
+#define THRIFT_NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  THRIFT_OK = 0,
+  THRIFT_ERR_ARG = -1,          /* bad pointer, size or flag */
+  THRIFT_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle */
+  THRIFT_ERR_CUDA = -3,         /* a CUDA runtime call failed */
+  THRIFT_ERR_TIMEOUT = -4       /* a device-side wait gave up */
+} thrift_status;
+
+typedef enum { THRIFT_F16 = 0, THRIFT_BF16 = 1 } thrift_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char* thrift_status_string(int status);
+
+/*
+ * Synchronises the calling thread with the current device and returns the
+ * device status word: THRIFT_OK, or THRIFT_ERR_TIMEOUT if any kernel of this
+ * library gave up on a bounded wait since the last reset.  reset != 0 clears
+ * the word.  Returns THRIFT_ERR_CUDA if the synchronisation itself fails.
+ */
+thrift_status thrift_device_status(int reset);
+
+/* ------------------------------------------------------------ quantiser --
+ * [SS] ScaleSearch; [AQ] E2M1.  Quantises x [rows, cols] (row-major, 16-bit)
+ * to NVFP4 with 16-element blocks along cols.
+ *   codes  [rows, cols/2] uint8 out;   scales [rows, cols/16] uint8 out.
+ *   tensor_scale: one float; read when tensor_scale_given != 0, else written
+ *     (g = amax/2688 over the whole, possibly rotated, tensor).
+ *   use_scalesearch: per block, among the bytes S0+f, f in {0,-2,-1,1,...,6}
+ *     that stay in 1..126, keep the first one of least error
+ *     (sum over the block, in order, of (t-q)^2 by fmaf) * S^2, where
+ *     t = x * (1/(S*g)) and q is t rounded to the E2M1 grid.
+ *   use_hadamard: rotate every row by the unnormalised Sylvester-Hadamard
+ *     transform first (cols must be 64 or 128).
+ * Requirements: rows >= 0, cols % 16 == 0, cols <= 4096.
+ * Workspace: nvfp4_quantize_workspace_size() bytes.
+ */
+size_t nvfp4_quantize_workspace_size(void);
+thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64_t cols,
+                             int use_scalesearch, int use_hadamard, int tensor_scale_given,
+                             uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Same, with 16-element blocks along ROWS (the token axis of V):
+ *   codes [cols, rows/2], scales [cols, rows/16].  rows % 16 == 0.
+ * No Hadamard option (the rotation applies to Q and K only). */
+thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t rows,
+                                       int64_t cols, int use_scalesearch,
+                                       int tensor_scale_given, uint8_t* codes,
+                                       uint8_t* scales, float* tensor_scale, void* workspace,
+                                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------- block selection --
+ * [TA] Metodologia step 1.  q [B,N,H,d], k [B,N,Hkv,d] 16-bit.  Blocks of
+ * blk tokens from the sequence start (the last may be partial).  Block means
+ * in fp64 (sequential sum in token order / count); scores by a sequential
+ * fp64 fma over channels; per (batch, head) the k = ceil(frac*n_valid - 1e-9)
+ * best valid pairs are selected (causal: j <= i), ties to the lower i*nB+j.
+ *   mask [B, H, nB, nB] uint8 out, 1 = FP16 pair.
+ * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, 0<=frac<=1,
+ * nB = ceil(N/blk) <= 1024.
+ */
+size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
+thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int B, int H,
+                              int Hkv, int N, int d, int blk, int causal, float topk_frac,
+                              uint8_t* mask, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- attention --
+ * [TA] + [SS] ScaleSearchAttention.  q [B,N,H,d], k, v [B,N,Hkv,d] 16-bit,
+ * contiguous.  Per (batch, head, query block of blk rows) the key blocks that
+ * were not selected run first on the NVFP4 path (block-scaled FP4 MMA, fp32
+ * accumulation; P quantised in two levels: a per-row, per-key-block fp32
+ * factor rowmax/2688 and NVFP4 16-key blocks), then the selected ones on the
+ * FP16 path (16-bit MMA with the unrotated inputs), merged by one online
+ * softmax.  Q, K, V are quantised inside the call (Q, K along d; V along
+ * tokens; use_scalesearch / use_hadamard as in nvfp4_quantize).
+ *   out [B,N,H,d] 16-bit out;  lse [B,H,N] fp32 out (natural log).
+ * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, N >= 1,
+ * 0 <= topk_frac <= 1, nB = ceil(N/blk) <= 1024.
+ */
+size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
+thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
+                              int B, int H, int Hkv, int N, int d, int blk, int causal,
+                              float topk_frac, int use_scalesearch, int use_hadamard, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* Varlen: q [total,H,d], k, v [total,Hkv,d] packed; cu_seqlens int32
+ * [nseq+1] on the DEVICE (cu_seqlens[0] = 0, cu_seqlens[nseq] = total,
+ * every length in 1..max_seqlen).  Each sequence is an independent problem
+ * (its own blocks and top-k); tensor scales cover the whole packed tensor.
+ *   out [total,H,d];  lse [H,total] fp32.
+ * Requirements as thrift_attn_fwd with N -> max_seqlen. */
+size_t thrift_attn_varlen_workspace_size(int nseq, int64_t total, int max_seqlen, int H,
+                                         int Hkv, int d, int blk);
+thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v,
+                                     thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                     int64_t total, int max_seqlen, int H, int Hkv, int d,
+                                     int blk, int causal, float topk_frac, int use_scalesearch,
+                                     int use_hadamard, void* out, float* lse, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------- kernel timing --
+ * Measurement aid (not part of the method).  While enabled, every
+ * thrift_attn_fwd / thrift_attn_fwd_varlen call records a CUDA event pair on
+ * its stream around the attention kernel launch.  thrift_kernel_timer_read
+ * waits for the recorded events, returns the summed kernel time in
+ * milliseconds and the number of timed launches, and clears the record.
+ * Host-side state shared by all threads of the process; not thread-safe.
+ * Events are created on first use and kept for reuse. */
+thrift_status thrift_kernel_timer_enable(int enable);
+thrift_status thrift_kernel_timer_read(double* total_ms, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THRIFT_NVFP4_H */

@@ -1,0 +1,122 @@
+"""GPU attention vs the oracle's emulation of the same quantisation and
+tiling (ThriftAttention Metodologia step 2; ScaleSearchAttention).
+
+Bar: max |out - oracle| <= 1e-2 and cosine >= 0.9999 over the compared rows;
+lse within 1e-2.  Error against unquantised fp64 attention is reported.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantization_b200 import ops, synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+MIN_COS = 0.9999
+
+
+def _to_f(orc, u16, dt):
+    return orc.half_to_float(u16, dt).astype(np.float64) if u16.size < 200000 else \
+        _fast_f(u16, dt)
+
+
+def _fast_f(u16, dt):
+    t = torch.from_numpy(u16.view(np.int16))
+    return (t.view(torch.bfloat16) if dt == 1 else t.view(torch.float16)).double().numpy()
+
+
+def _compare(got, want, what):
+    got = got.reshape(-1).astype(np.float64)
+    want = want.reshape(-1).astype(np.float64)
+    err = np.max(np.abs(got - want))
+    cos = float(got @ want / (np.linalg.norm(got) * np.linalg.norm(want) + 1e-300))
+    assert err <= MAX_ABS and cos >= MIN_COS, f"{what}: max abs {err:.3e}, cos {cos:.6f}"
+    return err, cos
+
+
+def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_off=3.0):
+    w = synth.AttnWorkload("case", B, H, Hkv, N, d, dtype, causal, blk, frac, ss, had,
+                           k_offset_std=k_off, seed=seed)
+    inp = synth.make_attn_inputs(w)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    out, lse = ops.thrift_attn_fwd(q.cuda(), k.cuda(), v.cuda(), blk=blk, causal=causal,
+                                   topk_frac=frac, use_scalesearch=ss, use_hadamard=had)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == ops.OK
+    dt = synth.dtype_code(dtype)
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    qp, kp, vp = (synth.as_u16(t.reshape(B * N, -1, d)) for t in (q, k, v))
+    r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had)
+    got = out.cpu().reshape(B * N, H, d)
+    gotf = got.double().numpy()
+    want = _to_f(orc, r["out"], dt)
+    _compare(gotf, want, "out")
+    lse_want = r["lse"].reshape(H, B, N).transpose(1, 0, 2)
+    assert np.max(np.abs(lse.cpu().numpy() - lse_want)) < 1e-2
+    return gotf, qp, kp, vp, cu, dt
+
+
+def test_tiny_workload(orc):
+    w = synth.TINY
+    gotf, qp, kp, vp, cu, dt = run_case(orc, w.B, w.N, w.H, w.Hkv, w.d, w.blk, w.causal,
+                                        w.topk_frac, w.use_scalesearch, w.use_hadamard, w.dtype,
+                                        k_off=0.0)
+    ref, _ = orc.attn_fp64(qp, kp, vp, dt, cu, w.causal)
+    print("tiny: max abs error vs fp64 attention", np.max(np.abs(gotf - ref)))
+
+
+CASES = [
+    # B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype
+    (1, 384, 2, 1, 128, 128, False, 0.0, False, False, torch.bfloat16),
+    (2, 300, 4, 2, 128, 128, True, 0.25, True, True, torch.bfloat16),
+    (1, 200, 2, 2, 64, 64, True, 0.5, False, True, torch.float16),
+    (1, 256, 2, 2, 64, 128, False, 1.0, False, False, torch.float16),
+    (1, 520, 2, 1, 128, 64, True, 0.1, True, False, torch.bfloat16),
+    (1, 129, 1, 1, 128, 128, True, 0.05, False, False, torch.float16),
+    (3, 17, 2, 2, 64, 64, False, 0.3, True, True, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(str(x) for x in c[:10]))
+def test_parity_cases(orc, case):
+    run_case(orc, *case)
+
+
+def test_varlen_parity(orc):
+    lens = [100, 257, 384, 1, 129]
+    H, Hkv, d, blk = 4, 2, 128, 128
+    total = sum(lens)
+    gen = torch.Generator().manual_seed(7)
+    q = torch.randn((total, H, d), generator=gen).to(torch.bfloat16)
+    k = (torch.randn((total, Hkv, d), generator=gen) + 2.0).to(torch.bfloat16)
+    v = torch.randn((total, Hkv, d), generator=gen).to(torch.bfloat16)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    cu_t = torch.from_numpy(cu).cuda()
+    for frac, ss, had in [(0.0, False, False), (0.25, True, True), (1.0, False, True)]:
+        out, lse = ops.thrift_attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu_t, max(lens),
+                                              blk=blk, causal=True, topk_frac=frac,
+                                              use_scalesearch=ss, use_hadamard=had)
+        torch.cuda.synchronize()
+        assert ops.device_status(reset=True) == ops.OK
+        r = orc.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), 1, cu, blk, True,
+                            frac, use_ss=ss, use_had=had)
+        _compare(out.cpu().double().numpy(), _to_f(orc, r["out"], 1), f"varlen frac={frac}")
+        assert np.max(np.abs(lse.cpu().numpy() - r["lse"])) < 1e-2
+
+
+def test_all_fp16_pairs_match_fp64(orc):
+    # topk_frac = 1: every pair on the FP16 path -> plain 16-bit attention.
+    gotf, qp, kp, vp, cu, dt = run_case(orc, 1, 256, 2, 2, 128, 128, True, 1.0, False, False,
+                                        torch.float16)
+    ref, _ = orc.attn_fp64(qp, kp, vp, dt, cu, True)
+    assert np.max(np.abs(gotf.reshape(ref.shape) - ref)) < 4e-3
+
+
+def test_deterministic():
+    inp = synth.make_attn_inputs(synth.TINY)
+    a = ops.thrift_attn_fwd(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), blk=64,
+                            topk_frac=0.25)[0]
+    b = ops.thrift_attn_fwd(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), blk=64,
+                            topk_frac=0.25)[0]
+    assert torch.equal(a, b)

@@ -1,0 +1,92 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point the header declares, and rejects bad arguments on the host before any
+launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from bit_quantization_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([a-z_][a-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            names.append(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _header_functions()
+    assert len(names) >= 11
+    assert set(names) == set(ops.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    assert ops.status_string(0) == "ok"
+    assert ops.status_string(-4) == "device wait timed out"
+
+
+def test_workspace_sizes_are_host_only(L):
+    assert L.nvfp4_quantize_workspace_size() >= 16
+    assert L.thrift_attn_workspace_size(1, 1, 1, 256, 64, 64) > 0
+    assert L.thrift_attn_workspace_size(1, 1, 1, 256, 96, 64) == 0
+    assert L.block_mean_topk_workspace_size(2, 32, 32, 8192, 128, 128) > 2 * 32 * 64 * 64 * 8
+    big = L.thrift_attn_workspace_size(1, 32, 8, 32768, 128, 128)
+    assert big < 1 << 31
+
+
+def test_bad_arguments_rejected_before_launch(L):
+    P = C.c_void_p
+    dummy = P(4096)
+    ws = P(8192)
+    # cols not a multiple of 16
+    assert L.nvfp4_quantize(dummy, 0, 4, 24, 0, 0, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_ARG
+    # Hadamard on an unsupported width
+    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 1, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_UNSUPPORTED
+    # workspace too small
+    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, 8, None) == ops.ERR_ARG
+    # misaligned input
+    assert L.nvfp4_quantize(P(4098), 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_ARG
+    # attention: unsupported head dim, bad GQA ratio, bad fraction, null pointer
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 96, 128, 0, C.c_float(0.1), 0, 0,
+                             dummy, dummy, ws, 1 << 40, None) == ops.ERR_UNSUPPORTED
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 3, 256, 128, 128, 0, C.c_float(0.1), 0, 0,
+                             dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(1.5), 0, 0,
+                             dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
+    assert L.thrift_attn_fwd(None, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0,
+                             dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0,
+                             dummy, dummy, ws, 16, None) == ops.ERR_ARG
+    assert L.block_mean_topk(dummy, dummy, 0, 1, 4, 4, 256, 128, 32, 0, C.c_float(0.1), dummy, ws,
+                             1 << 40, None) == ops.ERR_UNSUPPORTED
+    assert L.thrift_attn_fwd_varlen(dummy, dummy, dummy, 1, None, 2, 100, 64, 4, 4, 128, 128, 1,
+                                    C.c_float(0.1), 0, 0, dummy, dummy, ws, 1 << 40,
+                                    None) == ops.ERR_ARG
+
+
+def test_binding_fails_loudly_without_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    x = torch.zeros((16, 32), dtype=torch.float16)
+    with pytest.raises(ops.ThriftError):
+        ops.nvfp4_quantize(x)
