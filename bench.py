@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 / selective-FP16 attention forward on B200.
+
+One step = one thrift_attn_fwd call over one batch of the workload: tensor
+absmax, Q/K/V NVFP4 quantisation, block-mean top-k selection and the mixed
+NVFP4/FP16 attention kernel.  Prints one JSON line (rank 0).
+
+Default workload: B=2, H=32, N=8192, d=128, bf16, non-causal, 128x128 blocks,
+10% FP16 pairs, K with per-channel offsets N(0, 3).  Its inputs (3 x 134 MB)
+exceed L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference   # the CPU oracle on a bounded sample
+Multi-GPU (weak scaling, independent problems per rank, no collective on the
+data path): launched by torch.distributed.run, one rank per GPU.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_quantization_b200 import synth  # noqa: E402
+
+WORKLOADS = {
+    "b2h32n8192": synth.C_B2H32N8K,
+    "gqa32k": synth.C_GQA32K,
+    "tiny": synth.TINY,
+}
+
+METRIC = "NVFP4 attention fwd TFLOPS (whole step: quantise + select + attention)"
+UNIT = "TFLOP/s"
+KERNELS_PER_STEP = 11  # 3 absmax, 2 Q/K images, 1 V image, 2 block means, 1 scores, 1 top-k, 1 attention
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def pair_flops(mask, w, lengths):
+    """Algorithmic FLOPs (4*d per unmasked score element) split by path."""
+    blk, d = w.blk, w.d
+    f4 = f16 = 0.0
+    for b, L in enumerate(lengths):
+        nb = (L + blk - 1) // blk
+        for i in range(nb):
+            r0, r1 = i * blk, min(L, (i + 1) * blk)
+            for j in range(nb if not w.causal else i + 1):
+                c0, c1 = j * blk, min(L, (j + 1) * blk)
+                if w.causal:
+                    rows = np.arange(r0, r1)
+                    cnt = float(np.clip(np.minimum(rows + 1, c1) - c0, 0, None).sum())
+                else:
+                    cnt = float((r1 - r0) * (c1 - c0))
+                sel = mask[b, :, i, j]
+                n16 = float(sel.sum())
+                f16 += 4 * d * cnt * n16
+                f4 += 4 * d * cnt * (w.H - n16)
+    return f4, f16
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.proc = None
+        self.dev_id = None
+        try:
+            uuid = torch.cuda.get_device_properties(dev).uuid
+            self.dev_id = "GPU-" + str(uuid)
+        except Exception:
+            self.dev_id = str(dev.index or 0)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.dev_id, f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def oracle_sample(w, nunits, nthreads, inp=None):
+    """The CPU oracle on a bounded sample of the workload: one head of batch
+    entry 0 (full sequence length), `nunits` evenly spread query blocks.
+    Returns (seconds, algorithmic flops of the sampled rows, description)."""
+    import oracle
+    if inp is None:
+        inp = synth.make_attn_inputs(w)
+    N, d, blk = w.N, w.d, w.blk
+    q = inp["q"][0, :, 0:1].contiguous()
+    k = inp["k"][0, :, 0:1].contiguous()
+    v = inp["v"][0, :, 0:1].contiguous()
+    cu = np.array([0, N], np.int32)
+    nb = (N + blk - 1) // blk
+    blocks = np.unique(np.linspace(0, nb - 1, nunits).round().astype(int))
+    units = np.array([[0, 0, i] for i in blocks], np.int32)
+    t0 = time.perf_counter()
+    oracle.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), synth.dtype_code(w.dtype),
+                       cu, blk, w.causal, w.topk_frac, use_ss=w.use_scalesearch,
+                       use_had=w.use_hadamard, units=units, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    fl = 0.0
+    for i in blocks:
+        rows = np.arange(i * blk, min(N, (i + 1) * blk))
+        cnt = (rows + 1).sum() if w.causal else len(rows) * N
+        fl += 4.0 * d * cnt
+    desc = (f"1 of {w.B * w.H} heads (batch 0, head 0, full N={N}), {len(blocks)} of {nb} query "
+            f"blocks; includes that head's quantisation and selection")
+    return dt, fl, desc
+
+
+def run_reference(args, w):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return 0
+    cores = os.cpu_count() or 1
+    inp = synth.make_attn_inputs(w)
+    # Size the sample so the whole run stays within about two minutes.
+    dt0, _, _ = oracle_sample(w, 4, cores, inp)
+    budget = min(4.0, 120.0 / (args.steps + args.warmup))
+    units = int(max(1, min(args.ref_units, 4 * budget / max(dt0, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(w, units, cores, inp)
+    times, fl, desc = [], 0.0, ""
+    for _ in range(args.steps):
+        dt, fl, desc = oracle_sample(w, units, cores, inp)
+        times.append(dt)
+    t = sum(times)
+    val = fl * args.steps / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "dtype": str(w.dtype).replace("torch.", ""), "causal": w.causal, "blk": w.blk,
+            "topk_frac": w.topk_frac, "scalesearch": w.use_scalesearch,
+            "hadamard": w.use_hadamard, "k_offset_std": w.k_offset_std,
+            "l2": "inputs larger than L2 (no flush)", "parallelism": "independent problems per GPU"}
+
+
+def quantizer_line(dev, peaks):
+    """Quantiser-only workload (65536 x 128 fp16 with 4 outlier channels):
+    GB/s of algorithmic bytes (2 B read + 0.5625 B written per element).
+    Twelve rotating input copies (> L2); the calls are captured in one CUDA
+    graph so host-side launch gaps do not enter the timing."""
+    from bit_quantization_b200 import ops
+    x0 = synth.make_quant_input(synth.QUANT).to(dev)
+    xs = [x0.clone() for _ in range(12)]
+    rows, cols = x0.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    res = {}
+    algo = rows * cols * (2 + 0.5 + 0.0625)
+    n = 120
+    for ss in (False, True):
+        for i in range(6):
+            ops.nvfp4_quantize(xs[i % 12], ss, False, None, codes, scales, ws)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        with torch.cuda.graph(g, stream=side):
+            for i in range(n):
+                ops.nvfp4_quantize(xs[i % 12], ss, False, None, codes, scales, ws)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / (3 * n)
+        gbs = algo / (ms * 1e-3) / 1e9
+        res["scalesearch_on" if ss else "scalesearch_off"] = {
+            "us_per_call": 1e3 * ms, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "kernels_per_call": 2}
+        del g
+    res["workload"] = synth.QUANT.name
+    res["algorithmic_bytes"] = algo
+    res["timing"] = "CUDA graph of 120 calls, 12 rotating inputs (201 MB > L2)"
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="b2h32n8192", choices=sorted(WORKLOADS))
+    ap.add_argument("--ref-units", type=int, default=24)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quantizer", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    from bit_quantization_b200 import ops
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+
+    inp = synth.make_attn_inputs(w, seed=w.seed + rank)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(ops.thrift_attn_workspace_size(w.B, w.H, w.Hkv, w.N, w.d, w.blk),
+                     dtype=torch.uint8, device=dev)
+
+    def step(qq, kk, vv):
+        ops.thrift_attn_fwd(qq, kk, vv, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
+                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
+                            out=out, lse=lse, workspace=ws)
+
+    # FLOP split from the selection this input produces
+    mask = ops.block_mean_topk(q, k, w.blk, w.causal, w.topk_frac).cpu().numpy()
+    f4, f16 = pair_flops(mask, w, inp["lengths"])
+    flops = f4 + f16
+
+    for _ in range(args.warmup):
+        step(q, k, v)
+    torch.cuda.synchronize(dev)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    sampler = ClockSampler(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    ops.kernel_timer_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step(q, k, v)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ops.kernel_timer_enable(False)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = e0.elapsed_time(e1)
+    kms, klaunches = ops.kernel_timer_read()
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out during the timed region")
+    t = torch.tensor([ms_total, kms / max(klaunches, 1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_total, k_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    qh, kh, vh = (inp[n].pin_memory() for n in ("q", "k", "v"))
+    outh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(3, min(args.steps, 30))
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step(qd, kd, vd)
+        outh.copy_(out, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(te[0]) / e2e_steps
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = outh.numel() * outh.element_size() + lseh.numel() * lseh.element_size()
+
+    # roofline of the attention kernel (dominant): tensor-bound contraction;
+    # t_ideal = F4/P4 + F16/P16 with P16 the measured bf16 GEMM rate and
+    # P4 = 4 x P16 (nominal dense FP4 : BF16 ratio).
+    p16 = peaks["bf16_tflops_sustained"]
+    p4 = 4.0 * p16
+    t_ideal_ms = (f4 / (p4 * 1e12) + f16 / (p16 * 1e12)) * 1e3
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    peak_eff = flops / (t_ideal_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
+                "peak": peak_eff, "unit": "TFLOP/s", "frac": achieved / peak_eff,
+                "traffic": None,
+                "peak_note": (f"{peak_src} bf16 sustained {p16} TF/s x4 for the FP4 share, x1 for "
+                              f"the FP16 share ({100 * f16 / flops:.1f}% of flops)"),
+                "kernel_ms": k_ms, "fp4_flops": f4, "fp16_flops": f16}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
+            "data": "synthetic", "config": config_of(w), "roofline": roofline,
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_quantizer:
+        line["quantizer"] = quantizer_line(dev, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        dt, fl, desc = oracle_sample(w, args.ref_units, cores, inp)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

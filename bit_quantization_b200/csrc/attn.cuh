@@ -11,10 +11,13 @@
 // quantised in two levels (per row and key tile an fp32 factor rowmax/2688,
 // then NVFP4 16-key blocks).
 //
-// Roles (192 threads):
-//   warps 0-3  softmax + output: thread r owns query row r (TMEM lane r);
-//   warp 4     producer: bulk copies of the pre-quantised tile images;
-//   warp 5     tensor-memory owner and MMA issuer (one elected lane).
+// Roles (320 threads):
+//   warps 0-7  softmax + output: query row r (TMEM lane r) is shared by warps
+//              r/32 and r/32 + 4, each owning half of the key columns and
+//              half of the output columns; the two exchange their partial row
+//              max once per tile through shared memory;
+//   warp 8     producer: bulk copies of the pre-quantised tile images;
+//   warp 9     tensor-memory owner and MMA issuer (one elected lane).
 // Tensor memory (512 columns): S double buffer [2][BLK], PV [D], then the
 // scale factors of Q, K (x2), P (x2) and V (x2).
 // Every wait is bounded; a wait that gives up sets the device status word
@@ -42,12 +45,6 @@ struct AttnParams {
   float scale16;           // log2(e)/sqrt(d)
 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 template <int D, int BLK>
 struct AttnLayout {
   static constexpr uint32_t align(uint32_t x) { return (x + 1023u) & ~1023u; }
@@ -71,9 +68,10 @@ struct AttnLayout {
   static constexpr uint32_t OFF_P4 = OFF_STG + 2 * STG;
   static constexpr uint32_t OFF_P16 = OFF_P4 + 2 * PT4A;
   static constexpr uint32_t OFF_LIST = OFF_P16 + align(P16B);
-  static constexpr uint32_t MAX_TILES = 1024;
+  static constexpr uint32_t MAX_TILES = 512;  // key tiles per sequence
   static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
-  static constexpr uint32_t BYTES = OFF_BAR + 256;
+  static constexpr uint32_t OFF_XCH = OFF_BAR + 256;  // row-max / row-sum exchange
+  static constexpr uint32_t BYTES = OFF_XCH + 4 * 2 * 2 * 128 + 4 * 2 * 128;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
   // tensor-memory columns
   static constexpr uint32_t T_S = 0;
@@ -93,6 +91,22 @@ enum : int {
   B_SE = 8 /* 8,9 */, B_PF = 10 /* 10,11 */, B_OF = 12, B_OE = 13, B_DONE = 14, B_N = 15
 };
 
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kAttnThreads = 32 * (kSoftmaxWarps + 2);
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Waits with every lane of the warp; the result is uniform across the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -100,7 +114,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 template <int DT, int D, int BLK>
-__global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnParams p) {
   using L = AttnLayout<D, BLK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
   if (tid == 0) {
     for (int i = 0; i < B_N; ++i) {
       const uint32_t cnt = (i == B_SE || i == B_SE + 1 || i == B_PF || i == B_PF + 1 || i == B_OE)
-                               ? 128u : 1u;
+                               ? (uint32_t)kSoftmaxThreads : 1u;
       mbar_init(&bars[i], cnt);
     }
     *s_abort = 0;
@@ -149,7 +163,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
@@ -162,7 +176,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
   uint8_t* q4s = sm + L::OFF_Q4;
   uint8_t* q16s = sm + L::OFF_Q16;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------- producer --
     if (lane == 0) {
       const int64_t qtile = ((int64_t)seq * p.H + h) * p.nTq + qt;
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
       for (int st = 0; st < 2; ++st)
         if (issued[st] >= 0) mbar_wait(&bars[B_KVF + st], (issued[st] >> 1) & 1, never, 200000000ull);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ----------------------------------------------------- MMA issuer --
     if (lane == 0) {
       const uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
@@ -301,7 +315,12 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int r = tid;
+    // Two threads per query row: warp w owns TMEM lane quarter w % 4 and
+    // half hf = w / 4 of the key columns (and of the output columns).
+    constexpr int SC = BLK / 2;   // score columns per thread
+    constexpr int OC = D / 2;     // output columns per thread
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int r = q4 * 32 + lane;
     const int row = qt * 128 + r;
     const bool row_ok = row < len;
     const int qb = BLK == 128 ? qt : 2 * qt + (r >= 64 ? 1 : 0);
@@ -309,27 +328,28 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
     const float gk = tensor_scale_from_amax(p.amax[1]);
     const float gv = tensor_scale_from_amax(p.amax[2]);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    float O[D];
+    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+    float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][2 halves][128]
+    float O[OC];
 #pragma unroll
-    for (int c = 0; c < D; ++c) O[c] = 0.0f;
+    for (int c = 0; c < OC; ++c) O[c] = 0.0f;
     float m = -INFINITY, l = 0.0f;
     float pend_alpha = 1.0f, pend_sigma = 0.0f;
     int pending = -1;
     bool prev16 = false;
     bool ok = true;
 
+    // O <- alpha * O + sigma * PV(u) for this thread's output columns.
     auto accumulate = [&](int u) -> bool {
       if (!warp_wait(&bars[B_OF], u & 1, s_abort)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < OC / 32; ++c) {
         float v[32];
-        tmem_ld32(lane_base + L::T_PV + 32 * c, v);
+        tmem_ld32(lane_base + L::T_PV + hf * OC + 32 * c, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          O[32 * c + i] = fmaf(O[32 * c + i], pend_alpha, pend_sigma * v[i]);
+        for (int i = 0; i < 32; ++i) O[32 * c + i] = fmaf(O[32 * c + i], pend_alpha, pend_sigma * v[i]);
       }
       tc_fence_before();
       mbar_arrive(&bars[B_OE]);
@@ -342,88 +362,98 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
       const bool f16 = (s_list[t] >> 15) != 0;
       const bool pair_ok = row_ok && qb < nb && (!p.causal || j <= qb) &&
                            ((mrow[(int64_t)qb * p.nB + j] != 0) == f16);
-      const int lim = pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1;
+      // last valid score column of this thread's half (-1 or less: none)
+      const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - hf * SC;
+      const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
       const float cs = f16 ? p.scale16 : cs4;
-      if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t sb = lane_base + L::T_S + st * BLK;
-      // pass 1: tile row max of the scaled scores
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BLK / 32; ++c) {
-        float v[32];
-        tmem_ld32(sb + 32 * c, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * c + i <= lim) mt = fmaxf(mt, __fmul_rn(v[i], cs));
-      }
-      const float m_new = fmaxf(m, mt);
-      const float alpha = (m == -INFINITY) ? 1.0f : ex2_approx(__fsub_rn(m, m_new));
-      const float rowmax = (mt == -INFINITY) ? 0.0f : ex2_approx(__fsub_rn(mt, m_new));
-      l *= alpha;
-      // FP16 tiles share one P buffer: the previous FP16 PV must be done.
+      // FP16 tiles share one P buffer: the previous FP16 PV must be done
+      // (and folded into O) before this tile's P is written.
       if (f16 && prev16 && pending >= 0) {
         if (!accumulate(pending)) { ok = false; break; }
         pending = -1;
       }
-      const float inv = rowmax > 0.0f ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
-      const float sigma = f16 ? 1.0f : __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv);
+      if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+      tc_fence_after();
+      float a[SC];
+#pragma unroll
+      for (int c = 0; c < SC / 32; ++c)
+        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c,
+                  *reinterpret_cast<float(*)[32]>(a + 32 * c));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
+      // scaled scores (log2 domain) and this half's row max
+      float mh = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < SC; ++i) {
+          a[i] = __fmul_rn(a[i], cs);
+          mh = fmaxf(mh, a[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < SC; ++i) {
+          a[i] = i <= lim ? __fmul_rn(a[i], cs) : -INFINITY;
+          mh = fmaxf(mh, a[i]);
+        }
+      }
+      float* xs = xch + st * 256;
+      xs[hf * 128 + r] = mh;
+      named_bar_sync(1 + q4, 64);
+      const float mt = fmaxf(xs[r], xs[128 + r]);
+      const float m_new = fmaxf(m, mt);
+      const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(__fsub_rn(m, m_new));
+      const float rowmax = (mt == -INFINITY) ? 0.0f : ex2_ftz(__fsub_rn(mt, m_new));
+      const float msub = m_new == -INFINITY ? 0.0f : m_new;
+      l *= alpha;
       float lsum = 0.0f;
-      uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
-      uint8_t* p16 = sm + L::OFF_P16;
 #pragma unroll
-      for (int c = 0; c < BLK / 32; ++c) {
-        float v[32];
-        tmem_ld32(sb + 32 * c, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = __fmul_rn(v[i], cs);
-          v[i] = (32 * c + i <= lim) ? ex2_approx(__fsub_rn(a, m_new)) : 0.0f;
-          lsum += v[i];
-        }
-        if (!f16) {
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float ph[16];
-            float amax = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              ph[e] = __fmul_rn(v[16 * b + e], inv);
-              amax = fmaxf(amax, ph[e]);
-            }
-            const uint32_t S = ue4m3(__fdiv_rn(amax, 6.0f));
-            const float rr = S ? __frcp_rn(ue4m3_decode(S)) : 0.0f;
-            uint32_t cb[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              cb[e] = e2m1x2(__fmul_rn(ph[2 * e], rr), __fmul_rn(ph[2 * e + 1], rr));
-            const uint32_t k16 = 2 * c + b;
-            *reinterpret_cast<uint2*>(p4 + swz_offset(r, k16 * 8, BLK / 2)) =
-                make_uint2(cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24),
-                           cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24));
-            p4[128 * (BLK / 2) + sf_offset(r, k16)] = (uint8_t)S;
-          }
-        } else {
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = (uint32_t)f2h<DT>(v[8 * q8 + 2 * e]) |
-                     ((uint32_t)f2h<DT>(v[8 * q8 + 2 * e + 1]) << 16);
-            const uint32_t key0 = 32 * c + 8 * q8;
-            *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
-                                      swz_offset(r, (key0 % 64) * 2, 128)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+      for (int i = 0; i < SC; ++i) {
+        a[i] = ex2_ftz(__fsub_rn(a[i], msub));  // exp2(-inf) = 0 for masked columns
+        lsum += a[i];
       }
       l += lsum;
       m = m_new;
-      tc_fence_before();
-      mbar_arrive(&bars[B_SE + st]);
+      float sigma = 1.0f;
+      if (!f16) {
+        const float inv = rowmax > 0.0f ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
+        sigma = __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv);
+        uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+#pragma unroll
+        for (int b = 0; b < SC / 16; ++b) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            a[16 * b + e] = __fmul_rn(a[16 * b + e], inv);
+            amax = fmaxf(amax, a[16 * b + e]);
+          }
+          const uint32_t S = ue4m3(__fdiv_rn(amax, 6.0f));
+          const float rr = S ? __frcp_rn(ue4m3_decode(S)) : 0.0f;
+          uint32_t cb[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            cb[e] = e2m1x2(__fmul_rn(a[16 * b + 2 * e], rr), __fmul_rn(a[16 * b + 2 * e + 1], rr));
+          const uint32_t k16 = hf * (SC / 16) + b;
+          *reinterpret_cast<uint2*>(p4 + swz_offset(r, k16 * 8, BLK / 2)) =
+              make_uint2(cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24),
+                         cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24));
+          p4[128 * (BLK / 2) + sf_offset(r, k16)] = (uint8_t)S;
+        }
+      } else {
+        uint8_t* p16 = sm + L::OFF_P16;
+#pragma unroll
+        for (int q8 = 0; q8 < SC / 8; ++q8) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w4[e] = (uint32_t)f2h<DT>(a[8 * q8 + 2 * e]) |
+                    ((uint32_t)f2h<DT>(a[8 * q8 + 2 * e + 1]) << 16);
+          const uint32_t key0 = hf * SC + 8 * q8;
+          *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
+                                    swz_offset(r, (key0 % 64) * 2, 128)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_PF + st]);
       if (pending >= 0) {
@@ -435,12 +465,16 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
       prev16 = f16;
     }
     if (ok && pending >= 0) ok = accumulate(pending);
-    // epilogue
+    // combine the two halves' partial sums, then write this half of the row
+    float* xl = xch + 512;
+    xl[hf * 128 + r] = l;
+    named_bar_sync(1 + q4, 64);
+    const float lt = xl[r] + xl[128 + r];
     if (ok && row_ok) {
-      const float il = l > 0.0f ? 1.0f / l : 0.0f;
-      uint16_t* orow = p.out + ((start + row) * p.H + h) * D;
+      const float il = lt > 0.0f ? 1.0f / lt : 0.0f;
+      uint16_t* orow = p.out + ((start + row) * p.H + h) * D + hf * OC;
 #pragma unroll
-      for (int c = 0; c < D; c += 8) {
+      for (int c = 0; c < OC; c += 8) {
         uint4 w;
         w.x = (uint32_t)f2h<DT>(O[c] * il) | ((uint32_t)f2h<DT>(O[c + 1] * il) << 16);
         w.y = (uint32_t)f2h<DT>(O[c + 2] * il) | ((uint32_t)f2h<DT>(O[c + 3] * il) << 16);
@@ -448,15 +482,17 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const AttnParams p) {
         w.w = (uint32_t)f2h<DT>(O[c + 6] * il) | ((uint32_t)f2h<DT>(O[c + 7] * il) << 16);
         *reinterpret_cast<uint4*>(orow + c) = w;
       }
-      const float lse = l > 0.0f ? m * 0.6931471805599453f + logf(l) : -INFINITY;
-      const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
-                                      : ((int64_t)seq * p.H + h) * len + row;
-      p.lse[li] = lse;
+      if (hf == 0) {
+        const float lse = lt > 0.0f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
+        const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
+                                        : ((int64_t)seq * p.H + h) * len + row;
+        p.lse[li] = lse;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -157,7 +157,7 @@ thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) 
   dim3 grid(nTq, p.H, p.nseq);
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
-  attn_fwd_kernel<DT, D, BLK><<<grid, 192, L::SMEM_ALLOC, st>>>(p);
+  attn_fwd_kernel<DT, D, BLK><<<grid, kAttnThreads, L::SMEM_ALLOC, st>>>(p);
   const thrift_status s = launch_status();
   if (ev) cudaEventRecord(ev[1], st);
   return s;
@@ -230,7 +230,7 @@ thrift_status check_attn_args(const void* q, const void* k, const void* v, int d
   if (!(frac >= 0.0f && frac <= 1.0f)) return THRIFT_ERR_ARG;
   if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
   if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
-  if (ceil_div(maxlen, blk) > 1024) return THRIFT_ERR_UNSUPPORTED;
+  if (ceil_div(maxlen, blk) > 512) return THRIFT_ERR_UNSUPPORTED;
   if (H > 65535) return THRIFT_ERR_UNSUPPORTED;
   return THRIFT_OK;
 }

@@ -123,7 +123,7 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
  * tokens; use_scalesearch / use_hadamard as in nvfp4_quantize).
  *   out [B,N,H,d] 16-bit out;  lse [B,H,N] fp32 out (natural log).
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, N >= 1,
- * 0 <= topk_frac <= 1, nB = ceil(N/blk) <= 1024.
+ * 0 <= topk_frac <= 1, nB = ceil(N/blk) <= 512.
  */
 size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,

@@ -531,7 +531,8 @@ static inline double deq(uint8_t code, uint8_t sc, float g) {
 }
 
 // One query block i of sequence s, head h.  Writes out rows and lse.
-static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, float* lse) {
+static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, float* lse,
+                      double* out64) {
   const int d = C.d, blk = C.blk, H = C.H, Hkv = C.Hkv;
   const int64_t st = C.cu[s];
   const int len = C.cu[s + 1] - C.cu[s];
@@ -644,6 +645,7 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
     for (int c = 0; c < d; ++c) {
       double o = l[r] > 0.0 ? O[(size_t)r * d + c] / l[r] : 0.0;
       out[(tok * H + h) * d + c] = orc_double_to_half(o, C.dt);
+      if (out64) out64[(tok * H + h) * d + c] = o;
     }
     lse[(int64_t)h * C.total + tok] = l[r] > 0.0 ? (float)(m[r] * ln2 + std::log(l[r])) : -INFINITY;
   }
@@ -655,12 +657,13 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // it, else it is computed (reading R8) and written there.  units: optional
 // list of (sequence, head, query block) triples to compute (n_units = 0 means
 // every unit); rows of other units are left untouched.  gs_out (optional)
-// receives g_Q, g_K, g_V.
+// receives g_Q, g_K, g_V.  out64 (optional) receives the fp64 output before
+// its final rounding to the 16-bit type.
 int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
                     int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
                     float frac, int use_ss, int use_had, uint8_t* mask_io, int mask_given,
                     const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
-                    float* lse, float* gs_out) {
+                    float* lse, float* gs_out, double* out64) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
   if (use_had && (d & (d - 1))) return -1;
   AttnCtx C;
@@ -723,7 +726,7 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
     n_units = (int64_t)all.size() / 3;
   }
   parallel_for(n_units, nthreads, [&](int64_t u) {
-    attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse);
+    attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse, out64);
   });
   return 0;
 }

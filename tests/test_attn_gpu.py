@@ -1,8 +1,12 @@
 """GPU attention vs the oracle's emulation of the same quantisation and
 tiling (ThriftAttention Metodologia step 2; ScaleSearchAttention).
 
-Bar: max |out - oracle| <= 1e-2 and cosine >= 0.9999 over the compared rows;
-lse within 1e-2.  Error against unquantised fp64 attention is reported.
+Bar: |out - oracle| <= 1e-2 + half an ulp of the 16-bit output type at the
+oracle's value, element by element, and cosine >= 0.9999, against the
+oracle's output before its own final rounding (both sides round the same
+real result to bf16/fp16 once; for |out| >= 2 one bf16 ulp alone exceeds
+1e-2).  lse within 1e-2.  Error against unquantised fp64 attention is
+reported.
 """
 import numpy as np
 import pytest
@@ -26,13 +30,23 @@ def _fast_f(u16, dt):
     return (t.view(torch.bfloat16) if dt == 1 else t.view(torch.float16)).double().numpy()
 
 
-def _compare(got, want, what):
+def half_ulp(x, dtype):
+    """Half the spacing of the 16-bit type at |x| (subnormal floor included)."""
+    mant, emin = (7, -126) if dtype == torch.bfloat16 else (10, -14)
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** emin)))
+    return 0.5 * 2.0 ** (e - mant)
+
+
+def _compare(got, want64, what, dtype):
     got = got.reshape(-1).astype(np.float64)
-    want = want.reshape(-1).astype(np.float64)
-    err = np.max(np.abs(got - want))
+    want = want64.reshape(-1).astype(np.float64)
+    excess = np.abs(got - want) - half_ulp(want, dtype)
+    worst = int(np.argmax(excess))
     cos = float(got @ want / (np.linalg.norm(got) * np.linalg.norm(want) + 1e-300))
-    assert err <= MAX_ABS and cos >= MIN_COS, f"{what}: max abs {err:.3e}, cos {cos:.6f}"
-    return err, cos
+    assert excess[worst] <= MAX_ABS and cos >= MIN_COS, (
+        f"{what}: |err| - ulp/2 = {excess[worst]:.3e} at {worst} (got {got[worst]}, want "
+        f"{want[worst]}), cos {cos:.6f}")
+    return float(np.max(np.abs(got - want))), cos
 
 
 def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_off=3.0):
@@ -50,8 +64,7 @@ def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_
     r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had)
     got = out.cpu().reshape(B * N, H, d)
     gotf = got.double().numpy()
-    want = _to_f(orc, r["out"], dt)
-    _compare(gotf, want, "out")
+    _compare(gotf, r["out64"], "out", dtype)
     lse_want = r["lse"].reshape(H, B, N).transpose(1, 0, 2)
     assert np.max(np.abs(lse.cpu().numpy() - lse_want)) < 1e-2
     return gotf, qp, kp, vp, cu, dt
@@ -101,7 +114,7 @@ def test_varlen_parity(orc):
         assert ops.device_status(reset=True) == ops.OK
         r = orc.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), 1, cu, blk, True,
                             frac, use_ss=ss, use_had=had)
-        _compare(out.cpu().double().numpy(), _to_f(orc, r["out"], 1), f"varlen frac={frac}")
+        _compare(out.cpu().double().numpy(), r["out64"], f"varlen frac={frac}", torch.bfloat16)
         assert np.max(np.abs(lse.cpu().numpy() - r["lse"])) < 1e-2
 
 
