@@ -245,6 +245,27 @@ def quantizer_line(dev, peaks):
     return res
 
 
+def quantizer_only(args):
+    """A few plain (not graph-captured) quantiser calls on the quantiser
+    workload, ScaleSearch off then on; prints their event-timed durations."""
+    from bit_quantization_b200 import ops
+    dev = torch.device("cuda", 0)
+    x = synth.make_quant_input(synth.QUANT).to(dev)
+    res = {}
+    for ss in (False, True):
+        times = []
+        for _ in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ops.nvfp4_quantize(x, ss)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        res["ss_on" if ss else "ss_off"] = 1e3 * min(times[args.warmup:])
+    print(json.dumps({"mode": "quantizer", "workload": synth.QUANT.name, "us_min": res}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -255,11 +276,15 @@ def main():
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantizer", action="store_true")
+    ap.add_argument("--mode", default="attention", choices=["attention", "quantizer"],
+                    help="quantizer: only a few plain quantiser calls (profiling aid)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "quantizer":
+        return quantizer_only(args)
 
     from bit_quantization_b200 import ops
     world, rank, local = dist_setup(args)

@@ -107,6 +107,34 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
+// Eight fp32 values times c -> eight E2M1 codes packed in 32 bits (value
+// 2i in the low nibble of byte i).
+__device__ __forceinline__ uint32_t e2m1x8(const float* x, float c) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(x[0] * c), "f"(x[1] * c), "f"(x[2] * c), "f"(x[3] * c), "f"(x[4] * c),
+        "f"(x[5] * c), "f"(x[6] * c), "f"(x[7] * c));
+  return out;
+}
+
+// Two fp32 values -> packed 16-bit pair (lo in bits 0..15), nearest even.
+template <int DT>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (DT == 1) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
 // Waits with every lane of the warp; the result is uniform across the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -144,23 +172,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       mbar_init(&bars[i], cnt);
     }
     *s_abort = 0;
-    // Tile list: NVFP4 tiles ascending, then FP16 tiles ascending.
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    // Tile list: NVFP4 tiles ascending, then FP16 tiles ascending.  Entry:
+    // key tile j (bits 0..12), bit 13 + b set when query block b of this CTA
+    // (b = 0, 1; one block when BLK = 128) takes tile j on this path, bit 15
+    // the path (1 = FP16).  Built by one warp, 32 key tiles per step.
     const int qb0 = BLK == 128 ? qt : 2 * qt;
     const int nqb = BLK == 128 ? 1 : min(2, nb - 2 * qt);
     int n = 0;
     for (int pass = 0; pass < 2; ++pass) {
-      for (int j = 0; j < nb; ++j) {
-        bool need = false;
-        for (int b = qb0; b < qb0 + nqb; ++b) {
-          if (p.causal && j > b) continue;
-          if ((mrow[(int64_t)b * p.nB + j] != 0) == (pass == 1)) need = true;
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        uint32_t bits = 0;
+        if (j < nb) {
+          for (int b = 0; b < nqb; ++b) {
+            if (p.causal && j > qb0 + b) continue;
+            if ((__ldg(mrow + (int64_t)(qb0 + b) * p.nB + j) != 0) == (pass == 1))
+              bits |= 1u << (13 + b);
+          }
         }
-        if (need) s_list[n++] = (uint16_t)(j | (pass << 15));
+        const uint32_t vote = __ballot_sync(0xffffffffu, bits != 0);
+        if (bits) s_list[n + __popc(vote & ((1u << lane) - 1u))] = (uint16_t)(j | bits | (pass << 15));
+        n += __popc(vote);
       }
-      if (pass == 0) *s_n4 = n;
+      if (pass == 0 && lane == 0) *s_n4 = n;
     }
-    *s_n = n;
-    fence_mbar_init();
+    if (lane == 0) *s_n = n;
   }
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -189,7 +228,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       }
       for (int t = 0; t < n && !*s_abort; ++t) {
         const int st = t & 1;
-        const int j = s_list[t] & 0x7FFF;
+        const int j = s_list[t] & 0x1FFF;
         const bool f16 = (s_list[t] >> 15) != 0;
         if (t >= 2 && !mbar_wait(&bars[B_KVE + st], ((t >> 1) - 1) & 1, s_abort)) break;
         if (f16 && !q16_issued) {
@@ -319,38 +358,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     // half hf = w / 4 of the key columns (and of the output columns).
     constexpr int SC = BLK / 2;   // score columns per thread
     constexpr int OC = D / 2;     // output columns per thread
+    constexpr int NB = SC / 16;   // 16-key blocks per thread
     const int q4 = warp & 3, hf = warp >> 2;
     const int r = q4 * 32 + lane;
     const int row = qt * 128 + r;
     const bool row_ok = row < len;
-    const int qb = BLK == 128 ? qt : 2 * qt + (r >= 64 ? 1 : 0);
+    const int mbit = 13 + ((BLK == 64 && r >= 64) ? 1 : 0);  // tile-list bit of this row's block
     const float gq = tensor_scale_from_amax(p.amax[0]);
     const float gk = tensor_scale_from_amax(p.amax[1]);
     const float gv = tensor_scale_from_amax(p.amax[2]);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
     float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][2 halves][128]
+    // O holds the output divided by `ref`: the true accumulator is ref * O.
     float O[OC];
 #pragma unroll
     for (int c = 0; c < OC; ++c) O[c] = 0.0f;
+    float ref = 1.0f;
     float m = -INFINITY, l = 0.0f;
     float pend_alpha = 1.0f, pend_sigma = 0.0f;
     int pending = -1;
     bool prev16 = false;
     bool ok = true;
 
-    // O <- alpha * O + sigma * PV(u) for this thread's output columns.
+    // true O <- alpha * true O + sigma * PV(u), folded into one FMA per
+    // column by moving the reference factor to sigma.  Tiles whose sigma is
+    // negligible (< 2^-60 of the running maximum) only rescale.
     auto accumulate = [&](int u) -> bool {
       if (!warp_wait(&bars[B_OF], u & 1, s_abort)) return false;
       tc_fence_after();
+      const bool take = pend_sigma > 0.0f;
+      const float beta = take ? __fdiv_rn(pend_alpha * ref, pend_sigma) : 1.0f;
 #pragma unroll
       for (int c = 0; c < OC / 32; ++c) {
         float v[32];
         tmem_ld32(lane_base + L::T_PV + hf * OC + 32 * c, v);
         tmem_ld_wait();
+        if (take) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) O[32 * c + i] = fmaf(O[32 * c + i], pend_alpha, pend_sigma * v[i]);
+          for (int i = 0; i < 32; ++i) O[32 * c + i] = fmaf(O[32 * c + i], beta, v[i]);
+        }
       }
+      ref = take ? pend_sigma : ref * pend_alpha;
       tc_fence_before();
       mbar_arrive(&bars[B_OE]);
       return true;
@@ -358,11 +407,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
 
     for (int t = 0; t < n && ok; ++t) {
       const int st = t & 1;
-      const int j = s_list[t] & 0x7FFF;
-      const bool f16 = (s_list[t] >> 15) != 0;
-      const bool pair_ok = row_ok && qb < nb && (!p.causal || j <= qb) &&
-                           ((mrow[(int64_t)qb * p.nB + j] != 0) == f16);
-      // last valid score column of this thread's half (-1 or less: none)
+      const uint32_t ent = s_list[t];
+      const int j = ent & 0x1FFF;
+      const bool f16 = (ent >> 15) != 0;
+      const bool pair_ok = row_ok && ((ent >> mbit) & 1u);
+      // last valid score column of this thread's half (negative: none)
       const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - hf * SC;
       const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
       const float cs = f16 ? p.scale16 : cs4;
@@ -374,85 +423,101 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       }
       if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
-      float a[SC];
+      // pass 1: block maxima of the raw scores (the scale is positive, so
+      // the max of the scaled scores is the scaled max), 32 columns at a time
+      float bm[NB];
 #pragma unroll
-      for (int c = 0; c < SC / 32; ++c)
-        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c,
-                  *reinterpret_cast<float(*)[32]>(a + 32 * c));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
-      // scaled scores (log2 domain) and this half's row max
-      float mh = -INFINITY;
-      if (full) {
+      for (int c = 0; c < SC / 32; ++c) {
+        float a[32];
+        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c, a);
+        tmem_ld_wait();
+        if (!full) {
 #pragma unroll
-        for (int i = 0; i < SC; ++i) {
-          a[i] = __fmul_rn(a[i], cs);
-          mh = fmaxf(mh, a[i]);
+          for (int i = 0; i < 32; ++i) a[i] = 32 * c + i <= lim ? a[i] : -INFINITY;
         }
-      } else {
 #pragma unroll
-        for (int i = 0; i < SC; ++i) {
-          a[i] = i <= lim ? __fmul_rn(a[i], cs) : -INFINITY;
-          mh = fmaxf(mh, a[i]);
+        for (int bb = 0; bb < 2; ++bb) {
+          const float* x = a + 16 * bb;
+          float x0 = fmaxf(x[0], x[1]), x1 = fmaxf(x[2], x[3]);
+          float x2 = fmaxf(x[4], x[5]), x3 = fmaxf(x[6], x[7]);
+          x0 = fmaxf(x0, fmaxf(x[8], x[9]));
+          x1 = fmaxf(x1, fmaxf(x[10], x[11]));
+          x2 = fmaxf(x2, fmaxf(x[12], x[13]));
+          x3 = fmaxf(x3, fmaxf(x[14], x[15]));
+          bm[2 * c + bb] = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
         }
       }
+      float mh = bm[0];
+#pragma unroll
+      for (int b = 1; b < NB; ++b) mh = fmaxf(mh, bm[b]);
       float* xs = xch + st * 256;
       xs[hf * 128 + r] = mh;
       named_bar_sync(1 + q4, 64);
-      const float mt = fmaxf(xs[r], xs[128 + r]);
+      const float mt_raw = fmaxf(xs[r], xs[128 + r]);
+      const float mt = mt_raw * cs;
       const float m_new = fmaxf(m, mt);
-      const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(__fsub_rn(m, m_new));
-      const float rowmax = (mt == -INFINITY) ? 0.0f : ex2_ftz(__fsub_rn(mt, m_new));
-      const float msub = m_new == -INFINITY ? 0.0f : m_new;
+      const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(m - m_new);
+      const float negm = m_new == -INFINITY ? 0.0f : -m_new;
+      const float rowmax = (mt_raw == -INFINITY) ? 0.0f : ex2_ftz(fmaf(mt_raw, cs, negm));
       l *= alpha;
-      float lsum = 0.0f;
-#pragma unroll
-      for (int i = 0; i < SC; ++i) {
-        a[i] = ex2_ftz(__fsub_rn(a[i], msub));  // exp2(-inf) = 0 for masked columns
-        lsum += a[i];
-      }
-      l += lsum;
       m = m_new;
-      float sigma = 1.0f;
-      if (!f16) {
-        const float inv = rowmax > 0.0f ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
-        sigma = __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv);
-        uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+      // two-level quantisation of P: row factor rowmax/2688, NVFP4 blocks
+      const bool keep = rowmax >= 8.6736174e-19f;  // 2^-60
+      const float inv = (!f16 && keep) ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
+      const float sigma = f16 ? 1.0f : (keep ? __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv) : 0.0f);
+      uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+      uint8_t* p16 = sm + L::OFF_P16;
+      uint32_t sfw = 0;
+      float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      // pass 2: probabilities, 32 columns (two 16-key blocks) at a time
 #pragma unroll
-        for (int b = 0; b < SC / 16; ++b) {
-          float amax = 0.0f;
+      for (int c = 0; c < SC / 32; ++c) {
+        float a[32];
+        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c, a);
+        tmem_ld_wait();
+        if (!full) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            a[16 * b + e] = __fmul_rn(a[16 * b + e], inv);
-            amax = fmaxf(amax, a[16 * b + e]);
+          for (int i = 0; i < 32; ++i) a[i] = 32 * c + i <= lim ? a[i] : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          a[i] = ex2_ftz(fmaf(a[i], cs, negm));  // exp2(-inf) = 0 for masked columns
+          ls[i & 3] += a[i];
+        }
+        if (!f16) {
+          uint32_t cw[4];
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int b = 2 * c + bb;
+            const float pmax = bm[b] == -INFINITY ? 0.0f : ex2_ftz(fmaf(bm[b], cs, negm));
+            const uint32_t S = ue4m3(__fdiv_rn(__fmul_rn(pmax, inv), 6.0f));
+            const float cb = S ? __fmul_rn(inv, __frcp_rn(ue4m3_decode(S))) : 0.0f;
+            sfw |= S << (8 * b);
+            cw[2 * bb] = e2m1x8(a + 16 * bb, cb);
+            cw[2 * bb + 1] = e2m1x8(a + 16 * bb + 8, cb);
           }
-          const uint32_t S = ue4m3(__fdiv_rn(amax, 6.0f));
-          const float rr = S ? __frcp_rn(ue4m3_decode(S)) : 0.0f;
-          uint32_t cb[8];
+          *reinterpret_cast<uint4*>(p4 + swz_offset(r, (hf * NB + 2 * c) * 8, BLK / 2)) =
+              make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            cb[e] = e2m1x2(__fmul_rn(a[16 * b + 2 * e], rr), __fmul_rn(a[16 * b + 2 * e + 1], rr));
-          const uint32_t k16 = hf * (SC / 16) + b;
-          *reinterpret_cast<uint2*>(p4 + swz_offset(r, k16 * 8, BLK / 2)) =
-              make_uint2(cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24),
-                         cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24));
-          p4[128 * (BLK / 2) + sf_offset(r, k16)] = (uint8_t)S;
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w4[e] = pack2<DT>(a[8 * q8 + 2 * e], a[8 * q8 + 2 * e + 1]);
+            const uint32_t key0 = hf * SC + 32 * c + 8 * q8;
+            *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
+                                      swz_offset(r, (key0 % 64) * 2, 128)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
         }
-      } else {
-        uint8_t* p16 = sm + L::OFF_P16;
-#pragma unroll
-        for (int q8 = 0; q8 < SC / 8; ++q8) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w4[e] = (uint32_t)f2h<DT>(a[8 * q8 + 2 * e]) |
-                    ((uint32_t)f2h<DT>(a[8 * q8 + 2 * e + 1]) << 16);
-          const uint32_t key0 = hf * SC + 8 * q8;
-          *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
-                                    swz_offset(r, (key0 % 64) * 2, 128)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (!f16) {
+        uint8_t* sfp = p4 + 128 * (BLK / 2) + sf_offset(r, hf * NB);
+        if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(sfp) = sfw;
+        else *reinterpret_cast<uint16_t*>(sfp) = (uint16_t)sfw;
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_PF + st]);
@@ -471,15 +536,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     named_bar_sync(1 + q4, 64);
     const float lt = xl[r] + xl[128 + r];
     if (ok && row_ok) {
-      const float il = lt > 0.0f ? 1.0f / lt : 0.0f;
+      const float il = lt > 0.0f ? ref / lt : 0.0f;
       uint16_t* orow = p.out + ((start + row) * p.H + h) * D + hf * OC;
 #pragma unroll
       for (int c = 0; c < OC; c += 8) {
         uint4 w;
-        w.x = (uint32_t)f2h<DT>(O[c] * il) | ((uint32_t)f2h<DT>(O[c + 1] * il) << 16);
-        w.y = (uint32_t)f2h<DT>(O[c + 2] * il) | ((uint32_t)f2h<DT>(O[c + 3] * il) << 16);
-        w.z = (uint32_t)f2h<DT>(O[c + 4] * il) | ((uint32_t)f2h<DT>(O[c + 5] * il) << 16);
-        w.w = (uint32_t)f2h<DT>(O[c + 6] * il) | ((uint32_t)f2h<DT>(O[c + 7] * il) << 16);
+        w.x = pack2<DT>(O[c] * il, O[c + 1] * il);
+        w.y = pack2<DT>(O[c + 2] * il, O[c + 3] * il);
+        w.z = pack2<DT>(O[c + 4] * il, O[c + 5] * il);
+        w.w = pack2<DT>(O[c + 6] * il, O[c + 7] * il);
         *reinterpret_cast<uint4*>(orow + c) = w;
       }
       if (hf == 0) {

@@ -27,27 +27,69 @@ struct SeqInfo {
 };
 
 // ---------------------------------------------------------------- absmax --
-// Flat grid-stride loop over 16-element blocks of x (n_blocks of them).  G
-// lanes hold one row when rows are rotated (G = d/16), G = 0 for no rotation.
+
+// CTA-wide max of one value per thread; thread 0 then does one atomicMax on
+// the bit pattern of the (non-negative) result.
+__device__ __forceinline__ void cta_atomic_amax(float a, uint32_t* dst) {
+  __shared__ float red[32];
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+    if (threadIdx.x == 0 && a > 0.0f) atomicMax(dst, __float_as_uint(a));
+  }
+}
+
+// Loads the 32-byte block b (or zeros past the end) as raw 16-bit pairs.
+__device__ __forceinline__ void load_raw(const uint16_t* x, int64_t b, int64_t n_blocks,
+                                         uint4& r0, uint4& r1) {
+  if (b < n_blocks) {
+    r0 = __ldg(reinterpret_cast<const uint4*>(x + b * 16));
+    r1 = __ldg(reinterpret_cast<const uint4*>(x + b * 16) + 1);
+  } else {
+    r0 = r1 = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ void unpack16(const uint4& r0, const uint4& r1, float (&v)[16]) {
+  const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = h2f<DT>((uint16_t)(w[i] & 0xFFFF));
+    v[2 * i + 1] = h2f<DT>((uint16_t)(w[i] >> 16));
+  }
+}
+
+// Grid-stride absmax over 16-element blocks of x, KPT blocks in flight per
+// thread.  G lanes hold one row when rows are rotated (G = d/16), G = 0 for
+// no rotation.
+constexpr int kKPT = 4;
+
 template <int DT, int G>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x,
                                                    int64_t n_blocks, uint32_t* amax_out) {
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31;
   float a = 0.0f;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-       base < n_blocks; base += nthreads) {
-    const int64_t b = base + (threadIdx.x & 31);
-    float v[16];
-    if (b < n_blocks) {
-      load16<DT>(x + b * 16, v);
-    } else {
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n_blocks;
+       base += nthreads * kKPT) {
+    uint4 r[kKPT][2];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+    for (int k = 0; k < kKPT; ++k) load_raw(x, base + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+#pragma unroll
+    for (int k = 0; k < kKPT; ++k) {
+      float v[16];
+      unpack16<DT>(r[k][0], r[k][1], v);
+      if constexpr (G > 0) fwht_rows16<G>(v);
+      a = fmaxf(a, block_absmax(v));
     }
-    if constexpr (G > 0) fwht_rows16<G>(v);
-    a = fmaxf(a, block_absmax(v));
   }
-  warp_atomic_amax(a, amax_out);
+  cta_atomic_amax(a, amax_out);
 }
 
 // ------------------------------------------------- row-blocked quantiser --
@@ -60,16 +102,87 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   const float g = scale_given ? *tensor_scale : tensor_scale_from_amax(*amax_in);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-       base < n_blocks; base += nthreads) {
-    const int64_t b = base + (threadIdx.x & 31);
-    float v[16];
-    if (b < n_blocks) {
-      load16<DT>(x + b * 16, v);
-    } else {
+  const int64_t wbase0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = wbase0; base < n_blocks; base += nthreads * kKPT) {
+    uint4 r[kKPT][2];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+    for (int k = 0; k < kKPT; ++k) load_raw(x, base + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+#pragma unroll
+    for (int k = 0; k < kKPT; ++k) {
+      const int64_t b = base + lane + k * nthreads;
+      float v[16];
+      unpack16<DT>(r[k][0], r[k][1], v);
+      if constexpr (G > 0) fwht_rows16<G>(v);
+      if (b < n_blocks) {
+        uint32_t lo, hi;
+        const uint32_t S = quant_block16(v, g, SS, lo, hi);
+        *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
+        scales[b] = (uint8_t)S;
+      }
     }
+  }
+}
+
+// Single-pass quantiser: every thread stages kFusedKPT blocks in shared
+// memory, the grid agrees on the tensor absmax through one atomicMax per CTA
+// and a grid barrier, then quantises from shared memory, so x is read from
+// HBM once.  Launched cooperatively with a grid that covers the tensor in one
+// sweep (n_blocks <= threads * kFusedKPT).  sync[0] = absmax bits, sync[1] =
+// arrival counter, both zero at launch.  The barrier wait is bounded; on
+// timeout the device status word is set and the blocks are quantised with
+// the absmax seen so far.
+constexpr int kFusedKPT = 8;
+constexpr int kFusedSmem = kFusedKPT * 256 * 32;
+
+template <int DT, int G, bool SS>
+__global__ void __launch_bounds__(256) quant_rows_fused_kernel(
+    const uint16_t* __restrict__ x, int64_t n_blocks, uint32_t* sync, float* tensor_scale,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  extern __shared__ uint4 stage[];  // [kFusedKPT][256 threads][2]
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  float a = 0.0f;
+#pragma unroll
+  for (int k0 = 0; k0 < kFusedKPT; k0 += 4) {
+    uint4 r[4][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) load_raw(x, b0 + (k0 + k) * nthreads, n_blocks, r[k][0], r[k][1]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      stage[((k0 + k) * 256 + threadIdx.x) * 2] = r[k][0];
+      stage[((k0 + k) * 256 + threadIdx.x) * 2 + 1] = r[k][1];
+      float v[16];
+      unpack16<DT>(r[k][0], r[k][1], v);
+      if constexpr (G > 0) fwht_rows16<G>(v);
+      a = fmaxf(a, block_absmax(v));
+    }
+  }
+  cta_atomic_amax(a, &sync[0]);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(&sync[1], 1u);
+    const uint64_t t_start = globaltimer_ns();
+    uint32_t seen = 0;
+    for (uint32_t it = 0;; ++it) {
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(&sync[1]) : "memory");
+      if (seen >= gridDim.x) break;
+      if ((it & 63) == 63 && globaltimer_ns() - t_start > 1000000000ull) {
+        set_device_status(THRIFT_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  uint32_t amax_bits;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(&sync[0]) : "memory");
+  const float g = tensor_scale_from_amax(amax_bits);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+#pragma unroll 2
+  for (int k = 0; k < kFusedKPT; ++k) {
+    const int64_t b = b0 + k * nthreads;
+    float v[16];
+    unpack16<DT>(stage[(k * 256 + threadIdx.x) * 2], stage[(k * 256 + threadIdx.x) * 2 + 1], v);
     if constexpr (G > 0) fwht_rows16<G>(v);
     if (b < n_blocks) {
       uint32_t lo, hi;

@@ -43,10 +43,30 @@ struct Carve {
 
 // ------------------------------------------------------- quantiser glue --
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Grid for the streaming kernels: enough CTAs for kKPT blocks per thread,
+// at most four resident CTAs per SM (grid-stride beyond that).
+int stream_grid(int64_t n_blocks) {
+  int64_t g = ceil_div(n_blocks, (int64_t)kThreads * kKPT);
+  if (g < 1) g = 1;
+  if (g > 4LL * sm_count()) g = 4LL * sm_count();
+  return (int)g;
+}
+
 template <int DT>
 void launch_amax(const void* x, int64_t n_blocks, int G, uint32_t* out, cudaStream_t st) {
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  const int grid = grid_for(n_blocks);
+  const int grid = stream_grid(n_blocks);
   if (G == 8) amax_kernel<DT, 8><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
   else if (G == 4) amax_kernel<DT, 4><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
   else amax_kernel<DT, 0><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
@@ -55,23 +75,73 @@ void launch_amax(const void* x, int64_t n_blocks, int G, uint32_t* out, cudaStre
 template <int DT, int G, bool SS>
 void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, int given,
                          uint8_t* codes, uint8_t* scales, cudaStream_t st) {
-  quant_rows_kernel<DT, G, SS><<<grid_for(nb), kThreads, 0, st>>>(
+  quant_rows_kernel<DT, G, SS><<<stream_grid(nb), kThreads, 0, st>>>(
       static_cast<const uint16_t*>(x), nb, amax, ts, given, codes, scales);
 }
 
-template <int DT>
-void launch_quant_rows(const void* x, int64_t nb, int G, bool ss, uint32_t* amax, float* ts,
-                       int given, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
-  if (G == 8) {
-    if (ss) launch_quant_rows_t<DT, 8, true>(x, nb, amax, ts, given, codes, scales, st);
-    else launch_quant_rows_t<DT, 8, false>(x, nb, amax, ts, given, codes, scales, st);
-  } else if (G == 4) {
-    if (ss) launch_quant_rows_t<DT, 4, true>(x, nb, amax, ts, given, codes, scales, st);
-    else launch_quant_rows_t<DT, 4, false>(x, nb, amax, ts, given, codes, scales, st);
-  } else {
-    if (ss) launch_quant_rows_t<DT, 0, true>(x, nb, amax, ts, given, codes, scales, st);
-    else launch_quant_rows_t<DT, 0, false>(x, nb, amax, ts, given, codes, scales, st);
+// Single-pass quantiser (absmax agreed through a grid barrier) when one
+// resident grid covers the tensor with kFusedKPT blocks per thread; returns
+// false (nothing launched) when it does not.
+template <int DT, int G, bool SS>
+bool launch_quant_fused_t(const void* x, int64_t nb, uint32_t* sync, float* ts, uint8_t* codes,
+                          uint8_t* scales, cudaStream_t st, thrift_status* status) {
+  static int per_sm = -1;
+  if (per_sm < 0) {
+    per_sm = 0;
+    if (cudaFuncSetAttribute(quant_rows_fused_kernel<DT, G, SS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) ==
+            cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, quant_rows_fused_kernel<DT, G, SS>, kThreads, kFusedSmem) != cudaSuccess)
+      per_sm = 0;
   }
+  const int64_t need = ceil_div(nb, (int64_t)kThreads * kFusedKPT);
+  if (per_sm <= 0 || need > (int64_t)per_sm * sm_count()) return false;
+  if (cudaMemsetAsync(sync, 0, 8, st) != cudaSuccess) {
+    *status = THRIFT_ERR_CUDA;
+    return true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)need);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kFusedSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  *status = cudaLaunchKernelEx(&cfg, quant_rows_fused_kernel<DT, G, SS>, xp, nb, sync, ts, codes,
+                               scales) == cudaSuccess
+                ? THRIFT_OK
+                : THRIFT_ERR_CUDA;
+  return true;
+}
+
+template <int DT>
+thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_t* sync,
+                              float* ts, int given, uint8_t* codes, uint8_t* scales,
+                              cudaStream_t st) {
+#define THRIFT_QUANT_CASE(GG, SSV)                                                        \
+  if (G == GG && ss == SSV) {                                                              \
+    if (!given) {                                                                          \
+      thrift_status s = THRIFT_OK;                                                         \
+      if (launch_quant_fused_t<DT, GG, SSV>(x, nb, sync, ts, codes, scales, st, &s)) return s; \
+      if (cudaMemsetAsync(sync, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;          \
+      launch_amax<DT>(x, nb, GG, sync, st);                                                \
+    }                                                                                      \
+    launch_quant_rows_t<DT, GG, SSV>(x, nb, sync, ts, given, codes, scales, st);           \
+    return launch_status();                                                                \
+  }
+  THRIFT_QUANT_CASE(0, false)
+  THRIFT_QUANT_CASE(0, true)
+  THRIFT_QUANT_CASE(4, false)
+  THRIFT_QUANT_CASE(4, true)
+  THRIFT_QUANT_CASE(8, false)
+  THRIFT_QUANT_CASE(8, true)
+#undef THRIFT_QUANT_CASE
+  return THRIFT_ERR_UNSUPPORTED;
 }
 
 // ----------------------------------------------------- attention layout --
@@ -303,21 +373,14 @@ thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64
       (reinterpret_cast<uintptr_t>(codes) & 7))
     return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  uint32_t* sync = static_cast<uint32_t*>(workspace);
   const int64_t nb = rows * cols / 16;
   const int G = use_hadamard ? (int)(cols / 16) : 0;
-  if (!tensor_scale_given) {
-    if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
-    if (dt == THRIFT_BF16) launch_amax<1>(x, nb, G, amax, st);
-    else launch_amax<0>(x, nb, G, amax, st);
-  }
   if (dt == THRIFT_BF16)
-    launch_quant_rows<1>(x, nb, G, use_scalesearch != 0, amax, tensor_scale, tensor_scale_given,
-                         codes, scales, st);
-  else
-    launch_quant_rows<0>(x, nb, G, use_scalesearch != 0, amax, tensor_scale, tensor_scale_given,
-                         codes, scales, st);
-  return launch_status();
+    return launch_quantize<1>(x, nb, G, use_scalesearch != 0, sync, tensor_scale,
+                              tensor_scale_given, codes, scales, st);
+  return launch_quantize<0>(x, nb, G, use_scalesearch != 0, sync, tensor_scale,
+                            tensor_scale_given, codes, scales, st);
 }
 
 thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t rows,
@@ -342,7 +405,7 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
     else launch_amax<0>(x, rows * cols / 16, 0, amax, st);
   }
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  const int grid = grid_for((rows / 16) * cols);
+  const int grid = stream_grid((rows / 16) * cols / kKPT + 1);
   if (dt == THRIFT_BF16) {
     if (use_scalesearch)
       quant_cols_kernel<1, true><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,

@@ -102,3 +102,10 @@ def test_empty_rows():
     x = torch.zeros((0, 128), dtype=torch.float16, device="cuda")
     codes, scales, ts = ops.nvfp4_quantize(x)
     assert codes.shape == (0, 64)
+
+
+def test_two_pass_path_large_tensor(orc):
+    # 2^21 x 16 = 33.5M elements exceeds one resident grid of the single-pass
+    # kernel, so the absmax pass and the quantise pass run separately.
+    x = synth.randn16((1 << 21, 16), torch.bfloat16, seed=21)
+    _check_rows(orc, x, False, False)
