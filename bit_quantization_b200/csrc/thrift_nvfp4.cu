@@ -3,6 +3,7 @@
 // point are in include/thrift_nvfp4.h.
 #include <cmath>
 #include <cstdio>
+#include <mutex>
 #include <utility>
 #include <vector>
 
@@ -305,6 +306,28 @@ thrift_status check_attn_args(const void* q, const void* k, const void* v, int d
   return THRIFT_OK;
 }
 
+// Fixed scratch of block_mean_topk_noalloc.  In host code the array's name
+// is only a stand-in; its device address is looked up once per device (with
+// that device current) and cached.
+constexpr size_t kNoAllocScratchBytes = THRIFT_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+thrift_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return THRIFT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return THRIFT_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return THRIFT_OK;
+}
+
 }  // namespace
 }  // namespace thrift
 
@@ -319,6 +342,7 @@ const char* thrift_status_string(int s) {
     case THRIFT_ERR_UNSUPPORTED: return "unsupported";
     case THRIFT_ERR_CUDA: return "CUDA error";
     case THRIFT_ERR_TIMEOUT: return "device wait timed out";
+    case THRIFT_ERR_SCRATCH: return "problem exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
@@ -461,6 +485,20 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
   pair_scores_kernel<<<grid_for((int64_t)B * H * nB * nB), kThreads, 0, st>>>(mq, mk, si, B, H, Hkv, d, blk, nB, sc);
   topk_kernel<<<B * H, kTopkThreads, 0, st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
   return launch_status();
+}
+
+thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype dt, int B,
+                                      int H, int Hkv, int N, int d, int blk, int causal,
+                                      float topk_frac, uint8_t* mask, void* stream) {
+  if (!q || !k || !mask) return THRIFT_ERR_ARG;
+  const size_t need = block_mean_topk_workspace_size(B, H, Hkv, N, d, blk);
+  if (need == 0) return THRIFT_ERR_ARG;
+  if (need > kNoAllocScratchBytes) return THRIFT_ERR_SCRATCH;
+  void* scratch = nullptr;
+  const thrift_status s = noalloc_scratch(&scratch);
+  if (s != THRIFT_OK) return s;
+  return block_mean_topk(q, k, dt, B, H, Hkv, N, d, blk, causal, topk_frac, mask, scratch,
+                         kNoAllocScratchBytes, stream);
 }
 
 size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk) {

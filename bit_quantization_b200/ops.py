@@ -15,7 +15,8 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libthrift_nvfp4.so")
 
-OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH = 0, -1, -2, -3, -4, -5
+NOALLOC_SCRATCH_BYTES = 8 << 20
 F16, BF16 = 0, 1
 
 _lib = None
@@ -24,7 +25,7 @@ _lib = None
 EXPORTS = (
     "thrift_status_string", "thrift_device_status", "nvfp4_quantize_workspace_size",
     "nvfp4_quantize", "nvfp4_quantize_colblocks", "block_mean_topk_workspace_size",
-    "block_mean_topk", "thrift_attn_workspace_size", "thrift_attn_fwd",
+    "block_mean_topk", "block_mean_topk_noalloc", "thrift_attn_workspace_size", "thrift_attn_fwd",
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
     "thrift_kernel_timer_enable", "thrift_kernel_timer_read",
 )
@@ -57,6 +58,8 @@ def lib():
         L.block_mean_topk_workspace_size.argtypes = [i32] * 6
         L.block_mean_topk.restype = i32
         L.block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P, sz, P]
+        L.block_mean_topk_noalloc.restype = i32
+        L.block_mean_topk_noalloc.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P]
         L.thrift_attn_workspace_size.restype = sz
         L.thrift_attn_workspace_size.argtypes = [i32] * 6
         L.thrift_attn_fwd.restype = i32
@@ -195,6 +198,23 @@ def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, to
     _check(lib().block_mean_topk(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk, int(causal),
                                  float(topk_frac), _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
            "block_mean_topk")
+    return mask
+
+
+def block_mean_topk_noalloc(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool,
+                            topk_frac: float, mask: Optional[torch.Tensor] = None):
+    """block_mean_topk with the library's fixed scratch instead of a workspace,
+    for callers that cannot allocate device memory (see the header).  Pass
+    `mask` to avoid the one allocation this wrapper would otherwise make."""
+    _need_cuda(q, k)
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    nB = (N + blk - 1) // blk
+    if mask is None:
+        mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
+    _check(lib().block_mean_topk_noalloc(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk,
+                                         int(causal), float(topk_frac), _ptr(mask), _stream(q)),
+           "block_mean_topk_noalloc")
     return mask
 
 

@@ -51,7 +51,8 @@ typedef enum {
   THRIFT_ERR_ARG = -1,          /* bad pointer, size or flag */
   THRIFT_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle */
   THRIFT_ERR_CUDA = -3,         /* a CUDA runtime call failed */
-  THRIFT_ERR_TIMEOUT = -4       /* a device-side wait gave up */
+  THRIFT_ERR_TIMEOUT = -4,      /* a device-side wait gave up */
+  THRIFT_ERR_SCRATCH = -5       /* problem too large for a fixed scratch area */
 } thrift_status;
 
 typedef enum { THRIFT_F16 = 0, THRIFT_BF16 = 1 } thrift_dtype;
@@ -125,6 +126,26 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, N >= 1,
  * 0 <= topk_frac <= 1, nB = ceil(N/blk) <= 512.
  */
+/* Same selection without a workspace argument.  For callers that cannot
+ * allocate device memory: for example code that runs while a CUDA graph is
+ * being captured (cudaMalloc is not allowed there), or a plug-in handed only
+ * tensors and a stream by a host framework that owns all device memory.  The
+ * scratch (block means and pair scores) lives in one fixed array of
+ * THRIFT_NOALLOC_SCRATCH_BYTES in this library's device memory, held on every
+ * device that loads the library until the process exits; nothing in it has
+ * to start at zero.  The first call on a device looks up that array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Calls that overlap on the GPU share the
+ * array and race: issue them on one stream, or otherwise serialise them.
+ * Returns THRIFT_ERR_SCRATCH, launching nothing, when
+ * block_mean_topk_workspace_size(...) exceeds THRIFT_NOALLOC_SCRATCH_BYTES.
+ * Other arguments and results as block_mean_topk.  The method has no
+ * counterpart of this entry point; it only changes where scratch lives. */
+#define THRIFT_NOALLOC_SCRATCH_BYTES (8u << 20)
+thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype dt, int B,
+                                      int H, int Hkv, int N, int d, int blk, int causal,
+                                      float topk_frac, uint8_t* mask, void* stream);
+
 size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
                               int B, int H, int Hkv, int N, int d, int blk, int causal,
