@@ -11,13 +11,13 @@
 // quantised in two levels (per row and key tile an fp32 factor rowmax/2688,
 // then NVFP4 16-key blocks).
 //
-// Roles (320 threads):
-//   warps 0-7  softmax + output: query row r (TMEM lane r) is shared by warps
-//              r/32 and r/32 + 4, each owning half of the key columns and
-//              half of the output columns; the two exchange their partial row
-//              max once per tile through shared memory;
-//   warp 8     producer: bulk copies of the pre-quantised tile images;
-//   warp 9     tensor-memory owner and MMA issuer (one elected lane).
+// Roles (576 threads):
+//   warps 0-15 softmax + output: query row r (TMEM lane r) is shared by the
+//              four warps r/32 + 4f (f = 0..3), each owning a quarter of the
+//              key columns and of the output columns; they exchange their
+//              partial row max once per tile through shared memory;
+//   warp 16    producer: bulk copies of the pre-quantised tile images;
+//   warp 17    tensor-memory owner and MMA issuer (one elected lane).
 // Tensor memory (512 columns): S double buffer [2][BLK], PV [D], then the
 // scale factors of Q, K (x2), P (x2) and V (x2).
 // Every wait is bounded; a wait that gives up sets the device status word
@@ -71,7 +71,7 @@ struct AttnLayout {
   static constexpr uint32_t MAX_TILES = 512;  // key tiles per sequence
   static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
   static constexpr uint32_t OFF_XCH = OFF_BAR + 256;  // row-max / row-sum exchange
-  static constexpr uint32_t BYTES = OFF_XCH + 4 * 2 * 2 * 128 + 4 * 2 * 128;
+  static constexpr uint32_t BYTES = OFF_XCH + 4 * 2 * 4 * 128;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
   // tensor-memory columns
   static constexpr uint32_t T_S = 0;
@@ -91,7 +91,7 @@ enum : int {
   B_SE = 8 /* 8,9 */, B_PF = 10 /* 10,11 */, B_OF = 12, B_OE = 13, B_DONE = 14, B_N = 15
 };
 
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxWarps = 16;
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;
@@ -101,15 +101,53 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ float lg2_ftz(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// UE4M3 byte (0..126) -> value, with the subnormal case (m * 2^-9) formed by
+// the 2^23 magic-number conversion instead of an integer-to-float convert.
+__device__ __forceinline__ float ue4m3_decode_fast(uint32_t b) {
+  const uint32_t e = b >> 3, mt = b & 7u;
+  const float sub = (__uint_as_float(0x4B000000u | mt) - 8388608.0f) * 0.001953125f;
+  return e ? __uint_as_float(((e + 120u) << 23) | (mt << 20)) : sub;
+}
+
+__device__ __forceinline__ float rcp_ftz(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe, for x in [-125, 0]: x = n + f with n the nearest
+// integer (rounded by adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a
+// degree-6 polynomial interpolating 2^f at the Chebyshev nodes of
+// [-1/2, 1/2] (max relative error 8.2e-8); 2^n added to the exponent field.
+__device__ __forceinline__ float exp2_fma(float x) {
+  const float t = __fadd_rn(x, 12582912.0f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float fr = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+  float q = 1.5461444854736328e-04f;
+  q = fmaf(q, fr, 1.3400427997112274e-03f);
+  q = fmaf(q, fr, 9.6180569380521774e-03f);
+  q = fmaf(q, fr, 5.5503271520137787e-02f);
+  q = fmaf(q, fr, 2.4022650718688965e-01f);
+  q = fmaf(q, fr, 6.9314718246459961e-01f);
+  q = fmaf(q, fr, 1.0f);
+  return __int_as_float(__float_as_int(q) + (n << 23));
+}
+
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// Eight fp32 values times c -> eight E2M1 codes packed in 32 bits (value
-// 2i in the low nibble of byte i).
-__device__ __forceinline__ uint32_t e2m1x8(const float* x, float c) {
+// Eight fp32 values -> eight E2M1 codes packed in 32 bits (value 2i in the
+// low nibble of byte i), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e2m1x8(const float* x) {
   uint32_t out;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -118,8 +156,8 @@ __device__ __forceinline__ uint32_t e2m1x8(const float* x, float c) {
       "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(out)
-      : "f"(x[0] * c), "f"(x[1] * c), "f"(x[2] * c), "f"(x[3] * c), "f"(x[4] * c),
-        "f"(x[5] * c), "f"(x[6] * c), "f"(x[7] * c));
+      : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]),
+        "f"(x[7]));
   return out;
 }
 
@@ -354,12 +392,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     }
   } else {
     // -------------------------------------------------------- softmax --
-    // Two threads per query row: warp w owns TMEM lane quarter w % 4 and
-    // half hf = w / 4 of the key columns (and of the output columns).
-    constexpr int SC = BLK / 2;   // score columns per thread
-    constexpr int OC = D / 2;     // output columns per thread
+    // Four threads per query row: warp w owns TMEM lane quarter w % 4 and
+    // column quarter f = w / 4 of the key columns and of the output columns.
+    constexpr int SC = BLK / 4;   // score columns per thread
+    constexpr int OC = D / 4;     // output columns per thread
     constexpr int NB = SC / 16;   // 16-key blocks per thread
-    const int q4 = warp & 3, hf = warp >> 2;
+    const int q4 = warp & 3, f = warp >> 2;
     const int r = q4 * 32 + lane;
     const int row = qt * 128 + r;
     const bool row_ok = row < len;
@@ -369,39 +407,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     const float gv = tensor_scale_from_amax(p.amax[2]);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-    float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][2 halves][128]
+    float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][4 quarters][128]
     // O holds the output divided by `ref`: the true accumulator is ref * O.
     float O[OC];
 #pragma unroll
     for (int c = 0; c < OC; ++c) O[c] = 0.0f;
     float ref = 1.0f;
     float m = -INFINITY, l = 0.0f;
-    float pend_alpha = 1.0f, pend_sigma = 0.0f;
+    float pend_alpha = 1.0f, pend_sigma = 0.0f, pend_sigma_next = 0.0f;
     int pending = -1;
     bool prev16 = false;
     bool ok = true;
 
-    // true O <- alpha * true O + sigma * PV(u), folded into one FMA per
-    // column by moving the reference factor to sigma.  Tiles whose sigma is
-    // negligible (< 2^-60 of the running maximum) only rescale.
+    // true O <- alpha * true O + sigma * PV(u), one FMA per column: the
+    // reference factor moves to sigma.  Tiles whose sigma is negligible
+    // (< 2^-60 of the running maximum) only rescale.
     auto accumulate = [&](int u) -> bool {
       if (!warp_wait(&bars[B_OF], u & 1, s_abort)) return false;
       tc_fence_after();
-      const bool take = pend_sigma > 0.0f;
-      const float beta = take ? __fdiv_rn(pend_alpha * ref, pend_sigma) : 1.0f;
-#pragma unroll
-      for (int c = 0; c < OC / 32; ++c) {
-        float v[32];
-        tmem_ld32(lane_base + L::T_PV + hf * OC + 32 * c, v);
-        tmem_ld_wait();
-        if (take) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) O[32 * c + i] = fmaf(O[32 * c + i], beta, v[i]);
-        }
-      }
-      ref = take ? pend_sigma : ref * pend_alpha;
+      float v[OC];
+      tmem_ld_cols<OC>(lane_base + L::T_PV + f * OC, v);
+      tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars[B_OE]);
+      const bool take = pend_sigma > 0.0f;
+      const float beta = take ? pend_alpha * ref * rcp_ftz(pend_sigma) : 1.0f;
+      if (take) {
+#pragma unroll
+        for (int i = 0; i < OC; ++i) O[i] = fmaf(O[i], beta, v[i]);
+      }
+      ref = take ? pend_sigma : ref * pend_alpha;
       return true;
     };
 
@@ -411,8 +446,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const int j = ent & 0x1FFF;
       const bool f16 = (ent >> 15) != 0;
       const bool pair_ok = row_ok && ((ent >> mbit) & 1u);
-      // last valid score column of this thread's half (negative: none)
-      const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - hf * SC;
+      // last valid score column of this thread's quarter (negative: none)
+      const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - f * SC;
       const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
       const float cs = f16 ? p.scale16 : cs4;
       // FP16 tiles share one P buffer: the previous FP16 PV must be done
@@ -423,101 +458,107 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       }
       if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: block maxima of the raw scores (the scale is positive, so
-      // the max of the scaled scores is the scaled max), 32 columns at a time
+      float a[SC];
+      tmem_ld_cols<SC>(lane_base + L::T_S + st * BLK + f * SC, a);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
+      if (!full) {
+#pragma unroll
+        for (int i = 0; i < SC; ++i) a[i] = i <= lim ? a[i] : -INFINITY;
+      }
+      // block maxima of the raw scores (the scale is positive, so the max of
+      // the scaled scores is the scaled max)
       float bm[NB];
 #pragma unroll
-      for (int c = 0; c < SC / 32; ++c) {
-        float a[32];
-        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c, a);
-        tmem_ld_wait();
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = 32 * c + i <= lim ? a[i] : -INFINITY;
-        }
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const float* x = a + 16 * bb;
-          float x0 = fmaxf(x[0], x[1]), x1 = fmaxf(x[2], x[3]);
-          float x2 = fmaxf(x[4], x[5]), x3 = fmaxf(x[6], x[7]);
-          x0 = fmaxf(x0, fmaxf(x[8], x[9]));
-          x1 = fmaxf(x1, fmaxf(x[10], x[11]));
-          x2 = fmaxf(x2, fmaxf(x[12], x[13]));
-          x3 = fmaxf(x3, fmaxf(x[14], x[15]));
-          bm[2 * c + bb] = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-        }
+      for (int b = 0; b < NB; ++b) {
+        const float* x = a + 16 * b;
+        float x0 = fmaxf(x[0], x[1]), x1 = fmaxf(x[2], x[3]);
+        float x2 = fmaxf(x[4], x[5]), x3 = fmaxf(x[6], x[7]);
+        x0 = fmaxf(x0, fmaxf(x[8], x[9]));
+        x1 = fmaxf(x1, fmaxf(x[10], x[11]));
+        x2 = fmaxf(x2, fmaxf(x[12], x[13]));
+        x3 = fmaxf(x3, fmaxf(x[14], x[15]));
+        bm[b] = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
       }
       float mh = bm[0];
 #pragma unroll
       for (int b = 1; b < NB; ++b) mh = fmaxf(mh, bm[b]);
-      float* xs = xch + st * 256;
-      xs[hf * 128 + r] = mh;
-      named_bar_sync(1 + q4, 64);
-      const float mt_raw = fmaxf(xs[r], xs[128 + r]);
+      float* xs = xch + st * 512;
+      xs[f * 128 + r] = mh;
+      named_bar_sync(1 + q4, 128);
+      const float mt_raw = fmaxf(fmaxf(xs[r], xs[128 + r]), fmaxf(xs[256 + r], xs[384 + r]));
       const float mt = mt_raw * cs;
       const float m_new = fmaxf(m, mt);
       const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(m - m_new);
-      const float negm = m_new == -INFINITY ? 0.0f : -m_new;
-      const float rowmax = (mt_raw == -INFINITY) ? 0.0f : ex2_ftz(fmaf(mt_raw, cs, negm));
+      const bool live = mt_raw != -INFINITY;  // this row has a valid key in the tile
+      const float rowmax = live ? ex2_ftz(mt - m_new) : 0.0f;
       l *= alpha;
       m = m_new;
-      // two-level quantisation of P: row factor rowmax/2688, NVFP4 blocks
-      const bool keep = rowmax >= 8.6736174e-19f;  // 2^-60
-      const float inv = (!f16 && keep) ? __fdiv_rn(2688.0f, rowmax) : 0.0f;
-      const float sigma = f16 ? 1.0f : (keep ? __fmul_rn(__fdiv_rn(rowmax, 2688.0f), gv) : 0.0f);
-      uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
-      uint8_t* p16 = sm + L::OFF_P16;
-      uint32_t sfw = 0;
-      float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      // pass 2: probabilities, 32 columns (two 16-key blocks) at a time
-#pragma unroll
-      for (int c = 0; c < SC / 32; ++c) {
-        float a[32];
-        tmem_ld32(lane_base + L::T_S + st * BLK + hf * SC + 32 * c, a);
-        tmem_ld_wait();
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = 32 * c + i <= lim ? a[i] : -INFINITY;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          a[i] = ex2_ftz(fmaf(a[i], cs, negm));  // exp2(-inf) = 0 for masked columns
-          ls[i & 3] += a[i];
-        }
-        if (!f16) {
-          uint32_t cw[4];
-#pragma unroll
-          for (int bb = 0; bb < 2; ++bb) {
-            const int b = 2 * c + bb;
-            const float pmax = bm[b] == -INFINITY ? 0.0f : ex2_ftz(fmaf(bm[b], cs, negm));
-            const uint32_t S = ue4m3(__fdiv_rn(__fmul_rn(pmax, inv), 6.0f));
-            const float cb = S ? __fmul_rn(inv, __frcp_rn(ue4m3_decode(S))) : 0.0f;
-            sfw |= S << (8 * b);
-            cw[2 * bb] = e2m1x8(a + 16 * bb, cb);
-            cw[2 * bb + 1] = e2m1x8(a + 16 * bb + 8, cb);
-          }
-          *reinterpret_cast<uint4*>(p4 + swz_offset(r, (hf * NB + 2 * c) * 8, BLK / 2)) =
-              make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        } else {
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) w4[e] = pack2<DT>(a[8 * q8 + 2 * e], a[8 * q8 + 2 * e + 1]);
-            const uint32_t key0 = hf * SC + 32 * c + 8 * q8;
-            *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
-                                      swz_offset(r, (key0 % 64) * 2, 128)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float ls = 0.0f;
       if (!f16) {
-        uint8_t* sfp = p4 + 128 * (BLK / 2) + sf_offset(r, hf * NB);
-        if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(sfp) = sfw;
-        else *reinterpret_cast<uint16_t*>(sfp) = (uint16_t)sfw;
+        // Two-level quantisation of P.  Relative to the tile max the scaled
+        // probabilities are Phat = 2688 * 2^(s - mt) (row factor
+        // sigma = rowmax / 2688); block b gets the UE4M3 scale
+        // S_b = ue4m3(max Phat / 6) and the codes E2M1(Phat / S_b), computed
+        // as one exponential t = 2^(s + log2(2688) - mt - log2 S_b).
+        // l gets sum_b S_b * sum(t) * rowmax / 2688.
+        const bool keep = live && rowmax >= 8.6736174e-19f;  // 2^-60
+        const float sigma_raw = keep ? rowmax * (1.0f / 2688.0f) : 0.0f;
+        const float sigma = sigma_raw * gv;
+        uint32_t sfw = 0;
+        uint32_t cw[2 * NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
+          const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
+          const float dec = ue4m3_decode_fast(S);
+          const float c = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
+          float bs[2] = {0.0f, 0.0f};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            a[16 * b + i] = ex2_ftz(fmaf(a[16 * b + i], cs, c));
+            bs[i & 1] += a[16 * b + i];
+          }
+          ls = fmaf(bs[0] + bs[1], dec, ls);
+          sfw |= S << (8 * b);
+          cw[2 * b] = e2m1x8(a + 16 * b);
+          cw[2 * b + 1] = e2m1x8(a + 16 * b + 8);
+        }
+        l = fmaf(ls, sigma_raw, l);
+        uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+        if constexpr (NB == 2) {
+          *reinterpret_cast<uint4*>(p4 + swz_offset(r, f * NB * 8, BLK / 2)) =
+              make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint16_t*>(p4 + 128 * (BLK / 2) + sf_offset(r, f * NB)) =
+              (uint16_t)sfw;
+        } else {
+          *reinterpret_cast<uint2*>(p4 + swz_offset(r, f * NB * 8, BLK / 2)) =
+              make_uint2(cw[0], cw[1]);
+          p4[128 * (BLK / 2) + sf_offset(r, f * NB)] = (uint8_t)sfw;
+        }
+        pend_sigma_next = sigma;
+      } else {
+        const float negm = m_new == -INFINITY ? 0.0f : -m_new;
+        float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int i = 0; i < SC; ++i) {
+          a[i] = ex2_ftz(fmaf(a[i], cs, negm));  // exp2(-inf) = 0 for masked columns
+          l4[i & 3] += a[i];
+        }
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        uint8_t* p16 = sm + L::OFF_P16;
+#pragma unroll
+        for (int q8 = 0; q8 < SC / 8; ++q8) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w4[e] = pack2<DT>(a[8 * q8 + 2 * e], a[8 * q8 + 2 * e + 1]);
+          const uint32_t key0 = f * SC + 8 * q8;
+          *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
+                                    swz_offset(r, (key0 % 64) * 2, 128)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        pend_sigma_next = 1.0f;
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_PF + st]);
@@ -526,18 +567,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       }
       pending = t;
       pend_alpha = alpha;  // applied to O before PV(t) is added
-      pend_sigma = sigma;
+      pend_sigma = pend_sigma_next;
       prev16 = f16;
     }
     if (ok && pending >= 0) ok = accumulate(pending);
-    // combine the two halves' partial sums, then write this half of the row
-    float* xl = xch + 512;
-    xl[hf * 128 + r] = l;
-    named_bar_sync(1 + q4, 64);
-    const float lt = xl[r] + xl[128 + r];
+    // combine the four quarters' partial sums, then write this quarter of the
+    // row (the exchange area is free: every thread has passed its last tile)
+    named_bar_sync(1 + q4, 128);
+    float* xl = xch;
+    xl[f * 128 + r] = l;
+    named_bar_sync(1 + q4, 128);
+    const float lt = (xl[r] + xl[128 + r]) + (xl[256 + r] + xl[384 + r]);
     if (ok && row_ok) {
       const float il = lt > 0.0f ? ref / lt : 0.0f;
-      uint16_t* orow = p.out + ((start + row) * p.H + h) * D + hf * OC;
+      uint16_t* orow = p.out + ((start + row) * p.H + h) * D + f * OC;
 #pragma unroll
       for (int c = 0; c < OC; c += 8) {
         uint4 w;
@@ -547,7 +590,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         w.w = pack2<DT>(O[c + 6] * il, O[c + 7] * il);
         *reinterpret_cast<uint4*>(orow + c) = w;
       }
-      if (hf == 0) {
+      if (f == 0) {
         const float lse = lt > 0.0f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
         const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
                                         : ((int64_t)seq * p.H + h) * len + row;

@@ -67,7 +67,7 @@ def lib():
         L.orc_block_mean_topk_varlen.argtypes = [P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, P]
         L.orc_thrift_attn.restype = i32
         L.orc_thrift_attn.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, i32, i32,
-                                      P, i32, P, i64, i32, P, P, P, P]
+                                      P, i32, P, i64, i32, P, P, P, P, P]
         L.orc_attn_fp64.restype = i32
         L.orc_attn_fp64.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, P, i64, i32, P, P]
         _lib = L
@@ -252,8 +252,9 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
 
     q [total,H,d], k/v [total,Hkv,d] uint16; cu int32 [nseq+1].
     Returns dict(out uint16 [total,H,d], out64 fp64 [total,H,d] (before the
-    final rounding to the 16-bit type), lse f32 [H,total], mask flat uint8,
-    g (g_Q, g_K, g_V)).  ``units``: optional int array [n,3] of
+    final rounding to the 16-bit type), tol fp64 [total,H,d] (bound on the
+    effect of roundings that are not unique, see oracle.cpp), lse f32
+    [H,total], mask flat uint8, g (g_Q, g_K, g_V)).  ``units``: optional int array [n,3] of
     (sequence, head, query block) to compute; other rows stay 0 / NaN."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     cu = np.ascontiguousarray(cu, np.int32)
@@ -271,6 +272,7 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
         given = 1
     out = np.zeros((total, H, d), np.uint16)
     out64 = np.zeros((total, H, d), np.float64)
+    tol = np.zeros((total, H, d), np.float64)
     lse = np.full((H, total), np.nan, np.float32)
     gs = np.zeros(3, np.float32)
     if units is not None:
@@ -281,10 +283,10 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
     rc = lib().orc_thrift_attn(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
                                int(causal), float(frac), int(use_ss), int(use_had), _p(m), given,
                                _p(u), n_units, int(nthreads or nthreads_default()), _p(out),
-                               _p(lse), _p(gs), _p(out64))
+                               _p(lse), _p(gs), _p(out64), _p(tol))
     if rc:
         raise ValueError("oracle thrift_attn: bad arguments")
-    return {"out": out, "out64": out64, "lse": lse, "mask": m,
+    return {"out": out, "out64": out64, "tol": tol, "lse": lse, "mask": m,
             "g": tuple(float(x) for x in gs)}
 
 

@@ -531,8 +531,54 @@ static inline double deq(uint8_t code, uint8_t sc, float g) {
 }
 
 // One query block i of sequence s, head h.  Writes out rows and lse.
+// Relative distance within which a rounding decision of the oracle is treated
+// as not unique: the GPU computes the same quantities through fp32 MMA
+// accumulation and hardware exp2/log2, about 1e-6 relative from the oracle's
+// fp64 values, so a value this close to a rounding midpoint may land on
+// either side.
+static const double kAmbiguous = 2e-5;
+
+// E2M1 rounding midpoints between consecutive magnitudes and the code pair
+// on either side.
+static const double kE2M1Mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+
+// If |t| lies within kAmbiguous of an E2M1 midpoint, returns the magnitude of
+// the other code's value minus this code's value; else 0.
+static double e2m1_ambiguity(float t) {
+  const double a = std::fabs((double)t);
+  for (int k = 0; k < 7; ++k)
+    if (std::fabs(a - kE2M1Mid[k]) <= kAmbiguous * kE2M1Mid[k])
+      return (double)kE2M1Mag[k + 1] - (double)kE2M1Mag[k];
+  return 0.0;
+}
+
+// The UE4M3 byte on the other side of the nearest rounding midpoint when v
+// lies within kAmbiguous of it, else -1.
+static int ue4m3_ambiguous_neighbour(float v, uint8_t S) {
+  if (!(v > 0.0f)) return -1;
+  const double dv = (double)v, d0 = orc_ue4m3_decode(S);
+  for (int nb = (int)S - 1; nb <= (int)S + 1; nb += 2) {
+    if (nb < 0 || nb > 0x7E) continue;
+    const double mid = 0.5 * (d0 + (double)orc_ue4m3_decode((uint8_t)nb));
+    if (mid > 0.0 && std::fabs(dv - mid) <= kAmbiguous * mid) return nb;
+  }
+  return -1;
+}
+
+// Half the 16-bit spacing at x if x lies within kAmbiguous of a 16-bit
+// rounding midpoint (the other rounding is one spacing away), else 0.
+static double half_ambiguity(double x, int dt) {
+  if (x <= 0.0) return 0.0;
+  const double lo = orc_half_to_float(orc_double_to_half(x, dt), dt);
+  int e;
+  std::frexp(x, &e);
+  const double sp = std::ldexp(1.0, e - (dt == 1 ? 8 : 11));  // spacing in [2^(e-1), 2^e)
+  const double mid = lo + (x > lo ? 0.5 : -0.5) * sp;
+  return std::fabs(x - mid) <= kAmbiguous * x ? sp : 0.0;
+}
+
 static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, float* lse,
-                      double* out64) {
+                      double* out64, double* tol) {
   const int d = C.d, blk = C.blk, H = C.H, Hkv = C.Hkv;
   const int64_t st = C.cu[s];
   const int len = C.cu[s + 1] - C.cu[s];
@@ -561,6 +607,9 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
       q16[(size_t)r * d + c] = orc_half_to_float(C.q[e], C.dt);
     }
   std::vector<double> m(nr, -INFINITY), l(nr, 0.0), O((size_t)nr * d, 0.0);
+  // amb: bound on how far the non-unique roundings can move O (before / l)
+  std::vector<double> amb((size_t)nr * d, 0.0);
+  std::vector<double> dq(blk);
   std::vector<double> kt((size_t)blk * d), vt((size_t)blk * d), S(blk);
   std::vector<float> Pt(blk), Ph(blk);
   std::vector<double> Pq(blk);
@@ -599,7 +648,10 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
       const double mn = std::max(m[r], mt);
       const double alpha = std::exp2(m[r] - mn);  // 0 when m is still -inf
       l[r] *= alpha;
-      for (int c = 0; c < d; ++c) O[(size_t)r * d + c] *= alpha;
+      for (int c = 0; c < d; ++c) {
+        O[(size_t)r * d + c] *= alpha;
+        amb[(size_t)r * d + c] *= alpha;
+      }
       float rowmax = 0.0f;
       for (int t = 0; t < nk; ++t) {
         Pt[t] = S[t] == -INFINITY ? 0.0f : (float)std::exp2(S[t] - mn);
@@ -615,25 +667,46 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
         for (int b0 = 0; b0 < blk; b0 += 16) {
           float amax = 0.0f;
           for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
-          uint8_t sp = orc_ue4m3_encode(amax / 6.0f);
+          const float s_real = amax / 6.0f;
+          uint8_t sp = orc_ue4m3_encode(s_real);
           float dec = orc_ue4m3_decode(sp);
           float rr = 1.0f / dec;
-          for (int e = 0; e < 16; ++e)
-            Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr)) *
-                                             (double)dec;
+          for (int e = 0; e < 16; ++e) {
+            const float tq = Ph[b0 + e] * rr;
+            Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(tq)) * (double)dec;
+            dq[b0 + e] = sp == 0 ? 0.0 : e2m1_ambiguity(tq) * (double)dec;
+          }
+          // a block scale at a rounding midpoint: the other byte's block
+          const int alt = ue4m3_ambiguous_neighbour(s_real, sp);
+          if (alt > 0) {
+            const float dec2 = orc_ue4m3_decode((uint8_t)alt);
+            const float rr2 = 1.0f / dec2;
+            for (int e = 0; e < 16; ++e) {
+              const double q2 = (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr2)) * (double)dec2;
+              dq[b0 + e] = std::max(dq[b0 + e], std::fabs(q2 - Pq[b0 + e]));
+            }
+          }
         }
         for (int c = 0; c < d; ++c) {
-          double acc = 0.0;
-          for (int t = 0; t < nk; ++t) acc += Pq[t] * vt[(size_t)t * d + c];
+          double acc = 0.0, ab = 0.0;
+          for (int t = 0; t < nk; ++t) {
+            acc += Pq[t] * vt[(size_t)t * d + c];
+            ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
+          }
           O[(size_t)r * d + c] += (double)sigma * acc;
+          amb[(size_t)r * d + c] += (double)sigma * ab;
         }
       } else {
+        for (int t = 0; t < nk; ++t) dq[t] = half_ambiguity((double)Pt[t], C.dt);
         for (int c = 0; c < d; ++c) {
-          double acc = 0.0;
-          for (int t = 0; t < nk; ++t)
+          double acc = 0.0, ab = 0.0;
+          for (int t = 0; t < nk; ++t) {
             acc += (double)orc_half_to_float(orc_double_to_half((double)Pt[t], C.dt), C.dt) *
                    vt[(size_t)t * d + c];
+            ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
+          }
           O[(size_t)r * d + c] += acc;
+          amb[(size_t)r * d + c] += ab;
         }
       }
       m[r] = mn;
@@ -646,6 +719,7 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
       double o = l[r] > 0.0 ? O[(size_t)r * d + c] / l[r] : 0.0;
       out[(tok * H + h) * d + c] = orc_double_to_half(o, C.dt);
       if (out64) out64[(tok * H + h) * d + c] = o;
+      if (tol) tol[(tok * H + h) * d + c] = l[r] > 0.0 ? amb[(size_t)r * d + c] / l[r] : 0.0;
     }
     lse[(int64_t)h * C.total + tok] = l[r] > 0.0 ? (float)(m[r] * ln2 + std::log(l[r])) : -INFINITY;
   }
@@ -658,12 +732,16 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // list of (sequence, head, query block) triples to compute (n_units = 0 means
 // every unit); rows of other units are left untouched.  gs_out (optional)
 // receives g_Q, g_K, g_V.  out64 (optional) receives the fp64 output before
-// its final rounding to the 16-bit type.
+// its final rounding to the 16-bit type.  tol (optional) receives, per output
+// element, a bound on how far roundings that are not unique can move it: a
+// probability whose E2M1 code, UE4M3 block scale or 16-bit value lies within
+// 2e-5 relative of a rounding midpoint may take either side in an
+// implementation that evaluates the same arithmetic in another order.
 int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
                     int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
                     float frac, int use_ss, int use_had, uint8_t* mask_io, int mask_given,
                     const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
-                    float* lse, float* gs_out, double* out64) {
+                    float* lse, float* gs_out, double* out64, double* tol) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
   if (use_had && (d & (d - 1))) return -1;
   AttnCtx C;
@@ -726,7 +804,7 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
     n_units = (int64_t)all.size() / 3;
   }
   parallel_for(n_units, nthreads, [&](int64_t u) {
-    attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse, out64);
+    attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse, out64, tol);
   });
   return 0;
 }

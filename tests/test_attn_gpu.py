@@ -2,11 +2,15 @@
 tiling (ThriftAttention Metodologia step 2; ScaleSearchAttention).
 
 Bar: |out - oracle| <= 1e-2 + half an ulp of the 16-bit output type at the
-oracle's value, element by element, and cosine >= 0.9999, against the
-oracle's output before its own final rounding (both sides round the same
-real result to bf16/fp16 once; for |out| >= 2 one bf16 ulp alone exceeds
-1e-2).  lse within 1e-2.  Error against unquantised fp64 attention is
-reported.
+oracle's value + the oracle's bound for roundings that are not unique,
+element by element, and cosine >= 0.9999, against the oracle's output before
+its own final rounding.  Both sides round the same real result to bf16/fp16
+once (for |out| >= 2 one bf16 ulp alone exceeds 1e-2).  A probability whose
+E2M1 code, UE4M3 block scale or 16-bit value sits within the arithmetic's
+rounding noise of a rounding midpoint has two correct codes; the oracle
+bounds what the other choice moves each output (zero for almost every
+element) and that bound is added.  lse within 1e-2.  Error against
+unquantised fp64 attention is reported.
 """
 import numpy as np
 import pytest
@@ -37,10 +41,12 @@ def half_ulp(x, dtype):
     return 0.5 * 2.0 ** (e - mant)
 
 
-def _compare(got, want64, what, dtype):
+def _compare(got, want64, what, dtype, tol=None):
     got = got.reshape(-1).astype(np.float64)
     want = want64.reshape(-1).astype(np.float64)
     excess = np.abs(got - want) - half_ulp(want, dtype)
+    if tol is not None:
+        excess -= tol.reshape(-1)
     worst = int(np.argmax(excess))
     cos = float(got @ want / (np.linalg.norm(got) * np.linalg.norm(want) + 1e-300))
     assert excess[worst] <= MAX_ABS and cos >= MIN_COS, (
@@ -64,7 +70,7 @@ def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_
     r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had)
     got = out.cpu().reshape(B * N, H, d)
     gotf = got.double().numpy()
-    _compare(gotf, r["out64"], "out", dtype)
+    _compare(gotf, r["out64"], "out", dtype, r["tol"])
     lse_want = r["lse"].reshape(H, B, N).transpose(1, 0, 2)
     assert np.max(np.abs(lse.cpu().numpy() - lse_want)) < 1e-2
     return gotf, qp, kp, vp, cu, dt
@@ -114,7 +120,8 @@ def test_varlen_parity(orc):
         assert ops.device_status(reset=True) == ops.OK
         r = orc.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), 1, cu, blk, True,
                             frac, use_ss=ss, use_had=had)
-        _compare(out.cpu().double().numpy(), r["out64"], f"varlen frac={frac}", torch.bfloat16)
+        _compare(out.cpu().double().numpy(), r["out64"], f"varlen frac={frac}", torch.bfloat16,
+                 r["tol"])
         assert np.max(np.abs(lse.cpu().numpy() - r["lse"])) < 1e-2
 
 
