@@ -56,21 +56,30 @@ struct AttnLayout {
   static constexpr uint32_t VT16 = f16_tile_bytes(D, BLK);
   static constexpr uint32_t PT4 = fp4_tile_bytes(128, BLK);
   static constexpr uint32_t P16B = f16_tile_bytes(128, BLK);
-  static constexpr uint32_t V4_OFF = align(KT4);
-  static constexpr uint32_t V16_OFF = align(KT16);
-  static constexpr uint32_t STG = align(V4_OFF + VT4) > align(V16_OFF + VT16)
-                                      ? align(V4_OFF + VT4)
-                                      : align(V16_OFF + VT16);
-  static constexpr uint32_t OFF_Q4 = 0;
-  static constexpr uint32_t OFF_Q16 = OFF_Q4 + align(QT4);
-  static constexpr uint32_t OFF_STG = OFF_Q16 + align(Q16B);
   static constexpr uint32_t PT4A = align(PT4);  // one P slot
-  static constexpr uint32_t OFF_P4 = OFF_STG + 2 * STG;
-  static constexpr uint32_t OFF_P16 = OFF_P4 + 2 * PT4A;
-  static constexpr uint32_t OFF_LIST = OFF_P16 + align(P16B);
+  // One region serves the NVFP4 phase and then the FP16 phase of a CTA (all
+  // NVFP4 tiles come first); the producer enters the FP16 phase only after
+  // the last NVFP4 PV has retired.
+  //   NVFP4 view: Q4 | P4 x2 | NS4 stages (K4 + V4)
+  //   FP16 view:  Q16 | P16 | 2 stages (K16 + V16)
+  static constexpr uint32_t V4_OFF = align(KT4);
+  static constexpr uint32_t STG4 = V4_OFF + align(VT4);
+  static constexpr uint32_t V16_OFF = align(KT16);
+  static constexpr uint32_t STG16 = V16_OFF + align(VT16);
+  static constexpr uint32_t OFF4_Q = 0;
+  static constexpr uint32_t OFF4_P = align(QT4);
+  static constexpr uint32_t OFF4_STG = OFF4_P + 2 * PT4A;
+  static constexpr uint32_t OFF16_Q = 0;
+  static constexpr uint32_t OFF16_P = align(Q16B);
+  static constexpr uint32_t OFF16_STG = OFF16_P + align(P16B);
+  static constexpr uint32_t NS16 = 2;
+  static constexpr uint32_t REGION = OFF16_STG + NS16 * STG16;
+  static constexpr uint32_t NS4_FIT = (REGION - OFF4_STG) / STG4;
+  static constexpr uint32_t NS4 = NS4_FIT > 12 ? 12 : NS4_FIT;
+  static constexpr uint32_t OFF_LIST = REGION;
   static constexpr uint32_t MAX_TILES = 512;  // key tiles per sequence
   static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
-  static constexpr uint32_t OFF_XCH = OFF_BAR + 256;  // row-max / row-sum exchange
+  static constexpr uint32_t OFF_XCH = OFF_BAR + 512;  // row-max / row-sum exchange
   static constexpr uint32_t BYTES = OFF_XCH + 4 * 2 * 4 * 128;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
   // tensor-memory columns
@@ -82,13 +91,15 @@ struct AttnLayout {
   static constexpr uint32_t T_VSF = T_PSF + 2 * (BLK / 64) * 4;
   static constexpr uint32_t T_END = T_VSF + 2 * (BLK / 64) * 4;
   static_assert(T_END <= 512, "tensor memory budget");
+  static_assert(NS4 >= 2, "at least two NVFP4 stages");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 // Barrier slots inside the barrier area.
 enum : int {
-  B_Q4 = 0, B_Q16 = 1, B_KVF = 2 /* 2,3 */, B_KVE = 4 /* 4,5 */, B_SF = 6 /* 6,7 */,
-  B_SE = 8 /* 8,9 */, B_PF = 10 /* 10,11 */, B_OF = 12, B_OE = 13, B_DONE = 14, B_N = 15
+  B_Q4 = 0, B_Q16 = 1, B_SF = 2 /* 2,3 */, B_SE = 4 /* 4,5 */, B_PF = 6 /* 6,7 */, B_OF = 8,
+  B_OE = 9, B_DONE = 10, B_KVF16 = 11 /* 11,12 */, B_KVE16 = 13 /* 13,14 */,
+  B_KVF4 = 15 /* 15..26 */, B_KVE4 = 27 /* 27..38 */, B_N = 39
 };
 
 constexpr int kSoftmaxWarps = 16;
@@ -250,50 +261,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
   const uint32_t tmem = *s_tmem;
   const int n = *s_n, n4 = *s_n4;
 
-  uint8_t* q4s = sm + L::OFF_Q4;
-  uint8_t* q16s = sm + L::OFF_Q16;
+  uint8_t* q4s = sm + L::OFF4_Q;
+  uint8_t* q16s = sm + L::OFF16_Q;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------- producer --
     if (lane == 0) {
       const int64_t qtile = ((int64_t)seq * p.H + h) * p.nTq + qt;
       bool q4_issued = false, q16_issued = false;
-      int issued[2] = {-1, -1};
+      int last4[L::NS4], last16[L::NS16];
+      for (int i = 0; i < (int)L::NS4; ++i) last4[i] = -1;
+      for (int i = 0; i < (int)L::NS16; ++i) last16[i] = -1;
       if (n4 > 0) {
         mbar_arrive_expect_tx(&bars[B_Q4], L::QT4);
         bulk_g2s(q4s, p.q4 + qtile * L::QT4, L::QT4, &bars[B_Q4]);
         q4_issued = true;
       }
       for (int t = 0; t < n && !*s_abort; ++t) {
-        const int st = t & 1;
         const int j = s_list[t] & 0x1FFF;
-        const bool f16 = (s_list[t] >> 15) != 0;
-        if (t >= 2 && !mbar_wait(&bars[B_KVE + st], ((t >> 1) - 1) & 1, s_abort)) break;
-        if (f16 && !q16_issued) {
-          mbar_arrive_expect_tx(&bars[B_Q16], L::Q16B);
-          bulk_g2s(q16s, p.q16 + qtile * L::Q16B, L::Q16B, &bars[B_Q16]);
-          q16_issued = true;
-        }
-        uint8_t* stg = sm + L::OFF_STG + st * L::STG;
+        const bool f16 = t >= n4;
         const int64_t ktile = ((int64_t)seq * p.Hkv + hk) * p.nB + j;
         if (!f16) {
-          mbar_arrive_expect_tx(&bars[B_KVF + st], L::KT4 + L::VT4);
-          bulk_g2s(stg, p.k4 + ktile * L::KT4, L::KT4, &bars[B_KVF + st]);
-          bulk_g2s(stg + L::V4_OFF, p.v4 + ktile * L::VT4, L::VT4, &bars[B_KVF + st]);
+          const int i = t, sl = i % L::NS4;
+          if (i >= (int)L::NS4 &&
+              !mbar_wait(&bars[B_KVE4 + sl], ((i / L::NS4) - 1) & 1, s_abort))
+            break;
+          uint8_t* stg = sm + L::OFF4_STG + sl * L::STG4;
+          mbar_arrive_expect_tx(&bars[B_KVF4 + sl], L::KT4 + L::VT4);
+          bulk_g2s(stg, p.k4 + ktile * L::KT4, L::KT4, &bars[B_KVF4 + sl]);
+          bulk_g2s(stg + L::V4_OFF, p.v4 + ktile * L::VT4, L::VT4, &bars[B_KVF4 + sl]);
+          last4[sl] = i;
         } else {
-          mbar_arrive_expect_tx(&bars[B_KVF + st], L::KT16 + L::VT16);
-          bulk_g2s(stg, p.k16 + ktile * L::KT16, L::KT16, &bars[B_KVF + st]);
-          bulk_g2s(stg + L::V16_OFF, p.v16 + ktile * L::VT16, L::VT16, &bars[B_KVF + st]);
+          const int i = t - n4, sl = i % L::NS16;
+          if (i == 0) {
+            // the region switches to its FP16 view: the last NVFP4 PV (and
+            // with it every NVFP4 read of Q4, P4 and the stages) must be done
+            if (n4 > 0 && !mbar_wait(&bars[B_KVE4 + (n4 - 1) % L::NS4],
+                                     ((n4 - 1) / L::NS4) & 1, s_abort))
+              break;
+            mbar_arrive_expect_tx(&bars[B_Q16], L::Q16B);
+            bulk_g2s(q16s, p.q16 + qtile * L::Q16B, L::Q16B, &bars[B_Q16]);
+            q16_issued = true;
+          }
+          if (i >= (int)L::NS16 &&
+              !mbar_wait(&bars[B_KVE16 + sl], ((i / L::NS16) - 1) & 1, s_abort))
+            break;
+          uint8_t* stg = sm + L::OFF16_STG + sl * L::STG16;
+          mbar_arrive_expect_tx(&bars[B_KVF16 + sl], L::KT16 + L::VT16);
+          bulk_g2s(stg, p.k16 + ktile * L::KT16, L::KT16, &bars[B_KVF16 + sl]);
+          bulk_g2s(stg + L::V16_OFF, p.v16 + ktile * L::VT16, L::VT16, &bars[B_KVF16 + sl]);
+          last16[sl] = i;
         }
-        issued[st] = t;
       }
       // Drain: every copy this thread issued has landed before the CTA ends.
       int dummy = 0;
       volatile int* never = &dummy;
       if (q4_issued) mbar_wait(&bars[B_Q4], 0, never, 200000000ull);
       if (q16_issued) mbar_wait(&bars[B_Q16], 0, never, 200000000ull);
-      for (int st = 0; st < 2; ++st)
-        if (issued[st] >= 0) mbar_wait(&bars[B_KVF + st], (issued[st] >> 1) & 1, never, 200000000ull);
+      for (int sl = 0; sl < (int)L::NS4; ++sl)
+        if (last4[sl] >= 0)
+          mbar_wait(&bars[B_KVF4 + sl], (last4[sl] / L::NS4) & 1, never, 200000000ull);
+      for (int sl = 0; sl < (int)L::NS16; ++sl)
+        if (last16[sl] >= 0)
+          mbar_wait(&bars[B_KVF16 + sl], (last16[sl] / L::NS16) & 1, never, 200000000ull);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------- MMA issuer --
@@ -302,10 +332,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
       bool q4_ready = false, q16_ready = false;
       const uint32_t q4a = smem_u32(q4s), q16a = smem_u32(q16s);
+      // stage of tile t: NVFP4 tiles 0..n4-1 cycle through NS4 stages, FP16
+      // tiles through NS16
+      auto stage_of = [&](int t, uint32_t& addr, uint64_t*& full, uint64_t*& empty,
+                          uint32_t& parity) {
+        if (t < n4) {
+          const int sl = t % L::NS4;
+          addr = smem_u32(sm + L::OFF4_STG + sl * L::STG4);
+          full = &bars[B_KVF4 + sl];
+          empty = &bars[B_KVE4 + sl];
+          parity = (t / L::NS4) & 1;
+        } else {
+          const int i = t - n4, sl = i % L::NS16;
+          addr = smem_u32(sm + L::OFF16_STG + sl * L::STG16);
+          full = &bars[B_KVF16 + sl];
+          empty = &bars[B_KVE16 + sl];
+          parity = (i / L::NS16) & 1;
+        }
+      };
       auto issue_qk = [&](int t) -> bool {
         const int st = t & 1;
-        const bool f16 = (s_list[t] >> 15) != 0;
-        if (!mbar_wait(&bars[B_KVF + st], (t >> 1) & 1, s_abort)) return false;
+        const bool f16 = t >= n4;
+        uint32_t stg, par;
+        uint64_t *full, *empty;
+        stage_of(t, stg, full, empty, par);
+        if (!mbar_wait(full, par, s_abort)) return false;
         if (!f16 && !q4_ready) {
           if (!mbar_wait(&bars[B_Q4], 0, s_abort)) return false;
           tc_fence_after();
@@ -322,7 +373,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         if (t >= 2 && !mbar_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) return false;
         tc_fence_after();
         const uint32_t dS = tmem + L::T_S + st * BLK;
-        const uint32_t stg = smem_u32(sm + L::OFF_STG + st * L::STG);
         if (!f16) {
           const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
 #pragma unroll
@@ -346,14 +396,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       };
       auto issue_pv = [&](int t) -> bool {
         const int st = t & 1;
-        const bool f16 = (s_list[t] >> 15) != 0;
+        const bool f16 = t >= n4;
+        uint32_t stg, par;
+        uint64_t *full, *empty;
+        stage_of(t, stg, full, empty, par);
         if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) return false;
         if (t >= 1 && !mbar_wait(&bars[B_OE], (t - 1) & 1, s_abort)) return false;
         tc_fence_after();
         const uint32_t dO = tmem + L::T_PV;
-        const uint32_t stg = smem_u32(sm + L::OFF_STG + st * L::STG);
         if (!f16) {
-          const uint32_t p4 = smem_u32(sm + L::OFF_P4 + st * L::PT4A);
+          const uint32_t p4 = smem_u32(sm + L::OFF4_P + st * L::PT4A);
           const uint32_t v4 = stg + L::V4_OFF;
           const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
           const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
@@ -368,7 +420,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
                      make_sdesc(v4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
                      id_pv4, psf + 4 * s, vsf + 4 * s, s > 0);
         } else {
-          const uint32_t p16 = smem_u32(sm + L::OFF_P16);
+          const uint32_t p16 = smem_u32(sm + L::OFF16_P);
           const uint32_t v16 = stg + L::V16_OFF;
 #pragma unroll
           for (int s = 0; s < BLK / 16; ++s)
@@ -377,13 +429,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
                     id_pv16, s > 0);
         }
         tc_commit(&bars[B_OF]);
-        tc_commit(&bars[B_KVE + st]);
+        tc_commit(empty);
         return true;
       };
+      // QK^T of tile t+1 goes out before PV of tile t, except at the switch
+      // to the FP16 phase: the first FP16 tile is only loaded once the last
+      // NVFP4 PV has retired.
       bool ok = n > 0 ? issue_qk(0) : true;
       for (int t = 0; t < n && ok; ++t) {
-        if (t + 1 < n) ok = issue_qk(t + 1);
+        const bool crossing = t + 1 == n4;
+        if (t + 1 < n && !crossing) ok = issue_qk(t + 1);
         if (ok) ok = issue_pv(t);
+        if (ok && t + 1 < n && crossing) ok = issue_qk(t + 1);
       }
       tc_commit(&bars[B_DONE]);
       int dummy = 0;
@@ -526,7 +583,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           cw[2 * b + 1] = e2m1x8(a + 16 * b + 8);
         }
         l = fmaf(ls, sigma_raw, l);
-        uint8_t* p4 = sm + L::OFF_P4 + st * L::PT4A;
+        uint8_t* p4 = sm + L::OFF4_P + st * L::PT4A;
         if constexpr (NB == 2) {
           *reinterpret_cast<uint4*>(p4 + swz_offset(r, f * NB * 8, BLK / 2)) =
               make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -547,7 +604,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           l4[i & 3] += a[i];
         }
         l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-        uint8_t* p16 = sm + L::OFF_P16;
+        uint8_t* p16 = sm + L::OFF16_P;
 #pragma unroll
         for (int q8 = 0; q8 < SC / 8; ++q8) {
           uint32_t w4[4];
