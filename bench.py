@@ -51,6 +51,10 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+XU_OPS_PER_CLK_PER_SM = 16   # MUFU / conversion pipe lanes per SM (4 per sub-partition)
+XU_OPS_PER_ELEMENT = 1.5     # one exp2 and half of a two-value 4/16-bit convert per score
+
+
 def pair_flops(mask, w, lengths):
     """Algorithmic FLOPs (4*d per unmasked score element) split by path."""
     blk, d = w.blk, w.d
@@ -390,10 +394,24 @@ def main():
                               f"the FP16 share ({100 * f16 / flops:.1f}% of flops)"),
                 "kernel_ms": k_ms, "fp4_flops": f4, "fp16_flops": f16}
 
+    # ALU roofline of the same kernel: every score element needs one exp2 and
+    # half a packed conversion on the MUFU/convert pipe (16 lanes per SM).
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    elems = flops / (4.0 * w.d)
+    alu_peak = XU_OPS_PER_CLK_PER_SM * n_sm * sm_mhz * 1e6 / XU_OPS_PER_ELEMENT / 1e9
+    alu_achieved = elems / (k_ms * 1e-3) / 1e9
+    alu_roofline = {"bound": "alu", "kernel": "attn_fwd_kernel", "achieved": alu_achieved,
+                    "peak": alu_peak, "unit": "Gelem/s", "frac": alu_achieved / alu_peak,
+                    "peak_note": (f"{XU_OPS_PER_CLK_PER_SM} MUFU/convert lanes per SM x {n_sm} SMs x "
+                                  f"{sm_mhz:.0f} MHz / {XU_OPS_PER_ELEMENT} ops per score element"),
+                    "tflops_equivalent_peak": alu_peak * 1e9 * 4 * w.d / 1e12}
+
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
             "data": "synthetic", "config": config_of(w), "roofline": roofline,
+            "alu_roofline": alu_roofline,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
