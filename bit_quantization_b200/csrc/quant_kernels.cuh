@@ -124,75 +124,6 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   }
 }
 
-// Single-pass quantiser: every thread stages kFusedKPT blocks in shared
-// memory, the grid agrees on the tensor absmax through one atomicMax per CTA
-// and a grid barrier, then quantises from shared memory, so x is read from
-// HBM once.  Launched cooperatively with a grid that covers the tensor in one
-// sweep (n_blocks <= threads * kFusedKPT).  sync[0] = absmax bits, sync[1] =
-// arrival counter, both zero at launch.  The barrier wait is bounded; on
-// timeout the device status word is set and the blocks are quantised with
-// the absmax seen so far.
-constexpr int kFusedKPT = 8;
-constexpr int kFusedSmem = kFusedKPT * 256 * 32;
-
-template <int DT, int G, bool SS>
-__global__ void __launch_bounds__(256) quant_rows_fused_kernel(
-    const uint16_t* __restrict__ x, int64_t n_blocks, uint32_t* sync, float* tensor_scale,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  extern __shared__ uint4 stage[];  // [kFusedKPT][256 threads][2]
-  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
-  const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  float a = 0.0f;
-#pragma unroll
-  for (int k0 = 0; k0 < kFusedKPT; k0 += 4) {
-    uint4 r[4][2];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) load_raw(x, b0 + (k0 + k) * nthreads, n_blocks, r[k][0], r[k][1]);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      stage[((k0 + k) * 256 + threadIdx.x) * 2] = r[k][0];
-      stage[((k0 + k) * 256 + threadIdx.x) * 2 + 1] = r[k][1];
-      float v[16];
-      unpack16<DT>(r[k][0], r[k][1], v);
-      if constexpr (G > 0) fwht_rows16<G>(v);
-      a = fmaxf(a, block_absmax(v));
-    }
-  }
-  cta_atomic_amax(a, &sync[0]);
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(&sync[1], 1u);
-    const uint64_t t_start = globaltimer_ns();
-    uint32_t seen = 0;
-    for (uint32_t it = 0;; ++it) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(&sync[1]) : "memory");
-      if (seen >= gridDim.x) break;
-      if ((it & 63) == 63 && globaltimer_ns() - t_start > 1000000000ull) {
-        set_device_status(THRIFT_ERR_TIMEOUT);
-        break;
-      }
-    }
-  }
-  __syncthreads();
-  uint32_t amax_bits;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(&sync[0]) : "memory");
-  const float g = tensor_scale_from_amax(amax_bits);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-#pragma unroll 2
-  for (int k = 0; k < kFusedKPT; ++k) {
-    const int64_t b = b0 + k * nthreads;
-    float v[16];
-    unpack16<DT>(stage[(k * 256 + threadIdx.x) * 2], stage[(k * 256 + threadIdx.x) * 2 + 1], v);
-    if constexpr (G > 0) fwht_rows16<G>(v);
-    if (b < n_blocks) {
-      uint32_t lo, hi;
-      const uint32_t S = quant_block16(v, g, SS, lo, hi);
-      *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
-      scales[b] = (uint8_t)S;
-    }
-  }
-}
-
 // ---------------------------------------------- column-blocked quantiser --
 // x [rows, cols]; 16-blocks along rows.  codes [cols, rows/2], scales
 // [cols, rows/16].  One thread per (row block, column); columns fastest.

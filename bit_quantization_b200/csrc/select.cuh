@@ -13,7 +13,8 @@
 namespace thrift {
 
 // means [nseq, nh, nB, d] fp64 of x [total, nh, d]; one thread per
-// (sequence, head, block, channel), channels fastest.
+// (sequence, head, block, channel), channels fastest.  The sum runs in token
+// order; loads are issued eight tokens ahead of the additions.
 template <int DT>
 __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __restrict__ x,
                                                           SeqInfo seqs, int nseq, int nh, int d,
@@ -32,38 +33,91 @@ __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __rest
     const int t0 = i * blk;
     if (t0 >= len) continue;
     const int t1 = min(len, t0 + blk);
+    const uint16_t* px = x + ((start + t0) * nh + head) * d + c;
+    const int64_t stride = (int64_t)nh * d;
     double sum = 0.0;
-    for (int t = t0; t < t1; ++t)
-      sum = __dadd_rn(sum, (double)h2f<DT>(__ldg(x + ((start + t) * nh + head) * d + c)));
+    int t = t0;
+    for (; t + 8 <= t1; t += 8) {
+      uint16_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(px + (int64_t)(t - t0 + u) * stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum = __dadd_rn(sum, (double)h2f<DT>(v[u]));
+    }
+    for (; t < t1; ++t) sum = __dadd_rn(sum, (double)h2f<DT>(__ldg(px + (int64_t)(t - t0) * stride)));
     means[idx] = __ddiv_rn(sum, (double)(t1 - t0));
   }
 }
 
 // scores [nseq, H, nB, nB] fp64 (valid i, j < nb of the sequence only).
+// One CTA per (sequence, head, 16 query blocks); the key means pass through
+// shared memory transposed, 8 channels at a time, and every score keeps its
+// sequential fma order over the channels.  nB <= 512.
+constexpr int kScoreRows = 16, kScoreChunk = 8;
+
 __global__ void __launch_bounds__(256) pair_scores_kernel(const double* __restrict__ qm,
                                                           const double* __restrict__ km,
                                                           SeqInfo seqs, int nseq, int H,
                                                           int Hkv, int d, int blk, int nB,
                                                           double* __restrict__ scores) {
-  const int64_t n = (int64_t)nseq * H * nB * nB;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int j = (int)(idx % nB);
-    const int i = (int)((idx / nB) % nB);
-    const int h = (int)((idx / ((int64_t)nB * nB)) % H);
-    const int seq = (int)(idx / ((int64_t)nB * nB * H));
-    int64_t start;
-    int len;
-    seqs.get(seq, start, len);
-    const int nb = (int)ceil_div(len, blk);
-    if (i >= nb || j >= nb) continue;
-    const int hk = h / (H / Hkv);
-    const double* a = qm + (((int64_t)seq * H + h) * nB + i) * d;
-    const double* b = km + (((int64_t)seq * Hkv + hk) * nB + j) * d;
-    double acc = 0.0;
-    for (int c = 0; c < d; ++c) acc = __fma_rn(__ldg(a + c), __ldg(b + c), acc);
-    scores[idx] = acc;
+  extern __shared__ double ssm[];
+  double* qs = ssm;                                   // [kScoreRows][kScoreChunk]
+  double* ks = ssm + kScoreRows * kScoreChunk;        // [kScoreChunk][nB]
+  const int groups = (nB + kScoreRows - 1) / kScoreRows;
+  const int ig = blockIdx.x % groups;
+  const int h = (blockIdx.x / groups) % H;
+  const int seq = blockIdx.x / (groups * H);
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int nb = (int)ceil_div(len, blk);
+  const int i0 = ig * kScoreRows;
+  if (i0 >= nb) return;
+  const int hk = h / (H / Hkv);
+  const double* qrow = qm + (((int64_t)seq * H + h) * nB + i0) * d;
+  const double* krow = km + ((int64_t)seq * Hkv + hk) * nB * d;
+  double acc[kScoreRows][2];
+#pragma unroll
+  for (int a = 0; a < kScoreRows; ++a) acc[a][0] = acc[a][1] = 0.0;
+  const int j0 = threadIdx.x, j1 = threadIdx.x + 256;
+  for (int c0 = 0; c0 < d; c0 += kScoreChunk) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kScoreRows * kScoreChunk; e += blockDim.x) {
+      const int a = e / kScoreChunk, cc = e % kScoreChunk;
+      qs[e] = (i0 + a < nb) ? __ldg(qrow + (int64_t)a * d + c0 + cc) : 0.0;
+    }
+    for (int e = threadIdx.x; e < nb * kScoreChunk; e += blockDim.x) {
+      const int j = e / kScoreChunk, cc = e % kScoreChunk;
+      ks[cc * nB + j] = __ldg(krow + (int64_t)j * d + c0 + cc);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int cc = 0; cc < kScoreChunk; ++cc) {
+      const double k0 = j0 < nb ? ks[cc * nB + j0] : 0.0;
+      const double k1 = j1 < nb ? ks[cc * nB + j1] : 0.0;
+#pragma unroll
+      for (int a = 0; a < kScoreRows; ++a) {
+        const double q = qs[a * kScoreChunk + cc];
+        acc[a][0] = __fma_rn(q, k0, acc[a][0]);
+        acc[a][1] = __fma_rn(q, k1, acc[a][1]);
+      }
+    }
   }
+  double* out = scores + (((int64_t)seq * H + h) * nB + i0) * nB;
+#pragma unroll
+  for (int a = 0; a < kScoreRows; ++a) {
+    if (i0 + a >= nb) break;
+    if (j0 < nb) out[(int64_t)a * nB + j0] = acc[a][0];
+    if (j1 < nb) out[(int64_t)a * nB + j1] = acc[a][1];
+  }
+}
+
+inline size_t pair_scores_smem(int nB) {
+  return sizeof(double) * (kScoreRows * kScoreChunk + kScoreChunk * (size_t)nB);
+}
+
+inline int pair_scores_grid(int nseq, int H, int nB) {
+  return nseq * H * ((nB + kScoreRows - 1) / kScoreRows);
 }
 
 // Order-preserving map of a double to an unsigned 64-bit key.

@@ -80,46 +80,6 @@ void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, i
       static_cast<const uint16_t*>(x), nb, amax, ts, given, codes, scales);
 }
 
-// Single-pass quantiser (absmax agreed through a grid barrier) when one
-// resident grid covers the tensor with kFusedKPT blocks per thread; returns
-// false (nothing launched) when it does not.
-template <int DT, int G, bool SS>
-bool launch_quant_fused_t(const void* x, int64_t nb, uint32_t* sync, float* ts, uint8_t* codes,
-                          uint8_t* scales, cudaStream_t st, thrift_status* status) {
-  static int per_sm = -1;
-  if (per_sm < 0) {
-    per_sm = 0;
-    if (cudaFuncSetAttribute(quant_rows_fused_kernel<DT, G, SS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) ==
-            cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &per_sm, quant_rows_fused_kernel<DT, G, SS>, kThreads, kFusedSmem) != cudaSuccess)
-      per_sm = 0;
-  }
-  const int64_t need = ceil_div(nb, (int64_t)kThreads * kFusedKPT);
-  if (per_sm <= 0 || need > (int64_t)per_sm * sm_count()) return false;
-  if (cudaMemsetAsync(sync, 0, 8, st) != cudaSuccess) {
-    *status = THRIFT_ERR_CUDA;
-    return true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)need);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kFusedSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const uint16_t* xp = static_cast<const uint16_t*>(x);
-  *status = cudaLaunchKernelEx(&cfg, quant_rows_fused_kernel<DT, G, SS>, xp, nb, sync, ts, codes,
-                               scales) == cudaSuccess
-                ? THRIFT_OK
-                : THRIFT_ERR_CUDA;
-  return true;
-}
-
 template <int DT>
 thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_t* sync,
                               float* ts, int given, uint8_t* codes, uint8_t* scales,
@@ -127,8 +87,6 @@ thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_
 #define THRIFT_QUANT_CASE(GG, SSV)                                                        \
   if (G == GG && ss == SSV) {                                                              \
     if (!given) {                                                                          \
-      thrift_status s = THRIFT_OK;                                                         \
-      if (launch_quant_fused_t<DT, GG, SSV>(x, nb, sync, ts, codes, scales, st, &s)) return s; \
       if (cudaMemsetAsync(sync, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;          \
       launch_amax<DT>(x, nb, GG, sync, st);                                                \
     }                                                                                      \
@@ -267,7 +225,7 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
       static_cast<const uint16_t*>(q), si, nseq, H, d, blk, nB, w.means_q);
   block_means_kernel<DT><<<grid_for((int64_t)nseq * Hkv * nB * d), kThreads, 0, st>>>(
       static_cast<const uint16_t*>(k), si, nseq, Hkv, d, blk, nB, w.means_k);
-  pair_scores_kernel<<<grid_for((int64_t)nseq * H * nB * nB), kThreads, 0, st>>>(
+  pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, w.scores);
   topk_kernel<<<nseq * H, kTopkThreads, 0, st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
   if (launch_status() != THRIFT_OK) return THRIFT_ERR_CUDA;
@@ -464,7 +422,7 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
   if (!(topk_frac >= 0.0f && topk_frac <= 1.0f)) return THRIFT_ERR_ARG;
   if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
   if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
-  if (ceil_div(N, blk) > 1024) return THRIFT_ERR_UNSUPPORTED;
+  if (ceil_div(N, blk) > 512) return THRIFT_ERR_UNSUPPORTED;
   if (ws_bytes < block_mean_topk_workspace_size(B, H, Hkv, N, d, blk)) return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nB = (int)ceil_div(N, blk);
@@ -482,7 +440,8 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
     block_means_kernel<0><<<grid_for((int64_t)B * H * nB * d), kThreads, 0, st>>>(qp, si, B, H, d, blk, nB, mq);
     block_means_kernel<0><<<grid_for((int64_t)B * Hkv * nB * d), kThreads, 0, st>>>(kp, si, B, Hkv, d, blk, nB, mk);
   }
-  pair_scores_kernel<<<grid_for((int64_t)B * H * nB * nB), kThreads, 0, st>>>(mq, mk, si, B, H, Hkv, d, blk, nB, sc);
+  pair_scores_kernel<<<pair_scores_grid(B, H, nB), kThreads, pair_scores_smem(nB), st>>>(
+      mq, mk, si, B, H, Hkv, d, blk, nB, sc);
   topk_kernel<<<B * H, kTopkThreads, 0, st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
   return launch_status();
 }

@@ -106,7 +106,7 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
  * best valid pairs are selected (causal: j <= i), ties to the lower i*nB+j.
  *   mask [B, H, nB, nB] uint8 out, 1 = FP16 pair.
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, 0<=frac<=1,
- * nB = ceil(N/blk) <= 1024.
+ * nB = ceil(N/blk) <= 512.
  */
 size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int B, int H,
