@@ -132,24 +132,6 @@ __device__ __forceinline__ float rcp_ftz(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x in [-125, 0]: x = n + f with n the nearest
-// integer (rounded by adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a
-// degree-6 polynomial interpolating 2^f at the Chebyshev nodes of
-// [-1/2, 1/2] (max relative error 8.2e-8); 2^n added to the exponent field.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float t = __fadd_rn(x, 12582912.0f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  const float fr = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-  float q = 1.5461444854736328e-04f;
-  q = fmaf(q, fr, 1.3400427997112274e-03f);
-  q = fmaf(q, fr, 9.6180569380521774e-03f);
-  q = fmaf(q, fr, 5.5503271520137787e-02f);
-  q = fmaf(q, fr, 2.4022650718688965e-01f);
-  q = fmaf(q, fr, 6.9314718246459961e-01f);
-  q = fmaf(q, fr, 1.0f);
-  return __int_as_float(__float_as_int(q) + (n << 23));
-}
-
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -574,7 +556,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           float bs[2] = {0.0f, 0.0f};
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            a[16 * b + i] = ex2_ftz(fmaf(a[16 * b + i], cs, c));
+            a[16 * b + i] = ex2_ftz(fmaf(a[16 * b + i], cs, c));  // masked (-inf) -> 0
             bs[i & 1] += a[16 * b + i];
           }
           ls = fmaf(bs[0] + bs[1], dec, ls);
