@@ -112,6 +112,26 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Packed fp32 pairs (one instruction for two lanes' worth of fma / add;
+// each half rounds exactly as the scalar operation).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0,
+                                     float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ float lg2_ftz(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -447,6 +467,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
     float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][4 quarters][128]
+    // shared-memory offsets this thread writes every tile
+    const uint32_t p4_codes_off = swz_offset(r, f * NB * 8, BLK / 2);
+    const uint32_t p4_sf_off = 128 * (BLK / 2) + sf_offset(r, f * NB);
     // O holds the output divided by `ref`: the true accumulator is ref * O.
     float O[OC];
 #pragma unroll
@@ -473,7 +496,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const float beta = take ? pend_alpha * ref * rcp_ftz(pend_sigma) : 1.0f;
       if (take) {
 #pragma unroll
-        for (int i = 0; i < OC; ++i) O[i] = fmaf(O[i], beta, v[i]);
+        for (int i = 0; i < OC; i += 2)
+          fma2(O[i], O[i + 1], O[i], O[i + 1], beta, beta, v[i], v[i + 1]);
       }
       ref = take ? pend_sigma : ref * pend_alpha;
       return true;
@@ -553,13 +577,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
           const float dec = ue4m3_decode_fast(S);
           const float c = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
-          float bs[2] = {0.0f, 0.0f};
+          float bs0 = 0.0f, bs1 = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            a[16 * b + i] = ex2_ftz(fmaf(a[16 * b + i], cs, c));  // masked (-inf) -> 0
-            bs[i & 1] += a[16 * b + i];
+          for (int i = 0; i < 16; i += 2) {
+            float x0, x1;
+            fma2(x0, x1, a[16 * b + i], a[16 * b + i + 1], cs, cs, c, c);
+            a[16 * b + i] = ex2_ftz(x0);  // masked (-inf) -> 0
+            a[16 * b + i + 1] = ex2_ftz(x1);
+            add2(bs0, bs1, bs0, bs1, a[16 * b + i], a[16 * b + i + 1]);
           }
-          ls = fmaf(bs[0] + bs[1], dec, ls);
+          ls = fmaf(bs0 + bs1, dec, ls);
           sfw |= S << (8 * b);
           cw[2 * b] = e2m1x8(a + 16 * b);
           cw[2 * b + 1] = e2m1x8(a + 16 * b + 8);
@@ -567,25 +594,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         l = fmaf(ls, sigma_raw, l);
         uint8_t* p4 = sm + L::OFF4_P + st * L::PT4A;
         if constexpr (NB == 2) {
-          *reinterpret_cast<uint4*>(p4 + swz_offset(r, f * NB * 8, BLK / 2)) =
-              make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          *reinterpret_cast<uint16_t*>(p4 + 128 * (BLK / 2) + sf_offset(r, f * NB)) =
-              (uint16_t)sfw;
+          *reinterpret_cast<uint4*>(p4 + p4_codes_off) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint16_t*>(p4 + p4_sf_off) = (uint16_t)sfw;
         } else {
-          *reinterpret_cast<uint2*>(p4 + swz_offset(r, f * NB * 8, BLK / 2)) =
-              make_uint2(cw[0], cw[1]);
-          p4[128 * (BLK / 2) + sf_offset(r, f * NB)] = (uint8_t)sfw;
+          *reinterpret_cast<uint2*>(p4 + p4_codes_off) = make_uint2(cw[0], cw[1]);
+          p4[p4_sf_off] = (uint8_t)sfw;
         }
         pend_sigma_next = sigma;
       } else {
         const float negm = m_new == -INFINITY ? 0.0f : -m_new;
-        float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float l0 = 0.0f, l1 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < SC; ++i) {
-          a[i] = ex2_ftz(fmaf(a[i], cs, negm));  // exp2(-inf) = 0 for masked columns
-          l4[i & 3] += a[i];
+        for (int i = 0; i < SC; i += 2) {
+          float x0, x1;
+          fma2(x0, x1, a[i], a[i + 1], cs, cs, negm, negm);
+          a[i] = ex2_ftz(x0);  // exp2(-inf) = 0 for masked columns
+          a[i + 1] = ex2_ftz(x1);
+          add2(l0, l1, l0, l1, a[i], a[i + 1]);
         }
-        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        l += l0 + l1;
         uint8_t* p16 = sm + L::OFF16_P;
 #pragma unroll
         for (int q8 = 0; q8 < SC / 8; ++q8) {
