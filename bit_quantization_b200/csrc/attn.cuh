@@ -11,14 +11,19 @@
 // quantised in two levels (per row and key tile an fp32 factor rowmax/2688,
 // then NVFP4 16-key blocks).
 //
-// Roles (576 threads):
-//   warps 0-15 softmax + output: query row r (TMEM lane r) is shared by the
-//              four warps r/32 + 4f (f = 0..3), each owning a quarter of the
-//              key columns and of the output columns; they exchange their
-//              partial row max once per tile through shared memory;
-//   warp 16    producer: bulk copies of the pre-quantised tile images;
-//   warp 17    tensor-memory owner and MMA issuer (one elected lane).
-// Tensor memory (512 columns): S double buffer [2][BLK], PV [D], then the
+// Roles (704 threads):
+//   warps 0-15  softmax: query row r (TMEM lane r) is shared by the four
+//               warps r/32 + 4f (f = 0..3), each owning a quarter of the key
+//               columns; they exchange their partial row max once per tile
+//               through shared memory and publish the row's rescale factors;
+//   warps 16-19 correction + output: one thread per row rescales the output
+//               accumulator O (in tensor memory) between PV(t-1) and PV(t),
+//               then divides by the row sum and writes the output and LSE;
+//   warp 20     producer: bulk copies of the pre-quantised tile images;
+//   warp 21     tensor-memory owner and MMA issuer (one elected lane).
+// The MMA accumulates every PV straight into O, so the softmax warps never
+// wait on a PV product.
+// Tensor memory (512 columns): S double buffer [2][BLK], O [D], then the
 // scale factors of Q, K (x2), P (x2) and V (x2).
 // Every wait is bounded; a wait that gives up sets the device status word
 // and the CTA drains and exits.
@@ -79,13 +84,15 @@ struct AttnLayout {
   static constexpr uint32_t OFF_LIST = REGION;
   static constexpr uint32_t MAX_TILES = 512;  // key tiles per sequence
   static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
-  static constexpr uint32_t OFF_XCH = OFF_BAR + 512;  // row-max / row-sum exchange
-  static constexpr uint32_t BYTES = OFF_XCH + 4 * 2 * 4 * 128;
+  static constexpr uint32_t OFF_XCH = OFF_BAR + 512;      // row-max exchange [2][4][128]
+  static constexpr uint32_t OFF_STAT = OFF_XCH + 4 * 2 * 4 * 128;  // [2][alpha, sigma][128]
+  static constexpr uint32_t OFF_FIN = OFF_STAT + 4 * 2 * 2 * 128;  // row sums [4][128], max [128]
+  static constexpr uint32_t BYTES = OFF_FIN + 4 * 5 * 128;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
   // tensor-memory columns
   static constexpr uint32_t T_S = 0;
-  static constexpr uint32_t T_PV = 2 * BLK;
-  static constexpr uint32_t T_QSF = T_PV + D;
+  static constexpr uint32_t T_O = 2 * BLK;
+  static constexpr uint32_t T_QSF = T_O + D;
   static constexpr uint32_t T_KSF = T_QSF + (D / 64) * 4;
   static constexpr uint32_t T_PSF = T_KSF + 2 * (D / 64) * 4;
   static constexpr uint32_t T_VSF = T_PSF + 2 * (BLK / 64) * 4;
@@ -96,17 +103,26 @@ struct AttnLayout {
 };
 
 // Barrier slots inside the barrier area.
+//   SF/SE  S buffer full (MMA commit) / read (softmax)
+//   PF     P tile written (softmax)
+//   OD     PV(t) retired into O (MMA commit), one per P slot
+//   ST     rescale factors of tile t published (softmax, quarter 0)
+//   CF     O rescaled for tile t (correction)
+//   LF     row sums and max published after the last tile (softmax)
 enum : int {
-  B_Q4 = 0, B_Q16 = 1, B_SF = 2 /* 2,3 */, B_SE = 4 /* 4,5 */, B_PF = 6 /* 6,7 */, B_OF = 8,
-  B_OE = 9, B_DONE = 10, B_KVF16 = 11 /* 11,12 */, B_KVE16 = 13 /* 13,14 */,
-  B_KVF4 = 15 /* 15..26 */, B_KVE4 = 27 /* 27..38 */, B_N = 39
+  B_Q4 = 0, B_Q16 = 1, B_SF = 2 /* 2,3 */, B_SE = 4 /* 4,5 */, B_PF = 6 /* 6,7 */,
+  B_OD = 8 /* 8,9 */, B_DONE = 10, B_KVF16 = 11 /* 11,12 */, B_KVE16 = 13 /* 13,14 */,
+  B_KVF4 = 15 /* 15..26 */, B_KVE4 = 27 /* 27..38 */, B_ST = 39 /* 39,40 */, B_CF = 41,
+  B_LF = 42, B_N = 43
 };
 
 constexpr int kSoftmaxWarps = 16;
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
-constexpr int kProducerWarp = kSoftmaxWarps;
-constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kAttnThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kCorrWarp0 = kSoftmaxWarps;
+constexpr int kCorrThreads = 128;
+constexpr int kProducerWarp = kSoftmaxWarps + 4;
+constexpr int kMmaWarp = kSoftmaxWarps + 5;
+constexpr int kAttnThreads = 32 * (kSoftmaxWarps + 6);
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -218,8 +234,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
 
   if (tid == 0) {
     for (int i = 0; i < B_N; ++i) {
-      const uint32_t cnt = (i == B_SE || i == B_SE + 1 || i == B_PF || i == B_PF + 1 || i == B_OE)
-                               ? (uint32_t)kSoftmaxThreads : 1u;
+      uint32_t cnt = 1;
+      if (i == B_SE || i == B_SE + 1 || i == B_PF || i == B_PF + 1 || i == B_LF)
+        cnt = kSoftmaxThreads;
+      if (i == B_ST || i == B_ST + 1 || i == B_CF) cnt = 128;
       mbar_init(&bars[i], cnt);
     }
     *s_abort = 0;
@@ -403,9 +421,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         uint64_t *full, *empty;
         stage_of(t, stg, full, empty, par);
         if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) return false;
-        if (t >= 1 && !mbar_wait(&bars[B_OE], (t - 1) & 1, s_abort)) return false;
+        if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) return false;  // O rescaled for tile t
         tc_fence_after();
-        const uint32_t dO = tmem + L::T_PV;
+        const uint32_t dO = tmem + L::T_O;
         if (!f16) {
           const uint32_t p4 = smem_u32(sm + L::OFF4_P + st * L::PT4A);
           const uint32_t v4 = stg + L::V4_OFF;
@@ -420,7 +438,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           for (int s = 0; s < BLK / 64; ++s)
             mma_nvf4(dO, make_sdesc(p4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
                      make_sdesc(v4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
-                     id_pv4, psf + 4 * s, vsf + 4 * s, s > 0);
+                     id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
         } else {
           const uint32_t p16 = smem_u32(sm + L::OFF16_P);
           const uint32_t v16 = stg + L::V16_OFF;
@@ -428,9 +446,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           for (int s = 0; s < BLK / 16; ++s)
             mma_f16(dO, make_sdesc(p16 + (s / 4) * 128 * 128 + 32 * (s % 4), 16, 1024, SW_128B),
                     make_sdesc(v16 + (s / 4) * D * 128 + 32 * (s % 4), 16, 1024, SW_128B),
-                    id_pv16, s > 0);
+                    id_pv16, t > 0 || s > 0);
         }
-        tc_commit(&bars[B_OF]);
+        tc_commit(&bars[B_OD + st]);
         tc_commit(empty);
         return true;
       };
@@ -449,12 +467,106 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       volatile int* never = &dummy;
       mbar_wait(&bars[B_DONE], 0, never, 200000000ull);
     }
+  } else if (warp >= kCorrWarp0) {
+    // ----------------------------------------------------- correction --
+    // One thread per query row.  The true output accumulator is ref * O, O
+    // being the tensor-memory accumulator.  Tile t with factors
+    // (alpha, sigma) asks for  true O <- alpha * true O + sigma * PV(t); the
+    // MMA only adds PV(t), so before it does, O is multiplied by
+    // beta = alpha * ref / sigma and ref becomes sigma.  A tile with
+    // sigma = 0 adds nothing (the softmax zeroes its P) and only moves ref.
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int row = qt * 128 + r;
+    const bool row_ok = row < len;
+    const uint32_t o_base = tmem + ((uint32_t)(q4 * 32) << 16) + L::T_O;
+    const float* stat = reinterpret_cast<const float*>(sm + L::OFF_STAT);
+    float ref = 1.0f;
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      const int st = t & 1;
+      if (!warp_wait(&bars[B_ST + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+      const float alpha = stat[st * 256 + r];
+      const float sigma = stat[st * 256 + 128 + r];
+      float beta = 1.0f;
+      if (sigma > 0.0f) {
+        if (t > 0) beta = alpha * ref * rcp_ftz(sigma);
+        ref = sigma;
+      } else {
+        ref *= alpha;
+      }
+      // PV(t-1) has to be in O before O is rescaled.  The wait also keeps
+      // this arrival on CF from running a phase ahead of the MMA issuer,
+      // which consumed CF(t-1) before issuing PV(t-1).
+      if (t > 0 && !warp_wait(&bars[B_OD + ((t - 1) & 1)], ((t - 1) >> 1) & 1, s_abort)) {
+        ok = false;
+        break;
+      }
+      if (t > 0 && __any_sync(0xffffffffu, beta != 1.0f)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float v[32];
+          tmem_ld32(o_base + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float y0, y1;
+            fma2(y0, y1, v[i], v[i + 1], beta, beta, 0.0f, 0.0f);
+            v[i] = y0;
+            v[i + 1] = y1;
+          }
+          tmem_st32(o_base + c, v);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_CF]);
+    }
+    // epilogue: O * ref / l after the last PV
+    if (ok && n > 0) ok = warp_wait(&bars[B_OD + ((n - 1) & 1)], ((n - 1) >> 1) & 1, s_abort);
+    if (ok) ok = warp_wait(&bars[B_LF], 0, s_abort);
+    if (ok) {
+      tc_fence_after();
+      const float* fin = reinterpret_cast<const float*>(sm + L::OFF_FIN);
+      const float lt = (fin[r] + fin[128 + r]) + (fin[256 + r] + fin[384 + r]);
+      const float m = fin[512 + r];
+      const float il = (lt > 0.0f && n > 0) ? ref / lt : 0.0f;
+      uint16_t* orow = p.out + ((start + (row_ok ? row : 0)) * p.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float v[32];
+        if (n > 0) {
+          tmem_ld32(o_base + c, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 w;
+            w.x = pack2<DT>(v[i] * il, v[i + 1] * il);
+            w.y = pack2<DT>(v[i + 2] * il, v[i + 3] * il);
+            w.z = pack2<DT>(v[i + 4] * il, v[i + 5] * il);
+            w.w = pack2<DT>(v[i + 6] * il, v[i + 7] * il);
+            *reinterpret_cast<uint4*>(orow + c + i) = w;
+          }
+        }
+      }
+      if (row_ok) {
+        const float lse = lt > 0.0f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
+        const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
+                                        : ((int64_t)seq * p.H + h) * len + row;
+        p.lse[li] = lse;
+      }
+    }
   } else {
     // -------------------------------------------------------- softmax --
     // Four threads per query row: warp w owns TMEM lane quarter w % 4 and
-    // column quarter f = w / 4 of the key columns and of the output columns.
+    // column quarter f = w / 4 of the key columns.
     constexpr int SC = BLK / 4;   // score columns per thread
-    constexpr int OC = D / 4;     // output columns per thread
     constexpr int NB = SC / 16;   // 16-key blocks per thread
     const int q4 = warp & 3, f = warp >> 2;
     const int r = q4 * 32 + lane;
@@ -467,41 +579,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
     float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][4 quarters][128]
+    float* stat = reinterpret_cast<float*>(sm + L::OFF_STAT);
     // shared-memory offsets this thread writes every tile
     const uint32_t p4_codes_off = swz_offset(r, f * NB * 8, BLK / 2);
     const uint32_t p4_sf_off = 128 * (BLK / 2) + sf_offset(r, f * NB);
-    // O holds the output divided by `ref`: the true accumulator is ref * O.
-    float O[OC];
-#pragma unroll
-    for (int c = 0; c < OC; ++c) O[c] = 0.0f;
-    float ref = 1.0f;
     float m = -INFINITY, l = 0.0f;
-    float pend_alpha = 1.0f, pend_sigma = 0.0f, pend_sigma_next = 0.0f;
-    int pending = -1;
-    bool prev16 = false;
     bool ok = true;
-
-    // true O <- alpha * true O + sigma * PV(u), one FMA per column: the
-    // reference factor moves to sigma.  Tiles whose sigma is negligible
-    // (< 2^-60 of the running maximum) only rescale.
-    auto accumulate = [&](int u) -> bool {
-      if (!warp_wait(&bars[B_OF], u & 1, s_abort)) return false;
-      tc_fence_after();
-      float v[OC];
-      tmem_ld_cols<OC>(lane_base + L::T_PV + f * OC, v);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[B_OE]);
-      const bool take = pend_sigma > 0.0f;
-      const float beta = take ? pend_alpha * ref * rcp_ftz(pend_sigma) : 1.0f;
-      if (take) {
-#pragma unroll
-        for (int i = 0; i < OC; i += 2)
-          fma2(O[i], O[i + 1], O[i], O[i + 1], beta, beta, v[i], v[i + 1]);
-      }
-      ref = take ? pend_sigma : ref * pend_alpha;
-      return true;
-    };
 
     for (int t = 0; t < n && ok; ++t) {
       const int st = t & 1;
@@ -513,12 +596,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - f * SC;
       const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
       const float cs = f16 ? p.scale16 : cs4;
-      // FP16 tiles share one P buffer: the previous FP16 PV must be done
-      // (and folded into O) before this tile's P is written.
-      if (f16 && prev16 && pending >= 0) {
-        if (!accumulate(pending)) { ok = false; break; }
-        pending = -1;
-      }
       if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
       float a[SC];
@@ -558,7 +635,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const float rowmax = live ? ex2_ftz(mt - m_new) : 0.0f;
       l *= alpha;
       m = m_new;
-      float ls = 0.0f;
+      // Rescale factors of this tile: the contribution is sigma * PV(t).  An
+      // NVFP4 tile whose row factor is negligible (< 2^-60 of the running
+      // maximum) or not a normal float contributes nothing: its P is zero.
+      const float sigma_raw = (live && rowmax >= 8.6736174e-19f) ? rowmax * (1.0f / 2688.0f) : 0.0f;
+      float sigma = 1.0f;
+      if (!f16) {
+        sigma = sigma_raw * gv;
+        if (!(sigma >= 1.17549435e-38f)) sigma = 0.0f;
+      }
+      if (f == 0) {
+        stat[st * 256 + r] = alpha;
+        stat[st * 256 + 128 + r] = sigma;
+        mbar_arrive(&bars[B_ST + st]);
+      }
       if (!f16) {
         // Two-level quantisation of P.  Relative to the tile max the scaled
         // probabilities are Phat = 2688 * 2^(s - mt) (row factor
@@ -566,15 +656,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         // S_b = ue4m3(max Phat / 6) and the codes E2M1(Phat / S_b), computed
         // as one exponential t = 2^(s + log2(2688) - mt - log2 S_b).
         // l gets sum_b S_b * sum(t) * rowmax / 2688.
-        const bool keep = live && rowmax >= 8.6736174e-19f;  // 2^-60
-        const float sigma_raw = keep ? rowmax * (1.0f / 2688.0f) : 0.0f;
-        const float sigma = sigma_raw * gv;
+        const bool contrib = sigma > 0.0f;
+        float ls = 0.0f;
         uint32_t sfw = 0;
         uint32_t cw[2 * NB];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
-          const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
+          const uint32_t S = contrib ? ue4m3(448.0f * e) : 0u;
           const float dec = ue4m3_decode_fast(S);
           const float c = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
           float bs0 = 0.0f, bs1 = 0.0f;
@@ -592,6 +681,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           cw[2 * b + 1] = e2m1x8(a + 16 * b + 8);
         }
         l = fmaf(ls, sigma_raw, l);
+        // P slot st was last read by PV(t-2)
+        if (t >= 2 && !warp_wait(&bars[B_OD + st], ((t >> 1) - 1) & 1, s_abort)) {
+          ok = false;
+          break;
+        }
         uint8_t* p4 = sm + L::OFF4_P + st * L::PT4A;
         if constexpr (NB == 2) {
           *reinterpret_cast<uint4*>(p4 + p4_codes_off) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -600,7 +694,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           *reinterpret_cast<uint2*>(p4 + p4_codes_off) = make_uint2(cw[0], cw[1]);
           p4[p4_sf_off] = (uint8_t)sfw;
         }
-        pend_sigma_next = sigma;
       } else {
         const float negm = m_new == -INFINITY ? 0.0f : -m_new;
         float l0 = 0.0f, l1 = 0.0f;
@@ -613,6 +706,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           add2(l0, l1, l0, l1, a[i], a[i + 1]);
         }
         l += l0 + l1;
+        // FP16 tiles share one P buffer: the previous FP16 PV must be done.
+        // (The first FP16 tile needs no wait: its scores only arrive after
+        // the last NVFP4 PV has retired.)
+        if (t > n4 && !warp_wait(&bars[B_OD + ((t - 1) & 1)], ((t - 1) >> 1) & 1, s_abort)) {
+          ok = false;
+          break;
+        }
         uint8_t* p16 = sm + L::OFF16_P;
 #pragma unroll
         for (int q8 = 0; q8 < SC / 8; ++q8) {
@@ -624,45 +724,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
                                     swz_offset(r, (key0 % 64) * 2, 128)) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        pend_sigma_next = 1.0f;
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_PF + st]);
-      if (pending >= 0) {
-        if (!accumulate(pending)) { ok = false; break; }
-      }
-      pending = t;
-      pend_alpha = alpha;  // applied to O before PV(t) is added
-      pend_sigma = pend_sigma_next;
-      prev16 = f16;
     }
-    if (ok && pending >= 0) ok = accumulate(pending);
-    // combine the four quarters' partial sums, then write this quarter of the
-    // row (the exchange area is free: every thread has passed its last tile)
-    named_bar_sync(1 + q4, 128);
-    float* xl = xch;
-    xl[f * 128 + r] = l;
-    named_bar_sync(1 + q4, 128);
-    const float lt = (xl[r] + xl[128 + r]) + (xl[256 + r] + xl[384 + r]);
-    if (ok && row_ok) {
-      const float il = lt > 0.0f ? ref / lt : 0.0f;
-      uint16_t* orow = p.out + ((start + row) * p.H + h) * D + f * OC;
-#pragma unroll
-      for (int c = 0; c < OC; c += 8) {
-        uint4 w;
-        w.x = pack2<DT>(O[c] * il, O[c + 1] * il);
-        w.y = pack2<DT>(O[c + 2] * il, O[c + 3] * il);
-        w.z = pack2<DT>(O[c + 4] * il, O[c + 5] * il);
-        w.w = pack2<DT>(O[c + 6] * il, O[c + 7] * il);
-        *reinterpret_cast<uint4*>(orow + c) = w;
-      }
-      if (f == 0) {
-        const float lse = lt > 0.0f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
-        const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
-                                        : ((int64_t)seq * p.H + h) * len + row;
-        p.lse[li] = lse;
-      }
-    }
+    // publish this quarter's row sum (and the row max) for the output warps
+    float* fin = reinterpret_cast<float*>(sm + L::OFF_FIN);
+    fin[f * 128 + r] = l;
+    if (f == 0) fin[512 + r] = m;
+    mbar_arrive(&bars[B_LF]);
   }
   tc_fence_before();
   __syncthreads();
