@@ -12,15 +12,17 @@
 // then NVFP4 16-key blocks).
 //
 // Roles (704 threads):
-//   warps 0-15  softmax: query row r (TMEM lane r) is shared by the four
-//               warps r/32 + 4f (f = 0..3), each owning a quarter of the key
-//               columns; they exchange their partial row max once per tile
-//               through shared memory and publish the row's rescale factors;
-//   warps 16-19 correction + output: one thread per row rescales the output
-//               accumulator O (in tensor memory) between PV(t-1) and PV(t),
-//               then divides by the row sum and writes the output and LSE;
+//   warps 0-15  softmax, two groups of eight taking alternate key tiles;
+//               in a group, query row r (TMEM lane r) is shared by two
+//               warps, each owning half of the key columns; the groups take
+//               turns at the exponentials;
+//   warps 16-19 correction + output: one thread per row keeps the running
+//               max and sum, rescales the output accumulator O (in tensor
+//               memory) between PV(t-1) and PV(t), then divides by the row
+//               sum and writes the output and LSE;
 //   warp 20     producer: bulk copies of the pre-quantised tile images;
-//   warp 21     tensor-memory owner and MMA issuer (one elected lane).
+//   warp 21     tensor-memory owner and QK^T issuer (one elected lane);
+//   warp 22     PV issuer (one elected lane).
 // The MMA accumulates every PV straight into O, so the softmax warps never
 // wait on a PV product.
 // Tensor memory (512 columns): S double buffer [2][BLK], O [D], then the
@@ -84,10 +86,11 @@ struct AttnLayout {
   static constexpr uint32_t OFF_LIST = REGION;
   static constexpr uint32_t MAX_TILES = 512;  // key tiles per sequence
   static constexpr uint32_t OFF_BAR = OFF_LIST + 2 * 2 * MAX_TILES;
-  static constexpr uint32_t OFF_XCH = OFF_BAR + 512;      // row-max exchange [2][4][128]
-  static constexpr uint32_t OFF_STAT = OFF_XCH + 4 * 2 * 4 * 128;  // [2][alpha, sigma][128]
-  static constexpr uint32_t OFF_FIN = OFF_STAT + 4 * 2 * 2 * 128;  // row sums [4][128], max [128]
-  static constexpr uint32_t BYTES = OFF_FIN + 4 * 5 * 128;
+  static constexpr uint32_t OFF_XCH = OFF_BAR + 1024;  // half-row maxima [group][slot][half][128]
+  static constexpr uint32_t OFF_STA = OFF_XCH + 4 * 2 * 2 * 2 * 128;  // tile row max [4][128]
+  static constexpr uint32_t OFF_STB = OFF_STA + 4 * 4 * 128;          // tile row sums [4][2][128]
+  static constexpr uint32_t OFF_MR = OFF_STB + 4 * 4 * 2 * 128;       // running max [4][128]
+  static constexpr uint32_t BYTES = OFF_MR + 4 * 4 * 128;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // base alignment slack
   // tensor-memory columns
   static constexpr uint32_t T_S = 0;
@@ -103,30 +106,41 @@ struct AttnLayout {
 };
 
 // Barrier slots inside the barrier area.
-//   SF/SE  S buffer full (MMA commit) / read (softmax)
-//   PF     P tile written (softmax)
+//   SF/SE  S buffer full (MMA commit) / read (softmax group)
+//   PF     P tile written (softmax group)
 //   OD     PV(t) retired into O (MMA commit), one per P slot
-//   ST     rescale factors of tile t published (softmax, quarter 0)
+//   STA    row max of tile t published (softmax), four slots
+//   STB    row sums of tile t published (softmax), four slots
+//   MR     running max through tile t published (correction), four slots
 //   CF     O rescaled for tile t (correction)
-//   LF     row sums and max published after the last tile (softmax)
+//   XCH    half-row maxima exchanged, per (group, lane quarter, slot)
+//   TURN   turn at the exponentials, one per softmax group
+// Four-slot rings, each slot reused four tiles later:
+//   STA(t+4) is written by the group of tiles t, t+2, t+4 after it stored
+//   P(t+2), which waited for PV(t), issued after correction step t had read
+//   STA(t);
+//   STB(t) is read one correction step late (step t+1); STB(t+4) follows
+//   the group's P(t+4), which waited for PV(t+2), issued after step t+2;
+//   MR(t+4) is written by correction step t+4 after PV(t+3) retired; PV(t+1)
+//   was issued earlier by the same thread, after the softmax of tile t+1
+//   (the reader of MR(t)) had finished.
 enum : int {
   B_Q4 = 0, B_Q16 = 1, B_SF = 2 /* 2,3 */, B_SE = 4 /* 4,5 */, B_PF = 6 /* 6,7 */,
   B_OD = 8 /* 8,9 */, B_DONE = 10, B_KVF16 = 11 /* 11,12 */, B_KVE16 = 13 /* 13,14 */,
-  B_KVF4 = 15 /* 15..26 */, B_KVE4 = 27 /* 27..38 */, B_ST = 39 /* 39,40 */, B_CF = 41,
-  B_LF = 42, B_N = 43
+  B_KVF4 = 15 /* 15..26 */, B_KVE4 = 27 /* 27..38 */, B_STA = 39 /* 39..42 */,
+  B_STB = 43 /* 43..46 */, B_MR = 47 /* 47..50 */, B_CF = 51, B_XCH = 52 /* 52..67 */,
+  B_TURN = 68 /* 68,69 */, B_N = 70
 };
 
 constexpr int kSoftmaxWarps = 16;
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kGroupThreads = kSoftmaxThreads / 2;
 constexpr int kCorrWarp0 = kSoftmaxWarps;
 constexpr int kCorrThreads = 128;
 constexpr int kProducerWarp = kSoftmaxWarps + 4;
 constexpr int kMmaWarp = kSoftmaxWarps + 5;
-constexpr int kAttnThreads = 32 * (kSoftmaxWarps + 6);
-
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
+constexpr int kPvWarp = kSoftmaxWarps + 6;
+constexpr int kAttnThreads = 32 * (kSoftmaxWarps + 7);
 
 // Packed fp32 pairs (one instruction for two lanes' worth of fma / add;
 // each half rounds exactly as the scalar operation).
@@ -235,9 +249,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
   if (tid == 0) {
     for (int i = 0; i < B_N; ++i) {
       uint32_t cnt = 1;
-      if (i == B_SE || i == B_SE + 1 || i == B_PF || i == B_PF + 1 || i == B_LF)
-        cnt = kSoftmaxThreads;
-      if (i == B_ST || i == B_ST + 1 || i == B_CF) cnt = 128;
+      if ((i >= B_SE && i < B_SE + 2) || (i >= B_PF && i < B_PF + 2) ||
+          (i >= B_STB && i < B_STB + 4) || (i >= B_TURN && i < B_TURN + 2))
+        cnt = kGroupThreads;
+      if ((i >= B_STA && i < B_STA + 4) || (i >= B_MR && i < B_MR + 4) || i == B_CF) cnt = 128;
+      if (i >= B_XCH && i < B_XCH + 16) cnt = 64;
+      if (i == B_DONE) cnt = 2;  // one commit per MMA issuer
       mbar_init(&bars[i], cnt);
     }
     *s_abort = 0;
@@ -345,123 +362,130 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         if (last16[sl] >= 0)
           mbar_wait(&bars[B_KVF16 + sl], (last16[sl] / L::NS16) & 1, never, 200000000ull);
     }
-  } else if (warp == kMmaWarp) {
-    // ----------------------------------------------------- MMA issuer --
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // ---------------------------------------------------- MMA issuers --
+    // One elected lane issues QK^T for every tile in order (warp kMmaWarp),
+    // another PV (warp kPvWarp), so scores for the next tiles never queue
+    // behind a PV that waits for its P tile or for the correction step.
+    // QK^T(t) reads the K half of its stage before PV(t) is issued (PV(t)
+    // follows P(t), which follows the scores of tile t), so the PV side's
+    // commit alone frees the stage.
     if (lane == 0) {
-      const uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
-      const uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
-      bool q4_ready = false, q16_ready = false;
-      const uint32_t q4a = smem_u32(q4s), q16a = smem_u32(q16s);
-      // stage of tile t: NVFP4 tiles 0..n4-1 cycle through NS4 stages, FP16
-      // tiles through NS16
-      auto stage_of = [&](int t, uint32_t& addr, uint64_t*& full, uint64_t*& empty,
-                          uint32_t& parity) {
-        if (t < n4) {
-          const int sl = t % L::NS4;
-          addr = smem_u32(sm + L::OFF4_STG + sl * L::STG4);
-          full = &bars[B_KVF4 + sl];
-          empty = &bars[B_KVE4 + sl];
-          parity = (t / L::NS4) & 1;
-        } else {
-          const int i = t - n4, sl = i % L::NS16;
-          addr = smem_u32(sm + L::OFF16_STG + sl * L::STG16);
-          full = &bars[B_KVF16 + sl];
-          empty = &bars[B_KVE16 + sl];
-          parity = (i / L::NS16) & 1;
+      constexpr uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
+      constexpr uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
+      constexpr uint32_t swz_d = swz_mode_for_pitch(D / 2), swz_b = swz_mode_for_pitch(BLK / 2);
+      // Descriptors of every operand at stage / slot 0, built once: a
+      // descriptor's start field is the address in 16-byte units, so an
+      // operand at byte offset o further on is the descriptor + (o >> 4).
+      const uint32_t base = smem_u32(sm);
+      const uint64_t d_sf = make_sdesc(base, 512, 128, SW_NONE);  // + (byte offset >> 4)
+      int sl = 0, par = 0;  // stage ring position (NVFP4 ring, then FP16 ring)
+      auto advance = [&](int t) {
+        const int ns = t < n4 ? (int)L::NS4 : (int)L::NS16;
+        if (t + 1 == n4) {
+          sl = 0;
+          par = 0;
+        } else if (++sl == ns) {
+          sl = 0;
+          par ^= 1;
         }
       };
-      auto issue_qk = [&](int t) -> bool {
-        const int st = t & 1;
-        const bool f16 = t >= n4;
-        uint32_t stg, par;
-        uint64_t *full, *empty;
-        stage_of(t, stg, full, empty, par);
-        if (!mbar_wait(full, par, s_abort)) return false;
-        if (!f16 && !q4_ready) {
-          if (!mbar_wait(&bars[B_Q4], 0, s_abort)) return false;
-          tc_fence_after();
+      bool ok = true;
+      if (warp == kMmaWarp) {
+        const uint64_t d_q4 = make_sdesc(base + L::OFF4_Q, 16, 8 * (D / 2), swz_d);
+        const uint64_t d_k4 = make_sdesc(base + L::OFF4_STG, 16, 8 * (D / 2), swz_d);
+        const uint64_t d_q16 = make_sdesc(base + L::OFF16_Q, 16, 1024, SW_128B);
+        const uint64_t d_k16 = make_sdesc(base + L::OFF16_STG, 16, 1024, SW_128B);
+        bool q4_ready = false, q16_ready = false;
+        for (int t = 0; t < n && ok; ++t) {
+          const int st = t & 1;
+          const bool f16 = t >= n4;
+          uint64_t* full = f16 ? &bars[B_KVF16 + sl] : &bars[B_KVF4 + sl];
+          if (!mbar_wait(full, par, s_abort)) { ok = false; break; }
+          if (!f16 && !q4_ready) {
+            if (!mbar_wait(&bars[B_Q4], 0, s_abort)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int s = 0; s < D / 64; ++s)
-            tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
-                             make_sdesc(q4a + 128 * (D / 2) + 512 * s, 512, 128, SW_NONE));
-          q4_ready = true;
-        }
-        if (f16 && !q16_ready) {
-          if (!mbar_wait(&bars[B_Q16], 0, s_abort)) return false;
-          q16_ready = true;
-        }
-        if (t >= 2 && !mbar_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) return false;
-        tc_fence_after();
-        const uint32_t dS = tmem + L::T_S + st * BLK;
-        if (!f16) {
-          const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
-#pragma unroll
-          for (int s = 0; s < D / 64; ++s)
-            tc_cp_32x128b_x4(ksf + 4 * s,
-                             make_sdesc(stg + BLK * (D / 2) + 512 * s, 512, 128, SW_NONE));
-#pragma unroll
-          for (int s = 0; s < D / 64; ++s)
-            mma_nvf4(dS, make_sdesc(q4a + 32 * s, 16, 8 * (D / 2), swz_mode_for_pitch(D / 2)),
-                     make_sdesc(stg + 32 * s, 16, 8 * (D / 2), swz_mode_for_pitch(D / 2)),
-                     id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s, s > 0);
-        } else {
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s)
-            mma_f16(dS, make_sdesc(q16a + (s / 4) * 128 * 128 + 32 * (s % 4), 16, 1024, SW_128B),
-                    make_sdesc(stg + (s / 4) * BLK * 128 + 32 * (s % 4), 16, 1024, SW_128B),
-                    id_qk16, s > 0);
-        }
-        tc_commit(&bars[B_SF + st]);
-        return true;
-      };
-      auto issue_pv = [&](int t) -> bool {
-        const int st = t & 1;
-        const bool f16 = t >= n4;
-        uint32_t stg, par;
-        uint64_t *full, *empty;
-        stage_of(t, stg, full, empty, par);
-        if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) return false;
-        if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) return false;  // O rescaled for tile t
-        tc_fence_after();
-        const uint32_t dO = tmem + L::T_O;
-        if (!f16) {
-          const uint32_t p4 = smem_u32(sm + L::OFF4_P + st * L::PT4A);
-          const uint32_t v4 = stg + L::V4_OFF;
-          const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
-          const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
-#pragma unroll
-          for (int s = 0; s < BLK / 64; ++s) {
-            tc_cp_32x128b_x4(psf + 4 * s, make_sdesc(p4 + 128 * (BLK / 2) + 512 * s, 512, 128, SW_NONE));
-            tc_cp_32x128b_x4(vsf + 4 * s, make_sdesc(v4 + D * (BLK / 2) + 512 * s, 512, 128, SW_NONE));
+            for (int s = 0; s < D / 64; ++s)
+              tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
+                               d_sf + ((L::OFF4_Q + 128 * (D / 2) + 512 * s) >> 4));
+            q4_ready = true;
           }
+          if (f16 && !q16_ready) {
+            if (!mbar_wait(&bars[B_Q16], 0, s_abort)) { ok = false; break; }
+            q16_ready = true;
+          }
+          // the S buffer of tile t-2 has been read
+          if (t >= 2 && !mbar_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dS = tmem + L::T_S + st * BLK;
+          if (!f16) {
+            const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
+            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
 #pragma unroll
-          for (int s = 0; s < BLK / 64; ++s)
-            mma_nvf4(dO, make_sdesc(p4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
-                     make_sdesc(v4 + 32 * s, 16, 8 * (BLK / 2), swz_mode_for_pitch(BLK / 2)),
-                     id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
-        } else {
-          const uint32_t p16 = smem_u32(sm + L::OFF16_P);
-          const uint32_t v16 = stg + L::V16_OFF;
+            for (int s = 0; s < D / 64; ++s)
+              tc_cp_32x128b_x4(ksf + 4 * s,
+                               d_sf + ((L::OFF4_STG + BLK * (D / 2) + 512 * s) >> 4) + so);
 #pragma unroll
-          for (int s = 0; s < BLK / 16; ++s)
-            mma_f16(dO, make_sdesc(p16 + (s / 4) * 128 * 128 + 32 * (s % 4), 16, 1024, SW_128B),
-                    make_sdesc(v16 + (s / 4) * D * 128 + 32 * (s % 4), 16, 1024, SW_128B),
-                    id_pv16, t > 0 || s > 0);
+            for (int s = 0; s < D / 64; ++s)
+              mma_nvf4(dS, d_q4 + 2 * s, d_k4 + so + 2 * s, id_qk4, tmem + L::T_QSF + 4 * s,
+                       ksf + 4 * s, s > 0);
+          } else {
+            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+              mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                      d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
+          }
+          tc_commit(&bars[B_SF + st]);
+          advance(t);
         }
-        tc_commit(&bars[B_OD + st]);
-        tc_commit(empty);
-        return true;
-      };
-      // QK^T of tile t+1 goes out before PV of tile t, except at the switch
-      // to the FP16 phase: the first FP16 tile is only loaded once the last
-      // NVFP4 PV has retired.
-      bool ok = n > 0 ? issue_qk(0) : true;
-      for (int t = 0; t < n && ok; ++t) {
-        const bool crossing = t + 1 == n4;
-        if (t + 1 < n && !crossing) ok = issue_qk(t + 1);
-        if (ok) ok = issue_pv(t);
-        if (ok && t + 1 < n && crossing) ok = issue_qk(t + 1);
+      } else {
+        const uint64_t d_p4 = make_sdesc(base + L::OFF4_P, 16, 8 * (BLK / 2), swz_b);
+        const uint64_t d_v4 = make_sdesc(base + L::OFF4_STG + L::V4_OFF, 16, 8 * (BLK / 2), swz_b);
+        const uint64_t d_p16 = make_sdesc(base + L::OFF16_P, 16, 1024, SW_128B);
+        const uint64_t d_v16 = make_sdesc(base + L::OFF16_STG + L::V16_OFF, 16, 1024, SW_128B);
+        for (int t = 0; t < n && ok; ++t) {
+          const int st = t & 1;
+          const bool f16 = t >= n4;
+          uint64_t* empty = f16 ? &bars[B_KVE16 + sl] : &bars[B_KVE4 + sl];
+          if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
+          tc_fence_after();
+          const uint32_t dO = tmem + L::T_O;
+          if (!f16) {
+            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
+            const uint32_t po = (uint32_t)st * (L::PT4A >> 4);
+            const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
+            const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
+#pragma unroll
+            for (int s = 0; s < BLK / 64; ++s) {
+              tc_cp_32x128b_x4(psf + 4 * s,
+                               d_sf + ((L::OFF4_P + 128 * (BLK / 2) + 512 * s) >> 4) + po);
+              tc_cp_32x128b_x4(vsf + 4 * s, d_sf + ((L::OFF4_STG + L::V4_OFF + D * (BLK / 2) +
+                                                     512 * s) >> 4) + so);
+            }
+#pragma unroll
+            for (int s = 0; s < BLK / 64; ++s)
+              mma_nvf4(dO, d_p4 + po + 2 * s, d_v4 + so + 2 * s, id_pv4, psf + 4 * s,
+                       vsf + 4 * s, t > 0 || s > 0);
+          } else {
+            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
+#pragma unroll
+            for (int s = 0; s < BLK / 16; ++s)
+              mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                      d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
+                      t > 0 || s > 0);
+          }
+          tc_commit(&bars[B_OD + st]);
+          tc_commit(empty);
+          advance(t);
+        }
       }
+      // every MMA of both issuers has completed before the CTA ends
       tc_commit(&bars[B_DONE]);
       int dummy = 0;
       volatile int* never = &dummy;
@@ -469,25 +493,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     }
   } else if (warp >= kCorrWarp0) {
     // ----------------------------------------------------- correction --
-    // One thread per query row.  The true output accumulator is ref * O, O
-    // being the tensor-memory accumulator.  Tile t with factors
-    // (alpha, sigma) asks for  true O <- alpha * true O + sigma * PV(t); the
-    // MMA only adds PV(t), so before it does, O is multiplied by
-    // beta = alpha * ref / sigma and ref becomes sigma.  A tile with
-    // sigma = 0 adds nothing (the softmax zeroes its P) and only moves ref.
+    // One thread per query row; it owns the row's running max m and sum l.
+    // The true output accumulator is ref * O, O being the tensor-memory
+    // accumulator.  Tile t, taken by the softmax relative to its own row max
+    // mt (NVFP4) or to the running max (FP16), asks for
+    //   true O <- alpha * true O + sigma * PV(t)
+    // with alpha = 2^(m - m_new) and sigma = 2^(mt - m_new) / 2688 * g_V
+    // (NVFP4) or 1 (FP16).  The MMA only adds PV(t), so before it does, O is
+    // multiplied by beta = alpha * ref / sigma and ref becomes sigma.  An
+    // NVFP4 tile whose row factor is negligible (2^(mt - m_new) < 2^-60) or
+    // not a normal float adds nothing: its row of P gets zero block scales.
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const int row = qt * 128 + r;
     const bool row_ok = row < len;
     const uint32_t o_base = tmem + ((uint32_t)(q4 * 32) << 16) + L::T_O;
-    const float* stat = reinterpret_cast<const float*>(sm + L::OFF_STAT);
-    float ref = 1.0f;
+    const float* sta = reinterpret_cast<const float*>(sm + L::OFF_STA);
+    const float* stb = reinterpret_cast<const float*>(sm + L::OFF_STB);
+    float* mrw = reinterpret_cast<float*>(sm + L::OFF_MR);
+    const float gv = tensor_scale_from_amax(p.amax[2]);
+    float m = -INFINITY, l = 0.0f, ref = 1.0f;
+    float pend_alpha = 1.0f, pend_sigma_raw = 0.0f;
     bool ok = true;
+    // l <- alpha * l + sigma_raw * (row sum of tile u), in tile order
+    auto accumulate_l = [&](int u) -> bool {
+      const int s4 = u & 3;
+      if (!warp_wait(&bars[B_STB + s4], (u >> 2) & 1, s_abort)) return false;
+      const float ls = stb[(2 * s4) * 128 + r] + stb[(2 * s4 + 1) * 128 + r];
+      l *= pend_alpha;
+      l = u >= n4 ? l + ls : fmaf(ls, pend_sigma_raw, l);
+      return true;
+    };
     for (int t = 0; t < n; ++t) {
-      const int st = t & 1;
-      if (!warp_wait(&bars[B_ST + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
-      const float alpha = stat[st * 256 + r];
-      const float sigma = stat[st * 256 + 128 + r];
+      const int s4 = t & 3;
+      const bool f16 = t >= n4;
+      if (!warp_wait(&bars[B_STA + s4], (t >> 2) & 1, s_abort)) { ok = false; break; }
+      const float mt = sta[s4 * 128 + r];
+      const float m_new = fmaxf(m, mt);
+      const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(m - m_new);
+      float sigma = 1.0f, sigma_raw = 1.0f;
+      bool drop = false;
+      if (!f16) {
+        const bool live = mt != -INFINITY;
+        const float rowmax = live ? ex2_ftz(mt - m_new) : 0.0f;
+        sigma_raw = (live && rowmax >= 8.6736174e-19f) ? rowmax * (1.0f / 2688.0f) : 0.0f;  // 2^-60
+        sigma = sigma_raw * gv;
+        if (!(sigma >= 1.17549435e-38f)) sigma = sigma_raw = 0.0f;
+        drop = live && sigma == 0.0f;
+      }
+      // running max through tile t, for the FP16 softmax of tile t+1
+      mrw[s4 * 128 + r] = m_new;
+      mbar_arrive(&bars[B_MR + s4]);
+      m = m_new;
       float beta = 1.0f;
       if (sigma > 0.0f) {
         if (t > 0) beta = alpha * ref * rcp_ftz(sigma);
@@ -510,28 +567,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           tmem_ld32(o_base + c, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float y0, y1;
-            fma2(y0, y1, v[i], v[i + 1], beta, beta, 0.0f, 0.0f);
-            v[i] = y0;
-            v[i + 1] = y1;
-          }
+          for (int i = 0; i < 32; i += 2)
+            fma2(v[i], v[i + 1], v[i], v[i + 1], beta, beta, 0.0f, 0.0f);
           tmem_st32(o_base + c, v);
         }
         tmem_st_wait();
       }
+      if (__any_sync(0xffffffffu, drop)) {
+        // zero this row's block scales once P(t) is in shared memory
+        if (!warp_wait(&bars[B_PF + (t & 1)], (t >> 1) & 1, s_abort)) { ok = false; break; }
+        if (drop) {
+          uint8_t* psf = sm + L::OFF4_P + (t & 1) * L::PT4A + 128 * (BLK / 2);
+#pragma unroll
+          for (int a = 0; a < BLK / 64; ++a)
+            *reinterpret_cast<uint32_t*>(psf + sf_offset(r, 4 * a)) = 0u;
+        }
+        fence_proxy_async_smem();
+      }
       tc_fence_before();
       mbar_arrive(&bars[B_CF]);
+      // the row sum of tile t-1 (two column halves), one step late: it is
+      // published after P(t-1), which PV(t-1), waited for above, follows
+      if (t > 0) {
+        if (!accumulate_l(t - 1)) { ok = false; break; }
+      }
+      pend_alpha = alpha;
+      pend_sigma_raw = sigma_raw;
     }
+    if (ok && n > 0) ok = accumulate_l(n - 1);
     // epilogue: O * ref / l after the last PV
     if (ok && n > 0) ok = warp_wait(&bars[B_OD + ((n - 1) & 1)], ((n - 1) >> 1) & 1, s_abort);
-    if (ok) ok = warp_wait(&bars[B_LF], 0, s_abort);
     if (ok) {
       tc_fence_after();
-      const float* fin = reinterpret_cast<const float*>(sm + L::OFF_FIN);
-      const float lt = (fin[r] + fin[128 + r]) + (fin[256 + r] + fin[384 + r]);
-      const float m = fin[512 + r];
-      const float il = (lt > 0.0f && n > 0) ? ref / lt : 0.0f;
+      const float il = (l > 0.0f && n > 0) ? ref / l : 0.0f;
       uint16_t* orow = p.out + ((start + (row_ok ? row : 0)) * p.H + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
@@ -556,7 +624,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         }
       }
       if (row_ok) {
-        const float lse = lt > 0.0f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
+        const float lse = l > 0.0f ? m * 0.6931471805599453f + logf(l) : -INFINITY;
         const int64_t li = p.lse_varlen ? (int64_t)h * p.total + start + row
                                         : ((int64_t)seq * p.H + h) * len + row;
         p.lse[li] = lse;
@@ -564,175 +632,213 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     }
   } else {
     // -------------------------------------------------------- softmax --
-    // Four threads per query row: warp w owns TMEM lane quarter w % 4 and
-    // column quarter f = w / 4 of the key columns.
-    constexpr int SC = BLK / 4;   // score columns per thread
-    constexpr int NB = SC / 16;   // 16-key blocks per thread
-    const int q4 = warp & 3, f = warp >> 2;
+    // Two groups of eight warps take alternate key tiles: group g = w / 8
+    // the tiles t = g, g + 2, ... (S buffer and P slot g).  Within a group,
+    // query row r (TMEM lane r) is shared by the warps r/32 + 4(2g + hf),
+    // hf = 0, 1, each owning half of the key columns.  The groups take turns
+    // at the exponentials, so one group's loads and reductions run while the
+    // other keeps the MUFU busy.  No running state lives here: an NVFP4 tile
+    // is taken relative to its own row max, an FP16 tile relative to the
+    // running max published by the correction warps.
+    constexpr int SC = BLK / 2;   // score columns per thread
+    constexpr int NCH = SC / 32;  // 32-column chunks
+    const int q4 = warp & 3, f = warp >> 2, g = f >> 1, hf = f & 1;
     const int r = q4 * 32 + lane;
     const int row = qt * 128 + r;
     const bool row_ok = row < len;
     const int mbit = 13 + ((BLK == 64 && r >= 64) ? 1 : 0);  // tile-list bit of this row's block
     const float gq = tensor_scale_from_amax(p.amax[0]);
     const float gk = tensor_scale_from_amax(p.amax[1]);
-    const float gv = tensor_scale_from_amax(p.amax[2]);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
-    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-    float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH);  // [2 slots][4 quarters][128]
-    float* stat = reinterpret_cast<float*>(sm + L::OFF_STAT);
-    // shared-memory offsets this thread writes every tile
-    const uint32_t p4_codes_off = swz_offset(r, f * NB * 8, BLK / 2);
-    const uint32_t p4_sf_off = 128 * (BLK / 2) + sf_offset(r, f * NB);
-    float m = -INFINITY, l = 0.0f;
+    const uint32_t s_base = tmem + ((uint32_t)(q4 * 32) << 16) + L::T_S + g * BLK + hf * SC;
+    float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH) + g * 512;  // [2 slots][2 halves][128]
+    float* sta = reinterpret_cast<float*>(sm + L::OFF_STA);
+    float* stb = reinterpret_cast<float*>(sm + L::OFF_STB);
+    const float* mr = reinterpret_cast<const float*>(sm + L::OFF_MR);
+    uint64_t* xbar = &bars[B_XCH + (g * 4 + q4) * 2];
+    // shared-memory offsets this thread writes every NVFP4 tile
+    uint32_t p4_codes_off[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) p4_codes_off[c] = swz_offset(r, hf * (SC / 2) + 16 * c, BLK / 2);
+    const uint32_t p4_sf_off = 128 * (BLK / 2) + sf_offset(r, hf * (SC / 16));
+    uint8_t* p4 = sm + L::OFF4_P + g * L::PT4A;
+    uint8_t* p16 = sm + L::OFF16_P;
     bool ok = true;
+    // the first turn at the exponentials goes to group 0
+    if (g == 1) mbar_arrive(&bars[B_TURN]);
 
-    for (int t = 0; t < n && ok; ++t) {
-      const int st = t & 1;
+    for (int t = g; t < n && ok; t += 2) {
+      const int u = t >> 1;  // this group's tile count
       const uint32_t ent = s_list[t];
       const int j = ent & 0x1FFF;
       const bool f16 = (ent >> 15) != 0;
       const bool pair_ok = row_ok && ((ent >> mbit) & 1u);
-      // last valid score column of this thread's quarter (negative: none)
-      const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - f * SC;
+      // last valid score column of this thread's half (negative: none)
+      const int lim = (pair_ok ? min(len - 1, p.causal ? row : len - 1) - j * BLK : -1) - hf * SC;
       const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
       const float cs = f16 ? p.scale16 : cs4;
-      if (!warp_wait(&bars[B_SF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+      if (!warp_wait(&bars[B_SF + g], u & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
-      float a[SC];
-      tmem_ld_cols<SC>(lane_base + L::T_S + st * BLK + f * SC, a);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[B_SE + st]);  // S buffer free for QK^T of tile t+2
-      if (!full) {
+      // pass 1: block maxima of the raw scores (the scale is positive)
+      float bm[2 * NCH];
 #pragma unroll
-        for (int i = 0; i < SC; ++i) a[i] = i <= lim ? a[i] : -INFINITY;
-      }
-      // block maxima of the raw scores (the scale is positive, so the max of
-      // the scaled scores is the scaled max)
-      float bm[NB];
+      for (int c = 0; c < NCH; ++c) {
+        float a[32];
+        tmem_ld32(s_base + 32 * c, a);
+        tmem_ld_wait();
+        if (!full) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float* x = a + 16 * b;
-        float x0 = fmaxf(x[0], x[1]), x1 = fmaxf(x[2], x[3]);
-        float x2 = fmaxf(x[4], x[5]), x3 = fmaxf(x[6], x[7]);
-        x0 = fmaxf(x0, fmaxf(x[8], x[9]));
-        x1 = fmaxf(x1, fmaxf(x[10], x[11]));
-        x2 = fmaxf(x2, fmaxf(x[12], x[13]));
-        x3 = fmaxf(x3, fmaxf(x[14], x[15]));
-        bm[b] = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+          for (int i = 0; i < 32; ++i) a[i] = i + 32 * c <= lim ? a[i] : -INFINITY;
+        }
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const float* x = a + 16 * b;
+          float x0 = fmaxf(x[0], x[1]), x1 = fmaxf(x[2], x[3]);
+          float x2 = fmaxf(x[4], x[5]), x3 = fmaxf(x[6], x[7]);
+          x0 = fmaxf(x0, fmaxf(x[8], x[9]));
+          x1 = fmaxf(x1, fmaxf(x[10], x[11]));
+          x2 = fmaxf(x2, fmaxf(x[12], x[13]));
+          x3 = fmaxf(x3, fmaxf(x[14], x[15]));
+          bm[2 * c + b] = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        }
       }
       float mh = bm[0];
 #pragma unroll
-      for (int b = 1; b < NB; ++b) mh = fmaxf(mh, bm[b]);
-      float* xs = xch + st * 512;
-      xs[f * 128 + r] = mh;
-      named_bar_sync(1 + q4, 128);
-      const float mt_raw = fmaxf(fmaxf(xs[r], xs[128 + r]), fmaxf(xs[256 + r], xs[384 + r]));
-      const float mt = mt_raw * cs;
-      const float m_new = fmaxf(m, mt);
-      const float alpha = (m == -INFINITY) ? 1.0f : ex2_ftz(m - m_new);
+      for (int b = 1; b < 2 * NCH; ++b) mh = fmaxf(mh, bm[b]);
+      // exchange the half-row maxima with the partner warp
+      float* xs = xch + (u & 1) * 256;
+      xs[hf * 128 + r] = mh;
+      mbar_arrive(&xbar[u & 1]);
+      if (!warp_wait(&xbar[u & 1], (u >> 1) & 1, s_abort)) { ok = false; break; }
+      const float mt_raw = fmaxf(xs[r], xs[128 + r]);
       const bool live = mt_raw != -INFINITY;  // this row has a valid key in the tile
-      const float rowmax = live ? ex2_ftz(mt - m_new) : 0.0f;
-      l *= alpha;
-      m = m_new;
-      // Rescale factors of this tile: the contribution is sigma * PV(t).  An
-      // NVFP4 tile whose row factor is negligible (< 2^-60 of the running
-      // maximum) or not a normal float contributes nothing: its P is zero.
-      const float sigma_raw = (live && rowmax >= 8.6736174e-19f) ? rowmax * (1.0f / 2688.0f) : 0.0f;
-      float sigma = 1.0f;
-      if (!f16) {
-        sigma = sigma_raw * gv;
-        if (!(sigma >= 1.17549435e-38f)) sigma = 0.0f;
+      const float mt = mt_raw * cs;
+      if (hf == 0) {
+        sta[(t & 3) * 128 + r] = mt;
+        mbar_arrive(&bars[B_STA + (t & 3)]);
       }
-      if (f == 0) {
-        stat[st * 256 + r] = alpha;
-        stat[st * 256 + 128 + r] = sigma;
-        mbar_arrive(&bars[B_ST + st]);
-      }
+      float ls = 0.0f;
       if (!f16) {
         // Two-level quantisation of P.  Relative to the tile max the scaled
-        // probabilities are Phat = 2688 * 2^(s - mt) (row factor
-        // sigma = rowmax / 2688); block b gets the UE4M3 scale
-        // S_b = ue4m3(max Phat / 6) and the codes E2M1(Phat / S_b), computed
-        // as one exponential t = 2^(s + log2(2688) - mt - log2 S_b).
-        // l gets sum_b S_b * sum(t) * rowmax / 2688.
-        const bool contrib = sigma > 0.0f;
-        float ls = 0.0f;
+        // probabilities are Phat = 2688 * 2^(s - mt); block b gets the UE4M3
+        // scale S_b = ue4m3(max Phat / 6) and the codes E2M1(Phat / S_b),
+        // computed as one exponential t = 2^(s + log2(2688) - mt - log2 S_b).
+        // The row sum of the tile, relative to 2688 * 2^-mt, is
+        // sum_b S_b * sum(t).
+        if (!warp_wait(&bars[B_TURN + g], u & 1, s_abort)) { ok = false; break; }
         uint32_t sfw = 0;
-        uint32_t cw[2 * NB];
+        uint32_t cw[NCH][4];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
-          const uint32_t S = contrib ? ue4m3(448.0f * e) : 0u;
-          const float dec = ue4m3_decode_fast(S);
-          const float c = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
-          float bs0 = 0.0f, bs1 = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            float x0, x1;
-            fma2(x0, x1, a[16 * b + i], a[16 * b + i + 1], cs, cs, c, c);
-            a[16 * b + i] = ex2_ftz(x0);  // masked (-inf) -> 0
-            a[16 * b + i + 1] = ex2_ftz(x1);
-            add2(bs0, bs1, bs0, bs1, a[16 * b + i], a[16 * b + i + 1]);
+        for (int c = 0; c < NCH; ++c) {
+          float a[32];
+          tmem_ld32(s_base + 32 * c, a);
+          tmem_ld_wait();
+          if (c == NCH - 1) {
+            tc_fence_before();
+            mbar_arrive(&bars[B_SE + g]);  // S buffer free for QK^T of tile t+2
           }
-          ls = fmaf(bs0 + bs1, dec, ls);
-          sfw |= S << (8 * b);
-          cw[2 * b] = e2m1x8(a + 16 * b);
-          cw[2 * b + 1] = e2m1x8(a + 16 * b + 8);
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = i + 32 * c <= lim ? a[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int b2 = 0; b2 < 2; ++b2) {
+            const int b = 2 * c + b2;
+            const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
+            const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
+            const float dec = ue4m3_decode_fast(S);
+            const float cc = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
+            float bs0 = 0.0f, bs1 = 0.0f;
+            float* x = a + 16 * b2;
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              float x0, x1;
+              fma2(x0, x1, x[i], x[i + 1], cs, cs, cc, cc);
+              x[i] = ex2_ftz(x0);  // masked (-inf) -> 0
+              x[i + 1] = ex2_ftz(x1);
+              add2(bs0, bs1, bs0, bs1, x[i], x[i + 1]);
+            }
+            ls = fmaf(bs0 + bs1, dec, ls);
+            sfw |= S << (8 * b);
+            cw[c][2 * b2] = e2m1x8(x);
+            cw[c][2 * b2 + 1] = e2m1x8(x + 8);
+          }
         }
-        l = fmaf(ls, sigma_raw, l);
-        // P slot st was last read by PV(t-2)
-        if (t >= 2 && !warp_wait(&bars[B_OD + st], ((t >> 1) - 1) & 1, s_abort)) {
-          ok = false;
-          break;
-        }
-        uint8_t* p4 = sm + L::OFF4_P + st * L::PT4A;
-        if constexpr (NB == 2) {
-          *reinterpret_cast<uint4*>(p4 + p4_codes_off) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          *reinterpret_cast<uint16_t*>(p4 + p4_sf_off) = (uint16_t)sfw;
+        if (t + 1 < n) mbar_arrive(&bars[B_TURN + (1 - g)]);
+        // P slot g was last read by PV(t-2)
+        if (u >= 1 && !warp_wait(&bars[B_OD + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          *reinterpret_cast<uint4*>(p4 + p4_codes_off[c]) =
+              make_uint4(cw[c][0], cw[c][1], cw[c][2], cw[c][3]);
+        if constexpr (NCH == 2) {
+          *reinterpret_cast<uint32_t*>(p4 + p4_sf_off) = sfw;
         } else {
-          *reinterpret_cast<uint2*>(p4 + p4_codes_off) = make_uint2(cw[0], cw[1]);
-          p4[p4_sf_off] = (uint8_t)sfw;
+          *reinterpret_cast<uint16_t*>(p4 + p4_sf_off) = (uint16_t)sfw;
         }
       } else {
+        // FP16 tile: P = 2^(s - m_new) against the running max through t
+        float m_prev = -INFINITY;
+        if (t > 0) {
+          if (!warp_wait(&bars[B_MR + ((t - 1) & 3)], ((t - 1) >> 2) & 1, s_abort)) {
+            ok = false;
+            break;
+          }
+          m_prev = mr[((t - 1) & 3) * 128 + r];
+        }
+        const float m_new = fmaxf(m_prev, mt);
         const float negm = m_new == -INFINITY ? 0.0f : -m_new;
+        if (!warp_wait(&bars[B_TURN + g], u & 1, s_abort)) { ok = false; break; }
+        uint32_t w[NCH][16];
         float l0 = 0.0f, l1 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < SC; i += 2) {
-          float x0, x1;
-          fma2(x0, x1, a[i], a[i + 1], cs, cs, negm, negm);
-          a[i] = ex2_ftz(x0);  // exp2(-inf) = 0 for masked columns
-          a[i + 1] = ex2_ftz(x1);
-          add2(l0, l1, l0, l1, a[i], a[i + 1]);
+        for (int c = 0; c < NCH; ++c) {
+          float a[32];
+          tmem_ld32(s_base + 32 * c, a);
+          tmem_ld_wait();
+          if (c == NCH - 1) {
+            tc_fence_before();
+            mbar_arrive(&bars[B_SE + g]);
+          }
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = i + 32 * c <= lim ? a[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            fma2(x0, x1, a[i], a[i + 1], cs, cs, negm, negm);
+            a[i] = ex2_ftz(x0);  // exp2(-inf) = 0 for masked columns
+            a[i + 1] = ex2_ftz(x1);
+            add2(l0, l1, l0, l1, a[i], a[i + 1]);
+            w[c][i >> 1] = pack2<DT>(a[i], a[i + 1]);
+          }
         }
-        l += l0 + l1;
-        // FP16 tiles share one P buffer: the previous FP16 PV must be done.
-        // (The first FP16 tile needs no wait: its scores only arrive after
-        // the last NVFP4 PV has retired.)
+        ls = l0 + l1;
+        if (t + 1 < n) mbar_arrive(&bars[B_TURN + (1 - g)]);
+        // one P buffer: the previous FP16 PV must be done.  (The first FP16
+        // tile needs no wait: its scores only arrive after the last NVFP4
+        // PV has retired.)
         if (t > n4 && !warp_wait(&bars[B_OD + ((t - 1) & 1)], ((t - 1) >> 1) & 1, s_abort)) {
           ok = false;
           break;
         }
-        uint8_t* p16 = sm + L::OFF16_P;
 #pragma unroll
-        for (int q8 = 0; q8 < SC / 8; ++q8) {
-          uint32_t w4[4];
+        for (int c = 0; c < NCH; ++c) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) w4[e] = pack2<DT>(a[8 * q8 + 2 * e], a[8 * q8 + 2 * e + 1]);
-          const uint32_t key0 = f * SC + 8 * q8;
-          *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
-                                    swz_offset(r, (key0 % 64) * 2, 128)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const uint32_t key0 = hf * SC + 32 * c + 8 * q8;
+            *reinterpret_cast<uint4*>(p16 + (key0 / 64) * 128 * 128 +
+                                      swz_offset(r, (key0 % 64) * 2, 128)) =
+                make_uint4(w[c][4 * q8], w[c][4 * q8 + 1], w[c][4 * q8 + 2], w[c][4 * q8 + 3]);
+          }
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars[B_PF + st]);
+      mbar_arrive(&bars[B_PF + g]);
+      stb[(2 * (t & 3) + hf) * 128 + r] = ls;
+      mbar_arrive(&bars[B_STB + (t & 3)]);
     }
-    // publish this quarter's row sum (and the row max) for the output warps
-    float* fin = reinterpret_cast<float*>(sm + L::OFF_FIN);
-    fin[f * 128 + r] = l;
-    if (f == 0) fin[512 + r] = m;
-    mbar_arrive(&bars[B_LF]);
   }
   tc_fence_before();
   __syncthreads();
