@@ -216,6 +216,10 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// Materialises a value at this point of the program (an empty asm that
+// reads and rewrites it), so that it is not computed later.
+__device__ __forceinline__ void pin64(uint64_t& x) { asm volatile("" : "+l"(x)); }
+
 // Waits with every lane of the warp; the result is uniform across the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -401,6 +405,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           const int st = t & 1;
           const bool f16 = t >= n4;
           uint64_t* full = f16 ? &bars[B_KVF16 + sl] : &bars[B_KVF4 + sl];
+          // operands first, then the waits
+          constexpr int NI = D / 16;  // FP16 MMAs per tile (NVFP4: D / 64)
+          uint64_t da[NI], db[NI], cpk[D / 64];
+          const uint32_t dS = tmem + L::T_S + st * BLK;
+          const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
+          if (!f16) {
+            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
+#pragma unroll
+            for (int s = 0; s < D / 64; ++s) {
+              cpk[s] = d_sf + ((L::OFF4_STG + BLK * (D / 2) + 512 * s) >> 4) + so;
+              da[s] = d_q4 + 2 * s;
+              db[s] = d_k4 + so + 2 * s;
+              pin64(cpk[s]);
+              pin64(db[s]);
+            }
+          } else {
+            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
+#pragma unroll
+            for (int s = 0; s < NI; ++s) {
+              da[s] = d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4);
+              db[s] = d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4);
+              pin64(db[s]);
+            }
+          }
           if (!mbar_wait(full, par, s_abort)) { ok = false; break; }
           if (!f16 && !q4_ready) {
             if (!mbar_wait(&bars[B_Q4], 0, s_abort)) { ok = false; break; }
@@ -421,24 +449,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             break;
           }
           tc_fence_after();
-          const uint32_t dS = tmem + L::T_S + st * BLK;
           if (!f16) {
-            const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
-            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
+#pragma unroll
+            for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
 #pragma unroll
             for (int s = 0; s < D / 64; ++s)
-              tc_cp_32x128b_x4(ksf + 4 * s,
-                               d_sf + ((L::OFF4_STG + BLK * (D / 2) + 512 * s) >> 4) + so);
-#pragma unroll
-            for (int s = 0; s < D / 64; ++s)
-              mma_nvf4(dS, d_q4 + 2 * s, d_k4 + so + 2 * s, id_qk4, tmem + L::T_QSF + 4 * s,
-                       ksf + 4 * s, s > 0);
+              mma_nvf4(dS, da[s], db[s], id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s, s > 0);
           } else {
-            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
 #pragma unroll
-            for (int s = 0; s < D / 16; ++s)
-              mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
-                      d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
+            for (int s = 0; s < NI; ++s) mma_f16(dS, da[s], db[s], id_qk16, s > 0);
           }
           tc_commit(&bars[B_SF + st]);
           advance(t);
@@ -448,37 +467,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         const uint64_t d_v4 = make_sdesc(base + L::OFF4_STG + L::V4_OFF, 16, 8 * (BLK / 2), swz_b);
         const uint64_t d_p16 = make_sdesc(base + L::OFF16_P, 16, 1024, SW_128B);
         const uint64_t d_v16 = make_sdesc(base + L::OFF16_STG + L::V16_OFF, 16, 1024, SW_128B);
+        const uint32_t dO = tmem + L::T_O;
         for (int t = 0; t < n && ok; ++t) {
           const int st = t & 1;
           const bool f16 = t >= n4;
           uint64_t* empty = f16 ? &bars[B_KVE16 + sl] : &bars[B_KVE4 + sl];
-          if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
-          if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
-          tc_fence_after();
-          const uint32_t dO = tmem + L::T_O;
+          // Operands first: the waits below end when the correction step
+          // finishes, and from there on only the tensor instructions remain.
+          constexpr int NI = BLK / 16;  // FP16 MMAs per tile (NVFP4: BLK / 64)
+          uint64_t da[NI], db[NI], cpp[BLK / 64], cpv[BLK / 64];
+          uint32_t psf = 0, vsf = 0;
           if (!f16) {
             const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
             const uint32_t po = (uint32_t)st * (L::PT4A >> 4);
-            const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
-            const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
+            psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
+            vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
 #pragma unroll
             for (int s = 0; s < BLK / 64; ++s) {
-              tc_cp_32x128b_x4(psf + 4 * s,
-                               d_sf + ((L::OFF4_P + 128 * (BLK / 2) + 512 * s) >> 4) + po);
-              tc_cp_32x128b_x4(vsf + 4 * s, d_sf + ((L::OFF4_STG + L::V4_OFF + D * (BLK / 2) +
-                                                     512 * s) >> 4) + so);
+              cpp[s] = d_sf + ((L::OFF4_P + 128 * (BLK / 2) + 512 * s) >> 4) + po;
+              cpv[s] = d_sf + ((L::OFF4_STG + L::V4_OFF + D * (BLK / 2) + 512 * s) >> 4) + so;
+              da[s] = d_p4 + po + 2 * s;
+              db[s] = d_v4 + so + 2 * s;
+              pin64(cpp[s]);
+              pin64(cpv[s]);
+              pin64(da[s]);
+              pin64(db[s]);
             }
-#pragma unroll
-            for (int s = 0; s < BLK / 64; ++s)
-              mma_nvf4(dO, d_p4 + po + 2 * s, d_v4 + so + 2 * s, id_pv4, psf + 4 * s,
-                       vsf + 4 * s, t > 0 || s > 0);
           } else {
             const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
 #pragma unroll
-            for (int s = 0; s < BLK / 16; ++s)
-              mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
-                      d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
-                      t > 0 || s > 0);
+            for (int s = 0; s < NI; ++s) {
+              da[s] = d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4);
+              db[s] = d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4);
+              pin64(da[s]);
+              pin64(db[s]);
+            }
+          }
+          if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
+          tc_fence_after();
+          if (!f16) {
+#pragma unroll
+            for (int s = 0; s < BLK / 64; ++s) {
+              tc_cp_32x128b_x4(psf + 4 * s, cpp[s]);
+              tc_cp_32x128b_x4(vsf + 4 * s, cpv[s]);
+            }
+#pragma unroll
+            for (int s = 0; s < BLK / 64; ++s)
+              mma_nvf4(dO, da[s], db[s], id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
+          } else {
+#pragma unroll
+            for (int s = 0; s < NI; ++s) mma_f16(dO, da[s], db[s], id_pv16, t > 0 || s > 0);
           }
           tc_commit(&bars[B_OD + st]);
           tc_commit(empty);
@@ -725,8 +764,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         // computed as one exponential t = 2^(s + log2(2688) - mt - log2 S_b).
         // The row sum of the tile, relative to 2688 * 2^-mt, is
         // sum_b S_b * sum(t).
-        if (!warp_wait(&bars[B_TURN + g], u & 1, s_abort)) { ok = false; break; }
+        // block scales first, outside the turn
+        float dec[2 * NCH], cc[2 * NCH];
         uint32_t sfw = 0;
+#pragma unroll
+        for (int b = 0; b < 2 * NCH; ++b) {
+          const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
+          const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
+          dec[b] = ue4m3_decode_fast(S);
+          cc[b] = S ? 11.392317422778760f - mt - lg2_ftz(dec[b]) : -INFINITY;  // log2(2688)
+          sfw |= S << (8 * b);
+        }
+        if (!warp_wait(&bars[B_TURN + g], u & 1, s_abort)) { ok = false; break; }
         uint32_t cw[NCH][4];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
@@ -744,22 +793,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
             const int b = 2 * c + b2;
-            const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
-            const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
-            const float dec = ue4m3_decode_fast(S);
-            const float cc = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
             float bs0 = 0.0f, bs1 = 0.0f;
             float* x = a + 16 * b2;
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
               float x0, x1;
-              fma2(x0, x1, x[i], x[i + 1], cs, cs, cc, cc);
+              fma2(x0, x1, x[i], x[i + 1], cs, cs, cc[b], cc[b]);
               x[i] = ex2_ftz(x0);  // masked (-inf) -> 0
               x[i + 1] = ex2_ftz(x1);
               add2(bs0, bs1, bs0, bs1, x[i], x[i + 1]);
             }
-            ls = fmaf(bs0 + bs1, dec, ls);
-            sfw |= S << (8 * b);
+            ls = fmaf(bs0 + bs1, dec[b], ls);
             cw[c][2 * b2] = e2m1x8(x);
             cw[c][2 * b2 + 1] = e2m1x8(x + 8);
           }

@@ -43,17 +43,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       : "memory");
 }
 
-// Waits (suspended, not spinning) until the phase with the given parity has
-// completed or about `hint_ns` have passed; returns whether it completed.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
-                                              uint32_t hint_ns = 20000u) {
+// One potentially blocking test of the phase with the given parity (the
+// hardware may suspend the thread for a short, implementation-defined time);
+// returns whether the phase has completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
