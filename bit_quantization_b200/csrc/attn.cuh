@@ -793,17 +793,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
             const int b = 2 * c + b2;
-            float bs0 = 0.0f, bs1 = 0.0f;
             float* x = a + 16 * b2;
+            // all sixteen exponent arguments, then all sixteen exponentials
+            // (independent, so they stream through the MUFU back to back),
+            // then a sum tree
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              float x0, x1;
-              fma2(x0, x1, x[i], x[i + 1], cs, cs, cc[b], cc[b]);
-              x[i] = ex2_ftz(x0);  // masked (-inf) -> 0
-              x[i + 1] = ex2_ftz(x1);
-              add2(bs0, bs1, bs0, bs1, x[i], x[i + 1]);
-            }
-            ls = fmaf(bs0 + bs1, dec[b], ls);
+            for (int i = 0; i < 16; i += 2)
+              fma2(x[i], x[i + 1], x[i], x[i + 1], cs, cs, cc[b], cc[b]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = ex2_ftz(x[i]);  // masked (-inf) -> 0
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2)
+              add2(y[i], y[i + 1], x[2 * i], x[2 * i + 1], x[2 * i + 2], x[2 * i + 3]);
+            add2(y[0], y[1], y[0], y[1], y[2], y[3]);
+            add2(y[4], y[5], y[4], y[5], y[6], y[7]);
+            add2(y[0], y[1], y[0], y[1], y[4], y[5]);
+            ls = fmaf(y[0] + y[1], dec[b], ls);
             cw[c][2 * b2] = e2m1x8(x);
             cw[c][2 * b2 + 1] = e2m1x8(x + 8);
           }
@@ -849,13 +855,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             for (int i = 0; i < 32; ++i) a[i] = i + 32 * c <= lim ? a[i] : -INFINITY;
           }
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float x0, x1;
-            fma2(x0, x1, a[i], a[i + 1], cs, cs, negm, negm);
-            a[i] = ex2_ftz(x0);  // exp2(-inf) = 0 for masked columns
-            a[i + 1] = ex2_ftz(x1);
-            add2(l0, l1, l0, l1, a[i], a[i + 1]);
-            w[c][i >> 1] = pack2<DT>(a[i], a[i + 1]);
+          for (int h16 = 0; h16 < 32; h16 += 16) {
+            float* x = a + h16;
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) fma2(x[i], x[i + 1], x[i], x[i + 1], cs, cs, negm, negm);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = ex2_ftz(x[i]);  // exp2(-inf) = 0 when masked
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              add2(l0, l1, l0, l1, x[i], x[i + 1]);
+              w[c][(h16 + i) >> 1] = pack2<DT>(x[i], x[i + 1]);
+            }
           }
         }
         ls = l0 + l1;
