@@ -54,8 +54,8 @@ def load_peaks():
 # DRAM traffic of one attention launch measured by ncu (read + write bytes)
 # for the attention source with this hash; reported only while the source is
 # unchanged since the capture.
-ATTN_TRAFFIC = {"src_sha16": "4ccd12ef983ce6ad", "workload": "b2h32n8192d128_bf16_noncausal_top10",
-                "bytes": 519915008}
+ATTN_TRAFFIC = {"src_sha16": "069ff32032be3341", "workload": "b2h32n8192d128_bf16_noncausal_top10",
+                "bytes": 517434112}
 
 
 def attn_traffic(w):
@@ -67,8 +67,11 @@ def attn_traffic(w):
     return None
 
 
-XU_OPS_PER_CLK_PER_SM = 16   # MUFU / conversion pipe lanes per SM (4 per sub-partition)
-XU_OPS_PER_ELEMENT = 1.5     # one exp2 and half of a two-value 4/16-bit convert per score
+XU_OPS_PER_CLK_PER_SM = 16   # MUFU lanes per SM (4 per sub-partition)
+# MUFU operations per score element: one exp2, plus one exp2 and one log2 per
+# 16-key block for the block scale (the E2M1 / 16-bit converts do not use
+# this pipe: an instruction-class count of each convert shows none there)
+XU_OPS_PER_ELEMENT = 1.125
 
 
 def pair_flops(mask, w, lengths):
@@ -419,7 +422,7 @@ def main():
     alu_achieved = elems / (k_ms * 1e-3) / 1e9
     alu_roofline = {"bound": "alu", "kernel": "attn_fwd_kernel", "achieved": alu_achieved,
                     "peak": alu_peak, "unit": "Gelem/s", "frac": alu_achieved / alu_peak,
-                    "peak_note": (f"{XU_OPS_PER_CLK_PER_SM} MUFU/convert lanes per SM x {n_sm} SMs x "
+                    "peak_note": (f"{XU_OPS_PER_CLK_PER_SM} MUFU lanes per SM x {n_sm} SMs x "
                                   f"{sm_mhz:.0f} MHz / {XU_OPS_PER_ELEMENT} ops per score element"),
                     "tflops_equivalent_peak": alu_peak * 1e9 * 4 * w.d / 1e12}
 
