@@ -39,7 +39,7 @@ WORKLOADS = {
 
 METRIC = "NVFP4 attention fwd TFLOPS (whole step: quantise + select + attention)"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 11  # 3 absmax, 2 Q/K images, 1 V image, 2 block means, 1 scores, 1 top-k, 1 attention
+KERNELS_PER_STEP = 9  # 3 absmax, 2 Q/K images (with the block means), 1 V image, 1 scores, 1 top-k, 1 attention
 
 
 def load_peaks():

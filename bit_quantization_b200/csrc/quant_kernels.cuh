@@ -159,110 +159,126 @@ __host__ __device__ constexpr uint32_t f16_tile_bytes(uint32_t rows, uint32_t kd
   return rows * kdim * 2;
 }
 
-// Q or K ([total, nh, d] 16-bit) -> per (sequence, head, tile) images:
+// Q or K ([total, nh, d] 16-bit) -> per (sequence, head, tile) images, one
+// CTA per tile of tile_rows rows:
 //   img4:  codes [tile_rows, d/2] swizzled (pitch d/2), then scale factors;
 //   img16: the unrotated 16-bit rows, d/64 regions of [tile_rows, 128 B]
 //          with 128-byte swizzle.
-// Rows past the sequence end are written as zeros.  G = d/16.
+// Rows past the sequence end are written as zeros.  When means is given, the
+// CTA also writes the fp64 means [nseq, nh, nB, d] of the blk-row blocks in
+// its tile (ThriftAttention, Metodologia step 1): the unrotated values summed
+// in row order from the block start, divided by the row count.  The tile is
+// read from HBM once, with 16-byte loads, into shared memory.  G = d/16.
 template <int DT, int G, bool HAD, bool SS>
-__global__ void __launch_bounds__(256) qk_image_kernel(
-    const uint16_t* __restrict__ x, SeqInfo seqs, int nseq, int nh, int tile_rows, int ntiles,
-    const uint32_t* amax_in, uint8_t* __restrict__ img4, uint8_t* __restrict__ img16) {
+__global__ void __launch_bounds__(256) qk_tile_kernel(
+    const uint16_t* __restrict__ x, SeqInfo seqs, int nh, int tile_rows, int ntiles, int blk,
+    int nB, const uint32_t* amax_in, uint8_t* __restrict__ img4, uint8_t* __restrict__ img16,
+    double* __restrict__ means) {
   constexpr int D = G * 16;
+  extern __shared__ uint4 tsm[];  // [tile_rows][D] 16-bit values
+  const int tile = blockIdx.x, head = blockIdx.y, seq = blockIdx.z;
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int t0 = tile * tile_rows;
+  if (t0 >= len) return;
+  for (int i = threadIdx.x; i < tile_rows * (D / 8); i += blockDim.x) {
+    const int r = i / (D / 8), c8 = i % (D / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t0 + r < len)
+      v = __ldg(reinterpret_cast<const uint4*>(x + ((start + t0 + r) * nh + head) * D) + c8);
+    tsm[i] = v;
+  }
+  __syncthreads();
   const float g = tensor_scale_from_amax(*amax_in);
   const uint32_t t4 = fp4_tile_bytes(tile_rows, D), t16 = f16_tile_bytes(tile_rows, D);
-  const int64_t rows_per_seq = (int64_t)ntiles * tile_rows * nh;
-  const int64_t n_blocks = (int64_t)nseq * rows_per_seq * G;
-  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-       base < n_blocks; base += nthreads) {
-    const int64_t b = base + (threadIdx.x & 31);
-    const int kb = (int)(b % G);
-    const int64_t rho = b / G;
-    const int head = (int)(rho % nh);
-    const int64_t tp = (rho / nh) % ((int64_t)ntiles * tile_rows);
-    const int seq = (int)(rho / rows_per_seq);
-    bool write = false, real = false;
-    int64_t start = 0;
-    int len = 0;
-    if (b < n_blocks) {
-      seqs.get(seq, start, len);
-      write = tp < ceil_div(len, tile_rows) * tile_rows;
-      real = tp < len;
-    }
+  const int64_t tidx = ((int64_t)seq * nh + head) * ntiles + tile;
+  uint8_t* t4p = img4 + tidx * t4;
+  uint8_t* t16p = img16 + tidx * t16;
+  uint8_t* sf = t4p + (uint32_t)tile_rows * (D / 2);
+  // one 16-element block per thread and step; the G blocks of a row sit in
+  // G consecutive lanes (the Hadamard exchanges between them)
+  for (int i = threadIdx.x; i < tile_rows * G; i += blockDim.x) {
+    const int r = i / G, kb = i % G;
+    const uint4 raw0 = tsm[(r * D + kb * 16) / 8], raw1 = tsm[(r * D + kb * 16) / 8 + 1];
     float v[16];
-    uint4 raw0 = make_uint4(0, 0, 0, 0), raw1 = raw0;
-    if (real) {
-      const uint16_t* p = x + ((start + tp) * nh + head) * D + kb * 16;
-      raw0 = __ldg(reinterpret_cast<const uint4*>(p));
-      raw1 = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-    }
-    {
-      const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
+    const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = h2f<DT>((uint16_t)(w[i] & 0xFFFF));
-        v[2 * i + 1] = h2f<DT>((uint16_t)(w[i] >> 16));
-      }
+    for (int e = 0; e < 8; ++e) {
+      v[2 * e] = h2f<DT>((uint16_t)(w[e] & 0xFFFF));
+      v[2 * e + 1] = h2f<DT>((uint16_t)(w[e] >> 16));
     }
     if constexpr (HAD) fwht_rows16<G>(v);
-    if (write) {
-      const int tile = (int)(tp / tile_rows), r = (int)(tp % tile_rows);
-      const int64_t tidx = ((int64_t)seq * nh + head) * ntiles + tile;
-      uint8_t* t4p = img4 + tidx * t4;
-      uint32_t lo, hi;
-      const uint32_t S = quant_block16(v, g, SS, lo, hi);
-      *reinterpret_cast<uint2*>(t4p + swz_offset(r, kb * 8, D / 2)) = make_uint2(lo, hi);
-      uint8_t* sf = t4p + (uint32_t)tile_rows * (D / 2);
-      sf[sf_offset(r, kb)] = (uint8_t)S;
-      if (tile_rows == 64) sf[sf_offset(r + 64, kb)] = 0;
-      uint8_t* t16p = img16 + tidx * t16;
-      const uint32_t e0 = kb * 16;
-      uint8_t* reg = t16p + (e0 / 64) * ((uint32_t)tile_rows * 128);
-      *reinterpret_cast<uint4*>(reg + swz_offset(r, (e0 % 64) * 2, 128)) = raw0;
-      *reinterpret_cast<uint4*>(reg + swz_offset(r, (e0 % 64) * 2 + 16, 128)) = raw1;
+    uint32_t lo, hi;
+    const uint32_t S = quant_block16(v, g, SS, lo, hi);
+    *reinterpret_cast<uint2*>(t4p + swz_offset(r, kb * 8, D / 2)) = make_uint2(lo, hi);
+    sf[sf_offset(r, kb)] = (uint8_t)S;
+    if (tile_rows == 64) sf[sf_offset(r + 64, kb)] = 0;
+    const uint32_t e0 = kb * 16;
+    uint8_t* reg = t16p + (e0 / 64) * ((uint32_t)tile_rows * 128);
+    *reinterpret_cast<uint4*>(reg + swz_offset(r, (e0 % 64) * 2, 128)) = raw0;
+    *reinterpret_cast<uint4*>(reg + swz_offset(r, (e0 % 64) * 2 + 16, 128)) = raw1;
+  }
+  if (means != nullptr) {
+    const uint16_t* tv = reinterpret_cast<const uint16_t*>(tsm);
+    const int nbt = tile_rows / blk;  // selection blocks in this tile
+    for (int e = threadIdx.x; e < nbt * D; e += blockDim.x) {
+      const int c = e % D, bi = e / D;
+      const int b0 = t0 + bi * blk;
+      if (b0 >= len) continue;
+      const int b1 = min(len, b0 + blk);
+      double sum = 0.0;
+      for (int t = b0; t < b1; ++t) sum = __dadd_rn(sum, (double)h2f<DT>(tv[(t - t0) * D + c]));
+      means[(((int64_t)seq * nh + head) * nB + tile * nbt + bi) * D + c] =
+          __ddiv_rn(sum, (double)(b1 - b0));
     }
   }
 }
 
 // V ([total, Hkv, d] 16-bit) -> per (sequence, kv head, key tile) images with
-// 16-blocks along tokens: img4 codes [d, blk/2] swizzled (pitch blk/2) then
-// scale factors (rows = channels); img16 = V^T tile [d, blk] in blk/64
-// regions of [d, 128 B] with 128-byte swizzle.  Keys past the sequence end
-// are zeros.  One thread per (sequence, head, 16-token block, channel).
+// 16-blocks along tokens, one CTA per key tile: img4 codes [d, blk/2]
+// swizzled (pitch blk/2) then scale factors (rows = channels); img16 = V^T
+// tile [d, blk] in blk/64 regions of [d, 128 B] with 128-byte swizzle.  Keys
+// past the sequence end are zeros.  The tile is read once, with 16-byte
+// loads, into shared memory; each thread then takes one (channel, 16-key)
+// column block from there.
 template <int DT, bool SS>
-__global__ void __launch_bounds__(256) v_image_kernel(
-    const uint16_t* __restrict__ v, SeqInfo seqs, int nseq, int Hkv, int d, int blk, int ntiles,
+__global__ void __launch_bounds__(256) v_tile_kernel(
+    const uint16_t* __restrict__ v, SeqInfo seqs, int Hkv, int d, int blk, int ntiles,
     const uint32_t* amax_in, uint8_t* __restrict__ img4, uint8_t* __restrict__ img16) {
+  extern __shared__ uint4 tsm[];  // [blk][d] 16-bit values
+  const int j = blockIdx.x, hk = blockIdx.y, seq = blockIdx.z;
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int t0 = j * blk;
+  if (t0 >= len) return;
+  for (int i = threadIdx.x; i < blk * (d / 8); i += blockDim.x) {
+    const int r = i / (d / 8), c8 = i % (d / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (t0 + r < len)
+      val = __ldg(reinterpret_cast<const uint4*>(v + ((start + t0 + r) * Hkv + hk) * d) + c8);
+    tsm[i] = val;
+  }
+  __syncthreads();
   const float g = tensor_scale_from_amax(*amax_in);
   const uint32_t t4 = fp4_tile_bytes(d, blk), t16 = f16_tile_bytes(d, blk);
-  const int ntb = ntiles * blk / 16;
-  const int64_t n = (int64_t)nseq * Hkv * ntb * d;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int c = (int)(idx % d);
-    const int tb = (int)((idx / d) % ntb);
-    const int hk = (int)((idx / ((int64_t)d * ntb)) % Hkv);
-    const int seq = (int)(idx / ((int64_t)d * ntb * Hkv));
-    int64_t start;
-    int len;
-    seqs.get(seq, start, len);
-    const int t0 = tb * 16;
-    if (t0 >= ceil_div(len, blk) * blk) continue;
+  const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
+  uint8_t* t4p = img4 + tidx * t4;
+  uint8_t* sf = t4p + (uint32_t)d * (blk / 2);
+  const uint16_t* tv = reinterpret_cast<const uint16_t*>(tsm);
+  for (int i = threadIdx.x; i < d * (blk / 16); i += blockDim.x) {
+    const int c = i % d, kb = (i / d) * 16;
     float val[16];
     uint16_t raw[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      raw[e] = (t0 + e < len) ? __ldg(v + ((start + t0 + e) * Hkv + hk) * d + c) : (uint16_t)0;
+      raw[e] = tv[(kb + e) * d + c];
       val[e] = h2f<DT>(raw[e]);
     }
-    const int j = t0 / blk, kb = t0 % blk;
-    const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
-    uint8_t* t4p = img4 + tidx * t4;
     uint32_t lo, hi;
     const uint32_t S = quant_block16(val, g, SS, lo, hi);
     *reinterpret_cast<uint2*>(t4p + swz_offset(c, kb / 2, blk / 2)) = make_uint2(lo, hi);
-    uint8_t* sf = t4p + (uint32_t)d * (blk / 2);
     sf[sf_offset(c, kb / 16)] = (uint8_t)S;
     if (d == 64) sf[sf_offset(c + 64, kb / 16)] = 0;
     uint8_t* reg = img16 + tidx * t16 + (kb / 64) * ((uint32_t)d * 128);

@@ -134,24 +134,34 @@ AttnWs carve_attn(void* ws, int nseq, int maxlen, int H, int Hkv, int d, int blk
   return w;
 }
 
+// Image (and block-mean) launches: one CTA per (tile, head, sequence), the
+// tile staged in shared memory.
+struct TileArgs {
+  const void* x;
+  SeqInfo si;
+  int nseq, nh, rows, ntiles, blk, nB;
+  const uint32_t* amax;
+  uint8_t *i4, *i16;
+  double* means;
+};
+
 template <int DT, int G, bool HAD, bool SS>
-void launch_qk_image(const void* x, SeqInfo si, int nseq, int nh, int rows, int ntiles,
-                     const uint32_t* amax, uint8_t* i4, uint8_t* i16, cudaStream_t st) {
-  const int64_t nb = (int64_t)nseq * ntiles * rows * nh * G;
-  qk_image_kernel<DT, G, HAD, SS><<<grid_for(nb), kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(x), si, nseq, nh, rows, ntiles, amax, i4, i16);
+void launch_qk_tile(const TileArgs& a, cudaStream_t st) {
+  dim3 grid(a.ntiles, a.nh, a.nseq);
+  const size_t smem = (size_t)a.rows * G * 16 * 2;
+  qk_tile_kernel<DT, G, HAD, SS><<<grid, kThreads, smem, st>>>(
+      static_cast<const uint16_t*>(a.x), a.si, a.nh, a.rows, a.ntiles, a.blk, a.nB, a.amax, a.i4,
+      a.i16, a.means);
 }
 
 template <int DT, int G>
-void dispatch_qk_image(bool had, bool ss, const void* x, SeqInfo si, int nseq, int nh, int rows,
-                       int ntiles, const uint32_t* amax, uint8_t* i4, uint8_t* i16,
-                       cudaStream_t st) {
+void dispatch_qk_tile(bool had, bool ss, const TileArgs& a, cudaStream_t st) {
   if (had) {
-    if (ss) launch_qk_image<DT, G, true, true>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
-    else launch_qk_image<DT, G, true, false>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+    if (ss) launch_qk_tile<DT, G, true, true>(a, st);
+    else launch_qk_tile<DT, G, true, false>(a, st);
   } else {
-    if (ss) launch_qk_image<DT, G, false, true>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
-    else launch_qk_image<DT, G, false, false>(x, si, nseq, nh, rows, ntiles, amax, i4, i16, st);
+    if (ss) launch_qk_tile<DT, G, false, true>(a, st);
+    else launch_qk_tile<DT, G, false, false>(a, st);
   }
 }
 
@@ -204,27 +214,27 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   launch_amax<DT>(q, total * H * d / 16, had ? G : 0, w.amax + 0, st);
   launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, w.amax + 1, st);
   launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
+  // Q and K images, with the block means of the selection on the way
+  const TileArgs aq{q, si, nseq, H, 128, nTq, blk, nB, w.amax + 0, w.q4, w.q16, w.means_q};
+  const TileArgs ak{k, si, nseq, Hkv, blk, nB, blk, nB, w.amax + 1, w.k4, w.k16, w.means_k};
   if (G == 8) {
-    dispatch_qk_image<DT, 8>(had, ss, q, si, nseq, H, 128, nTq, w.amax + 0, w.q4, w.q16, st);
-    dispatch_qk_image<DT, 8>(had, ss, k, si, nseq, Hkv, blk, nB, w.amax + 1, w.k4, w.k16, st);
+    dispatch_qk_tile<DT, 8>(had, ss, aq, st);
+    dispatch_qk_tile<DT, 8>(had, ss, ak, st);
   } else {
-    dispatch_qk_image<DT, 4>(had, ss, q, si, nseq, H, 128, nTq, w.amax + 0, w.q4, w.q16, st);
-    dispatch_qk_image<DT, 4>(had, ss, k, si, nseq, Hkv, blk, nB, w.amax + 1, w.k4, w.k16, st);
+    dispatch_qk_tile<DT, 4>(had, ss, aq, st);
+    dispatch_qk_tile<DT, 4>(had, ss, ak, st);
   }
   {
-    const int64_t nv = (int64_t)nseq * Hkv * (nB * blk / 16) * d;
+    dim3 grid(nB, Hkv, nseq);
+    const size_t smem = (size_t)blk * d * 2;
     if (ss)
-      v_image_kernel<DT, true><<<grid_for(nv), kThreads, 0, st>>>(
-          static_cast<const uint16_t*>(v), si, nseq, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
+      v_tile_kernel<DT, true><<<grid, kThreads, smem, st>>>(
+          static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
     else
-      v_image_kernel<DT, false><<<grid_for(nv), kThreads, 0, st>>>(
-          static_cast<const uint16_t*>(v), si, nseq, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
+      v_tile_kernel<DT, false><<<grid, kThreads, smem, st>>>(
+          static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
   }
   // selection
-  block_means_kernel<DT><<<grid_for((int64_t)nseq * H * nB * d), kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(q), si, nseq, H, d, blk, nB, w.means_q);
-  block_means_kernel<DT><<<grid_for((int64_t)nseq * Hkv * nB * d), kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(k), si, nseq, Hkv, d, blk, nB, w.means_k);
   pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, w.scores);
   topk_kernel<<<nseq * H, kTopkThreads, 0, st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
@@ -484,6 +494,15 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrif
                         use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
   return attn_impl<0>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
                       use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
+}
+
+size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hkv, int d,
+                                         int blk) {
+  if (nseq <= 0 || max_seqlen <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || (d != 64 && d != 128) ||
+      (blk != 64 && blk != 128))
+    return 0;
+  const AttnWs w = carve_attn(nullptr, nseq, max_seqlen, H, Hkv, d, blk);
+  return (size_t)reinterpret_cast<uintptr_t>(w.mask);
 }
 
 size_t thrift_attn_varlen_workspace_size(int nseq, int64_t total, int max_seqlen, int H,

@@ -27,6 +27,7 @@ EXPORTS = (
     "nvfp4_quantize", "nvfp4_quantize_colblocks", "block_mean_topk_workspace_size",
     "block_mean_topk", "block_mean_topk_noalloc", "thrift_attn_workspace_size", "thrift_attn_fwd",
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
+    "thrift_attn_workspace_mask_offset",
     "thrift_kernel_timer_enable", "thrift_kernel_timer_read",
 )
 
@@ -67,6 +68,8 @@ def lib():
                                       i32, P, P, P, sz, P]
         L.thrift_attn_varlen_workspace_size.restype = sz
         L.thrift_attn_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+        L.thrift_attn_workspace_mask_offset.restype = sz
+        L.thrift_attn_workspace_mask_offset.argtypes = [i32, i32, i32, i32, i32, i32]
         L.thrift_attn_fwd_varlen.restype = i32
         L.thrift_attn_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
                                              i32, f32, i32, i32, P, P, P, sz, P]
@@ -243,6 +246,12 @@ def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesear
                                  int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                  _stream(q)), "thrift_attn_fwd")
     return out, lse
+
+
+def thrift_attn_workspace_mask_offset(nseq, max_seqlen, H, Hkv, d, blk) -> int:
+    """Byte offset of the selection mask [nseq, H, nB, nB] inside an attention
+    workspace (valid once the call that used the workspace has completed)."""
+    return int(lib().thrift_attn_workspace_mask_offset(nseq, max_seqlen, H, Hkv, d, blk))
 
 
 def thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk) -> int:

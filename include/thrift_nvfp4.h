@@ -167,6 +167,17 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
                                      int use_hadamard, void* out, float* lse, void* workspace,
                                      size_t ws_bytes, void* stream);
 
+/* Byte offset, inside the workspace of thrift_attn_fwd (nseq = B,
+ * max_seqlen = N) or thrift_attn_fwd_varlen, of the block-pair selection the
+ * call leaves there once it has completed on its stream: uint8
+ * [nseq, H, nB, nB], nB = ceil(max_seqlen / blk), 1 = the pair ran on the
+ * FP16 path ("ThriftAttention", Metodologia step 1); for a sequence with
+ * fewer blocks only its leading nb x nb pairs are meaningful.  Returns 0 for
+ * arguments the attention calls reject (0 is never a valid offset).  For
+ * inspection and tests; the workspace stays owned by the caller. */
+size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hkv, int d,
+                                         int blk);
+
 /* ----------------------------------------------------- kernel timing --
  * Measurement aid (not part of the method).  While enabled, every
  * thrift_attn_fwd / thrift_attn_fwd_varlen call records a CUDA event pair on
