@@ -49,75 +49,81 @@ __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __rest
   }
 }
 
-// scores [nseq, H, nB, nB] fp64 (valid i, j < nb of the sequence only).
-// One CTA per (sequence, head, 16 query blocks); the key means pass through
-// shared memory transposed, 8 channels at a time, and every score keeps its
-// sequential fma order over the channels.  nB <= 512.
-constexpr int kScoreRows = 16, kScoreChunk = 8;
+// scores [nseq, H, nB, nB] fp64 (valid i, j < nb of the sequence only;
+// causal: j <= i).  One CTA per (sequence, head, 64 x 64 tile of pairs);
+// each thread holds a 4 x 4 block of scores in registers, every score a
+// sequential fma over the channels in order.  The means pass through shared
+// memory 32 channels at a time, channel-major.  nB <= 512.
+constexpr int kPairTile = 64, kPairChunk = 32;
 
 __global__ void __launch_bounds__(256) pair_scores_kernel(const double* __restrict__ qm,
                                                           const double* __restrict__ km,
                                                           SeqInfo seqs, int nseq, int H,
                                                           int Hkv, int d, int blk, int nB,
+                                                          int causal,
                                                           double* __restrict__ scores) {
-  extern __shared__ double ssm[];
-  double* qs = ssm;                                   // [kScoreRows][kScoreChunk]
-  double* ks = ssm + kScoreRows * kScoreChunk;        // [kScoreChunk][nB]
-  const int groups = (nB + kScoreRows - 1) / kScoreRows;
-  const int ig = blockIdx.x % groups;
-  const int h = (blockIdx.x / groups) % H;
-  const int seq = blockIdx.x / (groups * H);
+  __shared__ double qs[kPairChunk][kPairTile + 1];
+  __shared__ double ks[kPairChunk][kPairTile + 1];
+  const int T = (nB + kPairTile - 1) / kPairTile;
+  const int tile = blockIdx.x % (T * T);
+  const int h = (blockIdx.x / (T * T)) % H;
+  const int seq = blockIdx.x / (T * T * H);
+  const int i0 = (tile / T) * kPairTile, j0 = (tile % T) * kPairTile;
   int64_t start;
   int len;
   seqs.get(seq, start, len);
   const int nb = (int)ceil_div(len, blk);
-  const int i0 = ig * kScoreRows;
-  if (i0 >= nb) return;
+  if (i0 >= nb || j0 >= nb || (causal && j0 > i0 + kPairTile - 1)) return;
   const int hk = h / (H / Hkv);
-  const double* qrow = qm + (((int64_t)seq * H + h) * nB + i0) * d;
+  const double* qrow = qm + ((int64_t)seq * H + h) * nB * d;
   const double* krow = km + ((int64_t)seq * Hkv + hk) * nB * d;
-  double acc[kScoreRows][2];
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  double acc[4][4];
 #pragma unroll
-  for (int a = 0; a < kScoreRows; ++a) acc[a][0] = acc[a][1] = 0.0;
-  const int j0 = threadIdx.x, j1 = threadIdx.x + 256;
-  for (int c0 = 0; c0 < d; c0 += kScoreChunk) {
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int c0 = 0; c0 < d; c0 += kPairChunk) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kScoreRows * kScoreChunk; e += blockDim.x) {
-      const int a = e / kScoreChunk, cc = e % kScoreChunk;
-      qs[e] = (i0 + a < nb) ? __ldg(qrow + (int64_t)a * d + c0 + cc) : 0.0;
-    }
-    for (int e = threadIdx.x; e < nb * kScoreChunk; e += blockDim.x) {
-      const int j = e / kScoreChunk, cc = e % kScoreChunk;
-      ks[cc * nB + j] = __ldg(krow + (int64_t)j * d + c0 + cc);
+    // rows i0.. / j0.. of the means, 32 channels each, transposed into
+    // shared memory (consecutive threads read consecutive channels)
+    for (int e = threadIdx.x; e < kPairTile * kPairChunk; e += blockDim.x) {
+      const int r = e / kPairChunk, c = e % kPairChunk;
+      qs[c][r] = (i0 + r < nb) ? __ldg(qrow + (int64_t)(i0 + r) * d + c0 + c) : 0.0;
+      ks[c][r] = (j0 + r < nb) ? __ldg(krow + (int64_t)(j0 + r) * d + c0 + c) : 0.0;
     }
     __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kPairChunk; ++c) {
+      double qv[4], kv[4];
 #pragma unroll
-    for (int cc = 0; cc < kScoreChunk; ++cc) {
-      const double k0 = j0 < nb ? ks[cc * nB + j0] : 0.0;
-      const double k1 = j1 < nb ? ks[cc * nB + j1] : 0.0;
+      for (int a = 0; a < 4; ++a) qv[a] = qs[c][4 * ti + a];
 #pragma unroll
-      for (int a = 0; a < kScoreRows; ++a) {
-        const double q = qs[a * kScoreChunk + cc];
-        acc[a][0] = __fma_rn(q, k0, acc[a][0]);
-        acc[a][1] = __fma_rn(q, k1, acc[a][1]);
-      }
+      for (int b = 0; b < 4; ++b) kv[b] = ks[c][tj + 16 * b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[a], kv[b], acc[a][b]);
     }
   }
-  double* out = scores + (((int64_t)seq * H + h) * nB + i0) * nB;
+  double* out = scores + ((int64_t)seq * H + h) * nB * nB;
 #pragma unroll
-  for (int a = 0; a < kScoreRows; ++a) {
-    if (i0 + a >= nb) break;
-    if (j0 < nb) out[(int64_t)a * nB + j0] = acc[a][0];
-    if (j1 < nb) out[(int64_t)a * nB + j1] = acc[a][1];
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + 4 * ti + a;
+    if (i >= nb) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + tj + 16 * b;
+      if (j < nb) out[(int64_t)i * nB + j] = acc[a][b];
+    }
   }
 }
 
-inline size_t pair_scores_smem(int nB) {
-  return sizeof(double) * (kScoreRows * kScoreChunk + kScoreChunk * (size_t)nB);
-}
+inline size_t pair_scores_smem(int) { return 0; }
 
 inline int pair_scores_grid(int nseq, int H, int nB) {
-  return nseq * H * ((nB + kScoreRows - 1) / kScoreRows);
+  const int T = (nB + kPairTile - 1) / kPairTile;
+  return nseq * H * T * T;
 }
 
 // Order-preserving map of a double to an unsigned 64-bit key.
@@ -164,9 +170,50 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   return r;
 }
 
+// Largest digit whose count, accumulated from digit 255 downwards, reaches
+// rem; returns it and the count strictly above it.  Warp 0 only: lane l takes
+// digits 255 - 8l ... 248 - 8l.
+__device__ __forceinline__ int select_digit(const int* hist, int64_t rem, int64_t* above) {
+  const int lane = threadIdx.x & 31;
+  int c[8];
+  int sum = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    c[e] = hist[255 - 8 * lane - e];
+    sum += c[e];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, (int64_t)incl >= rem);
+  const int src = hit ? __ffs(hit) - 1 : 31;
+  int64_t cum = (int64_t)(incl - sum);  // count above this lane's digits
+  int sel = 0;
+  if (lane == src) {
+    sel = 255 - 8 * lane - 7;
+    for (int e = 0; e < 8; ++e) {
+      if (cum + c[e] >= rem) {
+        sel = 255 - 8 * lane - e;
+        break;
+      }
+      cum += c[e];
+    }
+  }
+  sel = __shfl_sync(0xffffffffu, sel, src);
+  cum = __shfl_sync(0xffffffffu, cum, src);
+  *above = cum;
+  return sel;
+}
+
 // One CTA per (sequence, head): exact top-k by an 8-pass radix select on the
 // 64-bit keys, then ties at the threshold taken in ascending linear index.
-// mask [nseq, H, nB, nB] uint8 (1 = FP16 pair); every entry is written.
+// mask [nseq, H, nB, nB] uint8 (1 = FP16 pair); every entry is written.  The
+// keys are read once into shared memory when they fit (kTopkCache).
+constexpr int kTopkCache = 4096;  // 32 KB of keys: within the default shared-memory limit
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __restrict__ scores,
                                                             SeqInfo seqs, int H, int blk, int nB,
                                                             int causal, float frac,
@@ -176,6 +223,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
   __shared__ int s_total;
   __shared__ uint64_t s_prefix;
   __shared__ int64_t s_remaining;
+  extern __shared__ uint64_t kcache[];
   const int seq = blockIdx.x / H, h = blockIdx.x % H;
   int64_t start;
   int len;
@@ -195,45 +243,46 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
       mk[lin] = (k != 0 && valid(lin)) ? 1 : 0;
     return;
   }
+  const bool cached = npairs <= kTopkCache;
+  if (cached) {
+    for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x)
+      kcache[lin] = valid(lin) ? order_key(sc[lin]) : 0ull;
+  }
+  auto key_of = [&](int64_t lin) { return cached ? kcache[lin] : order_key(sc[lin]); };
   uint64_t prefix = 0, pmask = 0;
-  if (threadIdx.x == 0) s_remaining = k;
+  int64_t rem = k;
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x) {
       if (!valid(lin)) continue;
-      const uint64_t key = order_key(sc[lin]);
+      const uint64_t key = key_of(lin);
       if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int64_t rem = s_remaining, cum = 0;
-      int sel = 0;
-      for (int dgt = 255; dgt >= 0; --dgt) {
-        if (cum + hist[dgt] >= rem) {
-          sel = dgt;
-          break;
-        }
-        cum += hist[dgt];
+    if (threadIdx.x < 32) {
+      int64_t above;
+      const int sel = select_digit(hist, rem, &above);
+      if (threadIdx.x == 0) {
+        s_remaining = rem - above;
+        s_prefix = prefix | ((uint64_t)sel << shift);
       }
-      s_remaining = rem - cum;
-      s_prefix = prefix | ((uint64_t)sel << shift);
     }
     __syncthreads();
     prefix = s_prefix;
+    rem = s_remaining;
     pmask |= (uint64_t)255 << shift;
-    __syncthreads();
   }
   const uint64_t T = prefix;
-  const int64_t take_eq = s_remaining;
+  const int64_t take_eq = rem;
   int64_t taken = 0;
   for (int64_t base = 0; base < npairs; base += blockDim.x) {
     const int64_t lin = base + threadIdx.x;
     uint64_t key = 0;
     bool ok = false;
     if (lin < npairs && valid(lin)) {
-      key = order_key(sc[lin]);
+      key = key_of(lin);
       ok = true;
     }
     const int eq = (ok && key == T) ? 1 : 0;
@@ -242,6 +291,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
     taken += s_total;
     __syncthreads();
   }
+}
+
+inline size_t topk_smem(int nB) {
+  const int64_t np = (int64_t)nB * nB;
+  return np <= kTopkCache ? (size_t)np * 8 : 0;
 }
 
 }  // namespace thrift

@@ -236,8 +236,8 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   }
   // selection
   pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
-      w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, w.scores);
-  topk_kernel<<<nseq * H, kTopkThreads, 0, st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
+      w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, causal, w.scores);
+  topk_kernel<<<nseq * H, kTopkThreads, topk_smem(nB), st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
   if (launch_status() != THRIFT_OK) return THRIFT_ERR_CUDA;
 
   AttnParams p;
@@ -451,8 +451,8 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
     block_means_kernel<0><<<grid_for((int64_t)B * Hkv * nB * d), kThreads, 0, st>>>(kp, si, B, Hkv, d, blk, nB, mk);
   }
   pair_scores_kernel<<<pair_scores_grid(B, H, nB), kThreads, pair_scores_smem(nB), st>>>(
-      mq, mk, si, B, H, Hkv, d, blk, nB, sc);
-  topk_kernel<<<B * H, kTopkThreads, 0, st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
+      mq, mk, si, B, H, Hkv, d, blk, nB, causal, sc);
+  topk_kernel<<<B * H, kTopkThreads, topk_smem(nB), st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
   return launch_status();
 }
 
