@@ -289,6 +289,30 @@ def quantizer_only(args):
     return 0
 
 
+def nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4, steps=20):
+    """The attention kernel with no FP16 pairs (topk_frac = 0): every score
+    on the NVFP4 path, against the FP4 tensor peak alone."""
+    def step():
+        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=0.0,
+                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
+                            out=out, lse=lse, workspace=ws)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ops.kernel_timer_enable(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    ops.kernel_timer_enable(False)
+    kms, n = ops.kernel_timer_read()
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out (topk_frac = 0)")
+    k_ms = kms / max(n, 1)
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    return {"topk_frac": 0.0, "kernel": "attn_fwd_kernel", "kernel_ms": k_ms,
+            "achieved": achieved, "peak": p4, "unit": "TFLOP/s", "frac": achieved / p4}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -413,8 +437,8 @@ def main():
                               f"the FP16 share ({100 * f16 / flops:.1f}% of flops)"),
                 "kernel_ms": k_ms, "fp4_flops": f4, "fp16_flops": f16}
 
-    # ALU roofline of the same kernel: every score element needs one exp2 and
-    # half a packed conversion on the MUFU/convert pipe (16 lanes per SM).
+    # ALU roofline of the same kernel: the MUFU operations per score element
+    # (XU_OPS_PER_ELEMENT) against the MUFU lanes of the SMs.
     sm_mhz = clocks.get("sm_mhz") or 1965.0
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     elems = flops / (4.0 * w.d)
@@ -434,6 +458,8 @@ def main():
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
+    if rank == 0 and world == 1:
+        line["nvfp4_only"] = nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4)
     if rank == 0 and world == 1 and not args.no_quantizer:
         line["quantizer"] = quantizer_line(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -66,14 +66,6 @@ __device__ __forceinline__ float ue4m3_decode(uint32_t b) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// E2M1 code (4 bits) -> fp32 (exact).
-__device__ __forceinline__ float e2m1_decode(uint32_t c) {
-  const uint32_t m = c & 7u;
-  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 as bit patterns
-  const float mag = (m < 2) ? 0.5f * (float)m : __uint_as_float(((m >> 1) + 126u) << 23 | ((m & 1u) << 22));
-  return (c & 8u) ? -mag : mag;
-}
-
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace thrift

@@ -28,6 +28,20 @@ __device__ __forceinline__ float tensor_scale_from_amax(uint32_t amax_bits) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, kTensorScaleDiv);
 }
 
+// E2M1 round trip of two values: q = decode(E2M1(t)) (round to nearest
+// even, saturating), through the hardware converts to E2M1 and back to f16
+// (every E2M1 value, signed zeros included, is exact in f16 and in fp32).
+__device__ __forceinline__ void e2m1x2_roundtrip(float t0, float t1, float& q0, float& q1) {
+  asm("{\n\t.reg .b8 c;\n\t.reg .b32 h;\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %3, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h, c;\n\t"
+      "mov.b32 {lo, hi}, h;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t"
+      "cvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(q0), "=f"(q1)
+      : "f"(t0), "f"(t1));
+}
+
 // Block error of candidate byte S (see header comment).
 __device__ __forceinline__ double block_err(const float (&x)[16], float g, uint32_t S) {
   const float sv = ue4m3_decode(S);
@@ -36,8 +50,8 @@ __device__ __forceinline__ double block_err(const float (&x)[16], float g, uint3
 #pragma unroll
   for (int e = 0; e < 16; e += 2) {
     const float t0 = __fmul_rn(x[e], r), t1 = __fmul_rn(x[e + 1], r);
-    const uint32_t c = e2m1x2(t0, t1);
-    const float q0 = e2m1_decode(c & 15u), q1 = e2m1_decode(c >> 4);
+    float q0, q1;
+    e2m1x2_roundtrip(t0, t1, q0, q1);
     const float d0 = __fsub_rn(t0, q0), d1 = __fsub_rn(t1, q1);
     acc = __fmaf_rn(d0, d0, acc);
     acc = __fmaf_rn(d1, d1, acc);
@@ -59,18 +73,20 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], float g,
     return 0;
   }
   if (ss) {
-    const int order[9] = {0, -2, -1, 1, 2, 3, 4, 5, 6};
     double best = 0.0;
     int best_f = 0;
     bool have = false;
-#pragma unroll
+    // candidates in the order 0, -2, -1, 1, 2, ..., 6 (a rolled loop keeps
+    // the code small enough for the instruction cache)
+#pragma unroll 1
     for (int oi = 0; oi < 9; ++oi) {
-      const int b = (int)S + order[oi];
+      const int f = oi == 0 ? 0 : (oi <= 2 ? oi - 3 : oi - 2);
+      const int b = (int)S + f;
       if (b >= 1 && b <= 126) {
         const double err = block_err(x, g, (uint32_t)b);
         if (!have || err < best) {
           best = err;
-          best_f = order[oi];
+          best_f = f;
           have = true;
         }
       }

@@ -55,29 +55,45 @@ int sm_count() {
   return n;
 }
 
-// Grid for the streaming kernels: enough CTAs for kKPT blocks per thread,
-// at most four resident CTAs per SM (grid-stride beyond that).
-int stream_grid(int64_t n_blocks) {
+// Grid for the streaming (grid-stride) kernels: enough CTAs for kKPT blocks
+// per thread, capped at one full wave (resident CTAs per SM x SMs) so that no
+// partial second wave trails the launch.
+template <class Kernel>
+int stream_grid(Kernel kernel, int64_t n_blocks) {
+  static int resident = 0;  // per kernel instantiation
+  if (resident == 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
+            cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    resident = per_sm * sm_count();
+  }
   int64_t g = ceil_div(n_blocks, (int64_t)kThreads * kKPT);
   if (g < 1) g = 1;
-  if (g > 4LL * sm_count()) g = 4LL * sm_count();
+  if (g > resident) g = resident;
   return (int)g;
+}
+
+template <int DT, int G>
+void launch_amax_t(const uint16_t* xp, int64_t n_blocks, uint32_t* out, cudaStream_t st) {
+  amax_kernel<DT, G><<<stream_grid(amax_kernel<DT, G>, n_blocks), kThreads, 0, st>>>(
+      xp, n_blocks, out);
 }
 
 template <int DT>
 void launch_amax(const void* x, int64_t n_blocks, int G, uint32_t* out, cudaStream_t st) {
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  const int grid = stream_grid(n_blocks);
-  if (G == 8) amax_kernel<DT, 8><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
-  else if (G == 4) amax_kernel<DT, 4><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
-  else amax_kernel<DT, 0><<<grid, kThreads, 0, st>>>(xp, n_blocks, out);
+  if (G == 8) launch_amax_t<DT, 8>(xp, n_blocks, out, st);
+  else if (G == 4) launch_amax_t<DT, 4>(xp, n_blocks, out, st);
+  else launch_amax_t<DT, 0>(xp, n_blocks, out, st);
 }
 
 template <int DT, int G, bool SS>
 void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, int given,
                          uint8_t* codes, uint8_t* scales, cudaStream_t st) {
-  quant_rows_kernel<DT, G, SS><<<stream_grid(nb), kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(x), nb, amax, ts, given, codes, scales);
+  quant_rows_kernel<DT, G, SS><<<stream_grid(quant_rows_kernel<DT, G, SS>, nb), kThreads, 0,
+                                 st>>>(static_cast<const uint16_t*>(x), nb, amax, ts, given,
+                                       codes, scales);
 }
 
 template <int DT>
@@ -397,21 +413,26 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
     else launch_amax<0>(x, rows * cols / 16, 0, amax, st);
   }
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  const int grid = stream_grid((rows / 16) * cols / kKPT + 1);
+  // one thread per (row block, column): kKPT * threads items per CTA
+  const int64_t items = (rows / 16) * cols * kKPT;
   if (dt == THRIFT_BF16) {
     if (use_scalesearch)
-      quant_cols_kernel<1, true><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                                           tensor_scale_given, codes, scales);
+      quant_cols_kernel<1, true><<<stream_grid(quant_cols_kernel<1, true>, items), kThreads, 0,
+                                   st>>>(xp, rows, cols, amax, tensor_scale, tensor_scale_given,
+                                         codes, scales);
     else
-      quant_cols_kernel<1, false><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                                            tensor_scale_given, codes, scales);
+      quant_cols_kernel<1, false><<<stream_grid(quant_cols_kernel<1, false>, items), kThreads,
+                                    0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                             tensor_scale_given, codes, scales);
   } else {
     if (use_scalesearch)
-      quant_cols_kernel<0, true><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                                           tensor_scale_given, codes, scales);
+      quant_cols_kernel<0, true><<<stream_grid(quant_cols_kernel<0, true>, items), kThreads, 0,
+                                   st>>>(xp, rows, cols, amax, tensor_scale, tensor_scale_given,
+                                         codes, scales);
     else
-      quant_cols_kernel<0, false><<<grid, kThreads, 0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                                            tensor_scale_given, codes, scales);
+      quant_cols_kernel<0, false><<<stream_grid(quant_cols_kernel<0, false>, items), kThreads,
+                                    0, st>>>(xp, rows, cols, amax, tensor_scale,
+                                             tensor_scale_given, codes, scales);
   }
   return launch_status();
 }
