@@ -124,6 +124,98 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   }
 }
 
+// ------------------------------------------- one-pass row quantiser --
+// The whole tensor in one launch when it fits in shared memory: every CTA
+// (one per SM, co-resident by a cooperative launch) stages its contiguous
+// chunk of blocks once, takes the chunk absmax, publishes it, waits for all
+// CTAs (bounded wait), reduces the published maxima to the tensor absmax and
+// quantises its chunk from shared memory.  Same arithmetic as the two-pass
+// path.  sync[0] counts arrivals and sync[1] departures; the last CTA to
+// leave zeroes both, so the workspace is left as it was found (zeros).
+// partial[] has one float per CTA.  chunk is a multiple of 32 blocks (rows
+// stay whole for the Hadamard lanes).
+constexpr int kOnePassThreads = 512;
+
+template <int DT, int G, bool SS>
+__global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
+    const uint16_t* __restrict__ x, int64_t n_blocks, int64_t chunk, unsigned* sync,
+    float* partial, float* tensor_scale, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  extern __shared__ uint4 cs[];  // chunk blocks x 32 bytes
+  __shared__ float red[32];
+  __shared__ int s_ok;
+  const int64_t b0 = (int64_t)blockIdx.x * chunk;
+  float a = 0.0f;
+  for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
+    uint4 r0, r1;
+    load_raw(x, b0 + i, n_blocks, r0, r1);
+    cs[2 * i] = r0;
+    cs[2 * i + 1] = r1;
+    float v[16];
+    unpack16<DT>(r0, r1, v);
+    if constexpr (G > 0) fwht_rows16<G>(v);
+    a = fmaxf(a, block_absmax(v));
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float c = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c = fmaxf(c, red[w]);
+    partial[blockIdx.x] = c;
+    __threadfence();
+    atomicAdd(&sync[0], 1u);
+    // wait for every CTA's maximum (bounded)
+    int ok = 1;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      unsigned arrived;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(sync) : "memory");
+      if (arrived >= gridDim.x) break;
+      if (globaltimer_ns() - t0 > 2000000000ull) {
+        set_device_status(THRIFT_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  // tensor absmax from the published maxima (each thread folds a few)
+  float m = 0.0f;
+  for (int c = threadIdx.x; c < (int)gridDim.x; c += blockDim.x) m = fmaxf(m, __ldcg(partial + c));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = 0.0f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
+  const float g = tensor_scale_from_amax(__float_as_uint(amax));
+  if (threadIdx.x == 0) {
+    if (blockIdx.x == 0) *tensor_scale = g;
+    // the last CTA out leaves the counters at zero for the next call
+    if (atomicAdd(&sync[1], 1u) == gridDim.x - 1) {
+      sync[0] = 0u;
+      sync[1] = 0u;
+    }
+  }
+  for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
+    const int64_t b = b0 + i;
+    float v[16];
+    unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
+    if constexpr (G > 0) fwht_rows16<G>(v);
+    if (b < n_blocks) {
+      uint32_t lo, hi;
+      const uint32_t S = quant_block16(v, g, SS, lo, hi);
+      *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
+      scales[b] = (uint8_t)S;
+    }
+  }
+}
+
 // ---------------------------------------------- column-blocked quantiser --
 // x [rows, cols]; 16-blocks along rows.  codes [cols, rows/2], scales
 // [cols, rows/16].  One thread per (row block, column); columns fastest.

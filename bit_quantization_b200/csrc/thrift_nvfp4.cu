@@ -1,6 +1,7 @@
 // C-ABI entry points of libthrift_nvfp4.so: argument checks, workspace
 // carving and kernel launches.  Declarations and the contract of every entry
 // point are in include/thrift_nvfp4.h.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -96,17 +97,67 @@ void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, i
                                        codes, scales);
 }
 
+// Quantiser workspace: words 0 and 1 are the arrival and departure counts
+// of the one-pass kernel (zero between calls), word 2 the absmax of the
+// two-pass path, and from byte 256 one float per CTA of the one-pass kernel.
+constexpr size_t kQuantWsBytes = 4096;
+constexpr int kQuantMaxCtas = (int)((kQuantWsBytes - 256) / 4);
+constexpr int64_t kOnePassSmemMax = 200 * 1024;
+
+// The one-pass quantiser when the tensor fits in the SMs' shared memory;
+// returns false (nothing launched) when it does not or the cooperative
+// launch is refused.
+template <int DT, int G, bool SS>
+bool try_quant_onepass(const void* x, int64_t nb, uint32_t* ws, float* ts, uint8_t* codes,
+                       uint8_t* scales, cudaStream_t st) {
+  auto kern = quant_onepass_kernel<DT, G, SS>;
+  int grid = (int)std::min<int64_t>(std::min(sm_count(), kQuantMaxCtas), ceil_div(nb, 32));
+  const int64_t chunk = ceil_div(ceil_div(nb, (int64_t)grid), 32) * 32;
+  const int64_t smem = chunk * 32;
+  if (smem > kOnePassSmemMax) return false;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kOnePassSmemMax) != cudaSuccess)
+      return false;
+    attr = true;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kOnePassThreads,
+                                                    (size_t)smem) != cudaSuccess ||
+      per_sm < 1)
+    return false;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kOnePassThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  float* partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
+  return cudaLaunchKernelEx(&cfg, kern, xp, nb, chunk, ws, partial, ts, codes, scales) ==
+         cudaSuccess;
+}
+
 template <int DT>
-thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_t* sync,
+thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_t* ws,
                               float* ts, int given, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st) {
+  uint32_t* amax = ws + 2;
 #define THRIFT_QUANT_CASE(GG, SSV)                                                        \
   if (G == GG && ss == SSV) {                                                              \
     if (!given) {                                                                          \
-      if (cudaMemsetAsync(sync, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;          \
-      launch_amax<DT>(x, nb, GG, sync, st);                                                \
+      if (try_quant_onepass<DT, GG, SSV>(x, nb, ws, ts, codes, scales, st))                \
+        return launch_status();                                                            \
+      (void)cudaGetLastError();                                                            \
+      if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;          \
+      launch_amax<DT>(x, nb, GG, amax, st);                                                \
     }                                                                                      \
-    launch_quant_rows_t<DT, GG, SSV>(x, nb, sync, ts, given, codes, scales, st);           \
+    launch_quant_rows_t<DT, GG, SSV>(x, nb, amax, ts, given, codes, scales, st);           \
     return launch_status();                                                                \
   }
   THRIFT_QUANT_CASE(0, false)
@@ -365,7 +416,7 @@ thrift_status thrift_kernel_timer_read(double* total_ms, int* launches) {
   return THRIFT_OK;
 }
 
-size_t nvfp4_quantize_workspace_size(void) { return 256; }
+size_t nvfp4_quantize_workspace_size(void) { return kQuantWsBytes; }
 
 thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64_t cols,
                              int use_scalesearch, int use_hadamard, int tensor_scale_given,
@@ -381,13 +432,13 @@ thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64
       (reinterpret_cast<uintptr_t>(codes) & 7))
     return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* sync = static_cast<uint32_t*>(workspace);
+  uint32_t* wsw = static_cast<uint32_t*>(workspace);
   const int64_t nb = rows * cols / 16;
   const int G = use_hadamard ? (int)(cols / 16) : 0;
   if (dt == THRIFT_BF16)
-    return launch_quantize<1>(x, nb, G, use_scalesearch != 0, sync, tensor_scale,
+    return launch_quantize<1>(x, nb, G, use_scalesearch != 0, wsw, tensor_scale,
                               tensor_scale_given, codes, scales, st);
-  return launch_quantize<0>(x, nb, G, use_scalesearch != 0, sync, tensor_scale,
+  return launch_quantize<0>(x, nb, G, use_scalesearch != 0, wsw, tensor_scale,
                             tensor_scale_given, codes, scales, st);
 }
 
@@ -406,7 +457,7 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
     return THRIFT_ERR_ARG;
   if ((rows * cols) % 16) return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  uint32_t* amax = static_cast<uint32_t*>(workspace) + 2;  // word 2: see launch_quantize
   if (!tensor_scale_given) {
     if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
     if (dt == THRIFT_BF16) launch_amax<1>(x, rows * cols / 16, 0, amax, st);

@@ -132,19 +132,24 @@ def kernel_timer_read():
 
 
 class Workspace:
-    """Grow-only device scratch buffer reused across calls on one device."""
+    """Grow-only device scratch buffer reused across calls on one device
+    (zero-filled when allocated if ``zeroed``)."""
 
-    def __init__(self):
+    def __init__(self, zeroed=False):
         self.buf: Optional[torch.Tensor] = None
+        self.zeroed = zeroed
 
     def get(self, nbytes: int, device) -> torch.Tensor:
         nbytes = max(int(nbytes), 256)
         if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
-            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            alloc = torch.zeros if self.zeroed else torch.empty
+            self.buf = alloc(nbytes, dtype=torch.uint8, device=device)
         return self.buf
 
 
 _ws = Workspace()
+# the quantiser's own workspace: zero-filled, and left zero-filled by each call
+_qws = Workspace(zeroed=True)
 
 
 # ------------------------------------------------------------------ quantiser
@@ -162,8 +167,8 @@ def nvfp4_quantize(x: torch.Tensor, use_scalesearch=False, use_hadamard=False,
         scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
     given = tensor_scale is not None
     ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
-    ws = workspace if workspace is not None else _ws.get(lib().nvfp4_quantize_workspace_size(),
-                                                         x.device)
+    ws = workspace if workspace is not None else _qws.get(lib().nvfp4_quantize_workspace_size(),
+                                                          x.device)
     _check(lib().nvfp4_quantize(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
                                 int(use_hadamard), int(given), _ptr(codes), _ptr(scales),
                                 _ptr(ts), _ptr(ws), ws.numel(), _stream(x)), "nvfp4_quantize")
@@ -179,7 +184,7 @@ def nvfp4_quantize_colblocks(x: torch.Tensor, use_scalesearch=False,
     scales = torch.empty((cols, rows // 16), dtype=torch.uint8, device=x.device)
     given = tensor_scale is not None
     ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
-    ws = _ws.get(lib().nvfp4_quantize_workspace_size(), x.device)
+    ws = _qws.get(lib().nvfp4_quantize_workspace_size(), x.device)
     _check(lib().nvfp4_quantize_colblocks(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
                                           int(given), _ptr(codes), _ptr(scales), _ptr(ts),
                                           _ptr(ws), ws.numel(), _stream(x)),

@@ -81,7 +81,18 @@ thrift_status thrift_device_status(int reset);
  *   use_hadamard: rotate every row by the unnormalised Sylvester-Hadamard
  *     transform first (cols must be 64 or 128).
  * Requirements: rows >= 0, cols % 16 == 0, cols <= 4096.
- * Workspace: nvfp4_quantize_workspace_size() bytes.
+ * Workspace: nvfp4_quantize_workspace_size() bytes, 16-byte aligned, zero-
+ *   filled before its first use; every call that completes without a device
+ *   timeout leaves it zero-filled again (the one-pass kernel keeps two
+ *   counters there), so one buffer serves any number of calls issued in
+ *   stream order.  After THRIFT_ERR_TIMEOUT from thrift_device_status, zero
+ *   it again before reuse.  nvfp4_quantize_colblocks takes the same
+ *   workspace.
+ * Execution: when the tensor scale is computed and the tensor fits in the
+ *   SMs' shared memory (about 200 KB per SM), one cooperative launch stages
+ *   it once, exchanges the per-CTA maxima with a bounded grid-wide wait and
+ *   quantises from shared memory; otherwise an absmax pass and a quantise
+ *   pass.  Both give the same bytes.
  */
 size_t nvfp4_quantize_workspace_size(void);
 thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64_t cols,

@@ -57,14 +57,15 @@ def test_bad_arguments_rejected_before_launch(L):
     P = C.c_void_p
     dummy = P(4096)
     ws = P(8192)
+    qws = L.nvfp4_quantize_workspace_size()
     # cols not a multiple of 16
-    assert L.nvfp4_quantize(dummy, 0, 4, 24, 0, 0, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_ARG
+    assert L.nvfp4_quantize(dummy, 0, 4, 24, 0, 0, 0, dummy, dummy, dummy, ws, qws, None) == ops.ERR_ARG
     # Hadamard on an unsupported width
-    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 1, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_UNSUPPORTED
+    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 1, 0, dummy, dummy, dummy, ws, qws, None) == ops.ERR_UNSUPPORTED
     # workspace too small
-    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, 8, None) == ops.ERR_ARG
+    assert L.nvfp4_quantize(dummy, 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, qws - 1, None) == ops.ERR_ARG
     # misaligned input
-    assert L.nvfp4_quantize(P(4098), 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, 256, None) == ops.ERR_ARG
+    assert L.nvfp4_quantize(P(4098), 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, qws, None) == ops.ERR_ARG
     # attention: unsupported head dim, bad GQA ratio, bad fraction, null pointer
     assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 96, 128, 0, C.c_float(0.1), 0, 0,
                              dummy, dummy, ws, 1 << 40, None) == ops.ERR_UNSUPPORTED

@@ -109,3 +109,21 @@ def test_two_pass_path_large_tensor(orc):
     # kernel, so the absmax pass and the quantise pass run separately.
     x = synth.randn16((1 << 21, 16), torch.bfloat16, seed=21)
     _check_rows(orc, x, False, False)
+
+
+@pytest.mark.parametrize("had", [False, True])
+def test_one_pass_leaves_workspace_zeroed(orc, had):
+    # The one-pass kernel (tensor staged in shared memory, one grid-wide max
+    # exchange) keeps its counters in the caller's workspace and must leave
+    # them at zero; repeated calls on one workspace stay bit-exact.
+    ws = torch.zeros(ops.lib().nvfp4_quantize_workspace_size(), dtype=torch.uint8, device="cuda")
+    for seed in (11, 12, 13):
+        x = synth.randn16((4096, 128), torch.bfloat16, seed=seed, scale=2.0)
+        codes, scales, ts = ops.nvfp4_quantize(x.cuda(), use_hadamard=had, workspace=ws)
+        torch.cuda.synchronize()
+        assert ops.device_status() == ops.OK
+        assert not ws[:8].any().item()
+        c0, s0, g0, _ = orc.nvfp4_quantize(synth.as_u16(x), _dt(x.dtype), use_had=had)
+        assert ts.item() == np.float32(g0)
+        assert np.array_equal(scales.cpu().numpy(), s0)
+        assert np.array_equal(codes.cpu().numpy(), c0)
