@@ -239,15 +239,17 @@ def quantizer_line(dev, peaks):
     res = {}
     algo = rows * cols * (2 + 0.5 + 0.0625)
     n = 120
-    for ss in (False, True):
+    gts = ops.nvfp4_quantize(x0, False, False, None, codes, scales, ws)[2].clone()  # g of x0
+    for ss, given in ((False, False), (True, False), (False, True)):
+        ts = gts if given else None
         for i in range(6):
-            ops.nvfp4_quantize(xs[i % 12], ss, False, None, codes, scales, ws)
+            ops.nvfp4_quantize(xs[i % 12], ss, False, ts, codes, scales, ws)
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
         with torch.cuda.graph(g, stream=side):
             for i in range(n):
-                ops.nvfp4_quantize(xs[i % 12], ss, False, None, codes, scales, ws)
+                ops.nvfp4_quantize(xs[i % 12], ss, False, ts, codes, scales, ws)
         g.replay()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -258,9 +260,9 @@ def quantizer_line(dev, peaks):
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / (3 * n)
         gbs = algo / (ms * 1e-3) / 1e9
-        res["scalesearch_on" if ss else "scalesearch_off"] = {
-            "us_per_call": 1e3 * ms, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
-            "kernels_per_call": 1}
+        key = ("scalesearch_on" if ss else "scalesearch_off") + ("_scale_given" if given else "")
+        res[key] = {"us_per_call": 1e3 * ms, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                    "kernels_per_call": 1}
         del g
     res["workload"] = synth.QUANT.name
     res["algorithmic_bytes"] = algo

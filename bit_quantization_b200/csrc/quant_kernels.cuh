@@ -144,15 +144,37 @@ __global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
   extern __shared__ uint4 cs[];  // chunk blocks x 32 bytes
   __shared__ float red[32];
   __shared__ int s_ok;
+  __shared__ __align__(8) uint64_t s_bar;
   const int64_t b0 = (int64_t)blockIdx.x * chunk;
+  const int64_t nvalid = b0 < n_blocks ? min(chunk, n_blocks - b0) : 0;
+  // the chunk arrives by one bulk copy; blocks past the tensor end are zeros
+  for (int64_t i = nvalid + threadIdx.x; i < chunk; i += blockDim.x)
+    cs[2 * i] = cs[2 * i + 1] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    if (nvalid > 0) {
+      mbar_arrive_expect_tx(&s_bar, (uint32_t)(nvalid * 32));
+      bulk_g2s(cs, x + b0 * 16, (uint32_t)(nvalid * 32), &s_bar);
+    } else {
+      mbar_arrive(&s_bar);
+    }
+  }
+  __syncthreads();
+  {
+    int never = 0;
+    if (!mbar_wait(&s_bar, 0, &never)) {
+      // timed out (status word set): give the copy a last bounded wait so
+      // that it does not land after the CTA has left
+      int again = 0;
+      mbar_wait(&s_bar, 0, &again, 200000000ull);
+      return;
+    }
+  }
   float a = 0.0f;
   for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
-    uint4 r0, r1;
-    load_raw(x, b0 + i, n_blocks, r0, r1);
-    cs[2 * i] = r0;
-    cs[2 * i + 1] = r1;
     float v[16];
-    unpack16<DT>(r0, r1, v);
+    unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
     if constexpr (G > 0) fwht_rows16<G>(v);
     a = fmaxf(a, block_absmax(v));
   }
