@@ -62,12 +62,14 @@ def lib():
         L.orc_topk_count.restype = i64
         L.orc_topk_count.argtypes = [f32, i64]
         L.orc_block_mean_topk.restype = i32
-        L.orc_block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P]
+        L.orc_block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                          i32, P, P]
         L.orc_block_mean_topk_varlen.restype = i32
-        L.orc_block_mean_topk_varlen.argtypes = [P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, P]
+        L.orc_block_mean_topk_varlen.argtypes = [P, P, i32, i32, i32, P, i32, i32, i32, i32, f32,
+                                                 i32, i32, P]
         L.orc_thrift_attn.restype = i32
         L.orc_thrift_attn.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, i32, i32,
-                                      P, i32, P, i64, i32, P, P, P, P, P]
+                                      i32, i32, P, i32, P, i64, i32, P, P, P, P, P]
         L.orc_attn_fp64.restype = i32
         L.orc_attn_fp64.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, P, i64, i32, P, P]
         _lib = L
@@ -213,9 +215,10 @@ def topk_count(frac, n_valid):
     return lib().orc_topk_count(float(frac), int(n_valid))
 
 
-def block_mean_topk(q, k, dt, blk, causal, frac):
+def block_mean_topk(q, k, dt, blk, causal, frac, sink_blocks=0, recent_blocks=0):
     """q [B,N,H,d], k [B,N,Hkv,d] uint16.  Returns (mask uint8 [B,H,nB,nB],
-    scores fp64 [B,H,nB,nB])."""
+    scores fp64 [B,H,nB,nB]).  sink_blocks / recent_blocks: fixed FP16 pairs
+    OR-ed with the top-k ones (reading R14 of oracle.cpp)."""
     q, k = _u16(q), _u16(k)
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -223,13 +226,14 @@ def block_mean_topk(q, k, dt, blk, causal, frac):
     mask = np.zeros((B, H, nb, nb), np.uint8)
     scores = np.zeros((B, H, nb, nb), np.float64)
     rc = lib().orc_block_mean_topk(_p(q), _p(k), dt, B, H, Hkv, N, d, blk, int(causal),
-                                   float(frac), _p(mask), _p(scores))
+                                   float(frac), int(sink_blocks), int(recent_blocks), _p(mask),
+                                   _p(scores))
     if rc:
         raise ValueError("oracle block_mean_topk: bad arguments")
     return mask, scores
 
 
-def block_mean_topk_varlen(q, k, dt, cu, blk, causal, frac):
+def block_mean_topk_varlen(q, k, dt, cu, blk, causal, frac, sink_blocks=0, recent_blocks=0):
     """q [total,H,d], k [total,Hkv,d]; cu int32 [nseq+1].  Returns the flat
     mask (per sequence [H, nB_s, nB_s], concatenated)."""
     q, k = _u16(q), _u16(k)
@@ -239,15 +243,18 @@ def block_mean_topk_varlen(q, k, dt, cu, blk, causal, frac):
     lens = np.diff(cu)
     nbs = (lens + blk - 1) // blk
     mask = np.zeros(int(H * np.sum(nbs.astype(np.int64) ** 2)), np.uint8)
-    lib().orc_block_mean_topk_varlen(_p(q), _p(k), dt, H, Hkv, _p(cu), len(lens), d, blk,
-                                     int(causal), float(frac), _p(mask))
+    rc = lib().orc_block_mean_topk_varlen(_p(q), _p(k), dt, H, Hkv, _p(cu), len(lens), d, blk,
+                                          int(causal), float(frac), int(sink_blocks),
+                                          int(recent_blocks), _p(mask))
+    if rc:
+        raise ValueError("oracle block_mean_topk_varlen: bad arguments")
     return mask
 
 
 # ---------------------------------------------------------------- attention
 
 def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
-                mask=None, units=None, nthreads=None):
+                mask=None, units=None, nthreads=None, sink_blocks=0, recent_blocks=0):
     """Emulated NVFP4 + FP16 attention over packed sequences.
 
     q [total,H,d], k/v [total,Hkv,d] uint16; cu int32 [nseq+1].
@@ -281,7 +288,8 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
     else:
         u, n_units = None, 0
     rc = lib().orc_thrift_attn(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
-                               int(causal), float(frac), int(use_ss), int(use_had), _p(m), given,
+                               int(causal), float(frac), int(sink_blocks), int(recent_blocks),
+                               int(use_ss), int(use_had), _p(m), given,
                                _p(u), n_units, int(nthreads or nthreads_default()), _p(out),
                                _p(lse), _p(gs), _p(out64), _p(tol))
     if rc:

@@ -44,6 +44,10 @@
 //      over the valid pairs; ties go to the lower linear index i*nB + j.
 //  R9  FP16 path: unrotated 16-bit Q, K, V; P rounded to the input dtype;
 //      l accumulates the fp32 probabilities before rounding.
+//  R14 sink-aware mixed precision (optional, off when both counts are 0):
+//      the first `sink` key blocks, and the `recent` most recent key blocks a
+//      query block can see, run on the FP16 path for every query block; the
+//      fixed pairs are OR-ed with the top-k pairs, whose quota is unchanged.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -375,9 +379,19 @@ int64_t orc_topk_count(float frac, int64_t n_valid) {
 }
 
 // Selection for one (sequence, head): mask [nB, nB] (1 = FP16 pair).
+// Sink-aware fixed pairs (ScaleSearchAttention, the sink-aware mixed-
+// precision paragraph; reading R14): key block j is kept at full precision
+// for query block i when j is one of the first `sink` blocks, or one of the
+// `recent` most recent blocks i can see (causal: i - recent < j <= i;
+// non-causal: the last `recent` blocks of the sequence).
+static bool fixed_pair(int i, int j, int nb, int causal, int sink, int recent) {
+  if (j < sink) return true;
+  return causal ? (j > i - recent) : (j >= nb - recent);
+}
+
 static void select_one(const uint16_t* q, const uint16_t* k, int dt, int H, int Hkv,
                        int h, const SeqView& s, int d, int blk, int causal, float frac,
-                       uint8_t* mask, double* scores) {
+                       int sink, int recent, uint8_t* mask, double* scores) {
   int nb = (s.len + blk - 1) / blk;
   int hk = h / (H / Hkv);
   std::vector<double> qm, km;
@@ -401,21 +415,26 @@ static void select_one(const uint16_t* q, const uint16_t* k, int dt, int H, int 
     return a.second < b.second;
   });
   for (int64_t t = 0; t < kk; ++t) mask[cand[(size_t)t].second] = 1;
+  // the fixed pairs are added to the top-k ones (the quota is unchanged)
+  for (int i = 0; i < nb; ++i)
+    for (int j = 0; j < nb && (!causal || j <= i); ++j)
+      if (fixed_pair(i, j, nb, causal, sink, recent)) mask[(int64_t)i * nb + j] = 1;
 }
 
 // q [B, N, H, d], k [B, N, Hkv, d] 16-bit; mask out uint8 [B, H, nB, nB];
 // scores (optional) fp64 [B, H, nB, nB] (every pair, valid or not).
 int orc_block_mean_topk(const uint16_t* q, const uint16_t* k, int dt, int B, int H, int Hkv,
-                        int N, int d, int blk, int causal, float frac, uint8_t* mask,
-                        double* scores) {
+                        int N, int d, int blk, int causal, float frac, int sink, int recent,
+                        uint8_t* mask, double* scores) {
   if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || d <= 0 || blk <= 0) return -1;
+  if (sink < 0 || recent < 0) return -1;
   int nb = (N + blk - 1) / blk;
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < H; ++h) {
       SeqView s{0, N};
       int64_t off = ((int64_t)b * H + h) * nb * nb;
       select_one(q + (int64_t)b * N * H * d, k + (int64_t)b * N * Hkv * d, dt, H, Hkv, h, s, d,
-                 blk, causal, frac, mask + off, scores ? scores + off : nullptr);
+                 blk, causal, frac, sink, recent, mask + off, scores ? scores + off : nullptr);
     }
   return 0;
 }
@@ -425,13 +444,15 @@ int orc_block_mean_topk(const uint16_t* q, const uint16_t* k, int dt, int B, int
 // [H, nB_s, nB_s].
 int orc_block_mean_topk_varlen(const uint16_t* q, const uint16_t* k, int dt, int H, int Hkv,
                                const int32_t* cu, int nseq, int d, int blk, int causal,
-                               float frac, uint8_t* mask) {
+                               float frac, int sink, int recent, uint8_t* mask) {
+  if (sink < 0 || recent < 0) return -1;
   int64_t off = 0;
   for (int sq = 0; sq < nseq; ++sq) {
     SeqView s{cu[sq], cu[sq + 1] - cu[sq]};
     int nb = (s.len + blk - 1) / blk;
     for (int h = 0; h < H; ++h) {
-      select_one(q, k, dt, H, Hkv, h, s, d, blk, causal, frac, mask + off, nullptr);
+      select_one(q, k, dt, H, Hkv, h, s, d, blk, causal, frac, sink, recent, mask + off,
+                 nullptr);
       off += (int64_t)nb * nb;
     }
   }
@@ -739,7 +760,8 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // implementation that evaluates the same arithmetic in another order.
 int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
                     int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
-                    float frac, int use_ss, int use_had, uint8_t* mask_io, int mask_given,
+                    float frac, int sink, int recent, int use_ss, int use_had,
+                    uint8_t* mask_io, int mask_given,
                     const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
                     float* lse, float* gs_out, double* out64, double* tol) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
@@ -791,7 +813,8 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
   }
   if (gs_out) { gs_out[0] = C.gq; gs_out[1] = C.gk; gs_out[2] = C.gv; }
   if (!mask_given)
-    orc_block_mean_topk_varlen(q, k, dt, H, Hkv, cu, nseq, d, blk, causal, frac, mask_io);
+    orc_block_mean_topk_varlen(q, k, dt, H, Hkv, cu, nseq, d, blk, causal, frac, sink, recent,
+                               mask_io);
   C.mask = mask_io;
   std::vector<int32_t> all;
   if (n_units == 0) {

@@ -262,6 +262,33 @@ def test_selection_brute_force(orc, causal):
             assert np.array_equal(mask[b, h], want)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_sink_blocks_are_added_to_topk(orc, causal):
+    # ScaleSearchAttention, sink-aware mixed precision: the first and the
+    # most recent key blocks stay at full precision.  Brute force over the
+    # pairs: the selection is the top-k set (quota unchanged) united with
+    # the fixed pairs, and nothing outside the valid pairs.
+    B, N, H, Hkv, d, blk = 1, 300, 3, 1, 32, 32
+    q = synth.randn16((B, N, H, d), torch.bfloat16, 30)
+    k = synth.randn16((B, N, Hkv, d), torch.bfloat16, 31)
+    nb = (N + blk - 1) // blk
+    for frac, sink, recent in [(0.0, 1, 1), (0.2, 1, 2), (0.3, 2, 0), (0.1, 0, 3), (0.0, 20, 0)]:
+        base, _ = orc.block_mean_topk(synth.as_u16(q), synth.as_u16(k), 1, blk, causal, frac)
+        mask, _ = orc.block_mean_topk(synth.as_u16(q), synth.as_u16(k), 1, blk, causal, frac,
+                                      sink_blocks=sink, recent_blocks=recent)
+        for h in range(H):
+            for i in range(nb):
+                seen = [j for j in range(nb) if not causal or j <= i]
+                newest = seen[-recent:] if recent else []
+                for j in range(nb):
+                    fixed = j in seen and (j < sink or j in newest)
+                    want = 1 if (base[0, h, i, j] or fixed) else 0
+                    assert mask[0, h, i, j] == want, (frac, sink, recent, h, i, j)
+        if sink >= nb:  # every valid pair
+            valid = nb * (nb + 1) // 2 if causal else nb * nb
+            assert mask.sum() == H * valid
+
+
 def test_selection_ties_go_to_lower_index(orc):
     q = torch.ones((1, 128, 1, 16), dtype=torch.float16)
     k = torch.ones((1, 128, 1, 16), dtype=torch.float16)
