@@ -216,7 +216,8 @@ constexpr int kTopkCache = 4096;  // 32 KB of keys: within the default shared-me
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __restrict__ scores,
                                                             SeqInfo seqs, int H, int blk, int nB,
-                                                            int causal, float frac,
+                                                            int causal, float frac, int sink,
+                                                            int recent,
                                                             uint8_t* __restrict__ mask) {
   __shared__ int hist[256];
   __shared__ int warp_sums[32];
@@ -238,9 +239,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
     const int i = (int)(lin / nB), j = (int)(lin % nB);
     return i < nb && j < nb && (!causal || j <= i);
   };
+  // ScaleSearchAttention's sink-aware pairs, added to the top-k ones: the
+  // first `sink` key blocks and the `recent` newest ones query block i sees
+  auto fixed = [&](int64_t lin) {
+    const int i = (int)(lin / nB), j = (int)(lin % nB);
+    return j < sink || (causal ? (j > i - recent) : (j >= nb - recent));
+  };
   if (k == 0 || k == n_valid) {
     for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x)
-      mk[lin] = (k != 0 && valid(lin)) ? 1 : 0;
+      mk[lin] = (valid(lin) && (k != 0 || fixed(lin))) ? 1 : 0;
     return;
   }
   const bool cached = npairs <= kTopkCache;
@@ -287,7 +294,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
     }
     const int eq = (ok && key == T) ? 1 : 0;
     const int before = block_exclusive_scan(eq, warp_sums, &s_total);
-    if (lin < npairs) mk[lin] = (ok && (key > T || (eq && taken + before < take_eq))) ? 1 : 0;
+    if (lin < npairs)
+      mk[lin] = (ok && (key > T || (eq && taken + before < take_eq) || fixed(lin))) ? 1 : 0;
     taken += s_total;
     __syncthreads();
   }

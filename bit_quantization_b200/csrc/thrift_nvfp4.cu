@@ -272,8 +272,8 @@ thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) 
 template <int DT>
 thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
                         int64_t total, int maxlen, int H, int Hkv, int d, int blk, int causal,
-                        float frac, int ss, int had, void* out, float* lse, int lse_varlen,
-                        void* ws, cudaStream_t st) {
+                        float frac, int sink, int recent, int ss, int had, void* out, float* lse,
+                        int lse_varlen, void* ws, cudaStream_t st) {
   AttnWs w = carve_attn(ws, nseq, maxlen, H, Hkv, d, blk);
   const int nB = (int)ceil_div(maxlen, blk), nTq = (int)ceil_div(maxlen, 128);
   const int G = d / 16;
@@ -304,7 +304,8 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   // selection
   pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, causal, w.scores);
-  topk_kernel<<<nseq * H, kTopkThreads, topk_smem(nB), st>>>(w.scores, si, H, blk, nB, causal, frac, w.mask);
+  topk_kernel<<<nseq * H, kTopkThreads, topk_smem(nB), st>>>(w.scores, si, H, blk, nB, causal,
+                                                             frac, sink, recent, w.mask);
   if (launch_status() != THRIFT_OK) return THRIFT_ERR_CUDA;
 
   AttnParams p;
@@ -497,8 +498,10 @@ size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int b
 
 thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int B, int H,
                               int Hkv, int N, int d, int blk, int causal, float topk_frac,
-                              uint8_t* mask, void* workspace, size_t ws_bytes, void* stream) {
+                              int sink_blocks, int recent_blocks, uint8_t* mask,
+                              void* workspace, size_t ws_bytes, void* stream) {
   if (!q || !k || !mask || !workspace) return THRIFT_ERR_ARG;
+  if (sink_blocks < 0 || recent_blocks < 0) return THRIFT_ERR_ARG;
   if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
   if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0) return THRIFT_ERR_ARG;
   if (!(topk_frac >= 0.0f && topk_frac <= 1.0f)) return THRIFT_ERR_ARG;
@@ -524,13 +527,15 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
   }
   pair_scores_kernel<<<pair_scores_grid(B, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       mq, mk, si, B, H, Hkv, d, blk, nB, causal, sc);
-  topk_kernel<<<B * H, kTopkThreads, topk_smem(nB), st>>>(sc, si, H, blk, nB, causal, topk_frac, mask);
+  topk_kernel<<<B * H, kTopkThreads, topk_smem(nB), st>>>(sc, si, H, blk, nB, causal, topk_frac,
+                                                          sink_blocks, recent_blocks, mask);
   return launch_status();
 }
 
 thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype dt, int B,
                                       int H, int Hkv, int N, int d, int blk, int causal,
-                                      float topk_frac, uint8_t* mask, void* stream) {
+                                      float topk_frac, int sink_blocks, int recent_blocks,
+                                      uint8_t* mask, void* stream) {
   if (!q || !k || !mask) return THRIFT_ERR_ARG;
   const size_t need = block_mean_topk_workspace_size(B, H, Hkv, N, d, blk);
   if (need == 0) return THRIFT_ERR_ARG;
@@ -538,8 +543,8 @@ thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype
   void* scratch = nullptr;
   const thrift_status s = noalloc_scratch(&scratch);
   if (s != THRIFT_OK) return s;
-  return block_mean_topk(q, k, dt, B, H, Hkv, N, d, blk, causal, topk_frac, mask, scratch,
-                         kNoAllocScratchBytes, stream);
+  return block_mean_topk(q, k, dt, B, H, Hkv, N, d, blk, causal, topk_frac, sink_blocks,
+                         recent_blocks, mask, scratch, kNoAllocScratchBytes, stream);
 }
 
 size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk) {
@@ -551,9 +556,11 @@ size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk) 
 
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
                               int B, int H, int Hkv, int N, int d, int blk, int causal,
-                              float topk_frac, int use_scalesearch, int use_hadamard, void* out,
-                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
+                              float topk_frac, int sink_blocks, int recent_blocks,
+                              int use_scalesearch, int use_hadamard, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream) {
   thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, N, d, blk, topk_frac, out, lse);
+  if (sink_blocks < 0 || recent_blocks < 0) return THRIFT_ERR_ARG;
   if (s != THRIFT_OK) return s;
   if (B <= 0 || !workspace || !aligned16(workspace)) return THRIFT_ERR_ARG;
   if (ws_bytes < thrift_attn_workspace_size(B, H, Hkv, N, d, blk)) return THRIFT_ERR_ARG;
@@ -563,9 +570,10 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrif
   const int64_t total = (int64_t)B * N;
   if (dt == THRIFT_BF16)
     return attn_impl<1>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
-                        use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
-  return attn_impl<0>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
-                      use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
+                        sink_blocks, recent_blocks, use_scalesearch, use_hadamard, out, lse, 0,
+                        workspace, st);
+  return attn_impl<0>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac, sink_blocks,
+                      recent_blocks, use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
 }
 
 size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hkv, int d,
@@ -589,10 +597,12 @@ size_t thrift_attn_varlen_workspace_size(int nseq, int64_t total, int max_seqlen
 thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v,
                                      thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
                                      int64_t total, int max_seqlen, int H, int Hkv, int d,
-                                     int blk, int causal, float topk_frac, int use_scalesearch,
-                                     int use_hadamard, void* out, float* lse, void* workspace,
-                                     size_t ws_bytes, void* stream) {
+                                     int blk, int causal, float topk_frac, int sink_blocks,
+                                     int recent_blocks, int use_scalesearch, int use_hadamard,
+                                     void* out, float* lse, void* workspace, size_t ws_bytes,
+                                     void* stream) {
   thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, max_seqlen, d, blk, topk_frac, out, lse);
+  if (sink_blocks < 0 || recent_blocks < 0) return THRIFT_ERR_ARG;
   if (s != THRIFT_OK) return s;
   if (!cu_seqlens || nseq <= 0 || nseq > 65535 || total <= 0 || !workspace ||
       !aligned16(workspace))
@@ -603,9 +613,11 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == THRIFT_BF16)
     return attn_impl<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal,
-                        topk_frac, use_scalesearch, use_hadamard, out, lse, 1, workspace, st);
+                        topk_frac, sink_blocks, recent_blocks, use_scalesearch, use_hadamard,
+                        out, lse, 1, workspace, st);
   return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
-                      use_scalesearch, use_hadamard, out, lse, 1, workspace, st);
+                      sink_blocks, recent_blocks, use_scalesearch, use_hadamard, out, lse, 1,
+                      workspace, st);
 }
 
 }  // extern "C"

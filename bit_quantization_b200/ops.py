@@ -58,21 +58,23 @@ def lib():
         L.block_mean_topk_workspace_size.restype = sz
         L.block_mean_topk_workspace_size.argtypes = [i32] * 6
         L.block_mean_topk.restype = i32
-        L.block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P, sz, P]
+        L.block_mean_topk.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                      P, P, sz, P]
         L.block_mean_topk_noalloc.restype = i32
-        L.block_mean_topk_noalloc.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P]
+        L.block_mean_topk_noalloc.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                              i32, i32, P, P]
         L.thrift_attn_workspace_size.restype = sz
         L.thrift_attn_workspace_size.argtypes = [i32] * 6
         L.thrift_attn_fwd.restype = i32
         L.thrift_attn_fwd.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
-                                      i32, P, P, P, sz, P]
+                                      i32, i32, i32, P, P, P, sz, P]
         L.thrift_attn_varlen_workspace_size.restype = sz
         L.thrift_attn_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
         L.thrift_attn_workspace_mask_offset.restype = sz
         L.thrift_attn_workspace_mask_offset.argtypes = [i32, i32, i32, i32, i32, i32]
         L.thrift_attn_fwd_varlen.restype = i32
         L.thrift_attn_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
-                                             i32, f32, i32, i32, P, P, P, sz, P]
+                                             i32, f32, i32, i32, i32, i32, P, P, P, sz, P]
         L.thrift_kernel_timer_enable.restype = i32
         L.thrift_kernel_timer_enable.argtypes = [i32]
         L.thrift_kernel_timer_read.restype = i32
@@ -194,8 +196,11 @@ def nvfp4_quantize_colblocks(x: torch.Tensor, use_scalesearch=False,
 
 # ------------------------------------------------------------------ selection
 
-def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, topk_frac: float):
-    """q [B,N,H,d], k [B,N,Hkv,d] -> mask u8 [B,H,nB,nB] (1 = FP16 pair)."""
+def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, topk_frac: float,
+                    sink_blocks: int = 0, recent_blocks: int = 0):
+    """q [B,N,H,d], k [B,N,Hkv,d] -> mask u8 [B,H,nB,nB] (1 = FP16 pair).
+    sink_blocks / recent_blocks: fixed FP16 key blocks added to the top-k
+    pairs (see the header)."""
     _need_cuda(q, k)
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -204,13 +209,15 @@ def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, to
     need = lib().block_mean_topk_workspace_size(B, H, Hkv, N, d, blk)
     ws = _ws.get(need, q.device)
     _check(lib().block_mean_topk(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk, int(causal),
-                                 float(topk_frac), _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
+                                 float(topk_frac), int(sink_blocks), int(recent_blocks),
+                                 _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
            "block_mean_topk")
     return mask
 
 
 def block_mean_topk_noalloc(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool,
-                            topk_frac: float, mask: Optional[torch.Tensor] = None):
+                            topk_frac: float, mask: Optional[torch.Tensor] = None,
+                            sink_blocks: int = 0, recent_blocks: int = 0):
     """block_mean_topk with the library's fixed scratch instead of a workspace,
     for callers that cannot allocate device memory (see the header).  Pass
     `mask` to avoid the one allocation this wrapper would otherwise make."""
@@ -221,7 +228,8 @@ def block_mean_topk_noalloc(q: torch.Tensor, k: torch.Tensor, blk: int, causal: 
     if mask is None:
         mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
     _check(lib().block_mean_topk_noalloc(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk,
-                                         int(causal), float(topk_frac), _ptr(mask), _stream(q)),
+                                         int(causal), float(topk_frac), int(sink_blocks),
+                                         int(recent_blocks), _ptr(mask), _stream(q)),
            "block_mean_topk_noalloc")
     return mask
 
@@ -233,7 +241,8 @@ def thrift_attn_workspace_size(B, H, Hkv, N, d, blk) -> int:
 
 
 def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesearch=False,
-                    use_hadamard=False, out=None, lse=None, workspace=None):
+                    use_hadamard=False, out=None, lse=None, workspace=None, sink_blocks=0,
+                    recent_blocks=0):
     """q [B,N,H,d], k/v [B,N,Hkv,d] -> (out [B,N,H,d], lse f32 [B,H,N])."""
     _need_cuda(q, k, v)
     B, N, H, d = q.shape
@@ -247,9 +256,10 @@ def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesear
         raise ThriftError("thrift_attn_fwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
     _check(lib().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, Hkv, N, d, blk,
-                                 int(causal), float(topk_frac), int(use_scalesearch),
-                                 int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-                                 _stream(q)), "thrift_attn_fwd")
+                                 int(causal), float(topk_frac), int(sink_blocks),
+                                 int(recent_blocks), int(use_scalesearch), int(use_hadamard),
+                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
+           "thrift_attn_fwd")
     return out, lse
 
 
@@ -265,7 +275,7 @@ def thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk) -
 
 def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True,
                            topk_frac=0.0, use_scalesearch=False, use_hadamard=False, out=None,
-                           lse=None, workspace=None):
+                           lse=None, workspace=None, sink_blocks=0, recent_blocks=0):
     """q [total,H,d], k/v [total,Hkv,d], cu_seqlens int32 [nseq+1] (CUDA) ->
     (out [total,H,d], lse f32 [H,total])."""
     _need_cuda(q, k, v, cu_seqlens)
@@ -284,7 +294,8 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
     ws = workspace if workspace is not None else _ws.get(need, q.device)
     _check(lib().thrift_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens),
                                         nseq, total, int(max_seqlen), H, Hkv, d, blk,
-                                        int(causal), float(topk_frac), int(use_scalesearch),
+                                        int(causal), float(topk_frac), int(sink_blocks),
+                                        int(recent_blocks), int(use_scalesearch),
                                         int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws),
                                         ws.numel(), _stream(q)), "thrift_attn_fwd_varlen")
     return out, lse

@@ -116,13 +116,20 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
  * fp64 fma over channels; per (batch, head) the k = ceil(frac*n_valid - 1e-9)
  * best valid pairs are selected (causal: j <= i), ties to the lower i*nB+j.
  *   mask [B, H, nB, nB] uint8 out, 1 = FP16 pair.
+ * sink_blocks, recent_blocks >= 0 (0, 0: off): ScaleSearchAttention's
+ * sink-aware mixed precision.  For every query block i the first
+ * sink_blocks key blocks and the recent_blocks most recent key blocks i can
+ * see (causal: i - recent_blocks < j <= i; non-causal: the last
+ * recent_blocks blocks) are FP16 pairs too, added to the top-k pairs (whose
+ * count k is unchanged).
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, 0<=frac<=1,
  * nB = ceil(N/blk) <= 512.
  */
 size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int B, int H,
                               int Hkv, int N, int d, int blk, int causal, float topk_frac,
-                              uint8_t* mask, void* workspace, size_t ws_bytes, void* stream);
+                              int sink_blocks, int recent_blocks, uint8_t* mask,
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------- attention --
  * [TA] + [SS] ScaleSearchAttention.  q [B,N,H,d], k, v [B,N,Hkv,d] 16-bit,
@@ -134,8 +141,11 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
  * softmax.  Q, K, V are quantised inside the call (Q, K along d; V along
  * tokens; use_scalesearch / use_hadamard as in nvfp4_quantize).
  *   out [B,N,H,d] 16-bit out;  lse [B,H,N] fp32 out (natural log).
+ * The FP16 pairs are those of block_mean_topk with the same topk_frac,
+ * sink_blocks and recent_blocks.
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, N >= 1,
- * 0 <= topk_frac <= 1, nB = ceil(N/blk) <= 512.
+ * 0 <= topk_frac <= 1, sink_blocks, recent_blocks >= 0,
+ * nB = ceil(N/blk) <= 512.
  */
 /* Same selection without a workspace argument.  For callers that cannot
  * allocate device memory: for example code that runs while a CUDA graph is
@@ -155,13 +165,15 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
 #define THRIFT_NOALLOC_SCRATCH_BYTES (8u << 20)
 thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype dt, int B,
                                       int H, int Hkv, int N, int d, int blk, int causal,
-                                      float topk_frac, uint8_t* mask, void* stream);
+                                      float topk_frac, int sink_blocks, int recent_blocks,
+                                      uint8_t* mask, void* stream);
 
 size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
                               int B, int H, int Hkv, int N, int d, int blk, int causal,
-                              float topk_frac, int use_scalesearch, int use_hadamard, void* out,
-                              float* lse, void* workspace, size_t ws_bytes, void* stream);
+                              float topk_frac, int sink_blocks, int recent_blocks,
+                              int use_scalesearch, int use_hadamard, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /* Varlen: q [total,H,d], k, v [total,Hkv,d] packed; cu_seqlens int32
  * [nseq+1] on the DEVICE (cu_seqlens[0] = 0, cu_seqlens[nseq] = total,
@@ -174,9 +186,10 @@ size_t thrift_attn_varlen_workspace_size(int nseq, int64_t total, int max_seqlen
 thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v,
                                      thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
                                      int64_t total, int max_seqlen, int H, int Hkv, int d,
-                                     int blk, int causal, float topk_frac, int use_scalesearch,
-                                     int use_hadamard, void* out, float* lse, void* workspace,
-                                     size_t ws_bytes, void* stream);
+                                     int blk, int causal, float topk_frac, int sink_blocks,
+                                     int recent_blocks, int use_scalesearch, int use_hadamard,
+                                     void* out, float* lse, void* workspace, size_t ws_bytes,
+                                     void* stream);
 
 /* Byte offset, inside the workspace of thrift_attn_fwd (nseq = B,
  * max_seqlen = N) or thrift_attn_fwd_varlen, of the block-pair selection the

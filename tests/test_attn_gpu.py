@@ -55,19 +55,22 @@ def _compare(got, want64, what, dtype, tol=None):
     return float(np.max(np.abs(got - want))), cos
 
 
-def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_off=3.0):
+def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_off=3.0,
+             sink=0, recent=0):
     w = synth.AttnWorkload("case", B, H, Hkv, N, d, dtype, causal, blk, frac, ss, had,
                            k_offset_std=k_off, seed=seed)
     inp = synth.make_attn_inputs(w)
     q, k, v = inp["q"], inp["k"], inp["v"]
     out, lse = ops.thrift_attn_fwd(q.cuda(), k.cuda(), v.cuda(), blk=blk, causal=causal,
-                                   topk_frac=frac, use_scalesearch=ss, use_hadamard=had)
+                                   topk_frac=frac, use_scalesearch=ss, use_hadamard=had,
+                                   sink_blocks=sink, recent_blocks=recent)
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == ops.OK
     dt = synth.dtype_code(dtype)
     cu = np.arange(B + 1, dtype=np.int32) * N
     qp, kp, vp = (synth.as_u16(t.reshape(B * N, -1, d)) for t in (q, k, v))
-    r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had)
+    r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had,
+                        sink_blocks=sink, recent_blocks=recent)
     got = out.cpu().reshape(B * N, H, d)
     gotf = got.double().numpy()
     _compare(gotf, r["out64"], "out", dtype, r["tol"])
@@ -123,6 +126,22 @@ def test_varlen_parity(orc):
         _compare(out.cpu().double().numpy(), r["out64"], f"varlen frac={frac}", torch.bfloat16,
                  r["tol"])
         assert np.max(np.abs(lse.cpu().numpy() - r["lse"])) < 1e-2
+
+
+SINK_CASES = [
+    # B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, sink, recent
+    (1, 640, 2, 1, 128, 128, True, 0.1, True, True, torch.bfloat16, 1, 1),
+    (1, 512, 2, 2, 128, 128, False, 0.0, False, False, torch.bfloat16, 1, 1),
+    (2, 300, 2, 1, 64, 64, True, 0.05, False, True, torch.float16, 2, 2),
+]
+
+
+@pytest.mark.parametrize("case", SINK_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_sink_blocks_parity(orc, case):
+    # ScaleSearchAttention's sink-aware mixed precision: the first and the
+    # most recent key blocks on the FP16 path, on top of the top-k pairs
+    *args, sink, recent = case
+    run_case(orc, *args, sink=sink, recent=recent)
 
 
 def test_all_fp16_pairs_match_fp64(orc):

@@ -45,3 +45,16 @@ def test_full_size_workloads(orc, w):
     nb = w.N // w.blk
     n_valid = nb * (nb + 1) // 2 if w.causal else nb * nb
     assert (m.reshape(w.B * w.H, -1).sum(1) == orc.topk_count(w.topk_frac, n_valid)).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("frac,sink,recent", [(0.0, 1, 1), (0.1, 1, 2), (0.3, 3, 0), (1.0, 1, 1)])
+def test_sink_blocks_parity(orc, causal, frac, sink, recent):
+    # ScaleSearchAttention's sink-aware pairs OR-ed with the top-k selection
+    q = synth.randn16((2, 1000, 4, 128), torch.bfloat16, 5)
+    k = (synth.randn16((2, 1000, 2, 128), torch.float32, 6) + 1.5).to(torch.bfloat16)
+    mask = ops.block_mean_topk(q.cuda(), k.cuda(), 128, causal, frac, sink_blocks=sink,
+                               recent_blocks=recent).cpu().numpy()
+    m0, _ = orc.block_mean_topk(synth.as_u16(q), synth.as_u16(k), synth.dtype_code(q.dtype), 128,
+                                causal, frac, sink_blocks=sink, recent_blocks=recent)
+    assert np.array_equal(mask, m0), f"{np.argwhere(mask != m0)[:5]}"
