@@ -291,6 +291,44 @@ def quantizer_only(args):
     return 0
 
 
+def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20):
+    """Average attention-kernel time of the bench workload run with another
+    selection (CUDA events around each attention launch)."""
+    def step():
+        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=frac,
+                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
+                            out=out, lse=lse, workspace=ws, sink_blocks=sink, recent_blocks=recent)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ops.kernel_timer_enable(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    ops.kernel_timer_enable(False)
+    kms, n = ops.kernel_timer_read()
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out (selection variant)")
+    return kms / max(n, 1)
+
+
+def sink_line(ops, q, k, v, w, inp, out, lse, ws, p16, sink=1, recent=1):
+    """ScaleSearchAttention's sink-aware variant of the bench workload: the
+    first and the newest key block of every query block on the FP16 path on
+    top of the top-k pairs; the attention kernel's rate against the FP4 /
+    FP16 roofline of its own pair split."""
+    mask = ops.block_mean_topk(q, k, w.blk, w.causal, w.topk_frac, sink_blocks=sink,
+                               recent_blocks=recent).cpu().numpy()
+    f4, f16 = pair_flops(mask, w, inp["lengths"])
+    k_ms = variant_kernel_ms(ops, q, k, v, w, out, lse, ws, w.topk_frac, sink, recent)
+    t_ideal = f4 / (4.0 * p16 * 1e12) + f16 / (p16 * 1e12)
+    achieved = (f4 + f16) / (k_ms * 1e-3) / 1e12
+    return {"sink_blocks": sink, "recent_blocks": recent, "topk_frac": w.topk_frac,
+            "kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "achieved": achieved,
+            "unit": "TFLOP/s", "fp16_share": f16 / (f4 + f16),
+            "frac": (t_ideal / (k_ms * 1e-3))}
+
+
 def nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4, steps=20):
     """The attention kernel with no FP16 pairs (topk_frac = 0): every score
     on the NVFP4 path, against the FP4 tensor peak alone."""
@@ -462,6 +500,7 @@ def main():
             "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
     if rank == 0 and world == 1:
         line["nvfp4_only"] = nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4)
+        line["sink_aware"] = sink_line(ops, q, k, v, w, inp, out, lse, ws, p16)
     if rank == 0 and world == 1 and not args.no_quantizer:
         line["quantizer"] = quantizer_line(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
