@@ -430,37 +430,69 @@ def main():
     ms_step = ms_total / args.steps
     value = world * flops / (ms_step * 1e-3) / 1e12
 
-    # end to end through the public API with host buffers
+    # End to end through the public API with host buffers: every step copies
+    # its Q, K, V from pinned host memory and reads its output and LSE back.
+    # Steps are pipelined the way a serving loop streams batches: step s+1's
+    # inputs go up on a copy stream and step s-1's results come down on
+    # another while step s computes (two device buffer sets).
     qh, kh, vh = (inp[n].pin_memory() for n in ("q", "k", "v"))
-    outh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    e2e_steps = max(3, min(args.steps, 30))
+    outh = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    lseh = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    qd = [torch.empty_like(q) for _ in range(2)]
+    kd = [torch.empty_like(k) for _ in range(2)]
+    vd = [torch.empty_like(v) for _ in range(2)]
+    od = [torch.empty_like(out) for _ in range(2)]
+    ld = [torch.empty_like(lse) for _ in range(2)]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    e2e_steps = max(4, min(args.steps, 30))
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step(qd, kd, vd)
-        outh.copy_(out, non_blocking=True)
-        lseh.copy_(lse, non_blocking=True)
+    def e2e_run(nsteps):
+        for st in range(nsteps):
+            b = st % 2
+            with torch.cuda.stream(s_in):
+                if st >= 2:
+                    s_in.wait_event(ev_comp[b])  # step st-2 has consumed buffer b
+                qd[b].copy_(qh, non_blocking=True)
+                kd[b].copy_(kh, non_blocking=True)
+                vd[b].copy_(vh, non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[b])
+                if st >= 2:
+                    s_comp.wait_event(ev_out[b])  # step st-2's results have left buffer b
+                ops.thrift_attn_fwd(qd[b], kd[b], vd[b], blk=w.blk, causal=w.causal,
+                                    topk_frac=w.topk_frac, use_scalesearch=w.use_scalesearch,
+                                    use_hadamard=w.use_hadamard, out=od[b], lse=ld[b],
+                                    workspace=ws)
+                ev_comp[b].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                outh[b].copy_(od[b], non_blocking=True)
+                lseh[b].copy_(ld[b], non_blocking=True)
+                ev_out[b].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(2)
+    torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps)
+    for sx in (s_in, s_comp, s_out):
+        torch.cuda.current_stream(dev).wait_stream(sx)
     e1.record()
     torch.cuda.synchronize(dev)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the end-to-end loop")
     te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
     e2e_ms = float(te[0]) / e2e_steps
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
-    d2h = outh.numel() * outh.element_size() + lseh.numel() * lseh.element_size()
+    d2h = outh[0].numel() * outh[0].element_size() + lseh[0].numel() * lseh[0].element_size()
 
     # roofline of the attention kernel (dominant): tensor-bound contraction;
     # t_ideal = F4/P4 + F16/P16 with P16 the measured bf16 GEMM rate and
@@ -496,7 +528,9 @@ def main():
             "data": "synthetic", "config": config_of(w), "roofline": roofline,
             "alu_roofline": alu_roofline,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "pipelining": "inputs of step s+1 and results of step s-1 copied while "
+                                  "step s computes (two buffer sets, three streams)"},
             "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
     if rank == 0 and world == 1:
         line["nvfp4_only"] = nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4)
