@@ -273,6 +273,35 @@ __host__ __device__ constexpr uint32_t f16_tile_bytes(uint32_t rows, uint32_t kd
   return rows * kdim * 2;
 }
 
+// Stages rows [0, nrows) of a tile into shared memory (row r from
+// src + r * src_stride elements, row_bytes each, 16-byte aligned) with one
+// bulk copy per row issued by warp 0, and zero-fills rows [nvalid, nrows).
+// Every thread returns once the copies have landed; false if the wait timed
+// out (device status set, the copies given a last bounded wait).
+__device__ __forceinline__ bool stage_tile_rows(uint4* dst, const uint16_t* src,
+                                                int64_t src_stride, int nvalid, int nrows,
+                                                int row_bytes, uint64_t* bar) {
+  const int row16 = row_bytes / 16;
+  for (int i = nvalid * row16 + threadIdx.x; i < nrows * row16; i += blockDim.x)
+    dst[i] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x < 32) {
+    if (threadIdx.x == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(bar, (uint32_t)(nvalid * row_bytes));
+    }
+    __syncwarp();
+    for (int r = threadIdx.x; r < nvalid; r += 32)
+      bulk_g2s(dst + r * row16, src + r * src_stride, (uint32_t)row_bytes, bar);
+  }
+  __syncthreads();
+  int never = 0;
+  if (mbar_wait(bar, 0, &never)) return true;
+  int again = 0;
+  mbar_wait(bar, 0, &again, 200000000ull);
+  return false;
+}
+
 // Q or K ([total, nh, d] 16-bit) -> per (sequence, head, tile) images, one
 // CTA per tile of tile_rows rows:
 //   img4:  codes [tile_rows, d/2] swizzled (pitch d/2), then scale factors;
@@ -282,7 +311,7 @@ __host__ __device__ constexpr uint32_t f16_tile_bytes(uint32_t rows, uint32_t kd
 // CTA also writes the fp64 means [nseq, nh, nB, d] of the blk-row blocks in
 // its tile (ThriftAttention, Metodologia step 1): the unrotated values summed
 // in row order from the block start, divided by the row count.  The tile is
-// read from HBM once, with 16-byte loads, into shared memory.  G = d/16.
+// read from HBM once, one bulk copy per row, into shared memory.  G = d/16.
 template <int DT, int G, bool HAD, bool SS>
 __global__ void __launch_bounds__(256) qk_tile_kernel(
     const uint16_t* __restrict__ x, SeqInfo seqs, int nh, int tile_rows, int ntiles, int blk,
@@ -290,20 +319,16 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
     double* __restrict__ means) {
   constexpr int D = G * 16;
   extern __shared__ uint4 tsm[];  // [tile_rows][D] 16-bit values
+  __shared__ __align__(8) uint64_t s_bar;
   const int tile = blockIdx.x, head = blockIdx.y, seq = blockIdx.z;
   int64_t start;
   int len;
   seqs.get(seq, start, len);
   const int t0 = tile * tile_rows;
   if (t0 >= len) return;
-  for (int i = threadIdx.x; i < tile_rows * (D / 8); i += blockDim.x) {
-    const int r = i / (D / 8), c8 = i % (D / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (t0 + r < len)
-      v = __ldg(reinterpret_cast<const uint4*>(x + ((start + t0 + r) * nh + head) * D) + c8);
-    tsm[i] = v;
-  }
-  __syncthreads();
+  if (!stage_tile_rows(tsm, x + ((start + t0) * nh + head) * D, (int64_t)nh * D,
+                       min(tile_rows, len - t0), tile_rows, D * 2, &s_bar))
+    return;
   const float g = tensor_scale_from_amax(*amax_in);
   const uint32_t t4 = fp4_tile_bytes(tile_rows, D), t16 = f16_tile_bytes(tile_rows, D);
   const int64_t tidx = ((int64_t)seq * nh + head) * ntiles + tile;
@@ -353,28 +378,24 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
 // 16-blocks along tokens, one CTA per key tile: img4 codes [d, blk/2]
 // swizzled (pitch blk/2) then scale factors (rows = channels); img16 = V^T
 // tile [d, blk] in blk/64 regions of [d, 128 B] with 128-byte swizzle.  Keys
-// past the sequence end are zeros.  The tile is read once, with 16-byte
-// loads, into shared memory; each thread then takes one (channel, 16-key)
+// past the sequence end are zeros.  The tile is read once, one bulk copy per
+// row, into shared memory; each thread then takes one (channel, 16-key)
 // column block from there.
 template <int DT, bool SS>
 __global__ void __launch_bounds__(256) v_tile_kernel(
     const uint16_t* __restrict__ v, SeqInfo seqs, int Hkv, int d, int blk, int ntiles,
     const uint32_t* amax_in, uint8_t* __restrict__ img4, uint8_t* __restrict__ img16) {
   extern __shared__ uint4 tsm[];  // [blk][d] 16-bit values
+  __shared__ __align__(8) uint64_t s_bar;
   const int j = blockIdx.x, hk = blockIdx.y, seq = blockIdx.z;
   int64_t start;
   int len;
   seqs.get(seq, start, len);
   const int t0 = j * blk;
   if (t0 >= len) return;
-  for (int i = threadIdx.x; i < blk * (d / 8); i += blockDim.x) {
-    const int r = i / (d / 8), c8 = i % (d / 8);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (t0 + r < len)
-      val = __ldg(reinterpret_cast<const uint4*>(v + ((start + t0 + r) * Hkv + hk) * d) + c8);
-    tsm[i] = val;
-  }
-  __syncthreads();
+  if (!stage_tile_rows(tsm, v + ((start + t0) * Hkv + hk) * d, (int64_t)Hkv * d,
+                       min(blk, len - t0), blk, d * 2, &s_bar))
+    return;
   const float g = tensor_scale_from_amax(*amax_in);
   const uint32_t t4 = fp4_tile_bytes(d, blk), t16 = f16_tile_bytes(d, blk);
   const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
