@@ -50,11 +50,11 @@ __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __rest
 }
 
 // scores [nseq, H, nB, nB] fp64 (valid i, j < nb of the sequence only;
-// causal: j <= i).  One CTA per (sequence, head, 64 x 64 tile of pairs);
-// each thread holds a 4 x 4 block of scores in registers, every score a
+// causal: j <= i).  One CTA per (sequence, head, 32 x 32 tile of pairs);
+// each thread holds a 2 x 2 block of scores in registers, every score a
 // sequential fma over the channels in order.  The means pass through shared
 // memory 32 channels at a time, channel-major.  nB <= 512.
-constexpr int kPairTile = 64, kPairChunk = 32;
+constexpr int kPairTile = 32, kPairChunk = 32, kPairSub = kPairTile / 16;
 
 __global__ void __launch_bounds__(256) pair_scores_kernel(const double* __restrict__ qm,
                                                           const double* __restrict__ km,
@@ -78,11 +78,11 @@ __global__ void __launch_bounds__(256) pair_scores_kernel(const double* __restri
   const double* qrow = qm + ((int64_t)seq * H + h) * nB * d;
   const double* krow = km + ((int64_t)seq * Hkv + hk) * nB * d;
   const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
-  double acc[4][4];
+  double acc[kPairSub][kPairSub];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < kPairSub; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < kPairSub; ++b) acc[a][b] = 0.0;
   for (int c0 = 0; c0 < d; c0 += kPairChunk) {
     __syncthreads();
     // rows i0.. / j0.. of the means, 32 channels each, transposed into
@@ -93,26 +93,26 @@ __global__ void __launch_bounds__(256) pair_scores_kernel(const double* __restri
       ks[c][r] = (j0 + r < nb) ? __ldg(krow + (int64_t)(j0 + r) * d + c0 + c) : 0.0;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
     for (int c = 0; c < kPairChunk; ++c) {
-      double qv[4], kv[4];
+      double qv[kPairSub], kv[kPairSub];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qv[a] = qs[c][4 * ti + a];
+      for (int a = 0; a < kPairSub; ++a) qv[a] = qs[c][kPairSub * ti + a];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kv[b] = ks[c][tj + 16 * b];
+      for (int b = 0; b < kPairSub; ++b) kv[b] = ks[c][tj + 16 * b];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < kPairSub; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[a], kv[b], acc[a][b]);
+        for (int b = 0; b < kPairSub; ++b) acc[a][b] = __fma_rn(qv[a], kv[b], acc[a][b]);
     }
   }
   double* out = scores + ((int64_t)seq * H + h) * nB * nB;
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + 4 * ti + a;
+  for (int a = 0; a < kPairSub; ++a) {
+    const int i = i0 + kPairSub * ti + a;
     if (i >= nb) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < kPairSub; ++b) {
       const int j = j0 + tj + 16 * b;
       if (j < nb) out[(int64_t)i * nB + j] = acc[a][b];
     }
@@ -262,10 +262,19 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
     const int shift = 56 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x) {
-      if (!valid(lin)) continue;
-      const uint64_t key = key_of(lin);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+    // keys sharing a digit in a warp add to its bin once (the leading
+    // digits of nearby scores coincide, and same-address shared atomics
+    // serialise)
+    for (int64_t base = 0; base < npairs; base += blockDim.x) {
+      const int64_t lin = base + threadIdx.x;
+      int digit = -1;
+      if (lin < npairs && valid(lin)) {
+        const uint64_t key = key_of(lin);
+        if ((key & pmask) == prefix) digit = (int)((key >> shift) & 255);
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, digit);
+      if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
+        atomicAdd(&hist[digit], __popc(same));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
