@@ -274,27 +274,24 @@ __host__ __device__ constexpr uint32_t f16_tile_bytes(uint32_t rows, uint32_t kd
 }
 
 // Stages rows [0, nrows) of a tile into shared memory (row r from
-// src + r * src_stride elements, row_bytes each, 16-byte aligned) with one
-// bulk copy per row issued by warp 0, and zero-fills rows [nvalid, nrows).
+// src + r * src_stride elements, row_bytes each, 16-byte aligned), one bulk
+// copy per row spread over all threads, and zero-fills rows [nvalid, nrows).
 // Every thread returns once the copies have landed; false if the wait timed
 // out (device status set, the copies given a last bounded wait).
 __device__ __forceinline__ bool stage_tile_rows(uint4* dst, const uint16_t* src,
                                                 int64_t src_stride, int nvalid, int nrows,
                                                 int row_bytes, uint64_t* bar) {
   const int row16 = row_bytes / 16;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, (uint32_t)(nvalid * row_bytes));
+  }
   for (int i = nvalid * row16 + threadIdx.x; i < nrows * row16; i += blockDim.x)
     dst[i] = make_uint4(0, 0, 0, 0);
-  if (threadIdx.x < 32) {
-    if (threadIdx.x == 0) {
-      mbar_init(bar, 1);
-      fence_mbar_init();
-      mbar_arrive_expect_tx(bar, (uint32_t)(nvalid * row_bytes));
-    }
-    __syncwarp();
-    for (int r = threadIdx.x; r < nvalid; r += 32)
-      bulk_g2s(dst + r * row16, src + r * src_stride, (uint32_t)row_bytes, bar);
-  }
   __syncthreads();
+  for (int r = threadIdx.x; r < nvalid; r += blockDim.x)
+    bulk_g2s(dst + r * row16, src + r * src_stride, (uint32_t)row_bytes, bar);
   int never = 0;
   if (mbar_wait(bar, 0, &never)) return true;
   int again = 0;
