@@ -396,8 +396,11 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
   const float g = tensor_scale_from_amax(*amax_in);
   const uint32_t t4 = fp4_tile_bytes(d, blk), t16 = f16_tile_bytes(d, blk);
   const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
-  uint8_t* t4p = img4 + tidx * t4;
-  uint8_t* sf = t4p + (uint32_t)d * (blk / 2);
+  // the two output images are assembled in shared memory (transposed rows
+  // would make scattered global stores) and leave by two bulk copies
+  uint8_t* o4 = reinterpret_cast<uint8_t*>(tsm) + (size_t)blk * d * 2;
+  uint8_t* o16 = o4 + ((t4 + 127) & ~127u);
+  uint8_t* sf = o4 + (uint32_t)d * (blk / 2);
   const uint16_t* tv = reinterpret_cast<const uint16_t*>(tsm);
   for (int i = threadIdx.x; i < d * (blk / 16); i += blockDim.x) {
     const int c = i % d, kb = (i / d) * 16;
@@ -410,10 +413,10 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
     }
     uint32_t lo, hi;
     const uint32_t S = quant_block16(val, g, SS, lo, hi);
-    *reinterpret_cast<uint2*>(t4p + swz_offset(c, kb / 2, blk / 2)) = make_uint2(lo, hi);
+    *reinterpret_cast<uint2*>(o4 + swz_offset(c, kb / 2, blk / 2)) = make_uint2(lo, hi);
     sf[sf_offset(c, kb / 16)] = (uint8_t)S;
     if (d == 64) sf[sf_offset(c + 64, kb / 16)] = 0;
-    uint8_t* reg = img16 + tidx * t16 + (kb / 64) * ((uint32_t)d * 128);
+    uint8_t* reg = o16 + (kb / 64) * ((uint32_t)d * 128);
     uint4 h0, h1;
     h0.x = raw[0] | ((uint32_t)raw[1] << 16);
     h0.y = raw[2] | ((uint32_t)raw[3] << 16);
@@ -425,6 +428,13 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
     h1.w = raw[14] | ((uint32_t)raw[15] << 16);
     *reinterpret_cast<uint4*>(reg + swz_offset(c, (kb % 64) * 2, 128)) = h0;
     *reinterpret_cast<uint4*>(reg + swz_offset(c, (kb % 64) * 2 + 16, 128)) = h1;
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bulk_s2g(img4 + tidx * t4, o4, t4);
+    bulk_s2g(img16 + tidx * t16, o16, t16);
+    bulk_commit_and_wait_read();
   }
 }
 

@@ -292,14 +292,20 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
     dispatch_qk_tile<DT, 4>(had, ss, ak, st);
   }
   {
+    // input tile, then the NVFP4 and 16-bit output images (128-byte aligned)
     dim3 grid(nB, Hkv, nseq);
-    const size_t smem = (size_t)blk * d * 2;
-    if (ss)
-      v_tile_kernel<DT, true><<<grid, kThreads, smem, st>>>(
-          static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
-    else
-      v_tile_kernel<DT, false><<<grid, kThreads, smem, st>>>(
-          static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB, w.amax + 2, w.v4, w.v16);
+    const size_t smem = (size_t)blk * d * 2 + ((fp4_tile_bytes(d, blk) + 127) & ~127u) +
+                        f16_tile_bytes(d, blk);
+    auto kern = ss ? v_tile_kernel<DT, true> : v_tile_kernel<DT, false>;
+    static bool attr[2] = {false, false};
+    if (!attr[ss ? 1 : 0]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               96 * 1024) != cudaSuccess)
+        return THRIFT_ERR_CUDA;
+      attr[ss ? 1 : 0] = true;
+    }
+    kern<<<grid, kThreads, smem, st>>>(static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB,
+                                       w.amax + 2, w.v4, w.v16);
   }
   // selection
   pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
