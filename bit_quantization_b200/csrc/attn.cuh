@@ -405,29 +405,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           const int st = t & 1;
           const bool f16 = t >= n4;
           uint64_t* full = f16 ? &bars[B_KVF16 + sl] : &bars[B_KVF4 + sl];
-          // operands first, then the waits
-          constexpr int NI = D / 16;  // FP16 MMAs per tile (NVFP4: D / 64)
-          uint64_t da[NI], db[NI], cpk[D / 64];
+          // NVFP4 operands first, then the waits
           const uint32_t dS = tmem + L::T_S + st * BLK;
           const uint32_t ksf = tmem + L::T_KSF + st * (D / 64) * 4;
-          if (!f16) {
-            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
+          const uint32_t so = (uint32_t)sl * ((f16 ? L::STG16 : L::STG4) >> 4);
+          uint64_t cpk[D / 64], db[D / 64];
 #pragma unroll
-            for (int s = 0; s < D / 64; ++s) {
-              cpk[s] = d_sf + ((L::OFF4_STG + BLK * (D / 2) + 512 * s) >> 4) + so;
-              da[s] = d_q4 + 2 * s;
-              db[s] = d_k4 + so + 2 * s;
-              pin64(cpk[s]);
-              pin64(db[s]);
-            }
-          } else {
-            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
-#pragma unroll
-            for (int s = 0; s < NI; ++s) {
-              da[s] = d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4);
-              db[s] = d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4);
-              pin64(db[s]);
-            }
+          for (int s = 0; s < D / 64; ++s) {
+            cpk[s] = d_sf + ((L::OFF4_STG + BLK * (D / 2) + 512 * s) >> 4) + so;
+            db[s] = d_k4 + so + 2 * s;
+            pin64(cpk[s]);
+            pin64(db[s]);
           }
           if (!mbar_wait(full, par, s_abort)) { ok = false; break; }
           if (!f16 && !q4_ready) {
@@ -454,10 +442,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
 #pragma unroll
             for (int s = 0; s < D / 64; ++s)
-              mma_nvf4(dS, da[s], db[s], id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s, s > 0);
+              mma_nvf4(dS, d_q4 + 2 * s, db[s], id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s,
+                       s > 0);
           } else {
 #pragma unroll
-            for (int s = 0; s < NI; ++s) mma_f16(dS, da[s], db[s], id_qk16, s > 0);
+            for (int s = 0; s < D / 16; ++s)
+              mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                      d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
           }
           tc_commit(&bars[B_SF + st]);
           advance(t);
@@ -472,36 +463,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           const int st = t & 1;
           const bool f16 = t >= n4;
           uint64_t* empty = f16 ? &bars[B_KVE16 + sl] : &bars[B_KVE4 + sl];
-          // Operands first: the waits below end when the correction step
-          // finishes, and from there on only the tensor instructions remain.
-          constexpr int NI = BLK / 16;  // FP16 MMAs per tile (NVFP4: BLK / 64)
-          uint64_t da[NI], db[NI], cpp[BLK / 64], cpv[BLK / 64];
-          uint32_t psf = 0, vsf = 0;
-          if (!f16) {
-            const uint32_t so = (uint32_t)sl * (L::STG4 >> 4);
-            const uint32_t po = (uint32_t)st * (L::PT4A >> 4);
-            psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
-            vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
+          // NVFP4 operands first: the waits below end when the correction
+          // step finishes, and from there on only the tensor instructions
+          // remain.
+          const uint32_t so = (uint32_t)sl * ((f16 ? L::STG16 : L::STG4) >> 4);
+          const uint32_t po = (uint32_t)st * (L::PT4A >> 4);
+          const uint32_t psf = tmem + L::T_PSF + st * (BLK / 64) * 4;
+          const uint32_t vsf = tmem + L::T_VSF + st * (BLK / 64) * 4;
+          uint64_t da[BLK / 64], db[BLK / 64], cpp[BLK / 64], cpv[BLK / 64];
 #pragma unroll
-            for (int s = 0; s < BLK / 64; ++s) {
-              cpp[s] = d_sf + ((L::OFF4_P + 128 * (BLK / 2) + 512 * s) >> 4) + po;
-              cpv[s] = d_sf + ((L::OFF4_STG + L::V4_OFF + D * (BLK / 2) + 512 * s) >> 4) + so;
-              da[s] = d_p4 + po + 2 * s;
-              db[s] = d_v4 + so + 2 * s;
-              pin64(cpp[s]);
-              pin64(cpv[s]);
-              pin64(da[s]);
-              pin64(db[s]);
-            }
-          } else {
-            const uint32_t so = (uint32_t)sl * (L::STG16 >> 4);
-#pragma unroll
-            for (int s = 0; s < NI; ++s) {
-              da[s] = d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4);
-              db[s] = d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4);
-              pin64(da[s]);
-              pin64(db[s]);
-            }
+          for (int s = 0; s < BLK / 64; ++s) {
+            cpp[s] = d_sf + ((L::OFF4_P + 128 * (BLK / 2) + 512 * s) >> 4) + po;
+            cpv[s] = d_sf + ((L::OFF4_STG + L::V4_OFF + D * (BLK / 2) + 512 * s) >> 4) + so;
+            da[s] = d_p4 + po + 2 * s;
+            db[s] = d_v4 + so + 2 * s;
+            pin64(cpp[s]);
+            pin64(cpv[s]);
+            pin64(da[s]);
+            pin64(db[s]);
           }
           if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
           if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
@@ -517,7 +496,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
               mma_nvf4(dO, da[s], db[s], id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
           } else {
 #pragma unroll
-            for (int s = 0; s < NI; ++s) mma_f16(dO, da[s], db[s], id_pv16, t > 0 || s > 0);
+            for (int s = 0; s < BLK / 16; ++s)
+              mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                      d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
+                      t > 0 || s > 0);
           }
           tc_commit(&bars[B_OD + st]);
           tc_commit(empty);
