@@ -189,19 +189,7 @@ __global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
     __threadfence();
     atomicAdd(&sync[0], 1u);
     // wait for every CTA's maximum (bounded)
-    int ok = 1;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-      unsigned arrived;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(sync) : "memory");
-      if (arrived >= gridDim.x) break;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        set_device_status(THRIFT_ERR_TIMEOUT);
-        ok = 0;
-        break;
-      }
-    }
-    s_ok = ok;
+    s_ok = spin_until_geq(sync, gridDim.x) ? 1 : 0;
   }
   __syncthreads();
   if (!s_ok) return;

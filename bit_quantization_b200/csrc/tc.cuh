@@ -76,6 +76,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded spin until the global word reaches `target` (acquire loads at GPU
+// scope, so what the writers published before their release is visible
+// after).  Gives up after `limit_ns` of wall time, sets the device status
+// word and returns false.
+__device__ __forceinline__ bool spin_until_geq(const unsigned* word, unsigned target,
+                                               uint64_t limit_ns = 2000000000ull) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
+    if (v >= target) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_device_status(THRIFT_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------- bulk copies (TMA unit) --
 
 // Contiguous global -> shared copy completing on `bar` (transaction bytes).

@@ -370,6 +370,28 @@ thrift_status noalloc_scratch(void** out) {
   return THRIFT_OK;
 }
 
+// Failure-detection aid: one thread waits, with the library's own bounded
+// waits, on something that never completes: an mbarrier that nothing arrives
+// on (mode 0) or a global word that nothing writes (mode 1).  The wait gives
+// up after limit_ns, sets the device status word and the kernel returns.
+static __device__ unsigned g_never_written = 0u;
+
+__global__ void wait_timeout_kernel(int mode, uint64_t limit_ns) {
+  __shared__ uint64_t s_bar;
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  if (mode == 0)
+    mbar_wait(&s_bar, 0, &s_abort, limit_ns);
+  else
+    spin_until_geq(&g_never_written, 1u, limit_ns);
+}
+
 }  // namespace
 }  // namespace thrift
 
@@ -400,6 +422,14 @@ thrift_status thrift_device_status(int reset) {
       return THRIFT_ERR_CUDA;
   }
   return (thrift_status)v;
+}
+
+thrift_status thrift_test_wait_timeout(int mode, int limit_us, void* stream) {
+  if (mode != 0 && mode != 1) return THRIFT_ERR_ARG;
+  if (limit_us < 1 || limit_us > 1000000) return THRIFT_ERR_ARG;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      mode, (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
 thrift_status thrift_kernel_timer_enable(int enable) {

@@ -28,7 +28,7 @@ EXPORTS = (
     "block_mean_topk", "block_mean_topk_noalloc", "thrift_attn_workspace_size", "thrift_attn_fwd",
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
     "thrift_attn_workspace_mask_offset",
-    "thrift_kernel_timer_enable", "thrift_kernel_timer_read",
+    "thrift_kernel_timer_enable", "thrift_kernel_timer_read", "thrift_test_wait_timeout",
 )
 
 
@@ -79,6 +79,8 @@ def lib():
         L.thrift_kernel_timer_enable.argtypes = [i32]
         L.thrift_kernel_timer_read.restype = i32
         L.thrift_kernel_timer_read.argtypes = [P, P]
+        L.thrift_test_wait_timeout.restype = i32
+        L.thrift_test_wait_timeout.argtypes = [i32, i32, P]
         _lib = L
     return _lib
 
@@ -131,6 +133,16 @@ def kernel_timer_read():
     n = C.c_int(0)
     _check(lib().thrift_kernel_timer_read(C.byref(ms), C.byref(n)), "thrift_kernel_timer_read")
     return ms.value, n.value
+
+
+def test_wait_timeout(mode: int, limit_us: int, device=None):
+    """Failure-detection aid: launches a kernel whose bounded wait (mode 0 an
+    mbarrier nothing arrives on, mode 1 a global word nothing writes) gives
+    up after ``limit_us`` and sets the device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    st = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check(lib().thrift_test_wait_timeout(int(mode), int(limit_us), st),
+           "thrift_test_wait_timeout")
 
 
 class Workspace:

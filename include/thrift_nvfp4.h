@@ -213,6 +213,17 @@ size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hk
 thrift_status thrift_kernel_timer_enable(int enable);
 thrift_status thrift_kernel_timer_read(double* total_ms, int* launches);
 
+/* Failure-detection aid (not part of the method).  Launches one small kernel
+ * on `stream` whose single waiting thread uses the library's bounded waits on
+ * something that never completes: mode 0 an mbarrier that nothing arrives
+ * on (the wait every pipelined kernel here uses between its roles), mode 1
+ * a global word that nothing writes (the quantiser's grid-wide exchange).
+ * After limit_us microseconds (1 .. 1,000,000) the wait gives up, sets the
+ * device status word to THRIFT_ERR_TIMEOUT and the kernel returns normally:
+ * no trap, the context stays usable.  Returns THRIFT_ERR_ARG for a bad mode
+ * or limit (nothing launched), THRIFT_ERR_CUDA if the launch fails. */
+thrift_status thrift_test_wait_timeout(int mode, int limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,6 +87,10 @@ def test_bad_arguments_rejected_before_launch(L):
                              0, 0, dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
     assert L.block_mean_topk(dummy, dummy, 0, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, -2, dummy,
                              ws, 1 << 40, None) == ops.ERR_ARG
+    # failure-detection aid: unknown mode, limits outside 1 us .. 1 s
+    assert L.thrift_test_wait_timeout(2, 1000, None) == ops.ERR_ARG
+    assert L.thrift_test_wait_timeout(0, 0, None) == ops.ERR_ARG
+    assert L.thrift_test_wait_timeout(1, 1000001, None) == ops.ERR_ARG
 
 
 def test_binding_fails_loudly_without_device():
