@@ -72,6 +72,9 @@ def lib():
                                       i32, i32, P, i32, P, i64, i32, P, P, P, P, P]
         L.orc_attn_fp64.restype = i32
         L.orc_attn_fp64.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, P, i64, i32, P, P]
+        L.orc_thrift_decode.restype = i32
+        L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
+                                        i32, i32, i32, P, i32, i32, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -318,3 +321,39 @@ def attn_fp64(q, k, v, dt, cu, causal, rows=None, nthreads=None):
     if rc:
         raise ValueError("oracle attn_fp64: bad arguments")
     return out, lse
+
+
+# ------------------------------------------------------------------ decode
+
+def thrift_decode(q, k, v, dt, lens, blk, g_kv, frac, use_ss=False, sink_blocks=0,
+                  recent_blocks=0, mask=None, nthreads=None):
+    """One decode step over the double cache (reading R15 of oracle.cpp).
+
+    q [B,H,d] uint16; k/v [B,ncap,Hkv,d] uint16 (token t of sequence b at
+    [b, t]); lens int32 [B]; g_kv (g_K, g_V) floats.  Returns dict(out
+    uint16 [B,H,d], out64 fp64 [B,H,d], tol fp64 [B,H,d], lse f32 [B,H],
+    mask uint8 [B,H,nbcap], gq)."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, H, d = q.shape
+    ncap, Hkv = k.shape[1], k.shape[2]
+    lens = np.ascontiguousarray(lens, np.int32)
+    nbcap = (ncap + blk - 1) // blk
+    if mask is None:
+        m = np.zeros((B, H, nbcap), np.uint8)
+        given = 0
+    else:
+        m = np.ascontiguousarray(mask, np.uint8).reshape(B, H, nbcap).copy()
+        given = 1
+    gkv = np.ascontiguousarray(g_kv, np.float32).reshape(2)
+    out = np.zeros((B, H, d), np.uint16)
+    out64 = np.zeros((B, H, d), np.float64)
+    tol = np.zeros((B, H, d), np.float64)
+    lse = np.full((B, H), np.nan, np.float32)
+    gq = np.zeros(1, np.float32)
+    rc = lib().orc_thrift_decode(_p(q), _p(k), _p(v), dt, B, H, Hkv, ncap, d, blk, _p(lens),
+                                 _p(gkv), float(frac), int(sink_blocks), int(recent_blocks),
+                                 int(use_ss), _p(m), given, int(nthreads or nthreads_default()),
+                                 _p(out), _p(lse), _p(gq), _p(out64), _p(tol))
+    if rc:
+        raise ValueError("oracle thrift_decode: bad arguments")
+    return {"out": out, "out64": out64, "tol": tol, "lse": lse, "mask": m, "gq": float(gq[0])}

@@ -48,6 +48,21 @@
 //      the first `sink` key blocks, and the `recent` most recent key blocks a
 //      query block can see, run on the FP16 path for every query block; the
 //      fixed pairs are OR-ed with the top-k pairs, whose quota is unchanged.
+//  R15 decode on the double cache (ThriftAttention, Resultados: decode
+//      speed-up; Significado: the KV cache grows by 28% because every token
+//      is cached in FP16 and in FP4): one new query token per sequence
+//      attends to the len_b cached tokens of its sequence (its own key
+//      included).  The cache holds K and V in 16 bits and in NVFP4 (K
+//      blocks along d; V 16-token blocks along the tokens from token 0, the
+//      last block zero-padded) under per-tensor scales g_K, g_V fixed by the
+//      caller when the cache is filled (a growing cache cannot re-derive
+//      its amax).  q is quantised with g_Q = amax(q of the step) / 2688.
+//      Selection: the query block is the query itself (qbar = q), kbar_j
+//      the mean of the cached 16-bit keys of block j; k = ceil(frac * nb)
+//      per (sequence, head) over the nb key blocks, ties to the lower j;
+//      fixed pairs: j < sink or j >= nb - recent.  The row then follows the
+//      prefill steps: NVFP4 tiles ascending, then FP16 tiles ascending, one
+//      online softmax.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -828,6 +843,264 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
   }
   parallel_for(n_units, nthreads, [&](int64_t u) {
     attn_unit(C, units[3 * u], units[3 * u + 1], units[3 * u + 2], out, lse, out64, tol);
+  });
+  return 0;
+}
+
+// ------------------------------------------------------------- decode --
+//
+// Reading R15.  q [B, H, d]; k, v [B, ncap, Hkv, d] 16-bit (token t of
+// sequence b at row b * ncap + t); lens [B] cached tokens (0 <= len <= ncap).
+
+// Rows of a [rows, cols] 16-bit matrix quantised under a given tensor scale,
+// one unpacked 4-bit code per byte (same arithmetic as orc_nvfp4_quantize with
+// the scale given).
+static void quantize_rows_given(const uint16_t* x, int dt, int64_t rows, int cols, float g,
+                                int use_ss, int nthreads, std::vector<uint8_t>& codes,
+                                std::vector<uint8_t>& scales) {
+  const int64_t chunk = 4096;
+  const int64_t nchunks = (rows + chunk - 1) / chunk;
+  codes.assign((size_t)(rows * cols), 0);
+  scales.assign((size_t)(rows * (cols / 16)), 0);
+  parallel_for(nchunks, nthreads, [&](int64_t c) {
+    std::vector<float> row(cols);
+    uint8_t packed[8];
+    for (int64_t r = c * chunk; r < std::min(rows, (c + 1) * chunk); ++r) {
+      for (int e = 0; e < cols; ++e) row[e] = orc_half_to_float(x[r * cols + e], dt);
+      for (int b = 0; b < cols / 16; ++b) {
+        orc_quant_block(&row[b * 16], g, use_ss, packed, &scales[(size_t)(r * (cols / 16) + b)],
+                        nullptr);
+        for (int e = 0; e < 8; ++e) {
+          codes[(size_t)(r * cols + b * 16 + 2 * e)] = packed[e] & 0xF;
+          codes[(size_t)(r * cols + b * 16 + 2 * e + 1)] = packed[e] >> 4;
+        }
+      }
+    }
+  });
+}
+
+// Selection of one (sequence, head) at decode (reading R15): mask [nbcap],
+// 1 = FP16 key block; entries past the sequence are 0.
+static void decode_select_one(const uint16_t* q, const uint16_t* k, int dt, int H, int Hkv,
+                              int ncap, int d, int blk, int b, int h, int len, float frac,
+                              int sink, int recent, uint8_t* mask, int nbcap) {
+  const int nb = (len + blk - 1) / blk;
+  const int hk = h / (H / Hkv);
+  for (int j = 0; j < nbcap; ++j) mask[j] = 0;
+  if (nb == 0) return;
+  std::vector<double> qm(d), km(d);
+  for (int c = 0; c < d; ++c) qm[c] = (double)orc_half_to_float(q[((int64_t)b * H + h) * d + c], dt);
+  std::vector<std::pair<double, int64_t>> cand;
+  for (int j = 0; j < nb; ++j) {
+    const int t0 = j * blk, t1 = std::min(len, t0 + blk);
+    for (int c = 0; c < d; ++c) {
+      double sum = 0.0;
+      for (int t = t0; t < t1; ++t)
+        sum += (double)orc_half_to_float(k[(((int64_t)b * ncap + t) * Hkv + hk) * d + c], dt);
+      km[c] = sum / (double)(t1 - t0);
+    }
+    cand.push_back({pair_score(qm.data(), km.data(), d), j});
+  }
+  const int64_t kk = orc_topk_count(frac, nb);
+  std::sort(cand.begin(), cand.end(), [](const std::pair<double, int64_t>& a,
+                                         const std::pair<double, int64_t>& bb) {
+    if (a.first != bb.first) return a.first > bb.first;
+    return a.second < bb.second;
+  });
+  for (int64_t t = 0; t < kk; ++t) mask[cand[(size_t)t].second] = 1;
+  for (int j = 0; j < nb; ++j)
+    if (j < sink || j >= nb - recent) mask[j] = 1;
+}
+
+struct DecCtx {
+  int dt, B, H, Hkv, ncap, d, blk, nbcap;
+  const int32_t* lens;
+  const uint16_t *q, *k, *v;
+  std::vector<uint8_t> qc, qs, kc, ks, vc, vs;  // unpacked codes, scale bytes
+  float gq, gk, gv;
+  const uint8_t* mask;  // [B, H, nbcap]
+};
+
+// One query row (sequence b, head h): the steps of attn_unit for a single,
+// non-causal row over the cached tokens.
+static void decode_row(const DecCtx& C, int b, int h, uint16_t* out, float* lse, double* out64,
+                       double* tol) {
+  const int d = C.d, blk = C.blk, H = C.H, Hkv = C.Hkv;
+  const int len = C.lens[b];
+  const int nb = (len + blk - 1) / blk;
+  const int hk = h / (H / Hkv);
+  const int64_t orow = ((int64_t)b * H + h) * d;
+  const double l2e = 1.4426950408889634;
+  const double s4 = l2e / std::sqrt((double)d), s16 = s4;
+  const uint8_t* mk = C.mask + ((int64_t)b * H + h) * C.nbcap;
+  std::vector<int> order;
+  for (int pass = 0; pass < 2; ++pass)
+    for (int j = 0; j < nb; ++j)
+      if ((mk[j] != 0) == (pass == 1)) order.push_back(pass == 0 ? j : -1 - j);
+  std::vector<double> qh(d), q16(d);
+  for (int c = 0; c < d; ++c) {
+    qh[c] = deq(C.qc[(size_t)(orow + c)], C.qs[(size_t)((orow + c) / 16)], C.gq);
+    q16[c] = orc_half_to_float(C.q[orow + c], C.dt);
+  }
+  double m = -INFINITY, l = 0.0;
+  std::vector<double> O(d, 0.0), amb(d, 0.0), dq(blk), kt((size_t)blk * d), vt((size_t)blk * d),
+      S(blk), Pq(blk);
+  std::vector<float> Pt(blk), Ph(blk);
+  const int64_t vcol = C.nbcap * (int64_t)blk;  // padded tokens per V column
+  for (int code : order) {
+    const bool fp4 = code >= 0;
+    const int j = fp4 ? code : -1 - code;
+    const int k0 = j * blk, k1 = std::min(len, k0 + blk), nk = k1 - k0;
+    for (int t = 0; t < nk; ++t)
+      for (int c = 0; c < d; ++c) {
+        const int64_t e = (((int64_t)b * C.ncap + k0 + t) * Hkv + hk) * d + c;
+        if (fp4) {
+          kt[(size_t)t * d + c] = deq(C.kc[(size_t)e], C.ks[(size_t)(e / 16)], C.gk);
+          const int64_t ve = (((int64_t)b * Hkv + hk) * d + c) * vcol + k0 + t;
+          vt[(size_t)t * d + c] = deq(C.vc[(size_t)ve], C.vs[(size_t)(ve / 16)], C.gv);
+        } else {
+          kt[(size_t)t * d + c] = orc_half_to_float(C.k[e], C.dt);
+          vt[(size_t)t * d + c] = orc_half_to_float(C.v[e], C.dt);
+        }
+      }
+    const double* qv = fp4 ? qh.data() : q16.data();
+    double mt = -INFINITY;
+    for (int t = 0; t < nk; ++t) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += qv[c] * kt[(size_t)t * d + c];
+      S[t] = acc * (fp4 ? s4 : s16);
+      mt = std::max(mt, S[t]);
+    }
+    const double mn = std::max(m, mt);
+    const double alpha = std::exp2(m - mn);  // 0 when m is still -inf
+    l *= alpha;
+    for (int c = 0; c < d; ++c) {
+      O[c] *= alpha;
+      amb[c] *= alpha;
+    }
+    float rowmax = 0.0f;
+    for (int t = 0; t < nk; ++t) {
+      Pt[t] = (float)std::exp2(S[t] - mn);
+      l += (double)Pt[t];
+      rowmax = std::max(rowmax, Pt[t]);
+    }
+    if (fp4) {
+      if (rowmax == 0.0f) { m = mn; continue; }
+      const float inv = 2688.0f / rowmax;
+      const float sigma = rowmax / 2688.0f;
+      for (int t = 0; t < blk; ++t) Ph[t] = t < nk ? Pt[t] * inv : 0.0f;
+      for (int b0 = 0; b0 < blk; b0 += 16) {
+        float amax = 0.0f;
+        for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
+        const float s_real = amax / 6.0f;
+        const uint8_t sp = orc_ue4m3_encode(s_real);
+        const float dec = orc_ue4m3_decode(sp);
+        const float rr = 1.0f / dec;
+        for (int e = 0; e < 16; ++e) {
+          const float tq = Ph[b0 + e] * rr;
+          Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(tq)) * (double)dec;
+          dq[b0 + e] = sp == 0 ? 0.0 : e2m1_ambiguity(tq) * (double)dec;
+        }
+        const int alt = ue4m3_ambiguous_neighbour(s_real, sp);
+        if (alt > 0) {
+          const float dec2 = orc_ue4m3_decode((uint8_t)alt);
+          const float rr2 = 1.0f / dec2;
+          for (int e = 0; e < 16; ++e) {
+            const double q2 =
+                (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr2)) * (double)dec2;
+            dq[b0 + e] = std::max(dq[b0 + e], std::fabs(q2 - Pq[b0 + e]));
+          }
+        }
+      }
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0, ab = 0.0;
+        for (int t = 0; t < nk; ++t) {
+          acc += Pq[t] * vt[(size_t)t * d + c];
+          ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
+        }
+        O[c] += (double)sigma * acc;
+        amb[c] += (double)sigma * ab;
+      }
+    } else {
+      for (int t = 0; t < nk; ++t) dq[t] = half_ambiguity((double)Pt[t], C.dt);
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0, ab = 0.0;
+        for (int t = 0; t < nk; ++t) {
+          acc += (double)orc_half_to_float(orc_double_to_half((double)Pt[t], C.dt), C.dt) *
+                 vt[(size_t)t * d + c];
+          ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
+        }
+        O[c] += acc;
+        amb[c] += ab;
+      }
+    }
+    m = mn;
+  }
+  const double ln2 = 0.6931471805599453;
+  for (int c = 0; c < d; ++c) {
+    const double o = l > 0.0 ? O[c] / l : 0.0;
+    out[orow + c] = orc_double_to_half(o, C.dt);
+    if (out64) out64[orow + c] = o;
+    if (tol) tol[orow + c] = l > 0.0 ? amb[c] / l : 0.0;
+  }
+  lse[(int64_t)b * H + h] = l > 0.0 ? (float)(m * ln2 + std::log(l)) : -INFINITY;
+}
+
+// Decode step over the double cache (reading R15).  g_kv: g_K, g_V.
+// mask [B, H, nbcap] (nbcap = ceil(ncap / blk)): read when mask_given, else
+// computed and written.  out 16-bit [B, H, d]; lse fp32 [B, H] (natural log;
+// -inf and a zero row for an empty sequence).  gq_out (optional) receives
+// g_Q; out64 / tol (optional) as in orc_thrift_attn.
+int orc_thrift_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int B,
+                      int H, int Hkv, int ncap, int d, int blk, const int32_t* lens,
+                      const float* g_kv, float frac, int sink, int recent, int use_ss,
+                      uint8_t* mask_io, int mask_given, int nthreads, uint16_t* out, float* lse,
+                      float* gq_out, double* out64, double* tol) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || ncap <= 0 || d % 16 || blk % 16 || blk <= 0)
+    return -1;
+  if (sink < 0 || recent < 0 || !(frac >= 0.0f && frac <= 1.0f)) return -1;
+  for (int b = 0; b < B; ++b)
+    if (lens[b] < 0 || lens[b] > ncap) return -1;
+  DecCtx C;
+  C.dt = dt; C.B = B; C.H = H; C.Hkv = Hkv; C.ncap = ncap; C.d = d; C.blk = blk;
+  C.nbcap = (ncap + blk - 1) / blk;
+  C.lens = lens; C.q = q; C.k = k; C.v = v;
+  C.gk = g_kv[0];
+  C.gv = g_kv[1];
+  C.gq = quantize_rows_unpacked(q, dt, (int64_t)B * H, d, use_ss, 0, nthreads, C.qc, C.qs);
+  quantize_rows_given(k, dt, (int64_t)B * ncap * Hkv, d, C.gk, use_ss, nthreads, C.kc, C.ks);
+  // V: per (sequence, kv head, channel) column of nbcap * blk tokens, 16-blocks
+  // from token 0, tokens at or past len zero.
+  const int64_t vcol = (int64_t)C.nbcap * blk;
+  C.vc.assign((size_t)((int64_t)B * Hkv * d * vcol), 0);
+  C.vs.assign((size_t)((int64_t)B * Hkv * d * vcol / 16), 0);
+  parallel_for((int64_t)B * Hkv * d, nthreads, [&](int64_t bc) {
+    const int64_t b = bc / ((int64_t)Hkv * d), hk = (bc / d) % Hkv, c = bc % d;
+    float col[16];
+    uint8_t packed[8];
+    for (int64_t t0 = 0; t0 < vcol; t0 += 16) {
+      for (int e = 0; e < 16; ++e)
+        col[e] = t0 + e < lens[b]
+                     ? orc_half_to_float(v[((b * ncap + t0 + e) * Hkv + hk) * d + c], dt)
+                     : 0.0f;
+      const int64_t base = bc * vcol + t0;
+      orc_quant_block(col, C.gv, use_ss, packed, &C.vs[(size_t)(base / 16)], nullptr);
+      for (int e = 0; e < 8; ++e) {
+        C.vc[(size_t)(base + 2 * e)] = packed[e] & 0xF;
+        C.vc[(size_t)(base + 2 * e + 1)] = packed[e] >> 4;
+      }
+    }
+  });
+  if (gq_out) *gq_out = C.gq;
+  if (!mask_given)
+    parallel_for((int64_t)B * H, nthreads, [&](int64_t u) {
+      const int b = (int)(u / H), h = (int)(u % H);
+      decode_select_one(q, k, dt, H, Hkv, ncap, d, blk, b, h, lens[b], frac, sink, recent,
+                        mask_io + u * C.nbcap, C.nbcap);
+    });
+  C.mask = mask_io;
+  parallel_for((int64_t)B * H, nthreads, [&](int64_t u) {
+    decode_row(C, (int)(u / H), (int)(u % H), out, lse, out64, tol);
   });
   return 0;
 }
