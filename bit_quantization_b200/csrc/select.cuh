@@ -208,10 +208,90 @@ __device__ __forceinline__ int select_digit(const int* hist, int64_t rem, int64_
   return sel;
 }
 
-// One CTA per (sequence, head): exact top-k by an 8-pass radix select on the
-// 64-bit keys, then ties at the threshold taken in ascending linear index.
-// mask [nseq, H, nB, nB] uint8 (1 = FP16 pair); every entry is written.  The
-// keys are read once into shared memory when they fit (kTopkCache).
+// Exact top-k of one CTA over n entries by an 8-pass radix select on the
+// 64-bit order keys, then ties at the threshold taken in ascending index.
+// out[i] = 1 for the k largest valid entries and for every valid entry that
+// `fixed` names, else 0 (every out[i], i < n, is written).  The keys are read
+// once into `kcache` when it is given (n entries).  All threads of the CTA
+// call it.
+struct TopkShared {
+  int hist[256];
+  int warp_sums[32];
+  int total;
+  uint64_t prefix;
+  int64_t remaining;
+};
+
+template <class Valid, class Fixed, class Score>
+__device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, Fixed fixed,
+                           Score score, uint64_t* kcache, TopkShared& sh,
+                           uint8_t* __restrict__ out) {
+  if (k == 0 || k == n_valid) {
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x)
+      out[i] = (valid(i) && (k != 0 || fixed(i))) ? 1 : 0;
+    return;
+  }
+  if (kcache) {
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x)
+      kcache[i] = valid(i) ? order_key(score(i)) : 0ull;
+  }
+  auto key_of = [&](int64_t i) { return kcache ? kcache[i] : order_key(score(i)); };
+  uint64_t prefix = 0, pmask = 0;
+  int64_t rem = k;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
+    __syncthreads();
+    // keys sharing a digit in a warp add to its bin once (the leading
+    // digits of nearby scores coincide, and same-address shared atomics
+    // serialise)
+    for (int64_t base = 0; base < n; base += blockDim.x) {
+      const int64_t i = base + threadIdx.x;
+      int digit = -1;
+      if (i < n && valid(i)) {
+        const uint64_t key = key_of(i);
+        if ((key & pmask) == prefix) digit = (int)((key >> shift) & 255);
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, digit);
+      if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
+        atomicAdd(&sh.hist[digit], __popc(same));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int64_t above;
+      const int sel = select_digit(sh.hist, rem, &above);
+      if (threadIdx.x == 0) {
+        sh.remaining = rem - above;
+        sh.prefix = prefix | ((uint64_t)sel << shift);
+      }
+    }
+    __syncthreads();
+    prefix = sh.prefix;
+    rem = sh.remaining;
+    pmask |= (uint64_t)255 << shift;
+  }
+  const uint64_t T = prefix;
+  const int64_t take_eq = rem;
+  int64_t taken = 0;
+  for (int64_t base = 0; base < n; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    uint64_t key = 0;
+    bool ok = false;
+    if (i < n && valid(i)) {
+      key = key_of(i);
+      ok = true;
+    }
+    const int eq = (ok && key == T) ? 1 : 0;
+    const int before = block_exclusive_scan(eq, sh.warp_sums, &sh.total);
+    if (i < n) out[i] = (ok && (key > T || (eq && taken + before < take_eq) || fixed(i))) ? 1 : 0;
+    taken += sh.total;
+    __syncthreads();
+  }
+}
+
+// One CTA per (sequence, head) of the pair selection.  mask [nseq, H, nB, nB]
+// uint8 (1 = FP16 pair); every entry is written.  The keys are cached in
+// shared memory when they fit (kTopkCache).
 constexpr int kTopkCache = 4096;  // 32 KB of keys: within the default shared-memory limit
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __restrict__ scores,
@@ -219,11 +299,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
                                                             int causal, float frac, int sink,
                                                             int recent,
                                                             uint8_t* __restrict__ mask) {
-  __shared__ int hist[256];
-  __shared__ int warp_sums[32];
-  __shared__ int s_total;
-  __shared__ uint64_t s_prefix;
-  __shared__ int64_t s_remaining;
+  __shared__ TopkShared sh;
   extern __shared__ uint64_t kcache[];
   const int seq = blockIdx.x / H, h = blockIdx.x % H;
   int64_t start;
@@ -245,69 +321,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
     const int i = (int)(lin / nB), j = (int)(lin % nB);
     return j < sink || (causal ? (j > i - recent) : (j >= nb - recent));
   };
-  if (k == 0 || k == n_valid) {
-    for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x)
-      mk[lin] = (valid(lin) && (k != 0 || fixed(lin))) ? 1 : 0;
-    return;
-  }
-  const bool cached = npairs <= kTopkCache;
-  if (cached) {
-    for (int64_t lin = threadIdx.x; lin < npairs; lin += blockDim.x)
-      kcache[lin] = valid(lin) ? order_key(sc[lin]) : 0ull;
-  }
-  auto key_of = [&](int64_t lin) { return cached ? kcache[lin] : order_key(sc[lin]); };
-  uint64_t prefix = 0, pmask = 0;
-  int64_t rem = k;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    // keys sharing a digit in a warp add to its bin once (the leading
-    // digits of nearby scores coincide, and same-address shared atomics
-    // serialise)
-    for (int64_t base = 0; base < npairs; base += blockDim.x) {
-      const int64_t lin = base + threadIdx.x;
-      int digit = -1;
-      if (lin < npairs && valid(lin)) {
-        const uint64_t key = key_of(lin);
-        if ((key & pmask) == prefix) digit = (int)((key >> shift) & 255);
-      }
-      const unsigned same = __match_any_sync(0xffffffffu, digit);
-      if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
-        atomicAdd(&hist[digit], __popc(same));
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      int64_t above;
-      const int sel = select_digit(hist, rem, &above);
-      if (threadIdx.x == 0) {
-        s_remaining = rem - above;
-        s_prefix = prefix | ((uint64_t)sel << shift);
-      }
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    rem = s_remaining;
-    pmask |= (uint64_t)255 << shift;
-  }
-  const uint64_t T = prefix;
-  const int64_t take_eq = rem;
-  int64_t taken = 0;
-  for (int64_t base = 0; base < npairs; base += blockDim.x) {
-    const int64_t lin = base + threadIdx.x;
-    uint64_t key = 0;
-    bool ok = false;
-    if (lin < npairs && valid(lin)) {
-      key = key_of(lin);
-      ok = true;
-    }
-    const int eq = (ok && key == T) ? 1 : 0;
-    const int before = block_exclusive_scan(eq, warp_sums, &s_total);
-    if (lin < npairs)
-      mk[lin] = (ok && (key > T || (eq && taken + before < take_eq) || fixed(lin))) ? 1 : 0;
-    taken += s_total;
-    __syncthreads();
-  }
+  auto score = [&](int64_t lin) { return sc[lin]; };
+  radix_topk(npairs, k, n_valid, valid, fixed, score, npairs <= kTopkCache ? kcache : nullptr,
+             sh, mk);
 }
 
 inline size_t topk_smem(int nB) {

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "attn.cuh"
+#include "decode.cuh"
 #include "select.cuh"
 
 namespace thrift {
@@ -370,6 +371,155 @@ thrift_status noalloc_scratch(void** out) {
   return THRIFT_OK;
 }
 
+// ---------------------------------------------------------------- decode --
+
+constexpr int kDecMaxSplit = 32;  // CTAs per (sequence, kv head)
+
+bool decode_shape_ok(int H, int Hkv, int d, int blk, thrift_status* why) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv) { *why = THRIFT_ERR_ARG; return false; }
+  if (d != kDecD || blk != kDecTile || H / Hkv > kDecMaxG || H > 65535 || Hkv > 65535) {
+    *why = THRIFT_ERR_UNSUPPORTED;
+    return false;
+  }
+  return true;
+}
+
+CacheGeom cache_geom(int B, int Hkv, int capacity) {
+  CacheGeom cg;
+  cg.B = B;
+  cg.Hkv = Hkv;
+  cg.ntc = (int)ceil_div(capacity, kDecTile);
+  return cg;
+}
+
+struct DecWs {
+  uint32_t* amax;
+  uint8_t* q4;
+  uint8_t* q16;
+  double* scores;
+  uint8_t* mask;
+  float* part_o;
+  float* part_ml;
+  size_t bytes;
+};
+
+DecWs carve_decode(void* ws, int B, int H, int Hkv, int capacity) {
+  Carve c(ws);
+  DecWs w;
+  const int64_t nbcap = ceil_div(capacity, kDecTile);
+  w.amax = c.take<uint32_t>(16);
+  w.q4 = c.take<uint8_t>((size_t)B * Hkv * kDecQ4Bytes);
+  w.q16 = c.take<uint8_t>((size_t)B * Hkv * kDecQ16Bytes);
+  w.scores = c.take<double>((size_t)B * H * nbcap * 8);
+  w.mask = c.take<uint8_t>((size_t)B * H * nbcap);
+  w.part_o = c.take<float>((size_t)B * H * 2 * kDecMaxSplit * kDecD * 4);
+  w.part_ml = c.take<float>((size_t)B * H * 2 * kDecMaxSplit * 2 * 4);
+  w.bytes = (c.off + 1023) & ~(size_t)1023;
+  return w;
+}
+
+// CTAs per (sequence, kv head).  One CTA fits an SM, so the grid runs in
+// waves of sm_count CTAs: take the fewest waves (two at least, when the
+// problem has that many tiles) whose last wave is at least 90% full, else
+// the fullest; never more than one CTA per key tile, never a CTA with more
+// than 512 key tiles (each may appear in both lists).
+int decode_splits(int B, int Hkv, int ntc) {
+  const int64_t pairs = (int64_t)B * Hkv, sms = sm_count();
+  const int lo = std::max(1, (int)ceil_div(ntc, (int64_t)DecLayout::MAX_TILES / 2));
+  const int hi = std::max(lo, std::min(kDecMaxSplit, ntc));
+  int best = lo;
+  double best_eff = -1.0;
+  for (int waves = 1; waves <= 16; ++waves) {
+    int ns = (int)std::max<int64_t>(1, waves * sms / pairs);
+    ns = std::min(std::max(ns, lo), hi);
+    const int64_t ctas = pairs * ns;
+    const double eff = (double)ctas / (double)(ceil_div(ctas, sms) * sms);
+    if (waves >= 2 && eff >= 0.9) return ns;
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+  }
+  return best;
+}
+
+template <int DT, bool SS>
+void launch_kv_append(const void* kn, const void* vn, const CacheGeom& cg, int max_new,
+                      int capacity, const int32_t* cache_len, const int32_t* n_new,
+                      const float* kv_scale, uint8_t* cache, cudaStream_t st) {
+  kv_append_kernel<DT, SS><<<dim3(max_new, cg.Hkv, cg.B), kDecD, 0, st>>>(
+      static_cast<const uint16_t*>(kn), static_cast<const uint16_t*>(vn), cg, max_new, capacity,
+      cache_len, n_new, kv_scale, cache);
+  const int nv16 = (int)ceil_div(max_new, 16) + 1, nmt = (int)ceil_div(max_new, kDecTile) + 1;
+  kv_requant_kernel<DT, SS><<<dim3(nv16 + nmt, cg.Hkv, cg.B), kDecD, 0, st>>>(
+      cg, max_new, capacity, cache_len, n_new, kv_scale, nv16, cache);
+}
+
+template <int DT, int GC>
+thrift_status launch_decode_kernel(const DecParams& p, int B, int Hkv, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_decode_kernel<DT, GC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)DecLayout::SMEM_ALLOC) != cudaSuccess)
+      return THRIFT_ERR_CUDA;
+    attr_set = true;
+  }
+  cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
+  if (ev) cudaEventRecord(ev[0], st);
+  attn_decode_kernel<DT, GC><<<dim3(p.nsplit, Hkv, B), kDecThreads, DecLayout::SMEM_ALLOC, st>>>(p);
+  const thrift_status s = launch_status();
+  if (ev) cudaEventRecord(ev[1], st);
+  return s;
+}
+
+template <int DT>
+thrift_status decode_impl(const void* q, int B, int H, int Hkv, int capacity, const void* cache,
+                          const int32_t* seq_len, const float* kv_scale, float frac, int sink,
+                          int recent, int ss, void* out, float* lse, void* ws, cudaStream_t st) {
+  const DecWs w = carve_decode(ws, B, H, Hkv, capacity);
+  const CacheGeom cg = cache_geom(B, Hkv, capacity);
+  const int G = H / Hkv, nbcap = cg.ntc;
+  const uint16_t* qp = static_cast<const uint16_t*>(q);
+  if (cudaMemsetAsync(w.amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+  launch_amax<DT>(q, (int64_t)B * H * kDecD / 16, 0, w.amax, st);
+  if (ss)
+    dec_q_image_kernel<DT, true><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, w.q4, w.q16);
+  else
+    dec_q_image_kernel<DT, false><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, w.q4, w.q16);
+  const uint8_t* cp = static_cast<const uint8_t*>(cache);
+  dec_scores_kernel<DT><<<dim3((unsigned)ceil_div(nbcap, kDecScoreTiles), Hkv, B), 256, 0, st>>>(
+      qp, H, G, cg, cp, seq_len, capacity, nbcap, w.scores);
+  const size_t tsm = nbcap <= kTopkCache ? (size_t)nbcap * 8 : 0;
+  dec_topk_kernel<<<B * H, kTopkThreads, tsm, st>>>(w.scores, seq_len, capacity, H, nbcap, frac,
+                                                     sink, recent, w.mask);
+  thrift_status s = launch_status();
+  if (s != THRIFT_OK) return s;
+  DecParams p;
+  p.cache = cp;
+  p.cg = cg;
+  p.q4img = w.q4;
+  p.q16img = w.q16;
+  p.mask = w.mask;
+  p.seq_len = seq_len;
+  p.amax_q = w.amax;
+  p.kv_scale = kv_scale;
+  p.part_o = w.part_o;
+  p.part_ml = w.part_ml;
+  p.nbcap = nbcap;
+  p.capacity = capacity;
+  p.H = H;
+  p.G = G;
+  p.nsplit = decode_splits(B, Hkv, cg.ntc);
+  p.scale = (float)(1.4426950408889634 / std::sqrt((double)kDecD));
+  if (G <= 4) s = launch_decode_kernel<DT, 4>(p, B, Hkv, st);
+  else if (G <= 8) s = launch_decode_kernel<DT, 8>(p, B, Hkv, st);
+  else s = launch_decode_kernel<DT, 16>(p, B, Hkv, st);
+  if (s != THRIFT_OK) return s;
+  dec_combine_kernel<DT><<<B * H, kDecD, 0, st>>>(w.part_o, w.part_ml, 2 * p.nsplit,
+                                                  static_cast<uint16_t*>(out), lse);
+  return launch_status();
+}
+
 // Failure-detection aid: one thread waits, with the library's own bounded
 // waits, on something that never completes: an mbarrier that nothing arrives
 // on (mode 0) or a global word that nothing writes (mode 1).  The wait gives
@@ -654,6 +804,80 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
   return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
                       sink_blocks, recent_blocks, use_scalesearch, use_hadamard, out, lse, 1,
                       workspace, st);
+}
+
+size_t thrift_kv_cache_size(int B, int Hkv, int capacity, int d, int blk) {
+  thrift_status why;
+  if (B <= 0 || capacity <= 0 || !decode_shape_ok(Hkv, Hkv, d, blk, &why)) return 0;
+  return (size_t)cache_geom(B, Hkv, capacity).bytes();
+}
+
+thrift_status thrift_kv_cache_append(const void* k_new, const void* v_new, thrift_dtype dt, int B,
+                                     int Hkv, int d, int blk, int capacity,
+                                     const int32_t* cache_len, const int32_t* n_new, int max_new,
+                                     const float* kv_scale, int use_scalesearch, void* cache,
+                                     size_t cache_bytes, void* stream) {
+  thrift_status why;
+  if (!decode_shape_ok(Hkv, Hkv, d, blk, &why)) return why;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (B <= 0 || B > 65535 || capacity <= 0 || max_new < 0) return THRIFT_ERR_ARG;
+  if (!cache_len || !n_new || !kv_scale || !cache || !aligned16(cache)) return THRIFT_ERR_ARG;
+  if (cache_bytes < thrift_kv_cache_size(B, Hkv, capacity, d, blk)) return THRIFT_ERR_ARG;
+  if (max_new == 0) return THRIFT_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return THRIFT_ERR_ARG;
+  if (max_new > 0x7FFFFFFF / 2) return THRIFT_ERR_UNSUPPORTED;
+  const CacheGeom cg = cache_geom(B, Hkv, capacity);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* cp = static_cast<uint8_t*>(cache);
+  const bool ss = use_scalesearch != 0;
+  if (dt == THRIFT_BF16) {
+    if (ss) launch_kv_append<1, true>(k_new, v_new, cg, max_new, capacity, cache_len, n_new, kv_scale, cp, st);
+    else launch_kv_append<1, false>(k_new, v_new, cg, max_new, capacity, cache_len, n_new, kv_scale, cp, st);
+  } else {
+    if (ss) launch_kv_append<0, true>(k_new, v_new, cg, max_new, capacity, cache_len, n_new, kv_scale, cp, st);
+    else launch_kv_append<0, false>(k_new, v_new, cg, max_new, capacity, cache_len, n_new, kv_scale, cp, st);
+  }
+  return launch_status();
+}
+
+size_t thrift_attn_decode_workspace_size(int B, int H, int Hkv, int capacity, int d, int blk) {
+  thrift_status why;
+  if (B <= 0 || capacity <= 0 || !decode_shape_ok(H, Hkv, d, blk, &why)) return 0;
+  return carve_decode(nullptr, B, H, Hkv, capacity).bytes;
+}
+
+size_t thrift_attn_decode_mask_offset(int B, int H, int Hkv, int capacity, int d, int blk) {
+  thrift_status why;
+  if (B <= 0 || capacity <= 0 || !decode_shape_ok(H, Hkv, d, blk, &why)) return 0;
+  return (size_t)reinterpret_cast<uintptr_t>(carve_decode(nullptr, B, H, Hkv, capacity).mask);
+}
+
+thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, int Hkv, int d,
+                                 int blk, int capacity, const void* cache, size_t cache_bytes,
+                                 const int32_t* seq_len, const float* kv_scale, float topk_frac,
+                                 int sink_blocks, int recent_blocks, int use_scalesearch,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  thrift_status why;
+  if (!decode_shape_ok(H, Hkv, d, blk, &why)) return why;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (B <= 0 || B > 65535 || capacity <= 0) return THRIFT_ERR_ARG;
+  if (!(topk_frac >= 0.0f && topk_frac <= 1.0f) || sink_blocks < 0 || recent_blocks < 0)
+    return THRIFT_ERR_ARG;
+  if (!q || !cache || !seq_len || !kv_scale || !out || !lse || !workspace) return THRIFT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(out) || !aligned16(workspace))
+    return THRIFT_ERR_ARG;
+  if (cache_bytes < thrift_kv_cache_size(B, Hkv, capacity, d, blk)) return THRIFT_ERR_ARG;
+  if (ws_bytes < thrift_attn_decode_workspace_size(B, H, Hkv, capacity, d, blk))
+    return THRIFT_ERR_ARG;
+  if (ceil_div(cache_geom(B, Hkv, capacity).ntc, (int64_t)DecLayout::MAX_TILES / 2) > kDecMaxSplit)
+    return THRIFT_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == THRIFT_BF16)
+    return decode_impl<1>(q, B, H, Hkv, capacity, cache, seq_len, kv_scale, topk_frac,
+                          sink_blocks, recent_blocks, use_scalesearch, out, lse, workspace, st);
+  return decode_impl<0>(q, B, H, Hkv, capacity, cache, seq_len, kv_scale, topk_frac, sink_blocks,
+                        recent_blocks, use_scalesearch, out, lse, workspace, st);
 }
 
 }  // extern "C"

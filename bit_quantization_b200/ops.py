@@ -29,6 +29,8 @@ EXPORTS = (
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
     "thrift_attn_workspace_mask_offset",
     "thrift_kernel_timer_enable", "thrift_kernel_timer_read", "thrift_test_wait_timeout",
+    "thrift_kv_cache_size", "thrift_kv_cache_append", "thrift_attn_decode_workspace_size",
+    "thrift_attn_decode_mask_offset", "thrift_attn_decode",
 )
 
 
@@ -81,6 +83,18 @@ def lib():
         L.thrift_kernel_timer_read.argtypes = [P, P]
         L.thrift_test_wait_timeout.restype = i32
         L.thrift_test_wait_timeout.argtypes = [i32, i32, P]
+        L.thrift_kv_cache_size.restype = sz
+        L.thrift_kv_cache_size.argtypes = [i32] * 5
+        L.thrift_kv_cache_append.restype = i32
+        L.thrift_kv_cache_append.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, i32, P, i32,
+                                             P, sz, P]
+        L.thrift_attn_decode_workspace_size.restype = sz
+        L.thrift_attn_decode_workspace_size.argtypes = [i32] * 6
+        L.thrift_attn_decode_mask_offset.restype = sz
+        L.thrift_attn_decode_mask_offset.argtypes = [i32] * 6
+        L.thrift_attn_decode.restype = i32
+        L.thrift_attn_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, sz, P, P, f32,
+                                         i32, i32, i32, P, P, P, sz, P]
         _lib = L
     return _lib
 
@@ -310,4 +324,73 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
                                         int(recent_blocks), int(use_scalesearch),
                                         int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws),
                                         ws.numel(), _stream(q)), "thrift_attn_fwd_varlen")
+    return out, lse
+
+
+# ---------------------------------------------------------------- decode --
+
+def kv_cache_size(B, Hkv, capacity, d=128, blk=128) -> int:
+    return int(lib().thrift_kv_cache_size(B, Hkv, capacity, d, blk))
+
+
+def attn_decode_workspace_size(B, H, Hkv, capacity, d=128, blk=128) -> int:
+    return int(lib().thrift_attn_decode_workspace_size(B, H, Hkv, capacity, d, blk))
+
+
+def attn_decode_mask_offset(B, H, Hkv, capacity, d=128, blk=128) -> int:
+    return int(lib().thrift_attn_decode_mask_offset(B, H, Hkv, capacity, d, blk))
+
+
+class DoubleKVCache:
+    """The FP4 + 16-bit KV cache of ``B`` sequences (ThriftAttention decode):
+    one zero-filled device buffer in the library's format, the cached lengths
+    (int32, device) and the per-tensor scales (g_K, g_V) the NVFP4 part is
+    quantised with."""
+
+    def __init__(self, B, Hkv, capacity, kv_scale, dtype=torch.bfloat16, device="cuda",
+                 d=128, blk=128, use_scalesearch=False):
+        need = kv_cache_size(B, Hkv, capacity, d, blk)
+        if need == 0:
+            raise ThriftError("DoubleKVCache: unsupported shape")
+        self.B, self.Hkv, self.capacity, self.d, self.blk = B, Hkv, capacity, d, blk
+        self.dtype, self.use_scalesearch = dtype, use_scalesearch
+        self.buf = torch.zeros(need, dtype=torch.uint8, device=device)
+        self.lengths = torch.zeros(B, dtype=torch.int32, device=device)
+        self.kv_scale = torch.as_tensor(kv_scale, dtype=torch.float32, device=device).reshape(2)
+
+    def append(self, k_new, v_new, n_new=None):
+        """k_new, v_new [B, T, Hkv, d]; n_new int32 [B] (default: T each)."""
+        _need_cuda(k_new, v_new)
+        B, T, Hkv, d = k_new.shape
+        if n_new is None:
+            n_new = torch.full((B,), T, dtype=torch.int32, device=k_new.device)
+        _check(lib().thrift_kv_cache_append(_ptr(k_new), _ptr(v_new), _dt(k_new), B, Hkv, d,
+                                            self.blk, self.capacity, _ptr(self.lengths),
+                                            _ptr(n_new), T, _ptr(self.kv_scale),
+                                            int(self.use_scalesearch), _ptr(self.buf),
+                                            self.buf.numel(), _stream(k_new)),
+               "thrift_kv_cache_append")
+        self.lengths.add_(n_new)
+        self.lengths.clamp_(max=self.capacity)
+
+
+def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, recent_blocks=0,
+                       use_scalesearch=False, out=None, lse=None, workspace=None):
+    """q [B,H,d] -> (out [B,H,d], lse f32 [B,H]) against ``cache``."""
+    _need_cuda(q)
+    B, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = attn_decode_workspace_size(B, H, cache.Hkv, cache.capacity, d, cache.blk)
+    if need == 0:
+        raise ThriftError("thrift_attn_decode: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    _check(lib().thrift_attn_decode(_ptr(q), _dt(q), B, H, cache.Hkv, d, cache.blk,
+                                    cache.capacity, _ptr(cache.buf), cache.buf.numel(),
+                                    _ptr(cache.lengths), _ptr(cache.kv_scale), float(topk_frac),
+                                    int(sink_blocks), int(recent_blocks), int(use_scalesearch),
+                                    _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
+           "thrift_attn_decode")
     return out, lse

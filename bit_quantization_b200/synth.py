@@ -13,7 +13,12 @@ on; their datasets and model weights are not used):
   * K channel offsets: mu ~ 3 * randn(Hkv, d), added to K in fp32 before the
     cast and shared by every batch entry and token;
   * outlier channels (quantiser workload): 4 channels from ``randperm(cols)``
-    multiplied by 20 before the cast.
+    multiplied by 20 before the cast;
+  * decode (one query token per sequence against a cache): draw order
+    cached lengths (uniform on [lo, hi] unless given) -> K cache -> V cache
+    -> K channel offsets -> the step's query tokens; the cache tensors
+    [B, capacity, Hkv, d] are drawn whole, so tokens past a sequence's
+    length hold random values that a correct decode never reads.
 """
 from __future__ import annotations
 
@@ -53,6 +58,25 @@ class QuantWorkload:
     seed: int = 0
 
 
+@dataclass
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    capacity: int     # cache slots per sequence
+    lo: int           # cached lengths uniform on [lo, hi]
+    hi: int
+    d: int
+    dtype: torch.dtype
+    topk_frac: float
+    use_scalesearch: bool
+    k_offset_std: float = 3.0
+    sink_blocks: int = 0
+    recent_blocks: int = 0
+    seed: int = 0
+
+
 TINY = AttnWorkload("tiny_b1h1n256d64_fp16", 1, 1, 1, 256, 64, torch.float16, False, 64, 0.25,
                     False, False)
 QUANT = QuantWorkload("quant_65536x128_fp16_4outliers", 65536, 128, torch.float16, 4, 20.0)
@@ -63,6 +87,12 @@ C_GQA32K = AttnWorkload("b1h32hkv8n32768d128_bf16_causal_had_ss_top5", 1, 32, 8,
 C_VARLEN = AttnWorkload("varlen16_1k16k_h16d128_bf16_causal_had_ss", 16, 16, 16, 16384, 128,
                         torch.bfloat16, True, 128, 0.05, True, True, k_offset_std=3.0,
                         varlen={"nseq": 16, "lo": 1024, "hi": 16384})
+
+
+# Llama-3.1-8B attention shape (32 query heads, 8 kv heads, d = 128) at the
+# 131k context the pages quote decode at.
+C_DECODE131K = DecodeWorkload("decode_b4h32hkv8_ctx131072_bf16_top10", 4, 32, 8, 131072,
+                              131072, 131072, 128, torch.bfloat16, 0.10, False)
 
 
 def varlen_lengths(gen: torch.Generator, nseq: int, lo: int, hi: int):
@@ -94,6 +124,25 @@ def make_attn_inputs(w: AttnWorkload, seed: Optional[int] = None, lengths=None):
     cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
     return {"q": q.to(w.dtype), "k": k.to(w.dtype), "v": v.to(w.dtype), "cu_seqlens": cu,
             "lengths": list(lengths)}
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None, lengths=None,
+                       device="cpu"):
+    """Returns dict(q [B,H,d], k, v [B,capacity,Hkv,d], lengths (list)).
+    ``device`` = "cuda" draws on the GPU (for caches too large to move)."""
+    gen = torch.Generator(device=device).manual_seed(w.seed if seed is None else seed)
+    if lengths is None:
+        lengths = torch.randint(w.lo, w.hi + 1, (w.B,), generator=gen, device=device).tolist()
+    ks = (w.B, w.capacity, w.Hkv, w.d)
+    k = torch.randn(ks, generator=gen, dtype=torch.float32, device=device)
+    v = torch.randn(ks, generator=gen, dtype=torch.float32, device=device).to(w.dtype)
+    if w.k_offset_std:
+        mu = w.k_offset_std * torch.randn((w.Hkv, w.d), generator=gen, dtype=torch.float32,
+                                          device=device)
+        k += mu
+    k = k.to(w.dtype)
+    q = torch.randn((w.B, w.H, w.d), generator=gen, dtype=torch.float32, device=device)
+    return {"q": q.to(w.dtype), "k": k, "v": v, "lengths": list(lengths)}
 
 
 def make_quant_input(w: QuantWorkload, seed: Optional[int] = None):

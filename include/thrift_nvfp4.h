@@ -202,6 +202,75 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
 size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hkv, int d,
                                          int blk);
 
+/* -------------------------------------------------------------- decode --
+ * ThriftAttention decode over a double KV cache ("ThriftAttention",
+ * Resultados: decode speed-up; Significado: the KV cache grows by 28%
+ * because every token is kept in FP16 and in FP4).  One new query token per
+ * sequence attends to the len_b tokens cached for that sequence (its own key
+ * included: append it first).  Supported: d = 128, blk = 128, H % Hkv == 0,
+ * H / Hkv <= 16; other shapes return THRIFT_ERR_UNSUPPORTED.
+ *
+ * The cache is caller-owned device memory of thrift_kv_cache_size() bytes,
+ * ZERO-FILLED before its first use and before a sequence's slot is reused;
+ * its content is defined by this library.  Per (sequence b, kv head, key
+ * tile j of 128 tokens), in this order of regions, each region indexed by
+ * tile = (b * Hkv + hk) * ntile + j, ntile = ceil(capacity / 128):
+ *   K4   9216 B: NVFP4 K codes [128 tokens, 64 B] (byte 16i..16i+15 of a
+ *        row's 64 stored at chunk i XOR ((row / 2) mod 4)), then the UE4M3
+ *        scales of the 8 d-blocks in two 512-byte images (K-step s =
+ *        d-blocks 4s..4s+3: byte 512 s + (row mod 32) 16 + (row / 32) 4 +
+ *        (block mod 4));
+ *   V4   9216 B: the same for V^T: rows = channels, 16-token blocks along
+ *        the 128 tokens;
+ *   K16  32768 B: the 16-bit K rows, two 64-column regions [128, 128 B],
+ *        16-byte chunk i of a row at chunk i XOR (row mod 8);
+ *   V16  32768 B: the 16-bit V^T, the same with rows = channels;
+ *   MEAN 1024 B: fp64 mean over the cached tokens of the tile of each K
+ *        channel (tokens summed in order from the tile start).
+ * The 16-bit parts hold every cached value exactly; the NVFP4 parts are
+ * their quantisation under the caller's per-tensor scales g_K, g_V (V in
+ * 16-token blocks counted from token 0, the last block zero-padded).
+ *
+ * thrift_kv_cache_append: appends n_new[b] tokens (0 <= n_new[b] <=
+ * max_new) after cache_len[b] tokens of sequence b: k_new, v_new 16-bit
+ * [B, max_new, Hkv, 128] (token i of sequence b at [b, i]); cache_len,
+ * n_new int32 [B] on the device, read only (the caller advances its own
+ * lengths); kv_scale fp32 [2] on the device = (g_K, g_V).  Tokens that
+ * would land at or past `capacity` are dropped.  use_scalesearch as in
+ * nvfp4_quantize.  max_new = 0 launches nothing.  Appends to the same
+ * sequence must not overlap on the GPU.
+ *
+ * thrift_attn_decode: q 16-bit [B, H, 128]; seq_len int32 [B] on the
+ * device (tokens cached, clamped to [0, capacity]); kv_scale as above.
+ * The query tensor is quantised with g_Q = amax(q) / 2688 (use_scalesearch
+ * as in nvfp4_quantize); each (sequence, head) takes k = ceil(topk_frac *
+ * nb) of its nb = ceil(len / 128) key tiles on the FP16 path by the score
+ * q . kbar_j (fp64; ties to the lower tile), plus the first sink_blocks and
+ * the last recent_blocks tiles; the rest on the NVFP4 path; one online
+ * softmax (NVFP4 tiles, then FP16 tiles).
+ *   out 16-bit [B, H, 128] out;  lse fp32 [B, H] out (natural log; an
+ *   empty sequence gives a zero row and -inf).
+ * The workspace (thrift_attn_decode_workspace_size bytes, no initial
+ * content) also receives the selection, uint8 [B, H, ntile] (1 = FP16
+ * tile; tiles past a sequence's end 0) at thrift_attn_decode_mask_offset().
+ * Requirements: 0 <= topk_frac <= 1; sink_blocks, recent_blocks >= 0;
+ * capacity <= 32 * 512 * 128 tokens.  The kernel timer covers the decode
+ * attention kernel as well. */
+size_t thrift_kv_cache_size(int B, int Hkv, int capacity, int d, int blk);
+thrift_status thrift_kv_cache_append(const void* k_new, const void* v_new, thrift_dtype dt, int B,
+                                     int Hkv, int d, int blk, int capacity,
+                                     const int32_t* cache_len, const int32_t* n_new, int max_new,
+                                     const float* kv_scale, int use_scalesearch, void* cache,
+                                     size_t cache_bytes, void* stream);
+size_t thrift_attn_decode_workspace_size(int B, int H, int Hkv, int capacity, int d, int blk);
+size_t thrift_attn_decode_mask_offset(int B, int H, int Hkv, int capacity, int d, int blk);
+thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, int Hkv, int d,
+                                 int blk, int capacity, const void* cache, size_t cache_bytes,
+                                 const int32_t* seq_len, const float* kv_scale, float topk_frac,
+                                 int sink_blocks, int recent_blocks, int use_scalesearch,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
 /* ----------------------------------------------------- kernel timing --
  * Measurement aid (not part of the method).  While enabled, every
  * thrift_attn_fwd / thrift_attn_fwd_varlen call records a CUDA event pair on

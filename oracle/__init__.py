@@ -74,7 +74,7 @@ def lib():
         L.orc_attn_fp64.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, P, i64, i32, P, P]
         L.orc_thrift_decode.restype = i32
         L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
-                                        i32, i32, i32, P, i32, i32, P, P, P, P, P]
+                                        i32, i32, i32, P, i32, P, i32, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -326,13 +326,14 @@ def attn_fp64(q, k, v, dt, cu, causal, rows=None, nthreads=None):
 # ------------------------------------------------------------------ decode
 
 def thrift_decode(q, k, v, dt, lens, blk, g_kv, frac, use_ss=False, sink_blocks=0,
-                  recent_blocks=0, mask=None, nthreads=None):
+                  recent_blocks=0, mask=None, gq=None, nthreads=None):
     """One decode step over the double cache (reading R15 of oracle.cpp).
 
     q [B,H,d] uint16; k/v [B,ncap,Hkv,d] uint16 (token t of sequence b at
     [b, t]); lens int32 [B]; g_kv (g_K, g_V) floats.  Returns dict(out
     uint16 [B,H,d], out64 fp64 [B,H,d], tol fp64 [B,H,d], lse f32 [B,H],
-    mask uint8 [B,H,nbcap], gq)."""
+    mask uint8 [B,H,nbcap], gq).  ``gq``: optional given g_Q (for a sample
+    of the sequences of a larger step)."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, H, d = q.shape
     ncap, Hkv = k.shape[1], k.shape[2]
@@ -349,11 +350,14 @@ def thrift_decode(q, k, v, dt, lens, blk, g_kv, frac, use_ss=False, sink_blocks=
     out64 = np.zeros((B, H, d), np.float64)
     tol = np.zeros((B, H, d), np.float64)
     lse = np.full((B, H), np.nan, np.float32)
-    gq = np.zeros(1, np.float32)
+    gq_in = None if gq is None else np.array([gq], np.float32)
+    gq_out = np.zeros(1, np.float32)
     rc = lib().orc_thrift_decode(_p(q), _p(k), _p(v), dt, B, H, Hkv, ncap, d, blk, _p(lens),
                                  _p(gkv), float(frac), int(sink_blocks), int(recent_blocks),
-                                 int(use_ss), _p(m), given, int(nthreads or nthreads_default()),
-                                 _p(out), _p(lse), _p(gq), _p(out64), _p(tol))
+                                 int(use_ss), _p(m), given, _p(gq_in),
+                                 int(nthreads or nthreads_default()), _p(out), _p(lse),
+                                 _p(gq_out), _p(out64), _p(tol))
     if rc:
         raise ValueError("oracle thrift_decode: bad arguments")
-    return {"out": out, "out64": out64, "tol": tol, "lse": lse, "mask": m, "gq": float(gq[0])}
+    return {"out": out, "out64": out64, "tol": tol, "lse": lse, "mask": m,
+            "gq": float(gq_out[0])}

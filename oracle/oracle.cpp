@@ -1049,13 +1049,15 @@ static void decode_row(const DecCtx& C, int b, int h, uint16_t* out, float* lse,
 // Decode step over the double cache (reading R15).  g_kv: g_K, g_V.
 // mask [B, H, nbcap] (nbcap = ceil(ncap / blk)): read when mask_given, else
 // computed and written.  out 16-bit [B, H, d]; lse fp32 [B, H] (natural log;
-// -inf and a zero row for an empty sequence).  gq_out (optional) receives
-// g_Q; out64 / tol (optional) as in orc_thrift_attn.
+// -inf and a zero row for an empty sequence).  gq_in (optional) gives g_Q
+// (for a sample of the sequences of a larger step), else it is amax(q) /
+// 2688; gq_out (optional) receives it; out64 / tol (optional) as in
+// orc_thrift_attn.
 int orc_thrift_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int B,
                       int H, int Hkv, int ncap, int d, int blk, const int32_t* lens,
                       const float* g_kv, float frac, int sink, int recent, int use_ss,
-                      uint8_t* mask_io, int mask_given, int nthreads, uint16_t* out, float* lse,
-                      float* gq_out, double* out64, double* tol) {
+                      uint8_t* mask_io, int mask_given, const float* gq_in, int nthreads,
+                      uint16_t* out, float* lse, float* gq_out, double* out64, double* tol) {
   if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || ncap <= 0 || d % 16 || blk % 16 || blk <= 0)
     return -1;
   if (sink < 0 || recent < 0 || !(frac >= 0.0f && frac <= 1.0f)) return -1;
@@ -1067,7 +1069,12 @@ int orc_thrift_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
   C.lens = lens; C.q = q; C.k = k; C.v = v;
   C.gk = g_kv[0];
   C.gv = g_kv[1];
-  C.gq = quantize_rows_unpacked(q, dt, (int64_t)B * H, d, use_ss, 0, nthreads, C.qc, C.qs);
+  if (gq_in) {
+    C.gq = *gq_in;
+    quantize_rows_given(q, dt, (int64_t)B * H, d, C.gq, use_ss, nthreads, C.qc, C.qs);
+  } else {
+    C.gq = quantize_rows_unpacked(q, dt, (int64_t)B * H, d, use_ss, 0, nthreads, C.qc, C.qs);
+  }
   quantize_rows_given(k, dt, (int64_t)B * ncap * Hkv, d, C.gk, use_ss, nthreads, C.kc, C.ks);
   // V: per (sequence, kv head, channel) column of nbcap * blk tokens, 16-blocks
   // from token 0, tokens at or past len zero.

@@ -87,6 +87,35 @@ def test_bad_arguments_rejected_before_launch(L):
                              0, 0, dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
     assert L.block_mean_topk(dummy, dummy, 0, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, -2, dummy,
                              ws, 1 << 40, None) == ops.ERR_ARG
+    # decode: unsupported head dim / tile, too many heads per kv head, bad
+    # fraction, cache too small, workspace too small
+    big = 1 << 40
+    assert L.thrift_kv_cache_size(2, 4, 1024, 64, 128) == 0
+    assert L.thrift_kv_cache_size(2, 4, 1024, 128, 64) == 0
+    csz = L.thrift_kv_cache_size(2, 4, 1000, 128, 128)
+    assert csz == 2 * 4 * 8 * (9216 * 2 + 32768 * 2 + 1024)
+    assert L.thrift_attn_decode_workspace_size(2, 68, 4, 1024, 128, 128) == 0
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 4, 64, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(0.1), 0, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_UNSUPPORTED
+    assert L.thrift_attn_decode(dummy, 1, 2, 68, 4, 128, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(0.1), 0, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_UNSUPPORTED
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 3, 128, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(0.1), 0, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_ARG
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 4, 128, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(1.5), 0, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_ARG
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 4, 128, 128, 1024, dummy, 4096, dummy, dummy,
+                                C.c_float(0.1), 0, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_ARG
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 4, 128, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(0.1), 0, 0, 0, dummy, dummy, ws, 4096, None) == ops.ERR_ARG
+    assert L.thrift_attn_decode(dummy, 1, 2, 8, 4, 128, 128, 1024, dummy, big, dummy, dummy,
+                                C.c_float(0.1), -1, 0, 0, dummy, dummy, ws, big, None) == ops.ERR_ARG
+    assert L.thrift_kv_cache_append(dummy, dummy, 1, 2, 4, 128, 128, 1024, dummy, dummy, 4,
+                                    dummy, 0, dummy, 16, None) == ops.ERR_ARG
+    assert L.thrift_kv_cache_append(dummy, dummy, 1, 2, 4, 128, 128, 1024, dummy, dummy, -1,
+                                    dummy, 0, dummy, big, None) == ops.ERR_ARG
+    # nothing to append: accepted without a launch
+    assert L.thrift_kv_cache_append(None, None, 1, 2, 4, 128, 128, 1024, dummy, dummy, 0,
+                                    dummy, 0, dummy, big, None) == ops.OK
     # failure-detection aid: unknown mode, limits outside 1 us .. 1 s
     assert L.thrift_test_wait_timeout(2, 1000, None) == ops.ERR_ARG
     assert L.thrift_test_wait_timeout(0, 0, None) == ops.ERR_ARG

@@ -66,6 +66,9 @@ def test_decode_equals_prefill_last_row(orc, frac, sink, recent):
     g_kv = (orc.tensor_scale(K.reshape(-1, d), BF16), orc.tensor_scale(V.reshape(-1, d), BF16))
     dec = orc.thrift_decode(q, k, v, BF16, lens, blk, g_kv, frac, sink_blocks=sink,
                             recent_blocks=recent)
+    again = orc.thrift_decode(q, k, v, BF16, lens, blk, g_kv, frac, sink_blocks=sink,
+                              recent_blocks=recent, gq=dec["gq"])
+    assert np.array_equal(again["out64"], dec["out64"])  # g_Q given = g_Q derived
     o64, lse, tol, g = _prefill_last_rows(orc, q, k, v, lens, blk, dec["mask"])
     assert g[1] == g_kv[0] and g[2] == g_kv[1] and g[0] == dec["gq"]
     assert np.array_equal(dec["out64"], o64)
