@@ -304,11 +304,11 @@ struct DecLayout {
   static constexpr uint32_t P16B = 64 * kDecTile * 2;                 // 16384
   static constexpr uint32_t STG4 = CacheGeom::K4 + CacheGeom::V4;     // 18432
   static constexpr uint32_t STG16 = CacheGeom::K16 + CacheGeom::V16;  // 65536
-  //   NVFP4 view: Q4 | P4 x2 | NS4 stages (K4 + V4)
-  //   FP16 view:  Q16 | P16 x2 | NS16 stages (K16 + V16)
+  //   NVFP4 view: Q4 | P4 x4 (two per group) | NS4 stages (K4 + V4)
+  //   FP16 view:  Q16 | P16 x2 (one per group) | NS16 stages (K16 + V16)
   static constexpr uint32_t OFF4_Q = 0;
   static constexpr uint32_t OFF4_P = dec_align(kDecQ4Bytes);
-  static constexpr uint32_t OFF4_STG = OFF4_P + 2 * dec_align(P4B);
+  static constexpr uint32_t OFF4_STG = OFF4_P + 4 * dec_align(P4B);  // two slots per group
   static constexpr uint32_t OFF16_Q = 0;
   static constexpr uint32_t OFF16_P = dec_align(kDecQ16Bytes);
   static constexpr uint32_t OFF16_STG = OFF16_P + 2 * P16B;
@@ -326,20 +326,27 @@ struct DecLayout {
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
   // tensor-memory columns
   static constexpr uint32_t T_S = 0;      // + 64 g
-  static constexpr uint32_t T_O = 128;    // + 64 g
-  static constexpr uint32_t T_QSF = 256;  // + 8 g (two K-steps of 4 columns)
-  static constexpr uint32_t T_KSF = 272;  // + 8 g
-  static constexpr uint32_t T_PSF = 288;  // + 8 g
-  static constexpr uint32_t T_VSF = 304;  // + 8 g
+  static constexpr uint32_t T_O = 128;    // + 64 (2 g + slot)
+  static constexpr uint32_t T_QSF = 384;  // + 8 g (two K-steps of 4 columns)
+  static constexpr uint32_t T_KSF = 400;  // + 8 g
+  static constexpr uint32_t T_PSF = 416;  // + 8 g
+  static constexpr uint32_t T_VSF = 432;  // + 8 g
   static_assert(NS4 == 8, "barrier plan assumes eight NVFP4 stages");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// Barriers.  Per group g: SF/SE its S buffer full (QK commit) / read;
+// GB the group's own barrier (one phase per tile).  Per group g and slot s
+// (tile t of the group uses slot (t >> 1) & 1): PF its P tile written, OD
+// its PV retired into O buffer s, OE O buffer s folded (free again).  A
+// barrier of a slot only completes its next phase after its waiter has
+// passed the previous one: the slot's next PV waits OE, whose fold waited
+// OD; the slot's next P waits for that fold (or for OD, FP16).
 enum : int {
-  D_Q4 = 0, D_Q16 = 1, D_SF = 2 /* 2,3 */, D_SE = 4 /* 4,5 */, D_PF = 6 /* 6,7 */,
-  D_OD = 8 /* 8,9 */, D_OE = 10 /* 10,11 */, D_GB = 12 /* 12,13 */, D_P4DONE = 14,
-  D_DONE = 15, D_KVF16 = 16 /* 16,17 */, D_KVE16 = 18 /* 18,19 */, D_KVF4 = 20 /* 20..27 */,
-  D_KVE4 = 28 /* 28..35 */, D_N = 36
+  D_Q4 = 0, D_Q16 = 1, D_SF = 2 /* 2,3 */, D_SE = 4 /* 4,5 */, D_PF = 6 /* 6..9 */,
+  D_OD = 10 /* 10..13 */, D_OE = 14 /* 14..17 */, D_GB = 18 /* 18,19 */, D_P4DONE = 20,
+  D_DONE = 21, D_KVF16 = 22 /* 22,23 */, D_KVE16 = 24 /* 24,25 */, D_KVF4 = 26 /* 26..33 */,
+  D_KVE4 = 34 /* 34..41 */, D_N = 42
 };
 
 // warps 0..7 softmax (two groups), 8 producer, 9 + g the QK^T issuer of
@@ -386,8 +393,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
   if (tid == 0) {
     for (int i = 0; i < D_N; ++i) {
       uint32_t cnt = 1;
-      if ((i >= D_SE && i < D_SE + 2) || (i >= D_PF && i < D_PF + 2) ||
-          (i >= D_OE && i < D_OE + 2) || (i >= D_GB && i < D_GB + 2))
+      if ((i >= D_SE && i < D_SE + 2) || (i >= D_PF && i < D_PF + 4) ||
+          (i >= D_OE && i < D_OE + 4) || (i >= D_GB && i < D_GB + 2))
         cnt = 128;
       if (i == D_DONE) cnt = 4;     // one commit per MMA issuer
       if (i == D_P4DONE) cnt = 2;   // one commit per PV issuer
@@ -577,13 +584,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
           int sl, par;
           stage_of(t, sl, par);
           uint64_t* empty = f16 ? &bars[D_KVE16 + sl] : &bars[D_KVE4 + sl];
-          if (!mbar_wait(&bars[D_PF + g], u & 1, s_abort)) { ok = false; break; }
-          if (u >= 1 && !mbar_wait(&bars[D_OE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+          const int sl2 = u & 1, use = u >> 1;  // P / O slot and its use count
+          if (!mbar_wait(&bars[D_PF + 2 * g + sl2], use & 1, s_abort)) { ok = false; break; }
+          if (use >= 1 && !mbar_wait(&bars[D_OE + 2 * g + sl2], (use - 1) & 1, s_abort)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t dO = tmem + L::T_O + 64 * g;
+          const uint32_t dO = tmem + L::T_O + 64 * (2 * g + sl2);
           if (!f16) {
             const uint32_t stg = L::OFF4_STG + sl * L::STG4 + CacheGeom::K4;
-            const uint32_t pp = L::OFF4_P + g * dec_align(L::P4B);
+            const uint32_t pp = L::OFF4_P + (2 * g + sl2) * dec_align(L::P4B);
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
               tc_cp_32x128b_x4(vsf + 4 * s2, d_sf + ((stg + kDecD * (kDecTile / 2) + 512 * s2) >> 4));
@@ -601,7 +612,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
               mma_f16(dO, d16 + ((stg + (kk / 4) * 128 * 128) >> 4) + 2 * (kk % 4),
                       d16 + ((pp + (kk / 4) * 64 * 128) >> 4) + 2 * (kk % 4), id16, kk > 0);
           }
-          tc_commit(&bars[D_OD + g]);
+          tc_commit(&bars[D_OD + 2 * g + sl2]);
           tc_commit(empty);
           if (!p4_signalled && t + 2 >= n4) {
             tc_commit(&bars[D_P4DONE]);
@@ -625,8 +636,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     float* coef = reinterpret_cast<float*>(sm + L::OFF_COEF) + g * (2 * kDecMaxG * 2);
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_addr = lane_base + L::T_S + 64 * g;
-    const uint32_t o_addr = lane_base + L::T_O + 64 * g;
-    uint8_t* p4 = sm + L::OFF4_P + g * dec_align(L::P4B);
+    const uint32_t o_addr = lane_base + L::T_O + 64 * (2 * g);  // + 64 slot
+    uint8_t* p4g = sm + L::OFF4_P + 2 * g * dec_align(L::P4B);   // + slot * P4 slot
     uint8_t* p16 = sm + L::OFF16_P + g * L::P16B;
     // work item of this thread: block bb of head c
     const int c = i >> 3, bb = i & 7;
@@ -641,11 +652,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     // query image the producer loads at once when there is no NVFP4 tile:
     // the NVFP4 slot is only touched when that phase exists.
     if (n4 > 0) {
-      for (int e = i; e < (64 - GC) * 4; e += 128)
-        *reinterpret_cast<uint4*>(p4 + (GC + e / 4) * 64 + (e % 4) * 16) = make_uint4(0, 0, 0, 0);
-      for (int e = i; e < (64 - GC) * 8; e += 128)
-        p4[64 * (kDecTile / 2) + sf_offset(GC + e / 8, e % 8)] = 0;
+      for (int sl2 = 0; sl2 < 2; ++sl2) {
+        uint8_t* p4 = p4g + sl2 * dec_align(L::P4B);
+        for (int e = i; e < (64 - GC) * 4; e += 128)
+          *reinterpret_cast<uint4*>(p4 + (GC + e / 4) * 64 + (e % 4) * 16) = make_uint4(0, 0, 0, 0);
+        for (int e = i; e < (64 - GC) * 8; e += 128)
+          p4[64 * (kDecTile / 2) + sf_offset(GC + e / 8, e % 8)] = 0;
+      }
     }
+    // fold of the group's tile with use count v (slot v & 1): wait for its
+    // PV, add it to the running output with the coefficients its owners
+    // wrote, free the O buffer
+    auto fold = [&](int v) -> bool {
+      const int sl2 = v & 1;
+      if (!warp_wait(&bars[D_OD + 2 * g + sl2], (v >> 1) & 1, s_abort)) return false;
+      tc_fence_after();
+      float o[GC];
+      tmem_ld_cols<GC>(o_addr + 64 * sl2, o);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[D_OE + 2 * g + sl2]);
+      const float* cf = coef + sl2 * (kDecMaxG * 2);
+#pragma unroll
+      for (int k = 0; k < GC; ++k) orun[k] = fmaf(cf[2 * k], orun[k], cf[2 * k + 1] * o[k]);
+      return true;
+    };
     bool p16_ready = false;
     bool ok = true;
     int u_last = -1;
@@ -665,16 +696,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
         p16_ready = true;
       }
       float* sT = sT0 + (u & 1) * (L::ST_BYTES / 4);
-      // A: scores of key i for the group's heads -> transposed tile, and
-      // PV(t - 2) (channel i) into registers, both in one TMEM round trip
+      // A: scores of key i for the group's heads -> transposed tile
       if (!warp_wait(&bars[D_SF + g], u & 1, s_abort)) { ok = false; break; }
-      if (u >= 1 && !warp_wait(&bars[D_OD + g], (u - 1) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
-      float o[GC];
       {
         float a[GC];
         tmem_ld_cols<GC>(s_addr, a);
-        if (u >= 1) tmem_ld_cols<GC>(o_addr, o);
         tmem_ld_wait();
         const bool valid = j * kDecTile + i < len;
 #pragma unroll
@@ -682,16 +709,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       }
       tc_fence_before();
       mbar_arrive(&bars[D_SE + g]);
-      if (u >= 1) mbar_arrive(&bars[D_OE + g]);
       mbar_arrive(&bars[D_GB + g]);
       if (!warp_wait(&bars[D_GB + g], u & 1, s_abort)) { ok = false; break; }
-      // E: fold PV(t - 2) into the running output (its coefficients were
-      // written before the barrier)
-      if (u >= 1) {
-        const float* cf = coef + ((u - 1) & 1) * (kDecMaxG * 2);
-#pragma unroll
-        for (int k = 0; k < GC; ++k) orun[k] = fmaf(cf[2 * k], orun[k], cf[2 * k + 1] * o[k]);
+      // the single FP16 P buffer was last read by PV(t - 2)
+      if (f16 && u >= 1 &&
+          !warp_wait(&bars[D_OD + 2 * g + ((u - 1) & 1)], ((u - 1) >> 1) & 1, s_abort)) {
+        ok = false;
+        break;
       }
+      uint8_t* p4 = p4g + (u & 1) * dec_align(L::P4B);
       // C: probabilities of block bb of head c
       if (has_item) {
         float x[16];
@@ -795,7 +821,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       }
       // D: P(t) is in shared memory
       fence_proxy_async_smem();
-      mbar_arrive(&bars[D_PF + g]);
+      mbar_arrive(&bars[D_PF + 2 * g + (u & 1)]);
+      // E: fold PV(t - 2), now off the path from S(t) to P(t) (its
+      // coefficients were written before this tile's barrier)
+      if (u >= 1 && !fold(u - 1)) { ok = false; break; }
       u_last = u;
     }
     // the group's last PV, folded once every owner lane has written the
@@ -803,16 +832,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     if (ok && u_last >= 0) {
       mbar_arrive(&bars[D_GB + g]);
       ok = warp_wait(&bars[D_GB + g], (u_last + 1) & 1, s_abort);
-      if (ok) ok = warp_wait(&bars[D_OD + g], u_last & 1, s_abort);
-      if (ok) {
-        tc_fence_after();
-        float o[GC];
-        tmem_ld_cols<GC>(o_addr, o);
-        tmem_ld_wait();
-        const float* cf = coef + (u_last & 1) * (kDecMaxG * 2);
-#pragma unroll
-        for (int k = 0; k < GC; ++k) orun[k] = fmaf(cf[2 * k], orun[k], cf[2 * k + 1] * o[k]);
-      }
+      if (ok) ok = fold(u_last);
     }
     if (ok) {
       // this group's split: output relative to its running max, m and l
