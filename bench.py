@@ -9,12 +9,17 @@ Default workload: B=2, H=32, N=8192, d=128, bf16, non-causal, 128x128 blocks,
 10% FP16 pairs, K with per-channel offsets N(0, 3).  Its inputs (3 x 134 MB)
 exceed L2, so no flush is needed between steps.
 
+The line also carries "decode": one decode step of the double-cache decode
+path (Llama-3.1-8B attention shape, B=4, 131072 cached tokens, 10% FP16
+tiles): append the step's token, then attend; its kernel against HBM.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference   # the CPU oracle on a bounded sample
 Multi-GPU (weak scaling, independent problems per rank, no collective on the
 data path): launched by torch.distributed.run, one rank per GPU.
 """
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -291,6 +296,118 @@ def quantizer_only(args):
     return 0
 
 
+DECODE_KERNELS_PER_STEP = 8  # append (2), absmax, query images, scores, top-k, decode, merge
+
+
+def decode_setup(ops, dev, w, context=None):
+    """The decode workload's cache filled on the GPU: (cache, q, k_new,
+    v_new, L0, workspace, kv scales).  ``context`` overrides the cached
+    length (profiling on a smaller case)."""
+    if context is not None:
+        w = dataclasses.replace(w, capacity=context + 128, lo=context, hi=context)
+    inp = synth.make_decode_inputs(w, device=dev)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    L0 = inp["lengths"][0]
+    # the cache's per-tensor scales: the library's own quantiser over the
+    # cached tokens (g = amax / 2688, reading R1)
+    kv = torch.stack([ops.nvfp4_quantize(k[:, :L0].reshape(-1, w.d))[2].reshape(()),
+                      ops.nvfp4_quantize(v[:, :L0].reshape(-1, w.d))[2].reshape(())])
+    cache = ops.DoubleKVCache(w.B, w.Hkv, w.capacity, kv, dtype=w.dtype)
+    for t0 in range(0, L0, 32768):
+        t1 = min(L0, t0 + 32768)
+        cache.append(k[:, t0:t1].contiguous(), v[:, t0:t1].contiguous())
+    k_new = k[:, L0:L0 + 1].contiguous()
+    v_new = v[:, L0:L0 + 1].contiguous()
+    del k, v, inp
+    ws = torch.empty(ops.attn_decode_workspace_size(w.B, w.H, w.Hkv, w.capacity), dtype=torch.uint8,
+                     device=dev)
+    return w, cache, q, k_new, v_new, L0, ws
+
+
+def decode_line(ops, dev, peaks, steps=50, warmup=5):
+    """One decode step of the decode workload (Llama-3.1-8B attention shape,
+    131072 cached tokens per sequence): append the step's token to every
+    sequence's double cache, then attend.  The cached length is reset before
+    each step, so every step appends at the same position and attends over
+    131073 tokens."""
+    w, cache, q, k_new, v_new, L0, ws = decode_setup(ops, dev, synth.C_DECODE131K)
+    base = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
+
+    def step():
+        cache.lengths.copy_(base)
+        cache.append(k_new, v_new)
+        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, out=out, lse=lse, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the decode warm-up")
+    ops.kernel_timer_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    kms, nk = ops.kernel_timer_read()
+    ops.kernel_timer_enable(False)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the decode loop")
+    step_us = 1e3 * e0.elapsed_time(e1) / steps
+    k_us = 1e3 * kms / max(nk, 1)
+    # key tiles the decode kernel reads: per (sequence, kv head), every tile
+    # some query head takes in NVFP4 (K4 + V4 = 18432 B) and every tile some
+    # head takes in FP16 (K16 + V16 = 65536 B)
+    nbcap = (w.capacity + 127) // 128
+    mo = ops.attn_decode_mask_offset(w.B, w.H, w.Hkv, w.capacity)
+    G = w.H // w.Hkv
+    mask = ws[mo:mo + w.B * w.H * nbcap].view(w.B, w.Hkv, G, nbcap).bool()
+    nb = (L0 + 1 + 127) // 128
+    mask = mask[..., :nb]
+    t16 = int(mask.any(dim=2).sum())
+    t4 = int((~mask.all(dim=2)).sum())
+    kv_bytes = t4 * 18432 + t16 * 65536
+    achieved = kv_bytes / (k_us * 1e-6) / 1e9
+    hbm = peaks["hbm_gbs"]
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "d": w.d,
+            "cached_tokens": L0, "attended_tokens": L0 + 1, "topk_frac": w.topk_frac,
+            "us_per_step": step_us, "steps": steps,
+            "step": "append one token per sequence to the FP4 + 16-bit cache, then attend",
+            "kernel_us": k_us, "tiles_nvfp4": t4, "tiles_fp16": t16,
+            "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "algorithmic_bytes": kv_bytes},
+            "kernels_per_step": DECODE_KERNELS_PER_STEP}
+
+
+def decode_only(args):
+    """A few decode steps (profiling aid); ``--decode-context`` sets the
+    cached length."""
+    from bit_quantization_b200 import ops
+    dev = torch.device("cuda", 0)
+    w, cache, q, k_new, v_new, L0, ws = decode_setup(ops, dev, synth.C_DECODE131K,
+                                                   args.decode_context)
+    base = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    times = []
+    for _ in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cache.lengths.copy_(base)
+        e0.record()
+        cache.append(k_new, v_new)
+        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        times.append(1e3 * e0.elapsed_time(e1))
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out")
+    print(json.dumps({"mode": "decode", "workload": w.name, "cached_tokens": L0,
+                      "us_min": min(times[args.warmup:])}))
+    return 0
+
+
 def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20):
     """Average attention-kernel time of the bench workload run with another
     selection (CUDA events around each attention launch)."""
@@ -363,8 +480,11 @@ def main():
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantizer", action="store_true")
-    ap.add_argument("--mode", default="attention", choices=["attention", "quantizer"],
-                    help="quantizer: only a few plain quantiser calls (profiling aid)")
+    ap.add_argument("--mode", default="attention", choices=["attention", "quantizer", "decode"],
+                    help="quantizer / decode: only a few plain calls of that path (profiling aid)")
+    ap.add_argument("--decode-context", type=int, default=None,
+                    help="cached tokens per sequence in --mode decode (default: the workload's)")
+    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
@@ -372,6 +492,8 @@ def main():
         return run_reference(args, w)
     if args.mode == "quantizer":
         return quantizer_only(args)
+    if args.mode == "decode":
+        return decode_only(args)
 
     from bit_quantization_b200 import ops
     world, rank, local = dist_setup(args)
@@ -537,6 +659,10 @@ def main():
         line["sink_aware"] = sink_line(ops, q, k, v, w, inp, out, lse, ws, p16)
     if rank == 0 and world == 1 and not args.no_quantizer:
         line["quantizer"] = quantizer_line(dev, peaks)
+    if rank == 0 and world == 1 and not args.no_decode:
+        del qd, kd, vd, od, ld
+        torch.cuda.empty_cache()
+        line["decode"] = decode_line(ops, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
         dt, fl, desc = oracle_sample(w, args.ref_units, cores, inp)

@@ -299,6 +299,33 @@ __global__ void __launch_bounds__(kDecD) dec_combine_kernel(const float* __restr
 
 __host__ __device__ constexpr uint32_t dec_align(uint32_t x) { return (x + 1023u) & ~1023u; }
 
+// Sum of N values by a pairwise tree.
+template <int N>
+__device__ __forceinline__ float tree_sum(const float* x) {
+  float y[N];
+#pragma unroll
+  for (int e = 0; e < N; ++e) y[e] = x[e];
+#pragma unroll
+  for (int w = N / 2; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int e = 0; e < w; ++e) y[e] += y[e + w];
+  }
+  return y[0];
+}
+
+// Four fp32 values -> four E2M1 codes in the low 16 bits (value 2i in the
+// low nibble of byte i), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e2m1x4(const float* x) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
+      : "=r"(out)
+      : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]));
+  return out;
+}
+
 struct DecLayout {
   static constexpr uint32_t P4B = fp4_tile_bytes(64, kDecTile);       // 5120
   static constexpr uint32_t P16B = 64 * kDecTile * 2;                 // 16384
@@ -639,11 +666,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     const uint32_t o_addr = lane_base + L::T_O + 64 * (2 * g);  // + 64 slot
     uint8_t* p4g = sm + L::OFF4_P + 2 * g * dec_align(L::P4B);   // + slot * P4 slot
     uint8_t* p16 = sm + L::OFF16_P + g * L::P16B;
-    // work item of this thread: block bb of head c
-    const int c = i >> 3, bb = i & 7;
-    const bool has_item = i < 8 * GC;  // uniform over each warp
-    const int own = lane & ~7;
-    float m = -INFINITY, l = 0.0f;  // running state of head c (owner lanes, bb == 0)
+    // work item of this thread: keys [16 bb + KPL hb, + KPL) of head c, the
+    // LPB lanes of a 16-key block and the eight blocks of a head adjacent
+    constexpr int LPB = GC >= 16 ? 1 : (GC >= 8 ? 2 : 4);  // lanes per 16-key block
+    constexpr int KPL = 16 / LPB;                          // keys per lane
+    const int c = i / (8 * LPB), bb = (i / LPB) % 8, hb = i % LPB;
+    const bool has_item = i < 8 * LPB * GC;  // uniform over each warp
+    const int own = lane & ~(8 * LPB - 1);
+    const bool is_owner = (i % (8 * LPB)) == 0;
+    float m = -INFINITY, l = 0.0f;  // running state of head c (owner lanes)
     float orun[GC];
 #pragma unroll
     for (int k = 0; k < GC; ++k) orun[k] = 0.0f;
@@ -718,12 +749,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
         break;
       }
       uint8_t* p4 = p4g + (u & 1) * dec_align(L::P4B);
-      // C: probabilities of block bb of head c
+      // C: probabilities of keys [16 bb + KPL hb, + KPL) of head c
       if (has_item) {
-        float x[16];
-        const float4* src = reinterpret_cast<const float4*>(sT + c * L::ST_PITCH + 16 * bb);
+        float x[KPL];
+        const float4* src =
+            reinterpret_cast<const float4*>(sT + c * L::ST_PITCH + 16 * bb + KPL * hb);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < KPL / 4; ++q) {
           const float4 v4 = src[q];
           x[4 * q] = v4.x;
           x[4 * q + 1] = v4.y;
@@ -732,16 +764,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
         }
         float bm = x[0];
 #pragma unroll
-        for (int e = 1; e < 16; ++e) bm = fmaxf(bm, x[e]);
+        for (int e = 1; e < KPL; ++e) bm = fmaxf(bm, x[e]);
+#pragma unroll
+        for (int o = 1; o < LPB; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
         float mt_raw = bm;
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) mt_raw = fmaxf(mt_raw, __shfl_xor_sync(0xffffffffu, mt_raw, o));
+        for (int o = LPB; o < 8 * LPB; o <<= 1)
+          mt_raw = fmaxf(mt_raw, __shfl_xor_sync(0xffffffffu, mt_raw, o));
         const bool active = c < G && (((bits >> c) & 1u) != 0) == f16;
         const float m_old = __shfl_sync(0xffffffffu, m, own);
-        float alpha = 1.0f, sigma = 0.0f;
+        float alpha = 1.0f, sigma = 0.0f, ls = 0.0f;
         if (!f16) {
-          uint32_t lo = 0, hi = 0, S = 0;
-          float ls = 0.0f;
+          uint32_t S = 0;
+          uint32_t code[KPL / 8 > 0 ? KPL / 8 : 1] = {};
+          uint32_t code4 = 0;  // KPL == 4: two bytes
           bool drop = false;
           if (active) {
             const float mt = mt_raw * cs4;
@@ -751,15 +787,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             const float dec = ue4m3_decode_fast(S);
             const float cc = S ? 11.392317422778760f - mt - lg2_ftz(dec) : -INFINITY;  // log2(2688)
 #pragma unroll
-            for (int e2 = 0; e2 < 16; e2 += 2) fma2(x[e2], x[e2 + 1], x[e2], x[e2 + 1], cs4, cs4, cc, cc);
+            for (int e2 = 0; e2 < KPL; e2 += 2) fma2(x[e2], x[e2 + 1], x[e2], x[e2 + 1], cs4, cs4, cc, cc);
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) x[e2] = ex2_ftz(x[e2]);  // masked (-inf) -> 0
-            float sum = 0.0f;
+            for (int e2 = 0; e2 < KPL; ++e2) x[e2] = ex2_ftz(x[e2]);  // masked (-inf) -> 0
+            ls = tree_sum<KPL>(x) * dec;
+            if constexpr (KPL >= 8) {
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) sum += x[e2];
-            ls = sum * dec;
-            lo = e2m1x8(x);
-            hi = e2m1x8(x + 8);
+              for (int q = 0; q < KPL / 8; ++q) code[q] = e2m1x8(x + 8 * q);
+            } else {
+              code4 = e2m1x4(x);
+            }
             const float rowmax = ex2_ftz(mt - m_new);
             float sigma_raw = rowmax >= 8.6736174e-19f ? rowmax * (1.0f / 2688.0f) : 0.0f;  // 2^-60
             sigma = sigma_raw * gv;
@@ -767,53 +804,60 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             drop = sigma == 0.0f;
             alpha = m_old == -INFINITY ? 0.0f : ex2_ftz(m_old - m_new);
 #pragma unroll
-            for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-            if (bb == 0) {
+            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            if (is_owner) {
               l = fmaf(ls, sigma_raw, alpha * l);
               m = m_new;
             }
           } else {
 #pragma unroll
-            for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
           }
-          *reinterpret_cast<uint2*>(p4 + swz_offset(c, 8 * bb, kDecTile / 2)) = make_uint2(lo, hi);
-          p4[64 * (kDecTile / 2) + sf_offset(c, bb)] = drop ? 0 : (uint8_t)S;
+          uint8_t* dst = p4 + swz_offset(c, 8 * bb + (KPL / 2) * hb, kDecTile / 2);
+          if constexpr (KPL == 16) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(code[0], code[1]);
+          } else if constexpr (KPL == 8) {
+            *reinterpret_cast<uint32_t*>(dst) = code[0];
+          } else {
+            *reinterpret_cast<uint16_t*>(dst) = (uint16_t)code4;
+          }
+          if (hb == 0) p4[64 * (kDecTile / 2) + sf_offset(c, bb)] = drop ? 0 : (uint8_t)S;
         } else {
-          uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-          float ls = 0.0f;
+          uint32_t w[KPL / 2] = {};
           if (active) {
             const float mt = mt_raw * cs16;
             const float m_new = fmaxf(m_old, mt);
             const float negm = -m_new;
 #pragma unroll
-            for (int e2 = 0; e2 < 16; e2 += 2)
+            for (int e2 = 0; e2 < KPL; e2 += 2)
               fma2(x[e2], x[e2 + 1], x[e2], x[e2 + 1], cs16, cs16, negm, negm);
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) x[e2] = ex2_ftz(x[e2]);
+            for (int e2 = 0; e2 < KPL; ++e2) x[e2] = ex2_ftz(x[e2]);
+            ls = tree_sum<KPL>(x);
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) ls += x[e2];
-#pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2) w[e2] = pack2<DT>(x[2 * e2], x[2 * e2 + 1]);
+            for (int e2 = 0; e2 < KPL / 2; ++e2) w[e2] = pack2<DT>(x[2 * e2], x[2 * e2 + 1]);
             alpha = m_old == -INFINITY ? 0.0f : ex2_ftz(m_old - m_new);
             sigma = 1.0f;
 #pragma unroll
-            for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-            if (bb == 0) {
+            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            if (is_owner) {
               l = fmaf(alpha, l, ls);
               m = m_new;
             }
           } else {
 #pragma unroll
-            for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
           }
-          const uint32_t k0 = 16 * bb;
+          const uint32_t k0 = 16 * bb + KPL * hb;
           uint8_t* reg = p16 + (k0 / 64) * (64 * 128);
-          *reinterpret_cast<uint4*>(reg + swz_offset(c, (k0 % 64) * 2, 128)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(reg + swz_offset(c, (k0 % 64) * 2 + 16, 128)) =
-              make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+          for (int q = 0; q < KPL / 8; ++q)
+            *reinterpret_cast<uint4*>(reg + swz_offset(c, (k0 % 64) * 2 + 16 * q, 128)) =
+                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          if constexpr (KPL == 4)
+            *reinterpret_cast<uint2*>(reg + swz_offset(c, (k0 % 64) * 2, 128)) = make_uint2(w[0], w[1]);
         }
-        if (bb == 0) {
+        if (is_owner) {
           float* cf = coef + (u & 1) * (kDecMaxG * 2);
           cf[2 * c] = alpha;
           cf[2 * c + 1] = sigma;
@@ -841,7 +885,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
 #pragma unroll
       for (int k = 0; k < GC; ++k)
         if (k < G) p.part_o[((row0 + k) * ns + sidx) * kDecD + i] = orun[k];
-      if (has_item && bb == 0 && c < G) {
+      if (has_item && is_owner && c < G) {
         p.part_ml[((row0 + c) * ns + sidx) * 2] = m;
         p.part_ml[((row0 + c) * ns + sidx) * 2 + 1] = l;
       }

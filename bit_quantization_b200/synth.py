@@ -91,7 +91,8 @@ C_VARLEN = AttnWorkload("varlen16_1k16k_h16d128_bf16_causal_had_ss", 16, 16, 16,
 
 # Llama-3.1-8B attention shape (32 query heads, 8 kv heads, d = 128) at the
 # 131k context the pages quote decode at.
-C_DECODE131K = DecodeWorkload("decode_b4h32hkv8_ctx131072_bf16_top10", 4, 32, 8, 131072,
+# 131072 tokens cached per sequence, room for one more tile of new tokens.
+C_DECODE131K = DecodeWorkload("decode_b4h32hkv8_ctx131072_bf16_top10", 4, 32, 8, 131072 + 128,
                               131072, 131072, 128, torch.bfloat16, 0.10, False)
 
 

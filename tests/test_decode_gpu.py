@@ -227,11 +227,14 @@ def test_decode_full_size_sampled(orc):
     w = synth.C_DECODE131K
     inp = synth.make_decode_inputs(w, device="cuda")
     q, k, v, lengths = inp["q"], inp["k"], inp["v"], inp["lengths"]
-    kv = torch.stack([ops.nvfp4_quantize(k.reshape(-1, 128))[2].reshape(()),
-                      ops.nvfp4_quantize(v.reshape(-1, 128))[2].reshape(())])
+    kv = torch.stack([ops.nvfp4_quantize(k[:, :lengths[0]].reshape(-1, 128))[2].reshape(()),
+                      ops.nvfp4_quantize(v[:, :lengths[0]].reshape(-1, 128))[2].reshape(())])
     cache = ops.DoubleKVCache(w.B, w.Hkv, w.capacity, kv, dtype=w.dtype)
-    for t0 in range(0, w.capacity, 32768):
-        cache.append(k[:, t0:t0 + 32768].contiguous(), v[:, t0:t0 + 32768].contiguous())
+    L = lengths[0]
+    assert all(x == L for x in lengths)
+    for t0 in range(0, L, 32768):
+        t1 = min(L, t0 + 32768)
+        cache.append(k[:, t0:t1].contiguous(), v[:, t0:t1].contiguous())
     need = ops.attn_decode_workspace_size(w.B, w.H, w.Hkv, w.capacity)
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     out, lse = ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, workspace=ws)
