@@ -331,14 +331,18 @@ def decode_line(ops, dev, peaks, steps=50, warmup=5):
     each step, so every step appends at the same position and attends over
     131073 tokens."""
     w, cache, q, k_new, v_new, L0, ws = decode_setup(ops, dev, synth.C_DECODE131K)
-    base = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    # the serving loop's own length bookkeeping: every step writes its token
+    # at position L0 and attends over L0 + 1 tokens
+    at = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    ones = torch.ones(w.B, dtype=torch.int32, device=dev)
+    lens = at + ones
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
 
     def step():
-        cache.lengths.copy_(base)
-        cache.append(k_new, v_new)
-        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, out=out, lse=lse, workspace=ws)
+        cache.append(k_new, v_new, n_new=ones, cache_len=at)
+        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, out=out, lse=lse, workspace=ws,
+                               seq_len=lens)
 
     for _ in range(warmup):
         step()
@@ -390,14 +394,15 @@ def decode_only(args):
     dev = torch.device("cuda", 0)
     w, cache, q, k_new, v_new, L0, ws = decode_setup(ops, dev, synth.C_DECODE131K,
                                                    args.decode_context)
-    base = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    at = torch.full((w.B,), L0, dtype=torch.int32, device=dev)
+    ones = torch.ones(w.B, dtype=torch.int32, device=dev)
+    lens = at + ones
     times = []
     for _ in range(args.warmup + args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        cache.lengths.copy_(base)
         e0.record()
-        cache.append(k_new, v_new)
-        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, workspace=ws)
+        cache.append(k_new, v_new, n_new=ones, cache_len=at)
+        ops.thrift_attn_decode(q, cache, topk_frac=w.topk_frac, workspace=ws, seq_len=lens)
         e1.record()
         torch.cuda.synchronize(dev)
         times.append(1e3 * e0.elapsed_time(e1))

@@ -179,19 +179,26 @@ __global__ void __launch_bounds__(128) dec_q_image_kernel(const uint16_t* __rest
 // ------------------------------------------------------------- selection --
 
 // scores [B, H, nbcap] fp64: q . kbar_j by a sequential fp64 fma over d, the
-// query taken as its own block mean.  One CTA per (16 key tiles, kv head,
-// sequence); thread (tile, head of the group).
-constexpr int kDecScoreTiles = 16;
+// query taken as its own block mean.  One CTA per (32 key tiles, kv head,
+// sequence), 32 G threads: thread (tile, head of the group).  Shared memory
+// (dynamic, dec_scores_smem bytes): the tiles' means, rows padded to 129
+// doubles, then the G query rows.
+constexpr int kDecScoreTiles = 32;
+
+__host__ __device__ constexpr size_t dec_scores_smem(int G) {
+  return (size_t)kDecScoreTiles * (kDecD + 1) * 8 + (size_t)G * kDecD * 8;
+}
 
 template <int DT>
-__global__ void __launch_bounds__(256) dec_scores_kernel(const uint16_t* __restrict__ q, int H,
+__global__ void __launch_bounds__(512) dec_scores_kernel(const uint16_t* __restrict__ q, int H,
                                                          int G, CacheGeom cg,
                                                          const uint8_t* __restrict__ cache,
                                                          const int32_t* __restrict__ seq_len,
                                                          int capacity, int nbcap,
                                                          double* __restrict__ scores) {
-  __shared__ double km[kDecScoreTiles][kDecD + 1];
-  __shared__ double qm[kDecMaxG][kDecD];
+  extern __shared__ double dsm_scores[];
+  double* km = dsm_scores;                                 // [32][129]
+  double* qm = dsm_scores + kDecScoreTiles * (kDecD + 1);  // [G][128]
   const int j0 = blockIdx.x * kDecScoreTiles, hk = blockIdx.y, b = blockIdx.z;
   const int len = min(capacity, max(0, __ldg(seq_len + b)));
   const int nb = (int)ceil_div(len, kDecTile);
@@ -199,18 +206,38 @@ __global__ void __launch_bounds__(256) dec_scores_kernel(const uint16_t* __restr
   const int nj = min(kDecScoreTiles, nb - j0);
   const double* means =
       reinterpret_cast<const double*>(cache + cg.off_means()) + cg.tile(b, hk, j0) * kDecD;
-  for (int e = threadIdx.x; e < nj * kDecD; e += blockDim.x)
-    km[e / kDecD][e % kDecD] = __ldg(means + e);
+  // the means arrive as 16-byte pairs, eight loads in flight per thread
+  // before any is stored (the rows' padding breaks a single bulk copy)
+  const double2* m2 = reinterpret_cast<const double2*>(means);
+  const int npair = nj * kDecD / 2;
+  for (int e0 = threadIdx.x; e0 < npair; e0 += 8 * blockDim.x) {
+    double2 r[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = e0 + k * blockDim.x;
+      r[k] = e < npair ? __ldg(m2 + e) : make_double2(0.0, 0.0);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = 2 * (e0 + k * blockDim.x);
+      if (e < 2 * npair) {
+        double* dst = km + (e / kDecD) * (kDecD + 1) + e % kDecD;
+        dst[0] = r[k].x;
+        dst[1] = r[k].y;
+      }
+    }
+  }
   for (int e = threadIdx.x; e < G * kDecD; e += blockDim.x)
-    qm[e / kDecD][e % kDecD] =
-        (double)h2f<DT>(__ldg(q + ((int64_t)b * H + hk * G + e / kDecD) * kDecD + e % kDecD));
+    qm[e] = (double)h2f<DT>(__ldg(q + ((int64_t)b * H + hk * G + e / kDecD) * kDecD + e % kDecD));
   __syncthreads();
   for (int w = threadIdx.x; w < kDecScoreTiles * G; w += blockDim.x) {
     const int jj = w % kDecScoreTiles, gq = w / kDecScoreTiles;
     if (jj >= nj) continue;
+    const double* kr = km + jj * (kDecD + 1);
+    const double* qr = qm + gq * kDecD;
     double acc = 0.0;
 #pragma unroll 8
-    for (int c = 0; c < kDecD; ++c) acc = __fma_rn(qm[gq][c], km[jj][c], acc);
+    for (int c = 0; c < kDecD; ++c) acc = __fma_rn(qr[c], kr[c], acc);
     scores[((int64_t)b * H + hk * G + gq) * nbcap + j0 + jj] = acc;
   }
 }
@@ -218,7 +245,9 @@ __global__ void __launch_bounds__(256) dec_scores_kernel(const uint16_t* __restr
 // mask [B, H, nbcap] uint8 (1 = FP16 key tile): the k = ceil(frac * nb)
 // best tiles of each (sequence, head), ties to the lower tile, plus the
 // first `sink` and the last `recent` tiles.  One CTA per (sequence, head).
-__global__ void __launch_bounds__(kTopkThreads) dec_topk_kernel(
+constexpr int kDecTopkThreads = 1024;
+
+__global__ void __launch_bounds__(kDecTopkThreads) dec_topk_kernel(
     const double* __restrict__ scores, const int32_t* __restrict__ seq_len, int capacity, int H,
     int nbcap, float frac, int sink, int recent, uint8_t* __restrict__ mask) {
   __shared__ TopkShared sh;
@@ -237,7 +266,8 @@ __global__ void __launch_bounds__(kTopkThreads) dec_topk_kernel(
 
 // ----------------------------------------------------------------- merge --
 
-// Splits of one (sequence, head) merged: each split s left its output O_s
+// Splits of one (sequence, head) merged (at most 128 splits, one per
+// thread for the weights): each split s left its output O_s
 // relative to its own running max m_s (log2 units) and its sum l_s.
 //   M = max m_s,  out = sum 2^(m_s - M) O_s / sum 2^(m_s - M) l_s,
 //   lse = M ln 2 + ln(sum 2^(m_s - M) l_s).
@@ -247,27 +277,54 @@ __global__ void __launch_bounds__(kDecD) dec_combine_kernel(const float* __restr
                                                             const float* __restrict__ part_ml,
                                                             int nsplit, uint16_t* __restrict__ out,
                                                             float* __restrict__ lse) {
+  __shared__ float s_w[128];  // weight 2^(m_s - M) of each split (0: empty)
+  __shared__ float s_part[4];
+  __shared__ float s_ML[2];
   const int64_t bh = blockIdx.x;
   const float* ml = part_ml + bh * nsplit * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldg(ml + 2 * s));
-  float L = 0.0f, o = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = __ldg(ml + 2 * s);
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      L = fmaf(w, __ldg(ml + 2 * s + 1), L);
-      o = fmaf(w, __ldg(part_o + (bh * nsplit + s) * kDecD + threadIdx.x), o);
-    }
+  const int tid = threadIdx.x;
+  // splits spread over the threads: the maximum, then the weights and L
+  const float ms = tid < nsplit ? __ldg(ml + 2 * tid) : -INFINITY;
+  const float ls = tid < nsplit ? __ldg(ml + 2 * tid + 1) : 0.0f;
+  float M = ms;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if ((tid & 31) == 0) s_part[tid >> 5] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_part[0], s_part[1]), fmaxf(s_part[2], s_part[3]));
+  const float wgt = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
+  s_w[tid] = wgt;
+  float L = wgt * ls;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  __syncthreads();
+  if ((tid & 31) == 0) s_part[tid >> 5] = L;
+  __syncthreads();
+  if (tid == 0) {
+    s_ML[0] = M;
+    s_ML[1] = s_part[0] + s_part[1] + s_part[2] + s_part[3];
   }
+  __syncthreads();
+  L = s_ML[1];
+  // channel tid: the weighted sum over the splits, four loads in flight
+  const float* po = part_o + bh * nsplit * kDecD + tid;
+  float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
+  int s2 = 0;
+  for (; s2 + 4 <= nsplit; s2 += 4) {
+    o0 = fmaf(s_w[s2], __ldg(po + (int64_t)s2 * kDecD), o0);
+    o1 = fmaf(s_w[s2 + 1], __ldg(po + (int64_t)(s2 + 1) * kDecD), o1);
+    o2 = fmaf(s_w[s2 + 2], __ldg(po + (int64_t)(s2 + 2) * kDecD), o2);
+    o3 = fmaf(s_w[s2 + 3], __ldg(po + (int64_t)(s2 + 3) * kDecD), o3);
+  }
+  for (; s2 < nsplit; ++s2) o0 = fmaf(s_w[s2], __ldg(po + (int64_t)s2 * kDecD), o0);
+  const float o = (o0 + o1) + (o2 + o3);
   const float r = L > 0.0f ? o / L : 0.0f;
   if constexpr (DT == 1) {
-    out[bh * kDecD + threadIdx.x] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    out[bh * kDecD + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
   } else {
-    out[bh * kDecD + threadIdx.x] = __half_as_ushort(__float2half_rn(r));
+    out[bh * kDecD + tid] = __half_as_ushort(__float2half_rn(r));
   }
-  if (threadIdx.x == 0) lse[bh] = L > 0.0f ? M * 0.6931471805599453f + logf(L) : -INFINITY;
+  if (tid == 0) lse[bh] = L > 0.0f ? M * 0.6931471805599453f + logf(L) : -INFINITY;
 }
 
 // ------------------------------------------------------ attention kernel --
@@ -298,6 +355,13 @@ __global__ void __launch_bounds__(kDecD) dec_combine_kernel(const float* __restr
 // prefill kernel) and 1 for an FP16 one.
 
 __host__ __device__ constexpr uint32_t dec_align(uint32_t x) { return (x + 1023u) & ~1023u; }
+
+// Maximum of a float over the warp (one redux instruction).
+__device__ __forceinline__ float redux_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 
 // Sum of N values by a pairwise tree.
 template <int N>
@@ -347,8 +411,8 @@ struct DecLayout {
   static constexpr uint32_t ST_PITCH = kDecTile + 4;  // floats per transposed score row
   static constexpr uint32_t ST_BYTES = kDecMaxG * ST_PITCH * 4;
   static constexpr uint32_t OFF_ST = OFF_LIST + 4 * MAX_TILES;       // [group][2][16][132]
-  static constexpr uint32_t OFF_COEF = OFF_ST + 2 * 2 * ST_BYTES;    // [group][2][16][2]
-  static constexpr uint32_t OFF_BAR = OFF_COEF + 2 * 2 * kDecMaxG * 2 * 4;
+  static constexpr uint32_t OFF_COEF = OFF_ST + 2 * 2 * ST_BYTES;    // [group][4][16][2]
+  static constexpr uint32_t OFF_BAR = OFF_COEF + 2 * 4 * kDecMaxG * 2 * 4;
   static constexpr uint32_t BYTES = OFF_BAR + 512;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
   // tensor-memory columns
@@ -433,27 +497,40 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
   if (warp == 0) {
     // Tile list: tiles some head takes in NVFP4 (ascending), then tiles some
     // head takes in FP16 (ascending).  Entry: tile j (bits 0..14), the FP16
-    // heads of the group (bits 16..31).
+    // heads of the group (bits 16..31).  The mask bytes of up to 128 tiles
+    // are requested before any is used (one memory round trip per 128).
     const uint32_t all = (1u << G) - 1u;
     const uint8_t* mk = p.mask + ((int64_t)b * p.H + hk * G) * p.nbcap;
-    int n = 0;
-    for (int pass = 0; pass < 2; ++pass) {
-      for (int jb = j0; jb < j1; jb += 32) {
-        const int j = jb + lane;
-        uint32_t bits = 0;
-        bool take = false;
-        if (j < j1) {
+    int n = 0, nf = 0;
+    uint32_t* l16 = s_list + L::MAX_TILES / 2;  // FP16 entries, moved after the NVFP4 ones
+    for (int jb = j0; jb < j1; jb += 128) {
+      uint32_t bits[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = jb + 32 * r + lane;
+        if (j < j1)
           for (int c = 0; c < G; ++c)
-            if (__ldg(mk + (int64_t)c * p.nbcap + j) != 0) bits |= 1u << c;
-          take = pass == 0 ? bits != all : bits != 0;
-        }
-        const unsigned vote = __ballot_sync(0xffffffffu, take);
-        if (take) s_list[n + __popc(vote & ((1u << lane) - 1u))] = (uint32_t)j | (bits << 16);
-        n += __popc(vote);
+            bits[r] |= (uint32_t)(__ldg(mk + (int64_t)c * p.nbcap + j) != 0) << c;
       }
-      if (pass == 0 && lane == 0) *s_n4 = n;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = jb + 32 * r + lane;
+        const bool in = j < j1;
+        const bool t4 = in && bits[r] != all, t16 = in && bits[r] != 0;
+        const unsigned v4 = __ballot_sync(0xffffffffu, t4), v16 = __ballot_sync(0xffffffffu, t16);
+        const uint32_t e = (uint32_t)j | (bits[r] << 16);
+        if (t4) s_list[n + __popc(v4 & ((1u << lane) - 1u))] = e;
+        if (t16) l16[nf + __popc(v16 & ((1u << lane) - 1u))] = e;
+        n += __popc(v4);
+        nf += __popc(v16);
+      }
     }
-    if (lane == 0) *s_n = n;
+    __syncwarp();
+    for (int e = lane; e < nf; e += 32) s_list[n + e] = l16[e];
+    if (lane == 0) {
+      *s_n4 = n;
+      *s_n = n + nf;
+    }
   }
   __syncthreads();
   if (warp == kDecQkWarp) {
@@ -568,10 +645,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             if (!mbar_wait(&bars[D_Q16], 0, s_abort)) { ok = false; break; }
             q16_ready = true;
           }
-          if (u >= 1 && !mbar_wait(&bars[D_SE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t dS = tmem + L::T_S + 64 * g;
           if (!f16) {
+            // scale factors first: they wait only for the stage (the slot's
+            // previous reader, QK(t - 2), was issued earlier by this thread)
+            tc_fence_after();
             const uint32_t stg = L::OFF4_STG + sl * L::STG4;
             if (!q4_ready) {
 #pragma unroll
@@ -583,11 +661,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
               tc_cp_32x128b_x4(ksf + 4 * s2, d_sf + ((stg + kDecTile * (kDecD / 2) + 512 * s2) >> 4));
+            if (u >= 1 && !mbar_wait(&bars[D_SE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
               mma_nvf4(dS, d4 + (stg >> 4) + 2 * s2, d4 + (L::OFF4_Q >> 4) + 2 * s2, id4,
                        ksf + 4 * s2, qsf + 4 * s2, s2 > 0);
           } else {
+            if (u >= 1 && !mbar_wait(&bars[D_SE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+            tc_fence_after();
             const uint32_t stg = L::OFF16_STG + sl * L::STG16;
 #pragma unroll
             for (int kk = 0; kk < kDecD / 16; ++kk)
@@ -612,6 +694,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
           stage_of(t, sl, par);
           uint64_t* empty = f16 ? &bars[D_KVE16 + sl] : &bars[D_KVE4 + sl];
           const int sl2 = u & 1, use = u >> 1;  // P / O slot and its use count
+          if (!f16) {
+            // V's scale factors as soon as the stage has landed (the slot's
+            // previous reader, PV(t - 2), was issued earlier by this thread)
+            if (!mbar_wait(&bars[D_KVF4 + sl], par, s_abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t stg = L::OFF4_STG + sl * L::STG4 + CacheGeom::K4;
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2)
+              tc_cp_32x128b_x4(vsf + 4 * s2, d_sf + ((stg + kDecD * (kDecTile / 2) + 512 * s2) >> 4));
+          }
           if (!mbar_wait(&bars[D_PF + 2 * g + sl2], use & 1, s_abort)) { ok = false; break; }
           if (use >= 1 && !mbar_wait(&bars[D_OE + 2 * g + sl2], (use - 1) & 1, s_abort)) {
             ok = false;
@@ -623,10 +715,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             const uint32_t stg = L::OFF4_STG + sl * L::STG4 + CacheGeom::K4;
             const uint32_t pp = L::OFF4_P + (2 * g + sl2) * dec_align(L::P4B);
 #pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-              tc_cp_32x128b_x4(vsf + 4 * s2, d_sf + ((stg + kDecD * (kDecTile / 2) + 512 * s2) >> 4));
+            for (int s2 = 0; s2 < 2; ++s2)
               tc_cp_32x128b_x4(psf + 4 * s2, d_sf + ((pp + 64 * (kDecTile / 2) + 512 * s2) >> 4));
-            }
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
               mma_nvf4(dO, d4 + (stg >> 4) + 2 * s2, d4 + (pp >> 4) + 2 * s2, id4, vsf + 4 * s2,
@@ -660,7 +750,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     const float gk = __ldg(p.kv_scale), gv = __ldg(p.kv_scale + 1);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale), cs16 = p.scale;
     float* sT0 = reinterpret_cast<float*>(sm + L::OFF_ST) + g * 2 * (L::ST_BYTES / 4);
-    float* coef = reinterpret_cast<float*>(sm + L::OFF_COEF) + g * (2 * kDecMaxG * 2);
+    float* coef = reinterpret_cast<float*>(sm + L::OFF_COEF) + g * (4 * kDecMaxG * 2);
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_addr = lane_base + L::T_S + 64 * g;
     const uint32_t o_addr = lane_base + L::T_O + 64 * (2 * g);  // + 64 slot
@@ -672,9 +762,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     constexpr int KPL = 16 / LPB;                          // keys per lane
     const int c = i / (8 * LPB), bb = (i / LPB) % 8, hb = i % LPB;
     const bool has_item = i < 8 * LPB * GC;  // uniform over each warp
-    const int own = lane & ~(8 * LPB - 1);
     const bool is_owner = (i % (8 * LPB)) == 0;
-    float m = -INFINITY, l = 0.0f;  // running state of head c (owner lanes)
+    // running state of head c, kept by each of its 8 LPB lanes: the same
+    // max m on all of them, and each lane's share of the sum l (its keys'
+    // probabilities; the shares are added once, at the end)
+    float m = -INFINITY, l = 0.0f;
     float orun[GC];
 #pragma unroll
     for (int k = 0; k < GC; ++k) orun[k] = 0.0f;
@@ -692,21 +784,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       }
     }
     // fold of the group's tile with use count v (slot v & 1): wait for its
-    // PV, add it to the running output with the coefficients its owners
-    // wrote, free the O buffer
-    auto fold = [&](int v) -> bool {
-      const int sl2 = v & 1;
-      if (!warp_wait(&bars[D_OD + 2 * g + sl2], (v >> 1) & 1, s_abort)) return false;
+    // PV and start the load (fold_issue), then add it to the running output
+    // with the coefficients its owners wrote (slot v & 3) and free the O
+    // buffer (fold_finish, after tcgen05.wait::ld)
+    float o[GC];
+    auto fold_issue = [&](int v) -> bool {
+      if (!warp_wait(&bars[D_OD + 2 * g + (v & 1)], (v >> 1) & 1, s_abort)) return false;
       tc_fence_after();
-      float o[GC];
-      tmem_ld_cols<GC>(o_addr + 64 * sl2, o);
+      tmem_ld_cols<GC>(o_addr + 64 * (v & 1), o);
+      return true;
+    };
+    auto fold_finish = [&](int v) {
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars[D_OE + 2 * g + sl2]);
-      const float* cf = coef + sl2 * (kDecMaxG * 2);
+      mbar_arrive(&bars[D_OE + 2 * g + (v & 1)]);
+      const float* cf = coef + (v & 3) * (kDecMaxG * 2);
 #pragma unroll
       for (int k = 0; k < GC; ++k) orun[k] = fmaf(cf[2 * k], orun[k], cf[2 * k + 1] * o[k]);
-      return true;
     };
     bool p16_ready = false;
     bool ok = true;
@@ -742,12 +836,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       mbar_arrive(&bars[D_SE + g]);
       mbar_arrive(&bars[D_GB + g]);
       if (!warp_wait(&bars[D_GB + g], u & 1, s_abort)) { ok = false; break; }
-      // the single FP16 P buffer was last read by PV(t - 2)
-      if (f16 && u >= 1 &&
-          !warp_wait(&bars[D_OD + 2 * g + ((u - 1) & 1)], ((u - 1) >> 1) & 1, s_abort)) {
-        ok = false;
-        break;
-      }
+      // E (first half): PV(t - 2) retired (the single FP16 P buffer is then
+      // free too); its load runs while the probabilities are computed
+      if (u >= 1 && !fold_issue(u - 1)) { ok = false; break; }
       uint8_t* p4 = p4g + (u & 1) * dec_align(L::P4B);
       // C: probabilities of keys [16 bb + KPL hb, + KPL) of head c
       if (has_item) {
@@ -766,14 +857,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
 #pragma unroll
         for (int e = 1; e < KPL; ++e) bm = fmaxf(bm, x[e]);
 #pragma unroll
-        for (int o = 1; o < LPB; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-        float mt_raw = bm;
+        for (int o2 = 1; o2 < LPB; o2 <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o2));
+        float mt_raw;
+        if constexpr (8 * LPB == 32) {
+          mt_raw = redux_max_f32(bm);  // the head is the whole warp
+        } else {
+          mt_raw = bm;
 #pragma unroll
-        for (int o = LPB; o < 8 * LPB; o <<= 1)
-          mt_raw = fmaxf(mt_raw, __shfl_xor_sync(0xffffffffu, mt_raw, o));
+          for (int o2 = LPB; o2 < 8 * LPB; o2 <<= 1)
+            mt_raw = fmaxf(mt_raw, __shfl_xor_sync(0xffffffffu, mt_raw, o2));
+        }
         const bool active = c < G && (((bits >> c) & 1u) != 0) == f16;
-        const float m_old = __shfl_sync(0xffffffffu, m, own);
-        float alpha = 1.0f, sigma = 0.0f, ls = 0.0f;
+        float alpha = 1.0f, sigma = 0.0f;
         if (!f16) {
           uint32_t S = 0;
           uint32_t code[KPL / 8 > 0 ? KPL / 8 : 1] = {};
@@ -781,7 +876,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
           bool drop = false;
           if (active) {
             const float mt = mt_raw * cs4;
-            const float m_new = fmaxf(m_old, mt);
+            const float m_new = fmaxf(m, mt);
             const float e = ex2_ftz(fmaf(bm, cs4, -mt));  // block max / tile max
             S = ue4m3(448.0f * e);
             const float dec = ue4m3_decode_fast(S);
@@ -790,7 +885,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             for (int e2 = 0; e2 < KPL; e2 += 2) fma2(x[e2], x[e2 + 1], x[e2], x[e2 + 1], cs4, cs4, cc, cc);
 #pragma unroll
             for (int e2 = 0; e2 < KPL; ++e2) x[e2] = ex2_ftz(x[e2]);  // masked (-inf) -> 0
-            ls = tree_sum<KPL>(x) * dec;
+            const float ls = tree_sum<KPL>(x) * dec;
             if constexpr (KPL >= 8) {
 #pragma unroll
               for (int q = 0; q < KPL / 8; ++q) code[q] = e2m1x8(x + 8 * q);
@@ -802,16 +897,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             sigma = sigma_raw * gv;
             if (!(sigma >= 1.17549435e-38f)) sigma = sigma_raw = 0.0f;
             drop = sigma == 0.0f;
-            alpha = m_old == -INFINITY ? 0.0f : ex2_ftz(m_old - m_new);
-#pragma unroll
-            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-            if (is_owner) {
-              l = fmaf(ls, sigma_raw, alpha * l);
-              m = m_new;
-            }
-          } else {
-#pragma unroll
-            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            alpha = m == -INFINITY ? 0.0f : ex2_ftz(m - m_new);
+            l = fmaf(ls, sigma_raw, alpha * l);
+            m = m_new;
           }
           uint8_t* dst = p4 + swz_offset(c, 8 * bb + (KPL / 2) * hb, kDecTile / 2);
           if constexpr (KPL == 16) {
@@ -826,27 +914,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
           uint32_t w[KPL / 2] = {};
           if (active) {
             const float mt = mt_raw * cs16;
-            const float m_new = fmaxf(m_old, mt);
+            const float m_new = fmaxf(m, mt);
             const float negm = -m_new;
 #pragma unroll
             for (int e2 = 0; e2 < KPL; e2 += 2)
               fma2(x[e2], x[e2 + 1], x[e2], x[e2 + 1], cs16, cs16, negm, negm);
 #pragma unroll
             for (int e2 = 0; e2 < KPL; ++e2) x[e2] = ex2_ftz(x[e2]);
-            ls = tree_sum<KPL>(x);
+            const float ls = tree_sum<KPL>(x);
 #pragma unroll
             for (int e2 = 0; e2 < KPL / 2; ++e2) w[e2] = pack2<DT>(x[2 * e2], x[2 * e2 + 1]);
-            alpha = m_old == -INFINITY ? 0.0f : ex2_ftz(m_old - m_new);
+            alpha = m == -INFINITY ? 0.0f : ex2_ftz(m - m_new);
             sigma = 1.0f;
-#pragma unroll
-            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-            if (is_owner) {
-              l = fmaf(alpha, l, ls);
-              m = m_new;
-            }
-          } else {
-#pragma unroll
-            for (int o = 1; o < 8 * LPB; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            l = fmaf(alpha, l, ls);
+            m = m_new;
           }
           const uint32_t k0 = 16 * bb + KPL * hb;
           uint8_t* reg = p16 + (k0 / 64) * (64 * 128);
@@ -858,7 +939,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             *reinterpret_cast<uint2*>(reg + swz_offset(c, (k0 % 64) * 2, 128)) = make_uint2(w[0], w[1]);
         }
         if (is_owner) {
-          float* cf = coef + (u & 1) * (kDecMaxG * 2);
+          float* cf = coef + (u & 3) * (kDecMaxG * 2);
           cf[2 * c] = alpha;
           cf[2 * c + 1] = sigma;
         }
@@ -866,9 +947,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       // D: P(t) is in shared memory
       fence_proxy_async_smem();
       mbar_arrive(&bars[D_PF + 2 * g + (u & 1)]);
-      // E: fold PV(t - 2), now off the path from S(t) to P(t) (its
-      // coefficients were written before this tile's barrier)
-      if (u >= 1 && !fold(u - 1)) { ok = false; break; }
+      // E (second half): fold PV(t - 2) (its coefficients were written
+      // before this tile's barrier)
+      if (u >= 1) fold_finish(u - 1);
       u_last = u;
     }
     // the group's last PV, folded once every owner lane has written the
@@ -876,7 +957,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     if (ok && u_last >= 0) {
       mbar_arrive(&bars[D_GB + g]);
       ok = warp_wait(&bars[D_GB + g], (u_last + 1) & 1, s_abort);
-      if (ok) ok = fold(u_last);
+      if (ok) ok = fold_issue(u_last);
+      if (ok) fold_finish(u_last);
     }
     if (ok) {
       // this group's split: output relative to its running max, m and l
@@ -885,9 +967,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
 #pragma unroll
       for (int k = 0; k < GC; ++k)
         if (k < G) p.part_o[((row0 + k) * ns + sidx) * kDecD + i] = orun[k];
-      if (has_item && is_owner && c < G) {
-        p.part_ml[((row0 + c) * ns + sidx) * 2] = m;
-        p.part_ml[((row0 + c) * ns + sidx) * 2 + 1] = l;
+      if (has_item) {
+#pragma unroll
+        for (int o2 = 1; o2 < 8 * LPB; o2 <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+        if (is_owner && c < G) {
+          p.part_ml[((row0 + c) * ns + sidx) * 2] = m;
+          p.part_ml[((row0 + c) * ns + sidx) * 2 + 1] = l;
+        }
       }
     }
   }

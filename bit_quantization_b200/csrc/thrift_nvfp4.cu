@@ -487,11 +487,22 @@ thrift_status decode_impl(const void* q, int B, int H, int Hkv, int capacity, co
   else
     dec_q_image_kernel<DT, false><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, w.q4, w.q16);
   const uint8_t* cp = static_cast<const uint8_t*>(cache);
-  dec_scores_kernel<DT><<<dim3((unsigned)ceil_div(nbcap, kDecScoreTiles), Hkv, B), 256, 0, st>>>(
-      qp, H, G, cg, cp, seq_len, capacity, nbcap, w.scores);
+  {
+    static bool attr_set = false;
+    if (!attr_set) {
+      if (cudaFuncSetAttribute(dec_scores_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)dec_scores_smem(kDecMaxG)) != cudaSuccess)
+        return THRIFT_ERR_CUDA;
+      attr_set = true;
+    }
+    const int threads = kDecScoreTiles * std::max(G, 4);
+    dec_scores_kernel<DT><<<dim3((unsigned)ceil_div(nbcap, kDecScoreTiles), Hkv, B), threads,
+                            dec_scores_smem(G), st>>>(qp, H, G, cg, cp, seq_len, capacity, nbcap,
+                                                      w.scores);
+  }
   const size_t tsm = nbcap <= kTopkCache ? (size_t)nbcap * 8 : 0;
-  dec_topk_kernel<<<B * H, kTopkThreads, tsm, st>>>(w.scores, seq_len, capacity, H, nbcap, frac,
-                                                     sink, recent, w.mask);
+  dec_topk_kernel<<<B * H, kDecTopkThreads, tsm, st>>>(w.scores, seq_len, capacity, H, nbcap,
+                                                        frac, sink, recent, w.mask);
   thrift_status s = launch_status();
   if (s != THRIFT_OK) return s;
   DecParams p;

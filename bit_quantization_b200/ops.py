@@ -358,25 +358,31 @@ class DoubleKVCache:
         self.lengths = torch.zeros(B, dtype=torch.int32, device=device)
         self.kv_scale = torch.as_tensor(kv_scale, dtype=torch.float32, device=device).reshape(2)
 
-    def append(self, k_new, v_new, n_new=None):
-        """k_new, v_new [B, T, Hkv, d]; n_new int32 [B] (default: T each)."""
+    def append(self, k_new, v_new, n_new=None, cache_len=None):
+        """k_new, v_new [B, T, Hkv, d]; n_new int32 [B] (default: T each).
+        ``cache_len`` (int32 [B], device): the positions to write at, for a
+        caller that keeps its own lengths (``self.lengths`` is then left as
+        it is); by default ``self.lengths``, advanced by ``n_new``."""
         _need_cuda(k_new, v_new)
         B, T, Hkv, d = k_new.shape
         if n_new is None:
             n_new = torch.full((B,), T, dtype=torch.int32, device=k_new.device)
+        at = self.lengths if cache_len is None else cache_len
         _check(lib().thrift_kv_cache_append(_ptr(k_new), _ptr(v_new), _dt(k_new), B, Hkv, d,
-                                            self.blk, self.capacity, _ptr(self.lengths),
-                                            _ptr(n_new), T, _ptr(self.kv_scale),
-                                            int(self.use_scalesearch), _ptr(self.buf),
-                                            self.buf.numel(), _stream(k_new)),
+                                            self.blk, self.capacity, _ptr(at), _ptr(n_new), T,
+                                            _ptr(self.kv_scale), int(self.use_scalesearch),
+                                            _ptr(self.buf), self.buf.numel(), _stream(k_new)),
                "thrift_kv_cache_append")
-        self.lengths.add_(n_new)
-        self.lengths.clamp_(max=self.capacity)
+        if cache_len is None:
+            self.lengths.add_(n_new)
+            self.lengths.clamp_(max=self.capacity)
 
 
 def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, recent_blocks=0,
-                       use_scalesearch=False, out=None, lse=None, workspace=None):
-    """q [B,H,d] -> (out [B,H,d], lse f32 [B,H]) against ``cache``."""
+                       use_scalesearch=False, out=None, lse=None, workspace=None, seq_len=None):
+    """q [B,H,d] -> (out [B,H,d], lse f32 [B,H]) against ``cache``
+    (``seq_len``: int32 [B] device lengths to attend over instead of
+    ``cache.lengths``)."""
     _need_cuda(q)
     B, H, d = q.shape
     if out is None:
@@ -389,7 +395,8 @@ def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, re
     ws = workspace if workspace is not None else _ws.get(need, q.device)
     _check(lib().thrift_attn_decode(_ptr(q), _dt(q), B, H, cache.Hkv, d, cache.blk,
                                     cache.capacity, _ptr(cache.buf), cache.buf.numel(),
-                                    _ptr(cache.lengths), _ptr(cache.kv_scale), float(topk_frac),
+                                    _ptr(cache.lengths if seq_len is None else seq_len),
+                                    _ptr(cache.kv_scale), float(topk_frac),
                                     int(sink_blocks), int(recent_blocks), int(use_scalesearch),
                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
            "thrift_attn_decode")

@@ -252,3 +252,9 @@ def test_decode_full_size_sampled(orc):
     assert np.array_equal(mask[b:b + 1], r["mask"])
     _compare(out[b:b + 1].float().cpu().numpy(), r["out64"], r["tol"], w.dtype)
     assert np.max(np.abs(lse[b:b + 1].cpu().numpy() - r["lse"])) < 1e-2
+
+
+def test_decode_long_context(orc):
+    # 2049 key tiles: the selection's keys still fit the shared-memory cache,
+    # the tile list spans several list-building rounds
+    _decode_case(orc, _w(1, 4, 1, 2049 * 128, 0.05), lengths=[2049 * 128 - 77])
