@@ -144,13 +144,42 @@ __global__ void __launch_bounds__(kDecD) kv_requant_kernel(
 constexpr uint32_t kDecQ4Bytes = 64 * (kDecD / 2) + (kDecD / 64) * 512;  // 5120
 constexpr uint32_t kDecQ16Bytes = 64 * kDecD * 2;                        // 16384
 
+// amax: the query tensor's absmax (bits of a non-negative float), read when
+// self_amax == 0.  With self_amax != 0 every CTA reduces the whole query
+// tensor itself (q_elems values; for small tensors, read from L2, which saves
+// a launch) and CTA (0, 0) stores the result in *amax for the later kernels.
+constexpr int64_t kDecQSelfAmaxMax = 32768;
+
 template <int DT, bool SS>
 __global__ void __launch_bounds__(128) dec_q_image_kernel(const uint16_t* __restrict__ q, int H,
-                                                          int G, const uint32_t* amax,
+                                                          int G, uint32_t* amax, int self_amax,
+                                                          int64_t q_elems,
                                                           uint8_t* __restrict__ q4img,
                                                           uint8_t* __restrict__ q16img) {
   const int hk = blockIdx.x, b = blockIdx.y, Hkv = gridDim.x;
-  const float g = tensor_scale_from_amax(*amax);
+  float g;
+  if (!self_amax) {
+    g = tensor_scale_from_amax(*amax);
+  } else {
+    __shared__ float red[4];
+    float a = 0.0f;
+    const uint4* q8 = reinterpret_cast<const uint4*>(q);
+    for (int64_t e = threadIdx.x; e < q_elems / 8; e += blockDim.x) {
+      const uint4 r = __ldg(q8 + e);
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        a = fmaxf(a, fmaxf(fabsf(h2f<DT>((uint16_t)(w[k] & 0xFFFF))),
+                           fabsf(h2f<DT>((uint16_t)(w[k] >> 16)))));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    g = tensor_scale_from_amax(__float_as_uint(a));
+    if (hk == 0 && b == 0 && threadIdx.x == 0) *amax = __float_as_uint(a);
+  }
   const int64_t img = (int64_t)b * Hkv + hk;
   uint8_t* q4 = q4img + img * kDecQ4Bytes;
   uint8_t* q16 = q16img + img * kDecQ16Bytes;

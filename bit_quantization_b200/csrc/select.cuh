@@ -208,8 +208,11 @@ __device__ __forceinline__ int select_digit(const int* hist, int64_t rem, int64_
   return sel;
 }
 
-// Exact top-k of one CTA over n entries by an 8-pass radix select on the
-// 64-bit order keys, then ties at the threshold taken in ascending index.
+// Exact top-k of one CTA over n entries by a radix select on the 64-bit
+// order keys (up to 8 passes of 8 bits, most significant first), then ties
+// at the threshold taken in ascending index.  The select stops early once
+// the threshold digit's bucket holds exactly the entries still wanted: all
+// of them are taken, so the lower bits cannot change the result.
 // out[i] = 1 for the k largest valid entries and for every valid entry that
 // `fixed` names, else 0 (every out[i], i < n, is written).  The keys are read
 // once into `kcache` when it is given (n entries).  All threads of the CTA
@@ -218,6 +221,7 @@ struct TopkShared {
   int hist[256];
   int warp_sums[32];
   int total;
+  int done;
   uint64_t prefix;
   int64_t remaining;
 };
@@ -263,13 +267,17 @@ __device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, F
       if (threadIdx.x == 0) {
         sh.remaining = rem - above;
         sh.prefix = prefix | ((uint64_t)sel << shift);
+        sh.done = (int64_t)sh.hist[sel] == rem - above;
       }
     }
     __syncthreads();
     prefix = sh.prefix;
     rem = sh.remaining;
     pmask |= (uint64_t)255 << shift;
+    if (sh.done) break;  // uniform: every thread read the same word
   }
+  // compare on the decided bits only (all of them unless the select stopped
+  // early, when every key of the threshold bucket is taken)
   const uint64_t T = prefix;
   const int64_t take_eq = rem;
   int64_t taken = 0;
@@ -278,7 +286,7 @@ __device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, F
     uint64_t key = 0;
     bool ok = false;
     if (i < n && valid(i)) {
-      key = key_of(i);
+      key = key_of(i) & pmask;
       ok = true;
     }
     const int eq = (ok && key == T) ? 1 : 0;

@@ -480,12 +480,19 @@ thrift_status decode_impl(const void* q, int B, int H, int Hkv, int capacity, co
   const CacheGeom cg = cache_geom(B, Hkv, capacity);
   const int G = H / Hkv, nbcap = cg.ntc;
   const uint16_t* qp = static_cast<const uint16_t*>(q);
-  if (cudaMemsetAsync(w.amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
-  launch_amax<DT>(q, (int64_t)B * H * kDecD / 16, 0, w.amax, st);
+  const int64_t q_elems = (int64_t)B * H * kDecD;
+  // small query tensors: reduced inside the image kernel
+  const int self_amax = q_elems <= kDecQSelfAmaxMax ? 1 : 0;
+  if (!self_amax) {
+    if (cudaMemsetAsync(w.amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+    launch_amax<DT>(q, q_elems / 16, 0, w.amax, st);
+  }
   if (ss)
-    dec_q_image_kernel<DT, true><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, w.q4, w.q16);
+    dec_q_image_kernel<DT, true><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, self_amax,
+                                                               q_elems, w.q4, w.q16);
   else
-    dec_q_image_kernel<DT, false><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, w.q4, w.q16);
+    dec_q_image_kernel<DT, false><<<dim3(Hkv, B), 128, 0, st>>>(qp, H, G, w.amax, self_amax,
+                                                                q_elems, w.q4, w.q16);
   const uint8_t* cp = static_cast<const uint8_t*>(cache);
   {
     static bool attr_set = false;

@@ -258,3 +258,9 @@ def test_decode_long_context(orc):
     # 2049 key tiles: the selection's keys still fit the shared-memory cache,
     # the tile list spans several list-building rounds
     _decode_case(orc, _w(1, 4, 1, 2049 * 128, 0.05), lengths=[2049 * 128 - 77])
+
+
+def test_decode_large_batch(orc):
+    # a query tensor above the size reduced inside the query-image kernel:
+    # the separate absmax kernel runs
+    _decode_case(orc, _w(20, 16, 2, 512, 0.2), seed=5)
