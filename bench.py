@@ -324,6 +324,20 @@ def decode_setup(ops, dev, w, context=None):
     return w, cache, q, k_new, v_new, L0, ws
 
 
+def decode_tiles(ops, w, ws, L0):
+    """Key tiles the last decode step read, from the selection it left in
+    the workspace: per (sequence, kv head), every tile some query head took
+    in NVFP4 (K4 + V4 = 18432 B) and every tile some head took in FP16
+    (K16 + V16 = 65536 B).  Returns (tiles NVFP4, tiles FP16, bytes)."""
+    nbcap = (w.capacity + 127) // 128
+    mo = ops.attn_decode_mask_offset(w.B, w.H, w.Hkv, w.capacity)
+    mask = ws[mo:mo + w.B * w.H * nbcap].view(w.B, w.Hkv, w.H // w.Hkv, nbcap).bool()
+    mask = mask[..., :(L0 + 1 + 127) // 128]
+    t16 = int(mask.any(dim=2).sum())
+    t4 = int((~mask.all(dim=2)).sum())
+    return t4, t16, t4 * 18432 + t16 * 65536
+
+
 def decode_line(ops, dev, peaks, steps=50, warmup=5):
     """One decode step of the decode workload (Llama-3.1-8B attention shape,
     131072 cached tokens per sequence): append the step's token to every
@@ -362,18 +376,7 @@ def decode_line(ops, dev, peaks, steps=50, warmup=5):
         raise RuntimeError("device wait timed out in the decode loop")
     step_us = 1e3 * e0.elapsed_time(e1) / steps
     k_us = 1e3 * kms / max(nk, 1)
-    # key tiles the decode kernel reads: per (sequence, kv head), every tile
-    # some query head takes in NVFP4 (K4 + V4 = 18432 B) and every tile some
-    # head takes in FP16 (K16 + V16 = 65536 B)
-    nbcap = (w.capacity + 127) // 128
-    mo = ops.attn_decode_mask_offset(w.B, w.H, w.Hkv, w.capacity)
-    G = w.H // w.Hkv
-    mask = ws[mo:mo + w.B * w.H * nbcap].view(w.B, w.Hkv, G, nbcap).bool()
-    nb = (L0 + 1 + 127) // 128
-    mask = mask[..., :nb]
-    t16 = int(mask.any(dim=2).sum())
-    t4 = int((~mask.all(dim=2)).sum())
-    kv_bytes = t4 * 18432 + t16 * 65536
+    t4, t16, kv_bytes = decode_tiles(ops, w, ws, L0)
     achieved = kv_bytes / (k_us * 1e-6) / 1e9
     hbm = peaks["hbm_gbs"]
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "d": w.d,
@@ -408,8 +411,10 @@ def decode_only(args):
         times.append(1e3 * e0.elapsed_time(e1))
     if ops.device_status(reset=True) != ops.OK:
         raise RuntimeError("device wait timed out")
+    t4, t16, kv_bytes = decode_tiles(ops, w, ws, L0)
     print(json.dumps({"mode": "decode", "workload": w.name, "cached_tokens": L0,
-                      "us_min": min(times[args.warmup:])}))
+                      "us_min": min(times[args.warmup:]), "tiles_nvfp4": t4, "tiles_fp16": t16,
+                      "algorithmic_bytes": kv_bytes}))
     return 0
 
 
