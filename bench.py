@@ -296,7 +296,13 @@ def quantizer_only(args):
     return 0
 
 
-DECODE_KERNELS_PER_STEP = 8  # append (2), absmax, query images, scores, top-k, decode, merge
+DECODE_KERNELS_PER_STEP = 7  # append (2), query images (absmax fused), scores, top-k, decode, merge
+
+# DRAM traffic per algorithmic byte of the decode kernel, measured by ncu on
+# the 32768-token case of the decode workload (the traffic scales with the
+# tiles read); reported only while the decode source is unchanged since.
+DECODE_TRAFFIC = {"src_sha16": "7733001a3f2a47e2", "bytes_per_algorithmic_byte": 344.29 / 338.72,
+                  "captured_on": "decode workload with 32768 cached tokens"}
 
 
 def decode_setup(ops, dev, w, context=None):
@@ -322,6 +328,15 @@ def decode_setup(ops, dev, w, context=None):
     ws = torch.empty(ops.attn_decode_workspace_size(w.B, w.H, w.Hkv, w.capacity), dtype=torch.uint8,
                      device=dev)
     return w, cache, q, k_new, v_new, L0, ws
+
+
+def decode_traffic(kv_bytes):
+    import hashlib
+    with open(os.path.join(ROOT, "bit_quantization_b200", "csrc", "decode.cuh"), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if sha != DECODE_TRAFFIC["src_sha16"]:
+        return None
+    return kv_bytes * DECODE_TRAFFIC["bytes_per_algorithmic_byte"]
 
 
 def decode_tiles(ops, w, ws, L0):
@@ -385,8 +400,10 @@ def decode_line(ops, dev, peaks, steps=50, warmup=5):
             "step": "append one token per sequence to the FP4 + 16-bit cache, then attend",
             "kernel_us": k_us, "tiles_nvfp4": t4, "tiles_fp16": t16,
             "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
-                         "algorithmic_bytes": kv_bytes},
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": decode_traffic(kv_bytes), "algorithmic_bytes": kv_bytes,
+                         "traffic_note": "ncu DRAM bytes of a 32768-token launch per algorithmic "
+                                         "byte, times this launch's algorithmic bytes"},
             "kernels_per_step": DECODE_KERNELS_PER_STEP}
 
 
