@@ -72,6 +72,10 @@ def lib():
                                       i32, i32, P, i32, P, i64, i32, P, P, P, P, P]
         L.orc_attn_fp64.restype = i32
         L.orc_attn_fp64.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, P, i64, i32, P, P]
+        L.orc_thrift_attn_ex.restype = i32
+        L.orc_thrift_attn_ex.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, i32,
+                                         i32, i32, i32, i32, P, i32, P, i64, i32, P, P, P, P, P]
+        L.orc_k_channel_means.argtypes = [P, i32, i32, P, i32, i32, P]
         L.orc_thrift_decode.restype = i32
         L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
                                         i32, i32, i32, P, i32, P, i32, P, P, P, P, P]
@@ -256,8 +260,19 @@ def block_mean_topk_varlen(q, k, dt, cu, blk, causal, frac, sink_blocks=0, recen
 
 # ---------------------------------------------------------------- attention
 
+def k_channel_means(k, dt, cu):
+    """K channel means of reading R16: k [total, Hkv, d] -> fp32 [nseq, Hkv, d]."""
+    k = _u16(k)
+    cu = np.ascontiguousarray(cu, np.int32)
+    total, Hkv, d = k.shape
+    mu = np.zeros((len(cu) - 1, Hkv, d), np.float32)
+    lib().orc_k_channel_means(_p(k), dt, Hkv, _p(cu), len(cu) - 1, d, _p(mu))
+    return mu
+
+
 def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
-                mask=None, units=None, nthreads=None, sink_blocks=0, recent_blocks=0):
+                mask=None, units=None, nthreads=None, sink_blocks=0, recent_blocks=0,
+                smooth_k=False):
     """Emulated NVFP4 + FP16 attention over packed sequences.
 
     q [total,H,d], k/v [total,Hkv,d] uint16; cu int32 [nseq+1].
@@ -290,9 +305,9 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
         n_units = u.shape[0]
     else:
         u, n_units = None, 0
-    rc = lib().orc_thrift_attn(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
+    rc = lib().orc_thrift_attn_ex(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
                                int(causal), float(frac), int(sink_blocks), int(recent_blocks),
-                               int(use_ss), int(use_had), _p(m), given,
+                               int(use_ss), int(use_had), int(smooth_k), _p(m), given,
                                _p(u), n_units, int(nthreads or nthreads_default()), _p(out),
                                _p(lse), _p(gs), _p(out64), _p(tol))
     if rc:

@@ -48,6 +48,15 @@
 //      the first `sink` key blocks, and the `recent` most recent key blocks a
 //      query block can see, run on the FP16 path for every query block; the
 //      fixed pairs are OR-ed with the top-k pairs, whose quota is unchanged.
+//  R16 K smoothing (optional; "ThriftAttention" / Attn-QAT pages name Q/K
+//      smoothing among the outlier mitigations of earlier FP4 attention):
+//      mu = the mean of each K channel over the tokens of its sequence (per kv
+//      head): fp64 sums in token order within 128-token blocks, the block
+//      sums added in order, divided by the length, rounded to fp32.  The
+//      NVFP4 path quantises K' = fl32(k - mu) (its own tensor scale) and
+//      scores q^ . (k'^ + mu), i.e. the dequantised smoothed key with the
+//      mean added back, so both paths keep the same scores; the FP16 path and
+//      the selection use the raw K.  Not combined with the Hadamard rotation.
 //  R15 decode on the double cache (ThriftAttention, Resultados: decode
 //      speed-up; Significado: the KV cache grows by 28% because every token
 //      is cached in FP16 and in FP4): one new query token per sequence
@@ -550,7 +559,8 @@ static float quantize_rows_unpacked(const uint16_t* x, int dt, int64_t rows, int
 // tile is rounded to fp32 before it is quantised (reading R7).
 
 struct AttnCtx {
-  int dt, H, Hkv, d, blk, causal, use_had;
+  int dt, H, Hkv, d, blk, causal, use_had, smooth_k = 0;
+  std::vector<float> mu;  // K channel means [nseq, Hkv, d] (reading R16)
   const int32_t* cu;
   int nseq;
   int64_t total, ptot;
@@ -659,6 +669,7 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
         int64_t e = ((st + k0 + t) * Hkv + hk) * d + c;
         if (fp4) {
           kt[(size_t)t * d + c] = deq(C.kc[(size_t)e], C.ks[(size_t)(e / 16)], C.gk);
+          if (C.smooth_k) kt[(size_t)t * d + c] += (double)C.mu[((size_t)s * Hkv + hk) * d + c];
           int64_t ve = ((int64_t)hk * d + c) * C.ptot + C.pstart[s] + k0 + t;
           vt[(size_t)t * d + c] = deq(C.vc[(size_t)ve], C.vs[(size_t)(ve / 16)], C.gv);
         } else {
@@ -773,16 +784,82 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // probability whose E2M1 code, UE4M3 block scale or 16-bit value lies within
 // 2e-5 relative of a rounding midpoint may take either side in an
 // implementation that evaluates the same arithmetic in another order.
+// Quantiser of a [rows, cols] fp32 matrix (unpacked codes), tensor scale
+// amax/2688 over the whole matrix: the same arithmetic as
+// quantize_rows_unpacked on values that are not 16-bit.
+static float quantize_rows_f32(const float* x, int64_t rows, int cols, int use_ss, int nthreads,
+                               std::vector<uint8_t>& codes, std::vector<uint8_t>& scales) {
+  float amax = 0.0f;
+  for (int64_t e = 0; e < rows * cols; ++e) amax = std::max(amax, std::fabs(x[e]));
+  const float g = amax == 0.0f ? 1.0f : amax / 2688.0f;
+  codes.assign((size_t)(rows * cols), 0);
+  scales.assign((size_t)(rows * (cols / 16)), 0);
+  parallel_for((rows + 4095) / 4096, nthreads, [&](int64_t ch) {
+    uint8_t packed[8];
+    for (int64_t r = ch * 4096; r < std::min(rows, (ch + 1) * 4096); ++r)
+      for (int b = 0; b < cols / 16; ++b) {
+        orc_quant_block(&x[r * cols + b * 16], g, use_ss, packed,
+                        &scales[(size_t)(r * (cols / 16) + b)], nullptr);
+        for (int e = 0; e < 8; ++e) {
+          codes[(size_t)(r * cols + b * 16 + 2 * e)] = packed[e] & 0xF;
+          codes[(size_t)(r * cols + b * 16 + 2 * e + 1)] = packed[e] >> 4;
+        }
+      }
+  });
+  return g;
+}
+
+// K channel means of reading R16: [nseq, Hkv, d] fp32.
+void orc_k_channel_means(const uint16_t* k, int dt, int Hkv, const int32_t* cu, int nseq, int d,
+                         float* mu) {
+  for (int s = 0; s < nseq; ++s) {
+    const int64_t st = cu[s];
+    const int len = cu[s + 1] - cu[s];
+    for (int hk = 0; hk < Hkv; ++hk)
+      for (int c = 0; c < d; ++c) {
+        double total = 0.0;
+        for (int b0 = 0; b0 < len; b0 += 128) {
+          double sum = 0.0;
+          for (int t = b0; t < std::min(len, b0 + 128); ++t)
+            sum += (double)orc_half_to_float(k[((st + t) * Hkv + hk) * d + c], dt);
+          total += sum;
+        }
+        mu[((size_t)s * Hkv + hk) * d + c] = len > 0 ? (float)(total / (double)len) : 0.0f;
+      }
+  }
+}
+
+int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                       int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
+                       float frac, int sink, int recent, int use_ss, int use_had, int smooth_k,
+                       uint8_t* mask_io, int mask_given,
+                       const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
+                       float* lse, float* gs_out, double* out64, double* tol);
+
 int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
                     int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
                     float frac, int sink, int recent, int use_ss, int use_had,
                     uint8_t* mask_io, int mask_given,
                     const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
                     float* lse, float* gs_out, double* out64, double* tol) {
+  return orc_thrift_attn_ex(q, k, v, dt, H, Hkv, cu, nseq, d, blk, causal, frac, sink, recent,
+                            use_ss, use_had, 0, mask_io, mask_given, units, n_units, nthreads,
+                            out, lse, gs_out, out64, tol);
+}
+
+// As orc_thrift_attn, with optional K smoothing (reading R16).
+int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                       int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
+                       float frac, int sink, int recent, int use_ss, int use_had, int smooth_k,
+                       uint8_t* mask_io, int mask_given,
+                       const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
+                       float* lse, float* gs_out, double* out64, double* tol) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
   if (use_had && (d & (d - 1))) return -1;
+  if (smooth_k && use_had) return -1;
   AttnCtx C;
   C.dt = dt; C.H = H; C.Hkv = Hkv; C.d = d; C.blk = blk; C.causal = causal; C.use_had = use_had;
+  C.smooth_k = smooth_k;
   C.cu = cu; C.nseq = nseq; C.q = q; C.k = k; C.v = v;
   C.total = cu[nseq];
   C.pstart.resize(nseq + 1);
@@ -798,7 +875,21 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
   }
   C.ptot = C.pstart[nseq];
   C.gq = quantize_rows_unpacked(q, dt, C.total * H, d, use_ss, use_had, nthreads, C.qc, C.qs);
-  C.gk = quantize_rows_unpacked(k, dt, C.total * Hkv, d, use_ss, use_had, nthreads, C.kc, C.ks);
+  if (smooth_k) {
+    C.mu.assign((size_t)nseq * Hkv * d, 0.0f);
+    orc_k_channel_means(k, dt, Hkv, cu, nseq, d, C.mu.data());
+    std::vector<float> ks((size_t)(C.total * Hkv * d));
+    for (int s2 = 0; s2 < nseq; ++s2)
+      for (int64_t t = cu[s2]; t < cu[s2 + 1]; ++t)
+        for (int hk = 0; hk < Hkv; ++hk)
+          for (int c = 0; c < d; ++c) {
+            const int64_t e = (t * Hkv + hk) * d + c;
+            ks[(size_t)e] = orc_half_to_float(k[e], dt) - C.mu[((size_t)s2 * Hkv + hk) * d + c];
+          }
+    C.gk = quantize_rows_f32(ks.data(), C.total * Hkv, d, use_ss, nthreads, C.kc, C.ks);
+  } else {
+    C.gk = quantize_rows_unpacked(k, dt, C.total * Hkv, d, use_ss, use_had, nthreads, C.kc, C.ks);
+  }
   // V: 16-blocks along tokens, every sequence zero-padded to a whole number of
   // key blocks (reading R6).  The tensor scale covers the real tokens only.
   {
