@@ -50,6 +50,7 @@ struct AttnParams {
   int64_t total;
   float scale4;            // log2(e)/sqrt(d), divided by d with the rotation
   float scale16;           // log2(e)/sqrt(d)
+  const float* corr;       // K smoothing: q^ . mu per query row [nseq, H, nTq * 128], or null
 };
 
 template <int D, int BLK>
@@ -671,6 +672,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     const float gq = tensor_scale_from_amax(p.amax[0]);
     const float gk = tensor_scale_from_amax(p.amax[1]);
     const float cs4 = __fmul_rn(__fmul_rn(gq, gk), p.scale4);
+    const float corr_r =
+        (p.corr != nullptr && row_ok)
+            ? __ldg(p.corr + ((int64_t)seq * p.H + h) * ((int64_t)p.nTq * 128) + row) * p.scale4
+            : 0.0f;
     const uint32_t s_base = tmem + ((uint32_t)(q4 * 32) << 16) + L::T_S + g * BLK + hf * SC;
     float* xch = reinterpret_cast<float*>(sm + L::OFF_XCH) + g * 512;  // [2 slots][2 halves][128]
     float* sta = reinterpret_cast<float*>(sm + L::OFF_STA);
@@ -735,7 +740,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
       const bool live = mt_raw != -INFINITY;  // this row has a valid key in the tile
       const float mt = mt_raw * cs;
       if (hf == 0) {
-        sta[(t & 3) * 128 + r] = mt;
+        // with K smoothing the NVFP4 scores miss q^ . mu, a constant of the
+        // row: the probabilities (relative to mt) do not see it, the tile's
+        // maximum handed to the correction warps does
+        sta[(t & 3) * 128 + r] = (f16 || !live) ? mt : mt + corr_r;
         mbar_arrive(&bars[B_STA + (t & 3)]);
       }
       float ls = 0.0f;

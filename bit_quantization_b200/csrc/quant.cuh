@@ -42,6 +42,18 @@ __device__ __forceinline__ void e2m1x2_roundtrip(float t0, float t1, float& q0, 
       : "f"(t0), "f"(t1));
 }
 
+// A byte of two E2M1 codes (element 2i in the low nibble) -> their values.
+__device__ __forceinline__ void e2m1x2_values(uint32_t byte, float& v0, float& v1) {
+  asm("{\n\t.reg .b8 c;\n\t.reg .b32 h;\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.u8.u32 c, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h, c;\n\t"
+      "mov.b32 {lo, hi}, h;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t"
+      "cvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(v0), "=f"(v1)
+      : "r"(byte));
+}
+
 // Block error of candidate byte S (see header comment).
 __device__ __forceinline__ double block_err(const float (&x)[16], float g, uint32_t S) {
   const float sv = ue4m3_decode(S);

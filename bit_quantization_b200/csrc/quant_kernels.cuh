@@ -297,11 +297,19 @@ __device__ __forceinline__ bool stage_tile_rows(uint4* dst, const uint16_t* src,
 // its tile (ThriftAttention, Metodologia step 1): the unrotated values summed
 // in row order from the block start, divided by the row count.  The tile is
 // read from HBM once, one bulk copy per row, into shared memory.  G = d/16.
+//
+// K smoothing (optional): with mu and without corr (K) the row's channel
+// means mu [nseq, nh, D] are subtracted (fp32) before the NVFP4 quantisation;
+// the 16-bit image and the block means keep the raw values.  With mu and
+// corr (Q) the rows are quantised as usual and corr [nseq, nh, ntiles *
+// tile_rows] receives q^ . mu of the row's kv head (head / mu_group), the
+// dequantised NVFP4 row against the means (fp32).
 template <int DT, int G, bool HAD, bool SS>
 __global__ void __launch_bounds__(256) qk_tile_kernel(
     const uint16_t* __restrict__ x, SeqInfo seqs, int nh, int tile_rows, int ntiles, int blk,
     int nB, const uint32_t* amax_in, uint8_t* __restrict__ img4, uint8_t* __restrict__ img16,
-    double* __restrict__ means) {
+    double* __restrict__ means, const float* __restrict__ mu, int mu_group,
+    float* __restrict__ corr) {
   constexpr int D = G * 16;
   extern __shared__ uint4 tsm[];  // [tile_rows][D] 16-bit values
   __shared__ __align__(8) uint64_t s_bar;
@@ -332,9 +340,31 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
       v[2 * e] = h2f<DT>((uint16_t)(w[e] & 0xFFFF));
       v[2 * e + 1] = h2f<DT>((uint16_t)(w[e] >> 16));
     }
+    const float* mrow = mu ? mu + ((int64_t)seq * (nh / mu_group) + head / mu_group) * D + kb * 16
+                           : nullptr;
+    if (mrow && !corr) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], __ldg(mrow + e));
+    }
     if constexpr (HAD) fwht_rows16<G>(v);
     uint32_t lo, hi;
     const uint32_t S = quant_block16(v, g, SS, lo, hi);
+    if (mrow && corr) {
+      // q^ . mu over the row: this block's part, then the G lanes of the row
+      float part = 0.0f;
+      const uint32_t cw[2] = {lo, hi};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float c0, c1;
+        e2m1x2_values((cw[e / 4] >> (8 * (e % 4))) & 0xFFu, c0, c1);
+        part = fmaf(c0, __ldg(mrow + 2 * e), part);
+        part = fmaf(c1, __ldg(mrow + 2 * e + 1), part);
+      }
+      part *= ue4m3_decode(S) * g;
+#pragma unroll
+      for (int o = 1; o < G; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (kb == 0) corr[((int64_t)seq * nh + head) * ((int64_t)ntiles * tile_rows) + t0 + r] = part;
+    }
     *reinterpret_cast<uint2*>(t4p + swz_offset(r, kb * 8, D / 2)) = make_uint2(lo, hi);
     sf[sf_offset(r, kb)] = (uint8_t)S;
     if (tile_rows == 64) sf[sf_offset(r + 64, kb)] = 0;
@@ -357,6 +387,65 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
           __ddiv_rn(sum, (double)(b1 - b0));
     }
   }
+}
+
+// K smoothing statistics: per (sequence, kv head, 128-token block, channel)
+// the fp64 sum of the block's values in token order, their fp32 minimum and
+// maximum.  One CTA per (block, kv head, sequence), one thread per channel.
+template <int DT>
+__global__ void __launch_bounds__(128) k_stats_kernel(const uint16_t* __restrict__ k,
+                                                      SeqInfo seqs, int Hkv, int d, int nb128,
+                                                      double* __restrict__ sums,
+                                                      float* __restrict__ mins,
+                                                      float* __restrict__ maxs) {
+  const int b = blockIdx.x, hk = blockIdx.y, seq = blockIdx.z;
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int t0 = b * 128, t1 = min(len, t0 + 128);
+  const int64_t o = (((int64_t)seq * Hkv + hk) * nb128 + b) * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    double sum = 0.0;
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) {
+      const float xv = h2f<DT>(__ldg(k + ((start + t) * Hkv + hk) * d + c));
+      sum = __dadd_rn(sum, (double)xv);
+      mn = fminf(mn, xv);
+      mx = fmaxf(mx, xv);
+    }
+    sums[o + c] = sum;
+    mins[o + c] = mn;
+    maxs[o + c] = mx;
+  }
+}
+
+// mu [nseq, Hkv, d] = the block sums added in block order / length, rounded
+// to fp32; and the absmax of K - mu folded into *amax_k: over the blocks,
+// max(fl(max - mu), fl(mu - min)) (fp32 subtraction is monotone, so this is
+// the largest |fl(k - mu)| of the block).  One CTA per (kv head, sequence).
+__global__ void __launch_bounds__(128) k_mean_kernel(const double* __restrict__ sums,
+                                                     const float* __restrict__ mins,
+                                                     const float* __restrict__ maxs,
+                                                     SeqInfo seqs, int Hkv, int d, int nb128,
+                                                     float* __restrict__ mu,
+                                                     uint32_t* __restrict__ amax_k) {
+  const int hk = blockIdx.x, seq = blockIdx.y;
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int nb = (int)ceil_div(len, 128);
+  float a = 0.0f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const int64_t o = ((int64_t)seq * Hkv + hk) * nb128 * d + c;
+    double tot = 0.0;
+    for (int b = 0; b < nb; ++b) tot = __dadd_rn(tot, sums[o + (int64_t)b * d]);
+    const float m = len > 0 ? (float)__ddiv_rn(tot, (double)len) : 0.0f;
+    mu[((int64_t)seq * Hkv + hk) * d + c] = m;
+    for (int b = 0; b < nb; ++b)
+      a = fmaxf(a, fmaxf(__fsub_rn(maxs[o + (int64_t)b * d], m), __fsub_rn(m, mins[o + (int64_t)b * d])));
+  }
+  cta_atomic_amax(a, amax_k);
 }
 
 // V ([total, Hkv, d] 16-bit) -> per (sequence, kv head, key tile) images with

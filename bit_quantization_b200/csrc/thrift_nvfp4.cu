@@ -180,6 +180,10 @@ struct AttnWs {
   double* scores;
   uint8_t* mask;
   uint8_t *q4, *k4, *v4, *q16, *k16, *v16;
+  double* ksum;      // K smoothing: block sums [nseq, Hkv, nb128, d]
+  float *kmin, *kmax;
+  float* kmu;        // channel means [nseq, Hkv, d]
+  float* qcorr;      // q^ . mu per query row [nseq, H, nTq * 128]
   size_t bytes;
 };
 
@@ -198,6 +202,12 @@ AttnWs carve_attn(void* ws, int nseq, int maxlen, int H, int Hkv, int d, int blk
   w.q16 = c.take<uint8_t>((size_t)nseq * H * nTq * f16_tile_bytes(128, d));
   w.k16 = c.take<uint8_t>((size_t)nseq * Hkv * nB * f16_tile_bytes(blk, d));
   w.v16 = c.take<uint8_t>((size_t)nseq * Hkv * nB * f16_tile_bytes(d, blk));
+  const int64_t nb128 = ceil_div(maxlen, 128);
+  w.ksum = c.take<double>((size_t)nseq * Hkv * nb128 * d * 8);
+  w.kmin = c.take<float>((size_t)nseq * Hkv * nb128 * d * 4);
+  w.kmax = c.take<float>((size_t)nseq * Hkv * nb128 * d * 4);
+  w.kmu = c.take<float>((size_t)nseq * Hkv * d * 4);
+  w.qcorr = c.take<float>((size_t)nseq * H * nTq * 128 * 4);
   w.bytes = c.off + 1024;
   return w;
 }
@@ -211,6 +221,9 @@ struct TileArgs {
   const uint32_t* amax;
   uint8_t *i4, *i16;
   double* means;
+  const float* mu = nullptr;  // K smoothing (see qk_tile_kernel)
+  int mu_group = 1;
+  float* corr = nullptr;
 };
 
 template <int DT, int G, bool HAD, bool SS>
@@ -219,7 +232,7 @@ void launch_qk_tile(const TileArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.rows * G * 16 * 2;
   qk_tile_kernel<DT, G, HAD, SS><<<grid, kThreads, smem, st>>>(
       static_cast<const uint16_t*>(a.x), a.si, a.nh, a.rows, a.ntiles, a.blk, a.nB, a.amax, a.i4,
-      a.i16, a.means);
+      a.i16, a.means, a.mu, a.mu_group, a.corr);
 }
 
 template <int DT, int G>
@@ -273,18 +286,34 @@ thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) 
 template <int DT>
 thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
                         int64_t total, int maxlen, int H, int Hkv, int d, int blk, int causal,
-                        float frac, int sink, int recent, int ss, int had, void* out, float* lse,
-                        int lse_varlen, void* ws, cudaStream_t st) {
+                        float frac, int sink, int recent, int ss, int had, int smooth, void* out,
+                        float* lse, int lse_varlen, void* ws, cudaStream_t st) {
   AttnWs w = carve_attn(ws, nseq, maxlen, H, Hkv, d, blk);
   const int nB = (int)ceil_div(maxlen, blk), nTq = (int)ceil_div(maxlen, 128);
   const int G = d / 16;
   if (cudaMemsetAsync(w.amax, 0, 16, st) != cudaSuccess) return THRIFT_ERR_CUDA;
   launch_amax<DT>(q, total * H * d / 16, had ? G : 0, w.amax + 0, st);
-  launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, w.amax + 1, st);
+  if (smooth) {
+    // K smoothing: channel means per (sequence, kv head) and the absmax of
+    // K - mu, from one pass of block statistics over K
+    const int nb128 = (int)ceil_div(maxlen, 128);
+    k_stats_kernel<DT><<<dim3(nb128, Hkv, nseq), 128, 0, st>>>(
+        static_cast<const uint16_t*>(k), si, Hkv, d, nb128, w.ksum, w.kmin, w.kmax);
+    k_mean_kernel<<<dim3(Hkv, nseq), 128, 0, st>>>(w.ksum, w.kmin, w.kmax, si, Hkv, d, nb128,
+                                                   w.kmu, w.amax + 1);
+  } else {
+    launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, w.amax + 1, st);
+  }
   launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
   // Q and K images, with the block means of the selection on the way
-  const TileArgs aq{q, si, nseq, H, 128, nTq, blk, nB, w.amax + 0, w.q4, w.q16, w.means_q};
-  const TileArgs ak{k, si, nseq, Hkv, blk, nB, blk, nB, w.amax + 1, w.k4, w.k16, w.means_k};
+  TileArgs aq{q, si, nseq, H, 128, nTq, blk, nB, w.amax + 0, w.q4, w.q16, w.means_q};
+  TileArgs ak{k, si, nseq, Hkv, blk, nB, blk, nB, w.amax + 1, w.k4, w.k16, w.means_k};
+  if (smooth) {
+    aq.mu = w.kmu;
+    aq.mu_group = H / Hkv;
+    aq.corr = w.qcorr;
+    ak.mu = w.kmu;
+  }
   if (G == 8) {
     dispatch_qk_tile<DT, 8>(had, ss, aq, st);
     dispatch_qk_tile<DT, 8>(had, ss, ak, st);
@@ -325,6 +354,7 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   p.nseq = nseq; p.H = H; p.Hkv = Hkv; p.nB = nB; p.nTq = nTq; p.causal = causal;
   p.lse_varlen = lse_varlen;
   p.total = total;
+  p.corr = smooth ? w.qcorr : nullptr;
   const double l2e = 1.4426950408889634;
   p.scale16 = (float)(l2e / std::sqrt((double)d));
   p.scale4 = (float)(l2e / std::sqrt((double)d) / (had ? (double)d : 1.0));
@@ -761,11 +791,12 @@ size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk) 
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
                               int B, int H, int Hkv, int N, int d, int blk, int causal,
                               float topk_frac, int sink_blocks, int recent_blocks,
-                              int use_scalesearch, int use_hadamard, void* out, float* lse,
-                              void* workspace, size_t ws_bytes, void* stream) {
+                              int use_scalesearch, int use_hadamard, int smooth_k, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
   thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, N, d, blk, topk_frac, out, lse);
   if (sink_blocks < 0 || recent_blocks < 0) return THRIFT_ERR_ARG;
   if (s != THRIFT_OK) return s;
+  if (smooth_k && use_hadamard) return THRIFT_ERR_UNSUPPORTED;
   if (B <= 0 || !workspace || !aligned16(workspace)) return THRIFT_ERR_ARG;
   if (ws_bytes < thrift_attn_workspace_size(B, H, Hkv, N, d, blk)) return THRIFT_ERR_ARG;
   if ((int64_t)B * ceil_div(N, 128) > 0x7FFFFFFF || B > 65535) return THRIFT_ERR_UNSUPPORTED;
@@ -774,10 +805,11 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrif
   const int64_t total = (int64_t)B * N;
   if (dt == THRIFT_BF16)
     return attn_impl<1>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac,
-                        sink_blocks, recent_blocks, use_scalesearch, use_hadamard, out, lse, 0,
-                        workspace, st);
+                        sink_blocks, recent_blocks, use_scalesearch, use_hadamard, smooth_k, out,
+                        lse, 0, workspace, st);
   return attn_impl<0>(q, k, v, si, B, total, N, H, Hkv, d, blk, causal, topk_frac, sink_blocks,
-                      recent_blocks, use_scalesearch, use_hadamard, out, lse, 0, workspace, st);
+                      recent_blocks, use_scalesearch, use_hadamard, smooth_k, out, lse, 0,
+                      workspace, st);
 }
 
 size_t thrift_attn_workspace_mask_offset(int nseq, int max_seqlen, int H, int Hkv, int d,
@@ -803,11 +835,12 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
                                      int64_t total, int max_seqlen, int H, int Hkv, int d,
                                      int blk, int causal, float topk_frac, int sink_blocks,
                                      int recent_blocks, int use_scalesearch, int use_hadamard,
-                                     void* out, float* lse, void* workspace, size_t ws_bytes,
-                                     void* stream) {
+                                     int smooth_k, void* out, float* lse, void* workspace,
+                                     size_t ws_bytes, void* stream) {
   thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, max_seqlen, d, blk, topk_frac, out, lse);
   if (sink_blocks < 0 || recent_blocks < 0) return THRIFT_ERR_ARG;
   if (s != THRIFT_OK) return s;
+  if (smooth_k && use_hadamard) return THRIFT_ERR_UNSUPPORTED;
   if (!cu_seqlens || nseq <= 0 || nseq > 65535 || total <= 0 || !workspace ||
       !aligned16(workspace))
     return THRIFT_ERR_ARG;
@@ -818,10 +851,10 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
   if (dt == THRIFT_BF16)
     return attn_impl<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal,
                         topk_frac, sink_blocks, recent_blocks, use_scalesearch, use_hadamard,
-                        out, lse, 1, workspace, st);
+                        smooth_k, out, lse, 1, workspace, st);
   return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
-                      sink_blocks, recent_blocks, use_scalesearch, use_hadamard, out, lse, 1,
-                      workspace, st);
+                      sink_blocks, recent_blocks, use_scalesearch, use_hadamard, smooth_k, out,
+                      lse, 1, workspace, st);
 }
 
 size_t thrift_kv_cache_size(int B, int Hkv, int capacity, int d, int blk) {

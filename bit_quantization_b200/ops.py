@@ -69,14 +69,14 @@ def lib():
         L.thrift_attn_workspace_size.argtypes = [i32] * 6
         L.thrift_attn_fwd.restype = i32
         L.thrift_attn_fwd.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
-                                      i32, i32, i32, P, P, P, sz, P]
+                                      i32, i32, i32, i32, P, P, P, sz, P]
         L.thrift_attn_varlen_workspace_size.restype = sz
         L.thrift_attn_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
         L.thrift_attn_workspace_mask_offset.restype = sz
         L.thrift_attn_workspace_mask_offset.argtypes = [i32, i32, i32, i32, i32, i32]
         L.thrift_attn_fwd_varlen.restype = i32
         L.thrift_attn_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
-                                             i32, f32, i32, i32, i32, i32, P, P, P, sz, P]
+                                             i32, f32, i32, i32, i32, i32, i32, P, P, P, sz, P]
         L.thrift_kernel_timer_enable.restype = i32
         L.thrift_kernel_timer_enable.argtypes = [i32]
         L.thrift_kernel_timer_read.restype = i32
@@ -268,7 +268,7 @@ def thrift_attn_workspace_size(B, H, Hkv, N, d, blk) -> int:
 
 def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesearch=False,
                     use_hadamard=False, out=None, lse=None, workspace=None, sink_blocks=0,
-                    recent_blocks=0):
+                    recent_blocks=0, smooth_k=False):
     """q [B,N,H,d], k/v [B,N,Hkv,d] -> (out [B,N,H,d], lse f32 [B,H,N])."""
     _need_cuda(q, k, v)
     B, N, H, d = q.shape
@@ -284,7 +284,8 @@ def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesear
     _check(lib().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, Hkv, N, d, blk,
                                  int(causal), float(topk_frac), int(sink_blocks),
                                  int(recent_blocks), int(use_scalesearch), int(use_hadamard),
-                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
+                                 int(smooth_k), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                 _stream(q)),
            "thrift_attn_fwd")
     return out, lse
 
@@ -301,7 +302,8 @@ def thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk) -
 
 def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True,
                            topk_frac=0.0, use_scalesearch=False, use_hadamard=False, out=None,
-                           lse=None, workspace=None, sink_blocks=0, recent_blocks=0):
+                           lse=None, workspace=None, sink_blocks=0, recent_blocks=0,
+                           smooth_k=False):
     """q [total,H,d], k/v [total,Hkv,d], cu_seqlens int32 [nseq+1] (CUDA) ->
     (out [total,H,d], lse f32 [H,total])."""
     _need_cuda(q, k, v, cu_seqlens)
@@ -322,8 +324,9 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
                                         nseq, total, int(max_seqlen), H, Hkv, d, blk,
                                         int(causal), float(topk_frac), int(sink_blocks),
                                         int(recent_blocks), int(use_scalesearch),
-                                        int(use_hadamard), _ptr(out), _ptr(lse), _ptr(ws),
-                                        ws.numel(), _stream(q)), "thrift_attn_fwd_varlen")
+                                        int(use_hadamard), int(smooth_k), _ptr(out), _ptr(lse),
+                                        _ptr(ws), ws.numel(), _stream(q)),
+           "thrift_attn_fwd_varlen")
     return out, lse
 
 

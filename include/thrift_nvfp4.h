@@ -143,6 +143,17 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
  *   out [B,N,H,d] 16-bit out;  lse [B,H,N] fp32 out (natural log).
  * The FP16 pairs are those of block_mean_topk with the same topk_frac,
  * sink_blocks and recent_blocks.
+ * smooth_k != 0: K smoothing on the NVFP4 path (the Q/K smoothing the
+ * "Attn-QAT" and "ThriftAttention" pages name among the outlier
+ * mitigations of earlier FP4 attention; the pages give no formula, this is
+ * the reading): mu = the mean of each K channel over its sequence's tokens
+ * (per kv head; fp64 sums of 128-token blocks in token order, added in block
+ * order, divided by the length, rounded to fp32) is subtracted from K before
+ * the NVFP4 quantisation (own tensor scale for K - mu), and q^ . mu (the
+ * dequantised NVFP4 query row against the means) is added back to every
+ * NVFP4 score of the row, so the two paths keep one softmax scale.  The FP16
+ * path and the selection use the raw K.  Not combined with use_hadamard
+ * (THRIFT_ERR_UNSUPPORTED).
  * Requirements: H % Hkv == 0, d in {64,128}, blk in {64,128}, N >= 1,
  * 0 <= topk_frac <= 1, sink_blocks, recent_blocks >= 0,
  * nB = ceil(N/blk) <= 512.
@@ -172,8 +183,8 @@ size_t thrift_attn_workspace_size(int B, int H, int Hkv, int N, int d, int blk);
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, thrift_dtype dt,
                               int B, int H, int Hkv, int N, int d, int blk, int causal,
                               float topk_frac, int sink_blocks, int recent_blocks,
-                              int use_scalesearch, int use_hadamard, void* out, float* lse,
-                              void* workspace, size_t ws_bytes, void* stream);
+                              int use_scalesearch, int use_hadamard, int smooth_k, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* Varlen: q [total,H,d], k, v [total,Hkv,d] packed; cu_seqlens int32
  * [nseq+1] on the DEVICE (cu_seqlens[0] = 0, cu_seqlens[nseq] = total,
@@ -188,8 +199,8 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
                                      int64_t total, int max_seqlen, int H, int Hkv, int d,
                                      int blk, int causal, float topk_frac, int sink_blocks,
                                      int recent_blocks, int use_scalesearch, int use_hadamard,
-                                     void* out, float* lse, void* workspace, size_t ws_bytes,
-                                     void* stream);
+                                     int smooth_k, void* out, float* lse, void* workspace,
+                                     size_t ws_bytes, void* stream);
 
 /* Byte offset, inside the workspace of thrift_attn_fwd (nseq = B,
  * max_seqlen = N) or thrift_attn_fwd_varlen, of the block-pair selection the

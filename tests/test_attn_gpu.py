@@ -56,21 +56,21 @@ def _compare(got, want64, what, dtype, tol=None):
 
 
 def run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, had, dtype, seed=0, k_off=3.0,
-             sink=0, recent=0):
+             sink=0, recent=0, smooth=False):
     w = synth.AttnWorkload("case", B, H, Hkv, N, d, dtype, causal, blk, frac, ss, had,
                            k_offset_std=k_off, seed=seed)
     inp = synth.make_attn_inputs(w)
     q, k, v = inp["q"], inp["k"], inp["v"]
     out, lse = ops.thrift_attn_fwd(q.cuda(), k.cuda(), v.cuda(), blk=blk, causal=causal,
                                    topk_frac=frac, use_scalesearch=ss, use_hadamard=had,
-                                   sink_blocks=sink, recent_blocks=recent)
+                                   sink_blocks=sink, recent_blocks=recent, smooth_k=smooth)
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == ops.OK
     dt = synth.dtype_code(dtype)
     cu = np.arange(B + 1, dtype=np.int32) * N
     qp, kp, vp = (synth.as_u16(t.reshape(B * N, -1, d)) for t in (q, k, v))
     r = orc.thrift_attn(qp, kp, vp, dt, cu, blk, causal, frac, use_ss=ss, use_had=had,
-                        sink_blocks=sink, recent_blocks=recent)
+                        sink_blocks=sink, recent_blocks=recent, smooth_k=smooth)
     got = out.cpu().reshape(B * N, H, d)
     gotf = got.double().numpy()
     _compare(gotf, r["out64"], "out", dtype, r["tol"])
@@ -115,14 +115,16 @@ def test_varlen_parity(orc):
     v = torch.randn((total, Hkv, d), generator=gen).to(torch.bfloat16)
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     cu_t = torch.from_numpy(cu).cuda()
-    for frac, ss, had in [(0.0, False, False), (0.25, True, True), (1.0, False, True)]:
+    for frac, ss, had, smooth in [(0.0, False, False, False), (0.25, True, True, False),
+                                  (1.0, False, True, False), (0.25, False, False, True)]:
         out, lse = ops.thrift_attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu_t, max(lens),
                                               blk=blk, causal=True, topk_frac=frac,
-                                              use_scalesearch=ss, use_hadamard=had)
+                                              use_scalesearch=ss, use_hadamard=had,
+                                              smooth_k=smooth)
         torch.cuda.synchronize()
         assert ops.device_status(reset=True) == ops.OK
         r = orc.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), 1, cu, blk, True,
-                            frac, use_ss=ss, use_had=had)
+                            frac, use_ss=ss, use_had=had, smooth_k=smooth)
         _compare(out.cpu().double().numpy(), r["out64"], f"varlen frac={frac}", torch.bfloat16,
                  r["tol"])
         assert np.max(np.abs(lse.cpu().numpy() - r["lse"])) < 1e-2
@@ -159,3 +161,40 @@ def test_deterministic():
     b = ops.thrift_attn_fwd(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), blk=64,
                             topk_frac=0.25)[0]
     assert torch.equal(a, b)
+
+
+SMOOTH_CASES = [
+    # B, N, H, Hkv, d, blk, causal, frac, ss, dtype, K channel-offset std
+    (1, 384, 2, 1, 128, 128, False, 0.0, False, torch.bfloat16, 20.0),
+    (2, 300, 4, 2, 128, 128, True, 0.25, True, torch.bfloat16, 20.0),
+    (1, 520, 2, 1, 128, 64, True, 0.1, False, torch.float16, 8.0),
+    (1, 200, 2, 2, 64, 64, False, 0.5, True, torch.bfloat16, 3.0),
+]
+
+
+@pytest.mark.parametrize("case", SMOOTH_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_k_smoothing_parity(orc, case):
+    B, N, H, Hkv, d, blk, causal, frac, ss, dtype, k_off = case
+    run_case(orc, B, N, H, Hkv, d, blk, causal, frac, ss, False, dtype, k_off=k_off, smooth=True)
+
+
+def test_k_smoothing_improves_accuracy():
+    """Under strong K channel offsets the NVFP4 path loses most of K's
+    resolution to the offset; smoothing takes it back (error against fp64
+    attention at least halved)."""
+    import oracle as orc_mod
+    w = synth.AttnWorkload("case", 1, 4, 2, 1024, 128, torch.bfloat16, True, 128, 0.1, False,
+                           False, k_offset_std=20.0, seed=3)
+    inp = synth.make_attn_inputs(w)
+    q, k, v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
+    errs = []
+    cu = np.array([0, w.N], np.int32)
+    ref, _ = orc_mod.attn_fp64(synth.as_u16(inp["q"][0]), synth.as_u16(inp["k"][0]),
+                               synth.as_u16(inp["v"][0]), 1, cu, True)
+    for smooth in (False, True):
+        out, _ = ops.thrift_attn_fwd(q, k, v, blk=128, causal=True, topk_frac=0.1,
+                                     smooth_k=smooth)
+        torch.cuda.synchronize()
+        errs.append(float(np.sqrt(np.mean((out[0].double().cpu().numpy() - ref) ** 2))))
+    assert ops.device_status(reset=True) == ops.OK
+    assert errs[1] < 0.5 * errs[0], errs

@@ -67,24 +67,27 @@ def test_bad_arguments_rejected_before_launch(L):
     # misaligned input
     assert L.nvfp4_quantize(P(4098), 0, 4, 32, 0, 0, 0, dummy, dummy, dummy, ws, qws, None) == ops.ERR_ARG
     # attention: unsupported head dim, bad GQA ratio, bad fraction, null pointer
-    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 96, 128, 0, C.c_float(0.1), 0, 0, 0, 0,
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 96, 128, 0, C.c_float(0.1), 0, 0, 0, 0, 0,
                              dummy, dummy, ws, 1 << 40, None) == ops.ERR_UNSUPPORTED
-    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 3, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0,
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 3, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0, 0,
                              dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
-    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(1.5), 0, 0, 0, 0,
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(1.5), 0, 0, 0, 0, 0,
                              dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
-    assert L.thrift_attn_fwd(None, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0,
+    assert L.thrift_attn_fwd(None, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0, 0,
                              dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
-    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0,
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0, 0, 0, 0,
                              dummy, dummy, ws, 16, None) == ops.ERR_ARG
     assert L.block_mean_topk(dummy, dummy, 0, 1, 4, 4, 256, 128, 32, 0, C.c_float(0.1), 0, 0, dummy, ws,
                              1 << 40, None) == ops.ERR_UNSUPPORTED
     assert L.thrift_attn_fwd_varlen(dummy, dummy, dummy, 1, None, 2, 100, 64, 4, 4, 128, 128, 1,
-                                    C.c_float(0.1), 0, 0, 0, 0, dummy, dummy, ws, 1 << 40,
+                                    C.c_float(0.1), 0, 0, 0, 0, 0, dummy, dummy, ws, 1 << 40,
                                     None) == ops.ERR_ARG
     # negative sink / recent block counts
     assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), -1, 0,
-                             0, 0, dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
+                             0, 0, 0, dummy, dummy, ws, 1 << 40, None) == ops.ERR_ARG
+    # K smoothing with the Hadamard rotation: not supported
+    assert L.thrift_attn_fwd(dummy, dummy, dummy, 1, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, 0,
+                             0, 1, 1, dummy, dummy, ws, 1 << 40, None) == ops.ERR_UNSUPPORTED
     assert L.block_mean_topk(dummy, dummy, 0, 1, 4, 4, 256, 128, 128, 0, C.c_float(0.1), 0, -2, dummy,
                              ws, 1 << 40, None) == ops.ERR_ARG
     # decode: unsupported head dim / tile, too many heads per kv head, bad
