@@ -435,13 +435,15 @@ def decode_only(args):
     return 0
 
 
-def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20):
+def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20,
+                      smooth=False):
     """Average attention-kernel time of the bench workload run with another
-    selection (CUDA events around each attention launch)."""
+    selection or option (CUDA events around each attention launch)."""
     def step():
         ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=frac,
                             use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
-                            out=out, lse=lse, workspace=ws, sink_blocks=sink, recent_blocks=recent)
+                            out=out, lse=lse, workspace=ws, sink_blocks=sink, recent_blocks=recent,
+                            smooth_k=smooth)
     for _ in range(3):
         step()
     torch.cuda.synchronize()
@@ -471,6 +473,51 @@ def sink_line(ops, q, k, v, w, inp, out, lse, ws, p16, sink=1, recent=1):
             "kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "achieved": achieved,
             "unit": "TFLOP/s", "fp16_share": f16 / (f4 + f16),
             "frac": (t_ideal / (k_ms * 1e-3))}
+
+
+def smoothing_line(ops, q, k, v, w, out, lse, ws, steps=20, nrows=64):
+    """K smoothing on the bench workload: the attention kernel's and the whole
+    step's time with it, and the error of both variants against fp64
+    attention (torch, on the GPU) on a sample of output rows."""
+    dev = q.device
+    k_ms = variant_kernel_ms(ops, q, k, v, w, out, lse, ws, w.topk_frac, smooth=True)
+
+    def step_ms(smooth):
+        for _ in range(3):
+            ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
+                                out=out, lse=lse, workspace=ws, smooth_k=smooth)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
+                                out=out, lse=lse, workspace=ws, smooth_k=smooth)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    gen = torch.Generator().manual_seed(11)
+    rows = torch.randint(0, w.N, (nrows,), generator=gen).tolist()
+    heads = torch.randint(0, w.H, (nrows,), generator=gen).tolist()
+    g = w.H // w.Hkv
+    err = {}
+    for smooth in (False, True):
+        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac, out=out,
+                            lse=lse, workspace=ws, smooth_k=smooth)
+        torch.cuda.synchronize(dev)
+        se = 0.0
+        for t, h in zip(rows, heads):
+            qr = q[0, t, h].double()
+            kk = k[0, : (t + 1 if w.causal else w.N), h // g].double()
+            vv = v[0, : kk.shape[0], h // g].double()
+            p = torch.softmax(kk @ qr / (w.d ** 0.5), dim=0)
+            se += float(((out[0, t, h].double() - p @ vv) ** 2).sum())
+        err["on" if smooth else "off"] = (se / (nrows * w.d)) ** 0.5
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out (smoothing)")
+    return {"kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "step_ms": step_ms(True),
+            "step_ms_without": step_ms(False),
+            "rms_err_vs_fp64": err, "sample": f"{nrows} (token, head) rows of batch entry 0",
+            "reference": "torch fp64 softmax(q K^T / sqrt(d)) V of the 16-bit inputs"}
 
 
 def nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4, steps=20):
@@ -684,6 +731,8 @@ def main():
     if rank == 0 and world == 1:
         line["nvfp4_only"] = nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4)
         line["sink_aware"] = sink_line(ops, q, k, v, w, inp, out, lse, ws, p16)
+        if not w.use_hadamard:
+            line["k_smoothing"] = smoothing_line(ops, q, k, v, w, out, lse, ws)
     if rank == 0 and world == 1 and not args.no_quantizer:
         line["quantizer"] = quantizer_line(dev, peaks)
     if rank == 0 and world == 1 and not args.no_decode:
