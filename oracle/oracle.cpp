@@ -57,6 +57,15 @@
 //      scores q^ . (k'^ + mu), i.e. the dequantised smoothed key with the
 //      mean added back, so both paths keep the same scores; the FP16 path and
 //      the selection use the raw K.  Not combined with the Hadamard rotation.
+//  R17 Attn-QAT backward ("Attn-QAT", Metodologia A and B): the forward
+//      runs on fake-quantised NVFP4 Q^, K^, V^ (dequantised values) with the
+//      probabilities quantised in two levels per (row, key tile) as in R7;
+//      the backward treats every quantiser as the identity for gradients
+//      (straight-through), recomputes P = exp(S - lse) and its FP4 image P^
+//      from the same scales, and takes the scalar of the softmax gradient
+//      from a high-precision output O' = P V^ (not from the FP4 output
+//      O = P^ V^):  D = rowsum(dO o O'),  dV = P^T^ dO,  dP = dO V^T^,
+//      dS = P o (dP - D),  dQ = dS K^ / sqrt(d),  dK = dS^T Q^ / sqrt(d).
 //  R15 decode on the double cache (ThriftAttention, Resultados: decode
 //      speed-up; Significado: the KV cache grows by 28% because every token
 //      is cached in FP16 and in FP4): one new query token per sequence
@@ -1200,6 +1209,179 @@ int orc_thrift_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
   parallel_for((int64_t)B * H, nthreads, [&](int64_t u) {
     decode_row(C, (int)(u / H), (int)(u % H), out, lse, out64, tol);
   });
+  return 0;
+}
+
+// ------------------------------------------------ Attn-QAT backward --
+//
+// Reading R17.  q [total, H, d], k, v [total, Hkv, d], dout [total, H, d]
+// 16-bit over packed sequences cu [nseq+1]; blk = key tile of the P
+// quantisation.  Outputs (fp64): o (the FP4 forward output P^ V^), o_hp
+// (O' = P V^), lse [H, total] (natural log), dq [total, H, d], dk, dv
+// [total, Hkv, d] (summed over the query heads of a kv head).
+int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     const uint16_t* dout, int dt, int H, int Hkv, const int32_t* cu, int nseq,
+                     int d, int blk, int causal, int use_ss, int nthreads, double* o,
+                     double* o_hp, double* lse, double* dq, double* dk, double* dv) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
+  const int64_t total = cu[nseq];
+  std::vector<uint8_t> qc, qs, kc, ks, vc, vs;
+  const float gq = quantize_rows_unpacked(q, dt, total * H, d, use_ss, 0, nthreads, qc, qs);
+  const float gk = quantize_rows_unpacked(k, dt, total * Hkv, d, use_ss, 0, nthreads, kc, ks);
+  // V: 16-blocks along the tokens of each sequence (zero-padded), reading R6
+  std::vector<int64_t> pst(nseq + 1, 0);
+  for (int s = 0; s < nseq; ++s) {
+    const int len = cu[s + 1] - cu[s];
+    if (len <= 0) return -1;
+    pst[s + 1] = pst[s] + (len + 15) / 16 * 16;
+  }
+  const int64_t ptot = pst[nseq];
+  float vamax = 0.0f;
+  for (int64_t e = 0; e < total * Hkv * d; ++e) vamax = std::max(vamax, std::fabs(orc_half_to_float(v[e], dt)));
+  const float gv = vamax == 0.0f ? 1.0f : vamax / 2688.0f;
+  std::vector<uint8_t> vcol((size_t)(Hkv * d * ptot), 0), vsc((size_t)(Hkv * d * ptot / 16), 0);
+  for (int64_t hc = 0; hc < (int64_t)Hkv * d; ++hc) {
+    const int64_t hk = hc / d, c = hc % d;
+    float col[16];
+    uint8_t packed[8];
+    for (int s = 0; s < nseq; ++s) {
+      const int len = cu[s + 1] - cu[s];
+      for (int64_t t0 = 0; t0 < pst[s + 1] - pst[s]; t0 += 16) {
+        for (int e = 0; e < 16; ++e)
+          col[e] = t0 + e < len ? orc_half_to_float(v[((cu[s] + t0 + e) * Hkv + hk) * d + c], dt) : 0.0f;
+        const int64_t base = hc * ptot + pst[s] + t0;
+        orc_quant_block(col, gv, use_ss, packed, &vsc[(size_t)(base / 16)], nullptr);
+        for (int e = 0; e < 8; ++e) {
+          vcol[(size_t)(base + 2 * e)] = packed[e] & 0xF;
+          vcol[(size_t)(base + 2 * e + 1)] = packed[e] >> 4;
+        }
+      }
+    }
+  }
+  auto qhat = [&](int64_t t, int h, int c) {
+    const int64_t e = (t * H + h) * d + c;
+    return deq(qc[(size_t)e], qs[(size_t)(e / 16)], gq);
+  };
+  auto khat = [&](int64_t t, int hk, int c) {
+    const int64_t e = (t * Hkv + hk) * d + c;
+    return deq(kc[(size_t)e], ks[(size_t)(e / 16)], gk);
+  };
+  std::vector<int> seq_of((size_t)total);
+  for (int s = 0; s < nseq; ++s)
+    for (int64_t t = cu[s]; t < cu[s + 1]; ++t) seq_of[(size_t)t] = s;
+  auto vhat = [&](int64_t t, int hk, int c) {
+    const int s = seq_of[(size_t)t];
+    const int64_t ve = ((int64_t)hk * d + c) * ptot + pst[s] + (t - cu[s]);
+    return deq(vcol[(size_t)ve], vsc[(size_t)(ve / 16)], gv);
+  };
+  for (int64_t e = 0; e < total * Hkv * d; ++e) dk[e] = dv[e] = 0.0;
+  const double sc = 1.0 / std::sqrt((double)d);
+  // one (sequence, head) at a time: the kv-head gradients of different
+  // heads add into the same rows, so heads run in order
+  for (int s = 0; s < nseq; ++s) {
+    const int64_t st = cu[s];
+    const int len = cu[s + 1] - cu[s];
+    for (int h = 0; h < H; ++h) {
+      const int hk = h / (H / Hkv);
+      std::vector<double> P((size_t)len * len, 0.0), Ph((size_t)len * len, 0.0);
+      parallel_for(len, nthreads, [&](int64_t i) {
+        const int kend = causal ? (int)i + 1 : len;
+        std::vector<double> srow(len, -INFINITY);
+        double mx = -INFINITY;
+        for (int j = 0; j < kend; ++j) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += qhat(st + i, h, c) * khat(st + j, hk, c);
+          srow[j] = acc * sc;
+          mx = std::max(mx, srow[j]);
+        }
+        double den = 0.0;
+        for (int j = 0; j < kend; ++j) den += std::exp(srow[j] - mx);
+        const double lz = mx + std::log(den);
+        lse[(int64_t)h * total + st + i] = lz;
+        for (int j = 0; j < kend; ++j) P[(size_t)i * len + j] = std::exp(srow[j] - lz);
+        // P^: two-level FP4 image per key tile (reading R7 on the normalised row)
+        for (int j0 = 0; j0 < kend; j0 += blk) {
+          const int j1 = std::min(kend, j0 + blk);
+          std::vector<float> pt(blk, 0.0f);
+          float rowmax = 0.0f;
+          for (int j = j0; j < j1; ++j) {
+            pt[j - j0] = (float)P[(size_t)i * len + j];
+            rowmax = std::max(rowmax, pt[j - j0]);
+          }
+          if (rowmax == 0.0f) continue;
+          const float inv = 2688.0f / rowmax, sigma = rowmax / 2688.0f;
+          for (int b0 = 0; b0 < blk; b0 += 16) {
+            float ph[16], amax = 0.0f;
+            for (int e = 0; e < 16; ++e) {
+              ph[e] = pt[b0 + e] * inv;
+              amax = std::max(amax, ph[e]);
+            }
+            const uint8_t sp = orc_ue4m3_encode(amax / 6.0f);
+            const float dec = orc_ue4m3_decode(sp);
+            const float rr = 1.0f / dec;
+            for (int e = 0; e < 16; ++e) {
+              const int j = j0 + b0 + e;
+              if (j >= j1 || sp == 0) continue;
+              Ph[(size_t)i * len + j] = (double)orc_e2m1_decode(orc_e2m1_encode(ph[e] * rr)) *
+                                        (double)dec * (double)sigma;
+            }
+          }
+        }
+      });
+      // outputs, D, dP, dS and the gradients of this head
+      parallel_for(len, nthreads, [&](int64_t i) {
+        const int64_t ti = st + i;
+        std::vector<double> oh(d, 0.0), ohp(d, 0.0);
+        for (int j = 0; j < len; ++j) {
+          const double p = P[(size_t)i * len + j], ph = Ph[(size_t)i * len + j];
+          if (p == 0.0 && ph == 0.0) continue;
+          for (int c = 0; c < d; ++c) {
+            const double vv = vhat(st + j, hk, c);
+            oh[c] += ph * vv;
+            ohp[c] += p * vv;
+          }
+        }
+        double D = 0.0;
+        for (int c = 0; c < d; ++c) {
+          o[(ti * H + h) * d + c] = oh[c];
+          o_hp[(ti * H + h) * d + c] = ohp[c];
+          D += (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt) * ohp[c];
+        }
+        std::vector<double> dqr(d, 0.0);
+        for (int j = 0; j < len; ++j) {
+          const double p = P[(size_t)i * len + j];
+          if (p == 0.0) continue;
+          double dp = 0.0;
+          for (int c = 0; c < d; ++c)
+            dp += (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt) * vhat(st + j, hk, c);
+          const double ds = p * (dp - D);
+          for (int c = 0; c < d; ++c) dqr[c] += ds * khat(st + j, hk, c) * sc;
+        }
+        for (int c = 0; c < d; ++c) dq[(ti * H + h) * d + c] = dqr[c];
+      });
+      // dK, dV rows of this head: key j sums over the queries
+      parallel_for(len, nthreads, [&](int64_t j) {
+        const int64_t tj = st + j;
+        for (int64_t i = 0; i < len; ++i) {
+          const double p = P[(size_t)i * len + j], ph = Ph[(size_t)i * len + j];
+          if (p == 0.0 && ph == 0.0) continue;
+          const int64_t ti = st + i;
+          double dp = 0.0, D = 0.0;
+          for (int c = 0; c < d; ++c) {
+            const double g = (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt);
+            dp += g * vhat(tj, hk, c);
+            D += g * o_hp[(ti * H + h) * d + c];
+          }
+          const double ds = p * (dp - D);
+          for (int c = 0; c < d; ++c) {
+            const double g = (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt);
+            dv[(tj * Hkv + hk) * d + c] += ph * g;
+            dk[(tj * Hkv + hk) * d + c] += ds * qhat(ti, h, c) * sc;
+          }
+        }
+      });
+    }
+  }
   return 0;
 }
 
