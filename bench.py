@@ -391,12 +391,35 @@ def decode_line(ops, dev, peaks, steps=50, warmup=5):
         raise RuntimeError("device wait timed out in the decode loop")
     step_us = 1e3 * e0.elapsed_time(e1) / steps
     k_us = 1e3 * kms / max(nk, 1)
+    # the same step replayed from a CUDA graph (one capture, no per-kernel
+    # launch cost), the way a serving loop runs a fixed-shape decode step
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    graph_us = 1e3 * e0.elapsed_time(e1) / steps
+    del graph
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the decode graph")
     t4, t16, kv_bytes = decode_tiles(ops, w, ws, L0)
     achieved = kv_bytes / (k_us * 1e-6) / 1e9
     hbm = peaks["hbm_gbs"]
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "d": w.d,
             "cached_tokens": L0, "attended_tokens": L0 + 1, "topk_frac": w.topk_frac,
-            "us_per_step": step_us, "steps": steps,
+            "us_per_step": step_us, "us_per_step_graph": graph_us, "steps": steps,
             "step": "append one token per sequence to the FP4 + 16-bit cache, then attend",
             "kernel_us": k_us, "tiles_nvfp4": t4, "tiles_fp16": t16,
             "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel", "achieved": achieved,
