@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from bit_quantization_b200 import synth  # noqa: E402
+from bit_quantization_b200 import dist, synth  # noqa: E402
 
 WORKLOADS = {
     "b2h32n8192": synth.C_B2H32N8K,
@@ -151,17 +151,6 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    return world, rank, local
-
-
 def oracle_sample(w, nunits, nthreads, inp=None):
     """The CPU oracle on a bounded sample of the workload: one head of batch
     entry 0 (full sequence length), `nunits` evenly spread query blocks.
@@ -193,9 +182,9 @@ def oracle_sample(w, nunits, nthreads, inp=None):
 
 
 def run_reference(args, w):
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    world, rank, _ = dist.env()
     if rank != 0:
-        return 0
+        return 0  # the CPU reference runs once, on rank 0
     cores = os.cpu_count() or 1
     inp = synth.make_attn_inputs(w)
     # Size the sample so the whole run stays within about two minutes.
@@ -593,12 +582,12 @@ def main():
         return decode_only(args)
 
     from bit_quantization_b200 import ops
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist.setup("nccl")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
 
-    inp = synth.make_attn_inputs(w, seed=w.seed + rank)
+    inp = synth.make_attn_inputs(w, seed=dist.rank_seed(w.seed, rank))
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -622,8 +611,7 @@ def main():
         raise RuntimeError("device wait timed out during warm-up")
 
     sampler = ClockSampler(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier(world)
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
@@ -636,18 +624,15 @@ def main():
     torch.cuda.synchronize(dev)
     ops.kernel_timer_enable(False)
     clocks = sampler.stop()
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier(world)
     ms_total = e0.elapsed_time(e1)
     kms, klaunches = ops.kernel_timer_read()
     if ops.device_status(reset=True) != ops.OK:
         raise RuntimeError("device wait timed out during the timed region")
-    t = torch.tensor([ms_total, kms / max(klaunches, 1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_total, k_ms = float(t[0]), float(t[1])
+    ms_total, k_ms = dist.max_over_ranks([ms_total, kms / max(klaunches, 1)], world)
     ms_step = ms_total / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    job_flops = dist.sum_over_ranks([flops], world)[0]
+    value = dist.whole_job_rate(job_flops, ms_step) / 1e12
 
     # End to end through the public API with host buffers: every step copies
     # its Q, K, V from pinned host memory and reads its output and LSE back.
@@ -695,8 +680,7 @@ def main():
 
     e2e_run(2)
     torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier(world)
     torch.cuda.synchronize(dev)
     e0.record()
     e2e_run(e2e_steps)
@@ -706,10 +690,7 @@ def main():
     torch.cuda.synchronize(dev)
     if ops.device_status(reset=True) != ops.OK:
         raise RuntimeError("device wait timed out in the end-to-end loop")
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(te[0]) / e2e_steps
+    e2e_ms = dist.max_over_ranks([e0.elapsed_time(e1)], world)[0] / e2e_steps
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = outh[0].numel() * outh[0].element_size() + lseh[0].numel() * lseh[0].element_size()
 
@@ -746,7 +727,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
             "data": "synthetic", "config": config_of(w), "roofline": roofline,
             "alu_roofline": alu_roofline,
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "e2e": {"value": dist.whole_job_rate(job_flops, e2e_ms) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "pipelining": "inputs of step s+1 and results of step s-1 copied while "
                                   "step s computes (two buffer sets, three streams)"},
@@ -767,8 +748,7 @@ def main():
         dt, fl, desc = oracle_sample(w, args.ref_units, cores, inp)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores,
                                 "kind": "oracle", "sample": desc, "seconds": dt}
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    dist.teardown(world)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
