@@ -15,7 +15,7 @@
 // 16-bit) per kv head group, the block scores q . kbar_j and a top-k per
 // (sequence, head), then the attention kernel (split over the key tiles,
 // tensor cores with the key tile as the 128-row operand and the query group
-// as the 64-column one), and a merge of the splits.
+// as the 16-column one), and a merge of the splits.
 #pragma once
 
 #include "attn.cuh"
@@ -28,6 +28,7 @@ namespace thrift {
 constexpr int kDecTile = 128;  // tokens per key tile (= selection block)
 constexpr int kDecD = 128;     // head dimension
 constexpr int kDecMaxG = 16;   // query heads per kv head
+constexpr int kDecN = 16;      // MMA N: query columns of the S and O buffers (>= kDecMaxG)
 
 struct CacheGeom {
   int B, Hkv, ntc;  // key tiles per (sequence, kv head)
@@ -360,7 +361,8 @@ __global__ void __launch_bounds__(kDecD) dec_combine_kernel(const float* __restr
 //
 // One CTA per (split of the key tiles, kv head, sequence).  Tensor cores
 // compute S^T = K Q^T with the key tile as the 128-row A operand and the G
-// query heads of the group as the B operand (64 rows, G used), and
+// query heads of the group as the B operand (N = 16 rows of a 64-row image,
+// G used), and
 // O^T += V^T P^T with the 128 channels as A and the probability rows as B.
 // The key tiles whose heads all run on one path are read once per CTA in
 // that format; a tile some heads take in NVFP4 and others in FP16 is read in
@@ -444,29 +446,30 @@ struct DecLayout {
   static constexpr uint32_t OFF_BAR = OFF_COEF + 2 * 4 * kDecMaxG * 2 * 4;
   static constexpr uint32_t BYTES = OFF_BAR + 512;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
-  // tensor-memory columns
-  static constexpr uint32_t T_S = 0;      // + 64 g
-  static constexpr uint32_t T_O = 128;    // + 64 (2 g + slot)
-  static constexpr uint32_t T_QSF = 384;  // + 8 g (two K-steps of 4 columns)
-  static constexpr uint32_t T_KSF = 400;  // + 8 g
-  static constexpr uint32_t T_PSF = 416;  // + 8 g
-  static constexpr uint32_t T_VSF = 432;  // + 8 g
+  // tensor-memory columns (N = kDecN query columns per S or O buffer)
+  static constexpr uint32_t T_S = 0;      // + kDecN (2 g + slot)
+  static constexpr uint32_t T_O = 64;     // + kDecN (2 g + slot)
+  static constexpr uint32_t T_QSF = 128;  // + 8 g (two K-steps of 4 columns)
+  static constexpr uint32_t T_KSF = 144;  // + 8 g
+  static constexpr uint32_t T_PSF = 160;  // + 8 g
+  static constexpr uint32_t T_VSF = 176;  // + 8 g
+  static constexpr uint32_t T_COLS = 256;  // allocation
   static_assert(NS4 == 8, "barrier plan assumes eight NVFP4 stages");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-// Barriers.  Per group g: SF/SE its S buffer full (QK commit) / read;
-// GB the group's own barrier (one phase per tile).  Per group g and slot s
-// (tile t of the group uses slot (t >> 1) & 1): PF its P tile written, OD
-// its PV retired into O buffer s, OE O buffer s folded (free again).  A
+// Barriers.  GB: per group g, the group's own barrier (one phase per tile).
+// Per group g and slot s (tile t of the group uses slot (t >> 1) & 1): SF /
+// SE S buffer s full (QK commit) / read, PF its P tile written, OD its PV
+// retired into O buffer s, OE O buffer s folded (free again).  A
 // barrier of a slot only completes its next phase after its waiter has
 // passed the previous one: the slot's next PV waits OE, whose fold waited
 // OD; the slot's next P waits for that fold (or for OD, FP16).
 enum : int {
-  D_Q4 = 0, D_Q16 = 1, D_SF = 2 /* 2,3 */, D_SE = 4 /* 4,5 */, D_PF = 6 /* 6..9 */,
-  D_OD = 10 /* 10..13 */, D_OE = 14 /* 14..17 */, D_GB = 18 /* 18,19 */, D_P4DONE = 20,
-  D_DONE = 21, D_KVF16 = 22 /* 22,23 */, D_KVE16 = 24 /* 24,25 */, D_KVF4 = 26 /* 26..33 */,
-  D_KVE4 = 34 /* 34..41 */, D_N = 42
+  D_Q4 = 0, D_Q16 = 1, D_SF = 2 /* 2..5 */, D_SE = 6 /* 6..9 */, D_PF = 10 /* 10..13 */,
+  D_OD = 14 /* 14..17 */, D_OE = 18 /* 18..21 */, D_GB = 22 /* 22,23 */, D_P4DONE = 24,
+  D_DONE = 25, D_KVF16 = 26 /* 26,27 */, D_KVE16 = 28 /* 28,29 */, D_KVF4 = 30 /* 30..37 */,
+  D_KVE4 = 38 /* 38..45 */, D_N = 46
 };
 
 // warps 0..7 softmax (two groups), 8 producer, 9 + g the QK^T issuer of
@@ -513,7 +516,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
   if (tid == 0) {
     for (int i = 0; i < D_N; ++i) {
       uint32_t cnt = 1;
-      if ((i >= D_SE && i < D_SE + 2) || (i >= D_PF && i < D_PF + 4) ||
+      if ((i >= D_SE && i < D_SE + 4) || (i >= D_PF && i < D_PF + 4) ||
           (i >= D_OE && i < D_OE + 4) || (i >= D_GB && i < D_GB + 2))
         cnt = 128;
       if (i == D_DONE) cnt = 4;     // one commit per MMA issuer
@@ -563,7 +566,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
   }
   __syncthreads();
   if (warp == kDecQkWarp) {
-    tmem_alloc(s_tmem, 512);
+    tmem_alloc(s_tmem, L::T_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -640,7 +643,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     if (lane == 0) {
       const bool is_qk = warp < kDecPvWarp;
       const int g = is_qk ? warp - kDecQkWarp : warp - kDecPvWarp;
-      constexpr uint32_t id4 = idesc_nvf4(128, 64), id16 = idesc_f16(DT, 128, 64);
+      constexpr uint32_t id4 = idesc_nvf4(128, kDecN), id16 = idesc_f16(DT, 128, kDecN);
       const uint32_t base = smem_u32(sm);
       const uint64_t d_sf = make_sdesc(base, 512, 128, SW_NONE);  // + (byte offset >> 4)
       // operands of 64-byte rows (NVFP4, K = 128 elements) and of 128-byte
@@ -674,7 +677,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             if (!mbar_wait(&bars[D_Q16], 0, s_abort)) { ok = false; break; }
             q16_ready = true;
           }
-          const uint32_t dS = tmem + L::T_S + 64 * g;
+          const uint32_t dS = tmem + L::T_S + kDecN * (2 * g + (u & 1));
           if (!f16) {
             // scale factors first: they wait only for the stage (the slot's
             // previous reader, QK(t - 2), was issued earlier by this thread)
@@ -690,14 +693,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
               tc_cp_32x128b_x4(ksf + 4 * s2, d_sf + ((stg + kDecTile * (kDecD / 2) + 512 * s2) >> 4));
-            if (u >= 1 && !mbar_wait(&bars[D_SE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+            if (u >= 2 && !mbar_wait(&bars[D_SE + 2 * g + (u & 1)], ((u >> 1) - 1) & 1, s_abort)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
               mma_nvf4(dS, d4 + (stg >> 4) + 2 * s2, d4 + (L::OFF4_Q >> 4) + 2 * s2, id4,
                        ksf + 4 * s2, qsf + 4 * s2, s2 > 0);
           } else {
-            if (u >= 1 && !mbar_wait(&bars[D_SE + g], (u - 1) & 1, s_abort)) { ok = false; break; }
+            if (u >= 2 && !mbar_wait(&bars[D_SE + 2 * g + (u & 1)], ((u >> 1) - 1) & 1, s_abort)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t stg = L::OFF16_STG + sl * L::STG16;
 #pragma unroll
@@ -705,7 +714,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
               mma_f16(dS, d16 + ((stg + (kk / 4) * 128 * 128) >> 4) + 2 * (kk % 4),
                       d16 + ((L::OFF16_Q + (kk / 4) * 64 * 128) >> 4) + 2 * (kk % 4), id16, kk > 0);
           }
-          tc_commit(&bars[D_SF + g]);
+          tc_commit(&bars[D_SF + 2 * g + (u & 1)]);
         }
       } else {
         const uint32_t vsf = tmem + L::T_VSF + 8 * g, psf = tmem + L::T_PSF + 8 * g;
@@ -739,7 +748,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
             break;
           }
           tc_fence_after();
-          const uint32_t dO = tmem + L::T_O + 64 * (2 * g + sl2);
+          const uint32_t dO = tmem + L::T_O + kDecN * (2 * g + sl2);
           if (!f16) {
             const uint32_t stg = L::OFF4_STG + sl * L::STG4 + CacheGeom::K4;
             const uint32_t pp = L::OFF4_P + (2 * g + sl2) * dec_align(L::P4B);
@@ -781,8 +790,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     float* sT0 = reinterpret_cast<float*>(sm + L::OFF_ST) + g * 2 * (L::ST_BYTES / 4);
     float* coef = reinterpret_cast<float*>(sm + L::OFF_COEF) + g * (4 * kDecMaxG * 2);
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-    const uint32_t s_addr = lane_base + L::T_S + 64 * g;
-    const uint32_t o_addr = lane_base + L::T_O + 64 * (2 * g);  // + 64 slot
+    const uint32_t s_addr = lane_base + L::T_S + kDecN * (2 * g);  // + kDecN slot
+    const uint32_t o_addr = lane_base + L::T_O + kDecN * (2 * g);  // + kDecN slot
     uint8_t* p4g = sm + L::OFF4_P + 2 * g * dec_align(L::P4B);   // + slot * P4 slot
     uint8_t* p16 = sm + L::OFF16_P + g * L::P16B;
     // work item of this thread: keys [16 bb + KPL hb, + KPL) of head c, the
@@ -820,7 +829,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
     auto fold_issue = [&](int v) -> bool {
       if (!warp_wait(&bars[D_OD + 2 * g + (v & 1)], (v >> 1) & 1, s_abort)) return false;
       tc_fence_after();
-      tmem_ld_cols<GC>(o_addr + 64 * (v & 1), o);
+      tmem_ld_cols<GC>(o_addr + kDecN * (v & 1), o);
       return true;
     };
     auto fold_finish = [&](int v) {
@@ -851,18 +860,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
       }
       float* sT = sT0 + (u & 1) * (L::ST_BYTES / 4);
       // A: scores of key i for the group's heads -> transposed tile
-      if (!warp_wait(&bars[D_SF + g], u & 1, s_abort)) { ok = false; break; }
+      if (!warp_wait(&bars[D_SF + 2 * g + (u & 1)], (u >> 1) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
       {
         float a[GC];
-        tmem_ld_cols<GC>(s_addr, a);
+        tmem_ld_cols<GC>(s_addr + kDecN * (u & 1), a);
         tmem_ld_wait();
         const bool valid = j * kDecTile + i < len;
 #pragma unroll
         for (int k = 0; k < GC; ++k) sT[k * L::ST_PITCH + i] = valid ? a[k] : -INFINITY;
       }
       tc_fence_before();
-      mbar_arrive(&bars[D_SE + g]);
+      mbar_arrive(&bars[D_SE + 2 * g + (u & 1)]);
       mbar_arrive(&bars[D_GB + g]);
       if (!warp_wait(&bars[D_GB + g], u & 1, s_abort)) { ok = false; break; }
       // E (first half): PV(t - 2) retired (the single FP16 P buffer is then
@@ -1010,7 +1019,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const DecPa
   __syncthreads();
   if (warp == kDecQkWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, L::T_COLS);
   }
 }
 
