@@ -290,7 +290,7 @@ DECODE_KERNELS_PER_STEP = 7  # append (2), query images (absmax fused), scores, 
 # DRAM traffic per algorithmic byte of the decode kernel, measured by ncu on
 # the 32768-token case of the decode workload (the traffic scales with the
 # tiles read); reported only while the decode source is unchanged since.
-DECODE_TRAFFIC = {"src_sha16": "7733001a3f2a47e2", "bytes_per_algorithmic_byte": 344.29 / 338.72,
+DECODE_TRAFFIC = {"src_sha16": "a565554521ecf748", "bytes_per_algorithmic_byte": 344.61 / 338.72,
                   "captured_on": "decode workload with 32768 cached tokens"}
 
 
