@@ -78,7 +78,7 @@ def lib():
         L.orc_k_channel_means.argtypes = [P, i32, i32, P, i32, i32, P]
         L.orc_attn_qat_bwd.restype = i32
         L.orc_attn_qat_bwd.argtypes = [P, P, P, P, i32, i32, i32, P, i32, i32, i32, i32, i32, i32,
-                                       P, P, P, P, P, P]
+                                       P, P, P, P, P, P, P]
         L.orc_thrift_decode.restype = i32
         L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
                                         i32, i32, i32, P, i32, P, i32, P, P, P, P, P]
@@ -383,10 +383,12 @@ def thrift_decode(q, k, v, dt, lens, blk, g_kv, frac, use_ss=False, sink_blocks=
 
 # ---------------------------------------------------------- Attn-QAT bwd
 
-def attn_qat_bwd(q, k, v, dout, dt, cu, blk, causal, use_ss=False, nthreads=None):
+def attn_qat_bwd(q, k, v, dout, dt, cu, blk, causal, use_ss=False, nthreads=None, g=None):
     """Attn-QAT forward outputs and gradients (reading R17 of oracle.cpp).
 
     q, dout [total,H,d], k, v [total,Hkv,d] uint16; cu int32 [nseq+1].
+    g: optional tensor scales (gq, gk, gv) to use instead of those of the
+    given tensors (a slice of a larger problem keeps the whole tensors').
     Returns dict(o, o_hp [total,H,d], lse [H,total], dq [total,H,d],
     dk, dv [total,Hkv,d]), all fp64."""
     q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
@@ -399,8 +401,10 @@ def attn_qat_bwd(q, k, v, dout, dt, cu, blk, causal, use_ss=False, nthreads=None
     dq = np.zeros((total, H, d))
     dk = np.zeros((total, Hkv, d))
     dv = np.zeros((total, Hkv, d))
+    garr = None if g is None else np.ascontiguousarray(g, np.float32)
     rc = lib().orc_attn_qat_bwd(_p(q), _p(k), _p(v), _p(dout), dt, H, Hkv, _p(cu), len(cu) - 1, d,
                                 blk, int(causal), int(use_ss), int(nthreads or nthreads_default()),
+                                _p(garr) if garr is not None else None,
                                 _p(o), _p(o_hp), _p(lse), _p(dq), _p(dk), _p(dv))
     if rc:
         raise ValueError("oracle attn_qat_bwd: bad arguments")

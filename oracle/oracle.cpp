@@ -518,7 +518,8 @@ static void parallel_for(int64_t n, int nthreads, const std::function<void(int64
 // attention emulation below.  Same arithmetic as orc_nvfp4_quantize.
 static float quantize_rows_unpacked(const uint16_t* x, int dt, int64_t rows, int cols,
                                     int use_ss, int hadamard, int nthreads,
-                                    std::vector<uint8_t>& codes, std::vector<uint8_t>& scales) {
+                                    std::vector<uint8_t>& codes, std::vector<uint8_t>& scales,
+                                    const float* g_given = nullptr) {
   const int64_t chunk = 4096;
   const int64_t nchunks = (rows + chunk - 1) / chunk;
   std::vector<float> part(nchunks, 0.0f);
@@ -534,7 +535,7 @@ static float quantize_rows_unpacked(const uint16_t* x, int dt, int64_t rows, int
   });
   float amax = 0.0f;
   for (float a : part) amax = std::max(amax, a);
-  const float g = amax == 0.0f ? 1.0f : amax / 2688.0f;
+  const float g = g_given ? *g_given : (amax == 0.0f ? 1.0f : amax / 2688.0f);
   codes.assign((size_t)(rows * cols), 0);
   scales.assign((size_t)(rows * (cols / 16)), 0);
   parallel_for(nchunks, nthreads, [&](int64_t c) {
@@ -1218,16 +1219,21 @@ int orc_thrift_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
 // 16-bit over packed sequences cu [nseq+1]; blk = key tile of the P
 // quantisation.  Outputs (fp64): o (the FP4 forward output P^ V^), o_hp
 // (O' = P V^), lse [H, total] (natural log), dq [total, H, d], dk, dv
-// [total, Hkv, d] (summed over the query heads of a kv head).
+// [total, Hkv, d] (summed over the query heads of a kv head).  g_in
+// (optional, 3 floats): the tensor scales of Q, K, V to use instead of those
+// of the given tensors (a slice of a larger problem keeps the whole tensor's
+// scales, reading C3).
 int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      const uint16_t* dout, int dt, int H, int Hkv, const int32_t* cu, int nseq,
-                     int d, int blk, int causal, int use_ss, int nthreads, double* o,
-                     double* o_hp, double* lse, double* dq, double* dk, double* dv) {
+                     int d, int blk, int causal, int use_ss, int nthreads, const float* g_in,
+                     double* o, double* o_hp, double* lse, double* dq, double* dk, double* dv) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
   const int64_t total = cu[nseq];
   std::vector<uint8_t> qc, qs, kc, ks, vc, vs;
-  const float gq = quantize_rows_unpacked(q, dt, total * H, d, use_ss, 0, nthreads, qc, qs);
-  const float gk = quantize_rows_unpacked(k, dt, total * Hkv, d, use_ss, 0, nthreads, kc, ks);
+  const float gq = quantize_rows_unpacked(q, dt, total * H, d, use_ss, 0, nthreads, qc, qs,
+                                          g_in ? g_in + 0 : nullptr);
+  const float gk = quantize_rows_unpacked(k, dt, total * Hkv, d, use_ss, 0, nthreads, kc, ks,
+                                          g_in ? g_in + 1 : nullptr);
   // V: 16-blocks along the tokens of each sequence (zero-padded), reading R6
   std::vector<int64_t> pst(nseq + 1, 0);
   for (int s = 0; s < nseq; ++s) {
@@ -1238,7 +1244,7 @@ int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   const int64_t ptot = pst[nseq];
   float vamax = 0.0f;
   for (int64_t e = 0; e < total * Hkv * d; ++e) vamax = std::max(vamax, std::fabs(orc_half_to_float(v[e], dt)));
-  const float gv = vamax == 0.0f ? 1.0f : vamax / 2688.0f;
+  const float gv = g_in ? g_in[2] : (vamax == 0.0f ? 1.0f : vamax / 2688.0f);
   std::vector<uint8_t> vcol((size_t)(Hkv * d * ptot), 0), vsc((size_t)(Hkv * d * ptot / 16), 0);
   for (int64_t hc = 0; hc < (int64_t)Hkv * d; ++hc) {
     const int64_t hk = hc / d, c = hc % d;
@@ -1258,22 +1264,25 @@ int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
       }
     }
   }
-  auto qhat = [&](int64_t t, int h, int c) {
-    const int64_t e = (t * H + h) * d + c;
-    return deq(qc[(size_t)e], qs[(size_t)(e / 16)], gq);
-  };
-  auto khat = [&](int64_t t, int hk, int c) {
-    const int64_t e = (t * Hkv + hk) * d + c;
-    return deq(kc[(size_t)e], ks[(size_t)(e / 16)], gk);
-  };
-  std::vector<int> seq_of((size_t)total);
+  // dequantised values, tabulated once: Q^ [total, H, d], K^ and V^
+  // [total, Hkv, d], and dO as fp64
+  std::vector<double> qd((size_t)(total * H * d)), kd((size_t)(total * Hkv * d)),
+      vd((size_t)(total * Hkv * d)), dod((size_t)(total * H * d));
+  for (int64_t e = 0; e < total * H * d; ++e) {
+    qd[(size_t)e] = deq(qc[(size_t)e], qs[(size_t)(e / 16)], gq);
+    dod[(size_t)e] = (double)orc_half_to_float(dout[e], dt);
+  }
+  for (int64_t e = 0; e < total * Hkv * d; ++e) kd[(size_t)e] = deq(kc[(size_t)e], ks[(size_t)(e / 16)], gk);
   for (int s = 0; s < nseq; ++s)
-    for (int64_t t = cu[s]; t < cu[s + 1]; ++t) seq_of[(size_t)t] = s;
-  auto vhat = [&](int64_t t, int hk, int c) {
-    const int s = seq_of[(size_t)t];
-    const int64_t ve = ((int64_t)hk * d + c) * ptot + pst[s] + (t - cu[s]);
-    return deq(vcol[(size_t)ve], vsc[(size_t)(ve / 16)], gv);
-  };
+    for (int64_t t = cu[s]; t < cu[s + 1]; ++t)
+      for (int hk = 0; hk < Hkv; ++hk)
+        for (int c = 0; c < d; ++c) {
+          const int64_t ve = ((int64_t)hk * d + c) * ptot + pst[s] + (t - cu[s]);
+          vd[(size_t)((t * Hkv + hk) * d + c)] = deq(vcol[(size_t)ve], vsc[(size_t)(ve / 16)], gv);
+        }
+  auto qhat = [&](int64_t t, int h, int c) { return qd[(size_t)((t * H + h) * d + c)]; };
+  auto khat = [&](int64_t t, int hk, int c) { return kd[(size_t)((t * Hkv + hk) * d + c)]; };
+  auto vhat = [&](int64_t t, int hk, int c) { return vd[(size_t)((t * Hkv + hk) * d + c)]; };
   for (int64_t e = 0; e < total * Hkv * d; ++e) dk[e] = dv[e] = 0.0;
   const double sc = 1.0 / std::sqrt((double)d);
   // one (sequence, head) at a time: the kv-head gradients of different
@@ -1283,7 +1292,8 @@ int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     const int len = cu[s + 1] - cu[s];
     for (int h = 0; h < H; ++h) {
       const int hk = h / (H / Hkv);
-      std::vector<double> P((size_t)len * len, 0.0), Ph((size_t)len * len, 0.0);
+      std::vector<double> P((size_t)len * len, 0.0), Ph((size_t)len * len, 0.0),
+          dS((size_t)len * len, 0.0);
       parallel_for(len, nthreads, [&](int64_t i) {
         const int kend = causal ? (int)i + 1 : len;
         std::vector<double> srow(len, -INFINITY);
@@ -1345,7 +1355,7 @@ int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         for (int c = 0; c < d; ++c) {
           o[(ti * H + h) * d + c] = oh[c];
           o_hp[(ti * H + h) * d + c] = ohp[c];
-          D += (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt) * ohp[c];
+          D += dod[(size_t)((ti * H + h) * d + c)] * ohp[c];
         }
         std::vector<double> dqr(d, 0.0);
         for (int j = 0; j < len; ++j) {
@@ -1353,30 +1363,29 @@ int orc_attn_qat_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
           if (p == 0.0) continue;
           double dp = 0.0;
           for (int c = 0; c < d; ++c)
-            dp += (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt) * vhat(st + j, hk, c);
+            dp += dod[(size_t)((ti * H + h) * d + c)] * vhat(st + j, hk, c);
           const double ds = p * (dp - D);
+          dS[(size_t)i * len + j] = ds;
           for (int c = 0; c < d; ++c) dqr[c] += ds * khat(st + j, hk, c) * sc;
         }
         for (int c = 0; c < d; ++c) dq[(ti * H + h) * d + c] = dqr[c];
       });
-      // dK, dV rows of this head: key j sums over the queries
-      parallel_for(len, nthreads, [&](int64_t j) {
-        const int64_t tj = st + j;
+      // dK, dV rows of this head: key j sums over the queries in order
+      // (blocks of 64 keys keep the row reads of P^ and dS contiguous)
+      parallel_for((len + 63) / 64, nthreads, [&](int64_t jb) {
+        const int j0 = (int)jb * 64, j1 = std::min(len, j0 + 64);
         for (int64_t i = 0; i < len; ++i) {
-          const double p = P[(size_t)i * len + j], ph = Ph[(size_t)i * len + j];
-          if (p == 0.0 && ph == 0.0) continue;
           const int64_t ti = st + i;
-          double dp = 0.0, D = 0.0;
-          for (int c = 0; c < d; ++c) {
-            const double g = (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt);
-            dp += g * vhat(tj, hk, c);
-            D += g * o_hp[(ti * H + h) * d + c];
-          }
-          const double ds = p * (dp - D);
-          for (int c = 0; c < d; ++c) {
-            const double g = (double)orc_half_to_float(dout[(ti * H + h) * d + c], dt);
-            dv[(tj * Hkv + hk) * d + c] += ph * g;
-            dk[(tj * Hkv + hk) * d + c] += ds * qhat(ti, h, c) * sc;
+          for (int j = j0; j < j1; ++j) {
+            const double p = P[(size_t)i * len + j], ph = Ph[(size_t)i * len + j];
+            if (p == 0.0 && ph == 0.0) continue;
+            const double ds = dS[(size_t)i * len + j];
+            const int64_t tj = st + j;
+            for (int c = 0; c < d; ++c) {
+              const double g = dod[(size_t)((ti * H + h) * d + c)];
+              dv[(tj * Hkv + hk) * d + c] += ph * g;
+              dk[(tj * Hkv + hk) * d + c] += ds * qhat(ti, h, c) * sc;
+            }
           }
         }
       });
