@@ -1,0 +1,744 @@
+// Attn-QAT attention: forward on fake-quantised NVFP4 operands and the
+// backward with FP4 recomputation of the probabilities.
+//
+// Source: "Attn-QAT: 4-Bit Attention With Quantization-Aware Training",
+// Metodologia (1: the backward recomputes the probabilities at the forward's
+// FP4 precision; 2: the scalar term of the softmax gradient is taken from a
+// high-precision output O' kept beside the FP4 output).
+//
+// What is computed (every quantiser passes gradients straight through):
+//   Q^, K^  NVFP4 blocks of 16 along d; V^ blocks of 16 along the tokens of
+//           each sequence (zero padded); per-tensor scales g = amax / 2688
+//   S = Q^ K^T / sqrt(d),  lse = log sum_j exp S,  P = exp(S - lse)
+//   P^  two-level FP4 image of P per (row, key tile of blk keys):
+//       sigma = rowmax / 2688; the 16-key blocks of P / sigma are quantised
+//       with block scale E4M3(amax / 6) and no tensor scale
+//   O = P^ V^ (the FP4 output),  O' = P V^,  D = rowsum(dO o O')
+//   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),
+//   dQ = dS K^ / sqrt(d),  dK = dS^T Q^ / sqrt(d)
+//   (dK, dV summed over the query heads of a kv head)
+//
+// Design.  Memory-bound kernels write the fake-quantised images once: each
+// element is E2M1 value x UE4M3 block scale, exact in the 16-bit input type,
+// with the tensor scales applied to the fp32 accumulators instead.  The
+// three attention kernels run warp-level m16n8k16 MMAs (fp32 accumulate) on
+// those images; P^ enters the MMAs rounded to the 16-bit type, dS and the P
+// of O' as sums of two 16-bit parts.
+//   qat_fwd_kernel     per 64-query tile: pass 1 lse, pass 2 P, P^, O, O'
+//   qat_rowdot_kernel  D = rowsum(dO o O')
+//   qat_bwd_kv_kernel  per key tile of blk keys, over every 64-query chunk
+//                      of the kv head's query heads: S^T, P^T, its FP4
+//                      image, dP^T, dS^T; dV += P^^T dO, dK += dS^T Q^
+//   qat_bwd_q_kernel   per 64-query tile: S, P, dP, dS; dQ += dS K^
+#pragma once
+#include "quant_kernels.cuh"
+
+namespace thrift {
+
+constexpr int kQatRows = 64;   // query rows of a forward / dQ CTA (4 warps x 16)
+constexpr int kQatChunk = 64;  // query chunk of the key-tile kernel, key chunk of the dQ kernel
+constexpr float kQatLog2e = 1.4426950408889634f;
+constexpr float kQatLn2 = 0.6931471805599453f;
+
+struct QatParams {
+  const uint16_t* qi;  // fake-quantised images [total, H|Hkv, D] in the input type
+  const uint16_t* ki;
+  const uint16_t* vi;
+  const uint16_t* dout;  // [total, H, D] (backward)
+  const float* g;        // tensor scales of Q, K, V
+  SeqInfo si;
+  int H, Hkv;
+  int64_t total;
+  int causal;
+  float sc;          // 1 / sqrt(d)
+  uint16_t* out;     // forward: O [total, H, D] in the input type
+  float* out_hp;     // forward: O' [total, H, D]; backward: read
+  float* lse;        // [H, total], natural log
+  const float* dsum; // D [H, total]
+  float* dq;         // [total, H, D]
+  float* dk;         // [total, Hkv, D]
+  float* dv;
+};
+
+// ------------------------------------------------------- fake quantisers --
+
+// One 16-element value of a code byte (element 2i in the low nibble) times
+// the block scale, exact in either 16-bit type.
+template <int DT>
+__device__ __forceinline__ uint32_t fq_pair(uint32_t byte, float sv) {
+  float v0, v1;
+  e2m1x2_values(byte, v0, v1);
+  return (uint32_t)f2h<DT>(__fmul_rn(v0, sv)) | ((uint32_t)f2h<DT>(__fmul_rn(v1, sv)) << 16);
+}
+
+// Rows blocked along the contiguous axis (Q, K): n_blocks blocks of 16.
+template <int DT, bool SS>
+__global__ void __launch_bounds__(256) qat_fq_rows_kernel(const uint16_t* __restrict__ x,
+                                                          int64_t n_blocks, const uint32_t* amax,
+                                                          float* g_out,
+                                                          uint16_t* __restrict__ img) {
+  const float g = tensor_scale_from_amax(*amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    float v[16];
+    load16<DT>(x + b * 16, v);
+    uint32_t lo, hi;
+    const float sv = ue4m3_decode(quant_block16(v, g, SS, lo, hi));
+    uint4 w0, w1;
+    w0.x = fq_pair<DT>(lo & 0xFF, sv);
+    w0.y = fq_pair<DT>((lo >> 8) & 0xFF, sv);
+    w0.z = fq_pair<DT>((lo >> 16) & 0xFF, sv);
+    w0.w = fq_pair<DT>(lo >> 24, sv);
+    w1.x = fq_pair<DT>(hi & 0xFF, sv);
+    w1.y = fq_pair<DT>((hi >> 8) & 0xFF, sv);
+    w1.z = fq_pair<DT>((hi >> 16) & 0xFF, sv);
+    w1.w = fq_pair<DT>(hi >> 24, sv);
+    uint4* o = reinterpret_cast<uint4*>(img + b * 16);
+    o[0] = w0;
+    o[1] = w1;
+  }
+}
+
+// V: blocks of 16 tokens of one channel from each sequence's start, the last
+// block zero-padded.  grid (ceil(maxlen / 16), nseq); ncols = Hkv * d.
+template <int DT, bool SS>
+__global__ void __launch_bounds__(256) qat_fq_v_kernel(const uint16_t* __restrict__ v, SeqInfo si,
+                                                       int ncols, const uint32_t* amax,
+                                                       float* g_out, uint16_t* __restrict__ img) {
+  int64_t st;
+  int len;
+  si.get(blockIdx.y, st, len);
+  const float g = tensor_scale_from_amax(*amax);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+  const int t0 = blockIdx.x * 16;
+  if (t0 >= len) return;
+  const int n = min(16, len - t0);
+  for (int c = threadIdx.x; c < ncols; c += blockDim.x) {
+    float x[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      x[e] = e < n ? h2f<DT>(v[(st + t0 + e) * ncols + c]) : 0.0f;
+    uint32_t lo, hi;
+    const float sv = ue4m3_decode(quant_block16(x, g, SS, lo, hi));
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const uint32_t byte = ((e < 8 ? lo : hi) >> (8 * ((e & 7) >> 1))) & 0xFF;
+      const uint32_t pr = fq_pair<DT>(byte, sv);
+      if (e < n) img[(st + t0 + e) * ncols + c] = (uint16_t)(pr & 0xFFFF);
+      if (e + 1 < n) img[(st + t0 + e + 1) * ncols + c] = (uint16_t)(pr >> 16);
+    }
+  }
+}
+
+// ------------------------------------------------------------ warp MMAs --
+
+template <int DT>
+__device__ __forceinline__ uint32_t qpack2(float lo, float hi) {
+  return (uint32_t)f2h<DT>(lo) | ((uint32_t)f2h<DT>(hi) << 16);
+}
+
+// c += a (16 x 16, row) * b (16 x 8, col), fp32 accumulate.  Fragments:
+// a[0] (row g, k 2t..2t+1), a[1] (row g+8, same k), a[2] (row g, k 2t+8..),
+// a[3] (row g+8, k 2t+8..); b0 (k 2t..2t+1, col g), b1 (k 2t+8.., col g);
+// c[0..1] (row g, cols 2t, 2t+1), c[2..3] (row g+8, same cols); g = lane/4,
+// t = lane%4.
+template <int DT>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if constexpr (DT == 1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// Shared-memory tiles are row-major 16-bit with LD = cols + 8 elements per
+// row: a warp's fragment loads then touch 32 distinct banks, and every row
+// starts on a 16-byte boundary.
+template <int LD>
+__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const uint16_t* t, int row0, int k0,
+                                       int g, int tq) {
+  const uint16_t* p = t + (row0 + g) * LD + k0 + 2 * tq;
+  a[0] = *reinterpret_cast<const uint32_t*>(p);
+  a[1] = *reinterpret_cast<const uint32_t*>(p + 8 * LD);
+  a[2] = *reinterpret_cast<const uint32_t*>(p + 8);
+  a[3] = *reinterpret_cast<const uint32_t*>(p + 8 * LD + 8);
+}
+
+template <int LD>
+__device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const uint16_t* t, int n0, int k0,
+                                       int g, int tq) {
+  const uint16_t* p = t + (n0 + g) * LD + k0 + 2 * tq;
+  b0 = *reinterpret_cast<const uint32_t*>(p);
+  b1 = *reinterpret_cast<const uint32_t*>(p + 8);
+}
+
+// The A fragment of k-step s from accumulator tiles c[2s], c[2s+1] (the C
+// layout of two n-tiles is the A layout of one 16-wide k-step).
+template <int DT>
+__device__ __forceinline__ void c_to_a(uint32_t (&a)[4], const float (&c0)[4],
+                                       const float (&c1)[4]) {
+  a[0] = qpack2<DT>(c0[0], c0[1]);
+  a[1] = qpack2<DT>(c0[2], c0[3]);
+  a[2] = qpack2<DT>(c1[0], c1[1]);
+  a[3] = qpack2<DT>(c1[2], c1[3]);
+}
+
+// dS as the sum of two 16-bit parts, hi = round(dS) and lo = round(dS - hi),
+// for two MMAs into one accumulator: rows of dS sum to zero, and rounding
+// dS once would leave a residue that the products with K^ (whose channel
+// means can be large) or Q^ magnify; the split carries about 16 bits.
+template <int DT>
+__device__ __forceinline__ void c_to_a_split(uint32_t (&hi)[4], uint32_t (&lo)[4],
+                                             const float (&c0)[4], const float (&c1)[4]) {
+  const float* src[2] = {c0, c1};
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float* c = src[r >> 1] + 2 * (r & 1);
+    const uint32_t h = qpack2<DT>(c[0], c[1]);
+    hi[r] = h;
+    lo[r] = qpack2<DT>(c[0] - h2f<DT>((uint16_t)(h & 0xFFFF)), c[1] - h2f<DT>((uint16_t)(h >> 16)));
+  }
+}
+
+// rows [r0, r0 + R) of a [tokens, nh, D] image (head h) -> tile [R][LD]; rows
+// at or past len are zero.
+template <int D, int R, int LD>
+__device__ __forceinline__ void stage_rows(uint16_t* t, const uint16_t* x, int64_t st, int len,
+                                           int r0, int nh, int h) {
+  constexpr int CH = D / 8;
+  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
+    const int r = i / CH, c = i % CH;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + r < len) v = __ldg(reinterpret_cast<const uint4*>(x + ((st + r0 + r) * nh + h) * D) + c);
+    *reinterpret_cast<uint4*>(t + r * LD + 8 * c) = v;
+  }
+}
+
+// The same rows transposed: tile [D][LDT], element (c, r) = x[r0 + r][c].
+template <int D, int R, int LDT>
+__device__ __forceinline__ void stage_rows_t(uint16_t* t, const uint16_t* x, int64_t st, int len,
+                                             int r0, int nh, int h) {
+  constexpr int CH = D / 8;
+  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
+    const int r = i % R, c = i / R;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + r < len) v = __ldg(reinterpret_cast<const uint4*>(x + ((st + r0 + r) * nh + h) * D) + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      t[(8 * c + 2 * e) * LDT + r] = (uint16_t)(w[e] & 0xFFFF);
+      t[(8 * c + 2 * e + 1) * LDT + r] = (uint16_t)(w[e] >> 16);
+    }
+  }
+}
+
+__device__ __forceinline__ float quad_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+
+// FP4 value of a probability already divided by sigma: the 16-key block's
+// scale byte from amax (the block's largest scaled value), then the E2M1 code
+// of x / scale; returns code value x scale (0 when the byte is 0).
+struct PBlock {
+  float dec, rr;
+  bool zero;
+  __device__ __forceinline__ explicit PBlock(float amax) {
+    const uint32_t sp = ue4m3(__fdiv_rn(amax, 6.0f));
+    zero = sp == 0;
+    dec = ue4m3_decode(sp);
+    rr = zero ? 0.0f : __frcp_rn(dec);
+  }
+  __device__ __forceinline__ void apply(float x0, float x1, float& q0, float& q1) const {
+    e2m1x2_roundtrip(__fmul_rn(x0, rr), __fmul_rn(x1, rr), q0, q1);
+    q0 = zero ? 0.0f : __fmul_rn(q0, dec);
+    q1 = zero ? 0.0f : __fmul_rn(q1, dec);
+  }
+};
+
+template <int D, int BLK>
+struct QatFwdSmem {
+  static constexpr int LD = D + 8, LV = BLK + 8;
+  static constexpr int Q = 0;
+  static constexpr int K = Q + kQatRows * LD;
+  static constexpr int VT = K + BLK * LD;
+  static constexpr size_t BYTES = (size_t)(VT + D * LV) * 2;
+};
+
+// ------------------------------------------------------------- forward --
+// grid (ceil(maxlen / 64), H, nseq), 128 threads; warp w owns query rows
+// 16w..16w+15 of the tile.  Causal grids visit the tiles from the last (the
+// longest rows) first.
+template <int DT, int D, int BLK>
+__global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
+  using L = QatFwdSmem<D, BLK>;
+  constexpr int LD = L::LD, LV = L::LV, NT = BLK / 8, ND = D / 8;
+  extern __shared__ __align__(16) uint16_t qsm[];
+  uint16_t* sQ = qsm + L::Q;
+  uint16_t* sK = qsm + L::K;
+  uint16_t* sVt = qsm + L::VT;
+  int64_t st;
+  int len;
+  p.si.get(blockIdx.z, st, len);
+  const int tiles = (len + kQatRows - 1) / kQatRows;
+  if ((int)blockIdx.x >= tiles) return;
+  const int q0 = (p.causal ? tiles - 1 - (int)blockIdx.x : (int)blockIdx.x) * kQatRows;
+  const int h = blockIdx.y, hk = h / (p.H / p.Hkv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;
+  const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
+  const int kend = p.causal ? min(len, q0 + kQatRows) : len;
+  const int ntiles = (kend + BLK - 1) / BLK;
+
+  stage_rows<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+
+  auto scores = [&](float (&s)[NT][4], int j0) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t a[4];
+      frag_a<LD>(a, sQ, 16 * warp, 16 * kk, g, tq);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        uint32_t b0, b1;
+        frag_b<LD>(b0, b1, sK, 8 * n, 16 * kk, g, tq);
+        mma16816<DT>(s[n], a, b0, b1);
+      }
+    }
+    // scale to log2 units and mask
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j0 + 8 * n + 2 * tq + (e & 1), i = row[e >> 1];
+        const bool ok = j < len && (!p.causal || j <= i);
+        s[n][e] = ok ? s[n][e] * c2 : -INFINITY;
+      }
+  };
+
+  // pass 1: row max and sum of exp in log2 units
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+  for (int kt = 0; kt < ntiles; ++kt) {
+    __syncthreads();
+    stage_rows<D, BLK, LD>(sK, p.ki, st, len, kt * BLK, p.Hkv, hk);
+    __syncthreads();
+    float s[NT][4];
+    scores(s, kt * BLK);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
+      mx = quad_max(mx);
+      const float mn = fmaxf(m[r], mx);
+      if (mn == -INFINITY) continue;
+      float acc = m[r] == -INFINITY ? 0.0f : l[r] * exp2f(m[r] - mn);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) acc += exp2f(s[n][2 * r] - mn) + exp2f(s[n][2 * r + 1] - mn);
+      l[r] = acc;
+      m[r] = mn;
+    }
+  }
+  float lse2[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float t = l[r];
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    lse2[r] = m[r] + log2f(t);
+    if (tq == 0 && row[r] < len) p.lse[(int64_t)h * p.total + st + row[r]] = lse2[r] * kQatLn2;
+  }
+
+  // pass 2: P, its FP4 image, O and O'
+  float o[ND][4], oh[ND][4];
+#pragma unroll
+  for (int n = 0; n < ND; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[n][e] = oh[n][e] = 0.0f;
+  for (int kt = 0; kt < ntiles; ++kt) {
+    __syncthreads();
+    stage_rows<D, BLK, LD>(sK, p.ki, st, len, kt * BLK, p.Hkv, hk);
+    stage_rows_t<D, BLK, LV>(sVt, p.vi, st, len, kt * BLK, p.Hkv, hk);
+    __syncthreads();
+    float s[NT][4];
+    scores(s, kt * BLK);
+    float inv[2], sig[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mx = 0.0f;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        s[n][2 * r] = exp2f(s[n][2 * r] - lse2[r]);
+        s[n][2 * r + 1] = exp2f(s[n][2 * r + 1] - lse2[r]);
+        mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
+      }
+      mx = quad_max(mx);
+      inv[r] = mx > 0.0f ? __fdiv_rn(kTensorScaleDiv, mx) : 0.0f;
+      sig[r] = __fdiv_rn(mx, kTensorScaleDiv);
+    }
+#pragma unroll
+    for (int b = 0; b < NT / 2; ++b) {
+      float qv[2][4];  // P^ of n-tiles 2b, 2b+1 in C layout
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float x0 = __fmul_rn(s[2 * b][2 * r], inv[r]), x1 = __fmul_rn(s[2 * b][2 * r + 1], inv[r]);
+        const float x2 = __fmul_rn(s[2 * b + 1][2 * r], inv[r]);
+        const float x3 = __fmul_rn(s[2 * b + 1][2 * r + 1], inv[r]);
+        const PBlock pb(quad_max(fmaxf(fmaxf(x0, x1), fmaxf(x2, x3))));
+        float y0, y1, y2, y3;
+        pb.apply(x0, x1, y0, y1);
+        pb.apply(x2, x3, y2, y3);
+        qv[0][2 * r] = __fmul_rn(y0, sig[r]);
+        qv[0][2 * r + 1] = __fmul_rn(y1, sig[r]);
+        qv[1][2 * r] = __fmul_rn(y2, sig[r]);
+        qv[1][2 * r + 1] = __fmul_rn(y3, sig[r]);
+      }
+      // O' carries P in two parts: it sets D = rowsum(dO o O') of the
+      // backward, whose error reaches dQ multiplied by the keys' means
+      uint32_t aq[4], ph[4], pl[4];
+      c_to_a<DT>(aq, qv[0], qv[1]);
+      c_to_a_split<DT>(ph, pl, s[2 * b], s[2 * b + 1]);
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        uint32_t b0, b1;
+        frag_b<LV>(b0, b1, sVt, 8 * n, 16 * b, g, tq);
+        mma16816<DT>(o[n], aq, b0, b1);
+        mma16816<DT>(oh[n], ph, b0, b1);
+        mma16816<DT>(oh[n], pl, b0, b1);
+      }
+    }
+  }
+  const float gv = p.g[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    if (row[r] >= len) continue;
+    const int64_t base = ((st + row[r]) * p.H + h) * D;
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+      const int c = 8 * n + 2 * tq;
+      *reinterpret_cast<uint32_t*>(p.out + base + c) =
+          qpack2<DT>(o[n][2 * r] * gv, o[n][2 * r + 1] * gv);
+      *reinterpret_cast<float2*>(p.out_hp + base + c) =
+          make_float2(oh[n][2 * r] * gv, oh[n][2 * r + 1] * gv);
+    }
+  }
+}
+
+// D = rowsum(dO o O') per (token, head); one warp per row.
+template <int DT, int D>
+__global__ void __launch_bounds__(256) qat_rowdot_kernel(const uint16_t* __restrict__ dout,
+                                                         const float* __restrict__ out_hp,
+                                                         int64_t total, int H,
+                                                         float* __restrict__ dsum) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nrows = total * H;
+  for (int64_t rr = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; rr < nrows;
+       rr += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int c = lane; c < D; c += 32) acc = fmaf(h2f<DT>(dout[rr * D + c]), out_hp[rr * D + c], acc);
+#pragma unroll
+    for (int m2 = 16; m2 >= 1; m2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m2);
+    if (lane == 0) dsum[(rr % H) * total + rr / H] = acc;
+  }
+}
+
+template <int D, int BLK>
+struct QatKvSmem {
+  static constexpr int LD = D + 8, LT = kQatChunk + 8, NW = BLK / 16;
+  static constexpr int K = 0;
+  static constexpr int V = K + BLK * LD;
+  static constexpr int Q = V + BLK * LD;
+  static constexpr int DO = Q + kQatChunk * LD;
+  static constexpr int QT = DO + kQatChunk * LD;
+  static constexpr int DOT = QT + D * LT;
+  static constexpr int END16 = DOT + D * LT;  // 16-bit elements; fp32 arrays follow
+  static constexpr size_t BYTES = (size_t)END16 * 2 + (size_t)(2 + NW) * kQatChunk * 4;
+};
+
+// ------------------------------------------------- backward: dK and dV --
+// grid (ceil(maxlen / BLK), Hkv, nseq), BLK / 16 warps; warp w owns keys
+// 16w..16w+15 of the tile (one 16-key block of the P quantisation).
+template <int DT, int D, int BLK>
+__global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
+  using L = QatKvSmem<D, BLK>;
+  constexpr int LD = L::LD, LT = L::LT, NW = L::NW, QC = kQatChunk, NQ = QC / 8, ND = D / 8;
+  extern __shared__ __align__(16) uint16_t qsm[];
+  uint16_t* sK = qsm + L::K;
+  uint16_t* sV = qsm + L::V;
+  uint16_t* sQ = qsm + L::Q;
+  uint16_t* sdO = qsm + L::DO;
+  uint16_t* sQt = qsm + L::QT;
+  uint16_t* sdOt = qsm + L::DOT;
+  float* s_lse2 = reinterpret_cast<float*>(qsm + L::END16);
+  float* s_D = s_lse2 + QC;
+  float* s_cmax = s_D + QC;  // [NW][QC]
+  int64_t st;
+  int len;
+  p.si.get(blockIdx.z, st, len);
+  const int j0 = blockIdx.x * BLK;
+  if (j0 >= len) return;
+  const int hk = blockIdx.y, grp = p.H / p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
+  const int key[2] = {j0 + 16 * warp + g, j0 + 16 * warp + g + 8};
+
+  stage_rows<D, BLK, LD>(sK, p.ki, st, len, j0, p.Hkv, hk);
+  stage_rows<D, BLK, LD>(sV, p.vi, st, len, j0, p.Hkv, hk);
+  float dk[ND][4], dv[ND][4];
+#pragma unroll
+  for (int n = 0; n < ND; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.0f;
+
+  for (int hh = 0; hh < grp; ++hh) {
+    const int h = hk * grp + hh;
+    for (int qc0 = p.causal ? j0 / QC * QC : 0; qc0 < len; qc0 += QC) {
+      __syncthreads();
+      stage_rows<D, QC, LD>(sQ, p.qi, st, len, qc0, p.H, h);
+      stage_rows<D, QC, LD>(sdO, p.dout, st, len, qc0, p.H, h);
+      stage_rows_t<D, QC, LT>(sQt, p.qi, st, len, qc0, p.H, h);
+      stage_rows_t<D, QC, LT>(sdOt, p.dout, st, len, qc0, p.H, h);
+      for (int i = threadIdx.x; i < QC; i += blockDim.x) {
+        const bool ok = qc0 + i < len;
+        s_lse2[i] = ok ? p.lse[(int64_t)h * p.total + st + qc0 + i] * kQatLog2e : 0.0f;
+        s_D[i] = ok ? p.dsum[(int64_t)h * p.total + st + qc0 + i] : 0.0f;
+      }
+      __syncthreads();
+      // S^T (keys x queries) and P^T
+      float s[NQ][4];
+#pragma unroll
+      for (int n = 0; n < NQ; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4];
+        frag_a<LD>(a, sK, 16 * warp, 16 * kk, g, tq);
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) {
+          uint32_t b0, b1;
+          frag_b<LD>(b0, b1, sQ, 8 * n, 16 * kk, g, tq);
+          mma16816<DT>(s[n], a, b0, b1);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < NQ; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int il = 8 * n + 2 * tq + (e & 1), i = qc0 + il, j = key[e >> 1];
+          const bool ok = j < len && i < len && (!p.causal || j <= i);
+          s[n][e] = ok ? exp2f(s[n][e] * c2 - s_lse2[il]) : 0.0f;
+        }
+      // per query: max of P over the key tile (all warps)
+#pragma unroll
+      for (int n = 0; n < NQ; ++n)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float v = fmaxf(s[n][c], s[n][c + 2]);
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          if (g == 0) s_cmax[warp * QC + 8 * n + 2 * tq + c] = v;
+        }
+      __syncthreads();
+      // dV += P^^T dO, one 16-query k-step at a time
+#pragma unroll
+      for (int b = 0; b < NQ / 2; ++b) {
+        float qv[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int il = 8 * (2 * b + u) + 2 * tq + c;
+            float cm = 0.0f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) cm = fmaxf(cm, s_cmax[w * QC + il]);
+            const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
+            const float sig = __fdiv_rn(cm, kTensorScaleDiv);
+            const float x0 = __fmul_rn(s[2 * b + u][c], inv), x1 = __fmul_rn(s[2 * b + u][c + 2], inv);
+            float am = fmaxf(x0, x1);
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
+            const PBlock pb(am);
+            float y0, y1;
+            pb.apply(x0, x1, y0, y1);
+            qv[u][c] = __fmul_rn(y0, sig);
+            qv[u][c + 2] = __fmul_rn(y1, sig);
+          }
+        uint32_t a[4];
+        c_to_a<DT>(a, qv[0], qv[1]);
+#pragma unroll
+        for (int n = 0; n < ND; ++n) {
+          uint32_t b0, b1;
+          frag_b<LT>(b0, b1, sdOt, 8 * n, 16 * b, g, tq);
+          mma16816<DT>(dv[n], a, b0, b1);
+        }
+      }
+      // dP^T = V^ dO^T, dS^T = P^T o (dP^T - D)
+      float dp[NQ][4];
+#pragma unroll
+      for (int n = 0; n < NQ; ++n) dp[n][0] = dp[n][1] = dp[n][2] = dp[n][3] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4];
+        frag_a<LD>(a, sV, 16 * warp, 16 * kk, g, tq);
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) {
+          uint32_t b0, b1;
+          frag_b<LD>(b0, b1, sdO, 8 * n, 16 * kk, g, tq);
+          mma16816<DT>(dp[n], a, b0, b1);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < NQ; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int il = 8 * n + 2 * tq + (e & 1);
+          dp[n][e] = s[n][e] * (dp[n][e] * gv - s_D[il]);
+        }
+      // dK += dS^T Q^
+#pragma unroll
+      for (int b = 0; b < NQ / 2; ++b) {
+        uint32_t ah[4], al[4];
+        c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
+#pragma unroll
+        for (int n = 0; n < ND; ++n) {
+          uint32_t b0, b1;
+          frag_b<LT>(b0, b1, sQt, 8 * n, 16 * b, g, tq);
+          mma16816<DT>(dk[n], ah, b0, b1);
+          mma16816<DT>(dk[n], al, b0, b1);
+        }
+      }
+    }
+  }
+  const float kscale = p.g[0] * p.sc;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    if (key[r] >= len) continue;
+    const int64_t base = ((st + key[r]) * p.Hkv + hk) * D;
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+      const int c = 8 * n + 2 * tq;
+      *reinterpret_cast<float2*>(p.dk + base + c) =
+          make_float2(dk[n][2 * r] * kscale, dk[n][2 * r + 1] * kscale);
+      *reinterpret_cast<float2*>(p.dv + base + c) = make_float2(dv[n][2 * r], dv[n][2 * r + 1]);
+    }
+  }
+}
+
+template <int D>
+struct QatQSmem {
+  static constexpr int LD = D + 8, LT = kQatChunk + 8;
+  static constexpr int Q = 0;
+  static constexpr int DO = Q + kQatRows * LD;
+  static constexpr int K = DO + kQatRows * LD;
+  static constexpr int V = K + kQatChunk * LD;
+  static constexpr int KT = V + kQatChunk * LD;
+  static constexpr size_t BYTES = (size_t)(KT + D * LT) * 2;
+};
+
+// ------------------------------------------------------ backward: dQ --
+// grid (ceil(maxlen / 64), H, nseq), 128 threads; warp w owns query rows
+// 16w..16w+15; keys in chunks of 64.
+template <int DT, int D>
+__global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
+  using L = QatQSmem<D>;
+  constexpr int LD = L::LD, LT = L::LT, KC = kQatChunk, NK = KC / 8, ND = D / 8;
+  extern __shared__ __align__(16) uint16_t qsm[];
+  uint16_t* sQ = qsm + L::Q;
+  uint16_t* sdO = qsm + L::DO;
+  uint16_t* sK = qsm + L::K;
+  uint16_t* sV = qsm + L::V;
+  uint16_t* sKt = qsm + L::KT;
+  int64_t st;
+  int len;
+  p.si.get(blockIdx.z, st, len);
+  const int tiles = (len + kQatRows - 1) / kQatRows;
+  if ((int)blockIdx.x >= tiles) return;
+  const int q0 = (p.causal ? tiles - 1 - (int)blockIdx.x : (int)blockIdx.x) * kQatRows;
+  const int h = blockIdx.y, hk = h / (p.H / p.Hkv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
+  const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
+  float lse2[2], dsum[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const bool ok = row[r] < len;
+    lse2[r] = ok ? p.lse[(int64_t)h * p.total + st + row[r]] * kQatLog2e : 0.0f;
+    dsum[r] = ok ? p.dsum[(int64_t)h * p.total + st + row[r]] : 0.0f;
+  }
+  stage_rows<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+  stage_rows<D, kQatRows, LD>(sdO, p.dout, st, len, q0, p.H, h);
+  float dq[ND][4];
+#pragma unroll
+  for (int n = 0; n < ND; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.0f;
+  const int kend = p.causal ? min(len, q0 + kQatRows) : len;
+  for (int k0 = 0; k0 < kend; k0 += KC) {
+    __syncthreads();
+    stage_rows<D, KC, LD>(sK, p.ki, st, len, k0, p.Hkv, hk);
+    stage_rows<D, KC, LD>(sV, p.vi, st, len, k0, p.Hkv, hk);
+    stage_rows_t<D, KC, LT>(sKt, p.ki, st, len, k0, p.Hkv, hk);
+    __syncthreads();
+    float s[NK][4], dp[NK][4];
+#pragma unroll
+    for (int n = 0; n < NK; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t aq[4], ad[4];
+      frag_a<LD>(aq, sQ, 16 * warp, 16 * kk, g, tq);
+      frag_a<LD>(ad, sdO, 16 * warp, 16 * kk, g, tq);
+#pragma unroll
+      for (int n = 0; n < NK; ++n) {
+        uint32_t b0, b1;
+        frag_b<LD>(b0, b1, sK, 8 * n, 16 * kk, g, tq);
+        mma16816<DT>(s[n], aq, b0, b1);
+        frag_b<LD>(b0, b1, sV, 8 * n, 16 * kk, g, tq);
+        mma16816<DT>(dp[n], ad, b0, b1);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NK; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = k0 + 8 * n + 2 * tq + (e & 1), r = e >> 1, i = row[r];
+        const bool ok = j < len && i < len && (!p.causal || j <= i);
+        const float pr = ok ? exp2f(s[n][e] * c2 - lse2[r]) : 0.0f;
+        dp[n][e] = pr * (dp[n][e] * gv - dsum[r]);
+      }
+#pragma unroll
+    for (int b = 0; b < NK / 2; ++b) {
+      uint32_t ah[4], al[4];
+      c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        uint32_t b0, b1;
+        frag_b<LT>(b0, b1, sKt, 8 * n, 16 * b, g, tq);
+        mma16816<DT>(dq[n], ah, b0, b1);
+        mma16816<DT>(dq[n], al, b0, b1);
+      }
+    }
+  }
+  const float qscale = p.g[1] * p.sc;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    if (row[r] >= len) continue;
+    const int64_t base = ((st + row[r]) * p.H + h) * D;
+#pragma unroll
+    for (int n = 0; n < ND; ++n)
+      *reinterpret_cast<float2*>(p.dq + base + 8 * n + 2 * tq) =
+          make_float2(dq[n][2 * r] * qscale, dq[n][2 * r + 1] * qscale);
+  }
+}
+
+}  // namespace thrift

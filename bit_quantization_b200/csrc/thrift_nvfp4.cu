@@ -10,6 +10,7 @@
 
 #include "attn.cuh"
 #include "decode.cuh"
+#include "qat.cuh"
 #include "select.cuh"
 
 namespace thrift {
@@ -590,6 +591,133 @@ __global__ void wait_timeout_kernel(int mode, uint64_t limit_ns) {
     spin_until_geq(&g_never_written, 1u, limit_ns);
 }
 
+
+// ---------------------------------------------------------- Attn-QAT glue --
+
+struct QatWs {
+  uint16_t* qi;
+  uint16_t* ki;
+  uint16_t* vi;
+  uint32_t* amax;  // [4]
+  float* g;        // [4]
+  float* dsum;     // [H, total]
+  size_t bytes;
+};
+
+QatWs carve_qat(void* base, int64_t total, int H, int Hkv, int d) {
+  Carve c(base);
+  QatWs w;
+  w.qi = c.take<uint16_t>((size_t)total * H * d * 2);
+  w.ki = c.take<uint16_t>((size_t)total * Hkv * d * 2);
+  w.vi = c.take<uint16_t>((size_t)total * Hkv * d * 2);
+  w.amax = c.take<uint32_t>(16);
+  w.g = c.take<float>(16);
+  w.dsum = c.take<float>((size_t)total * H * 4);
+  w.bytes = c.off;
+  return w;
+}
+
+template <class Kernel>
+thrift_status qat_smem_attr(Kernel kernel, size_t bytes, bool& done) {
+  if (!done) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+      return THRIFT_ERR_CUDA;
+    done = true;
+  }
+  return THRIFT_OK;
+}
+
+// Fake-quantised images of Q, K, V and their tensor scales.
+template <int DT>
+void qat_images(const void* q, const void* k, const void* v, SeqInfo si, int nseq, int64_t total,
+                int maxlen, int H, int Hkv, int d, int ss, const QatWs& w, cudaStream_t st) {
+  cudaMemsetAsync(w.amax, 0, 16, st);
+  launch_amax<DT>(q, total * H * d / 16, 0, w.amax + 0, st);
+  launch_amax<DT>(k, total * Hkv * d / 16, 0, w.amax + 1, st);
+  launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
+  const auto* qp = static_cast<const uint16_t*>(q);
+  const auto* kp = static_cast<const uint16_t*>(k);
+  const auto* vp = static_cast<const uint16_t*>(v);
+  const int64_t nq = total * H * d / 16, nk = total * Hkv * d / 16;
+  if (ss) {
+    qat_fq_rows_kernel<DT, true><<<grid_for(nq), kThreads, 0, st>>>(qp, nq, w.amax, w.g, w.qi);
+    qat_fq_rows_kernel<DT, true><<<grid_for(nk), kThreads, 0, st>>>(kp, nk, w.amax + 1, w.g + 1, w.ki);
+    qat_fq_v_kernel<DT, true><<<dim3((unsigned)ceil_div(maxlen, 16), nseq), kThreads, 0, st>>>(
+        vp, si, Hkv * d, w.amax + 2, w.g + 2, w.vi);
+  } else {
+    qat_fq_rows_kernel<DT, false><<<grid_for(nq), kThreads, 0, st>>>(qp, nq, w.amax, w.g, w.qi);
+    qat_fq_rows_kernel<DT, false><<<grid_for(nk), kThreads, 0, st>>>(kp, nk, w.amax + 1, w.g + 1, w.ki);
+    qat_fq_v_kernel<DT, false><<<dim3((unsigned)ceil_div(maxlen, 16), nseq), kThreads, 0, st>>>(
+        vp, si, Hkv * d, w.amax + 2, w.g + 2, w.vi);
+  }
+}
+
+template <int DT, int D, int BLK>
+thrift_status qat_fwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
+  static bool attr = false;
+  const size_t smem = QatFwdSmem<D, BLK>::BYTES;
+  if (qat_smem_attr(qat_fwd_kernel<DT, D, BLK>, smem, attr) != THRIFT_OK) return THRIFT_ERR_CUDA;
+  const dim3 grid((unsigned)ceil_div(maxlen, kQatRows), p.H, nseq);
+  cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
+  if (ev) cudaEventRecord(ev[0], st);
+  qat_fwd_kernel<DT, D, BLK><<<grid, 128, smem, st>>>(p);
+  const thrift_status s = launch_status();
+  if (ev) cudaEventRecord(ev[1], st);
+  return s;
+}
+
+template <int DT, int D, int BLK>
+thrift_status qat_bwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
+  static bool attr_kv = false, attr_q = false;
+  const size_t skv = QatKvSmem<D, BLK>::BYTES, sq = QatQSmem<D>::BYTES;
+  if (qat_smem_attr(qat_bwd_kv_kernel<DT, D, BLK>, skv, attr_kv) != THRIFT_OK) return THRIFT_ERR_CUDA;
+  if (qat_smem_attr(qat_bwd_q_kernel<DT, D>, sq, attr_q) != THRIFT_OK) return THRIFT_ERR_CUDA;
+  const int64_t rows = p.total * p.H;
+  qat_rowdot_kernel<DT, D><<<grid_for(rows * 32), kThreads, 0, st>>>(p.dout, p.out_hp, p.total,
+                                                                    p.H, const_cast<float*>(p.dsum));
+  cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
+  if (ev) cudaEventRecord(ev[0], st);
+  qat_bwd_kv_kernel<DT, D, BLK><<<dim3((unsigned)ceil_div(maxlen, BLK), p.Hkv, nseq), BLK * 2, skv,
+                                  st>>>(p);
+  qat_bwd_q_kernel<DT, D><<<dim3((unsigned)ceil_div(maxlen, kQatRows), p.H, nseq), 128, sq, st>>>(p);
+  const thrift_status s = launch_status();
+  if (ev) cudaEventRecord(ev[1], st);
+  return s;
+}
+
+template <int DT>
+thrift_status qat_fwd_dispatch(const QatParams& p, int nseq, int maxlen, int d, int blk,
+                               cudaStream_t st) {
+  if (d == 128 && blk == 128) return qat_fwd_launch<DT, 128, 128>(p, nseq, maxlen, st);
+  if (d == 128 && blk == 64) return qat_fwd_launch<DT, 128, 64>(p, nseq, maxlen, st);
+  if (d == 64 && blk == 128) return qat_fwd_launch<DT, 64, 128>(p, nseq, maxlen, st);
+  return qat_fwd_launch<DT, 64, 64>(p, nseq, maxlen, st);
+}
+
+template <int DT>
+thrift_status qat_bwd_dispatch(const QatParams& p, int nseq, int maxlen, int d, int blk,
+                               cudaStream_t st) {
+  if (d == 128 && blk == 128) return qat_bwd_launch<DT, 128, 128>(p, nseq, maxlen, st);
+  if (d == 128 && blk == 64) return qat_bwd_launch<DT, 128, 64>(p, nseq, maxlen, st);
+  if (d == 64 && blk == 128) return qat_bwd_launch<DT, 64, 128>(p, nseq, maxlen, st);
+  return qat_bwd_launch<DT, 64, 64>(p, nseq, maxlen, st);
+}
+
+thrift_status check_qat_args(const void* q, const void* k, const void* v, int dt,
+                             const int32_t* cu, int nseq, int64_t total, int maxlen, int H,
+                             int Hkv, int d, int blk, const void* ws, size_t ws_bytes) {
+  if (!q || !k || !v || !cu || !ws) return THRIFT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(ws)) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (H <= 0 || Hkv <= 0 || H % Hkv || maxlen <= 0 || nseq <= 0 || total <= 0) return THRIFT_ERR_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (H > 65535 || nseq > 65535) return THRIFT_ERR_UNSUPPORTED;
+  if (ws_bytes < carve_qat(nullptr, total, H, Hkv, d).bytes) return THRIFT_ERR_ARG;
+  return THRIFT_OK;
+}
+
 }  // namespace
 }  // namespace thrift
 
@@ -929,6 +1057,90 @@ thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, i
                           sink_blocks, recent_blocks, use_scalesearch, out, lse, workspace, st);
   return decode_impl<0>(q, B, H, Hkv, capacity, cache, seq_len, kv_scale, topk_frac, sink_blocks,
                         recent_blocks, use_scalesearch, out, lse, workspace, st);
+}
+
+// ------------------------------------------------------------ Attn-QAT --
+
+size_t thrift_qat_workspace_size(int64_t total, int H, int Hkv, int d) {
+  if (total <= 0 || H <= 0 || Hkv <= 0 || (d != 64 && d != 128)) return 0;
+  return carve_qat(nullptr, total, H, Hkv, d).bytes;
+}
+
+thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v, thrift_dtype dt,
+                                    const int32_t* cu_seqlens, int nseq, int64_t total,
+                                    int max_seqlen, int H, int Hkv, int d, int blk, int causal,
+                                    int use_scalesearch, void* out, float* out_hp, float* lse,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  thrift_status s = check_qat_args(q, k, v, dt, cu_seqlens, nseq, total, max_seqlen, H, Hkv, d,
+                                   blk, workspace, ws_bytes);
+  if (s != THRIFT_OK) return s;
+  if (!out || !out_hp || !lse || !aligned16(out) || !aligned16(out_hp)) return THRIFT_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const QatWs w = carve_qat(workspace, total, H, Hkv, d);
+  const SeqInfo si{cu_seqlens, 0};
+  QatParams p{};
+  p.qi = w.qi;
+  p.ki = w.ki;
+  p.vi = w.vi;
+  p.g = w.g;
+  p.si = si;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.total = total;
+  p.causal = causal ? 1 : 0;
+  p.sc = (float)(1.0 / std::sqrt((double)d));
+  p.out = static_cast<uint16_t*>(out);
+  p.out_hp = out_hp;
+  p.lse = lse;
+  if (dt == THRIFT_BF16) {
+    qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+    return qat_fwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
+  }
+  qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+  return qat_fwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
+}
+
+thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v, const void* dout,
+                                    thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                    int64_t total, int max_seqlen, int H, int Hkv, int d, int blk,
+                                    int causal, int use_scalesearch, int reuse_images,
+                                    const float* out_hp, const float* lse, float* dq, float* dk,
+                                    float* dv, void* workspace, size_t ws_bytes, void* stream) {
+  thrift_status s = check_qat_args(q, k, v, dt, cu_seqlens, nseq, total, max_seqlen, H, Hkv, d,
+                                   blk, workspace, ws_bytes);
+  if (s != THRIFT_OK) return s;
+  if (!dout || !out_hp || !lse || !dq || !dk || !dv) return THRIFT_ERR_ARG;
+  if (!aligned16(dout) || !aligned16(out_hp) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return THRIFT_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const QatWs w = carve_qat(workspace, total, H, Hkv, d);
+  const SeqInfo si{cu_seqlens, 0};
+  QatParams p{};
+  p.qi = w.qi;
+  p.ki = w.ki;
+  p.vi = w.vi;
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.g = w.g;
+  p.si = si;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.total = total;
+  p.causal = causal ? 1 : 0;
+  p.sc = (float)(1.0 / std::sqrt((double)d));
+  p.out_hp = const_cast<float*>(out_hp);
+  p.lse = const_cast<float*>(lse);
+  p.dsum = w.dsum;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  if (dt == THRIFT_BF16) {
+    if (!reuse_images)
+      qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+    return qat_bwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
+  }
+  if (!reuse_images)
+    qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+  return qat_bwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
 }
 
 }  // extern "C"

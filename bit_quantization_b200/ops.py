@@ -31,6 +31,7 @@ EXPORTS = (
     "thrift_kernel_timer_enable", "thrift_kernel_timer_read", "thrift_test_wait_timeout",
     "thrift_kv_cache_size", "thrift_kv_cache_append", "thrift_attn_decode_workspace_size",
     "thrift_attn_decode_mask_offset", "thrift_attn_decode",
+    "thrift_qat_workspace_size", "thrift_qat_fwd_varlen", "thrift_qat_bwd_varlen",
 )
 
 
@@ -95,6 +96,14 @@ def lib():
         L.thrift_attn_decode.restype = i32
         L.thrift_attn_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, sz, P, P, f32,
                                          i32, i32, i32, P, P, P, sz, P]
+        L.thrift_qat_workspace_size.restype = sz
+        L.thrift_qat_workspace_size.argtypes = [i64, i32, i32, i32]
+        L.thrift_qat_fwd_varlen.restype = i32
+        L.thrift_qat_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
+                                            i32, i32, P, P, P, P, sz, P]
+        L.thrift_qat_bwd_varlen.restype = i32
+        L.thrift_qat_bwd_varlen.argtypes = [P, P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
+                                            i32, i32, i32, P, P, P, P, P, P, sz, P]
         _lib = L
     return _lib
 
@@ -404,3 +413,89 @@ def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, re
                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
            "thrift_attn_decode")
     return out, lse
+
+
+# --------------------------------------------------------------- Attn-QAT --
+
+def qat_workspace_size(total, H, Hkv, d=128) -> int:
+    return int(lib().thrift_qat_workspace_size(int(total), H, Hkv, d))
+
+
+def _qat_pack(q, k, v, cu_seqlens, max_seqlen):
+    """[B,N,H,d] inputs -> packed [B*N,H,d] with uniform cu_seqlens; packed
+    inputs pass through."""
+    if q.dim() == 4:
+        B, N = q.shape[0], q.shape[1]
+        cu = torch.arange(0, B * N + 1, N, dtype=torch.int32, device=q.device)
+        return (q.reshape(B * N, *q.shape[2:]), k.reshape(B * N, *k.shape[2:]),
+                v.reshape(B * N, *v.shape[2:]), cu, N)
+    if cu_seqlens is None or max_seqlen is None:
+        raise ThriftError("packed inputs need cu_seqlens and max_seqlen")
+    if cu_seqlens.dtype != torch.int32:
+        raise ThriftError("cu_seqlens must be int32")
+    return q, k, v, cu_seqlens, int(max_seqlen)
+
+
+def thrift_qat_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, blk=128, causal=True,
+                   use_scalesearch=False, workspace=None):
+    """Attn-QAT forward.  q [B,N,H,d] or packed [total,H,d] (with cu_seqlens,
+    max_seqlen), k/v likewise with Hkv heads.  Returns (out like q in its
+    dtype: the FP4 output, out_hp f32 like q: the high-precision output,
+    lse f32 [H, total])."""
+    _need_cuda(q, k, v)
+    shape = q.shape
+    qp, kp, vp, cu, maxlen = _qat_pack(q, k, v, cu_seqlens, max_seqlen)
+    for t in (qp, kp, vp):
+        if not t.is_contiguous():
+            raise ThriftError("thrift_qat_fwd: inputs must be contiguous")
+    total, H, d = qp.shape
+    Hkv = kp.shape[1]
+    out = torch.empty_like(qp)
+    out_hp = torch.empty(qp.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    need = qat_workspace_size(total, H, Hkv, d)
+    if need == 0:
+        raise ThriftError("thrift_qat_fwd: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    _check(lib().thrift_qat_fwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _dt(q), _ptr(cu),
+                                       cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
+                                       int(use_scalesearch), _ptr(out), _ptr(out_hp), _ptr(lse),
+                                       _ptr(ws), ws.numel(), _stream(q)),
+           "thrift_qat_fwd_varlen")
+    return out.reshape(shape), out_hp.reshape(shape), lse
+
+
+def thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu_seqlens=None, max_seqlen=None, blk=128,
+                   causal=True, use_scalesearch=False, reuse_images=False, workspace=None):
+    """Attn-QAT backward: (dq like q, dk and dv like k, all f32).
+    reuse_images takes the fake-quantised images from ``workspace`` as the
+    forward on the same inputs left them (an explicit workspace is then
+    required)."""
+    _need_cuda(q, k, v, dout, out_hp, lse)
+    if reuse_images and workspace is None:
+        raise ThriftError("reuse_images needs the forward's workspace")
+    qshape, kshape = q.shape, k.shape
+    qp, kp, vp, cu, maxlen = _qat_pack(q, k, v, cu_seqlens, max_seqlen)
+    dop = dout.reshape(qp.shape)
+    ohp = out_hp.reshape(qp.shape)
+    for t in (qp, kp, vp, dop, ohp, lse):
+        if not t.is_contiguous():
+            raise ThriftError("thrift_qat_bwd: inputs must be contiguous")
+    if dout.dtype != q.dtype or out_hp.dtype != torch.float32 or lse.dtype != torch.float32:
+        raise ThriftError("thrift_qat_bwd: dout in the input type, out_hp and lse float32")
+    total, H, d = qp.shape
+    Hkv = kp.shape[1]
+    dq = torch.empty(qp.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(kp.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(kp.shape, dtype=torch.float32, device=q.device)
+    need = qat_workspace_size(total, H, Hkv, d)
+    if need == 0:
+        raise ThriftError("thrift_qat_bwd: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    _check(lib().thrift_qat_bwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(dop), _dt(q), _ptr(cu),
+                                       cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
+                                       int(use_scalesearch), int(reuse_images), _ptr(ohp),
+                                       _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                       ws.numel(), _stream(q)),
+           "thrift_qat_bwd_varlen")
+    return dq.reshape(qshape), dk.reshape(kshape), dv.reshape(kshape)

@@ -96,6 +96,28 @@ C_DECODE131K = DecodeWorkload("decode_b4h32hkv8_ctx131072_bf16_top10", 4, 32, 8,
                               131072, 131072, 128, torch.bfloat16, 0.10, False)
 
 
+@dataclass
+class QatWorkload:
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    N: int
+    d: int
+    dtype: torch.dtype
+    causal: bool
+    blk: int
+    use_scalesearch: bool
+    k_offset_std: float = 3.0
+    seed: int = 0
+
+
+# Attn-QAT training step (forward + backward) at the Llama-3.1-8B attention
+# shape and a 4k training context; the pages give no training shapes.
+C_QAT4K = QatWorkload("qat_b1h32hkv8n4096d128_bf16_causal", 1, 32, 8, 4096, 128, torch.bfloat16,
+                      True, 128, False)
+
+
 def varlen_lengths(gen: torch.Generator, nseq: int, lo: int, hi: int):
     """Integer lengths uniform on [lo, hi] (inclusive)."""
     return torch.randint(lo, hi + 1, (nseq,), generator=gen).tolist()
@@ -169,3 +191,25 @@ def as_u16(t: torch.Tensor):
 
 def dtype_code(dtype: torch.dtype) -> int:
     return {torch.float16: 0, torch.bfloat16: 1}[dtype]
+
+
+def make_qat_inputs(w: QatWorkload, seed: Optional[int] = None, lengths=None, device="cpu"):
+    """Returns dict(q [total,H,d], k, v [total,Hkv,d], dout [total,H,d],
+    cu_seqlens int32 [nseq+1], lengths).  Draw order: lengths (given, else
+    B x N) -> Q -> K -> V -> K channel offsets -> dO (the output gradient,
+    N(0,1))."""
+    gen = torch.Generator(device=device).manual_seed(w.seed if seed is None else seed)
+    if lengths is None:
+        lengths = [w.N] * w.B
+    total = int(sum(lengths))
+    f32 = torch.float32
+    q = torch.randn((total, w.H, w.d), generator=gen, dtype=f32, device=device)
+    k = torch.randn((total, w.Hkv, w.d), generator=gen, dtype=f32, device=device)
+    v = torch.randn((total, w.Hkv, w.d), generator=gen, dtype=f32, device=device)
+    if w.k_offset_std:
+        k += w.k_offset_std * torch.randn((w.Hkv, w.d), generator=gen, dtype=f32, device=device)
+    dout = torch.randn((total, w.H, w.d), generator=gen, dtype=f32, device=device)
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    return {"q": q.to(w.dtype), "k": k.to(w.dtype), "v": v.to(w.dtype), "dout": dout.to(w.dtype),
+            "cu_seqlens": cu, "lengths": list(lengths)}

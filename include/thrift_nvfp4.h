@@ -282,10 +282,63 @@ thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, i
                                  void* out, float* lse, void* workspace, size_t ws_bytes,
                                  void* stream);
 
+/* ------------------------------------------------------------ Attn-QAT --
+ * "Attn-QAT: 4-Bit Attention With Quantization-Aware Training",
+ * Metodologia: attention trained through a fake-quantised NVFP4 forward.
+ * The forward quantises Q and K (16-blocks along d), V (16-blocks along the
+ * tokens of each sequence, the last block zero-padded) with per-tensor
+ * scales g = amax / 2688 and the block scales of max scaling (ScaleSearch
+ * when use_scalesearch), computes S = Q^ K^T / sqrt(d),
+ * lse = log sum_j exp S, P = exp(S - lse), its two-level FP4 image P^ per
+ * (row, key tile of blk keys from the sequence start: sigma = tile row max /
+ * 2688, 16-key blocks of P / sigma with scale E4M3(amax / 6)), the FP4
+ * output O = P^ V^ and the high-precision output O' = P V^ (Metodologia 2).
+ * The backward recomputes P and P^ at the forward's precision (Metodologia
+ * 1) and returns, with every quantiser passing gradients straight through,
+ *   D = rowsum(dO o O'),  dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),
+ *   dQ = dS K^ / sqrt(d),  dK = dS^T Q^ / sqrt(d),
+ * dK and dV summed over the query heads of each kv head (H % Hkv == 0).
+ *
+ * Layout: packed sequences as in thrift_attn_fwd_varlen: q, dout 16-bit
+ * [total, H, d], k, v [total, Hkv, d], cu_seqlens int32 [nseq + 1] on the
+ * device (cu[0] = 0, non-decreasing, cu[nseq] = total), all contiguous and
+ * 16-byte aligned; max_seqlen >= every length.  causal: key j visible to
+ * query i iff j <= i within a sequence.  d in {64, 128}, blk in {64, 128}
+ * (else THRIFT_ERR_UNSUPPORTED).
+ *
+ * Outputs (caller-owned device memory): out [total, H, d] in the input
+ * type (O), out_hp fp32 [total, H, d] (O'), lse fp32 [H, total] (natural
+ * log); dq fp32 [total, H, d], dk, dv fp32 [total, Hkv, d].
+ *
+ * Workspace: thrift_qat_workspace_size(total, H, Hkv, d) bytes of device
+ * memory, 16-byte aligned; it holds the fake-quantised images (each element
+ * E2M1 value x UE4M3 block scale, exact in the input type), the tensor
+ * scales and D.  thrift_qat_bwd_varlen with reuse_images != 0 takes the
+ * images and scales from the workspace as a thrift_qat_fwd_varlen call on
+ * the same q, k, v, flags and workspace left them; with 0 it recomputes them.
+ *
+ * Errors: THRIFT_ERR_ARG for null or misaligned pointers, bad shapes or a
+ * short workspace (returned before any launch); THRIFT_ERR_CUDA if a launch
+ * fails.  Asynchronous on `stream`. */
+size_t thrift_qat_workspace_size(int64_t total, int H, int Hkv, int d);
+thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v, thrift_dtype dt,
+                                    const int32_t* cu_seqlens, int nseq, int64_t total,
+                                    int max_seqlen, int H, int Hkv, int d, int blk, int causal,
+                                    int use_scalesearch, void* out, float* out_hp, float* lse,
+                                    void* workspace, size_t ws_bytes, void* stream);
+thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v, const void* dout,
+                                    thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                    int64_t total, int max_seqlen, int H, int Hkv, int d, int blk,
+                                    int causal, int use_scalesearch, int reuse_images,
+                                    const float* out_hp, const float* lse, float* dq, float* dk,
+                                    float* dv, void* workspace, size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------- kernel timing --
  * Measurement aid (not part of the method).  While enabled, every
  * thrift_attn_fwd / thrift_attn_fwd_varlen call records a CUDA event pair on
- * its stream around the attention kernel launch.  thrift_kernel_timer_read
+ * its stream around the attention kernel launch (thrift_qat_fwd_varlen:
+ * around the forward kernel; thrift_qat_bwd_varlen: around its two
+ * gradient kernels).  thrift_kernel_timer_read
  * waits for the recorded events, returns the summed kernel time in
  * milliseconds and the number of timed launches, and clears the record.
  * Host-side state shared by all threads of the process; not thread-safe.
