@@ -447,6 +447,142 @@ def decode_only(args):
     return 0
 
 
+def qat_setup(ops, dev, w):
+    inp = synth.make_qat_inputs(w, device=dev)
+    q, k, v, dout = (inp[n] for n in ("q", "k", "v", "dout"))
+    cu = inp["cu_seqlens"].to(dev)
+    ws = torch.empty(ops.qat_workspace_size(q.shape[0], w.H, w.Hkv, w.d), dtype=torch.uint8,
+                     device=dev)
+    return inp, q, k, v, dout, cu, ws
+
+
+def qat_flops(w, lengths):
+    """Algorithmic FLOPs of one Attn-QAT step: the forward's S, P^V and PV and
+    the backward's dP, dV, dK and dQ, 2 d flops per visible (query, key)
+    pair each."""
+    pairs = sum(L * (L + 1) // 2 if w.causal else L * L for L in lengths) * w.H
+    return 7 * 2 * pairs * w.d, pairs
+
+
+# forward: 3 tensor absmax, 3 image kernels, the attention forward; backward
+# (images reused): D, the key-tile and the query-tile gradient kernels
+QAT_KERNELS_PER_STEP = 10
+
+
+def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
+    """Attn-QAT training step (forward + backward) of the QAT workload: the
+    forward quantises Q, K, V and writes O, O', lse; the backward reuses the
+    forward's images and returns dQ, dK, dV."""
+    w = synth.C_QAT4K
+    inp, q, k, v, dout, cu, ws = qat_setup(ops, dev, w)
+    N = w.N
+
+    def fwd():
+        return ops.thrift_qat_fwd(q, k, v, cu, N, blk=w.blk, causal=w.causal,
+                                  use_scalesearch=w.use_scalesearch, workspace=ws)
+
+    out, out_hp, lse = fwd()
+
+    def bwd():
+        return ops.thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu, N, blk=w.blk, causal=w.causal,
+                                  use_scalesearch=w.use_scalesearch, reuse_images=True,
+                                  workspace=ws)
+
+    for _ in range(warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the QAT warm-up")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps + 1)]
+    ev[0].record()
+    for i in range(steps):
+        fwd()
+        ev[2 * i + 1].record()
+        bwd()
+        ev[2 * i + 2].record()
+    torch.cuda.synchronize(dev)
+    fwd_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)) / steps
+    bwd_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(steps)) / steps
+    # the three attention kernels alone (event pairs around them)
+    ops.kernel_timer_enable(True)
+    for _ in range(steps):
+        fwd()
+        bwd()
+    kms, nk = ops.kernel_timer_read()
+    ops.kernel_timer_enable(False)
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out in the QAT loop")
+    flops, pairs = qat_flops(w, inp["lengths"])
+    step_ms = fwd_ms + bwd_ms
+    attn_ms = kms / steps
+    p16, src = peaks["bf16_tflops_sustained"], peak_src
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    line = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "causal": w.causal, "blk": w.blk, "dtype": "bf16",
+            "step": "forward (quantise, O, O', lse) + backward (dQ, dK, dV) reusing the "
+                    "forward's fake-quantised images",
+            "value": flops / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": step_ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "attention_kernels_ms": attn_ms, "algorithmic_flops": flops,
+            "roofline": {"bound": "tensor", "kernel": "qat_fwd + qat_bwd_kv + qat_bwd_q",
+                         "achieved": achieved, "peak": p16, "unit": "TFLOP/s",
+                         "frac": achieved / p16, "traffic": None,
+                         "peak_note": f"{src} bf16 sustained (the kernels run 16-bit MMAs)",
+                         "executed_mma_flops": 14 * 2 * pairs * w.d,
+                         "note": "7 algorithmic products; the kernels execute 14 (S recomputed "
+                                 "in each pass, dS and the P of O' as two 16-bit parts)"},
+            "kernels_per_step": QAT_KERNELS_PER_STEP, "steps": steps}
+    if not args.no_cpu_baseline:
+        # the oracle on a causal prefix of kv head 0 with its query heads: a
+        # complete smaller problem of the same shape per head
+        import oracle
+        cores = os.cpu_count() or 1
+        L = 1024
+        grp = w.H // w.Hkv
+        host = synth.make_qat_inputs(w)
+        sl = {n: synth.as_u16(host[n][:L, :grp].contiguous()) for n in ("q", "dout")}
+        sl.update({n: synth.as_u16(host[n][:L, :1].contiguous()) for n in ("k", "v")})
+        t0 = time.perf_counter()
+        oracle.attn_qat_bwd(sl["q"], sl["k"], sl["v"], sl["dout"], synth.dtype_code(w.dtype),
+                            np.array([0, L], np.int32), w.blk, w.causal, nthreads=cores)
+        dt = time.perf_counter() - t0
+        fl = 7 * 2 * (L * (L + 1) // 2) * grp * w.d
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "seconds": dt,
+                                "sample": f"first {L} tokens of kv head 0 with its {grp} query "
+                                          f"heads (a complete causal problem)"}
+    del q, k, v, dout, ws, out, out_hp, lse
+    torch.cuda.empty_cache()
+    return line
+
+
+def qat_only(args):
+    """A few Attn-QAT steps (profiling aid)."""
+    from bit_quantization_b200 import ops
+    dev = torch.device("cuda", 0)
+    w = synth.C_QAT4K
+    inp, q, k, v, dout, cu, ws = qat_setup(ops, dev, w)
+    times = []
+    for _ in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out, out_hp, lse = ops.thrift_qat_fwd(q, k, v, cu, w.N, blk=w.blk, causal=w.causal,
+                                              workspace=ws)
+        ops.thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu, w.N, blk=w.blk, causal=w.causal,
+                           reuse_images=True, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+    if ops.device_status(reset=True) != ops.OK:
+        raise RuntimeError("device wait timed out")
+    flops, _ = qat_flops(w, inp["lengths"])
+    best = min(times[args.warmup:])
+    print(json.dumps({"mode": "qat", "workload": w.name, "ms_min": best,
+                      "tflops": flops / (best * 1e-3) / 1e12}))
+    return 0
+
+
 def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20,
                       smooth=False):
     """Average attention-kernel time of the bench workload run with another
@@ -566,11 +702,13 @@ def main():
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantizer", action="store_true")
-    ap.add_argument("--mode", default="attention", choices=["attention", "quantizer", "decode"],
+    ap.add_argument("--mode", default="attention",
+                    choices=["attention", "quantizer", "decode", "qat"],
                     help="quantizer / decode: only a few plain calls of that path (profiling aid)")
     ap.add_argument("--decode-context", type=int, default=None,
                     help="cached tokens per sequence in --mode decode (default: the workload's)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-qat", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
@@ -580,6 +718,8 @@ def main():
         return quantizer_only(args)
     if args.mode == "decode":
         return decode_only(args)
+    if args.mode == "qat":
+        return qat_only(args)
 
     from bit_quantization_b200 import ops
     world, rank, local = dist.setup("nccl")
@@ -743,6 +883,8 @@ def main():
         del qd, kd, vd, od, ld
         torch.cuda.empty_cache()
         line["decode"] = decode_line(ops, dev, peaks)
+    if rank == 0 and world == 1 and not args.no_qat:
+        line["qat"] = qat_line(ops, dev, peaks, peak_src, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
         dt, fl, desc = oracle_sample(w, args.ref_units, cores, inp)

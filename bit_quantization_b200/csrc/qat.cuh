@@ -180,6 +180,20 @@ __device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const uint16_
   b1 = *reinterpret_cast<const uint32_t*>(p + 8);
 }
 
+// B fragments of n-tiles n0 and n0 + 8 for the k-step at row k0 of a
+// row-major tile whose rows run along the contraction (k) axis, transposed
+// on the way in by ldmatrix: b[0], b[1] for n-tile n0, b[2], b[3] for n0 + 8.
+// Lane l addresses row k0 + (l & 15), column n0 + 8 (l >> 4); rows are
+// 16-byte aligned and 8 consecutive rows hit distinct banks (LD = cols + 8).
+template <int LD>
+__device__ __forceinline__ void frag_b_t2(uint32_t (&b)[4], const uint16_t* t, int k0, int n0,
+                                          int lane) {
+  const uint32_t a = smem_u32(t + (k0 + (lane & 15)) * LD + n0 + 8 * (lane >> 4));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+               : "r"(a));
+}
+
 // The A fragment of k-step s from accumulator tiles c[2s], c[2s+1] (the C
 // layout of two n-tiles is the A layout of one 16-wide k-step).
 template <int DT>
@@ -222,24 +236,6 @@ __device__ __forceinline__ void stage_rows(uint16_t* t, const uint16_t* x, int64
   }
 }
 
-// The same rows transposed: tile [D][LDT], element (c, r) = x[r0 + r][c].
-template <int D, int R, int LDT>
-__device__ __forceinline__ void stage_rows_t(uint16_t* t, const uint16_t* x, int64_t st, int len,
-                                             int r0, int nh, int h) {
-  constexpr int CH = D / 8;
-  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
-    const int r = i % R, c = i / R;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r0 + r < len) v = __ldg(reinterpret_cast<const uint4*>(x + ((st + r0 + r) * nh + h) * D) + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      t[(8 * c + 2 * e) * LDT + r] = (uint16_t)(w[e] & 0xFFFF);
-      t[(8 * c + 2 * e + 1) * LDT + r] = (uint16_t)(w[e] >> 16);
-    }
-  }
-}
-
 __device__ __forceinline__ float quad_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
@@ -266,32 +262,32 @@ struct PBlock {
 
 template <int D, int BLK>
 struct QatFwdSmem {
-  static constexpr int LD = D + 8, LV = BLK + 8;
+  static constexpr int LD = D + 8;
   static constexpr int Q = 0;
   static constexpr int K = Q + kQatRows * LD;
-  static constexpr int VT = K + BLK * LD;
-  static constexpr size_t BYTES = (size_t)(VT + D * LV) * 2;
+  static constexpr int V = K + BLK * LD;
+  static constexpr size_t BYTES = (size_t)(V + BLK * LD) * 2;
 };
 
 // ------------------------------------------------------------- forward --
-// grid (ceil(maxlen / 64), H, nseq), 128 threads; warp w owns query rows
-// 16w..16w+15 of the tile.  Causal grids visit the tiles from the last (the
-// longest rows) first.
+// grid (ceil(maxlen / 64) * H, nseq), 128 threads, the tile index the
+// slowest: causal grids start the longest rows of every head first.  Warp w
+// owns query rows 16w..16w+15 of the tile.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
   using L = QatFwdSmem<D, BLK>;
-  constexpr int LD = L::LD, LV = L::LV, NT = BLK / 8, ND = D / 8;
+  constexpr int LD = L::LD, NT = BLK / 8, ND = D / 8;
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sQ = qsm + L::Q;
   uint16_t* sK = qsm + L::K;
-  uint16_t* sVt = qsm + L::VT;
+  uint16_t* sV = qsm + L::V;
   int64_t st;
   int len;
-  p.si.get(blockIdx.z, st, len);
+  p.si.get(blockIdx.y, st, len);
   const int tiles = (len + kQatRows - 1) / kQatRows;
-  if ((int)blockIdx.x >= tiles) return;
-  const int q0 = (p.causal ? tiles - 1 - (int)blockIdx.x : (int)blockIdx.x) * kQatRows;
-  const int h = blockIdx.y, hk = h / (p.H / p.Hkv);
+  const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
+  if (ti >= tiles) return;
+  const int q0 = (p.causal ? tiles - 1 - ti : ti) * kQatRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;
   const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
@@ -367,7 +363,7 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
   for (int kt = 0; kt < ntiles; ++kt) {
     __syncthreads();
     stage_rows<D, BLK, LD>(sK, p.ki, st, len, kt * BLK, p.Hkv, hk);
-    stage_rows_t<D, BLK, LV>(sVt, p.vi, st, len, kt * BLK, p.Hkv, hk);
+    stage_rows<D, BLK, LD>(sV, p.vi, st, len, kt * BLK, p.Hkv, hk);
     __syncthreads();
     float s[NT][4];
     scores(s, kt * BLK);
@@ -408,12 +404,15 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
       c_to_a<DT>(aq, qv[0], qv[1]);
       c_to_a_split<DT>(ph, pl, s[2 * b], s[2 * b + 1]);
 #pragma unroll
-      for (int n = 0; n < ND; ++n) {
-        uint32_t b0, b1;
-        frag_b<LV>(b0, b1, sVt, 8 * n, 16 * b, g, tq);
-        mma16816<DT>(o[n], aq, b0, b1);
-        mma16816<DT>(oh[n], ph, b0, b1);
-        mma16816<DT>(oh[n], pl, b0, b1);
+      for (int n = 0; n < ND; n += 2) {
+        uint32_t bb[4];
+        frag_b_t2<LD>(bb, sV, 16 * b, 8 * n, lane);
+        mma16816<DT>(o[n], aq, bb[0], bb[1]);
+        mma16816<DT>(oh[n], ph, bb[0], bb[1]);
+        mma16816<DT>(oh[n], pl, bb[0], bb[1]);
+        mma16816<DT>(o[n + 1], aq, bb[2], bb[3]);
+        mma16816<DT>(oh[n + 1], ph, bb[2], bb[3]);
+        mma16816<DT>(oh[n + 1], pl, bb[2], bb[3]);
       }
     }
   }
@@ -454,40 +453,37 @@ __global__ void __launch_bounds__(256) qat_rowdot_kernel(const uint16_t* __restr
 
 template <int D, int BLK>
 struct QatKvSmem {
-  static constexpr int LD = D + 8, LT = kQatChunk + 8, NW = BLK / 16;
+  static constexpr int LD = D + 8, NW = BLK / 16;
   static constexpr int K = 0;
   static constexpr int V = K + BLK * LD;
   static constexpr int Q = V + BLK * LD;
   static constexpr int DO = Q + kQatChunk * LD;
-  static constexpr int QT = DO + kQatChunk * LD;
-  static constexpr int DOT = QT + D * LT;
-  static constexpr int END16 = DOT + D * LT;  // 16-bit elements; fp32 arrays follow
+  static constexpr int END16 = DO + kQatChunk * LD;  // 16-bit elements; fp32 arrays follow
   static constexpr size_t BYTES = (size_t)END16 * 2 + (size_t)(2 + NW) * kQatChunk * 4;
 };
 
 // ------------------------------------------------- backward: dK and dV --
-// grid (ceil(maxlen / BLK), Hkv, nseq), BLK / 16 warps; warp w owns keys
-// 16w..16w+15 of the tile (one 16-key block of the P quantisation).
+// grid (ceil(maxlen / BLK) * Hkv, nseq), BLK / 16 warps, the key tile the
+// slowest (causal grids start the tiles with the most queries first); warp w
+// owns keys 16w..16w+15 of the tile (one 16-key block of the P
+// quantisation).
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
   using L = QatKvSmem<D, BLK>;
-  constexpr int LD = L::LD, LT = L::LT, NW = L::NW, QC = kQatChunk, NQ = QC / 8, ND = D / 8;
+  constexpr int LD = L::LD, NW = L::NW, QC = kQatChunk, NQ = QC / 8, ND = D / 8;
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sK = qsm + L::K;
   uint16_t* sV = qsm + L::V;
   uint16_t* sQ = qsm + L::Q;
   uint16_t* sdO = qsm + L::DO;
-  uint16_t* sQt = qsm + L::QT;
-  uint16_t* sdOt = qsm + L::DOT;
   float* s_lse2 = reinterpret_cast<float*>(qsm + L::END16);
   float* s_D = s_lse2 + QC;
   float* s_cmax = s_D + QC;  // [NW][QC]
   int64_t st;
   int len;
-  p.si.get(blockIdx.z, st, len);
-  const int j0 = blockIdx.x * BLK;
+  p.si.get(blockIdx.y, st, len);
+  const int j0 = (int)blockIdx.x / p.Hkv * BLK, hk = (int)blockIdx.x % p.Hkv, grp = p.H / p.Hkv;
   if (j0 >= len) return;
-  const int hk = blockIdx.y, grp = p.H / p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
   const int key[2] = {j0 + 16 * warp + g, j0 + 16 * warp + g + 8};
@@ -506,8 +502,6 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
       __syncthreads();
       stage_rows<D, QC, LD>(sQ, p.qi, st, len, qc0, p.H, h);
       stage_rows<D, QC, LD>(sdO, p.dout, st, len, qc0, p.H, h);
-      stage_rows_t<D, QC, LT>(sQt, p.qi, st, len, qc0, p.H, h);
-      stage_rows_t<D, QC, LT>(sdOt, p.dout, st, len, qc0, p.H, h);
       for (int i = threadIdx.x; i < QC; i += blockDim.x) {
         const bool ok = qc0 + i < len;
         s_lse2[i] = ok ? p.lse[(int64_t)h * p.total + st + qc0 + i] * kQatLog2e : 0.0f;
@@ -577,10 +571,11 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
         uint32_t a[4];
         c_to_a<DT>(a, qv[0], qv[1]);
 #pragma unroll
-        for (int n = 0; n < ND; ++n) {
-          uint32_t b0, b1;
-          frag_b<LT>(b0, b1, sdOt, 8 * n, 16 * b, g, tq);
-          mma16816<DT>(dv[n], a, b0, b1);
+        for (int n = 0; n < ND; n += 2) {
+          uint32_t bb[4];
+          frag_b_t2<LD>(bb, sdO, 16 * b, 8 * n, lane);
+          mma16816<DT>(dv[n], a, bb[0], bb[1]);
+          mma16816<DT>(dv[n + 1], a, bb[2], bb[3]);
         }
       }
       // dP^T = V^ dO^T, dS^T = P^T o (dP^T - D)
@@ -611,11 +606,13 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
         uint32_t ah[4], al[4];
         c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
 #pragma unroll
-        for (int n = 0; n < ND; ++n) {
-          uint32_t b0, b1;
-          frag_b<LT>(b0, b1, sQt, 8 * n, 16 * b, g, tq);
-          mma16816<DT>(dk[n], ah, b0, b1);
-          mma16816<DT>(dk[n], al, b0, b1);
+        for (int n = 0; n < ND; n += 2) {
+          uint32_t bb[4];
+          frag_b_t2<LD>(bb, sQ, 16 * b, 8 * n, lane);
+          mma16816<DT>(dk[n], ah, bb[0], bb[1]);
+          mma16816<DT>(dk[n], al, bb[0], bb[1]);
+          mma16816<DT>(dk[n + 1], ah, bb[2], bb[3]);
+          mma16816<DT>(dk[n + 1], al, bb[2], bb[3]);
         }
       }
     }
@@ -637,35 +634,34 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
 
 template <int D>
 struct QatQSmem {
-  static constexpr int LD = D + 8, LT = kQatChunk + 8;
+  static constexpr int LD = D + 8;
   static constexpr int Q = 0;
   static constexpr int DO = Q + kQatRows * LD;
   static constexpr int K = DO + kQatRows * LD;
   static constexpr int V = K + kQatChunk * LD;
-  static constexpr int KT = V + kQatChunk * LD;
-  static constexpr size_t BYTES = (size_t)(KT + D * LT) * 2;
+  static constexpr size_t BYTES = (size_t)(V + kQatChunk * LD) * 2;
 };
 
 // ------------------------------------------------------ backward: dQ --
-// grid (ceil(maxlen / 64), H, nseq), 128 threads; warp w owns query rows
-// 16w..16w+15; keys in chunks of 64.
+// grid (ceil(maxlen / 64) * H, nseq), 128 threads, the tile index the
+// slowest (causal grids start the longest rows first); warp w owns query
+// rows 16w..16w+15; keys in chunks of 64.
 template <int DT, int D>
 __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
   using L = QatQSmem<D>;
-  constexpr int LD = L::LD, LT = L::LT, KC = kQatChunk, NK = KC / 8, ND = D / 8;
+  constexpr int LD = L::LD, KC = kQatChunk, NK = KC / 8, ND = D / 8;
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sQ = qsm + L::Q;
   uint16_t* sdO = qsm + L::DO;
   uint16_t* sK = qsm + L::K;
   uint16_t* sV = qsm + L::V;
-  uint16_t* sKt = qsm + L::KT;
   int64_t st;
   int len;
-  p.si.get(blockIdx.z, st, len);
+  p.si.get(blockIdx.y, st, len);
   const int tiles = (len + kQatRows - 1) / kQatRows;
-  if ((int)blockIdx.x >= tiles) return;
-  const int q0 = (p.causal ? tiles - 1 - (int)blockIdx.x : (int)blockIdx.x) * kQatRows;
-  const int h = blockIdx.y, hk = h / (p.H / p.Hkv);
+  const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
+  if (ti >= tiles) return;
+  const int q0 = (p.causal ? tiles - 1 - ti : ti) * kQatRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
   const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
@@ -686,7 +682,6 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
     __syncthreads();
     stage_rows<D, KC, LD>(sK, p.ki, st, len, k0, p.Hkv, hk);
     stage_rows<D, KC, LD>(sV, p.vi, st, len, k0, p.Hkv, hk);
-    stage_rows_t<D, KC, LT>(sKt, p.ki, st, len, k0, p.Hkv, hk);
     __syncthreads();
     float s[NK][4], dp[NK][4];
 #pragma unroll
@@ -721,11 +716,13 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
       uint32_t ah[4], al[4];
       c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
 #pragma unroll
-      for (int n = 0; n < ND; ++n) {
-        uint32_t b0, b1;
-        frag_b<LT>(b0, b1, sKt, 8 * n, 16 * b, g, tq);
-        mma16816<DT>(dq[n], ah, b0, b1);
-        mma16816<DT>(dq[n], al, b0, b1);
+      for (int n = 0; n < ND; n += 2) {
+        uint32_t bb[4];
+        frag_b_t2<LD>(bb, sK, 16 * b, 8 * n, lane);
+        mma16816<DT>(dq[n], ah, bb[0], bb[1]);
+        mma16816<DT>(dq[n], al, bb[0], bb[1]);
+        mma16816<DT>(dq[n + 1], ah, bb[2], bb[3]);
+        mma16816<DT>(dq[n + 1], al, bb[2], bb[3]);
       }
     }
   }
