@@ -24,7 +24,8 @@
 // three attention kernels run warp-level m16n8k16 MMAs (fp32 accumulate) on
 // those images; P^ enters the MMAs rounded to the 16-bit type, dS and the P
 // of O' as sums of two 16-bit parts.
-//   qat_fwd_kernel     per 64-query tile: pass 1 lse, pass 2 P, P^, O, O'
+//   qat_fwd_kernel     per 64-query tile, one pass over the key tiles:
+//                      running max, P, its FP4 image, O, O', lse
 //   qat_rowdot_kernel  D = rowsum(dO o O')
 //   qat_bwd_kv_kernel  per key tile of blk keys, over every 64-query chunk
 //                      of the kv head's query heads: S^T, P^T, its FP4
@@ -236,6 +237,29 @@ __device__ __forceinline__ void stage_rows(uint16_t* t, const uint16_t* x, int64
   }
 }
 
+// The same rows through cp.async (16 bytes a copy, rows at or past len
+// zero-filled); the caller commits the group and waits for it.
+template <int D, int R, int LD>
+__device__ __forceinline__ void stage_rows_async(uint16_t* t, const uint16_t* x, int64_t st,
+                                                 int len, int r0, int nh, int h) {
+  constexpr int CH = D / 8;
+  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
+    const int r = i / CH, c = i % CH;
+    const bool ok = r0 + r < len;
+    const uint16_t* src = ok ? x + ((st + r0 + r) * nh + h) * D + 8 * c : x;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(t + r * LD + 8 * c)),
+                 "l"(src), "r"(ok ? 16 : 0)
+                 : "memory");
+  }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ float quad_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
@@ -264,23 +288,28 @@ template <int D, int BLK>
 struct QatFwdSmem {
   static constexpr int LD = D + 8;
   static constexpr int Q = 0;
-  static constexpr int K = Q + kQatRows * LD;
-  static constexpr int V = K + BLK * LD;
-  static constexpr size_t BYTES = (size_t)(V + BLK * LD) * 2;
+  static constexpr int K = Q + kQatRows * LD;  // two buffers of K and V each: the
+  static constexpr int V = K + 2 * BLK * LD;   // key tile in use and the next one
+  static constexpr size_t BYTES = (size_t)(V + 2 * BLK * LD) * 2;
 };
 
 // ------------------------------------------------------------- forward --
 // grid (ceil(maxlen / 64) * H, nseq), 128 threads, the tile index the
 // slowest: causal grids start the longest rows of every head first.  Warp w
 // owns query rows 16w..16w+15 of the tile.
+//
+// One pass over the key tiles with a running maximum m (log2 units): the
+// FP4 image of P on a key tile does not depend on lse, because
+// P / sigma = 2688 exp(S - max_tile S); the tile's sigma =
+// exp(max_tile S - lse) / 2688 enters as exp2(mt - m) / 2688 x (the rescale
+// of the running sums to the final m and the division by l), the same
+// bookkeeping as O' = sum exp2(s - m) V / l.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
   using L = QatFwdSmem<D, BLK>;
   constexpr int LD = L::LD, NT = BLK / 8, ND = D / 8;
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sQ = qsm + L::Q;
-  uint16_t* sK = qsm + L::K;
-  uint16_t* sV = qsm + L::V;
   int64_t st;
   int len;
   p.si.get(blockIdx.y, st, len);
@@ -294,9 +323,34 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
   const int kend = p.causal ? min(len, q0 + kQatRows) : len;
   const int ntiles = (kend + BLK - 1) / BLK;
 
-  stage_rows<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+  auto issue = [&](int kt) {
+    const int buf = kt & 1;
+    stage_rows_async<D, BLK, LD>(qsm + L::K + buf * BLK * LD, p.ki, st, len, kt * BLK, p.Hkv, hk);
+    stage_rows_async<D, BLK, LD>(qsm + L::V + buf * BLK * LD, p.vi, st, len, kt * BLK, p.Hkv, hk);
+  };
+  stage_rows_async<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+  issue(0);
+  cp_async_commit();
 
-  auto scores = [&](float (&s)[NT][4], int j0) {
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+  float o[ND][4], oh[ND][4];
+#pragma unroll
+  for (int n = 0; n < ND; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[n][e] = oh[n][e] = 0.0f;
+  for (int kt = 0; kt < ntiles; ++kt) {
+    const uint16_t* sK = qsm + L::K + (kt & 1) * BLK * LD;
+    const uint16_t* sV = qsm + L::V + (kt & 1) * BLK * LD;
+    if (kt + 1 < ntiles) {
+      issue(kt + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int j0 = kt * BLK;
+    float s[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
 #pragma unroll
@@ -310,7 +364,8 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
         mma16816<DT>(s[n], a, b0, b1);
       }
     }
-    // scale to log2 units and mask
+    // scores in log2 units, masked; tile row maxima; running maxima
+    float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -318,91 +373,62 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
         const int j = j0 + 8 * n + 2 * tq + (e & 1), i = row[e >> 1];
         const bool ok = j < len && (!p.causal || j <= i);
         s[n][e] = ok ? s[n][e] * c2 : -INFINITY;
+        mt[e >> 1] = fmaxf(mt[e >> 1], s[n][e]);
       }
-  };
-
-  // pass 1: row max and sum of exp in log2 units
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
-  for (int kt = 0; kt < ntiles; ++kt) {
-    __syncthreads();
-    stage_rows<D, BLK, LD>(sK, p.ki, st, len, kt * BLK, p.Hkv, hk);
-    __syncthreads();
-    float s[NT][4];
-    scores(s, kt * BLK);
+    float fct[2], inv2688 = 1.0f / kTensorScaleDiv;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int n = 0; n < NT; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
-      mx = quad_max(mx);
-      const float mn = fmaxf(m[r], mx);
-      if (mn == -INFINITY) continue;
-      float acc = m[r] == -INFINITY ? 0.0f : l[r] * exp2f(m[r] - mn);
-#pragma unroll
-      for (int n = 0; n < NT; ++n) acc += exp2f(s[n][2 * r] - mn) + exp2f(s[n][2 * r + 1] - mn);
-      l[r] = acc;
+      mt[r] = quad_max(mt[r]);
+      const float mn = fmaxf(m[r], mt[r]);
+      const float alpha = (m[r] == -INFINITY || mn == -INFINITY) ? 0.0f : exp2f(m[r] - mn);
       m[r] = mn;
-    }
-  }
-  float lse2[2];
+      l[r] *= alpha;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float t = l[r];
-    t += __shfl_xor_sync(0xffffffffu, t, 1);
-    t += __shfl_xor_sync(0xffffffffu, t, 2);
-    lse2[r] = m[r] + log2f(t);
-    if (tq == 0 && row[r] < len) p.lse[(int64_t)h * p.total + st + row[r]] = lse2[r] * kQatLn2;
-  }
-
-  // pass 2: P, its FP4 image, O and O'
-  float o[ND][4], oh[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[n][e] = oh[n][e] = 0.0f;
-  for (int kt = 0; kt < ntiles; ++kt) {
-    __syncthreads();
-    stage_rows<D, BLK, LD>(sK, p.ki, st, len, kt * BLK, p.Hkv, hk);
-    stage_rows<D, BLK, LD>(sV, p.vi, st, len, kt * BLK, p.Hkv, hk);
-    __syncthreads();
-    float s[NT][4];
-    scores(s, kt * BLK);
-    float inv[2], sig[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      float mx = 0.0f;
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        s[n][2 * r] = exp2f(s[n][2 * r] - lse2[r]);
-        s[n][2 * r + 1] = exp2f(s[n][2 * r + 1] - lse2[r]);
-        mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
+      for (int n = 0; n < ND; ++n) {
+        o[n][2 * r] *= alpha;
+        o[n][2 * r + 1] *= alpha;
+        oh[n][2 * r] *= alpha;
+        oh[n][2 * r + 1] *= alpha;
       }
-      mx = quad_max(mx);
-      inv[r] = mx > 0.0f ? __fdiv_rn(kTensorScaleDiv, mx) : 0.0f;
-      sig[r] = __fdiv_rn(mx, kTensorScaleDiv);
+      // sigma of this tile relative to the running maximum
+      fct[r] = mt[r] == -INFINITY ? 0.0f : exp2f(mt[r] - mn) * inv2688;
     }
+    // a row without a visible key in the tile has s = -inf throughout:
+    // finite references keep its exponentials at 0
+    const float mr[2] = {m[0] == -INFINITY ? 0.0f : m[0], m[1] == -INFINITY ? 0.0f : m[1]};
+    const float mtr[2] = {mt[0] == -INFINITY ? 0.0f : mt[0], mt[1] == -INFINITY ? 0.0f : mt[1]};
 #pragma unroll
     for (int b = 0; b < NT / 2; ++b) {
-      float qv[2][4];  // P^ of n-tiles 2b, 2b+1 in C layout
+      float qv[2][4], pe[2][4];  // P^ / (tile factor) and exp2(s - m), C layout
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float s0 = s[2 * b + u][2 * r], s1 = s[2 * b + u][2 * r + 1];
+          pe[u][2 * r] = exp2f(s0 - mr[r]);
+          pe[u][2 * r + 1] = exp2f(s1 - mr[r]);
+          l[r] += pe[u][2 * r] + pe[u][2 * r + 1];
+          // P / sigma of the oracle's reading: 2688 exp(S - max_tile S)
+          qv[u][2 * r] = kTensorScaleDiv * exp2f(s0 - mtr[r]);
+          qv[u][2 * r + 1] = kTensorScaleDiv * exp2f(s1 - mtr[r]);
+        }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const float x0 = __fmul_rn(s[2 * b][2 * r], inv[r]), x1 = __fmul_rn(s[2 * b][2 * r + 1], inv[r]);
-        const float x2 = __fmul_rn(s[2 * b + 1][2 * r], inv[r]);
-        const float x3 = __fmul_rn(s[2 * b + 1][2 * r + 1], inv[r]);
-        const PBlock pb(quad_max(fmaxf(fmaxf(x0, x1), fmaxf(x2, x3))));
-        float y0, y1, y2, y3;
-        pb.apply(x0, x1, y0, y1);
-        pb.apply(x2, x3, y2, y3);
-        qv[0][2 * r] = __fmul_rn(y0, sig[r]);
-        qv[0][2 * r + 1] = __fmul_rn(y1, sig[r]);
-        qv[1][2 * r] = __fmul_rn(y2, sig[r]);
-        qv[1][2 * r + 1] = __fmul_rn(y3, sig[r]);
+        const PBlock pb(quad_max(fmaxf(fmaxf(qv[0][2 * r], qv[0][2 * r + 1]),
+                                       fmaxf(qv[1][2 * r], qv[1][2 * r + 1]))));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          float y0, y1;
+          pb.apply(qv[u][2 * r], qv[u][2 * r + 1], y0, y1);
+          qv[u][2 * r] = __fmul_rn(y0, fct[r]);
+          qv[u][2 * r + 1] = __fmul_rn(y1, fct[r]);
+        }
       }
       // O' carries P in two parts: it sets D = rowsum(dO o O') of the
       // backward, whose error reaches dQ multiplied by the keys' means
       uint32_t aq[4], ph[4], pl[4];
       c_to_a<DT>(aq, qv[0], qv[1]);
-      c_to_a_split<DT>(ph, pl, s[2 * b], s[2 * b + 1]);
+      c_to_a_split<DT>(ph, pl, pe[0], pe[1]);
 #pragma unroll
       for (int n = 0; n < ND; n += 2) {
         uint32_t bb[4];
@@ -415,19 +441,25 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
         mma16816<DT>(oh[n + 1], pl, bb[2], bb[3]);
       }
     }
+    __syncthreads();  // every read of this buffer done before it is refilled
   }
   const float gv = p.g[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
+    float t = l[r];
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
     if (row[r] >= len) continue;
+    if (tq == 0) p.lse[(int64_t)h * p.total + st + row[r]] = (m[r] + log2f(t)) * kQatLn2;
+    const float sc_out = gv / t;
     const int64_t base = ((st + row[r]) * p.H + h) * D;
 #pragma unroll
     for (int n = 0; n < ND; ++n) {
       const int c = 8 * n + 2 * tq;
       *reinterpret_cast<uint32_t*>(p.out + base + c) =
-          qpack2<DT>(o[n][2 * r] * gv, o[n][2 * r + 1] * gv);
+          qpack2<DT>(o[n][2 * r] * sc_out, o[n][2 * r + 1] * sc_out);
       *reinterpret_cast<float2*>(p.out_hp + base + c) =
-          make_float2(oh[n][2 * r] * gv, oh[n][2 * r + 1] * gv);
+          make_float2(oh[n][2 * r] * sc_out, oh[n][2 * r + 1] * sc_out);
     }
   }
 }
@@ -456,10 +488,11 @@ struct QatKvSmem {
   static constexpr int LD = D + 8, NW = BLK / 16;
   static constexpr int K = 0;
   static constexpr int V = K + BLK * LD;
-  static constexpr int Q = V + BLK * LD;
-  static constexpr int DO = Q + kQatChunk * LD;
-  static constexpr int END16 = DO + kQatChunk * LD;  // 16-bit elements; fp32 arrays follow
-  static constexpr size_t BYTES = (size_t)END16 * 2 + (size_t)(2 + NW) * kQatChunk * 4;
+  static constexpr int Q = V + BLK * LD;             // two buffers of [64][LD] each:
+  static constexpr int DO = Q + 2 * kQatChunk * LD;  // the chunk in use and the next one
+  static constexpr int END16 = DO + 2 * kQatChunk * LD;  // 16-bit elements; fp32 arrays follow
+  // fp32: lse (log2 units) [2][64], D [2][64], column maxima [NW][64]
+  static constexpr size_t BYTES = (size_t)END16 * 2 + (size_t)(4 + NW) * kQatChunk * 4;
 };
 
 // ------------------------------------------------- backward: dK and dV --
@@ -474,11 +507,9 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sK = qsm + L::K;
   uint16_t* sV = qsm + L::V;
-  uint16_t* sQ = qsm + L::Q;
-  uint16_t* sdO = qsm + L::DO;
-  float* s_lse2 = reinterpret_cast<float*>(qsm + L::END16);
-  float* s_D = s_lse2 + QC;
-  float* s_cmax = s_D + QC;  // [NW][QC]
+  float* s_lse2b = reinterpret_cast<float*>(qsm + L::END16);  // [2][QC]
+  float* s_Db = s_lse2b + 2 * QC;                               // [2][QC]
+  float* s_cmax = s_Db + 2 * QC;                                // [NW][QC]
   int64_t st;
   int len;
   p.si.get(blockIdx.y, st, len);
@@ -487,27 +518,47 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
   const int key[2] = {j0 + 16 * warp + g, j0 + 16 * warp + g + 8};
+  // query chunks: every head of the group, from the first chunk that sees a
+  // key of this tile; chunk it + 1 is fetched while chunk it is computed
+  const int qstart = p.causal ? j0 / QC * QC : 0;
+  const int nch = (len - qstart + QC - 1) / QC;
+  const int n_it = grp * nch;
+  auto issue = [&](int it) {
+    const int buf = it & 1, h = hk * grp + it / nch, qc0 = qstart + (it % nch) * QC;
+    stage_rows_async<D, QC, LD>(qsm + L::Q + buf * QC * LD, p.qi, st, len, qc0, p.H, h);
+    stage_rows_async<D, QC, LD>(qsm + L::DO + buf * QC * LD, p.dout, st, len, qc0, p.H, h);
+    for (int i = threadIdx.x; i < QC; i += blockDim.x) {
+      const bool ok = qc0 + i < len;
+      s_lse2b[buf * QC + i] = ok ? p.lse[(int64_t)h * p.total + st + qc0 + i] * kQatLog2e : 0.0f;
+      s_Db[buf * QC + i] = ok ? p.dsum[(int64_t)h * p.total + st + qc0 + i] : 0.0f;
+    }
+  };
 
-  stage_rows<D, BLK, LD>(sK, p.ki, st, len, j0, p.Hkv, hk);
-  stage_rows<D, BLK, LD>(sV, p.vi, st, len, j0, p.Hkv, hk);
+  stage_rows_async<D, BLK, LD>(sK, p.ki, st, len, j0, p.Hkv, hk);
+  stage_rows_async<D, BLK, LD>(sV, p.vi, st, len, j0, p.Hkv, hk);
+  issue(0);
+  cp_async_commit();
   float dk[ND][4], dv[ND][4];
 #pragma unroll
   for (int n = 0; n < ND; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.0f;
 
-  for (int hh = 0; hh < grp; ++hh) {
-    const int h = hk * grp + hh;
-    for (int qc0 = p.causal ? j0 / QC * QC : 0; qc0 < len; qc0 += QC) {
-      __syncthreads();
-      stage_rows<D, QC, LD>(sQ, p.qi, st, len, qc0, p.H, h);
-      stage_rows<D, QC, LD>(sdO, p.dout, st, len, qc0, p.H, h);
-      for (int i = threadIdx.x; i < QC; i += blockDim.x) {
-        const bool ok = qc0 + i < len;
-        s_lse2[i] = ok ? p.lse[(int64_t)h * p.total + st + qc0 + i] * kQatLog2e : 0.0f;
-        s_D[i] = ok ? p.dsum[(int64_t)h * p.total + st + qc0 + i] : 0.0f;
-      }
-      __syncthreads();
+  for (int it = 0; it < n_it; ++it) {
+    if (it + 1 < n_it) {
+      issue(it + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    {
+      const int buf = it & 1, qc0 = qstart + (it % nch) * QC;
+      const uint16_t* sQ = qsm + L::Q + buf * QC * LD;
+      const uint16_t* sdO = qsm + L::DO + buf * QC * LD;
+      const float* s_lse2 = s_lse2b + buf * QC;
+      const float* s_D = s_Db + buf * QC;
       // S^T (keys x queries) and P^T
       float s[NQ][4];
 #pragma unroll
@@ -616,6 +667,7 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
         }
       }
     }
+    __syncthreads();  // every read of this buffer done before it is refilled
   }
   const float kscale = p.g[0] * p.sc;
 #pragma unroll
@@ -637,9 +689,9 @@ struct QatQSmem {
   static constexpr int LD = D + 8;
   static constexpr int Q = 0;
   static constexpr int DO = Q + kQatRows * LD;
-  static constexpr int K = DO + kQatRows * LD;
-  static constexpr int V = K + kQatChunk * LD;
-  static constexpr size_t BYTES = (size_t)(V + kQatChunk * LD) * 2;
+  static constexpr int K = DO + kQatRows * LD;  // two buffers each: the key chunk
+  static constexpr int V = K + 2 * kQatChunk * LD;  // in use and the next one
+  static constexpr size_t BYTES = (size_t)(V + 2 * kQatChunk * LD) * 2;
 };
 
 // ------------------------------------------------------ backward: dQ --
@@ -653,8 +705,6 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sQ = qsm + L::Q;
   uint16_t* sdO = qsm + L::DO;
-  uint16_t* sK = qsm + L::K;
-  uint16_t* sV = qsm + L::V;
   int64_t st;
   int len;
   p.si.get(blockIdx.y, st, len);
@@ -672,16 +722,32 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
     lse2[r] = ok ? p.lse[(int64_t)h * p.total + st + row[r]] * kQatLog2e : 0.0f;
     dsum[r] = ok ? p.dsum[(int64_t)h * p.total + st + row[r]] : 0.0f;
   }
-  stage_rows<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
-  stage_rows<D, kQatRows, LD>(sdO, p.dout, st, len, q0, p.H, h);
   float dq[ND][4];
 #pragma unroll
   for (int n = 0; n < ND; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.0f;
   const int kend = p.causal ? min(len, q0 + kQatRows) : len;
-  for (int k0 = 0; k0 < kend; k0 += KC) {
-    __syncthreads();
-    stage_rows<D, KC, LD>(sK, p.ki, st, len, k0, p.Hkv, hk);
-    stage_rows<D, KC, LD>(sV, p.vi, st, len, k0, p.Hkv, hk);
+  const int n_it = (kend + KC - 1) / KC;
+  // key chunk it + 1 is fetched while chunk it is computed
+  auto issue = [&](int it) {
+    const int buf = it & 1;
+    stage_rows_async<D, KC, LD>(qsm + L::K + buf * KC * LD, p.ki, st, len, it * KC, p.Hkv, hk);
+    stage_rows_async<D, KC, LD>(qsm + L::V + buf * KC * LD, p.vi, st, len, it * KC, p.Hkv, hk);
+  };
+  stage_rows_async<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+  stage_rows_async<D, kQatRows, LD>(sdO, p.dout, st, len, q0, p.H, h);
+  issue(0);
+  cp_async_commit();
+  for (int it = 0; it < n_it; ++it) {
+    const int k0 = it * KC;
+    const uint16_t* sK = qsm + L::K + (it & 1) * KC * LD;
+    const uint16_t* sV = qsm + L::V + (it & 1) * KC * LD;
+    if (it + 1 < n_it) {
+      issue(it + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
     float s[NK][4], dp[NK][4];
 #pragma unroll
@@ -725,6 +791,7 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
         mma16816<DT>(dq[n + 1], al, bb[2], bb[3]);
       }
     }
+    __syncthreads();  // every read of this buffer done before it is refilled
   }
   const float qscale = p.g[1] * p.sc;
 #pragma unroll
