@@ -24,7 +24,7 @@
 // three attention kernels run warp-level m16n8k16 MMAs (fp32 accumulate) on
 // those images; P^ enters the MMAs rounded to the 16-bit type, dS and the P
 // of O' as sums of two 16-bit parts.
-//   qat_fwd_kernel     per 64-query tile, one pass over the key tiles:
+//   qat_fwd_kernel     per 128-query tile, one pass over the key tiles:
 //                      running max, P, its FP4 image, O, O', lse
 //   qat_rowdot_kernel  D = rowsum(dO o O')
 //   qat_bwd_kv_kernel  per key tile of blk keys, over every 64-query chunk
@@ -36,7 +36,8 @@
 
 namespace thrift {
 
-constexpr int kQatRows = 64;   // query rows of a forward / dQ CTA (4 warps x 16)
+constexpr int kQatFwdRows = 128;  // query rows of a forward CTA (8 warps x 16)
+constexpr int kQatRows = 64;   // query rows of a dQ CTA (4 warps x 16)
 constexpr int kQatChunk = 64;  // query chunk of the key-tile kernel, key chunk of the dQ kernel
 constexpr float kQatLog2e = 1.4426950408889634f;
 constexpr float kQatLn2 = 0.6931471805599453f;
@@ -288,15 +289,16 @@ template <int D, int BLK>
 struct QatFwdSmem {
   static constexpr int LD = D + 8;
   static constexpr int Q = 0;
-  static constexpr int K = Q + kQatRows * LD;  // two buffers of K and V each: the
+  static constexpr int K = Q + kQatFwdRows * LD;  // two buffers of K and V each: the
   static constexpr int V = K + 2 * BLK * LD;   // key tile in use and the next one
   static constexpr size_t BYTES = (size_t)(V + 2 * BLK * LD) * 2;
 };
 
 // ------------------------------------------------------------- forward --
-// grid (ceil(maxlen / 64) * H, nseq), 128 threads, the tile index the
+// grid (ceil(maxlen / 128) * H, nseq), 256 threads, the tile index the
 // slowest: causal grids start the longest rows of every head first.  Warp w
-// owns query rows 16w..16w+15 of the tile.
+// owns query rows 16w..16w+15 of the tile; the eight warps share the
+// double-buffered K and V tiles.
 //
 // One pass over the key tiles with a running maximum m (log2 units): the
 // FP4 image of P on a key tile does not depend on lse, because
@@ -305,22 +307,22 @@ struct QatFwdSmem {
 // of the running sums to the final m and the division by l), the same
 // bookkeeping as O' = sum exp2(s - m) V / l.
 template <int DT, int D, int BLK>
-__global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
+__global__ void __launch_bounds__(256) qat_fwd_kernel(QatParams p) {
   using L = QatFwdSmem<D, BLK>;
-  constexpr int LD = L::LD, NT = BLK / 8, ND = D / 8;
+  constexpr int LD = L::LD, NT = BLK / 8, ND = D / 8, ROWS = kQatFwdRows;
   extern __shared__ __align__(16) uint16_t qsm[];
   uint16_t* sQ = qsm + L::Q;
   int64_t st;
   int len;
   p.si.get(blockIdx.y, st, len);
-  const int tiles = (len + kQatRows - 1) / kQatRows;
+  const int tiles = (len + ROWS - 1) / ROWS;
   const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
   if (ti >= tiles) return;
-  const int q0 = (p.causal ? tiles - 1 - ti : ti) * kQatRows;
+  const int q0 = (p.causal ? tiles - 1 - ti : ti) * ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;
   const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
-  const int kend = p.causal ? min(len, q0 + kQatRows) : len;
+  const int kend = p.causal ? min(len, q0 + ROWS) : len;
   const int ntiles = (kend + BLK - 1) / BLK;
 
   auto issue = [&](int kt) {
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
     stage_rows_async<D, BLK, LD>(qsm + L::K + buf * BLK * LD, p.ki, st, len, kt * BLK, p.Hkv, hk);
     stage_rows_async<D, BLK, LD>(qsm + L::V + buf * BLK * LD, p.vi, st, len, kt * BLK, p.Hkv, hk);
   };
-  stage_rows_async<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
+  stage_rows_async<D, ROWS, LD>(sQ, p.qi, st, len, q0, p.H, h);
   issue(0);
   cp_async_commit();
 
@@ -433,11 +435,11 @@ __global__ void __launch_bounds__(128) qat_fwd_kernel(QatParams p) {
       for (int n = 0; n < ND; n += 2) {
         uint32_t bb[4];
         frag_b_t2<LD>(bb, sV, 16 * b, 8 * n, lane);
-        mma16816<DT>(o[n], aq, bb[0], bb[1]);
         mma16816<DT>(oh[n], ph, bb[0], bb[1]);
-        mma16816<DT>(oh[n], pl, bb[0], bb[1]);
-        mma16816<DT>(o[n + 1], aq, bb[2], bb[3]);
         mma16816<DT>(oh[n + 1], ph, bb[2], bb[3]);
+        mma16816<DT>(o[n], aq, bb[0], bb[1]);
+        mma16816<DT>(o[n + 1], aq, bb[2], bb[3]);
+        mma16816<DT>(oh[n], pl, bb[0], bb[1]);
         mma16816<DT>(oh[n + 1], pl, bb[2], bb[3]);
       }
     }
@@ -661,8 +663,8 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
           uint32_t bb[4];
           frag_b_t2<LD>(bb, sQ, 16 * b, 8 * n, lane);
           mma16816<DT>(dk[n], ah, bb[0], bb[1]);
-          mma16816<DT>(dk[n], al, bb[0], bb[1]);
           mma16816<DT>(dk[n + 1], ah, bb[2], bb[3]);
+          mma16816<DT>(dk[n], al, bb[0], bb[1]);
           mma16816<DT>(dk[n + 1], al, bb[2], bb[3]);
         }
       }
@@ -786,8 +788,8 @@ __global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
         uint32_t bb[4];
         frag_b_t2<LD>(bb, sK, 16 * b, 8 * n, lane);
         mma16816<DT>(dq[n], ah, bb[0], bb[1]);
-        mma16816<DT>(dq[n], al, bb[0], bb[1]);
         mma16816<DT>(dq[n + 1], ah, bb[2], bb[3]);
+        mma16816<DT>(dq[n], al, bb[0], bb[1]);
         mma16816<DT>(dq[n + 1], al, bb[2], bb[3]);
       }
     }

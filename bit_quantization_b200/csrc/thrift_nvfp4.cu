@@ -658,10 +658,10 @@ thrift_status qat_fwd_launch(const QatParams& p, int nseq, int maxlen, cudaStrea
   static bool attr = false;
   const size_t smem = QatFwdSmem<D, BLK>::BYTES;
   if (qat_smem_attr(qat_fwd_kernel<DT, D, BLK>, smem, attr) != THRIFT_OK) return THRIFT_ERR_CUDA;
-  const dim3 grid((unsigned)(ceil_div(maxlen, kQatRows) * p.H), nseq);
+  const dim3 grid((unsigned)(ceil_div(maxlen, kQatFwdRows) * p.H), nseq);
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
-  qat_fwd_kernel<DT, D, BLK><<<grid, 128, smem, st>>>(p);
+  qat_fwd_kernel<DT, D, BLK><<<grid, 256, smem, st>>>(p);
   const thrift_status s = launch_status();
   if (ev) cudaEventRecord(ev[1], st);
   return s;

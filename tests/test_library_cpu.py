@@ -132,3 +132,37 @@ def test_binding_fails_loudly_without_device():
     x = torch.zeros((16, 32), dtype=torch.float16)
     with pytest.raises(ops.ThriftError):
         ops.nvfp4_quantize(x)
+
+
+def test_qat_entry_points_check_arguments_before_launch(L):
+    """Attn-QAT: workspace size on the host, argument errors returned before
+    any launch (no device needed)."""
+    P = C.c_void_p
+    dummy, ws, big = P(4096), P(8192), 1 << 40
+    size = L.thrift_qat_workspace_size(1000, 8, 2, 128)
+    # three images in the input type, 2 x 16-byte scalars, D in fp32 (1024-byte slices)
+    assert size >= 1000 * (8 + 2 + 2) * 128 * 2 + 1000 * 8 * 4
+    assert L.thrift_qat_workspace_size(1000, 8, 2, 96) == 0
+    assert L.thrift_qat_workspace_size(0, 8, 2, 128) == 0
+
+    def fwd(d=128, blk=128, H=8, Hkv=2, q=dummy, cu=dummy, wsb=big, out=dummy):
+        return L.thrift_qat_fwd_varlen(q, dummy, dummy, 1, cu, 2, 1000, 600, H, Hkv, d, blk, 1, 0,
+                                       out, dummy, dummy, ws, wsb, None)
+
+    assert fwd(d=96) == ops.ERR_UNSUPPORTED
+    assert fwd(blk=32) == ops.ERR_UNSUPPORTED
+    assert fwd(Hkv=3) == ops.ERR_ARG
+    assert fwd(q=None) == ops.ERR_ARG
+    assert fwd(cu=None) == ops.ERR_ARG
+    assert fwd(out=None) == ops.ERR_ARG
+    assert fwd(q=P(4098)) == ops.ERR_ARG
+    assert fwd(wsb=16) == ops.ERR_ARG
+
+    def bwd(dout=dummy, dq=dummy, wsb=big):
+        return L.thrift_qat_bwd_varlen(dummy, dummy, dummy, dout, 1, dummy, 2, 1000, 600, 8, 2, 128,
+                                       128, 1, 0, 1, dummy, dummy, dq, dummy, dummy, ws, wsb, None)
+
+    assert bwd(dout=None) == ops.ERR_ARG
+    assert bwd(dq=None) == ops.ERR_ARG
+    assert bwd(dq=P(4100)) == ops.ERR_ARG
+    assert bwd(wsb=16) == ops.ERR_ARG
