@@ -72,6 +72,22 @@ def attn_traffic(w):
     return None
 
 
+# DRAM traffic per step of the three Attn-QAT attention kernels (forward,
+# key-tile and query-tile backward) from the ncu launch list of the QAT source
+# with this hash; reported only while the source is unchanged.
+QAT_TRAFFIC = {"src_sha16": "2359dd27247327d3", "workload": "qat_b1h32hkv8n4096d128_bf16_causal",
+               "bytes": int((97.8 + 91.5 + 110.9) * 1e6)}
+
+
+def qat_traffic(w):
+    import hashlib
+    path = os.path.join(ROOT, "bit_quantization_b200", "csrc", "qat.cuh")
+    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    if sha == QAT_TRAFFIC["src_sha16"] and w.name == QAT_TRAFFIC["workload"]:
+        return QAT_TRAFFIC["bytes"]
+    return None
+
+
 XU_OPS_PER_CLK_PER_SM = 16   # MUFU lanes per SM (4 per sub-partition)
 # MUFU operations per score element: one exp2, plus one exp2 and one log2 per
 # 16-key block for the block scale (the E2M1 / 16-bit converts do not use
@@ -527,7 +543,7 @@ def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
             "attention_kernels_ms": attn_ms, "algorithmic_flops": flops,
             "roofline": {"bound": "tensor", "kernel": "qat_fwd + qat_bwd_kv + qat_bwd_q",
                          "achieved": achieved, "peak": p16, "unit": "TFLOP/s",
-                         "frac": achieved / p16, "traffic": None,
+                         "frac": achieved / p16, "traffic": qat_traffic(w),
                          "peak_note": f"{src} bf16 sustained (the kernels run 16-bit MMAs)",
                          "executed_mma_flops": 14 * 2 * pairs * w.d,
                          "note": "7 algorithmic products; the kernels execute 14 (S recomputed "
