@@ -224,22 +224,9 @@ __device__ __forceinline__ void c_to_a_split(uint32_t (&hi)[4], uint32_t (&lo)[4
   }
 }
 
-// rows [r0, r0 + R) of a [tokens, nh, D] image (head h) -> tile [R][LD]; rows
-// at or past len are zero.
-template <int D, int R, int LD>
-__device__ __forceinline__ void stage_rows(uint16_t* t, const uint16_t* x, int64_t st, int len,
-                                           int r0, int nh, int h) {
-  constexpr int CH = D / 8;
-  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
-    const int r = i / CH, c = i % CH;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r0 + r < len) v = __ldg(reinterpret_cast<const uint4*>(x + ((st + r0 + r) * nh + h) * D) + c);
-    *reinterpret_cast<uint4*>(t + r * LD + 8 * c) = v;
-  }
-}
-
-// The same rows through cp.async (16 bytes a copy, rows at or past len
-// zero-filled); the caller commits the group and waits for it.
+// Rows [r0, r0 + R) of a [tokens, nh, D] image (head h) -> tile [R][LD]
+// through cp.async, 16 bytes a copy; rows at or past len are zero-filled.
+// The caller commits the group and waits for it.
 template <int D, int R, int LD>
 __device__ __forceinline__ void stage_rows_async(uint16_t* t, const uint16_t* x, int64_t st,
                                                  int len, int r0, int nh, int h) {
