@@ -630,9 +630,10 @@ thrift_status qat_smem_attr(Kernel kernel, size_t bytes, bool& done) {
 
 // Fake-quantised images of Q, K, V and their tensor scales.
 template <int DT>
-void qat_images(const void* q, const void* k, const void* v, SeqInfo si, int nseq, int64_t total,
-                int maxlen, int H, int Hkv, int d, int ss, const QatWs& w, cudaStream_t st) {
-  cudaMemsetAsync(w.amax, 0, 16, st);
+thrift_status qat_images(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
+                         int64_t total, int maxlen, int H, int Hkv, int d, int ss, const QatWs& w,
+                         cudaStream_t st) {
+  if (cudaMemsetAsync(w.amax, 0, 16, st) != cudaSuccess) return THRIFT_ERR_CUDA;
   launch_amax<DT>(q, total * H * d / 16, 0, w.amax + 0, st);
   launch_amax<DT>(k, total * Hkv * d / 16, 0, w.amax + 1, st);
   launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
@@ -651,6 +652,7 @@ void qat_images(const void* q, const void* k, const void* v, SeqInfo si, int nse
     qat_fq_v_kernel<DT, false><<<dim3((unsigned)ceil_div(maxlen, 16), nseq), kThreads, 0, st>>>(
         vp, si, Hkv * d, w.amax + 2, w.g + 2, w.vi);
   }
+  return launch_status();
 }
 
 template <int DT, int D, int BLK>
@@ -1094,11 +1096,11 @@ thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v,
   p.out_hp = out_hp;
   p.lse = lse;
   if (dt == THRIFT_BF16) {
-    qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-    return qat_fwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
+    s = qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+    return s != THRIFT_OK ? s : qat_fwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
   }
-  qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-  return qat_fwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
+  s = qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+  return s != THRIFT_OK ? s : qat_fwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
 }
 
 thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v, const void* dout,
@@ -1136,12 +1138,12 @@ thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v,
   p.dv = dv;
   if (dt == THRIFT_BF16) {
     if (!reuse_images)
-      qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-    return qat_bwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
+      s = qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+    return s != THRIFT_OK ? s : qat_bwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
   }
   if (!reuse_images)
-    qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-  return qat_bwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
+    s = qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
+  return s != THRIFT_OK ? s : qat_bwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
 }
 
 }  // extern "C"
