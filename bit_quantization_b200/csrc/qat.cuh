@@ -256,14 +256,16 @@ __device__ __forceinline__ float quad_max(float v) {
 // FP4 value of a probability already divided by sigma: the 16-key block's
 // scale byte from amax (the block's largest scaled value), then the E2M1 code
 // of x / scale; returns code value x scale (0 when the byte is 0).
+// rcp: the correctly rounded reciprocals of the UE4M3 values by byte
+// (qat_rcp_table), read instead of recomputed.
 struct PBlock {
   float dec, rr;
   bool zero;
-  __device__ __forceinline__ explicit PBlock(float amax) {
+  __device__ __forceinline__ PBlock(float amax, const float* rcp) {
     const uint32_t sp = ue4m3(__fdiv_rn(amax, 6.0f));
     zero = sp == 0;
     dec = ue4m3_decode(sp);
-    rr = zero ? 0.0f : __frcp_rn(dec);
+    rr = rcp[sp];
   }
   __device__ __forceinline__ void apply(float x0, float x1, float& q0, float& q1) const {
     e2m1x2_roundtrip(__fmul_rn(x0, rr), __fmul_rn(x1, rr), q0, q1);
@@ -272,13 +274,21 @@ struct PBlock {
   }
 };
 
+// Fills rcp[b] = 1 / ue4m3_value(b) for the bytes 1..126 (rcp[0] = 0) in
+// shared memory; the caller synchronises before use.
+__device__ __forceinline__ void qat_rcp_table(float* rcp) {
+  for (int b = threadIdx.x; b < 128; b += blockDim.x)
+    rcp[b] = (b == 0 || b == 127) ? 0.0f : __frcp_rn(ue4m3_decode((uint32_t)b));
+}
+
 template <int D, int BLK>
 struct QatFwdSmem {
   static constexpr int LD = D + 8;
   static constexpr int Q = 0;
   static constexpr int K = Q + kQatFwdRows * LD;  // two buffers of K and V each: the
   static constexpr int V = K + 2 * BLK * LD;   // key tile in use and the next one
-  static constexpr size_t BYTES = (size_t)(V + 2 * BLK * LD) * 2;
+  static constexpr int RCP = V + 2 * BLK * LD;  // 128 floats follow the 16-bit tiles
+  static constexpr size_t BYTES = (size_t)RCP * 2 + 128 * 4;
 };
 
 // ------------------------------------------------------------- forward --
@@ -317,6 +327,8 @@ __global__ void __launch_bounds__(256) qat_fwd_kernel(QatParams p) {
     stage_rows_async<D, BLK, LD>(qsm + L::K + buf * BLK * LD, p.ki, st, len, kt * BLK, p.Hkv, hk);
     stage_rows_async<D, BLK, LD>(qsm + L::V + buf * BLK * LD, p.vi, st, len, kt * BLK, p.Hkv, hk);
   };
+  float* s_rcp = reinterpret_cast<float*>(qsm + L::RCP);
+  qat_rcp_table(s_rcp);  // visible after the first barrier of the loop
   stage_rows_async<D, ROWS, LD>(sQ, p.qi, st, len, q0, p.H, h);
   issue(0);
   cp_async_commit();
@@ -404,7 +416,8 @@ __global__ void __launch_bounds__(256) qat_fwd_kernel(QatParams p) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const PBlock pb(quad_max(fmaxf(fmaxf(qv[0][2 * r], qv[0][2 * r + 1]),
-                                       fmaxf(qv[1][2 * r], qv[1][2 * r + 1]))));
+                                       fmaxf(qv[1][2 * r], qv[1][2 * r + 1]))),
+                        s_rcp);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           float y0, y1;
@@ -480,8 +493,10 @@ struct QatKvSmem {
   static constexpr int Q = V + BLK * LD;             // two buffers of [64][LD] each:
   static constexpr int DO = Q + 2 * kQatChunk * LD;  // the chunk in use and the next one
   static constexpr int END16 = DO + 2 * kQatChunk * LD;  // 16-bit elements; fp32 arrays follow
-  // fp32: lse (log2 units) [2][64], D [2][64], column maxima [NW][64]
-  static constexpr size_t BYTES = (size_t)END16 * 2 + (size_t)(4 + NW) * kQatChunk * 4;
+  // fp32: lse (log2 units) [2][64], D [2][64], column maxima [NW][64], the
+  // columns' 2688 / max and max / 2688 [2][64], UE4M3 reciprocals [128]
+  static constexpr size_t BYTES =
+      (size_t)END16 * 2 + (size_t)(6 + NW) * kQatChunk * 4 + 128 * 4;
 };
 
 // ------------------------------------------------- backward: dK and dV --
@@ -499,6 +514,9 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
   float* s_lse2b = reinterpret_cast<float*>(qsm + L::END16);  // [2][QC]
   float* s_Db = s_lse2b + 2 * QC;                               // [2][QC]
   float* s_cmax = s_Db + 2 * QC;                                // [NW][QC]
+  float* s_cinv = s_cmax + NW * QC;                             // [QC]
+  float* s_csig = s_cinv + QC;                                  // [QC]
+  float* s_rcp = s_csig + QC;                                   // [128]
   int64_t st;
   int len;
   p.si.get(blockIdx.y, st, len);
@@ -523,6 +541,7 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
     }
   };
 
+  qat_rcp_table(s_rcp);  // visible after the first barrier of the loop
   stage_rows_async<D, BLK, LD>(sK, p.ki, st, len, j0, p.Hkv, hk);
   stage_rows_async<D, BLK, LD>(sV, p.vi, st, len, j0, p.Hkv, hk);
   issue(0);
@@ -583,6 +602,15 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
           if (g == 0) s_cmax[warp * QC + 8 * n + 2 * tq + c] = v;
         }
       __syncthreads();
+      // per query column, once: the max over the key tile and its factors
+      for (int c = threadIdx.x; c < QC; c += blockDim.x) {
+        float cm = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) cm = fmaxf(cm, s_cmax[w * QC + c]);
+        s_cinv[c] = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
+        s_csig[c] = __fdiv_rn(cm, kTensorScaleDiv);
+      }
+      __syncthreads();
       // dV += P^^T dO, one 16-query k-step at a time
 #pragma unroll
       for (int b = 0; b < NQ / 2; ++b) {
@@ -592,17 +620,13 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int il = 8 * (2 * b + u) + 2 * tq + c;
-            float cm = 0.0f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) cm = fmaxf(cm, s_cmax[w * QC + il]);
-            const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
-            const float sig = __fdiv_rn(cm, kTensorScaleDiv);
+            const float inv = s_cinv[il], sig = s_csig[il];
             const float x0 = __fmul_rn(s[2 * b + u][c], inv), x1 = __fmul_rn(s[2 * b + u][c + 2], inv);
             float am = fmaxf(x0, x1);
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
-            const PBlock pb(am);
+            const PBlock pb(am, s_rcp);
             float y0, y1;
             pb.apply(x0, x1, y0, y1);
             qv[u][c] = __fmul_rn(y0, sig);
