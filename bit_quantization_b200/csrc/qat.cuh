@@ -14,7 +14,7 @@
 //       sigma = rowmax / 2688; the 16-key blocks of P / sigma are quantised
 //       with block scale E4M3(amax / 6) and no tensor scale
 //   O = P^ V^ (the FP4 output),  O' = P V^,  D = rowsum(dO o O')
-//   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),
+//   dV = (P^)^T dO,  dP = dO V^T,  dS = P o (dP - D),
 //   dQ = dS K^ / sqrt(d),  dK = dS^T Q^ / sqrt(d)
 //   (dK, dV summed over the query heads of a kv head)
 //
@@ -23,13 +23,15 @@
 // with the tensor scales applied to the fp32 accumulators instead.  The
 // three attention kernels run warp-level m16n8k16 MMAs (fp32 accumulate) on
 // those images; P^ enters the MMAs rounded to the 16-bit type, dS and the P
-// of O' as sums of two 16-bit parts.
+// of O' as sums of two 16-bit parts.  Operand tiles are staged by cp.async
+// with the next tile in flight; B operands that run along the rows of a
+// staged tile are transposed by ldmatrix.
 //   qat_fwd_kernel     per 128-query tile, one pass over the key tiles:
 //                      running max, P, its FP4 image, O, O', lse
 //   qat_rowdot_kernel  D = rowsum(dO o O')
 //   qat_bwd_kv_kernel  per key tile of blk keys, over every 64-query chunk
 //                      of the kv head's query heads: S^T, P^T, its FP4
-//                      image, dP^T, dS^T; dV += P^^T dO, dK += dS^T Q^
+//                      image, dP^T, dS^T; dV += (P^)^T dO, dK += dS^T Q^
 //   qat_bwd_q_kernel   per 64-query tile: S, P, dP, dS; dQ += dS K^
 #pragma once
 #include "quant_kernels.cuh"
@@ -611,7 +613,7 @@ __global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
         s_csig[c] = __fdiv_rn(cm, kTensorScaleDiv);
       }
       __syncthreads();
-      // dV += P^^T dO, one 16-query k-step at a time
+      // dV += (P^)^T dO, one 16-query k-step at a time
 #pragma unroll
       for (int b = 0; b < NQ / 2; ++b) {
         float qv[2][4];
