@@ -3,6 +3,8 @@ the bench times: the GPU computes every output; the oracle computes the
 whole quantisation and selection and then a sample of query blocks (first,
 last, middle and diagonal-heavy ones), compared row by row with the bar of
 test_attn_gpu.py.  Also the longest sequence a call accepts (512 key tiles).
+Each case also prints its error against unquantised fp64 attention on the
+sampled rows (a report, not a bound).
 """
 import numpy as np
 import pytest
@@ -63,7 +65,19 @@ def _run(orc, w, picks, lengths=None):
     units = _units_for(lengths, w.H, w.blk, picks)
     r = orc.thrift_attn(qp, kp, vp, synth.dtype_code(w.dtype), cu, w.blk, w.causal, w.topk_frac,
                         use_ss=w.use_scalesearch, use_had=w.use_hadamard, units=units)
-    return _check_units(orc, gotf, r, cu, units, w.blk, w.dtype)
+    err = _check_units(orc, gotf, r, cu, units, w.blk, w.dtype)
+    # reported, not asserted: the error of the quantised result against
+    # unquantised fp64 attention on the same rows
+    rows = np.array([(t, h) for s, h, i in units
+                     for t in range(cu[s] + i * w.blk, min(cu[s + 1], cu[s] + (i + 1) * w.blk))],
+                    np.int64)
+    ref, _ = orc.attn_fp64(qp, kp, vp, synth.dtype_code(w.dtype), cu, w.causal, rows=rows)
+    g = gotf[rows[:, 0], rows[:, 1]].ravel()
+    f = ref[rows[:, 0], rows[:, 1]].ravel()
+    print(f"\n{w.name} topk {w.topk_frac}: vs unquantised fp64 attention on {len(rows)} rows: "
+          f"max abs {np.abs(g - f).max():.3e}, rms {np.sqrt(np.mean((g - f) ** 2)):.3e} "
+          f"(rms of the fp64 output {np.sqrt(np.mean(f ** 2)):.3e})")
+    return err
 
 
 def test_b2h32n8192_noncausal_top10(orc):
