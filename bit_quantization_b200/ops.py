@@ -125,6 +125,35 @@ def _dt(t: torch.Tensor) -> int:
     raise ThriftError(f"unsupported dtype {t.dtype}")
 
 
+def _check_qkv(q, k, v=None, packed=False):
+    """Shapes and dtypes of attention inputs, checked before anything reaches
+    the device: q [B,N,H,d] (packed: [total,H,d]), k and v [B,N,Hkv,d]
+    ([total,Hkv,d]) in one 16-bit type, H a multiple of Hkv."""
+    nd = 3 if packed else 4
+    ts = [("q", q), ("k", k)] + ([("v", v)] if v is not None else [])
+    for name, t in ts:
+        if t.dim() != nd:
+            raise ThriftError(f"{name} must have {nd} dimensions, got {tuple(t.shape)}")
+        if t.dtype != q.dtype:
+            raise ThriftError(f"{name} has dtype {t.dtype}, q has {q.dtype}")
+    _dt(q)
+    if v is not None and v.shape != k.shape:
+        raise ThriftError(f"v {tuple(v.shape)} and k {tuple(k.shape)} differ")
+    if q.shape[:-2] != k.shape[:-2] or q.shape[-1] != k.shape[-1]:
+        raise ThriftError(f"q {tuple(q.shape)} and k {tuple(k.shape)} differ outside the head axis")
+    if k.shape[-2] <= 0 or q.shape[-2] % k.shape[-2]:
+        raise ThriftError("the query heads must be a multiple of the kv heads")
+
+
+def _check_like(t, shape, dtype, name):
+    """A caller-supplied output or auxiliary tensor of a given shape and type."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ThriftError(f"{name} must be {dtype} of shape {tuple(shape)}, got {t.dtype} "
+                          f"{tuple(t.shape)}")
+
+
 def _need_cuda(*ts):
     for t in ts:
         if not t.is_cuda:
@@ -236,6 +265,7 @@ def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, to
     """q [B,N,H,d], k [B,N,Hkv,d] -> mask u8 [B,H,nB,nB] (1 = FP16 pair).
     sink_blocks / recent_blocks: fixed FP16 key blocks added to the top-k
     pairs (see the header)."""
+    _check_qkv(q, k)
     _need_cuda(q, k)
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -256,10 +286,12 @@ def block_mean_topk_noalloc(q: torch.Tensor, k: torch.Tensor, blk: int, causal: 
     """block_mean_topk with the library's fixed scratch instead of a workspace,
     for callers that cannot allocate device memory (see the header).  Pass
     `mask` to avoid the one allocation this wrapper would otherwise make."""
-    _need_cuda(q, k)
+    _check_qkv(q, k)
     B, N, H, d = q.shape
-    Hkv = k.shape[2]
     nB = (N + blk - 1) // blk
+    _check_like(mask, (B, H, nB, nB), torch.uint8, "mask")
+    _need_cuda(q, k)
+    Hkv = k.shape[2]
     if mask is None:
         mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
     _check(lib().block_mean_topk_noalloc(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk,
@@ -279,8 +311,11 @@ def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesear
                     use_hadamard=False, out=None, lse=None, workspace=None, sink_blocks=0,
                     recent_blocks=0, smooth_k=False):
     """q [B,N,H,d], k/v [B,N,Hkv,d] -> (out [B,N,H,d], lse f32 [B,H,N])."""
-    _need_cuda(q, k, v)
+    _check_qkv(q, k, v)
     B, N, H, d = q.shape
+    _check_like(out, q.shape, q.dtype, "out")
+    _check_like(lse, (B, H, N), torch.float32, "lse")
+    _need_cuda(q, k, v)
     Hkv = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
@@ -315,9 +350,12 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
                            smooth_k=False):
     """q [total,H,d], k/v [total,Hkv,d], cu_seqlens int32 [nseq+1] (CUDA) ->
     (out [total,H,d], lse f32 [H,total])."""
+    _check_qkv(q, k, v, packed=True)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ThriftError("cu_seqlens must be int32 [nseq + 1]")
+    _check_like(out, q.shape, q.dtype, "out")
+    _check_like(lse, (q.shape[1], q.shape[0]), torch.float32, "lse")
     _need_cuda(q, k, v, cu_seqlens)
-    if cu_seqlens.dtype != torch.int32:
-        raise ThriftError("cu_seqlens must be int32")
     total, H, d = q.shape
     Hkv = k.shape[1]
     nseq = cu_seqlens.numel() - 1
@@ -375,6 +413,11 @@ class DoubleKVCache:
         ``cache_len`` (int32 [B], device): the positions to write at, for a
         caller that keeps its own lengths (``self.lengths`` is then left as
         it is); by default ``self.lengths``, advanced by ``n_new``."""
+        if (k_new.dim() != 4 or k_new.shape != v_new.shape or k_new.shape[0] != self.B
+                or k_new.shape[2] != self.Hkv or k_new.shape[3] != self.d):
+            raise ThriftError(f"k_new, v_new must both be [B={self.B}, T, {self.Hkv}, {self.d}]")
+        if k_new.dtype != self.dtype or v_new.dtype != self.dtype:
+            raise ThriftError(f"k_new, v_new must be {self.dtype}")
         _need_cuda(k_new, v_new)
         B, T, Hkv, d = k_new.shape
         if n_new is None:
@@ -395,6 +438,12 @@ def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, re
     """q [B,H,d] -> (out [B,H,d], lse f32 [B,H]) against ``cache``
     (``seq_len``: int32 [B] device lengths to attend over instead of
     ``cache.lengths``)."""
+    if q.dim() != 3 or q.shape[0] != cache.B or q.shape[2] != cache.d or q.shape[1] % cache.Hkv:
+        raise ThriftError(f"q must be [B={cache.B}, H (a multiple of {cache.Hkv}), {cache.d}]")
+    if q.dtype != cache.dtype:
+        raise ThriftError(f"q has dtype {q.dtype}, the cache holds {cache.dtype}")
+    _check_like(out, q.shape, q.dtype, "out")
+    _check_like(lse, q.shape[:2], torch.float32, "lse")
     _need_cuda(q)
     B, H, d = q.shape
     if out is None:
@@ -442,6 +491,7 @@ def thrift_qat_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, blk=128, causal=Tr
     max_seqlen), k/v likewise with Hkv heads.  Returns (out like q in its
     dtype: the FP4 output, out_hp f32 like q: the high-precision output,
     lse f32 [H, total])."""
+    _check_qkv(q, k, v, packed=q.dim() == 3)
     _need_cuda(q, k, v)
     shape = q.shape
     qp, kp, vp, cu, maxlen = _qat_pack(q, k, v, cu_seqlens, max_seqlen)
@@ -471,6 +521,11 @@ def thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu_seqlens=None, max_seqlen=None,
     reuse_images takes the fake-quantised images from ``workspace`` as the
     forward on the same inputs left them (an explicit workspace is then
     required)."""
+    _check_qkv(q, k, v, packed=q.dim() == 3)
+    total_rows = q.shape[0] * (q.shape[1] if q.dim() == 4 else 1)
+    _check_like(dout, q.shape, q.dtype, "dout")
+    _check_like(out_hp, q.shape, torch.float32, "out_hp")
+    _check_like(lse, (q.shape[-2], total_rows), torch.float32, "lse")
     _need_cuda(q, k, v, dout, out_hp, lse)
     if reuse_images and workspace is None:
         raise ThriftError("reuse_images needs the forward's workspace")

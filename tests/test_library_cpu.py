@@ -166,3 +166,37 @@ def test_qat_entry_points_check_arguments_before_launch(L):
     assert bwd(dq=None) == ops.ERR_ARG
     assert bwd(dq=P(4100)) == ops.ERR_ARG
     assert bwd(wsb=16) == ops.ERR_ARG
+
+
+def test_binding_checks_shapes_before_the_device():
+    """Mismatched inputs are rejected on the host with their shapes, before
+    anything reaches a device (here: CPU tensors, so a consistent call only
+    fails for want of a device)."""
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros((1, 64, 4, 128), dtype=bf)
+    k = torch.zeros((1, 64, 2, 128), dtype=bf)
+    with pytest.raises(ops.ThriftError, match="differ"):
+        ops.thrift_attn_fwd(q, k, torch.zeros((1, 64, 2, 64), dtype=bf))
+    with pytest.raises(ops.ThriftError, match="differ outside the head axis"):
+        ops.thrift_attn_fwd(q, torch.zeros((1, 32, 2, 128), dtype=bf), torch.zeros((1, 32, 2, 128), dtype=bf))
+    with pytest.raises(ops.ThriftError, match="multiple of the kv heads"):
+        ops.thrift_attn_fwd(q, torch.zeros((1, 64, 3, 128), dtype=bf), torch.zeros((1, 64, 3, 128), dtype=bf))
+    with pytest.raises(ops.ThriftError, match="dtype"):
+        ops.thrift_attn_fwd(q, k.half(), k.half())
+    with pytest.raises(ops.ThriftError, match="lse must be"):
+        ops.thrift_attn_fwd(q, k, k, lse=torch.zeros((1, 4, 32)))
+    with pytest.raises(ops.ThriftError, match="dimensions"):
+        ops.block_mean_topk(q[0], k[0], 64, False, 0.1)
+    with pytest.raises(ops.ThriftError, match="cu_seqlens"):
+        ops.thrift_attn_fwd_varlen(q[0], k[0], k[0], torch.zeros(3, dtype=torch.int64), 64)
+    with pytest.raises(ops.ThriftError, match="dout must be"):
+        ops.thrift_qat_bwd(q, k, k, q.half(), torch.zeros(q.shape), torch.zeros((4, 64)))
+    with pytest.raises(ops.ThriftError, match="lse must be"):
+        ops.thrift_qat_bwd(q, k, k, q, torch.zeros(q.shape), torch.zeros((4, 32)))
+    # consistent shapes: only the device is missing
+    if not torch.cuda.is_available():
+        with pytest.raises(ops.ThriftError, match="CUDA device"):
+            ops.thrift_attn_fwd(q, k, k)
+        with pytest.raises(ops.ThriftError, match="CUDA device"):
+            ops.thrift_qat_bwd(q, k, k, q, torch.zeros(q.shape), torch.zeros((4, 64)))
