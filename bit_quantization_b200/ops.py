@@ -225,8 +225,15 @@ def nvfp4_quantize(x: torch.Tensor, use_scalesearch=False, use_hadamard=False,
                    workspace: Optional[torch.Tensor] = None):
     """x [rows, cols] fp16/bf16 on CUDA -> (codes u8 [rows, cols/2],
     scales u8 [rows, cols/16], tensor_scale f32 [1])."""
-    _need_cuda(x)
+    if x.dim() != 2:
+        raise ThriftError(f"x must be [rows, cols], got {tuple(x.shape)}")
     rows, cols = x.shape
+    _check_like(codes, (rows, cols // 2), torch.uint8, "codes")
+    _check_like(scales, (rows, cols // 16), torch.uint8, "scales")
+    if tensor_scale is not None and (tensor_scale.dtype != torch.float32 or
+                                     tensor_scale.numel() < 1):
+        raise ThriftError("tensor_scale must be float32 with at least one element")
+    _need_cuda(x)
     if codes is None:
         codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
     if scales is None:
@@ -244,6 +251,11 @@ def nvfp4_quantize(x: torch.Tensor, use_scalesearch=False, use_hadamard=False,
 def nvfp4_quantize_colblocks(x: torch.Tensor, use_scalesearch=False,
                              tensor_scale: Optional[torch.Tensor] = None):
     """x [rows, cols] -> (codes [cols, rows/2], scales [cols, rows/16], g)."""
+    if x.dim() != 2:
+        raise ThriftError(f"x must be [rows, cols], got {tuple(x.shape)}")
+    if tensor_scale is not None and (tensor_scale.dtype != torch.float32 or
+                                     tensor_scale.numel() < 1):
+        raise ThriftError("tensor_scale must be float32 with at least one element")
     _need_cuda(x)
     rows, cols = x.shape
     codes = torch.empty((cols, rows // 2), dtype=torch.uint8, device=x.device)

@@ -200,3 +200,16 @@ def test_binding_checks_shapes_before_the_device():
             ops.thrift_attn_fwd(q, k, k)
         with pytest.raises(ops.ThriftError, match="CUDA device"):
             ops.thrift_qat_bwd(q, k, k, q, torch.zeros(q.shape), torch.zeros((4, 64)))
+
+
+def test_quantiser_binding_checks_buffers_before_the_device():
+    import torch
+    x = torch.zeros((32, 64), dtype=torch.float16)
+    with pytest.raises(ops.ThriftError, match=r"x must be \[rows, cols\]"):
+        ops.nvfp4_quantize(x.reshape(2, 16, 64))
+    with pytest.raises(ops.ThriftError, match="codes must be"):
+        ops.nvfp4_quantize(x, codes=torch.zeros((32, 16), dtype=torch.uint8))
+    with pytest.raises(ops.ThriftError, match="scales must be"):
+        ops.nvfp4_quantize(x, scales=torch.zeros((32, 4), dtype=torch.int8))
+    with pytest.raises(ops.ThriftError, match="tensor_scale"):
+        ops.nvfp4_quantize_colblocks(x, tensor_scale=torch.zeros(1, dtype=torch.float16))
