@@ -57,7 +57,7 @@
 //      scores q^ . (k'^ + mu), i.e. the dequantised smoothed key with the
 //      mean added back, so both paths keep the same scores; the FP16 path and
 //      the selection use the raw K.  Not combined with the Hadamard rotation.
-//  R17 Attn-QAT backward ("Attn-QAT", Metodologia A and B): the forward
+//  R17 Attn-QAT backward ("Attn-QAT", Metodologia, items 1 and 2): the forward
 //      runs on fake-quantised NVFP4 Q^, K^, V^ (dequantised values) with the
 //      probabilities quantised in two levels per (row, key tile) as in R7;
 //      the backward treats every quantiser as the identity for gradients

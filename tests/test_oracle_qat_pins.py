@@ -1,5 +1,5 @@
 """Pins of the oracle's Attn-QAT backward (reading R17; "Attn-QAT",
-Metodologia A and B) against torch fp64 autograd of the same fake-quantised
+Metodologia, items 1 and 2) against torch fp64 autograd of the same fake-quantised
 graph with straight-through quantisers, an implementation of the gradient
 independent of the oracle's.  Autograd takes the softmax gradient's row
 scalar as rowsum(P o dP) = dO . (P V^), i.e. from the high-precision output
