@@ -106,3 +106,48 @@ def test_gradients_match_autograd_with_straight_through(orc, causal, H, Hkv):
     dS = P.detach() * (dP - Dn.T[:, :, None])
     dq_naive = torch.einsum("hij,jhc->ihc", dS, Kx.detach()) / np.sqrt(d)
     assert np.abs(dq_naive.numpy() - r["dq"]).max() > 1e-4 * np.abs(r["dq"]).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_p_hat_structure_through_identity_values(orc, causal):
+    """With V the identity (d = L), V^ = v I, so the oracle's outputs expose
+    the probabilities row by row: O' = v P and O = v P^.  Closed-form
+    properties of the two-level quantisation (reading R7 on the normalised
+    rows): on each key tile sigma = max P / 2688; each 16-key block of P^ is
+    (an E2M1 value) x (one UE4M3 value) x sigma; the tile maximum is
+    reproduced exactly (2688 / 6 = 448, the largest UE4M3 value, with code
+    6); and no element moves by more than one grid unit (the gap 4 -> 6 is
+    the widest) times its block's scale."""
+    rng = np.random.default_rng(11)
+    L, blk = 64, 32
+    q16 = _bf16(rng.standard_normal((L, 1, L)))
+    k16 = _bf16(rng.standard_normal((L, 1, L)))
+    v16 = _bf16(np.eye(L).reshape(L, 1, L))
+    do16 = _bf16(rng.standard_normal((L, 1, L)))
+    r = orc.attn_qat_bwd(q16, k16, v16, do16, BF16, np.array([0, L], np.int32), blk, causal)
+    vhat = _deq_v(orc, v16, L, 1, L)[:, 0, :]
+    vv = vhat[0, 0]
+    assert np.array_equal(vhat, vv * np.eye(L))  # one value on the diagonal
+    P = r["o_hp"][:, 0, :] / vv
+    Ph = r["o"][:, 0, :] / vv
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    scales = np.array([orc.ue4m3_decode([b])[0] for b in range(1, 127)], np.float64)
+    for i in range(L):
+        kend = i + 1 if causal else L
+        assert np.all(P[i, kend:] == 0) and np.all(Ph[i, kend:] == 0)
+        for j0 in range(0, kend, blk):
+            p, ph = P[i, j0:min(kend, j0 + blk)], Ph[i, j0:min(kend, j0 + blk)]
+            m = p.max()
+            sigma = float(np.float32(np.float32(m) / np.float32(2688.0)))
+            jm = int(np.argmax(p))
+            assert abs(ph[jm] - m) <= 4e-7 * m, (i, j0)
+            for b0 in range(0, len(p), 16):
+                blkv = ph[b0:b0 + 16] / sigma
+                if not blkv.any():
+                    continue
+                # one UE4M3 scale puts every element on the E2M1 grid
+                ok = [s for s in scales
+                      if np.all(np.min(np.abs(blkv[:, None] / s - grid[None, :]), axis=1) <= 1e-5)]
+                assert ok, (i, j0, b0)
+                s = min(ok, key=lambda x: abs(blkv.max() / x - 6))
+                assert np.all(np.abs(ph[b0:b0 + 16] - p[b0:b0 + 16]) <= (1.0 + 1e-5) * s * sigma)
