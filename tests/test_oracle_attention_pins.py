@@ -165,3 +165,56 @@ def test_sampled_units_equal_full_run(orc):
         rows = slice(cu[s] + 32 * i, cu[s] + 32 * (i + 1))
         assert np.array_equal(part["out"][rows, h], full["out"][rows, h])
         assert np.array_equal(part["lse"][h, rows], full["lse"][h, rows])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_nvfp4_probability_structure_through_identity_values(orc, causal):
+    """Two-level P quantisation (reading C8) seen through V = the identity
+    (d = N, every pair on the NVFP4 path): V^ is one value v on the diagonal,
+    so output column j of a row is v x (its FP4 probability) x a factor that
+    is constant over a key tile (sigma, the running-max rescale, 1 / l).  On
+    each key tile, 2688 x O_ij / O_i,argmax is then (an E2M1 value) x (one
+    UE4M3 value per 16-key block) -- the tile maximum maps to 2688 / 6 = 448
+    with code 6, as does every block maximum under a normal scale (max
+    scaling) -- and lies within one grid unit of the block scale from
+    2688 exp(S_ij - max_tile S), S the scores of the quantised Q and K."""
+    N, d, blk = 64, 64, 32
+    gen = torch.Generator().manual_seed(21)
+    q = torch.randn((N, 1, d), generator=gen).to(torch.bfloat16)
+    k = torch.randn((N, 1, d), generator=gen).to(torch.bfloat16)
+    v = torch.eye(N).reshape(N, 1, N).to(torch.bfloat16)
+    cu = np.array([0, N], np.int32)
+    r = orc.thrift_attn(synth.as_u16(q), synth.as_u16(k), synth.as_u16(v), 1, cu, blk, causal, 0.0)
+    O = r["out64"][:, 0, :]
+
+    def deq(x):
+        codes, scales, g, _ = orc.nvfp4_quantize(synth.as_u16(x).reshape(N, d), 1)
+        return orc.dequantize(codes, scales, g).astype(np.float64)
+
+    S = deq(q) @ deq(k).T / np.sqrt(d)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    scales = np.array([orc.ue4m3_decode([b])[0] for b in range(1, 127)], np.float64)
+    for i in range(N):
+        kend = i + 1 if causal else N
+        assert np.all(O[i, kend:] == 0)
+        for j0 in range(0, kend, blk):
+            j1 = min(kend, j0 + blk)
+            o, s = O[i, j0:j1], S[i, j0:j1]
+            jm = int(np.argmax(s))
+            assert o[jm] > 0 and o[jm] == o.max(), (i, j0)
+            rq = 2688.0 * o / o[jm]
+            exact = 2688.0 * np.exp(s - s[jm])
+            for b0 in range(0, j1 - j0, 16):
+                blkv = rq[b0:b0 + 16]
+                if not blkv.any():
+                    continue
+                ok = [t for t in scales
+                      if np.all(np.min(np.abs(blkv[:, None] / t - grid[None, :]), axis=1) <= 1e-6)]
+                assert ok, (i, j0, b0)
+                t = min(ok, key=lambda x: abs(blkv.max() / x - 6))
+                # max scaling: the block maximum carries code 6 (a normal
+                # UE4M3 scale rounds amax / 6 within 2^-4, so amax / S is in
+                # [5.65, 6.4] and rounds to 6)
+                if t >= 2.0 ** -6:
+                    assert abs(blkv.max() / t - 6.0) <= 1e-9, (i, j0, b0)
+                assert np.all(np.abs(blkv - exact[b0:b0 + 16]) <= (1.0 + 1e-4) * t), (i, j0, b0)

@@ -150,4 +150,7 @@ def test_p_hat_structure_through_identity_values(orc, causal):
                       if np.all(np.min(np.abs(blkv[:, None] / s - grid[None, :]), axis=1) <= 1e-5)]
                 assert ok, (i, j0, b0)
                 s = min(ok, key=lambda x: abs(blkv.max() / x - 6))
+                # max scaling: the block maximum carries code 6 (normal scales)
+                if s >= 2.0 ** -6:
+                    assert abs(blkv.max() / s - 6.0) <= 1e-5, (i, j0, b0)
                 assert np.all(np.abs(ph[b0:b0 + 16] - p[b0:b0 + 16]) <= (1.0 + 1e-5) * s * sigma)
