@@ -11,7 +11,7 @@
 // quantised in two levels (per row and key tile an fp32 factor rowmax/2688,
 // then NVFP4 16-key blocks).
 //
-// Roles (704 threads):
+// Roles (23 warps, 736 threads):
 //   warps 0-15  softmax, two groups of eight taking alternate key tiles;
 //               in a group, query row r (TMEM lane r) is shared by two
 //               warps, each owning half of the key columns; the groups take

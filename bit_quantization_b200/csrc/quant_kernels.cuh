@@ -130,10 +130,11 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
 // chunk of blocks once, takes the chunk absmax, publishes it, waits for all
 // CTAs (bounded wait), reduces the published maxima to the tensor absmax and
 // quantises its chunk from shared memory.  Same arithmetic as the two-pass
-// path.  sync[0] counts arrivals and sync[1] departures; the last CTA to
-// leave zeroes both, so the workspace is left as it was found (zeros).
-// partial[] has one float per CTA.  chunk is a multiple of 32 blocks (rows
-// stay whole for the Hadamard lanes).
+// path.  sync[0] counts arrivals; the launching code zeroes it on the stream
+// right before every launch, so nothing depends on what an earlier call (one
+// that timed out included) left in the workspace.  partial[] has one float
+// per CTA.  chunk is a multiple of 32 blocks (rows stay whole for the
+// Hadamard lanes).
 constexpr int kOnePassThreads = 512;
 
 template <int DT, int G, bool SS>
@@ -204,14 +205,7 @@ __global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
   float amax = 0.0f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
   const float g = tensor_scale_from_amax(__float_as_uint(amax));
-  if (threadIdx.x == 0) {
-    if (blockIdx.x == 0) *tensor_scale = g;
-    // the last CTA out leaves the counters at zero for the next call
-    if (atomicAdd(&sync[1], 1u) == gridDim.x - 1) {
-      sync[0] = 0u;
-      sync[1] = 0u;
-    }
-  }
+  if (threadIdx.x == 0 && blockIdx.x == 0) *tensor_scale = g;
   for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
     const int64_t b = b0 + i;
     float v[16];

@@ -2,6 +2,7 @@
 // carving and kernel launches.  Declarations and the contract of every entry
 // point are in include/thrift_nvfp4.h.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -45,17 +46,50 @@ struct Carve {
   }
 };
 
+// Device-side settings (function attributes, occupancy queries) apply to
+// the current device, so each is made once per device: bit `dev` of a
+// DeviceSet records that it has succeeded there.
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+struct DeviceSet {
+  std::atomic<uint64_t> bits{0};
+  bool has(int dev) const { return (bits.load() >> dev) & 1u; }
+  void add(int dev) { bits.fetch_or(1ull << dev); }
+};
+
+// Raises the dynamic shared-memory limit of `kernel` to `bytes` on the
+// current device (once per device).
+template <class Kernel>
+bool smem_attr(Kernel kernel, size_t bytes, DeviceSet& done) {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  if (done.has(dev)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return false;
+  done.add(dev);
+  return true;
+}
+
 // ------------------------------------------------------- quantiser glue --
 
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> n[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  if (n[dev].load() == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    n[dev].store(v);
   }
-  return n;
+  return n[dev].load();
 }
 
 // Grid for the streaming (grid-stride) kernels: enough CTAs for kKPT blocks
@@ -63,13 +97,16 @@ int sm_count() {
 // partial second wave trails the launch.
 template <class Kernel>
 int stream_grid(Kernel kernel, int64_t n_blocks) {
-  static int resident = 0;  // per kernel instantiation
+  static std::atomic<int> per_dev[kMaxDevices] = {};  // per kernel instantiation
+  const int dev = current_device();
+  int resident = dev < 0 ? 0 : per_dev[dev].load();
   if (resident == 0) {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
             cudaSuccess || per_sm < 1)
       per_sm = 1;
     resident = per_sm * sm_count();
+    if (dev >= 0) per_dev[dev].store(resident);
   }
   int64_t g = ceil_div(n_blocks, (int64_t)kThreads * kKPT);
   if (g < 1) g = 1;
@@ -99,9 +136,10 @@ void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, i
                                        codes, scales);
 }
 
-// Quantiser workspace: words 0 and 1 are the arrival and departure counts
-// of the one-pass kernel (zero between calls), word 2 the absmax of the
-// two-pass path, and from byte 256 one float per CTA of the one-pass kernel.
+// Quantiser workspace: word 0 is the arrival count of the one-pass kernel
+// (zeroed on the stream before each of its launches), word 2 the absmax of
+// the two-pass path, and from byte 256 one float per CTA of the one-pass
+// kernel.  No call depends on the workspace's earlier contents.
 constexpr size_t kQuantWsBytes = 4096;
 constexpr int kQuantMaxCtas = (int)((kQuantWsBytes - 256) / 4);
 constexpr int64_t kOnePassSmemMax = 200 * 1024;
@@ -117,13 +155,8 @@ bool try_quant_onepass(const void* x, int64_t nb, uint32_t* ws, float* ts, uint8
   const int64_t chunk = ceil_div(ceil_div(nb, (int64_t)grid), 32) * 32;
   const int64_t smem = chunk * 32;
   if (smem > kOnePassSmemMax) return false;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kOnePassSmemMax) != cudaSuccess)
-      return false;
-    attr = true;
-  }
+  static DeviceSet attr;
+  if (!smem_attr(kern, kOnePassSmemMax, attr)) return false;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kOnePassThreads,
                                                     (size_t)smem) != cudaSuccess ||
@@ -141,6 +174,8 @@ bool try_quant_onepass(const void* x, int64_t nb, uint32_t* ws, float* ts, uint8
   cfg.numAttrs = 1;
   const uint16_t* xp = static_cast<const uint16_t*>(x);
   float* partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
+  // the arrival counter starts from zero whatever an earlier call left there
+  if (cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return false;
   return cudaLaunchKernelEx(&cfg, kern, xp, nb, chunk, ws, partial, ts, codes, scales) ==
          cudaSuccess;
 }
@@ -267,14 +302,8 @@ KernelTimer g_timer;
 template <int DT, int D, int BLK>
 thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) {
   using L = AttnLayout<D, BLK>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<DT, D, BLK>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)L::SMEM_ALLOC) != cudaSuccess)
-      return THRIFT_ERR_CUDA;
-    attr_set = true;
-  }
+  static DeviceSet attr;
+  if (!smem_attr(attn_fwd_kernel<DT, D, BLK>, L::SMEM_ALLOC, attr)) return THRIFT_ERR_CUDA;
   dim3 grid(nTq, p.H, p.nseq);
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
@@ -328,13 +357,8 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
     const size_t smem = (size_t)blk * d * 2 + ((fp4_tile_bytes(d, blk) + 127) & ~127u) +
                         f16_tile_bytes(d, blk);
     auto kern = ss ? v_tile_kernel<DT, true> : v_tile_kernel<DT, false>;
-    static bool attr[2] = {false, false};
-    if (!attr[ss ? 1 : 0]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               96 * 1024) != cudaSuccess)
-        return THRIFT_ERR_CUDA;
-      attr[ss ? 1 : 0] = true;
-    }
+    static DeviceSet attr[2];
+    if (!smem_attr(kern, 96 * 1024, attr[ss ? 1 : 0])) return THRIFT_ERR_CUDA;
     kern<<<grid, kThreads, smem, st>>>(static_cast<const uint16_t*>(v), si, Hkv, d, blk, nB,
                                        w.amax + 2, w.v4, w.v16);
   }
@@ -385,13 +409,12 @@ thrift_status check_attn_args(const void* q, const void* k, const void* v, int d
 // that device current) and cached.
 constexpr size_t kNoAllocScratchBytes = THRIFT_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-constexpr int kMaxDevices = 64;
 void* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 thrift_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return THRIFT_ERR_CUDA;
+  const int dev = current_device();
+  if (dev < 0) return THRIFT_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
@@ -488,13 +511,8 @@ void launch_kv_append(const void* kn, const void* vn, const CacheGeom& cg, int m
 
 template <int DT, int GC>
 thrift_status launch_decode_kernel(const DecParams& p, int B, int Hkv, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_decode_kernel<DT, GC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)DecLayout::SMEM_ALLOC) != cudaSuccess)
-      return THRIFT_ERR_CUDA;
-    attr_set = true;
-  }
+  static DeviceSet attr;
+  if (!smem_attr(attn_decode_kernel<DT, GC>, DecLayout::SMEM_ALLOC, attr)) return THRIFT_ERR_CUDA;
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
   attn_decode_kernel<DT, GC><<<dim3(p.nsplit, Hkv, B), kDecThreads, DecLayout::SMEM_ALLOC, st>>>(p);
@@ -526,13 +544,8 @@ thrift_status decode_impl(const void* q, int B, int H, int Hkv, int capacity, co
                                                                 q_elems, w.q4, w.q16);
   const uint8_t* cp = static_cast<const uint8_t*>(cache);
   {
-    static bool attr_set = false;
-    if (!attr_set) {
-      if (cudaFuncSetAttribute(dec_scores_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)dec_scores_smem(kDecMaxG)) != cudaSuccess)
-        return THRIFT_ERR_CUDA;
-      attr_set = true;
-    }
+    static DeviceSet attr;
+    if (!smem_attr(dec_scores_kernel<DT>, dec_scores_smem(kDecMaxG), attr)) return THRIFT_ERR_CUDA;
     const int threads = kDecScoreTiles * std::max(G, 4);
     dec_scores_kernel<DT><<<dim3((unsigned)ceil_div(nbcap, kDecScoreTiles), Hkv, B), threads,
                             dec_scores_smem(G), st>>>(qp, H, G, cg, cp, seq_len, capacity, nbcap,
@@ -617,16 +630,6 @@ QatWs carve_qat(void* base, int64_t total, int H, int Hkv, int d) {
   return w;
 }
 
-template <class Kernel>
-thrift_status qat_smem_attr(Kernel kernel, size_t bytes, bool& done) {
-  if (!done) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
-      return THRIFT_ERR_CUDA;
-    done = true;
-  }
-  return THRIFT_OK;
-}
 
 // Fake-quantised images of Q, K, V and their tensor scales.
 template <int DT>
@@ -657,9 +660,9 @@ thrift_status qat_images(const void* q, const void* k, const void* v, SeqInfo si
 
 template <int DT, int D, int BLK>
 thrift_status qat_fwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
-  static bool attr = false;
+  static DeviceSet attr;
   const size_t smem = QatFwdSmem<D, BLK>::BYTES;
-  if (qat_smem_attr(qat_fwd_kernel<DT, D, BLK>, smem, attr) != THRIFT_OK) return THRIFT_ERR_CUDA;
+  if (!smem_attr(qat_fwd_kernel<DT, D, BLK>, smem, attr)) return THRIFT_ERR_CUDA;
   const dim3 grid((unsigned)(ceil_div(maxlen, kQatFwdRows) * p.H), nseq);
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
@@ -671,10 +674,10 @@ thrift_status qat_fwd_launch(const QatParams& p, int nseq, int maxlen, cudaStrea
 
 template <int DT, int D, int BLK>
 thrift_status qat_bwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
-  static bool attr_kv = false, attr_q = false;
+  static DeviceSet attr_kv, attr_q;
   const size_t skv = QatKvSmem<D, BLK>::BYTES, sq = QatQSmem<D>::BYTES;
-  if (qat_smem_attr(qat_bwd_kv_kernel<DT, D, BLK>, skv, attr_kv) != THRIFT_OK) return THRIFT_ERR_CUDA;
-  if (qat_smem_attr(qat_bwd_q_kernel<DT, D>, sq, attr_q) != THRIFT_OK) return THRIFT_ERR_CUDA;
+  if (!smem_attr(qat_bwd_kv_kernel<DT, D, BLK>, skv, attr_kv)) return THRIFT_ERR_CUDA;
+  if (!smem_attr(qat_bwd_q_kernel<DT, D>, sq, attr_q)) return THRIFT_ERR_CUDA;
   const int64_t rows = p.total * p.H;
   qat_rowdot_kernel<DT, D><<<grid_for(rows * 32), kThreads, 0, st>>>(p.dout, p.out_hp, p.total,
                                                                     p.H, const_cast<float*>(p.dsum));
@@ -750,6 +753,19 @@ thrift_status thrift_device_status(int reset) {
     if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess)
       return THRIFT_ERR_CUDA;
   }
+  return (thrift_status)v;
+}
+
+thrift_status thrift_stream_status(void* stream, int reset) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&word), g_device_status) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, word, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (reset && cudaMemsetAsync(word, 0, sizeof(int), st) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return THRIFT_ERR_CUDA;
   return (thrift_status)v;
 }
 

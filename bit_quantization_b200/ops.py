@@ -23,7 +23,8 @@ _lib = None
 
 # Exported names of the C ABI, in header order.
 EXPORTS = (
-    "thrift_status_string", "thrift_device_status", "nvfp4_quantize_workspace_size",
+    "thrift_status_string", "thrift_device_status", "thrift_stream_status",
+    "nvfp4_quantize_workspace_size",
     "nvfp4_quantize", "nvfp4_quantize_colblocks", "block_mean_topk_workspace_size",
     "block_mean_topk", "block_mean_topk_noalloc", "thrift_attn_workspace_size", "thrift_attn_fwd",
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
@@ -52,6 +53,8 @@ def lib():
         L.thrift_status_string.argtypes = [i32]
         L.thrift_device_status.restype = i32
         L.thrift_device_status.argtypes = [i32]
+        L.thrift_stream_status.restype = i32
+        L.thrift_stream_status.argtypes = [P, i32]
         L.nvfp4_quantize_workspace_size.restype = sz
         L.nvfp4_quantize_workspace_size.argtypes = []
         L.nvfp4_quantize.restype = i32
@@ -175,6 +178,21 @@ def device_status(reset: bool = False) -> int:
     return lib().thrift_device_status(int(reset))
 
 
+def stream_status(stream: Optional[torch.cuda.Stream] = None, reset: bool = False) -> int:
+    """Waits for ``stream`` only (default: the current stream) and returns the
+    device status word (OK or ERR_TIMEOUT), clearing it when ``reset``."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.device(st.device):
+        return lib().thrift_stream_status(C.c_void_p(st.cuda_stream), int(reset))
+
+
+def _on(t: torch.Tensor):
+    """Makes the tensor's device current around a library call (the library
+    resolves per-device state, such as the no-allocation scratch address, on
+    the current device)."""
+    return torch.cuda.device(t.device)
+
+
 def kernel_timer_enable(enable: bool):
     _check(lib().thrift_kernel_timer_enable(int(enable)), "thrift_kernel_timer_enable")
 
@@ -198,24 +216,31 @@ def test_wait_timeout(mode: int, limit_us: int, device=None):
 
 
 class Workspace:
-    """Grow-only device scratch buffer reused across calls on one device
-    (zero-filled when allocated if ``zeroed``)."""
+    """Grow-only device scratch buffers reused across calls, one per (device,
+    stream): a call uses the buffer of the stream it is queued on, so calls on
+    different streams never share scratch, and a buffer that grows is freed
+    back to the one stream that used it (allocated while that stream is
+    current, so the caching allocator reuses it only in that stream's order)."""
 
-    def __init__(self, zeroed=False):
-        self.buf: Optional[torch.Tensor] = None
-        self.zeroed = zeroed
+    def __init__(self):
+        self.bufs = {}
 
     def get(self, nbytes: int, device) -> torch.Tensor:
         nbytes = max(int(nbytes), 256)
-        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
-            alloc = torch.zeros if self.zeroed else torch.empty
-            self.buf = alloc(nbytes, dtype=torch.uint8, device=device)
-        return self.buf
+        device = torch.device(device)
+        stream = torch.cuda.current_stream(device)
+        key = (device.index, stream.cuda_stream)
+        buf = self.bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            self.bufs.pop(key, None)
+            with torch.cuda.device(device), torch.cuda.stream(stream):
+                buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            self.bufs[key] = buf
+        return buf
 
 
 _ws = Workspace()
-# the quantiser's own workspace: zero-filled, and left zero-filled by each call
-_qws = Workspace(zeroed=True)
+_qws = Workspace()  # the quantiser's (needs no initial contents)
 
 
 # ------------------------------------------------------------------ quantiser
@@ -242,9 +267,10 @@ def nvfp4_quantize(x: torch.Tensor, use_scalesearch=False, use_hadamard=False,
     ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
     ws = workspace if workspace is not None else _qws.get(lib().nvfp4_quantize_workspace_size(),
                                                           x.device)
-    _check(lib().nvfp4_quantize(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
-                                int(use_hadamard), int(given), _ptr(codes), _ptr(scales),
-                                _ptr(ts), _ptr(ws), ws.numel(), _stream(x)), "nvfp4_quantize")
+    with _on(x):
+        _check(lib().nvfp4_quantize(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
+                                    int(use_hadamard), int(given), _ptr(codes), _ptr(scales),
+                                    _ptr(ts), _ptr(ws), ws.numel(), _stream(x)), "nvfp4_quantize")
     return codes, scales, ts
 
 
@@ -263,10 +289,11 @@ def nvfp4_quantize_colblocks(x: torch.Tensor, use_scalesearch=False,
     given = tensor_scale is not None
     ts = tensor_scale if given else torch.empty(1, dtype=torch.float32, device=x.device)
     ws = _qws.get(lib().nvfp4_quantize_workspace_size(), x.device)
-    _check(lib().nvfp4_quantize_colblocks(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
-                                          int(given), _ptr(codes), _ptr(scales), _ptr(ts),
-                                          _ptr(ws), ws.numel(), _stream(x)),
-           "nvfp4_quantize_colblocks")
+    with _on(x):
+        _check(lib().nvfp4_quantize_colblocks(_ptr(x), _dt(x), rows, cols, int(use_scalesearch),
+                                              int(given), _ptr(codes), _ptr(scales), _ptr(ts),
+                                              _ptr(ws), ws.numel(), _stream(x)),
+               "nvfp4_quantize_colblocks")
     return codes, scales, ts
 
 
@@ -285,10 +312,11 @@ def block_mean_topk(q: torch.Tensor, k: torch.Tensor, blk: int, causal: bool, to
     mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
     need = lib().block_mean_topk_workspace_size(B, H, Hkv, N, d, blk)
     ws = _ws.get(need, q.device)
-    _check(lib().block_mean_topk(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk, int(causal),
-                                 float(topk_frac), int(sink_blocks), int(recent_blocks),
-                                 _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
-           "block_mean_topk")
+    with _on(q):
+        _check(lib().block_mean_topk(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk, int(causal),
+                                     float(topk_frac), int(sink_blocks), int(recent_blocks),
+                                     _ptr(mask), _ptr(ws), ws.numel(), _stream(q)),
+               "block_mean_topk")
     return mask
 
 
@@ -306,10 +334,11 @@ def block_mean_topk_noalloc(q: torch.Tensor, k: torch.Tensor, blk: int, causal: 
     Hkv = k.shape[2]
     if mask is None:
         mask = torch.empty((B, H, nB, nB), dtype=torch.uint8, device=q.device)
-    _check(lib().block_mean_topk_noalloc(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk,
-                                         int(causal), float(topk_frac), int(sink_blocks),
-                                         int(recent_blocks), _ptr(mask), _stream(q)),
-           "block_mean_topk_noalloc")
+    with _on(q):
+        _check(lib().block_mean_topk_noalloc(_ptr(q), _ptr(k), _dt(q), B, H, Hkv, N, d, blk,
+                                             int(causal), float(topk_frac), int(sink_blocks),
+                                             int(recent_blocks), _ptr(mask), _stream(q)),
+               "block_mean_topk_noalloc")
     return mask
 
 
@@ -337,12 +366,13 @@ def thrift_attn_fwd(q, k, v, blk=128, causal=False, topk_frac=0.0, use_scalesear
     if need == 0:
         raise ThriftError("thrift_attn_fwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
-    _check(lib().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, Hkv, N, d, blk,
-                                 int(causal), float(topk_frac), int(sink_blocks),
-                                 int(recent_blocks), int(use_scalesearch), int(use_hadamard),
-                                 int(smooth_k), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-                                 _stream(q)),
-           "thrift_attn_fwd")
+    with _on(q):
+        _check(lib().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, Hkv, N, d, blk,
+                                     int(causal), float(topk_frac), int(sink_blocks),
+                                     int(recent_blocks), int(use_scalesearch), int(use_hadamard),
+                                     int(smooth_k), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                     _stream(q)),
+               "thrift_attn_fwd")
     return out, lse
 
 
@@ -379,13 +409,14 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
     if need == 0:
         raise ThriftError("thrift_attn_fwd_varlen: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
-    _check(lib().thrift_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens),
-                                        nseq, total, int(max_seqlen), H, Hkv, d, blk,
-                                        int(causal), float(topk_frac), int(sink_blocks),
-                                        int(recent_blocks), int(use_scalesearch),
-                                        int(use_hadamard), int(smooth_k), _ptr(out), _ptr(lse),
-                                        _ptr(ws), ws.numel(), _stream(q)),
-           "thrift_attn_fwd_varlen")
+    with _on(q):
+        _check(lib().thrift_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens),
+                                            nseq, total, int(max_seqlen), H, Hkv, d, blk,
+                                            int(causal), float(topk_frac), int(sink_blocks),
+                                            int(recent_blocks), int(use_scalesearch),
+                                            int(use_hadamard), int(smooth_k), _ptr(out), _ptr(lse),
+                                            _ptr(ws), ws.numel(), _stream(q)),
+               "thrift_attn_fwd_varlen")
     return out, lse
 
 
@@ -435,11 +466,12 @@ class DoubleKVCache:
         if n_new is None:
             n_new = torch.full((B,), T, dtype=torch.int32, device=k_new.device)
         at = self.lengths if cache_len is None else cache_len
-        _check(lib().thrift_kv_cache_append(_ptr(k_new), _ptr(v_new), _dt(k_new), B, Hkv, d,
-                                            self.blk, self.capacity, _ptr(at), _ptr(n_new), T,
-                                            _ptr(self.kv_scale), int(self.use_scalesearch),
-                                            _ptr(self.buf), self.buf.numel(), _stream(k_new)),
-               "thrift_kv_cache_append")
+        with _on(k_new):
+            _check(lib().thrift_kv_cache_append(_ptr(k_new), _ptr(v_new), _dt(k_new), B, Hkv, d,
+                                                self.blk, self.capacity, _ptr(at), _ptr(n_new), T,
+                                                _ptr(self.kv_scale), int(self.use_scalesearch),
+                                                _ptr(self.buf), self.buf.numel(), _stream(k_new)),
+                   "thrift_kv_cache_append")
         if cache_len is None:
             self.lengths.add_(n_new)
             self.lengths.clamp_(max=self.capacity)
@@ -466,13 +498,14 @@ def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, re
     if need == 0:
         raise ThriftError("thrift_attn_decode: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
-    _check(lib().thrift_attn_decode(_ptr(q), _dt(q), B, H, cache.Hkv, d, cache.blk,
-                                    cache.capacity, _ptr(cache.buf), cache.buf.numel(),
-                                    _ptr(cache.lengths if seq_len is None else seq_len),
-                                    _ptr(cache.kv_scale), float(topk_frac),
-                                    int(sink_blocks), int(recent_blocks), int(use_scalesearch),
-                                    _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
-           "thrift_attn_decode")
+    with _on(q):
+        _check(lib().thrift_attn_decode(_ptr(q), _dt(q), B, H, cache.Hkv, d, cache.blk,
+                                        cache.capacity, _ptr(cache.buf), cache.buf.numel(),
+                                        _ptr(cache.lengths if seq_len is None else seq_len),
+                                        _ptr(cache.kv_scale), float(topk_frac),
+                                        int(sink_blocks), int(recent_blocks), int(use_scalesearch),
+                                        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)),
+               "thrift_attn_decode")
     return out, lse
 
 
@@ -519,11 +552,12 @@ def thrift_qat_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, blk=128, causal=Tr
     if need == 0:
         raise ThriftError("thrift_qat_fwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
-    _check(lib().thrift_qat_fwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _dt(q), _ptr(cu),
-                                       cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
-                                       int(use_scalesearch), _ptr(out), _ptr(out_hp), _ptr(lse),
-                                       _ptr(ws), ws.numel(), _stream(q)),
-           "thrift_qat_fwd_varlen")
+    with _on(q):
+        _check(lib().thrift_qat_fwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _dt(q), _ptr(cu),
+                                           cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
+                                           int(use_scalesearch), _ptr(out), _ptr(out_hp), _ptr(lse),
+                                           _ptr(ws), ws.numel(), _stream(q)),
+               "thrift_qat_fwd_varlen")
     return out.reshape(shape), out_hp.reshape(shape), lse
 
 
@@ -559,10 +593,11 @@ def thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu_seqlens=None, max_seqlen=None,
     if need == 0:
         raise ThriftError("thrift_qat_bwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
-    _check(lib().thrift_qat_bwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(dop), _dt(q), _ptr(cu),
-                                       cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
-                                       int(use_scalesearch), int(reuse_images), _ptr(ohp),
-                                       _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
-                                       ws.numel(), _stream(q)),
-           "thrift_qat_bwd_varlen")
+    with _on(q):
+        _check(lib().thrift_qat_bwd_varlen(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(dop), _dt(q), _ptr(cu),
+                                           cu.numel() - 1, total, maxlen, H, Hkv, d, blk, int(causal),
+                                           int(use_scalesearch), int(reuse_images), _ptr(ohp),
+                                           _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                           ws.numel(), _stream(q)),
+               "thrift_qat_bwd_varlen")
     return dq.reshape(qshape), dk.reshape(kshape), dv.reshape(kshape)

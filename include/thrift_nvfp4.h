@@ -68,6 +68,17 @@ const char* thrift_status_string(int status);
  */
 thrift_status thrift_device_status(int reset);
 
+/*
+ * Per-stream form of thrift_device_status: waits only for the work already
+ * queued on `stream` (cudaStreamSynchronize), then reads the device status
+ * word through that stream, and with reset != 0 clears it (also on that
+ * stream, before returning).  Other streams keep running.  The word itself
+ * is shared by every stream of the current device: a timeout raised by a
+ * kernel on another stream shows here too once it has happened.  Returns
+ * THRIFT_ERR_CUDA if a CUDA call fails.
+ */
+thrift_status thrift_stream_status(void* stream, int reset);
+
 /* ------------------------------------------------------------ quantiser --
  * [SS] ScaleSearch; [AQ] E2M1.  Quantises x [rows, cols] (row-major, 16-bit)
  * to NVFP4 with 16-element blocks along cols.
@@ -81,13 +92,12 @@ thrift_status thrift_device_status(int reset);
  *   use_hadamard: rotate every row by the unnormalised Sylvester-Hadamard
  *     transform first (cols must be 64 or 128).
  * Requirements: rows >= 0, cols % 16 == 0, cols <= 4096.
- * Workspace: nvfp4_quantize_workspace_size() bytes, 16-byte aligned, zero-
- *   filled before its first use; every call that completes without a device
- *   timeout leaves it zero-filled again (the one-pass kernel keeps two
- *   counters there), so one buffer serves any number of calls issued in
- *   stream order.  After THRIFT_ERR_TIMEOUT from thrift_device_status, zero
- *   it again before reuse.  nvfp4_quantize_colblocks takes the same
- *   workspace.
+ * Workspace: nvfp4_quantize_workspace_size() bytes, 16-byte aligned, no
+ *   initial contents required: the one-pass kernel's arrival counter is
+ *   cleared on the stream before each of its launches, so one buffer serves
+ *   any number of calls issued in stream order, after a device timeout too.
+ *   Calls that overlap on the GPU must not share a workspace.
+ *   nvfp4_quantize_colblocks takes the same workspace.
  * Execution: when the tensor scale is computed and the tensor fits in the
  *   SMs' shared memory (about 200 KB per SM), one cooperative launch stages
  *   it once, exchanges the per-CTA maxima with a bounded grid-wide wait and

@@ -54,3 +54,23 @@ def test_attention_after_a_timeout():
     torch.cuda.synchronize()
     assert ops.device_status() == ops.OK
     assert torch.isfinite(out.float()).all()
+
+
+def test_stream_status_waits_for_its_own_stream_only():
+    """thrift_stream_status synchronises one stream: while a bounded wait of
+    300 ms runs on stream A, a status read through stream B returns at once
+    (OK: the wait has not given up yet); the read through A waits for it and
+    reports the timeout, and its reset clears the word."""
+    assert ops.device_status(reset=True) == ops.OK
+    a, b = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(a):
+        ops.test_wait_timeout(0, 300000)
+    t0 = time.perf_counter()
+    got_b = ops.stream_status(b)
+    t_b = time.perf_counter() - t0
+    got_a = ops.stream_status(a, reset=True)
+    t_a = time.perf_counter() - t0
+    assert got_b == ops.OK and t_b < 0.2, (got_b, t_b)
+    assert got_a == ops.ERR_TIMEOUT and t_a >= 0.25, (got_a, t_a)
+    assert ops.stream_status(b) == ops.OK
+    assert ops.device_status() == ops.OK

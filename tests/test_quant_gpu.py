@@ -112,18 +112,22 @@ def test_two_pass_path_large_tensor(orc):
 
 
 @pytest.mark.parametrize("had", [False, True])
-def test_one_pass_leaves_workspace_zeroed(orc, had):
+@pytest.mark.parametrize("fill", [0x00, 0x5A, 0xFF])
+def test_one_pass_any_workspace_contents(orc, had, fill):
     # The one-pass kernel (tensor staged in shared memory, one grid-wide max
-    # exchange) keeps its counters in the caller's workspace and must leave
-    # them at zero; repeated calls on one workspace stay bit-exact.
-    ws = torch.zeros(ops.lib().nvfp4_quantize_workspace_size(), dtype=torch.uint8, device="cuda")
+    # exchange) counts arrivals in the caller's workspace.  The counter is
+    # cleared on the stream before each launch, so a workspace full of
+    # leftovers (non-zero counters, stale per-CTA maxima) still gives
+    # bit-exact codes, call after call on the same buffer.
+    ws = torch.full((ops.lib().nvfp4_quantize_workspace_size(),), fill, dtype=torch.uint8,
+                    device="cuda")
     for seed in (11, 12, 13):
         x = synth.randn16((4096, 128), torch.bfloat16, seed=seed, scale=2.0)
         codes, scales, ts = ops.nvfp4_quantize(x.cuda(), use_hadamard=had, workspace=ws)
         torch.cuda.synchronize()
-        assert ops.device_status() == ops.OK
-        assert not ws[:8].any().item()
+        assert ops.stream_status() == ops.OK
         c0, s0, g0, _ = orc.nvfp4_quantize(synth.as_u16(x), _dt(x.dtype), use_had=had)
         assert ts.item() == np.float32(g0)
         assert np.array_equal(scales.cpu().numpy(), s0)
         assert np.array_equal(codes.cpu().numpy(), c0)
+        ws[:8].fill_(fill)  # leftovers again before the next call
