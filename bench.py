@@ -1,17 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 / selective-FP16 attention forward on B200.
 
-One step = one thrift_attn_fwd call over one batch of the workload: tensor
-absmax, Q/K/V NVFP4 quantisation, block-mean top-k selection and the mixed
-NVFP4/FP16 attention kernel.  Prints one JSON line (rank 0).
+One step = one attention call over one batch of the workload: tensor absmax,
+Q/K/V NVFP4 quantisation (Hadamard and ScaleSearch when the workload asks),
+block-mean top-k selection and the mixed NVFP4/FP16 attention kernel.
+Prints one JSON line (rank 0).
 
-Default workload: B=2, H=32, N=8192, d=128, bf16, non-causal, 128x128 blocks,
-10% FP16 pairs, K with per-channel offsets N(0, 3).  Its inputs (3 x 134 MB)
-exceed L2, so no flush is needed between steps.
+Headline workload (default): the largest single-GPU configuration, causal
+GQA B=1, H=32, Hkv=8, N=32768, d=128, bf16, 128x128 blocks, 128-point
+Hadamard on Q/K, ScaleSearch, 5% FP16 pairs, K with per-channel offsets
+N(0, 3).  Its inputs (268 + 2 x 67 MB) exceed L2, so no flush is needed
+between steps.
 
-The line also carries "decode": one decode step of the double-cache decode
-path (Llama-3.1-8B attention shape, B=4, 131072 cached tokens, 10% FP16
-tiles): append the step's token, then attend; its kernel against HBM.
+The line also carries one object per other attention configuration ("configs":
+B2 H32 N8192 non-causal top 10%, and the varlen batch of 16 sequences at top
+0/5/25%), each with its own kernel roofline, oracle time and error against
+unquantised fp64 attention; the quantiser workload ("quantizer"); one decode
+step over the double cache ("decode"); and one Attn-QAT training step ("qat").
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference   # the CPU oracle on a bounded sample
@@ -37,14 +42,29 @@ if ROOT not in sys.path:
 from bit_quantization_b200 import dist, synth  # noqa: E402
 
 WORKLOADS = {
-    "b2h32n8192": synth.C_B2H32N8K,
     "gqa32k": synth.C_GQA32K,
+    "b2h32n8192": synth.C_B2H32N8K,
+    "varlen": synth.C_VARLEN,
     "tiny": synth.TINY,
 }
+# The other attention configurations reported beside the headline, each as
+# its own object: (key, workload).
+SECONDARY = [
+    ("b2h32n8192_top10", synth.C_B2H32N8K),
+    ("varlen_top0", dataclasses.replace(synth.C_VARLEN, topk_frac=0.0)),
+    ("varlen_top5", dataclasses.replace(synth.C_VARLEN, topk_frac=0.05)),
+    ("varlen_top25", dataclasses.replace(synth.C_VARLEN, topk_frac=0.25)),
+]
 
 METRIC = "NVFP4 attention fwd TFLOPS (whole step: quantise + select + attention)"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 9  # 3 absmax, 2 Q/K images (with the block means), 1 V image, 1 scores, 1 top-k, 1 attention
+# 3 absmax, 2 Q/K images (with the block means), 1 V image, 1 scores, 1 top-k,
+# 1 attention
+KERNELS_PER_STEP = 9
+# Nominal dense peaks of one B200 (context beside the measured ones)
+NOMINAL_FP4_TFLOPS = 9000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
 
 
 def load_peaks():
@@ -56,6 +76,12 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def _src_sha(name):
+    import hashlib
+    with open(os.path.join(ROOT, "bit_quantization_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
 # DRAM traffic of one attention launch measured by ncu (read + write bytes)
 # for the attention source with this hash; reported only while the source is
 # unchanged since the capture.
@@ -64,10 +90,7 @@ ATTN_TRAFFIC = {"src_sha16": "aed717716c579cc9", "workload": "b2h32n8192d128_bf1
 
 
 def attn_traffic(w):
-    import hashlib
-    path = os.path.join(ROOT, "bit_quantization_b200", "csrc", "attn.cuh")
-    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
-    if sha == ATTN_TRAFFIC["src_sha16"] and w.name == ATTN_TRAFFIC["workload"]:
+    if _src_sha("attn.cuh") == ATTN_TRAFFIC["src_sha16"] and w.name == ATTN_TRAFFIC["workload"]:
         return ATTN_TRAFFIC["bytes"]
     return None
 
@@ -80,10 +103,7 @@ QAT_TRAFFIC = {"src_sha16": "932e539dcdf5cdaa", "workload": "qat_b1h32hkv8n4096d
 
 
 def qat_traffic(w):
-    import hashlib
-    path = os.path.join(ROOT, "bit_quantization_b200", "csrc", "qat.cuh")
-    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
-    if sha == QAT_TRAFFIC["src_sha16"] and w.name == QAT_TRAFFIC["workload"]:
+    if _src_sha("qat.cuh") == QAT_TRAFFIC["src_sha16"] and w.name == QAT_TRAFFIC["workload"]:
         return QAT_TRAFFIC["bytes"]
     return None
 
@@ -93,10 +113,14 @@ XU_OPS_PER_CLK_PER_SM = 16   # MUFU lanes per SM (4 per sub-partition)
 # 16-key block for the block scale (the E2M1 / 16-bit converts do not use
 # this pipe: an instruction-class count of each convert shows none there)
 XU_OPS_PER_ELEMENT = 1.125
+# Warp instructions one sub-partition issues per clock (4 per SM)
+ISSUE_PER_CLK_PER_SM = 4
 
 
 def pair_flops(mask, w, lengths):
-    """Algorithmic FLOPs (4*d per unmasked score element) split by path."""
+    """Algorithmic FLOPs (4*d per unmasked score element) split by path.
+    mask [nseq, H, nB, nB] (1 = FP16 pair); sequence b uses its first
+    ceil(L_b / blk) block rows and columns."""
     blk, d = w.blk, w.d
     f4 = f16 = 0.0
     for b, L in enumerate(lengths):
@@ -115,6 +139,42 @@ def pair_flops(mask, w, lengths):
                 f16 += 4 * d * cnt * n16
                 f4 += 4 * d * cnt * (w.H - n16)
     return f4, f16
+
+
+def tensor_roofline(f4, f16, k_ms, peaks, peak_src):
+    """Roofline of the attention kernel: a tensor-bound contraction with
+    t_ideal = F4 / P4 + F16 / P16.  P16 is the measured bf16 GEMM burst rate
+    (the kernel is timed over tens of milliseconds, not a seconds-long
+    power-capped loop) and P4 = 4 x P16 (the nominal dense FP4 : BF16 ratio).
+    The same fraction against the nominal dense peaks is given beside it."""
+    p16 = peaks["bf16_tflops"]
+    p4 = 4.0 * p16
+    flops = f4 + f16
+    t_ideal = f4 / (p4 * 1e12) + f16 / (p16 * 1e12)
+    t_nom = f4 / (NOMINAL_FP4_TFLOPS * 1e12) + f16 / (NOMINAL_BF16_TFLOPS * 1e12)
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    peak_eff = flops / t_ideal / 1e12
+    return {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
+            "peak": peak_eff, "unit": "TFLOP/s", "frac": achieved / peak_eff,
+            "peak_note": (f"{peak_src} bf16 burst {p16} TF/s x4 for the FP4 share, x1 for the "
+                          f"FP16 share ({100 * f16 / max(flops, 1):.1f}% of flops)"),
+            "frac_of_nominal": t_nom / (k_ms * 1e-3),
+            "nominal_note": f"against nominal dense {NOMINAL_FP4_TFLOPS:.0f} TF/s FP4 and "
+                            f"{NOMINAL_BF16_TFLOPS:.0f} TF/s BF16",
+            "kernel_ms": k_ms, "fp4_flops": f4, "fp16_flops": f16}
+
+
+def alu_roofline(flops, d, k_ms, sm_mhz, n_sm):
+    """ALU roofline of the attention kernel: the MUFU operations per score
+    element (XU_OPS_PER_ELEMENT) against the MUFU lanes of the SMs."""
+    elems = flops / (4.0 * d)
+    peak = XU_OPS_PER_CLK_PER_SM * n_sm * sm_mhz * 1e6 / XU_OPS_PER_ELEMENT / 1e9
+    achieved = elems / (k_ms * 1e-3) / 1e9
+    return {"bound": "alu", "kernel": "attn_fwd_kernel", "achieved": achieved, "peak": peak,
+            "unit": "Gelem/s", "frac": achieved / peak,
+            "peak_note": (f"{XU_OPS_PER_CLK_PER_SM} MUFU lanes per SM x {n_sm} SMs x "
+                          f"{sm_mhz:.0f} MHz / {XU_OPS_PER_ELEMENT} ops per score element"),
+            "tflops_equivalent_peak": peak * 1e9 * 4 * d / 1e12}
 
 
 class ClockSampler:
@@ -168,16 +228,18 @@ class ClockSampler:
 
 
 def oracle_sample(w, nunits, nthreads, inp=None):
-    """The CPU oracle on a bounded sample of the workload: one head of batch
-    entry 0 (full sequence length), `nunits` evenly spread query blocks.
+    """The CPU oracle on a bounded sample of the workload: one head of the
+    first sequence (full length), `nunits` evenly spread query blocks.
     Returns (seconds, algorithmic flops of the sampled rows, description)."""
     import oracle
     if inp is None:
         inp = synth.make_attn_inputs(w)
-    N, d, blk = w.N, w.d, w.blk
-    q = inp["q"][0, :, 0:1].contiguous()
-    k = inp["k"][0, :, 0:1].contiguous()
-    v = inp["v"][0, :, 0:1].contiguous()
+    d, blk = w.d, w.blk
+    N = inp["lengths"][0]
+    if w.varlen is None:
+        q, k, v = (inp[n][0, :, 0:1].contiguous() for n in ("q", "k", "v"))
+    else:
+        q, k, v = (inp[n][:N, 0:1].contiguous() for n in ("q", "k", "v"))
     cu = np.array([0, N], np.int32)
     nb = (N + blk - 1) // blk
     blocks = np.unique(np.linspace(0, nb - 1, nunits).round().astype(int))
@@ -191,10 +253,23 @@ def oracle_sample(w, nunits, nthreads, inp=None):
     for i in blocks:
         rows = np.arange(i * blk, min(N, (i + 1) * blk))
         cnt = (rows + 1).sum() if w.causal else len(rows) * N
-        fl += 4.0 * d * cnt
-    desc = (f"1 of {w.B * w.H} heads (batch 0, head 0, full N={N}), {len(blocks)} of {nb} query "
-            f"blocks; includes that head's quantisation and selection")
+        fl += 4.0 * d * float(cnt)
+    nheads = w.B * w.H if w.varlen is None else len(inp["lengths"]) * w.H
+    desc = (f"1 of {nheads} (sequence, head) problems (sequence 0, head 0, full length {N}), "
+            f"{len(blocks)} of {nb} query blocks; includes that head's quantisation and "
+            f"selection")
     return dt, fl, desc
+
+
+def cpu_baseline(w, inp, budget_s=10.0, max_units=64):
+    """The oracle timed on the host cores on a sample sized to about
+    `budget_s` seconds, its rate in the line's unit."""
+    cores = os.cpu_count() or 1
+    dt0, fl0, _ = oracle_sample(w, 2, cores, inp)
+    units = int(max(2, min(max_units, 2 * budget_s / max(dt0, 1e-3))))
+    dt, fl, desc = oracle_sample(w, units, cores, inp)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": desc, "seconds": dt}
 
 
 def run_reference(args, w):
@@ -218,7 +293,7 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(w),
+            "data": "synthetic", "config": config_of(w, inp["lengths"]),
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -226,28 +301,46 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w):
-    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-            "dtype": str(w.dtype).replace("torch.", ""), "causal": w.causal, "blk": w.blk,
-            "topk_frac": w.topk_frac, "scalesearch": w.use_scalesearch,
-            "hadamard": w.use_hadamard, "k_offset_std": w.k_offset_std,
-            "l2": "inputs larger than L2 (no flush)", "parallelism": "independent problems per GPU"}
+def config_of(w, lengths=None):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+         "dtype": str(w.dtype).replace("torch.", ""), "causal": w.causal, "blk": w.blk,
+         "topk_frac": w.topk_frac, "scalesearch": w.use_scalesearch,
+         "hadamard": w.use_hadamard, "k_offset_std": w.k_offset_std,
+         "l2": "inputs larger than L2 (no flush)", "parallelism": "independent problems per GPU"}
+    if w.varlen is not None:
+        c.update({"nseq": len(lengths), "lengths": list(lengths), "total_tokens": int(sum(lengths))})
+        c["B"] = len(lengths)
+    return c
 
 
-def quantizer_line(dev, peaks):
+# Issue slots per element of the ScaleSearch-on quantiser, counted from the
+# source (quant_block16 and block_err): per candidate and 16-block about 110
+# instructions (UE4M3 decode 5, scale product 1, correctly rounded reciprocal
+# ~10, 16 products, 8 E2M1 round trips of 4 converts, 16 differences, 16
+# sequential fmaf, the fp64 error and compare ~9, loop ~5) for 9 candidates,
+# plus ~70 for max scaling and the final codes and ~16 for the loads:
+# (9 x 110 + 86) / 16 = 67 per element.
+QUANT_SS_ISSUE_PER_ELEM = 67.0
+QUANT_SS_ISSUE_NOTE = ("issue slots per element counted from the source (9 candidates x ~110 "
+                       "instructions per 16-block + ~86 for max scaling, codes and loads)")
+
+
+def quantizer_line(dev, peaks, with_oracle=True):
     """Quantiser-only workload (65536 x 128 fp16 with 4 outlier channels):
     GB/s of algorithmic bytes (2 B read + 0.5625 B written per element).
     Twelve rotating input copies (> L2); the calls are captured in one CUDA
-    graph so host-side launch gaps do not enter the timing."""
+    graph so host-side launch gaps do not enter the timing.  The oracle
+    quantises the whole tensor on the host cores beside it."""
     from bit_quantization_b200 import ops
     x0 = synth.make_quant_input(synth.QUANT).to(dev)
     xs = [x0.clone() for _ in range(12)]
     rows, cols = x0.shape
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
-    ws = torch.zeros(ops.lib().nvfp4_quantize_workspace_size(), dtype=torch.uint8, device=dev)
+    ws = torch.empty(ops.lib().nvfp4_quantize_workspace_size(), dtype=torch.uint8, device=dev)
     res = {}
-    algo = rows * cols * (2 + 0.5 + 0.0625)
+    elems = rows * cols
+    algo = elems * (2 + 0.5 + 0.0625)
     n = 120
     gts = ops.nvfp4_quantize(x0, False, False, None, codes, scales, ws)[2].clone()  # g of x0
     for ss, given in ((False, False), (True, False), (False, True)):
@@ -272,11 +365,39 @@ def quantizer_line(dev, peaks):
         gbs = algo / (ms * 1e-3) / 1e9
         key = ("scalesearch_on" if ss else "scalesearch_off") + ("_scale_given" if given else "")
         res[key] = {"us_per_call": 1e3 * ms, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
-                    "kernels_per_call": 1}
+                    "frac_of_nominal_hbm": gbs / NOMINAL_HBM_GBS}
+        if ss:
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            clk = peaks.get("sm_max_mhz", 1965.0)
+            peak_elem = ISSUE_PER_CLK_PER_SM * 32 * n_sm * clk * 1e6 / QUANT_SS_ISSUE_PER_ELEM
+            ach_elem = elems / (ms * 1e-3)
+            res[key]["alu_roofline"] = {
+                "bound": "alu", "achieved": ach_elem / 1e9, "peak": peak_elem / 1e9,
+                "unit": "Gelem/s", "frac": ach_elem / peak_elem,
+                "peak_note": f"{ISSUE_PER_CLK_PER_SM} warp instructions per clock per SM x 32 "
+                             f"lanes x {n_sm} SMs x {clk:.0f} MHz / {QUANT_SS_ISSUE_PER_ELEM} "
+                             f"({QUANT_SS_ISSUE_NOTE})",
+                "gbs_equivalent_peak": peak_elem * 2.5625 / 1e9}
         del g
     res["workload"] = synth.QUANT.name
     res["algorithmic_bytes"] = algo
+    res["kernels_per_call"] = 1
     res["timing"] = "CUDA graph of 120 calls, 12 rotating inputs (201 MB > L2)"
+    if with_oracle:
+        import oracle
+        cores = os.cpu_count() or 1
+        xh = synth.as_u16(synth.make_quant_input(synth.QUANT))
+        ob = {}
+        for ss in (False, True):
+            t0 = time.perf_counter()
+            oracle.nvfp4_quantize(xh, synth.dtype_code(synth.QUANT.dtype), use_ss=ss)
+            dt = time.perf_counter() - t0
+            ob["scalesearch_on" if ss else "scalesearch_off"] = {
+                "seconds": dt, "gbs": algo / dt / 1e9, "unit": "GB/s"}
+        res["cpu_baseline"] = {"kind": "oracle", "cores": 1, "host_cores": cores,
+                               "sample": "the whole 65536 x 128 tensor (tensor absmax, block "
+                                         "scales, codes), one thread",
+                               "value": ob["scalesearch_off"]["gbs"], "unit": "GB/s", **ob}
     return res
 
 
@@ -532,7 +653,7 @@ def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
     flops, pairs = qat_flops(w, inp["lengths"])
     step_ms = fwd_ms + bwd_ms
     attn_ms = kms / steps
-    p16, src = peaks["bf16_tflops_sustained"], peak_src
+    p16, src = peaks["bf16_tflops"], peak_src
     achieved = flops / (attn_ms * 1e-3) / 1e12
     line = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
             "causal": w.causal, "blk": w.blk, "dtype": "bf16",
@@ -544,7 +665,9 @@ def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
             "roofline": {"bound": "tensor", "kernel": "qat_fwd + qat_bwd_kv + qat_bwd_q",
                          "achieved": achieved, "peak": p16, "unit": "TFLOP/s",
                          "frac": achieved / p16, "traffic": qat_traffic(w),
-                         "peak_note": f"{src} bf16 sustained (the kernels run 16-bit MMAs)",
+                         "peak_note": f"{src} bf16 burst (the kernels run 16-bit MMAs; the "
+                                      f"timed region is tens of milliseconds)",
+                         "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                          "executed_mma_flops": 14 * 2 * pairs * w.d,
                          "note": "7 algorithmic products; the kernels execute 14 (S recomputed "
                                  "in each pass, dS and the P of O' as two 16-bit parts)"},
@@ -599,128 +722,229 @@ def qat_only(args):
     return 0
 
 
-def variant_kernel_ms(ops, q, k, v, w, out, lse, ws, frac, sink=0, recent=0, steps=20,
-                      smooth=False):
-    """Average attention-kernel time of the bench workload run with another
-    selection or option (CUDA events around each attention launch)."""
-    def step():
-        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=frac,
-                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
-                            out=out, lse=lse, workspace=ws, sink_blocks=sink, recent_blocks=recent,
-                            smooth_k=smooth)
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    ops.kernel_timer_enable(True)
-    for _ in range(steps):
-        step()
-    torch.cuda.synchronize()
-    ops.kernel_timer_enable(False)
-    kms, n = ops.kernel_timer_read()
-    if ops.device_status(reset=True) != ops.OK:
-        raise RuntimeError("device wait timed out (selection variant)")
-    return kms / max(n, 1)
+class AttnCase:
+    """One attention workload resident on the device: inputs, outputs,
+    workspace and the call one step makes (the packed entry point for a
+    varlen batch)."""
+
+    def __init__(self, ops, dev, w, seed=None):
+        self.ops, self.dev, self.w = ops, dev, w
+        self.inp = synth.make_attn_inputs(w, seed=seed)
+        self.lengths = self.inp["lengths"]
+        self.q, self.k, self.v = (self.inp[n].to(dev) for n in ("q", "k", "v"))
+        self.varlen = w.varlen is not None
+        self.out = torch.empty_like(self.q)
+        if self.varlen:
+            self.nseq, self.maxlen = len(self.lengths), max(self.lengths)
+            total = self.q.shape[0]
+            self.cu = self.inp["cu_seqlens"].to(dev)
+            self.lse = torch.empty((w.H, total), dtype=torch.float32, device=dev)
+            need = ops.thrift_attn_varlen_workspace_size(self.nseq, total, self.maxlen, w.H, w.Hkv,
+                                                         w.d, w.blk)
+        else:
+            self.nseq, self.maxlen = w.B, w.N
+            self.cu = None
+            self.lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+            need = ops.thrift_attn_workspace_size(w.B, w.H, w.Hkv, w.N, w.d, w.blk)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def run(self, q=None, k=None, v=None, out=None, lse=None, frac=None, sink=0, recent=0,
+            smooth=False):
+        w, ops = self.w, self.ops
+        q = self.q if q is None else q
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
+        frac = w.topk_frac if frac is None else frac
+        if self.varlen:
+            ops.thrift_attn_fwd_varlen(q, k, v, self.cu, self.maxlen, blk=w.blk, causal=w.causal,
+                                       topk_frac=frac, use_scalesearch=w.use_scalesearch,
+                                       use_hadamard=w.use_hadamard, out=out, lse=lse,
+                                       workspace=self.ws, sink_blocks=sink, recent_blocks=recent,
+                                       smooth_k=smooth)
+        else:
+            ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=frac,
+                                use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
+                                out=out, lse=lse, workspace=self.ws, sink_blocks=sink,
+                                recent_blocks=recent, smooth_k=smooth)
+
+    def mask(self):
+        """The selection [nseq, H, nB, nB] the last call left in the workspace."""
+        w = self.w
+        nB = (self.maxlen + w.blk - 1) // w.blk
+        off = self.ops.thrift_attn_workspace_mask_offset(self.nseq, self.maxlen, w.H, w.Hkv,
+                                                         w.d, w.blk)
+        n = self.nseq * w.H * nB * nB
+        return self.ws[off:off + n].view(self.nseq, w.H, nB, nB).cpu().numpy()
+
+    def flops(self, **kw):
+        """(F4, F16) of the selection one call with these options makes."""
+        self.run(**kw)
+        torch.cuda.synchronize(self.dev)
+        return pair_flops(self.mask(), self.w, self.lengths)
+
+    def kernel_ms(self, steps=20, **kw):
+        """Average attention-kernel time (CUDA events around each launch on
+        its stream) over `steps` calls with these options."""
+        ops = self.ops
+        for _ in range(3):
+            self.run(**kw)
+        torch.cuda.synchronize(self.dev)
+        ops.kernel_timer_enable(True)
+        for _ in range(steps):
+            self.run(**kw)
+        torch.cuda.synchronize(self.dev)
+        ops.kernel_timer_enable(False)
+        kms, n = ops.kernel_timer_read()
+        if ops.device_status(reset=True) != ops.OK:
+            raise RuntimeError("device wait timed out")
+        return kms / max(n, 1)
+
+    def err_vs_fp64(self, nrows=128, seed=11):
+        """Error of the last call's output against unquantised fp64 attention
+        (torch, on the device) of the same 16-bit inputs, on `nrows` seeded
+        (sequence, token, head) rows; a report, not a bound."""
+        w = self.w
+        g = w.H // w.Hkv
+        gen = torch.Generator().manual_seed(seed)
+        seqs = torch.randint(0, self.nseq, (nrows,), generator=gen).tolist()
+        fr = torch.rand((nrows,), generator=gen).tolist()
+        heads = torch.randint(0, w.H, (nrows,), generator=gen).tolist()
+        se = ref2 = 0.0
+        mx = 0.0
+        for s, f, h in zip(seqs, fr, heads):
+            L = self.lengths[s]
+            t = min(L - 1, int(f * L))
+            n_keys = t + 1 if w.causal else L
+            if self.varlen:
+                a = int(self.inp["cu_seqlens"][s])
+                qr, o = self.q[a + t, h], self.out[a + t, h]
+                kk, vv = self.k[a:a + n_keys, h // g], self.v[a:a + n_keys, h // g]
+            else:
+                qr, o = self.q[s, t, h], self.out[s, t, h]
+                kk, vv = self.k[s, :n_keys, h // g], self.v[s, :n_keys, h // g]
+            p = torch.softmax(kk.double() @ qr.double() / (w.d ** 0.5), dim=0)
+            ref = p @ vv.double()
+            dlt = o.double() - ref
+            se += float((dlt ** 2).sum())
+            ref2 += float((ref ** 2).sum())
+            mx = max(mx, float(dlt.abs().max()))
+        n = nrows * w.d
+        return {"max_abs": mx, "rms": (se / n) ** 0.5, "rms_of_reference": (ref2 / n) ** 0.5,
+                "rows": nrows, "sample": "seeded uniform (sequence, token, head) rows",
+                "reference": "torch fp64 softmax(q K^T / sqrt(d)) V of the 16-bit inputs"}
 
 
-def sink_line(ops, q, k, v, w, inp, out, lse, ws, p16, sink=1, recent=1):
-    """ScaleSearchAttention's sink-aware variant of the bench workload: the
-    first and the newest key block of every query block on the FP16 path on
-    top of the top-k pairs; the attention kernel's rate against the FP4 /
-    FP16 roofline of its own pair split."""
-    mask = ops.block_mean_topk(q, k, w.blk, w.causal, w.topk_frac, sink_blocks=sink,
-                               recent_blocks=recent).cpu().numpy()
-    f4, f16 = pair_flops(mask, w, inp["lengths"])
-    k_ms = variant_kernel_ms(ops, q, k, v, w, out, lse, ws, w.topk_frac, sink, recent)
-    t_ideal = f4 / (4.0 * p16 * 1e12) + f16 / (p16 * 1e12)
+def nvfp4_only_object(case, peaks, peak_src, steps=20):
+    """The attention kernel with no FP16 pairs (topk_frac = 0): every score
+    on the NVFP4 path, against the FP4 tensor peak alone."""
+    f4, f16 = case.flops(frac=0.0)
+    k_ms = case.kernel_ms(steps, frac=0.0)
+    p4 = 4.0 * peaks["bf16_tflops"]
     achieved = (f4 + f16) / (k_ms * 1e-3) / 1e12
-    return {"sink_blocks": sink, "recent_blocks": recent, "topk_frac": w.topk_frac,
-            "kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "achieved": achieved,
-            "unit": "TFLOP/s", "fp16_share": f16 / (f4 + f16),
-            "frac": (t_ideal / (k_ms * 1e-3))}
+    return {"topk_frac": 0.0, "kernel": "attn_fwd_kernel", "kernel_ms": k_ms,
+            "achieved": achieved, "peak": p4, "unit": "TFLOP/s", "frac": achieved / p4,
+            "peak_note": f"{peak_src} bf16 burst x4",
+            "frac_of_nominal": achieved / NOMINAL_FP4_TFLOPS}
 
 
-def smoothing_line(ops, q, k, v, w, out, lse, ws, steps=20, nrows=64):
-    """K smoothing on the bench workload: the attention kernel's and the whole
-    step's time with it, and the error of both variants against fp64
-    attention (torch, on the GPU) on a sample of output rows."""
-    dev = q.device
-    k_ms = variant_kernel_ms(ops, q, k, v, w, out, lse, ws, w.topk_frac, smooth=True)
+def sink_object(case, peaks, peak_src, sink=1, recent=1):
+    """ScaleSearchAttention's sink-aware variant: the first and the newest key
+    block of every query block on the FP16 path on top of the top-k pairs;
+    the attention kernel's rate against the FP4 / FP16 roofline of its own
+    pair split."""
+    f4, f16 = case.flops(sink=sink, recent=recent)
+    k_ms = case.kernel_ms(sink=sink, recent=recent)
+    r = tensor_roofline(f4, f16, k_ms, peaks, peak_src)
+    return {"sink_blocks": sink, "recent_blocks": recent, "topk_frac": case.w.topk_frac,
+            "kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "achieved": r["achieved"],
+            "unit": "TFLOP/s", "fp16_share": f16 / (f4 + f16), "frac": r["frac"]}
+
+
+def smoothing_object(case, steps=20):
+    """K smoothing: the attention kernel's and the whole step's time with it,
+    and the error of both variants against fp64 attention."""
+    dev = case.dev
+    k_ms = case.kernel_ms(smooth=True)
 
     def step_ms(smooth):
         for _ in range(3):
-            ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
-                                out=out, lse=lse, workspace=ws, smooth_k=smooth)
+            case.run(smooth=smooth)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(steps):
-            ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
-                                out=out, lse=lse, workspace=ws, smooth_k=smooth)
+            case.run(smooth=smooth)
         e1.record()
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / steps
 
-    gen = torch.Generator().manual_seed(11)
-    rows = torch.randint(0, w.N, (nrows,), generator=gen).tolist()
-    heads = torch.randint(0, w.H, (nrows,), generator=gen).tolist()
-    g = w.H // w.Hkv
     err = {}
     for smooth in (False, True):
-        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac, out=out,
-                            lse=lse, workspace=ws, smooth_k=smooth)
+        case.run(smooth=smooth)
         torch.cuda.synchronize(dev)
-        se = 0.0
-        for t, h in zip(rows, heads):
-            qr = q[0, t, h].double()
-            kk = k[0, : (t + 1 if w.causal else w.N), h // g].double()
-            vv = v[0, : kk.shape[0], h // g].double()
-            p = torch.softmax(kk @ qr / (w.d ** 0.5), dim=0)
-            se += float(((out[0, t, h].double() - p @ vv) ** 2).sum())
-        err["on" if smooth else "off"] = (se / (nrows * w.d)) ** 0.5
-    if ops.device_status(reset=True) != ops.OK:
+        err["on" if smooth else "off"] = case.err_vs_fp64(64)["rms"]
+    if case.ops.device_status(reset=True) != case.ops.OK:
         raise RuntimeError("device wait timed out (smoothing)")
     return {"kernel": "attn_fwd_kernel", "kernel_ms": k_ms, "step_ms": step_ms(True),
-            "step_ms_without": step_ms(False),
-            "rms_err_vs_fp64": err, "sample": f"{nrows} (token, head) rows of batch entry 0",
+            "step_ms_without": step_ms(False), "rms_err_vs_fp64": err,
             "reference": "torch fp64 softmax(q K^T / sqrt(d)) V of the 16-bit inputs"}
 
 
-def nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4, steps=20):
-    """The attention kernel with no FP16 pairs (topk_frac = 0): every score
-    on the NVFP4 path, against the FP4 tensor peak alone."""
-    def step():
-        ops.thrift_attn_fwd(q, k, v, blk=w.blk, causal=w.causal, topk_frac=0.0,
-                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
-                            out=out, lse=lse, workspace=ws)
+def config_object(case, peaks, peak_src, steps, sm_mhz, n_sm, with_cpu=True,
+                  with_nvfp4_only=False):
+    """One attention configuration: whole-step rate, the attention kernel's
+    tensor and ALU rooflines, error against fp64 attention and the oracle on
+    the host cores."""
+    ops, w, dev = case.ops, case.w, case.dev
+    f4, f16 = case.flops()
+    flops = f4 + f16
     for _ in range(3):
-        step()
-    torch.cuda.synchronize()
+        case.run()
+    torch.cuda.synchronize(dev)
     ops.kernel_timer_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
     for _ in range(steps):
-        step()
-    torch.cuda.synchronize()
+        case.run()
+    e1.record()
+    torch.cuda.synchronize(dev)
     ops.kernel_timer_enable(False)
     kms, n = ops.kernel_timer_read()
     if ops.device_status(reset=True) != ops.OK:
-        raise RuntimeError("device wait timed out (topk_frac = 0)")
+        raise RuntimeError(f"device wait timed out ({w.name})")
+    step_ms = e0.elapsed_time(e1) / steps
     k_ms = kms / max(n, 1)
-    achieved = flops / (k_ms * 1e-3) / 1e12
-    return {"topk_frac": 0.0, "kernel": "attn_fwd_kernel", "kernel_ms": k_ms,
-            "achieved": achieved, "peak": p4, "unit": "TFLOP/s", "frac": achieved / p4}
+    obj = {"workload": w.name, "config": config_of(w, case.lengths),
+           "value": flops / (step_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": step_ms,
+           "steps": steps, "kernel_ms": k_ms, "algorithmic_flops": flops,
+           "roofline": tensor_roofline(f4, f16, k_ms, peaks, peak_src),
+           "alu_roofline": alu_roofline(flops, w.d, k_ms, sm_mhz, n_sm),
+           "err_vs_fp64": case.err_vs_fp64(), "gpu_launches": KERNELS_PER_STEP * steps}
+    obj["roofline"]["traffic"] = attn_traffic(w)
+    if with_nvfp4_only:
+        obj["nvfp4_only"] = nvfp4_only_object(case, peaks, peak_src)
+    if with_cpu:
+        obj["cpu_baseline"] = cpu_baseline(w, case.inp)
+    return obj
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="b2h32n8192", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="gqa32k", choices=sorted(WORKLOADS))
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quantizer", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the objects of the other attention configurations")
     ap.add_argument("--mode", default="attention",
                     choices=["attention", "quantizer", "decode", "qat"],
-                    help="quantizer / decode: only a few plain calls of that path (profiling aid)")
+                    help="quantizer / decode / qat: only a few plain calls of that path "
+                         "(profiling aid)")
     ap.add_argument("--decode-context", type=int, default=None,
                     help="cached tokens per sequence in --mode decode (default: the workload's)")
     ap.add_argument("--no-decode", action="store_true")
@@ -742,26 +966,15 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
 
-    inp = synth.make_attn_inputs(w, seed=dist.rank_seed(w.seed, rank))
-    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
-    out = torch.empty_like(q)
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-    ws = torch.empty(ops.thrift_attn_workspace_size(w.B, w.H, w.Hkv, w.N, w.d, w.blk),
-                     dtype=torch.uint8, device=dev)
-
-    def step(qq, kk, vv):
-        ops.thrift_attn_fwd(qq, kk, vv, blk=w.blk, causal=w.causal, topk_frac=w.topk_frac,
-                            use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
-                            out=out, lse=lse, workspace=ws)
-
+    case = AttnCase(ops, dev, w, seed=dist.rank_seed(w.seed, rank))
     # FLOP split from the selection this input produces
-    mask = ops.block_mean_topk(q, k, w.blk, w.causal, w.topk_frac).cpu().numpy()
-    f4, f16 = pair_flops(mask, w, inp["lengths"])
+    f4, f16 = case.flops()
     flops = f4 + f16
 
     for _ in range(args.warmup):
-        step(q, k, v)
+        case.run()
     torch.cuda.synchronize(dev)
     if ops.device_status(reset=True) != ops.OK:
         raise RuntimeError("device wait timed out during warm-up")
@@ -775,7 +988,7 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        step(q, k, v)
+        case.run()
     e1.record()
     torch.cuda.synchronize(dev)
     ops.kernel_timer_enable(False)
@@ -795,14 +1008,14 @@ def main():
     # Steps are pipelined the way a serving loop streams batches: step s+1's
     # inputs go up on a copy stream and step s-1's results come down on
     # another while step s computes (two device buffer sets).
-    qh, kh, vh = (inp[n].pin_memory() for n in ("q", "k", "v"))
-    outh = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
-    lseh = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
-    qd = [torch.empty_like(q) for _ in range(2)]
-    kd = [torch.empty_like(k) for _ in range(2)]
-    vd = [torch.empty_like(v) for _ in range(2)]
-    od = [torch.empty_like(out) for _ in range(2)]
-    ld = [torch.empty_like(lse) for _ in range(2)]
+    qh, kh, vh = (case.inp[n].pin_memory() for n in ("q", "k", "v"))
+    outh = [torch.empty(case.out.shape, dtype=case.out.dtype).pin_memory() for _ in range(2)]
+    lseh = [torch.empty(case.lse.shape, dtype=case.lse.dtype).pin_memory() for _ in range(2)]
+    qd = [torch.empty_like(case.q) for _ in range(2)]
+    kd = [torch.empty_like(case.k) for _ in range(2)]
+    vd = [torch.empty_like(case.v) for _ in range(2)]
+    od = [torch.empty_like(case.out) for _ in range(2)]
+    ld = [torch.empty_like(case.lse) for _ in range(2)]
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
@@ -823,10 +1036,7 @@ def main():
                 s_comp.wait_event(ev_in[b])
                 if st >= 2:
                     s_comp.wait_event(ev_out[b])  # step st-2's results have left buffer b
-                ops.thrift_attn_fwd(qd[b], kd[b], vd[b], blk=w.blk, causal=w.causal,
-                                    topk_frac=w.topk_frac, use_scalesearch=w.use_scalesearch,
-                                    use_hadamard=w.use_hadamard, out=od[b], lse=ld[b],
-                                    workspace=ws)
+                case.run(qd[b], kd[b], vd[b], od[b], ld[b])
                 ev_comp[b].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[b])
@@ -849,63 +1059,51 @@ def main():
     e2e_ms = dist.max_over_ranks([e0.elapsed_time(e1)], world)[0] / e2e_steps
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = outh[0].numel() * outh[0].element_size() + lseh[0].numel() * lseh[0].element_size()
-
-    # roofline of the attention kernel (dominant): tensor-bound contraction;
-    # t_ideal = F4/P4 + F16/P16 with P16 the measured bf16 GEMM rate and
-    # P4 = 4 x P16 (nominal dense FP4 : BF16 ratio).
-    p16 = peaks["bf16_tflops_sustained"]
-    p4 = 4.0 * p16
-    t_ideal_ms = (f4 / (p4 * 1e12) + f16 / (p16 * 1e12)) * 1e3
-    achieved = flops / (k_ms * 1e-3) / 1e12
-    peak_eff = flops / (t_ideal_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
-                "peak": peak_eff, "unit": "TFLOP/s", "frac": achieved / peak_eff,
-                "traffic": attn_traffic(w),
-                "peak_note": (f"{peak_src} bf16 sustained {p16} TF/s x4 for the FP4 share, x1 for "
-                              f"the FP16 share ({100 * f16 / flops:.1f}% of flops)"),
-                "kernel_ms": k_ms, "fp4_flops": f4, "fp16_flops": f16}
-
-    # ALU roofline of the same kernel: the MUFU operations per score element
-    # (XU_OPS_PER_ELEMENT) against the MUFU lanes of the SMs.
+    del qd, kd, vd, od, ld, outh, lseh
     sm_mhz = clocks.get("sm_mhz") or 1965.0
-    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-    elems = flops / (4.0 * w.d)
-    alu_peak = XU_OPS_PER_CLK_PER_SM * n_sm * sm_mhz * 1e6 / XU_OPS_PER_ELEMENT / 1e9
-    alu_achieved = elems / (k_ms * 1e-3) / 1e9
-    alu_roofline = {"bound": "alu", "kernel": "attn_fwd_kernel", "achieved": alu_achieved,
-                    "peak": alu_peak, "unit": "Gelem/s", "frac": alu_achieved / alu_peak,
-                    "peak_note": (f"{XU_OPS_PER_CLK_PER_SM} MUFU lanes per SM x {n_sm} SMs x "
-                                  f"{sm_mhz:.0f} MHz / {XU_OPS_PER_ELEMENT} ops per score element"),
-                    "tflops_equivalent_peak": alu_peak * 1e9 * 4 * w.d / 1e12}
 
+    roofline = tensor_roofline(f4, f16, k_ms, peaks, peak_src)
+    roofline["traffic"] = attn_traffic(w)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
-            "data": "synthetic", "config": config_of(w), "roofline": roofline,
-            "alu_roofline": alu_roofline,
+            "data": "synthetic", "config": config_of(w, case.lengths), "roofline": roofline,
+            "alu_roofline": alu_roofline(flops, w.d, k_ms, sm_mhz, n_sm),
             "e2e": {"value": dist.whole_job_rate(job_flops, e2e_ms) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "pipelining": "inputs of step s+1 and results of step s-1 copied while "
                                   "step s computes (two buffer sets, three streams)"},
             "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks}
     if rank == 0 and world == 1:
-        line["nvfp4_only"] = nvfp4_only_line(ops, q, k, v, w, out, lse, ws, flops, p4)
-        line["sink_aware"] = sink_line(ops, q, k, v, w, inp, out, lse, ws, p16)
-        if not w.use_hadamard:
-            line["k_smoothing"] = smoothing_line(ops, q, k, v, w, out, lse, ws)
+        case.run()
+        torch.cuda.synchronize(dev)
+        line["err_vs_fp64"] = case.err_vs_fp64()
+        line["nvfp4_only"] = nvfp4_only_object(case, peaks, peak_src)
+        line["sink_aware"] = sink_object(case, peaks, peak_src)
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, case.inp)
+    del case
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_configs:
+        configs = {}
+        for key, cw in SECONDARY:
+            if cw.name == w.name and cw.topk_frac == w.topk_frac:
+                continue
+            c = AttnCase(ops, dev, cw)
+            configs[key] = config_object(c, peaks, peak_src, 20, sm_mhz, n_sm,
+                                         with_cpu=not args.no_cpu_baseline,
+                                         with_nvfp4_only=cw is synth.C_B2H32N8K)
+            if cw is synth.C_B2H32N8K:
+                configs[key]["k_smoothing"] = smoothing_object(c)
+            del c
+            torch.cuda.empty_cache()
+        line["configs"] = configs
     if rank == 0 and world == 1 and not args.no_quantizer:
-        line["quantizer"] = quantizer_line(dev, peaks)
+        line["quantizer"] = quantizer_line(dev, peaks, with_oracle=not args.no_cpu_baseline)
     if rank == 0 and world == 1 and not args.no_decode:
-        del qd, kd, vd, od, ld
-        torch.cuda.empty_cache()
         line["decode"] = decode_line(ops, dev, peaks)
     if rank == 0 and world == 1 and not args.no_qat:
         line["qat"] = qat_line(ops, dev, peaks, peak_src, args)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = os.cpu_count() or 1
-        dt, fl, desc = oracle_sample(w, args.ref_units, cores, inp)
-        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores,
-                                "kind": "oracle", "sample": desc, "seconds": dt}
     dist.teardown(world)
     if rank == 0:
         print(json.dumps(line), flush=True)
