@@ -82,6 +82,8 @@ def lib():
         L.orc_thrift_decode.restype = i32
         L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
                                         i32, i32, i32, P, i32, P, i32, P, P, P, P, P]
+        L.orc_set_test_hooks.restype = None
+        L.orc_set_test_hooks.argtypes = [C.c_double, C.c_uint64, i32, i32, i32, i32, f32, i32]
         _lib = L
     return _lib
 
@@ -409,3 +411,27 @@ def attn_qat_bwd(q, k, v, dout, dt, cu, blk, causal, use_ss=False, nthreads=None
     if rc:
         raise ValueError("oracle attn_qat_bwd: bad arguments")
     return {"o": o, "o_hp": o_hp, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+
+
+# ------------------------------------------------------------ test hooks
+
+class test_hooks:
+    """Context manager that sets the emulation's test hooks (pins of the
+    non-unique-rounding bound ``tol`` only; see oracle.cpp) and clears them
+    on exit.  pert: every rounding input of the probabilities is multiplied by
+    1 + pert * rho * u, u in [-1, 1) from a hash of (seed, position); plant:
+    (sequence, head, row, key) whose scaled NVFP4 probability becomes plant_t
+    and whose E2M1 code then moves ``force`` grid steps."""
+
+    def __init__(self, pert=0.0, seed=0, plant=None, plant_t=0.0, force=0):
+        self.args = (float(pert), int(seed)) + (tuple(plant) if plant else (-1, -1, -1, -1)) + (
+            float(plant_t), int(force))
+
+    def __enter__(self):
+        lib().orc_set_test_hooks(*self.args)
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_test_hooks(0.0, 0, -1, -1, -1, -1, 0.0, 0)
+        return False
+

@@ -586,53 +586,183 @@ static inline double deq(uint8_t code, uint8_t sc, float g) {
   return (double)orc_e2m1_decode(code) * (double)orc_ue4m3_decode(sc) * (double)g;
 }
 
-// One query block i of sequence s, head h.  Writes out rows and lse.
-// Relative distance within which a rounding decision of the oracle is treated
-// as not unique: the GPU computes the same quantities through fp32 MMA
-// accumulation and hardware exp2/log2, about 1e-6 relative from the oracle's
-// fp64 values, so a value this close to a rounding midpoint may land on
-// either side.
-static const double kAmbiguous = 2e-5;
-
-// E2M1 rounding midpoints between consecutive magnitudes and the code pair
-// on either side.
-static const double kE2M1Mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
-
-// If |t| lies within kAmbiguous of an E2M1 midpoint, returns the magnitude of
-// the other code's value minus this code's value; else 0.
-static double e2m1_ambiguity(float t) {
-  const double a = std::fabs((double)t);
-  for (int k = 0; k < 7; ++k)
-    if (std::fabs(a - kE2M1Mid[k]) <= kAmbiguous * kE2M1Mid[k])
-      return (double)kE2M1Mag[k + 1] - (double)kE2M1Mag[k];
-  return 0.0;
+// ------------------------------------------ roundings that are not unique --
+//
+// The GPU evaluates the quantities of this emulation in another order: scores
+// by fp32 accumulation in the tensor cores, the exponent argument of each
+// probability in fp32, exp2 and log2 by the hardware approximations.  A
+// probability whose E2M1 code, UE4M3 block scale or 16-bit value lies within
+// that arithmetic's error of a rounding midpoint may round to either side,
+// and both results are correct evaluations of the method.  The emulation
+// reports, per output element, a bound `tol` on how far such roundings can
+// move it.  The radius (relative) within which a rounding counts as not
+// unique is taken per row and key tile from the error bounds of that
+// arithmetic, in log2 units of the exponent argument:
+//   * each score and the maximum it is taken against come from an fp32
+//     accumulation of d exact products with at most one ulp of error per
+//     addition: 2 d 2^-23 A, A = the tile's largest sum over channels of
+//     |q_c k_c| (softmax scale included);
+//   * the fp32 roundings of the scale product, the maximum, the constant part
+//     of the argument (log2 2688 - log2 S_b, the log2 approximation adding at
+//     most 2^-22 per unit of its result) and the fused argument itself:
+//     2^-22 (|S|max + |m| + 24), 24 bounding |log2 2688| + |log2 S_b| <= 20.4;
+// plus, relative, the exp2 approximation (2 ulp, 2^-22) and this emulation's
+// own fp32 chain (P, 1/rowmax, P/rowmax, 1/S_b, t: five roundings of 2^-24):
+//   rho = ln 2 (2 d 2^-23 A + 2^-22 (|S|max + |m| + 24)) + 2^-22 + 5 2^-24.
+static double tile_radius(int d, double A, double smax_abs, double m_abs) {
+  const double u23 = std::ldexp(1.0, -23), u22 = std::ldexp(1.0, -22);
+  const double dx = 2.0 * d * u23 * A + u22 * (smax_abs + m_abs + 24.0);
+  return 0.6931471805599453 * dx + u22 + 5.0 * std::ldexp(1.0, -24);
 }
 
-// The UE4M3 byte on the other side of the nearest rounding midpoint when v
-// lies within kAmbiguous of it, else -1.
-static int ue4m3_ambiguous_neighbour(float v, uint8_t S) {
-  if (!(v > 0.0f)) return -1;
-  const double dv = (double)v, d0 = orc_ue4m3_decode(S);
-  for (int nb = (int)S - 1; nb <= (int)S + 1; nb += 2) {
-    if (nb < 0 || nb > 0x7E) continue;
-    const double mid = 0.5 * (d0 + (double)orc_ue4m3_decode((uint8_t)nb));
-    if (mid > 0.0 && std::fabs(dv - mid) <= kAmbiguous * mid) return nb;
+// Every rounding below is monotone, so the roundings a value x can take
+// when it is changed by a factor in [1 - rho, 1 + rho] lie between the
+// roundings of the two ends of that interval.  The ends carry 2^-23 of
+// margin for the fp32 rounding of a changed value.
+static double widen(double rho) { return rho + std::ldexp(1.0, -23); }
+
+// E2M1 value of t (round to nearest even, saturating).
+static double e2m1_val(double t) { return (double)orc_e2m1_decode(orc_e2m1_encode((float)t)); }
+
+// How far the E2M1 value of t can move under a change of t within rho.
+static double e2m1_reach(float t, double rho) {
+  const double r = widen(rho), q0 = e2m1_val(t);
+  return std::max(std::fabs(e2m1_val((double)t * (1.0 + r)) - q0),
+                  std::fabs(e2m1_val((double)t * (1.0 - r)) - q0));
+}
+
+// How far the 16-bit rounding of x can move under a change of x within rho.
+static double half_reach(double x, int dt, double rho) {
+  const double r = widen(rho);
+  const double q0 = orc_half_to_float(orc_double_to_half(x, dt), dt);
+  const double qh = orc_half_to_float(orc_double_to_half(x * (1.0 + r), dt), dt);
+  const double ql = orc_half_to_float(orc_double_to_half(x * (1.0 - r), dt), dt);
+  return std::max(std::fabs(qh - q0), std::fabs(ql - q0));
+}
+
+// Test hooks (pins of `tol` only; off unless set by orc_set_test_hooks).
+//   pert: every rounding input of the probabilities -- the scaled P whose
+//     E2M1 code is taken, the block-scale argument, the P rounded to 16 bits
+//     -- is multiplied by 1 + pert * rho * u, u in [-1, 1) a hash of (seed,
+//     sequence, head, row, key, kind); with |pert| <= 1 only roundings within
+//     the radius can change.
+//   plant: on the NVFP4 path of one (sequence, head, row, key) the scaled
+//     probability t takes the value plant_t, and its E2M1 code then moves
+//     `force` grid steps (+1 up, -1 down, 0 none).
+struct OrcHooks {
+  double pert = 0.0;
+  uint64_t seed = 0;
+  int s = -1, h = -1, row = -1, key = -1;
+  float plant_t = 0.0f;
+  int force = 0;
+};
+static OrcHooks g_hooks;
+
+void orc_set_test_hooks(double pert, uint64_t seed, int s, int h, int row, int key,
+                        float plant_t, int force) {
+  g_hooks.pert = pert;
+  g_hooks.seed = seed;
+  g_hooks.s = s;
+  g_hooks.h = h;
+  g_hooks.row = row;
+  g_hooks.key = key;
+  g_hooks.plant_t = plant_t;
+  g_hooks.force = force;
+}
+
+// splitmix64 finaliser of the hooks' hash.
+static uint64_t mix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// fp32 x * (1 + pert * rho * u) for the hooks' perturbation (x when off).
+static float hook_perturb(float x, double rho, int s, int h, int row, int key, int kind) {
+  if (g_hooks.pert == 0.0) return x;
+  uint64_t z = mix64(g_hooks.seed ^ ((uint64_t)(uint32_t)s << 40));
+  z = mix64(z ^ ((uint64_t)(uint32_t)h << 20) ^ (uint64_t)(uint32_t)row);
+  z = mix64(z ^ ((uint64_t)(uint32_t)key << 8) ^ (uint64_t)kind);
+  const double u = (double)(z >> 11) * std::ldexp(1.0, -52) - 1.0;
+  return (float)((double)x * (1.0 + g_hooks.pert * rho * u));
+}
+
+static bool hook_planted(int s, int h, int row, int key) {
+  return s == g_hooks.s && h == g_hooks.h && row == g_hooks.row && key == g_hooks.key;
+}
+
+// Two-level quantisation of one row's probability tile (reading R7): Pt[t],
+// t < nk, the fp32 probabilities relative to the running max; returns
+// sigma = rowmax / 2688 (0 when the row has no live key: the tile adds
+// nothing) and, for t < nk, Pq[t] = the value of P^ (E2M1 value times UE4M3
+// block scale; the tile adds sigma * sum_t Pq[t] v[t]) and dq[t] = how far a
+// rounding that is not unique within radius rho can move Pq[t].
+// (s, h, row, key0) locate the tile for the test hooks.
+static float p_tile_fp4(const float* Pt, int nk, int blk, double rho, int s, int h, int row,
+                        int key0, double* Pq, double* dq) {
+  float rowmax = 0.0f;
+  for (int t = 0; t < nk; ++t) rowmax = std::max(rowmax, Pt[t]);
+  if (rowmax == 0.0f) return 0.0f;
+  const float inv = 2688.0f / rowmax;
+  const float sigma = rowmax / 2688.0f;
+  std::vector<float> Ph(blk);
+  for (int t = 0; t < blk; ++t) Ph[t] = t < nk ? Pt[t] * inv : 0.0f;
+  for (int b0 = 0; b0 < blk && b0 < nk; b0 += 16) {
+    const int ne = std::min(16, nk - b0);
+    float amax = 0.0f;
+    for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
+    const float s_real = hook_perturb(amax / 6.0f, rho, s, h, row, key0 + b0, 1);
+    const uint8_t sp = orc_ue4m3_encode(s_real);
+    const float dec = orc_ue4m3_decode(sp);
+    const float rr = 1.0f / dec;
+    for (int e = 0; e < ne; ++e) {
+      const int key = key0 + b0 + e;
+      float tq = Ph[b0 + e] * rr;
+      const bool planted = hook_planted(s, h, row, key);
+      if (planted) tq = g_hooks.plant_t;
+      tq = hook_perturb(tq, rho, s, h, row, key, 0);
+      uint8_t code = orc_e2m1_encode(tq);
+      if (planted && g_hooks.force != 0) {
+        const int mag = std::min(7, std::max(0, (int)(code & 7) + g_hooks.force));
+        code = (uint8_t)((code & 8) | mag);
+      }
+      Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(code) * (double)dec;
+      dq[b0 + e] = sp == 0 ? 0.0 : e2m1_reach(tq, rho) * (double)dec;
+    }
+    // block-scale bytes the scale argument can round to within the radius:
+    // under each other byte, the block's codes (each within the radius too)
+    const double rw = widen(rho);
+    const int lo_b = orc_ue4m3_encode((float)((double)s_real * (1.0 - rw)));
+    const int hi_b = orc_ue4m3_encode((float)((double)s_real * (1.0 + rw)));
+    for (int alt = lo_b; alt <= hi_b; ++alt) {
+      if (alt == (int)sp) continue;
+      const float dec2 = orc_ue4m3_decode((uint8_t)alt);
+      const float rr2 = alt == 0 ? 0.0f : 1.0f / dec2;
+      for (int e = 0; e < ne; ++e) {
+        const float t2 = Ph[b0 + e] * rr2;
+        const double q2 = alt == 0 ? 0.0 : e2m1_val(t2) * (double)dec2;
+        const double r2 = alt == 0 ? 0.0 : e2m1_reach(t2, rho) * (double)dec2;
+        dq[b0 + e] = std::max(dq[b0 + e], std::fabs(q2 - Pq[b0 + e]) + r2);
+      }
+    }
   }
-  return -1;
+  return sigma;
 }
 
-// Half the 16-bit spacing at x if x lies within kAmbiguous of a 16-bit
-// rounding midpoint (the other rounding is one spacing away), else 0.
-static double half_ambiguity(double x, int dt) {
-  if (x <= 0.0) return 0.0;
-  const double lo = orc_half_to_float(orc_double_to_half(x, dt), dt);
-  int e;
-  std::frexp(x, &e);
-  const double sp = std::ldexp(1.0, e - (dt == 1 ? 8 : 11));  // spacing in [2^(e-1), 2^e)
-  const double mid = lo + (x > lo ? 0.5 : -0.5) * sp;
-  return std::fabs(x - mid) <= kAmbiguous * x ? sp : 0.0;
+// FP16 path of one row's tile (reading R9): P16[t] = Pt[t] rounded to the
+// input type, dq[t] = how far that rounding can move under a change of Pt[t]
+// within radius rho.
+static void p_tile_16(const float* Pt, int nk, int dt, double rho, int s, int h, int row,
+                      int key0, double* P16, double* dq) {
+  for (int t = 0; t < nk; ++t) {
+    const float x = hook_perturb(Pt[t], rho, s, h, row, key0 + t, 2);
+    P16[t] = (double)orc_half_to_float(orc_double_to_half((double)x, dt), dt);
+    dq[t] = half_reach((double)x, dt, rho);
+  }
 }
 
+// One query block i of sequence s, head h.  Writes out rows and lse.
 static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, float* lse,
                       double* out64, double* tol) {
   const int d = C.d, blk = C.blk, H = C.H, Hkv = C.Hkv;
@@ -665,9 +795,11 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
   std::vector<double> m(nr, -INFINITY), l(nr, 0.0), O((size_t)nr * d, 0.0);
   // amb: bound on how far the non-unique roundings can move O (before / l)
   std::vector<double> amb((size_t)nr * d, 0.0);
+  // arun: the largest sum of |q_c k_c| of the row so far (error of its max)
+  std::vector<double> arun(nr, 0.0);
   std::vector<double> dq(blk);
   std::vector<double> kt((size_t)blk * d), vt((size_t)blk * d), S(blk);
-  std::vector<float> Pt(blk), Ph(blk);
+  std::vector<float> Pt(blk);
   std::vector<double> Pq(blk);
 
   for (int code : order) {
@@ -690,60 +822,42 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
     for (int r = 0; r < nr; ++r) {
       const int row = r0 + r;
       const double* qv = fp4 ? &qh[(size_t)r * d] : &q16[(size_t)r * d];
-      double mt = -INFINITY;
+      double mt = -INFINITY, amx = 0.0, smx = 0.0;
       for (int t = 0; t < nk; ++t) {
         if (C.causal && k0 + t > row) {
           S[t] = -INFINITY;
           continue;
         }
-        double acc = 0.0;
-        for (int c = 0; c < d; ++c) acc += qv[c] * kt[(size_t)t * d + c];
+        double acc = 0.0, aabs = 0.0;
+        for (int c = 0; c < d; ++c) {
+          acc += qv[c] * kt[(size_t)t * d + c];
+          aabs += std::fabs(qv[c] * kt[(size_t)t * d + c]);
+        }
         S[t] = acc * (fp4 ? s4 : s16);
         mt = std::max(mt, S[t]);
+        amx = std::max(amx, aabs * (fp4 ? s4 : s16));
+        smx = std::max(smx, std::fabs(S[t]));
       }
       if (mt == -INFINITY) continue;
       const double mn = std::max(m[r], mt);
       const double alpha = std::exp2(m[r] - mn);  // 0 when m is still -inf
+      arun[r] = std::max(arun[r], amx);
       l[r] *= alpha;
       for (int c = 0; c < d; ++c) {
         O[(size_t)r * d + c] *= alpha;
         amb[(size_t)r * d + c] *= alpha;
       }
-      float rowmax = 0.0f;
       for (int t = 0; t < nk; ++t) {
         Pt[t] = S[t] == -INFINITY ? 0.0f : (float)std::exp2(S[t] - mn);
         l[r] += (double)Pt[t];
-        rowmax = std::max(rowmax, Pt[t]);
       }
       if (fp4) {
-        // Two-level quantisation of the probability row tile (reading R7).
-        if (rowmax == 0.0f) { m[r] = mn; continue; }
-        const float inv = 2688.0f / rowmax;
-        const float sigma = rowmax / 2688.0f;
-        for (int t = 0; t < blk; ++t) Ph[t] = t < nk ? Pt[t] * inv : 0.0f;
-        for (int b0 = 0; b0 < blk; b0 += 16) {
-          float amax = 0.0f;
-          for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
-          const float s_real = amax / 6.0f;
-          uint8_t sp = orc_ue4m3_encode(s_real);
-          float dec = orc_ue4m3_decode(sp);
-          float rr = 1.0f / dec;
-          for (int e = 0; e < 16; ++e) {
-            const float tq = Ph[b0 + e] * rr;
-            Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(tq)) * (double)dec;
-            dq[b0 + e] = sp == 0 ? 0.0 : e2m1_ambiguity(tq) * (double)dec;
-          }
-          // a block scale at a rounding midpoint: the other byte's block
-          const int alt = ue4m3_ambiguous_neighbour(s_real, sp);
-          if (alt > 0) {
-            const float dec2 = orc_ue4m3_decode((uint8_t)alt);
-            const float rr2 = 1.0f / dec2;
-            for (int e = 0; e < 16; ++e) {
-              const double q2 = (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr2)) * (double)dec2;
-              dq[b0 + e] = std::max(dq[b0 + e], std::fabs(q2 - Pq[b0 + e]));
-            }
-          }
-        }
+        // Two-level quantisation of the probability row tile (reading R7),
+        // each row's P taken relative to the tile maximum on the GPU.
+        const double rho = tile_radius(d, amx, smx, std::fabs(mt));
+        const float sigma = p_tile_fp4(Pt.data(), nk, blk, rho, s, h, row, k0, Pq.data(),
+                                       dq.data());
+        if (sigma == 0.0f) { m[r] = mn; continue; }
         for (int c = 0; c < d; ++c) {
           double acc = 0.0, ab = 0.0;
           for (int t = 0; t < nk; ++t) {
@@ -754,12 +868,13 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
           amb[(size_t)r * d + c] += (double)sigma * ab;
         }
       } else {
-        for (int t = 0; t < nk; ++t) dq[t] = half_ambiguity((double)Pt[t], C.dt);
+        // FP16 path: P taken against the running max on the GPU
+        const double rho = tile_radius(d, arun[r], smx, std::fabs(mn));
+        p_tile_16(Pt.data(), nk, C.dt, rho, s, h, row, k0, Pq.data(), dq.data());
         for (int c = 0; c < d; ++c) {
           double acc = 0.0, ab = 0.0;
           for (int t = 0; t < nk; ++t) {
-            acc += (double)orc_half_to_float(orc_double_to_half((double)Pt[t], C.dt), C.dt) *
-                   vt[(size_t)t * d + c];
+            acc += Pq[t] * vt[(size_t)t * d + c];
             ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
           }
           O[(size_t)r * d + c] += acc;
@@ -792,8 +907,9 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // its final rounding to the 16-bit type.  tol (optional) receives, per output
 // element, a bound on how far roundings that are not unique can move it: a
 // probability whose E2M1 code, UE4M3 block scale or 16-bit value lies within
-// 2e-5 relative of a rounding midpoint may take either side in an
-// implementation that evaluates the same arithmetic in another order.
+// the radius of tile_radius() of a rounding midpoint may take either side in
+// an implementation that evaluates the same arithmetic in another order.
+
 // Quantiser of a [rows, cols] fp32 matrix (unpacked codes), tensor scale
 // amax/2688 over the whole matrix: the same arithmetic as
 // quantize_rows_unpacked on values that are not 16-bit.
@@ -1043,10 +1159,10 @@ static void decode_row(const DecCtx& C, int b, int h, uint16_t* out, float* lse,
     qh[c] = deq(C.qc[(size_t)(orow + c)], C.qs[(size_t)((orow + c) / 16)], C.gq);
     q16[c] = orc_half_to_float(C.q[orow + c], C.dt);
   }
-  double m = -INFINITY, l = 0.0;
+  double m = -INFINITY, l = 0.0, arun = 0.0;
   std::vector<double> O(d, 0.0), amb(d, 0.0), dq(blk), kt((size_t)blk * d), vt((size_t)blk * d),
       S(blk), Pq(blk);
-  std::vector<float> Pt(blk), Ph(blk);
+  std::vector<float> Pt(blk);
   const int64_t vcol = C.nbcap * (int64_t)blk;  // padded tokens per V column
   for (int code : order) {
     const bool fp4 = code >= 0;
@@ -1065,54 +1181,34 @@ static void decode_row(const DecCtx& C, int b, int h, uint16_t* out, float* lse,
         }
       }
     const double* qv = fp4 ? qh.data() : q16.data();
-    double mt = -INFINITY;
+    double mt = -INFINITY, amx = 0.0, smx = 0.0;
     for (int t = 0; t < nk; ++t) {
-      double acc = 0.0;
-      for (int c = 0; c < d; ++c) acc += qv[c] * kt[(size_t)t * d + c];
+      double acc = 0.0, aabs = 0.0;
+      for (int c = 0; c < d; ++c) {
+        acc += qv[c] * kt[(size_t)t * d + c];
+        aabs += std::fabs(qv[c] * kt[(size_t)t * d + c]);
+      }
       S[t] = acc * (fp4 ? s4 : s16);
       mt = std::max(mt, S[t]);
+      amx = std::max(amx, aabs * (fp4 ? s4 : s16));
+      smx = std::max(smx, std::fabs(S[t]));
     }
     const double mn = std::max(m, mt);
     const double alpha = std::exp2(m - mn);  // 0 when m is still -inf
+    arun = std::max(arun, amx);
     l *= alpha;
     for (int c = 0; c < d; ++c) {
       O[c] *= alpha;
       amb[c] *= alpha;
     }
-    float rowmax = 0.0f;
     for (int t = 0; t < nk; ++t) {
       Pt[t] = (float)std::exp2(S[t] - mn);
       l += (double)Pt[t];
-      rowmax = std::max(rowmax, Pt[t]);
     }
     if (fp4) {
-      if (rowmax == 0.0f) { m = mn; continue; }
-      const float inv = 2688.0f / rowmax;
-      const float sigma = rowmax / 2688.0f;
-      for (int t = 0; t < blk; ++t) Ph[t] = t < nk ? Pt[t] * inv : 0.0f;
-      for (int b0 = 0; b0 < blk; b0 += 16) {
-        float amax = 0.0f;
-        for (int e = 0; e < 16; ++e) amax = std::max(amax, Ph[b0 + e]);
-        const float s_real = amax / 6.0f;
-        const uint8_t sp = orc_ue4m3_encode(s_real);
-        const float dec = orc_ue4m3_decode(sp);
-        const float rr = 1.0f / dec;
-        for (int e = 0; e < 16; ++e) {
-          const float tq = Ph[b0 + e] * rr;
-          Pq[b0 + e] = sp == 0 ? 0.0 : (double)orc_e2m1_decode(orc_e2m1_encode(tq)) * (double)dec;
-          dq[b0 + e] = sp == 0 ? 0.0 : e2m1_ambiguity(tq) * (double)dec;
-        }
-        const int alt = ue4m3_ambiguous_neighbour(s_real, sp);
-        if (alt > 0) {
-          const float dec2 = orc_ue4m3_decode((uint8_t)alt);
-          const float rr2 = 1.0f / dec2;
-          for (int e = 0; e < 16; ++e) {
-            const double q2 =
-                (double)orc_e2m1_decode(orc_e2m1_encode(Ph[b0 + e] * rr2)) * (double)dec2;
-            dq[b0 + e] = std::max(dq[b0 + e], std::fabs(q2 - Pq[b0 + e]));
-          }
-        }
-      }
+      const double rho = tile_radius(d, amx, smx, std::fabs(mt));
+      const float sigma = p_tile_fp4(Pt.data(), nk, blk, rho, b, h, 0, k0, Pq.data(), dq.data());
+      if (sigma == 0.0f) { m = mn; continue; }
       for (int c = 0; c < d; ++c) {
         double acc = 0.0, ab = 0.0;
         for (int t = 0; t < nk; ++t) {
@@ -1123,12 +1219,12 @@ static void decode_row(const DecCtx& C, int b, int h, uint16_t* out, float* lse,
         amb[c] += (double)sigma * ab;
       }
     } else {
-      for (int t = 0; t < nk; ++t) dq[t] = half_ambiguity((double)Pt[t], C.dt);
+      const double rho = tile_radius(d, arun, smx, std::fabs(mn));
+      p_tile_16(Pt.data(), nk, C.dt, rho, b, h, 0, k0, Pq.data(), dq.data());
       for (int c = 0; c < d; ++c) {
         double acc = 0.0, ab = 0.0;
         for (int t = 0; t < nk; ++t) {
-          acc += (double)orc_half_to_float(orc_double_to_half((double)Pt[t], C.dt), C.dt) *
-                 vt[(size_t)t * d + c];
+          acc += Pq[t] * vt[(size_t)t * d + c];
           ab += dq[t] * std::fabs(vt[(size_t)t * d + c]);
         }
         O[c] += acc;

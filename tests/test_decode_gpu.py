@@ -25,26 +25,11 @@ from bit_quantization_b200 import ops, synth
 
 pytestmark = pytest.mark.gpu
 
-MAX_ABS = 1e-2
-MIN_COS = 0.9999
-
-
-def half_ulp(x, dtype):
-    mant, emin = (7, -126) if dtype == torch.bfloat16 else (10, -14)
-    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** emin)))
-    return 0.5 * 2.0 ** (e - mant)
+from parity_bars import compare
 
 
 def _compare(got, want64, tol, dtype, what="out"):
-    got = got.reshape(-1).astype(np.float64)
-    want = want64.reshape(-1)
-    excess = np.abs(got - want) - half_ulp(want, dtype) - tol.reshape(-1)
-    worst = int(np.argmax(excess))
-    nrm = np.linalg.norm(got) * np.linalg.norm(want)
-    cos = float(got @ want / nrm) if nrm > 0 else 1.0
-    assert excess[worst] <= MAX_ABS and cos >= MIN_COS, (
-        f"{what}: |err| - ulp/2 - tol = {excess[worst]:.3e} at {worst} (got {got[worst]}, "
-        f"want {want[worst]}), cos {cos:.6f}")
+    compare(got, want64, dtype, tol, what)
 
 
 def _gkv(orc, k, v, lengths, dt):
