@@ -127,57 +127,82 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
 // ------------------------------------------- one-pass row quantiser --
 // The whole tensor in one launch when it fits in shared memory: every CTA
 // (one per SM, co-resident by a cooperative launch) stages its contiguous
-// chunk of blocks once, takes the chunk absmax, publishes it, waits for all
-// CTAs (bounded wait), reduces the published maxima to the tensor absmax and
-// quantises its chunk from shared memory.  Same arithmetic as the two-pass
-// path.  sync[0] counts arrivals; the launching code zeroes it on the stream
-// right before every launch, so nothing depends on what an earlier call (one
-// that timed out included) left in the workspace.  partial[] has one float
-// per CTA.  chunk is a multiple of 32 blocks (rows stay whole for the
-// Hadamard lanes).
+// chunk of blocks in pieces, takes the chunk absmax as the pieces land,
+// publishes it in its own slot of the workspace tagged with this launch's
+// grid identifier, waits until every CTA's slot carries that tag (bounded
+// wait), reduces the published maxima to the tensor absmax and quantises its
+// chunk from shared memory.  Same arithmetic as the two-pass path.
+// The grid identifier (%gridid) is unique per launch in the context, each
+// replay of a CUDA graph included, so slots written by earlier launches, or
+// any other contents of the workspace, never match: the workspace needs no
+// initial contents and nothing resets it.  A slot is 16 bytes: the tag (64
+// bits, written last with release semantics) and the CTA's maximum.  chunk
+// is a multiple of 32 blocks (rows stay whole for the Hadamard lanes, and
+// every lane of a warp runs the same number of iterations).
 constexpr int kOnePassThreads = 512;
+constexpr int kOnePassPieces = 4;
+
+__device__ __forceinline__ uint64_t grid_id() {
+  uint64_t g;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+  return g;
+}
 
 template <int DT, int G, bool SS>
 __global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
-    const uint16_t* __restrict__ x, int64_t n_blocks, int64_t chunk, unsigned* sync,
-    float* partial, float* tensor_scale, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales) {
+    const uint16_t* __restrict__ x, int64_t n_blocks, int64_t chunk, uint8_t* slots,
+    float* tensor_scale, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   extern __shared__ uint4 cs[];  // chunk blocks x 32 bytes
   __shared__ float red[32];
   __shared__ int s_ok;
-  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ __align__(8) uint64_t s_bar[kOnePassPieces];
   const int64_t b0 = (int64_t)blockIdx.x * chunk;
   const int64_t nvalid = b0 < n_blocks ? min(chunk, n_blocks - b0) : 0;
-  // the chunk arrives by one bulk copy; blocks past the tensor end are zeros
+  // pieces of whole warps' worth of blocks; the last may be short or empty
+  const int64_t pc = ((chunk / kOnePassPieces + 31) / 32) * 32;
+  const uint64_t gid = grid_id();
+  // blocks past the tensor end are zeros
   for (int64_t i = nvalid + threadIdx.x; i < chunk; i += blockDim.x)
     cs[2 * i] = cs[2 * i + 1] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
-    mbar_init(&s_bar, 1);
+    for (int p = 0; p < kOnePassPieces; ++p) mbar_init(&s_bar[p], 1);
     fence_mbar_init();
-    if (nvalid > 0) {
-      mbar_arrive_expect_tx(&s_bar, (uint32_t)(nvalid * 32));
-      bulk_g2s(cs, x + b0 * 16, (uint32_t)(nvalid * 32), &s_bar);
-    } else {
-      mbar_arrive(&s_bar);
+    for (int p = 0; p < kOnePassPieces; ++p) {
+      const int64_t lo = min(p * pc, nvalid), hi = min((p + 1) * pc, nvalid);
+      if (hi > lo) {
+        mbar_arrive_expect_tx(&s_bar[p], (uint32_t)((hi - lo) * 32));
+        bulk_g2s(cs + 2 * lo, x + (b0 + lo) * 16, (uint32_t)((hi - lo) * 32), &s_bar[p]);
+      } else {
+        mbar_arrive(&s_bar[p]);
+      }
     }
   }
   __syncthreads();
-  {
+  float a = 0.0f;
+  bool ok = true;
+  for (int p = 0; p < kOnePassPieces && ok; ++p) {
     int never = 0;
-    if (!mbar_wait(&s_bar, 0, &never)) {
-      // timed out (status word set): give the copy a last bounded wait so
-      // that it does not land after the CTA has left
-      int again = 0;
-      mbar_wait(&s_bar, 0, &again, 200000000ull);
-      return;
+    // one decision per warp: the Hadamard lanes exchange values in the loop
+    if (!__all_sync(0xffffffffu, mbar_wait(&s_bar[p], 0, &never))) {
+      ok = false;
+      break;
+    }
+    for (int64_t i = p * pc + threadIdx.x; i < min((p + 1) * pc, chunk); i += blockDim.x) {
+      float v[16];
+      unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
+      if constexpr (G > 0) fwht_rows16<G>(v);
+      a = fmaxf(a, block_absmax(v));
     }
   }
-  float a = 0.0f;
-  for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
-    float v[16];
-    unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
-    if constexpr (G > 0) fwht_rows16<G>(v);
-    a = fmaxf(a, block_absmax(v));
+  if (__syncthreads_or(!ok)) {
+    // timed out (status word set): give every copy a last bounded wait so
+    // that none lands after the CTA has left
+    if (threadIdx.x == 0)
+      for (int p = 0; p < kOnePassPieces; ++p) {
+        int again = 0;
+        mbar_wait(&s_bar[p], 0, &again, 200000000ull);
+      }
+    return;
   }
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
@@ -186,22 +211,25 @@ __global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
   if (threadIdx.x == 0) {
     float c = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c = fmaxf(c, red[w]);
-    partial[blockIdx.x] = c;
-    __threadfence();
-    atomicAdd(&sync[0], 1u);
-    // wait for every CTA's maximum (bounded)
-    s_ok = spin_until_geq(sync, gridDim.x) ? 1 : 0;
+    uint8_t* my = slots + 16 * (int64_t)blockIdx.x;
+    *reinterpret_cast<volatile float*>(my + 8) = c;
+    store_release64(my, gid);
+    s_ok = 1;
   }
   __syncthreads();
-  if (!s_ok) return;
-  // tensor absmax from the published maxima (each thread folds a few)
+  // every CTA's maximum, one slot per thread (bounded wait on its tag)
   float m = 0.0f;
-  for (int c = threadIdx.x; c < (int)gridDim.x; c += blockDim.x) m = fmaxf(m, __ldcg(partial + c));
+  for (int c = threadIdx.x; c < (int)gridDim.x; c += blockDim.x) {
+    const uint8_t* sl = slots + 16 * (int64_t)c;
+    if (!spin_until_eq64(sl, gid)) s_ok = 0;
+    m = fmaxf(m, *reinterpret_cast<const volatile float*>(sl + 8));
+  }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   __syncthreads();
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
+  if (!s_ok) return;
   float amax = 0.0f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
   const float g = tensor_scale_from_amax(__float_as_uint(amax));

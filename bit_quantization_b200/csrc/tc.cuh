@@ -94,6 +94,30 @@ __device__ __forceinline__ bool spin_until_geq(const unsigned* word, unsigned ta
   }
 }
 
+// Bounded spin until the 64-bit global word equals `tag` (acquire loads at
+// GPU scope, so what the writer stored before its release store of the tag
+// is visible after).  Gives up after `limit_ns` of wall time, sets the device
+// status word and returns false.
+__device__ __forceinline__ bool spin_until_eq64(const void* word, uint64_t tag,
+                                                uint64_t limit_ns = 2000000000ull) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
+    if (v == tag) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_device_status(THRIFT_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Release store of a 64-bit word at GPU scope: this thread's earlier writes
+// are visible to a thread that reads the word with acquire semantics.
+__device__ __forceinline__ void store_release64(void* word, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(word), "l"(v) : "memory");
+}
+
 // ------------------------------------------------- bulk copies (TMA unit) --
 
 // Contiguous global -> shared copy completing on `bar` (transaction bytes).

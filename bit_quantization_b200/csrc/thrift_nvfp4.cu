@@ -136,12 +136,12 @@ void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, i
                                        codes, scales);
 }
 
-// Quantiser workspace: word 0 is the arrival count of the one-pass kernel
-// (zeroed on the stream before each of its launches), word 2 the absmax of
-// the two-pass path, and from byte 256 one float per CTA of the one-pass
-// kernel.  No call depends on the workspace's earlier contents.
+// Quantiser workspace: word 2 is the absmax of the two-pass path, and from
+// byte 256 one 16-byte slot per CTA of the one-pass kernel (its maximum,
+// tagged with the launch's grid identifier).  No call depends on the
+// workspace's earlier contents.
 constexpr size_t kQuantWsBytes = 4096;
-constexpr int kQuantMaxCtas = (int)((kQuantWsBytes - 256) / 4);
+constexpr int kQuantMaxCtas = (int)((kQuantWsBytes - 256) / 16);
 constexpr int64_t kOnePassSmemMax = 200 * 1024;
 
 // The one-pass quantiser when the tensor fits in the SMs' shared memory;
@@ -173,11 +173,8 @@ bool try_quant_onepass(const void* x, int64_t nb, uint32_t* ws, float* ts, uint8
   cfg.attrs = at;
   cfg.numAttrs = 1;
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  float* partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
-  // the arrival counter starts from zero whatever an earlier call left there
-  if (cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return false;
-  return cudaLaunchKernelEx(&cfg, kern, xp, nb, chunk, ws, partial, ts, codes, scales) ==
-         cudaSuccess;
+  uint8_t* slots = reinterpret_cast<uint8_t*>(ws) + 256;
+  return cudaLaunchKernelEx(&cfg, kern, xp, nb, chunk, slots, ts, codes, scales) == cudaSuccess;
 }
 
 template <int DT>

@@ -93,10 +93,11 @@ thrift_status thrift_stream_status(void* stream, int reset);
  *     transform first (cols must be 64 or 128).
  * Requirements: rows >= 0, cols % 16 == 0, cols <= 4096.
  * Workspace: nvfp4_quantize_workspace_size() bytes, 16-byte aligned, no
- *   initial contents required: the one-pass kernel's arrival counter is
- *   cleared on the stream before each of its launches, so one buffer serves
- *   any number of calls issued in stream order, after a device timeout too.
- *   Calls that overlap on the GPU must not share a workspace.
+ *   initial contents required: the one-pass kernel's per-CTA maxima are
+ *   tagged with the launch's grid identifier, so nothing from an earlier
+ *   call (a timed-out one included) or any other contents can be taken for
+ *   this call's; one buffer serves any number of calls issued in stream
+ *   order.  Calls that overlap on the GPU must not share a workspace.
  *   nvfp4_quantize_colblocks takes the same workspace.
  * Execution: when the tensor scale is computed and the tensor fits in the
  *   SMs' shared memory (about 200 KB per SM), one cooperative launch stages
