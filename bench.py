@@ -769,6 +769,28 @@ class AttnCase:
                                 out=out, lse=lse, workspace=self.ws, sink_blocks=sink,
                                 recent_blocks=recent, smooth_k=smooth)
 
+    def run_sharded(self, world, q=None, k=None, v=None, out=None, lse=None):
+        """One step of a problem split across `world` ranks, on this rank's
+        shard (its inputs): the shard's three tensor absmaxes, their maximum
+        over the ranks (one all-reduce of 3 floats), then the attention under
+        the agreed absmaxes.  With one rank the same calls, no all-reduce."""
+        from bit_quantization_b200 import shard
+        w, ops = self.w, self.ops
+        q = self.q if q is None else q
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
+        if not hasattr(self, "amax"):
+            self.amax = torch.empty(3, dtype=torch.float32, device=self.dev)
+        ops.thrift_attn_absmax(q, k, v, self.cu, self.maxlen, blk=w.blk,
+                               use_hadamard=w.use_hadamard, amax=self.amax, workspace=self.ws)
+        shard.agree_absmax(self.amax, world)
+        ops.thrift_attn_fwd_absmax(q, k, v, self.amax, self.cu, self.maxlen, blk=w.blk,
+                                   causal=w.causal, topk_frac=w.topk_frac,
+                                   use_scalesearch=w.use_scalesearch, use_hadamard=w.use_hadamard,
+                                   out=out, lse=lse, workspace=self.ws)
+
     def mask(self):
         """The selection [nseq, H, nB, nB] the last call left in the workspace."""
         w = self.w
@@ -973,8 +995,12 @@ def main():
     f4, f16 = case.flops()
     flops = f4 + f16
 
+    # Each rank holds one shard (its own batch entries: seed + rank) of one
+    # problem of world x B sequences; the step agrees the tensor absmaxes
+    # across ranks by one max all-reduce of 3 floats (NCCL), so every code is
+    # the one-GPU run's of that whole problem.
     for _ in range(args.warmup):
-        case.run()
+        case.run_sharded(world)
     torch.cuda.synchronize(dev)
     if ops.device_status(reset=True) != ops.OK:
         raise RuntimeError("device wait timed out during warm-up")
@@ -988,7 +1014,7 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        case.run()
+        case.run_sharded(world)
     e1.record()
     torch.cuda.synchronize(dev)
     ops.kernel_timer_enable(False)
@@ -1036,7 +1062,7 @@ def main():
                 s_comp.wait_event(ev_in[b])
                 if st >= 2:
                     s_comp.wait_event(ev_out[b])  # step st-2's results have left buffer b
-                case.run(qd[b], kd[b], vd[b], od[b], ld[b])
+                case.run_sharded(world, qd[b], kd[b], vd[b], od[b], ld[b])
                 ev_comp[b].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[b])
@@ -1067,7 +1093,10 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
-            "data": "synthetic", "config": config_of(w, case.lengths), "roofline": roofline,
+            "data": "synthetic", "config": dict(config_of(w, case.lengths), parallelism=(
+                f"one problem of {world} x {w.B if w.varlen is None else len(case.lengths)} "
+                f"sequences split by batch across {world} GPU(s); per step one max all-reduce "
+                f"of the 3 tensor absmaxes")), "roofline": roofline,
             "alu_roofline": alu_roofline(flops, w.d, k_ms, sm_mhz, n_sm),
             "e2e": {"value": dist.whole_job_rate(job_flops, e2e_ms) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,

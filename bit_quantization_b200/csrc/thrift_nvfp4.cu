@@ -310,16 +310,16 @@ thrift_status launch_attn_kernel(const AttnParams& p, int nTq, cudaStream_t st) 
   return s;
 }
 
+// The three tensor absmaxes of an attention call into amax[0..2] (bit
+// patterns of non-negative floats): Q and K rotated when `had`, K - mu with
+// K smoothing (whose channel means land in w.kmu on the way).
 template <int DT>
-thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
-                        int64_t total, int maxlen, int H, int Hkv, int d, int blk, int causal,
-                        float frac, int sink, int recent, int ss, int had, int smooth, void* out,
-                        float* lse, int lse_varlen, void* ws, cudaStream_t st) {
-  AttnWs w = carve_attn(ws, nseq, maxlen, H, Hkv, d, blk);
-  const int nB = (int)ceil_div(maxlen, blk), nTq = (int)ceil_div(maxlen, 128);
+thrift_status attn_absmax(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
+                          int64_t total, int maxlen, int H, int Hkv, int d, int had, int smooth,
+                          const AttnWs& w, uint32_t* amax, cudaStream_t st) {
   const int G = d / 16;
-  if (cudaMemsetAsync(w.amax, 0, 16, st) != cudaSuccess) return THRIFT_ERR_CUDA;
-  launch_amax<DT>(q, total * H * d / 16, had ? G : 0, w.amax + 0, st);
+  if (cudaMemsetAsync(amax, 0, 12, st) != cudaSuccess) return THRIFT_ERR_CUDA;
+  launch_amax<DT>(q, total * H * d / 16, had ? G : 0, amax + 0, st);
   if (smooth) {
     // K smoothing: channel means per (sequence, kv head) and the absmax of
     // K - mu, from one pass of block statistics over K
@@ -327,11 +327,40 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
     k_stats_kernel<DT><<<dim3(nb128, Hkv, nseq), 128, 0, st>>>(
         static_cast<const uint16_t*>(k), si, Hkv, d, nb128, w.ksum, w.kmin, w.kmax);
     k_mean_kernel<<<dim3(Hkv, nseq), 128, 0, st>>>(w.ksum, w.kmin, w.kmax, si, Hkv, d, nb128,
-                                                   w.kmu, w.amax + 1);
+                                                   w.kmu, amax + 1);
   } else {
-    launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, w.amax + 1, st);
+    launch_amax<DT>(k, total * Hkv * d / 16, had ? G : 0, amax + 1, st);
   }
-  launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
+  launch_amax<DT>(v, total * Hkv * d / 16, 0, amax + 2, st);
+  return launch_status();
+}
+
+// One attention call.  amax_given (device, 3 floats) replaces the call's own
+// tensor absmaxes when not null (a shard of a larger problem).
+template <int DT>
+thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
+                        int64_t total, int maxlen, int H, int Hkv, int d, int blk, int causal,
+                        float frac, int sink, int recent, int ss, int had, int smooth, void* out,
+                        float* lse, int lse_varlen, void* ws, cudaStream_t st,
+                        const float* amax_given = nullptr) {
+  AttnWs w = carve_attn(ws, nseq, maxlen, H, Hkv, d, blk);
+  const int nB = (int)ceil_div(maxlen, blk), nTq = (int)ceil_div(maxlen, 128);
+  const int G = d / 16;
+  if (amax_given) {
+    // the given absmaxes; K smoothing still needs this shard's channel means
+    // (its own absmax goes to a spare word)
+    if (smooth) {
+      const thrift_status s0 = attn_absmax<DT>(q, k, v, si, nseq, total, maxlen, H, Hkv, d, had,
+                                               smooth, w, w.amax + 4, st);
+      if (s0 != THRIFT_OK) return s0;
+    }
+    if (cudaMemcpyAsync(w.amax, amax_given, 12, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return THRIFT_ERR_CUDA;
+  } else {
+    const thrift_status s0 = attn_absmax<DT>(q, k, v, si, nseq, total, maxlen, H, Hkv, d, had,
+                                             smooth, w, w.amax, st);
+    if (s0 != THRIFT_OK) return s0;
+  }
   // Q and K images, with the block means of the selection on the way
   TileArgs aq{q, si, nseq, H, 128, nTq, blk, nB, w.amax + 0, w.q4, w.q16, w.means_q};
   TileArgs ak{k, si, nseq, Hkv, blk, nB, blk, nB, w.amax + 1, w.k4, w.k16, w.means_k};
@@ -999,6 +1028,61 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
   return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
                       sink_blocks, recent_blocks, use_scalesearch, use_hadamard, smooth_k, out,
                       lse, 1, workspace, st);
+}
+
+thrift_status thrift_attn_absmax(const void* q, const void* k, const void* v, thrift_dtype dt,
+                                 const int32_t* cu_seqlens, int nseq, int64_t total,
+                                 int max_seqlen, int H, int Hkv, int d, int blk, int use_hadamard,
+                                 int smooth_k, float* amax_out, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  if (!q || !k || !v || !amax_out || !workspace || !aligned16(workspace)) return THRIFT_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return THRIFT_ERR_ARG;
+  if (dt != THRIFT_F16 && dt != THRIFT_BF16) return THRIFT_ERR_ARG;
+  if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || max_seqlen <= 0 || total <= 0)
+    return THRIFT_ERR_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (smooth_k && use_hadamard) return THRIFT_ERR_UNSUPPORTED;
+  if (!cu_seqlens && total != (int64_t)nseq * max_seqlen) return THRIFT_ERR_ARG;
+  if (ws_bytes < thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk))
+    return THRIFT_ERR_ARG;
+  const SeqInfo si{cu_seqlens, cu_seqlens ? 0 : max_seqlen};
+  const AttnWs w = carve_attn(workspace, nseq, max_seqlen, H, Hkv, d, blk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* a = reinterpret_cast<uint32_t*>(amax_out);
+  if (dt == THRIFT_BF16)
+    return attn_absmax<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_hadamard,
+                          smooth_k, w, a, st);
+  return attn_absmax<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_hadamard, smooth_k,
+                        w, a, st);
+}
+
+thrift_status thrift_attn_fwd_absmax(const void* q, const void* k, const void* v,
+                                     thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                     int64_t total, int max_seqlen, int H, int Hkv, int d,
+                                     int blk, int causal, float topk_frac, int sink_blocks,
+                                     int recent_blocks, int use_scalesearch, int use_hadamard,
+                                     int smooth_k, const float* amax_in, void* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  thrift_status s = check_attn_args(q, k, v, dt, H, Hkv, max_seqlen, d, blk, topk_frac, out, lse);
+  if (s != THRIFT_OK) return s;
+  if (sink_blocks < 0 || recent_blocks < 0 || !amax_in) return THRIFT_ERR_ARG;
+  if (smooth_k && use_hadamard) return THRIFT_ERR_UNSUPPORTED;
+  if (nseq <= 0 || nseq > 65535 || total <= 0 || !workspace || !aligned16(workspace))
+    return THRIFT_ERR_ARG;
+  if (!cu_seqlens && total != (int64_t)nseq * max_seqlen) return THRIFT_ERR_ARG;
+  if (ws_bytes < thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H, Hkv, d, blk))
+    return THRIFT_ERR_ARG;
+  const SeqInfo si{cu_seqlens, cu_seqlens ? 0 : max_seqlen};
+  const int lse_varlen = cu_seqlens ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == THRIFT_BF16)
+    return attn_impl<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
+                        sink_blocks, recent_blocks, use_scalesearch, use_hadamard, smooth_k, out,
+                        lse, lse_varlen, workspace, st, amax_in);
+  return attn_impl<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, blk, causal, topk_frac,
+                      sink_blocks, recent_blocks, use_scalesearch, use_hadamard, smooth_k, out,
+                      lse, lse_varlen, workspace, st, amax_in);
 }
 
 size_t thrift_kv_cache_size(int B, int Hkv, int capacity, int d, int blk) {

@@ -28,7 +28,7 @@ EXPORTS = (
     "nvfp4_quantize", "nvfp4_quantize_colblocks", "block_mean_topk_workspace_size",
     "block_mean_topk", "block_mean_topk_noalloc", "thrift_attn_workspace_size", "thrift_attn_fwd",
     "thrift_attn_varlen_workspace_size", "thrift_attn_fwd_varlen",
-    "thrift_attn_workspace_mask_offset",
+    "thrift_attn_absmax", "thrift_attn_fwd_absmax", "thrift_attn_workspace_mask_offset",
     "thrift_kernel_timer_enable", "thrift_kernel_timer_read", "thrift_test_wait_timeout",
     "thrift_kv_cache_size", "thrift_kv_cache_append", "thrift_attn_decode_workspace_size",
     "thrift_attn_decode_mask_offset", "thrift_attn_decode",
@@ -76,6 +76,12 @@ def lib():
                                       i32, i32, i32, i32, P, P, P, sz, P]
         L.thrift_attn_varlen_workspace_size.restype = sz
         L.thrift_attn_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+        L.thrift_attn_absmax.restype = i32
+        L.thrift_attn_absmax.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32, i32,
+                                         i32, P, P, sz, P]
+        L.thrift_attn_fwd_absmax.restype = i32
+        L.thrift_attn_fwd_absmax.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
+                                             i32, f32, i32, i32, i32, i32, i32, P, P, P, P, sz, P]
         L.thrift_attn_workspace_mask_offset.restype = sz
         L.thrift_attn_workspace_mask_offset.argtypes = [i32, i32, i32, i32, i32, i32]
         L.thrift_attn_fwd_varlen.restype = i32
@@ -417,6 +423,77 @@ def thrift_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, blk=128, causal=True
                                             int(use_hadamard), int(smooth_k), _ptr(out), _ptr(lse),
                                             _ptr(ws), ws.numel(), _stream(q)),
                "thrift_attn_fwd_varlen")
+    return out, lse
+
+
+def _shape_of(q, k, cu_seqlens, max_seqlen):
+    """(nseq, total, max_seqlen, H, Hkv, d) of [B,N,H,d] or packed inputs."""
+    if q.dim() == 4:
+        B, N, H, d = q.shape
+        return B, B * N, N, H, k.shape[2], d
+    if cu_seqlens is None or max_seqlen is None:
+        raise ThriftError("packed inputs need cu_seqlens and max_seqlen")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ThriftError("cu_seqlens must be int32 [nseq + 1]")
+    total, H, d = q.shape
+    return cu_seqlens.numel() - 1, total, int(max_seqlen), H, k.shape[1], d
+
+
+def thrift_attn_absmax(q, k, v, cu_seqlens=None, max_seqlen=None, blk=128, use_hadamard=False,
+                       smooth_k=False, amax=None, workspace=None):
+    """The three tensor absmaxes (Q, K rotated when use_hadamard, V) of an
+    attention call's inputs: float32 [3] on the device.  q [B,N,H,d] or
+    packed [total,H,d] with cu_seqlens / max_seqlen."""
+    _check_qkv(q, k, v, packed=q.dim() == 3)
+    _need_cuda(q, k, v)
+    nseq, total, maxlen, H, Hkv, d = _shape_of(q, k, cu_seqlens, max_seqlen)
+    _check_like(amax, (3,), torch.float32, "amax")
+    if amax is None:
+        amax = torch.empty(3, dtype=torch.float32, device=q.device)
+    need = thrift_attn_varlen_workspace_size(nseq, total, maxlen, H, Hkv, d, blk)
+    if need == 0:
+        raise ThriftError("thrift_attn_absmax: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    with _on(q):
+        _check(lib().thrift_attn_absmax(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens), nseq,
+                                        total, maxlen, H, Hkv, d, blk, int(use_hadamard),
+                                        int(smooth_k), _ptr(amax), _ptr(ws), ws.numel(),
+                                        _stream(q)),
+               "thrift_attn_absmax")
+    return amax
+
+
+def thrift_attn_fwd_absmax(q, k, v, amax, cu_seqlens=None, max_seqlen=None, blk=128,
+                           causal=False, topk_frac=0.0, use_scalesearch=False, use_hadamard=False,
+                           out=None, lse=None, workspace=None, sink_blocks=0, recent_blocks=0,
+                           smooth_k=False):
+    """thrift_attn_fwd (q [B,N,H,d]; lse [B,H,N]) or thrift_attn_fwd_varlen
+    (packed, cu_seqlens; lse [H,total]) with the three tensor absmaxes given
+    (float32 [3] on the device, e.g. agreed across the shards of a problem)."""
+    _check_qkv(q, k, v, packed=q.dim() == 3)
+    nseq, total, maxlen, H, Hkv, d = _shape_of(q, k, cu_seqlens, max_seqlen)
+    lse_shape = (H, total) if q.dim() == 3 else (nseq, H, maxlen)
+    _check_like(amax, (3,), torch.float32, "amax")
+    _check_like(out, q.shape, q.dtype, "out")
+    _check_like(lse, lse_shape, torch.float32, "lse")
+    _need_cuda(q, k, v, amax)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    need = thrift_attn_varlen_workspace_size(nseq, total, maxlen, H, Hkv, d, blk)
+    if need == 0:
+        raise ThriftError("thrift_attn_fwd_absmax: unsupported shape")
+    ws = workspace if workspace is not None else _ws.get(need, q.device)
+    with _on(q):
+        _check(lib().thrift_attn_fwd_absmax(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(cu_seqlens),
+                                            nseq, total, maxlen, H, Hkv, d, blk, int(causal),
+                                            float(topk_frac), int(sink_blocks),
+                                            int(recent_blocks), int(use_scalesearch),
+                                            int(use_hadamard), int(smooth_k), _ptr(amax),
+                                            _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                            _stream(q)),
+               "thrift_attn_fwd_absmax")
     return out, lse
 
 

@@ -213,6 +213,44 @@ thrift_status thrift_attn_fwd_varlen(const void* q, const void* k, const void* v
                                      int smooth_k, void* out, float* lse, void* workspace,
                                      size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------- one problem on several GPUs --
+ * [TA] Metodologia step 1: block means, scores and selection are per
+ * (sequence, head), and so are the NVFP4 blocks of Q, K and V and the
+ * attention itself; the only quantity coupling the heads and sequences of one
+ * problem is the per-tensor FP32 scale g = amax/2688 of Q, K and V.  A
+ * problem split by (sequence, kv-head group) across GPUs therefore gives the
+ * same codes, scales, selection and output as on one GPU once every shard
+ * uses the whole problem's three absmaxes: each shard computes its own with
+ * thrift_attn_absmax, the shards agree on the elementwise maximum (a 3-float
+ * max all-reduce), and each runs thrift_attn_fwd_absmax with it.
+ *
+ * thrift_attn_absmax: amax_out[3] (device fp32, written) = the absmax of Q
+ * and of K (after the Hadamard rotation when use_hadamard; of K - mu with
+ * smooth_k, mu the per-sequence channel means of reading R16) and of V over
+ * this call's tensors.  cu_seqlens: device [nseq+1] for packed sequences, or
+ * NULL for nseq sequences of max_seqlen tokens each ([nseq, max_seqlen, .]
+ * layout, total = nseq * max_seqlen).  workspace: as thrift_attn_fwd_absmax.
+ *
+ * thrift_attn_fwd_absmax: thrift_attn_fwd / thrift_attn_fwd_varlen (chosen
+ * by cu_seqlens as above; lse [nseq, H, max_seqlen] without cu_seqlens,
+ * [H, total] with them) with the three tensor absmaxes read from amax_in
+ * (device fp32 [3]) instead of computed: g = amax/2688 (1 for 0) as always.
+ * Workspace: thrift_attn_varlen_workspace_size(nseq, total, max_seqlen, H,
+ * Hkv, d, blk) bytes.  Other arguments, requirements and errors as those
+ * calls. */
+thrift_status thrift_attn_absmax(const void* q, const void* k, const void* v, thrift_dtype dt,
+                                 const int32_t* cu_seqlens, int nseq, int64_t total,
+                                 int max_seqlen, int H, int Hkv, int d, int blk, int use_hadamard,
+                                 int smooth_k, float* amax_out, void* workspace, size_t ws_bytes,
+                                 void* stream);
+thrift_status thrift_attn_fwd_absmax(const void* q, const void* k, const void* v,
+                                     thrift_dtype dt, const int32_t* cu_seqlens, int nseq,
+                                     int64_t total, int max_seqlen, int H, int Hkv, int d,
+                                     int blk, int causal, float topk_frac, int sink_blocks,
+                                     int recent_blocks, int use_scalesearch, int use_hadamard,
+                                     int smooth_k, const float* amax_in, void* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
 /* Byte offset, inside the workspace of thrift_attn_fwd (nseq = B,
  * max_seqlen = N) or thrift_attn_fwd_varlen, of the block-pair selection the
  * call leaves there once it has completed on its stream: uint8

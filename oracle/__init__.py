@@ -82,6 +82,11 @@ def lib():
         L.orc_thrift_decode.restype = i32
         L.orc_thrift_decode.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, f32,
                                         i32, i32, i32, P, i32, P, i32, P, P, P, P, P]
+        L.orc_thrift_attn_g.restype = i32
+        L.orc_thrift_attn_g.argtypes = [P, P, P, i32, i32, i32, P, i32, i32, i32, i32, f32, i32,
+                                        i32, i32, i32, i32, P, P, i32, P, i64, i32, P, P, P, P, P]
+        L.orc_tensor_absmax.restype = f32
+        L.orc_tensor_absmax.argtypes = [P, i32, i64, i64, i32]
         L.orc_set_test_hooks.restype = None
         L.orc_set_test_hooks.argtypes = [C.c_double, C.c_uint64, i32, i32, i32, i32, f32, i32]
         _lib = L
@@ -172,6 +177,20 @@ def tensor_scale(x, dt, hadamard=False):
     x = _u16(x)
     cols = x.shape[-1]
     return lib().orc_tensor_scale(_p(x), dt, x.size // cols, cols, int(hadamard))
+
+
+def tensor_absmax(x, dt, hadamard=False):
+    """max |x| over a [..., cols] 16-bit tensor (rows rotated first with
+    hadamard)."""
+    x = _u16(x)
+    cols = x.shape[-1]
+    return lib().orc_tensor_absmax(_p(x), dt, x.size // cols, cols, int(hadamard))
+
+
+def scale_from_absmax(amax):
+    """g = amax / 2688 in fp32 (1 for amax = 0), reading R1."""
+    a = np.float32(amax)
+    return float(np.float32(1.0)) if a == 0 else float(a / np.float32(2688.0))
 
 
 def nvfp4_quantize(x, dt, use_ss=False, use_had=False, g=None):
@@ -277,7 +296,7 @@ def k_channel_means(k, dt, cu):
 
 def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
                 mask=None, units=None, nthreads=None, sink_blocks=0, recent_blocks=0,
-                smooth_k=False):
+                smooth_k=False, g=None):
     """Emulated NVFP4 + FP16 attention over packed sequences.
 
     q [total,H,d], k/v [total,Hkv,d] uint16; cu int32 [nseq+1].
@@ -285,7 +304,8 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
     final rounding to the 16-bit type), tol fp64 [total,H,d] (bound on the
     effect of roundings that are not unique, see oracle.cpp), lse f32
     [H,total], mask flat uint8, g (g_Q, g_K, g_V)).  ``units``: optional int array [n,3] of
-    (sequence, head, query block) to compute; other rows stay 0 / NaN."""
+    (sequence, head, query block) to compute; other rows stay 0 / NaN.  ``g``: optional
+    given (g_Q, g_K, g_V) (a shard of a larger problem), else computed (reading R1)."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     cu = np.ascontiguousarray(cu, np.int32)
     total, H, d = q.shape
@@ -310,11 +330,12 @@ def thrift_attn(q, k, v, dt, cu, blk, causal, frac, use_ss=False, use_had=False,
         n_units = u.shape[0]
     else:
         u, n_units = None, 0
-    rc = lib().orc_thrift_attn_ex(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
-                               int(causal), float(frac), int(sink_blocks), int(recent_blocks),
-                               int(use_ss), int(use_had), int(smooth_k), _p(m), given,
-                               _p(u), n_units, int(nthreads or nthreads_default()), _p(out),
-                               _p(lse), _p(gs), _p(out64), _p(tol))
+    g_in = None if g is None else np.ascontiguousarray(g, np.float32).reshape(3)
+    rc = lib().orc_thrift_attn_g(_p(q), _p(k), _p(v), dt, H, Hkv, _p(cu), len(lens), d, blk,
+                                 int(causal), float(frac), int(sink_blocks), int(recent_blocks),
+                                 int(use_ss), int(use_had), int(smooth_k), _p(g_in), _p(m), given,
+                                 _p(u), n_units, int(nthreads or nthreads_default()), _p(out),
+                                 _p(lse), _p(gs), _p(out64), _p(tol))
     if rc:
         raise ValueError("oracle thrift_attn: bad arguments")
     return {"out": out, "out64": out64, "tol": tol, "lse": lse, "mask": m,

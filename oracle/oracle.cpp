@@ -261,6 +261,14 @@ float orc_tensor_scale(const uint16_t* x, int dt, int64_t rows, int64_t cols, in
   return tensor_scale_of(load_rows(x, dt, rows, cols, hadamard));
 }
 
+// max |x| over a [rows, cols] 16-bit matrix (rows rotated first when
+// hadamard): the quantity g = amax / 2688 of reading R1 is taken from.
+float orc_tensor_absmax(const uint16_t* x, int dt, int64_t rows, int64_t cols, int hadamard) {
+  float amax = 0.0f;
+  for (float f : load_rows(x, dt, rows, cols, hadamard)) amax = std::max(amax, std::fabs(f));
+  return amax;
+}
+
 // ScaleSearch error of one candidate scale byte for a block of 16 values x
 // under tensor scale g (reading R4): t = x * (1/(S g)), q = E2M1 grid value
 // of t, err = (sum over the block, in order, of (t-q)^2 with fmaf) * S^2.
@@ -914,10 +922,11 @@ static void attn_unit(const AttnCtx& C, int s, int h, int i, uint16_t* out, floa
 // amax/2688 over the whole matrix: the same arithmetic as
 // quantize_rows_unpacked on values that are not 16-bit.
 static float quantize_rows_f32(const float* x, int64_t rows, int cols, int use_ss, int nthreads,
-                               std::vector<uint8_t>& codes, std::vector<uint8_t>& scales) {
+                               std::vector<uint8_t>& codes, std::vector<uint8_t>& scales,
+                               const float* g_given = nullptr) {
   float amax = 0.0f;
   for (int64_t e = 0; e < rows * cols; ++e) amax = std::max(amax, std::fabs(x[e]));
-  const float g = amax == 0.0f ? 1.0f : amax / 2688.0f;
+  const float g = g_given ? *g_given : (amax == 0.0f ? 1.0f : amax / 2688.0f);
   codes.assign((size_t)(rows * cols), 0);
   scales.assign((size_t)(rows * (cols / 16)), 0);
   parallel_for((rows + 4095) / 4096, nthreads, [&](int64_t ch) {
@@ -973,6 +982,13 @@ int orc_thrift_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
                             out, lse, gs_out, out64, tol);
 }
 
+int orc_thrift_attn_g(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                      int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
+                      float frac, int sink, int recent, int use_ss, int use_had, int smooth_k,
+                      const float* g_in, uint8_t* mask_io, int mask_given,
+                      const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
+                      float* lse, float* gs_out, double* out64, double* tol);
+
 // As orc_thrift_attn, with optional K smoothing (reading R16).
 int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
                        int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
@@ -980,6 +996,20 @@ int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                        uint8_t* mask_io, int mask_given,
                        const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
                        float* lse, float* gs_out, double* out64, double* tol) {
+  return orc_thrift_attn_g(q, k, v, dt, H, Hkv, cu, nseq, d, blk, causal, frac, sink, recent,
+                           use_ss, use_had, smooth_k, nullptr, mask_io, mask_given, units,
+                           n_units, nthreads, out, lse, gs_out, out64, tol);
+}
+
+// As orc_thrift_attn_ex, with the tensor scales g_Q, g_K, g_V given (g_in,
+// 3 floats; NULL: computed from the tensors, reading R1): a shard of a larger
+// problem quantised under that problem's scales.
+int orc_thrift_attn_g(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dt, int H,
+                      int Hkv, const int32_t* cu, int nseq, int d, int blk, int causal,
+                      float frac, int sink, int recent, int use_ss, int use_had, int smooth_k,
+                      const float* g_in, uint8_t* mask_io, int mask_given,
+                      const int32_t* units, int64_t n_units, int nthreads, uint16_t* out,
+                      float* lse, float* gs_out, double* out64, double* tol) {
   if (H <= 0 || Hkv <= 0 || H % Hkv || nseq <= 0 || d % 16 || blk % 16 || blk <= 0) return -1;
   if (use_had && (d & (d - 1))) return -1;
   if (smooth_k && use_had) return -1;
@@ -1000,7 +1030,8 @@ int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     C.moff[s + 1] = C.moff[s] + (int64_t)H * nb * nb;
   }
   C.ptot = C.pstart[nseq];
-  C.gq = quantize_rows_unpacked(q, dt, C.total * H, d, use_ss, use_had, nthreads, C.qc, C.qs);
+  C.gq = quantize_rows_unpacked(q, dt, C.total * H, d, use_ss, use_had, nthreads, C.qc, C.qs,
+                                g_in ? &g_in[0] : nullptr);
   if (smooth_k) {
     C.mu.assign((size_t)nseq * Hkv * d, 0.0f);
     orc_k_channel_means(k, dt, Hkv, cu, nseq, d, C.mu.data());
@@ -1012,16 +1043,18 @@ int orc_thrift_attn_ex(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
             const int64_t e = (t * Hkv + hk) * d + c;
             ks[(size_t)e] = orc_half_to_float(k[e], dt) - C.mu[((size_t)s2 * Hkv + hk) * d + c];
           }
-    C.gk = quantize_rows_f32(ks.data(), C.total * Hkv, d, use_ss, nthreads, C.kc, C.ks);
+    C.gk = quantize_rows_f32(ks.data(), C.total * Hkv, d, use_ss, nthreads, C.kc, C.ks,
+                             g_in ? &g_in[1] : nullptr);
   } else {
-    C.gk = quantize_rows_unpacked(k, dt, C.total * Hkv, d, use_ss, use_had, nthreads, C.kc, C.ks);
+    C.gk = quantize_rows_unpacked(k, dt, C.total * Hkv, d, use_ss, use_had, nthreads, C.kc, C.ks,
+                                  g_in ? &g_in[1] : nullptr);
   }
   // V: 16-blocks along tokens, every sequence zero-padded to a whole number of
   // key blocks (reading R6).  The tensor scale covers the real tokens only.
   {
     float amax = 0.0f;
     for (int64_t e = 0; e < C.total * Hkv * d; ++e) amax = std::max(amax, std::fabs(orc_half_to_float(v[e], dt)));
-    C.gv = amax == 0.0f ? 1.0f : amax / 2688.0f;
+    C.gv = g_in ? g_in[2] : (amax == 0.0f ? 1.0f : amax / 2688.0f);
     C.vc.assign((size_t)(Hkv * d * C.ptot), 0);
     C.vs.assign((size_t)(Hkv * d * C.ptot / 16), 0);
     parallel_for((int64_t)Hkv * d, nthreads, [&](int64_t hc) {
