@@ -92,22 +92,90 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
   cta_atomic_amax(a, amax_out);
 }
 
-// ------------------------------------------------- row-blocked quantiser --
-// codes [rows, cols/2], scales [rows, cols/16] as flat arrays of blocks.
-template <int DT, int G, bool SS>
-__global__ void __launch_bounds__(256) quant_rows_kernel(
-    const uint16_t* __restrict__ x, int64_t n_blocks, const uint32_t* amax_in,
-    float* tensor_scale, int scale_given, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales) {
-  const float g = scale_given ? *tensor_scale : tensor_scale_from_amax(*amax_in);
-  if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+// ------------------------------------------- quantiser: partial maxima --
+// First kernel of the quantiser when the tensor scale is computed: CTA c
+// writes the absmax of its share of x (blocks c*KPT*256 + ..., grid-stride)
+// to partial[c].  Launched with programmatic dependent launch: the loads
+// and the maximum run while the previous kernel of the stream may still be
+// finishing (a quantise kernel of an earlier call reading these same
+// partial slots), and only the store waits for it.
+template <int DT, int G>
+__global__ void __launch_bounds__(256) amax_partial_kernel(const uint16_t* __restrict__ x,
+                                                           int64_t n_blocks, float* partial) {
+  __shared__ float red[8];
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
-  const int64_t wbase0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
   const int lane = threadIdx.x & 31;
-  for (int64_t base = wbase0; base < n_blocks; base += nthreads * kKPT) {
+  float a = 0.0f;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n_blocks;
+       base += nthreads * kKPT) {
     uint4 r[kKPT][2];
 #pragma unroll
     for (int k = 0; k < kKPT; ++k) load_raw(x, base + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+#pragma unroll
+    for (int k = 0; k < kKPT; ++k) {
+      float v[16];
+      unpack16<DT>(r[k][0], r[k][1], v);
+      if constexpr (G > 0) fwht_rows16<G>(v);
+      a = fmaxf(a, block_absmax(v));
+    }
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+  if (lane == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
+    pdl_wait();
+    partial[blockIdx.x] = a;
+  }
+  pdl_trigger();
+}
+
+// The tensor scale of a quantise kernel: given (read once the previous
+// kernel of the stream, which may have written it, is done), or g of the
+// largest of the n_partial maxima of amax_partial_kernel.
+__device__ __forceinline__ float quant_tensor_scale(const float* partial, int n_partial,
+                                                    const float* tensor_scale, int given) {
+  __shared__ float red[8];
+  pdl_wait();
+  if (given) return *tensor_scale;
+  float m = 0.0f;
+  for (int c = threadIdx.x; c < n_partial; c += blockDim.x) m = fmaxf(m, partial[c]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+  return tensor_scale_from_amax(__float_as_uint(m));
+}
+
+// ------------------------------------------------- row-blocked quantiser --
+// codes [rows, cols/2], scales [rows, cols/16] as flat arrays of blocks.
+// Programmatic dependent launch: the first blocks' loads are issued before
+// the wait for the previous kernel of the stream; everything it may have
+// written (the partial maxima, a given tensor scale, the outputs) is touched
+// after it.
+template <int DT, int G, bool SS>
+__global__ void __launch_bounds__(256) quant_rows_kernel(
+    const uint16_t* __restrict__ x, int64_t n_blocks, const float* partial, int n_partial,
+    float* tensor_scale, int scale_given, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int64_t wbase0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  const int lane = threadIdx.x & 31;
+  uint4 r[kKPT][2];
+#pragma unroll
+  for (int k = 0; k < kKPT; ++k) load_raw(x, wbase0 + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+  pdl_trigger();
+  const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
+  if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+  for (int64_t base = wbase0; base < n_blocks; base += nthreads * kKPT) {
+    if (base != wbase0) {
+#pragma unroll
+      for (int k = 0; k < kKPT; ++k)
+        load_raw(x, base + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+    }
 #pragma unroll
     for (int k = 0; k < kKPT; ++k) {
       const int64_t b = base + lane + k * nthreads;
@@ -124,139 +192,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   }
 }
 
-// ------------------------------------------- one-pass row quantiser --
-// The whole tensor in one launch when it fits in shared memory: every CTA
-// (one per SM, co-resident by a cooperative launch) stages its contiguous
-// chunk of blocks in pieces, takes the chunk absmax as the pieces land,
-// publishes it in its own slot of the workspace tagged with this launch's
-// grid identifier, waits until every CTA's slot carries that tag (bounded
-// wait), reduces the published maxima to the tensor absmax and quantises its
-// chunk from shared memory.  Same arithmetic as the two-pass path.
-// The grid identifier (%gridid) is unique per launch in the context, each
-// replay of a CUDA graph included, so slots written by earlier launches, or
-// any other contents of the workspace, never match: the workspace needs no
-// initial contents and nothing resets it.  A slot is 16 bytes: the tag (64
-// bits, written last with release semantics) and the CTA's maximum.  chunk
-// is a multiple of 32 blocks (rows stay whole for the Hadamard lanes, and
-// every lane of a warp runs the same number of iterations).
-constexpr int kOnePassThreads = 512;
-constexpr int kOnePassPieces = 4;
-
-__device__ __forceinline__ uint64_t grid_id() {
-  uint64_t g;
-  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
-  return g;
-}
-
-template <int DT, int G, bool SS>
-__global__ void __launch_bounds__(kOnePassThreads, 1) quant_onepass_kernel(
-    const uint16_t* __restrict__ x, int64_t n_blocks, int64_t chunk, uint8_t* slots,
-    float* tensor_scale, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  extern __shared__ uint4 cs[];  // chunk blocks x 32 bytes
-  __shared__ float red[32];
-  __shared__ int s_ok;
-  __shared__ __align__(8) uint64_t s_bar[kOnePassPieces];
-  const int64_t b0 = (int64_t)blockIdx.x * chunk;
-  const int64_t nvalid = b0 < n_blocks ? min(chunk, n_blocks - b0) : 0;
-  // pieces of whole warps' worth of blocks; the last may be short or empty
-  const int64_t pc = ((chunk / kOnePassPieces + 31) / 32) * 32;
-  const uint64_t gid = grid_id();
-  // blocks past the tensor end are zeros
-  for (int64_t i = nvalid + threadIdx.x; i < chunk; i += blockDim.x)
-    cs[2 * i] = cs[2 * i + 1] = make_uint4(0, 0, 0, 0);
-  if (threadIdx.x == 0) {
-    for (int p = 0; p < kOnePassPieces; ++p) mbar_init(&s_bar[p], 1);
-    fence_mbar_init();
-    for (int p = 0; p < kOnePassPieces; ++p) {
-      const int64_t lo = min(p * pc, nvalid), hi = min((p + 1) * pc, nvalid);
-      if (hi > lo) {
-        mbar_arrive_expect_tx(&s_bar[p], (uint32_t)((hi - lo) * 32));
-        bulk_g2s(cs + 2 * lo, x + (b0 + lo) * 16, (uint32_t)((hi - lo) * 32), &s_bar[p]);
-      } else {
-        mbar_arrive(&s_bar[p]);
-      }
-    }
-  }
-  __syncthreads();
-  float a = 0.0f;
-  bool ok = true;
-  for (int p = 0; p < kOnePassPieces && ok; ++p) {
-    int never = 0;
-    // one decision per warp: the Hadamard lanes exchange values in the loop
-    if (!__all_sync(0xffffffffu, mbar_wait(&s_bar[p], 0, &never))) {
-      ok = false;
-      break;
-    }
-    for (int64_t i = p * pc + threadIdx.x; i < min((p + 1) * pc, chunk); i += blockDim.x) {
-      float v[16];
-      unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
-      if constexpr (G > 0) fwht_rows16<G>(v);
-      a = fmaxf(a, block_absmax(v));
-    }
-  }
-  if (__syncthreads_or(!ok)) {
-    // timed out (status word set): give every copy a last bounded wait so
-    // that none lands after the CTA has left
-    if (threadIdx.x == 0)
-      for (int p = 0; p < kOnePassPieces; ++p) {
-        int again = 0;
-        mbar_wait(&s_bar[p], 0, &again, 200000000ull);
-      }
-    return;
-  }
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float c = 0.0f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c = fmaxf(c, red[w]);
-    uint8_t* my = slots + 16 * (int64_t)blockIdx.x;
-    *reinterpret_cast<volatile float*>(my + 8) = c;
-    store_release64(my, gid);
-    s_ok = 1;
-  }
-  __syncthreads();
-  // every CTA's maximum, one slot per thread (bounded wait on its tag)
-  float m = 0.0f;
-  for (int c = threadIdx.x; c < (int)gridDim.x; c += blockDim.x) {
-    const uint8_t* sl = slots + 16 * (int64_t)c;
-    if (!spin_until_eq64(sl, gid)) s_ok = 0;
-    m = fmaxf(m, *reinterpret_cast<const volatile float*>(sl + 8));
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (!s_ok) return;
-  float amax = 0.0f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
-  const float g = tensor_scale_from_amax(__float_as_uint(amax));
-  if (threadIdx.x == 0 && blockIdx.x == 0) *tensor_scale = g;
-  for (int64_t i = threadIdx.x; i < chunk; i += blockDim.x) {
-    const int64_t b = b0 + i;
-    float v[16];
-    unpack16<DT>(cs[2 * i], cs[2 * i + 1], v);
-    if constexpr (G > 0) fwht_rows16<G>(v);
-    if (b < n_blocks) {
-      uint32_t lo, hi;
-      const uint32_t S = quant_block16(v, g, SS, lo, hi);
-      *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
-      scales[b] = (uint8_t)S;
-    }
-  }
-}
-
 // ---------------------------------------------- column-blocked quantiser --
 // x [rows, cols]; 16-blocks along rows.  codes [cols, rows/2], scales
 // [cols, rows/16].  One thread per (row block, column); columns fastest.
 template <int DT, bool SS>
 __global__ void __launch_bounds__(256) quant_cols_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const uint32_t* amax_in,
-    float* tensor_scale, int scale_given, uint8_t* __restrict__ codes,
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const float* partial,
+    int n_partial, float* tensor_scale, int scale_given, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales) {
-  const float g = scale_given ? *tensor_scale : tensor_scale_from_amax(*amax_in);
+  pdl_trigger();
+  const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
   const int64_t n = (rows / 16) * cols;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;

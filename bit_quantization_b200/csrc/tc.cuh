@@ -94,28 +94,17 @@ __device__ __forceinline__ bool spin_until_geq(const unsigned* word, unsigned ta
   }
 }
 
-// Bounded spin until the 64-bit global word equals `tag` (acquire loads at
-// GPU scope, so what the writer stored before its release store of the tag
-// is visible after).  Gives up after `limit_ns` of wall time, sets the device
-// status word and returns false.
-__device__ __forceinline__ bool spin_until_eq64(const void* word, uint64_t tag,
-                                                uint64_t limit_ns = 2000000000ull) {
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    uint64_t v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
-    if (v == tag) return true;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      set_device_status(THRIFT_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// Release store of a 64-bit word at GPU scope: this thread's earlier writes
-// are visible to a thread that reads the word with acquire semantics.
-__device__ __forceinline__ void store_release64(void* word, uint64_t v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(word), "l"(v) : "memory");
+// Programmatic dependent launch.  pdl_wait: waits until the grid this one
+// depends on in its stream has completed and its memory operations are
+// visible (returns at once when there is none: a kernel launched without the
+// programmatic-serialisation attribute, or whose predecessor has finished);
+// it is the stream order itself, only moved inside the kernel.  pdl_trigger:
+// lets the next kernel of the stream that was launched with that attribute
+// be scheduled before this grid completes (it then waits in its own
+// pdl_wait for what it must not overtake).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------- bulk copies (TMA unit) --
@@ -280,6 +269,11 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
   }
 }
 
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(v));
+  tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -301,6 +295,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
         "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+  tmem_st32(taddr, *reinterpret_cast<const float(*)[32]>(v));
+  tmem_st32(taddr + 32, *reinterpret_cast<const float(*)[32]>(v + 32));
 }
 
 __device__ __forceinline__ void tmem_st_wait() {

@@ -128,72 +128,70 @@ void launch_amax(const void* x, int64_t n_blocks, int G, uint32_t* out, cudaStre
   else launch_amax_t<DT, 0>(xp, n_blocks, out, st);
 }
 
-template <int DT, int G, bool SS>
-void launch_quant_rows_t(const void* x, int64_t nb, uint32_t* amax, float* ts, int given,
-                         uint8_t* codes, uint8_t* scales, cudaStream_t st) {
-  quant_rows_kernel<DT, G, SS><<<stream_grid(quant_rows_kernel<DT, G, SS>, nb), kThreads, 0,
-                                 st>>>(static_cast<const uint16_t*>(x), nb, amax, ts, given,
-                                       codes, scales);
-}
-
-// Quantiser workspace: word 2 is the absmax of the two-pass path, and from
-// byte 256 one 16-byte slot per CTA of the one-pass kernel (its maximum,
-// tagged with the launch's grid identifier).  No call depends on the
-// workspace's earlier contents.
-constexpr size_t kQuantWsBytes = 4096;
-constexpr int kQuantMaxCtas = (int)((kQuantWsBytes - 256) / 16);
-constexpr int64_t kOnePassSmemMax = 200 * 1024;
-
-// The one-pass quantiser when the tensor fits in the SMs' shared memory;
-// returns false (nothing launched) when it does not or the cooperative
-// launch is refused.
-template <int DT, int G, bool SS>
-bool try_quant_onepass(const void* x, int64_t nb, uint32_t* ws, float* ts, uint8_t* codes,
-                       uint8_t* scales, cudaStream_t st) {
-  auto kern = quant_onepass_kernel<DT, G, SS>;
-  int grid = (int)std::min<int64_t>(std::min(sm_count(), kQuantMaxCtas), ceil_div(nb, 32));
-  const int64_t chunk = ceil_div(ceil_div(nb, (int64_t)grid), 32) * 32;
-  const int64_t smem = chunk * 32;
-  if (smem > kOnePassSmemMax) return false;
-  static DeviceSet attr;
-  if (!smem_attr(kern, kOnePassSmemMax, attr)) return false;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kOnePassThreads,
-                                                    (size_t)smem) != cudaSuccess ||
-      per_sm < 1)
-    return false;
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel of the stream finishes; it waits for it
+// (pdl_wait) before touching anything that kernel may write.
+template <class Kernel, class... Args>
+cudaError_t launch_pdl(Kernel kernel, int grid, int threads, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kOnePassThreads);
-  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeCooperative;
-  at[0].val.cooperative = 1;
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Quantiser workspace: from byte 256, the per-CTA maxima of the partial
+// absmax kernel (one float each).  Every call that computes the tensor scale
+// writes the slots it then reads, so no call depends on the workspace's
+// earlier contents.
+constexpr size_t kQuantWsBytes = 4096;
+constexpr int kQuantMaxPartials = (int)((kQuantWsBytes - 256) / 4);
+
+float* quant_partials(uint32_t* ws) {
+  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
+}
+
+// The partial absmax kernel over n_blocks 16-element blocks of x (rows
+// rotated when G > 0); returns its grid (the number of partial maxima).
+template <int DT, int G>
+int launch_amax_partial(const uint16_t* xp, int64_t nb, float* partial, cudaStream_t st,
+                        thrift_status* s) {
+  auto kern = amax_partial_kernel<DT, G>;
+  const int grid = std::min(kQuantMaxPartials, stream_grid(kern, nb));
+  *s = launch_pdl(kern, grid, kThreads, st, xp, nb, partial) == cudaSuccess ? THRIFT_OK
+                                                                             : THRIFT_ERR_CUDA;
+  return grid;
+}
+
+template <int DT, int G, bool SS>
+thrift_status quantize_rows(const void* x, int64_t nb, uint32_t* ws, float* ts, int given,
+                            uint8_t* codes, uint8_t* scales, cudaStream_t st) {
   const uint16_t* xp = static_cast<const uint16_t*>(x);
-  uint8_t* slots = reinterpret_cast<uint8_t*>(ws) + 256;
-  return cudaLaunchKernelEx(&cfg, kern, xp, nb, chunk, slots, ts, codes, scales) == cudaSuccess;
+  float* partial = quant_partials(ws);
+  int np = 0;
+  thrift_status s = THRIFT_OK;
+  if (!given) np = launch_amax_partial<DT, G>(xp, nb, partial, st, &s);
+  if (s != THRIFT_OK) return s;
+  auto kern = quant_rows_kernel<DT, G, SS>;
+  return launch_pdl(kern, stream_grid(kern, nb), kThreads, st, xp, nb,
+                    static_cast<const float*>(partial), np, ts, given, codes, scales) ==
+                 cudaSuccess
+             ? THRIFT_OK
+             : THRIFT_ERR_CUDA;
 }
 
 template <int DT>
 thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_t* ws,
                               float* ts, int given, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st) {
-  uint32_t* amax = ws + 2;
-#define THRIFT_QUANT_CASE(GG, SSV)                                                        \
-  if (G == GG && ss == SSV) {                                                              \
-    if (!given) {                                                                          \
-      if (try_quant_onepass<DT, GG, SSV>(x, nb, ws, ts, codes, scales, st))                \
-        return launch_status();                                                            \
-      (void)cudaGetLastError();                                                            \
-      if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;          \
-      launch_amax<DT>(x, nb, GG, amax, st);                                                \
-    }                                                                                      \
-    launch_quant_rows_t<DT, GG, SSV>(x, nb, amax, ts, given, codes, scales, st);           \
-    return launch_status();                                                                \
-  }
+#define THRIFT_QUANT_CASE(GG, SSV) \
+  if (G == GG && ss == SSV) return quantize_rows<DT, GG, SSV>(x, nb, ws, ts, given, codes, scales, st);
   THRIFT_QUANT_CASE(0, false)
   THRIFT_QUANT_CASE(0, true)
   THRIFT_QUANT_CASE(4, false)
@@ -409,6 +407,10 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   const double l2e = 1.4426950408889634;
   p.scale16 = (float)(l2e / std::sqrt((double)d));
   p.scale4 = (float)(l2e / std::sqrt((double)d) / (had ? (double)d : 1.0));
+  for (int m = 0; m < 8; ++m) {
+    p.log2_sf[m] = (float)std::log2(1.0 + m / 8.0);
+    p.log2_sf[8 + m] = m == 0 ? 0.0f : (float)(std::log2((double)m) - 2.0);
+  }
   if (d == 128 && blk == 128) return launch_attn_kernel<DT, 128, 128>(p, nTq, st);
   if (d == 128 && blk == 64) return launch_attn_kernel<DT, 128, 64>(p, nTq, st);
   if (d == 64 && blk == 128) return launch_attn_kernel<DT, 64, 128>(p, nTq, st);
@@ -865,35 +867,39 @@ thrift_status nvfp4_quantize_colblocks(const void* x, thrift_dtype dt, int64_t r
     return THRIFT_ERR_ARG;
   if ((rows * cols) % 16) return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* amax = static_cast<uint32_t*>(workspace) + 2;  // word 2: see launch_quantize
-  if (!tensor_scale_given) {
-    if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return THRIFT_ERR_CUDA;
-    if (dt == THRIFT_BF16) launch_amax<1>(x, rows * cols / 16, 0, amax, st);
-    else launch_amax<0>(x, rows * cols / 16, 0, amax, st);
-  }
   const uint16_t* xp = static_cast<const uint16_t*>(x);
+  float* partial = quant_partials(static_cast<uint32_t*>(workspace));
+  int np = 0;
+  thrift_status s = THRIFT_OK;
+  if (!tensor_scale_given) {
+    np = dt == THRIFT_BF16 ? launch_amax_partial<1, 0>(xp, rows * cols / 16, partial, st, &s)
+                           : launch_amax_partial<0, 0>(xp, rows * cols / 16, partial, st, &s);
+    if (s != THRIFT_OK) return s;
+  }
   // one thread per (row block, column): kKPT * threads items per CTA
   const int64_t items = (rows / 16) * cols * kKPT;
+  const float* pc = partial;
+  cudaError_t e;
   if (dt == THRIFT_BF16) {
     if (use_scalesearch)
-      quant_cols_kernel<1, true><<<stream_grid(quant_cols_kernel<1, true>, items), kThreads, 0,
-                                   st>>>(xp, rows, cols, amax, tensor_scale, tensor_scale_given,
-                                         codes, scales);
+      e = launch_pdl(quant_cols_kernel<1, true>, stream_grid(quant_cols_kernel<1, true>, items),
+                     kThreads, st, xp, rows, cols, pc, np, tensor_scale, tensor_scale_given, codes,
+                     scales);
     else
-      quant_cols_kernel<1, false><<<stream_grid(quant_cols_kernel<1, false>, items), kThreads,
-                                    0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                             tensor_scale_given, codes, scales);
+      e = launch_pdl(quant_cols_kernel<1, false>, stream_grid(quant_cols_kernel<1, false>, items),
+                     kThreads, st, xp, rows, cols, pc, np, tensor_scale, tensor_scale_given, codes,
+                     scales);
   } else {
     if (use_scalesearch)
-      quant_cols_kernel<0, true><<<stream_grid(quant_cols_kernel<0, true>, items), kThreads, 0,
-                                   st>>>(xp, rows, cols, amax, tensor_scale, tensor_scale_given,
-                                         codes, scales);
+      e = launch_pdl(quant_cols_kernel<0, true>, stream_grid(quant_cols_kernel<0, true>, items),
+                     kThreads, st, xp, rows, cols, pc, np, tensor_scale, tensor_scale_given, codes,
+                     scales);
     else
-      quant_cols_kernel<0, false><<<stream_grid(quant_cols_kernel<0, false>, items), kThreads,
-                                    0, st>>>(xp, rows, cols, amax, tensor_scale,
-                                             tensor_scale_given, codes, scales);
+      e = launch_pdl(quant_cols_kernel<0, false>, stream_grid(quant_cols_kernel<0, false>, items),
+                     kThreads, st, xp, rows, cols, pc, np, tensor_scale, tensor_scale_given, codes,
+                     scales);
   }
-  return launch_status();
+  return e == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
 size_t block_mean_topk_workspace_size(int B, int H, int Hkv, int N, int d, int blk) {

@@ -93,17 +93,23 @@ thrift_status thrift_stream_status(void* stream, int reset);
  *     transform first (cols must be 64 or 128).
  * Requirements: rows >= 0, cols % 16 == 0, cols <= 4096.
  * Workspace: nvfp4_quantize_workspace_size() bytes, 16-byte aligned, no
- *   initial contents required: the one-pass kernel's per-CTA maxima are
- *   tagged with the launch's grid identifier, so nothing from an earlier
- *   call (a timed-out one included) or any other contents can be taken for
- *   this call's; one buffer serves any number of calls issued in stream
- *   order.  Calls that overlap on the GPU must not share a workspace.
- *   nvfp4_quantize_colblocks takes the same workspace.
- * Execution: when the tensor scale is computed and the tensor fits in the
- *   SMs' shared memory (about 200 KB per SM), one cooperative launch stages
- *   it once, exchanges the per-CTA maxima with a bounded grid-wide wait and
- *   quantises from shared memory; otherwise an absmax pass and a quantise
- *   pass.  Both give the same bytes.
+ *   initial contents required (a call that computes the tensor scale writes
+ *   every per-CTA maximum it then reads); one buffer serves any number of
+ *   calls issued in stream order.  Calls that overlap on the GPU must not
+ *   share a workspace.  nvfp4_quantize_colblocks takes the same workspace.
+ * Execution: with the tensor scale computed, a partial-absmax kernel (one
+ *   maximum per CTA into the workspace) and a quantise kernel that reduces
+ *   those maxima to g and quantises (x read twice: from L2 the second time
+ *   when it fits); with the scale given, the quantise kernel alone.  Both are
+ *   launched with programmatic dependent launch: a kernel's first input loads
+ *   may run while the previous kernel of the stream finishes, and whatever
+ *   that kernel may write (the maxima, a given tensor scale, the outputs) is
+ *   touched only after it has completed.  Hence x must already be final when
+ *   the previous kernel of the stream lets its dependents start: x must not
+ *   alias a previous quantiser call's codes, scales or tensor scale, and a
+ *   predecessor that triggers its dependents early itself
+ *   (griddepcontrol.launch_dependents) must have written x before it does;
+ *   every other predecessor is waited for in full.
  */
 size_t nvfp4_quantize_workspace_size(void);
 thrift_status nvfp4_quantize(const void* x, thrift_dtype dt, int64_t rows, int64_t cols,
