@@ -51,10 +51,6 @@ struct AttnParams {
   float scale4;            // log2(e)/sqrt(d), divided by d with the rotation
   float scale16;           // log2(e)/sqrt(d)
   const float* corr;       // K smoothing: q^ . mu per query row [nseq, H, nTq * 128], or null
-  // log2 of the UE4M3 mantissa factors: [m] = log2(1 + m/8) (normal bytes),
-  // [8 + m] = log2(m) - 2 (subnormal bytes), so that log2(value(S)) =
-  // (S >> 3) - 7 + log2_sf[...] exactly to fp32 rounding
-  float log2_sf[16];
 };
 
 template <int D, int BLK>
@@ -193,38 +189,6 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
-// 2^x for two values on the FMA pipe (no MUFU).  Range reduction x = n + f,
-// n = round(x) by adding and subtracting 1.5 * 2^23 (f in [-1/2, 1/2],
-// exact); 2^f by the quartic of bit_quantization_b200/fit_exp2.py, which
-// interpolates 2^f exactly at the fractional positions where 2^x crosses an
-// E2M1 rounding midpoint (so the E2M1 codes of its results are those of the
-// exact exponential up to fp32 evaluation rounding) and stays within
-// 1.5e-5 relative elsewhere; 2^n added to the exponent field.  x is clamped
-// at -126 first (2^-126 and below are zero for every code and sum here).
-constexpr float kExp2C1 = 0.6931387f, kExp2C2 = 0.24022177f, kExp2C3 = 0.055751342f,
-                kExp2C4 = 0.009595151f;
-
-__device__ __forceinline__ void exp2_fma2(float& x0, float& x1) {
-  constexpr float M = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
-  float j0, j1, n0, n1, f0, f1, p0, p1;
-  add2(j0, j1, x0, x1, M, M);                       // M + round(x)
-  add2(n0, n1, j0, j1, -M, -M);                     // round(x)
-  fma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);       // f = x - round(x), exact
-  fma2(p0, p1, kExp2C4, kExp2C4, f0, f1, kExp2C3, kExp2C3);
-  fma2(p0, p1, p0, p1, f0, f1, kExp2C2, kExp2C2);
-  fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-  fma2(p0, p1, p0, p1, f0, f1, 1.0f, 1.0f);
-  // the low bits of M + round(x) hold round(x): shifted into the exponent
-  x0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
-  x1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
-}
-
-// Probabilities of each 16-key block of an NVFP4 tile taken on the FMA pipe
-// by exp2_fma2 (the others by the MUFU's ex2): the two pipes share the work.
-constexpr int kPolyPerBlock = 4;
-
 // Eight fp32 values -> eight E2M1 codes packed in 32 bits (value 2i in the
 // low nibble of byte i), round to nearest even, saturating.
 __device__ __forceinline__ uint32_t e2m1x8(const float* x) {
@@ -275,7 +239,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
   int* s_n = reinterpret_cast<int*>(sm + L::OFF_BAR + 8 * B_N + 4);
   int* s_n4 = s_n + 1;
   volatile int* s_abort = s_n + 2;
-  float* s_lg = reinterpret_cast<float*>(sm + L::OFF_BAR + 8 * B_N + 32);  // [16]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
@@ -302,7 +265,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     *s_abort = 0;
     fence_mbar_init();
   }
-  if (tid < 16) s_lg[tid] = p.log2_sf[tid];
   if (warp == 0) {
     // Tile list: NVFP4 tiles ascending, then FP16 tiles ascending.  Entry:
     // key tile j (bits 0..12), bit 13 + b set when query block b of this CTA
@@ -800,11 +762,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           const float e = ex2_ftz(fmaf(bm[b], cs, -mt));  // block max / tile max
           const uint32_t S = live ? ue4m3(448.0f * e) : 0u;
           dec[b] = ue4m3_decode_fast(S);
-          // log2(2688) - mt - log2(value(S)), the last from the exponent
-          // field and the mantissa table (exact to fp32 rounding, no MUFU)
-          const uint32_t ex = S >> 3;
-          const float l2s = (float)((int)ex - 7) + s_lg[(ex == 0 ? 8u : 0u) + (S & 7u)];
-          cc[b] = S ? (11.392317422778760f - mt) - l2s : -INFINITY;
+          cc[b] = S ? 11.392317422778760f - mt - lg2_ftz(dec[b]) : -INFINITY;  // log2(2688)
           sfw |= S << (8 * b);
         }
         if (!warp_wait(&bars[B_TURN + g], u & 1, s_abort)) { ok = false; break; }
@@ -833,9 +791,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             for (int i = 0; i < 16; i += 2)
               fma2(x[i], x[i + 1], x[i], x[i + 1], cs, cs, cc[b], cc[b]);
 #pragma unroll
-            for (int i = 0; i < kPolyPerBlock; i += 2) exp2_fma2(x[i], x[i + 1]);
-#pragma unroll
-            for (int i = kPolyPerBlock; i < 16; ++i) x[i] = ex2_ftz(x[i]);  // masked (-inf) -> 0
+            for (int i = 0; i < 16; ++i) x[i] = ex2_ftz(x[i]);  // masked (-inf) -> 0
             float y[8];
 #pragma unroll
             for (int i = 0; i < 8; i += 2)

@@ -269,11 +269,6 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
   }
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(v));
-  tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -295,11 +290,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
         "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
-}
-
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
-  tmem_st32(taddr, *reinterpret_cast<const float(*)[32]>(v));
-  tmem_st32(taddr + 32, *reinterpret_cast<const float(*)[32]>(v + 32));
 }
 
 __device__ __forceinline__ void tmem_st_wait() {

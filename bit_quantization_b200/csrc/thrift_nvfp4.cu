@@ -407,10 +407,6 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   const double l2e = 1.4426950408889634;
   p.scale16 = (float)(l2e / std::sqrt((double)d));
   p.scale4 = (float)(l2e / std::sqrt((double)d) / (had ? (double)d : 1.0));
-  for (int m = 0; m < 8; ++m) {
-    p.log2_sf[m] = (float)std::log2(1.0 + m / 8.0);
-    p.log2_sf[8 + m] = m == 0 ? 0.0f : (float)(std::log2((double)m) - 2.0);
-  }
   if (d == 128 && blk == 128) return launch_attn_kernel<DT, 128, 128>(p, nTq, st);
   if (d == 128 && blk == 64) return launch_attn_kernel<DT, 128, 64>(p, nTq, st);
   if (d == 64 && blk == 128) return launch_attn_kernel<DT, 64, 128>(p, nTq, st);

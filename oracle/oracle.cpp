@@ -614,16 +614,13 @@ static inline double deq(uint8_t code, uint8_t sc, float g) {
 //     of the argument (log2 2688 - log2 S_b, the log2 approximation adding at
 //     most 2^-22 per unit of its result) and the fused argument itself:
 //     2^-22 (|S|max + |m| + 24), 24 bounding |log2 2688| + |log2 S_b| <= 20.4;
-// plus, relative, the exponential itself (the hardware exp2 approximation,
-// 2 ulp = 2^-22, or a polynomial on the FMA pipe that interpolates 2^x at
-// the E2M1 rounding midpoints, exact there up to its fp32 evaluation: 2^-21
-// covers both) and this emulation's own fp32 chain (P, 1/rowmax, P/rowmax,
-// 1/S_b, t: five roundings of 2^-24):
-//   rho = ln 2 (2 d 2^-23 A + 2^-22 (|S|max + |m| + 24)) + 2^-21 + 5 2^-24.
+// plus, relative, the exp2 approximation (2 ulp, 2^-22) and this emulation's
+// own fp32 chain (P, 1/rowmax, P/rowmax, 1/S_b, t: five roundings of 2^-24):
+//   rho = ln 2 (2 d 2^-23 A + 2^-22 (|S|max + |m| + 24)) + 2^-22 + 5 2^-24.
 static double tile_radius(int d, double A, double smax_abs, double m_abs) {
   const double u23 = std::ldexp(1.0, -23), u22 = std::ldexp(1.0, -22);
   const double dx = 2.0 * d * u23 * A + u22 * (smax_abs + m_abs + 24.0);
-  return 0.6931471805599453 * dx + std::ldexp(1.0, -21) + 5.0 * std::ldexp(1.0, -24);
+  return 0.6931471805599453 * dx + u22 + 5.0 * std::ldexp(1.0, -24);
 }
 
 // Every rounding below is monotone, so the roundings a value x can take
