@@ -170,6 +170,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   pdl_trigger();
   const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+  __shared__ float rtab[128];
+  build_rcp_table(rtab, g);
+  __syncthreads();
   for (int64_t base = wbase0; base < n_blocks; base += nthreads * kKPT) {
     if (base != wbase0) {
 #pragma unroll
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
       if constexpr (G > 0) fwht_rows16<G>(v);
       if (b < n_blocks) {
         uint32_t lo, hi;
-        const uint32_t S = quant_block16(v, g, SS, lo, hi);
+        const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
         *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
         scales[b] = (uint8_t)S;
       }
@@ -203,6 +206,9 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
   pdl_trigger();
   const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+  __shared__ float rtab[128];
+  build_rcp_table(rtab, g);
+  __syncthreads();
   const int64_t n = (rows / 16) * cols;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -211,7 +217,7 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
 #pragma unroll
     for (int e = 0; e < 16; ++e) v[e] = h2f<DT>(__ldg(x + (rb * 16 + e) * cols + c));
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(v, g, SS, lo, hi);
+    const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
     *reinterpret_cast<uint2*>(codes + c * (rows / 2) + rb * 8) = make_uint2(lo, hi);
     scales[c * (rows / 16) + rb] = (uint8_t)S;
   }
@@ -290,6 +296,9 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
                        min(tile_rows, len - t0), tile_rows, D * 2, &s_bar))
     return;
   const float g = tensor_scale_from_amax(*amax_in);
+  __shared__ float rtab[128];
+  build_rcp_table(rtab, g);
+  __syncthreads();
   const uint32_t t4 = fp4_tile_bytes(tile_rows, D), t16 = f16_tile_bytes(tile_rows, D);
   const int64_t tidx = ((int64_t)seq * nh + head) * ntiles + tile;
   uint8_t* t4p = img4 + tidx * t4;
@@ -315,7 +324,7 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
     }
     if constexpr (HAD) fwht_rows16<G>(v);
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(v, g, SS, lo, hi);
+    const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
     if (mrow && corr) {
       // q^ . mu over the row: this block's part, then the G lanes of the row
       float part = 0.0f;
@@ -438,6 +447,9 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
                        min(blk, len - t0), blk, d * 2, &s_bar))
     return;
   const float g = tensor_scale_from_amax(*amax_in);
+  __shared__ float rtab[128];
+  build_rcp_table(rtab, g);
+  __syncthreads();
   const uint32_t t4 = fp4_tile_bytes(d, blk), t16 = f16_tile_bytes(d, blk);
   const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
   // the two output images are assembled in shared memory (transposed rows
@@ -456,7 +468,7 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
       val[e] = h2f<DT>(raw[e]);
     }
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(val, g, SS, lo, hi);
+    const uint32_t S = quant_block16(val, g, SS, lo, hi, rtab);
     *reinterpret_cast<uint2*>(o4 + swz_offset(c, kb / 2, blk / 2)) = make_uint2(lo, hi);
     sf[sf_offset(c, kb / 16)] = (uint8_t)S;
     if (d == 64) sf[sf_offset(c + 64, kb / 16)] = 0;
