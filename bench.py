@@ -85,8 +85,8 @@ def _src_sha(name):
 # DRAM traffic of one attention launch measured by ncu (read + write bytes)
 # for the attention source with this hash; reported only while the source is
 # unchanged since the capture.
-ATTN_TRAFFIC = {"src_sha16": "aed717716c579cc9", "workload": "b2h32n8192d128_bf16_noncausal_top10",
-                "bytes": 396740352 + 123007744}
+ATTN_TRAFFIC = {"src_sha16": "abe4ba02cd17350b", "workload": "b2h32n8192d128_bf16_noncausal_top10",
+                "bytes": 395558144 + 121920256}
 
 
 def attn_traffic(w):
@@ -969,11 +969,15 @@ def main():
                          "(profiling aid)")
     ap.add_argument("--decode-context", type=int, default=None,
                     help="cached tokens per sequence in --mode decode (default: the workload's)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="tokens per sequence of a fixed-length workload (profiling a smaller case)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-qat", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
+    if args.seq_len is not None and w.varlen is None:
+        w = dataclasses.replace(w, N=args.seq_len, name=f"{w.name}_n{args.seq_len}")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.mode == "quantizer":

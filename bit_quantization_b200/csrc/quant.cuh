@@ -54,9 +54,10 @@ __device__ __forceinline__ void e2m1x2_values(uint32_t byte, float& v0, float& v
       : "r"(byte));
 }
 
-// Block error of candidate byte S with value sv and r = 1/(sv g)
-// correctly rounded (see header comment).
-__device__ __forceinline__ double block_err_r(const float (&x)[16], float sv, float r) {
+// Block error of candidate byte S (see header comment).
+__device__ __forceinline__ double block_err(const float (&x)[16], float g, uint32_t S) {
+  const float sv = ue4m3_decode(S);
+  const float r = __frcp_rn(__fmul_rn(sv, g));
   float acc = 0.0f;
 #pragma unroll
   for (int e = 0; e < 16; e += 2) {
@@ -71,26 +72,10 @@ __device__ __forceinline__ double block_err_r(const float (&x)[16], float sv, fl
   return __dmul_rn((double)acc, __dmul_rn(s, s));
 }
 
-__device__ __forceinline__ double block_err(const float (&x)[16], float g, uint32_t S) {
-  const float sv = ue4m3_decode(S);
-  return block_err_r(x, sv, __frcp_rn(__fmul_rn(sv, g)));
-}
-
-// rtab[S] = 1/(value(S) g), correctly rounded, for every UE4M3 byte S
-// (entry 0 unused): the same reciprocals the quantiser would compute per
-// block and candidate, once per CTA.  Call with all threads; the caller
-// synchronises before use.
-__device__ __forceinline__ void build_rcp_table(float* rtab, float g) {
-  for (int b = threadIdx.x; b < 128; b += blockDim.x)
-    rtab[b] = (b == 0 || b == 127) ? 0.0f : __frcp_rn(__fmul_rn(ue4m3_decode((uint32_t)b), g));
-}
-
 // Quantises one 16-element block.  Returns the scale byte; codes in
 // lo (elements 0..7) and hi (elements 8..15), element 2c in the low nibble.
-// rtab (optional): the reciprocal table of build_rcp_table for this g.
 __device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], float g, bool ss,
-                                                  uint32_t& lo, uint32_t& hi,
-                                                  const float* rtab = nullptr) {
+                                                  uint32_t& lo, uint32_t& hi) {
   float amax = 0.0f;
 #pragma unroll
   for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
@@ -110,9 +95,7 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], float g,
       const int f = oi == 0 ? 0 : (oi <= 2 ? oi - 3 : oi - 2);
       const int b = (int)S + f;
       if (b >= 1 && b <= 126) {
-        const float sv = ue4m3_decode((uint32_t)b);
-        const double err =
-            block_err_r(x, sv, rtab ? rtab[b] : __frcp_rn(__fmul_rn(sv, g)));
+        const double err = block_err(x, g, (uint32_t)b);
         if (!have || err < best) {
           best = err;
           best_f = f;
@@ -122,7 +105,7 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], float g,
     }
     S = (uint32_t)((int)S + best_f);
   }
-  const float r = rtab ? rtab[S] : __frcp_rn(__fmul_rn(ue4m3_decode(S), g));
+  const float r = __frcp_rn(__fmul_rn(ue4m3_decode(S), g));
   uint32_t c[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) c[i] = e2m1x2(__fmul_rn(x[2 * i], r), __fmul_rn(x[2 * i + 1], r));

@@ -156,38 +156,39 @@ __device__ __forceinline__ float quant_tensor_scale(const float* partial, int n_
 // the wait for the previous kernel of the stream; everything it may have
 // written (the partial maxima, a given tensor scale, the outputs) is touched
 // after it.
+// Blocks in flight per thread in the quantise kernel: two, so that four
+// CTAs of 256 threads fit an SM (64 registers a thread).
+constexpr int kQuantKPT = 2;
+
 template <int DT, int G, bool SS>
-__global__ void __launch_bounds__(256) quant_rows_kernel(
+__global__ void __launch_bounds__(256, 4) quant_rows_kernel(
     const uint16_t* __restrict__ x, int64_t n_blocks, const float* partial, int n_partial,
     float* tensor_scale, int scale_given, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales) {
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
   const int64_t wbase0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
   const int lane = threadIdx.x & 31;
-  uint4 r[kKPT][2];
+  uint4 r[kQuantKPT][2];
 #pragma unroll
-  for (int k = 0; k < kKPT; ++k) load_raw(x, wbase0 + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
+  for (int k = 0; k < kQuantKPT; ++k) load_raw(x, wbase0 + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
   pdl_trigger();
   const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-  __shared__ float rtab[128];
-  build_rcp_table(rtab, g);
-  __syncthreads();
-  for (int64_t base = wbase0; base < n_blocks; base += nthreads * kKPT) {
+  for (int64_t base = wbase0; base < n_blocks; base += nthreads * kQuantKPT) {
     if (base != wbase0) {
 #pragma unroll
-      for (int k = 0; k < kKPT; ++k)
+      for (int k = 0; k < kQuantKPT; ++k)
         load_raw(x, base + lane + k * nthreads, n_blocks, r[k][0], r[k][1]);
     }
 #pragma unroll
-    for (int k = 0; k < kKPT; ++k) {
+    for (int k = 0; k < kQuantKPT; ++k) {
       const int64_t b = base + lane + k * nthreads;
       float v[16];
       unpack16<DT>(r[k][0], r[k][1], v);
       if constexpr (G > 0) fwht_rows16<G>(v);
       if (b < n_blocks) {
         uint32_t lo, hi;
-        const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
+        const uint32_t S = quant_block16(v, g, SS, lo, hi);
         *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
         scales[b] = (uint8_t)S;
       }
@@ -206,9 +207,6 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
   pdl_trigger();
   const float g = quant_tensor_scale(partial, n_partial, tensor_scale, scale_given);
   if (!scale_given && blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-  __shared__ float rtab[128];
-  build_rcp_table(rtab, g);
-  __syncthreads();
   const int64_t n = (rows / 16) * cols;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -217,7 +215,7 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
 #pragma unroll
     for (int e = 0; e < 16; ++e) v[e] = h2f<DT>(__ldg(x + (rb * 16 + e) * cols + c));
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
+    const uint32_t S = quant_block16(v, g, SS, lo, hi);
     *reinterpret_cast<uint2*>(codes + c * (rows / 2) + rb * 8) = make_uint2(lo, hi);
     scales[c * (rows / 16) + rb] = (uint8_t)S;
   }
@@ -296,9 +294,6 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
                        min(tile_rows, len - t0), tile_rows, D * 2, &s_bar))
     return;
   const float g = tensor_scale_from_amax(*amax_in);
-  __shared__ float rtab[128];
-  build_rcp_table(rtab, g);
-  __syncthreads();
   const uint32_t t4 = fp4_tile_bytes(tile_rows, D), t16 = f16_tile_bytes(tile_rows, D);
   const int64_t tidx = ((int64_t)seq * nh + head) * ntiles + tile;
   uint8_t* t4p = img4 + tidx * t4;
@@ -324,7 +319,7 @@ __global__ void __launch_bounds__(256) qk_tile_kernel(
     }
     if constexpr (HAD) fwht_rows16<G>(v);
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(v, g, SS, lo, hi, rtab);
+    const uint32_t S = quant_block16(v, g, SS, lo, hi);
     if (mrow && corr) {
       // q^ . mu over the row: this block's part, then the G lanes of the row
       float part = 0.0f;
@@ -447,9 +442,6 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
                        min(blk, len - t0), blk, d * 2, &s_bar))
     return;
   const float g = tensor_scale_from_amax(*amax_in);
-  __shared__ float rtab[128];
-  build_rcp_table(rtab, g);
-  __syncthreads();
   const uint32_t t4 = fp4_tile_bytes(d, blk), t16 = f16_tile_bytes(d, blk);
   const int64_t tidx = ((int64_t)seq * Hkv + hk) * ntiles + j;
   // the two output images are assembled in shared memory (transposed rows
@@ -468,7 +460,7 @@ __global__ void __launch_bounds__(256) v_tile_kernel(
       val[e] = h2f<DT>(raw[e]);
     }
     uint32_t lo, hi;
-    const uint32_t S = quant_block16(val, g, SS, lo, hi, rtab);
+    const uint32_t S = quant_block16(val, g, SS, lo, hi);
     *reinterpret_cast<uint2*>(o4 + swz_offset(c, kb / 2, blk / 2)) = make_uint2(lo, hi);
     sf[sf_offset(c, kb / 16)] = (uint8_t)S;
     if (d == 64) sf[sf_offset(c + 64, kb / 16)] = 0;

@@ -96,7 +96,7 @@ int sm_count() {
 // per thread, capped at one full wave (resident CTAs per SM x SMs) so that no
 // partial second wave trails the launch.
 template <class Kernel>
-int stream_grid(Kernel kernel, int64_t n_blocks) {
+int stream_grid(Kernel kernel, int64_t n_blocks, int kpt = kKPT) {
   static std::atomic<int> per_dev[kMaxDevices] = {};  // per kernel instantiation
   const int dev = current_device();
   int resident = dev < 0 ? 0 : per_dev[dev].load();
@@ -108,7 +108,7 @@ int stream_grid(Kernel kernel, int64_t n_blocks) {
     resident = per_sm * sm_count();
     if (dev >= 0) per_dev[dev].store(resident);
   }
-  int64_t g = ceil_div(n_blocks, (int64_t)kThreads * kKPT);
+  int64_t g = ceil_div(n_blocks, (int64_t)kThreads * kpt);
   if (g < 1) g = 1;
   if (g > resident) g = resident;
   return (int)g;
@@ -179,7 +179,7 @@ thrift_status quantize_rows(const void* x, int64_t nb, uint32_t* ws, float* ts, 
   if (!given) np = launch_amax_partial<DT, G>(xp, nb, partial, st, &s);
   if (s != THRIFT_OK) return s;
   auto kern = quant_rows_kernel<DT, G, SS>;
-  return launch_pdl(kern, stream_grid(kern, nb), kThreads, st, xp, nb,
+  return launch_pdl(kern, stream_grid(kern, nb, kQuantKPT), kThreads, st, xp, nb,
                     static_cast<const float*>(partial), np, ts, given, codes, scales) ==
                  cudaSuccess
              ? THRIFT_OK
