@@ -319,14 +319,16 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
   uint8_t* mk = mask + ((int64_t)seq * H + h) * npairs;
   const int64_t n_valid = causal ? (int64_t)nb * (nb + 1) / 2 : (int64_t)nb * nb;
   const int64_t k = topk_count_dev(frac, n_valid);
+  // pair indices fit 32 bits (nB <= 512): a 32-bit division, not the
+  // software-emulated 64-bit one
   auto valid = [&](int64_t lin) {
-    const int i = (int)(lin / nB), j = (int)(lin % nB);
+    const int l = (int)lin, i = l / nB, j = l - i * nB;
     return i < nb && j < nb && (!causal || j <= i);
   };
   // ScaleSearchAttention's sink-aware pairs, added to the top-k ones: the
   // first `sink` key blocks and the `recent` newest ones query block i sees
   auto fixed = [&](int64_t lin) {
-    const int i = (int)(lin / nB), j = (int)(lin % nB);
+    const int l = (int)lin, i = l / nB, j = l - i * nB;
     return j < sink || (causal ? (j > i - recent) : (j >= nb - recent));
   };
   auto score = [&](int64_t lin) { return sc[lin]; };
