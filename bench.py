@@ -588,8 +588,8 @@ def qat_setup(ops, dev, w):
     inp = synth.make_qat_inputs(w, device=dev)
     q, k, v, dout = (inp[n] for n in ("q", "k", "v", "dout"))
     cu = inp["cu_seqlens"].to(dev)
-    ws = torch.empty(ops.qat_workspace_size(q.shape[0], w.H, w.Hkv, w.d), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(ops.qat_workspace_size(q.shape[0], w.H, w.Hkv, w.d, cu.numel() - 1),
+                     dtype=torch.uint8, device=dev)
     return inp, q, k, v, dout, cu, ws
 
 
@@ -669,8 +669,9 @@ def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
                                       f"timed region is tens of milliseconds)",
                          "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                          "executed_mma_flops": 14 * 2 * pairs * w.d,
-                         "note": "7 algorithmic products; the kernels execute 14 (S recomputed "
-                                 "in each pass, dS and the P of O' as two 16-bit parts)"},
+                         "note": "7 algorithmic products; the kernels execute 14 (the forward "
+                                 "computes S in both of its passes, each gradient kernel S and "
+                                 "dP again; dS and the P of O' enter as two 16-bit parts)"},
             "kernels_per_step": QAT_KERNELS_PER_STEP, "steps": steps}
     if not args.no_cpu_baseline:
         # the oracle on a causal prefix of kv head 0 with its query heads: a

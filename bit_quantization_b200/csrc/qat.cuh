@@ -1,5 +1,6 @@
 // Attn-QAT attention: forward on fake-quantised NVFP4 operands and the
-// backward with FP4 recomputation of the probabilities.
+// backward with FP4 recomputation of the probabilities, on the Blackwell
+// tensor cores (tcgen05 kind::f16, fp32 accumulators in tensor memory).
 //
 // Source: "Attn-QAT: 4-Bit Attention With Quantization-Aware Training",
 // Metodologia (1: the backward recomputes the probabilities at the forward's
@@ -18,51 +19,105 @@
 //   dQ = dS K^ / sqrt(d),  dK = dS^T Q^ / sqrt(d)
 //   (dK, dV summed over the query heads of a kv head)
 //
-// Design.  Memory-bound kernels write the fake-quantised images once: each
-// element is E2M1 value x UE4M3 block scale, exact in the 16-bit input type,
-// with the tensor scales applied to the fp32 accumulators instead.  The
-// three attention kernels run warp-level m16n8k16 MMAs (fp32 accumulate) on
-// those images; P^ enters the MMAs rounded to the 16-bit type, dS and the P
-// of O' as sums of two 16-bit parts.  Operand tiles are staged by cp.async
-// with the next tile in flight; B operands that run along the rows of a
-// staged tile are transposed by ldmatrix.
-//   qat_fwd_kernel     per 128-query tile, one pass over the key tiles:
-//                      running max, P, its FP4 image, O, O', lse
-//   qat_rowdot_kernel  D = rowsum(dO o O')
-//   qat_bwd_kv_kernel  per key tile of blk keys, over every 64-query chunk
-//                      of the kv head's query heads: S^T, P^T, its FP4
-//                      image, dP^T, dS^T; dV += (P^)^T dO, dK += dS^T Q^
-//   qat_bwd_q_kernel   per 64-query tile: S, P, dP, dS; dQ += dS K^
+// Operand tiles.  Every 16-bit operand lives in HBM as tiles of 128 rows:
+// D / 64 regions of [128 rows][128 B] with the 128-byte swizzle, element
+// (r, c) at (c / 64) * 16384 + swizzle(r, 2 (c % 64)).  A tile is a K-major
+// operand when its rows are the M or N dimension of a product and an
+// MN-major one when its rows run along the contraction, so no transposed
+// copy is ever made: O = P^ V^ and dQ = dS K^ read V^ and K^ MN-major,
+// dV = P^T dO and dK = dS^T Q^ read both operands MN-major.  The tiles of a
+// sequence s that starts at token st are slots st / 128 + s + t
+// (t < ceil(len / 128)) of its head; nslot = total / 128 + nseq bounds them.
+// The fake-quantised elements (E2M1 value x UE4M3 block scale) are exact in
+// the 16-bit input type; the tensor scales multiply the fp32 accumulators.
+// P^ enters the products rounded to the 16-bit type, P (of O') and dS as
+// two 16-bit parts, hi = round(x) and lo = round(x - hi): rows of dS sum to
+// zero, and one rounding would leave a residue that the products with K^ or
+// Q^ (whose channel means can be large) magnify.
+//
+// Kernels.
+//   qat_fq_tile_kernel      Q, K (blocks along d) or V (blocks along the
+//                           tokens) -> fake-quantised tiles, one 128-row
+//                           tile per CTA staged in shared memory
+//   qat_rowdot_tile_kernel  D = rowsum(dO o O') and the dO tiles
+//   qat_fwd_kernel          per 128 query rows: pass A over the key tiles
+//                           for the row maxima (S only), pass B for P, P^,
+//                           O = P^ V^ and O' = P V^ against the final
+//                           maxima (no rescaling of the accumulators), lse
+//   qat_bwd_q_kernel        per 128 query rows: S, dP, dS; dQ += dS K^
+//   qat_bwd_kv_kernel       per 128-key tile over the 128-row query chunks
+//                           of its query heads: S, dP, P, P^, dS;
+//                           dV += P^T dO, dK += dS^T Q^
+// The three attention kernels have ten warps: warps 0-7 own the rows (two
+// per tensor-memory lane quarter, each taking half of the 128 columns of
+// a score tile), warp 8 moves tiles with bulk copies, warp 9 issues the MMAs
+// from one thread.  Every wait is bounded.
 #pragma once
-#include "quant_kernels.cuh"
+#include "attn.cuh"
 
 namespace thrift {
 
-constexpr int kQatFwdRows = 128;  // query rows of a forward CTA (8 warps x 16)
-constexpr int kQatRows = 64;   // query rows of a dQ CTA (4 warps x 16)
-constexpr int kQatChunk = 64;  // query chunk of the key-tile kernel, key chunk of the dQ kernel
 constexpr float kQatLog2e = 1.4426950408889634f;
 constexpr float kQatLn2 = 0.6931471805599453f;
 
+constexpr int kQtWarps = 8;             // row-owning warps, two per lane quarter
+constexpr int kQtProducer = kQtWarps;   // warp 8
+constexpr int kQtMma = kQtWarps + 1;    // warp 9
+constexpr int kQtThreads = 32 * (kQtWarps + 2);
+constexpr uint32_t kQtPTile = 128u * 128u * 2u;  // [128][128] 16-bit
+constexpr uint32_t kQtShBytes = 2048;            // barriers, flags, tables
+
+__host__ __device__ constexpr uint32_t qt_tile_bytes(int d) { return 128u * (uint32_t)d * 2u; }
+__host__ __device__ constexpr int64_t qat_nslot(int64_t total, int nseq) {
+  return total / 128 + nseq;
+}
+
 struct QatParams {
-  const uint16_t* qi;  // fake-quantised images [total, H|Hkv, D] in the input type
-  const uint16_t* ki;
-  const uint16_t* vi;
-  const uint16_t* dout;  // [total, H, D] (backward)
-  const float* g;        // tensor scales of Q, K, V
+  const uint8_t* qt;   // fake-quantised tiles: Q [H][nslot], K, V [Hkv][nslot]
+  const uint8_t* kt;
+  const uint8_t* vt;
+  const uint8_t* dot;  // dO tiles [H][nslot] (backward)
+  int64_t nslot;
+  const float* g;      // tensor scales of Q, K, V
   SeqInfo si;
   int H, Hkv;
   int64_t total;
   int causal;
-  float sc;          // 1 / sqrt(d)
-  uint16_t* out;     // forward: O [total, H, D] in the input type
-  float* out_hp;     // forward: O' [total, H, D]; backward: read
-  float* lse;        // [H, total], natural log
-  const float* dsum; // D [H, total]
-  float* dq;         // [total, H, D]
-  float* dk;         // [total, Hkv, D]
+  float sc;            // 1 / sqrt(d)
+  uint16_t* out;       // forward: O [total, H, D] in the input type
+  float* out_hp;       // forward: O' [total, H, D]
+  float* lse;          // [H, total], natural log
+  const float* dsum;   // D [H, total]
+  float* dq;           // [total, H, D]
+  float* dk;           // [total, Hkv, D]
   float* dv;
 };
+
+__device__ __forceinline__ int64_t qat_slot(int hd, int64_t nslot, int64_t st, int seq, int t) {
+  return (int64_t)hd * nslot + st / 128 + seq + t;
+}
+
+// Byte offset of element (r, c) of a 128-row tile.
+__device__ __forceinline__ uint32_t qt_elem(int r, int c) {
+  return (uint32_t)(c >> 6) * 16384u + swz_offset((uint32_t)r, (uint32_t)(c & 63) * 2u, 128);
+}
+
+// K-major operand of a 128-row tile, K-step s (16 elements along the row):
+// 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t qt_desc_k(uint32_t tile, int s) {
+  return make_sdesc(tile + (uint32_t)(s >> 2) * 16384u + 32u * (uint32_t)(s & 3), 16, 1024,
+                    SW_128B);
+}
+
+// MN-major operand of a 128-row tile whose rows run along the contraction:
+// K-step s takes rows 16s..16s+15; the 64-element groups along M or N are
+// 16384 bytes apart (leading offset), the 8-row groups along K 1024
+// (stride offset).
+__device__ __forceinline__ uint64_t qt_desc_mn(uint32_t tile, int s) {
+  return make_sdesc(tile + (uint32_t)s * 2048u, 16384, 1024, SW_128B);
+}
+
+constexpr uint32_t kIdescAmn = 1u << 15, kIdescBmn = 1u << 16;
 
 // ------------------------------------------------------- fake quantisers --
 
@@ -75,185 +130,108 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t byte, float sv) {
   return (uint32_t)f2h<DT>(__fmul_rn(v0, sv)) | ((uint32_t)f2h<DT>(__fmul_rn(v1, sv)) << 16);
 }
 
-// Rows blocked along the contiguous axis (Q, K): n_blocks blocks of 16.
-template <int DT, bool SS>
-__global__ void __launch_bounds__(256) qat_fq_rows_kernel(const uint16_t* __restrict__ x,
-                                                          int64_t n_blocks, const uint32_t* amax,
-                                                          float* g_out,
-                                                          uint16_t* __restrict__ img) {
+// x [total, nh, D] -> fake-quantised tiles.  COLS = false: blocks of 16
+// along d (Q, K); COLS = true: blocks of 16 tokens of one channel from the
+// sequence's start (V; the 128-row tiles hold whole blocks).  Rows past the
+// sequence end are zero.  grid (ceil(maxlen / 128), nh, nseq), 256 threads.
+template <int DT, bool SS, int D, bool COLS>
+__global__ void __launch_bounds__(256) qat_fq_tile_kernel(const uint16_t* __restrict__ x,
+                                                          SeqInfo si, int nh, int64_t nslot,
+                                                          const uint32_t* amax, float* g_out,
+                                                          uint8_t* __restrict__ tiles) {
+  __shared__ __align__(128) uint8_t img[128 * D * 2];
+  const int t = blockIdx.x, hd = blockIdx.y, seq = blockIdx.z;
   const float g = tensor_scale_from_amax(*amax);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks;
-       b += (int64_t)gridDim.x * blockDim.x) {
-    float v[16];
-    load16<DT>(x + b * 16, v);
-    uint32_t lo, hi;
-    const float sv = ue4m3_decode(quant_block16(v, g, SS, lo, hi));
-    uint4 w0, w1;
-    w0.x = fq_pair<DT>(lo & 0xFF, sv);
-    w0.y = fq_pair<DT>((lo >> 8) & 0xFF, sv);
-    w0.z = fq_pair<DT>((lo >> 16) & 0xFF, sv);
-    w0.w = fq_pair<DT>(lo >> 24, sv);
-    w1.x = fq_pair<DT>(hi & 0xFF, sv);
-    w1.y = fq_pair<DT>((hi >> 8) & 0xFF, sv);
-    w1.z = fq_pair<DT>((hi >> 16) & 0xFF, sv);
-    w1.w = fq_pair<DT>(hi >> 24, sv);
-    uint4* o = reinterpret_cast<uint4*>(img + b * 16);
-    o[0] = w0;
-    o[1] = w1;
-  }
-}
-
-// V: blocks of 16 tokens of one channel from each sequence's start, the last
-// block zero-padded.  grid (ceil(maxlen / 16), nseq); ncols = Hkv * d.
-template <int DT, bool SS>
-__global__ void __launch_bounds__(256) qat_fq_v_kernel(const uint16_t* __restrict__ v, SeqInfo si,
-                                                       int ncols, const uint32_t* amax,
-                                                       float* g_out, uint16_t* __restrict__ img) {
+  if ((t | hd | seq) == 0 && threadIdx.x == 0) *g_out = g;
   int64_t st;
   int len;
-  si.get(blockIdx.y, st, len);
-  const float g = tensor_scale_from_amax(*amax);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
-  const int t0 = blockIdx.x * 16;
-  if (t0 >= len) return;
-  const int n = min(16, len - t0);
-  for (int c = threadIdx.x; c < ncols; c += blockDim.x) {
-    float x[16];
+  si.get(seq, st, len);
+  const int r0 = t * 128;
+  if (r0 >= len) return;
+  const int n = min(128, len - r0);
+  constexpr int NB = 128 * D / 16;
+  for (int b = threadIdx.x; b < NB; b += blockDim.x) {
+    float v[16];
+    int r, c;
+    if constexpr (!COLS) {
+      r = b / (D / 16);
+      c = (b % (D / 16)) * 16;
+      if (r < n) {
+        load16<DT>(x + ((st + r0 + r) * nh + hd) * D + c, v);
+      } else {
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
-      x[e] = e < n ? h2f<DT>(v[(st + t0 + e) * ncols + c]) : 0.0f;
+        for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+      }
+    } else {
+      c = b % D;
+      r = (b / D) * 16;
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        v[e] = r + e < n ? h2f<DT>(x[((st + r0 + r + e) * nh + hd) * D + c]) : 0.0f;
+    }
     uint32_t lo, hi;
-    const float sv = ue4m3_decode(quant_block16(x, g, SS, lo, hi));
+    const float sv = ue4m3_decode(quant_block16(v, g, SS, lo, hi));
+    uint32_t w[8];
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {
-      const uint32_t byte = ((e < 8 ? lo : hi) >> (8 * ((e & 7) >> 1))) & 0xFF;
-      const uint32_t pr = fq_pair<DT>(byte, sv);
-      if (e < n) img[(st + t0 + e) * ncols + c] = (uint16_t)(pr & 0xFFFF);
-      if (e + 1 < n) img[(st + t0 + e + 1) * ncols + c] = (uint16_t)(pr >> 16);
+    for (int i = 0; i < 8; ++i) w[i] = fq_pair<DT>(((i < 4 ? lo : hi) >> (8 * (i & 3))) & 0xFF, sv);
+    if constexpr (!COLS) {
+      *reinterpret_cast<uint4*>(img + qt_elem(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(img + qt_elem(r, c + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        *reinterpret_cast<uint16_t*>(img + qt_elem(r + 2 * i, c)) = (uint16_t)(w[i] & 0xFFFF);
+        *reinterpret_cast<uint16_t*>(img + qt_elem(r + 2 * i + 1, c)) = (uint16_t)(w[i] >> 16);
+      }
     }
   }
+  __syncthreads();
+  uint4* dst = reinterpret_cast<uint4*>(tiles + qat_slot(hd, nslot, st, seq, t) * qt_tile_bytes(D));
+  const uint4* src = reinterpret_cast<const uint4*>(img);
+  for (int i = threadIdx.x; i < 128 * D / 8; i += blockDim.x) dst[i] = src[i];
 }
 
-// ------------------------------------------------------------ warp MMAs --
-
-template <int DT>
-__device__ __forceinline__ uint32_t qpack2(float lo, float hi) {
-  return (uint32_t)f2h<DT>(lo) | ((uint32_t)f2h<DT>(hi) << 16);
-}
-
-// c += a (16 x 16, row) * b (16 x 8, col), fp32 accumulate.  Fragments:
-// a[0] (row g, k 2t..2t+1), a[1] (row g+8, same k), a[2] (row g, k 2t+8..),
-// a[3] (row g+8, k 2t+8..); b0 (k 2t..2t+1, col g), b1 (k 2t+8.., col g);
-// c[0..1] (row g, cols 2t, 2t+1), c[2..3] (row g+8, same cols); g = lane/4,
-// t = lane%4.
-template <int DT>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  if constexpr (DT == 1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  } else {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-}
-
-// Shared-memory tiles are row-major 16-bit with LD = cols + 8 elements per
-// row: a warp's fragment loads then touch 32 distinct banks, and every row
-// starts on a 16-byte boundary.
-template <int LD>
-__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const uint16_t* t, int row0, int k0,
-                                       int g, int tq) {
-  const uint16_t* p = t + (row0 + g) * LD + k0 + 2 * tq;
-  a[0] = *reinterpret_cast<const uint32_t*>(p);
-  a[1] = *reinterpret_cast<const uint32_t*>(p + 8 * LD);
-  a[2] = *reinterpret_cast<const uint32_t*>(p + 8);
-  a[3] = *reinterpret_cast<const uint32_t*>(p + 8 * LD + 8);
-}
-
-template <int LD>
-__device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const uint16_t* t, int n0, int k0,
-                                       int g, int tq) {
-  const uint16_t* p = t + (n0 + g) * LD + k0 + 2 * tq;
-  b0 = *reinterpret_cast<const uint32_t*>(p);
-  b1 = *reinterpret_cast<const uint32_t*>(p + 8);
-}
-
-// B fragments of n-tiles n0 and n0 + 8 for the k-step at row k0 of a
-// row-major tile whose rows run along the contraction (k) axis, transposed
-// on the way in by ldmatrix: b[0], b[1] for n-tile n0, b[2], b[3] for n0 + 8.
-// Lane l addresses row k0 + (l & 15), column n0 + 8 (l >> 4); rows are
-// 16-byte aligned and 8 consecutive rows hit distinct banks (LD = cols + 8).
-template <int LD>
-__device__ __forceinline__ void frag_b_t2(uint32_t (&b)[4], const uint16_t* t, int k0, int n0,
-                                          int lane) {
-  const uint32_t a = smem_u32(t + (k0 + (lane & 15)) * LD + n0 + 8 * (lane >> 4));
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
-               : "r"(a));
-}
-
-// The A fragment of k-step s from accumulator tiles c[2s], c[2s+1] (the C
-// layout of two n-tiles is the A layout of one 16-wide k-step).
-template <int DT>
-__device__ __forceinline__ void c_to_a(uint32_t (&a)[4], const float (&c0)[4],
-                                       const float (&c1)[4]) {
-  a[0] = qpack2<DT>(c0[0], c0[1]);
-  a[1] = qpack2<DT>(c0[2], c0[3]);
-  a[2] = qpack2<DT>(c1[0], c1[1]);
-  a[3] = qpack2<DT>(c1[2], c1[3]);
-}
-
-// dS as the sum of two 16-bit parts, hi = round(dS) and lo = round(dS - hi),
-// for two MMAs into one accumulator: rows of dS sum to zero, and rounding
-// dS once would leave a residue that the products with K^ (whose channel
-// means can be large) or Q^ magnify; the split carries about 16 bits.
-template <int DT>
-__device__ __forceinline__ void c_to_a_split(uint32_t (&hi)[4], uint32_t (&lo)[4],
-                                             const float (&c0)[4], const float (&c1)[4]) {
-  const float* src[2] = {c0, c1};
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float* c = src[r >> 1] + 2 * (r & 1);
-    const uint32_t h = qpack2<DT>(c[0], c[1]);
-    hi[r] = h;
-    lo[r] = qpack2<DT>(c[0] - h2f<DT>((uint16_t)(h & 0xFFFF)), c[1] - h2f<DT>((uint16_t)(h >> 16)));
-  }
-}
-
-// Rows [r0, r0 + R) of a [tokens, nh, D] image (head h) -> tile [R][LD]
-// through cp.async, 16 bytes a copy; rows at or past len are zero-filled.
-// The caller commits the group and waits for it.
-template <int D, int R, int LD>
-__device__ __forceinline__ void stage_rows_async(uint16_t* t, const uint16_t* x, int64_t st,
-                                                 int len, int r0, int nh, int h) {
+// D = rowsum(dO o O') per (token, head), and the dO tiles.  One thread per
+// 16-byte chunk of dO; the D / 8 chunks of a row are consecutive lanes.
+// grid (ceil(maxlen / 128), H, nseq), 256 threads.
+template <int DT, int D>
+__global__ void __launch_bounds__(256) qat_rowdot_tile_kernel(
+    const uint16_t* __restrict__ dout, const float* __restrict__ out_hp, SeqInfo si, int H,
+    int64_t total, int64_t nslot, float* __restrict__ dsum, uint8_t* __restrict__ tiles) {
   constexpr int CH = D / 8;
-  for (int i = threadIdx.x; i < R * CH; i += blockDim.x) {
+  const int t = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+  int64_t st;
+  int len;
+  si.get(seq, st, len);
+  const int r0 = t * 128;
+  if (r0 >= len) return;
+  uint8_t* tile = tiles + qat_slot(h, nslot, st, seq, t) * qt_tile_bytes(D);
+  for (int i = threadIdx.x; i < 128 * CH; i += blockDim.x) {  // 128 * CH: a multiple of 256
     const int r = i / CH, c = i % CH;
     const bool ok = r0 + r < len;
-    const uint16_t* src = ok ? x + ((st + r0 + r) * nh + h) * D + 8 * c : x;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(t + r * LD + 8 * c)),
-                 "l"(src), "r"(ok ? 16 : 0)
-                 : "memory");
+    uint4 v = make_uint4(0, 0, 0, 0);
+    float acc = 0.0f;
+    if (ok) {
+      const int64_t e = ((st + r0 + r) * H + h) * D + 8 * c;
+      v = __ldg(reinterpret_cast<const uint4*>(dout + e));
+      const float4 o0 = __ldg(reinterpret_cast<const float4*>(out_hp + e));
+      const float4 o1 = __ldg(reinterpret_cast<const float4*>(out_hp + e) + 1);
+      const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc = fmaf(h2f<DT>((uint16_t)(w[k] & 0xFFFF)), o[2 * k], acc);
+        acc = fmaf(h2f<DT>((uint16_t)(w[k] >> 16)), o[2 * k + 1], acc);
+      }
+    }
+#pragma unroll
+    for (int m = CH / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (ok && c == 0) dsum[(int64_t)h * total + st + r0 + r] = acc;
+    *reinterpret_cast<uint4*>(tile + qt_elem(r, 8 * c)) = v;
   }
 }
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ float quad_max(float v) {
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-}
+// ------------------------------------------------------ shared helpers --
 
 // FP4 value of a probability already divided by sigma: the 16-key block's
 // scale byte from amax (the block's largest scaled value), then the E2M1 code
@@ -283,541 +261,725 @@ __device__ __forceinline__ void qat_rcp_table(float* rcp) {
     rcp[b] = (b == 0 || b == 127) ? 0.0f : __frcp_rn(ue4m3_decode((uint32_t)b));
 }
 
-template <int D, int BLK>
-struct QatFwdSmem {
-  static constexpr int LD = D + 8;
-  static constexpr int Q = 0;
-  static constexpr int K = Q + kQatFwdRows * LD;  // two buffers of K and V each: the
-  static constexpr int V = K + 2 * BLK * LD;   // key tile in use and the next one
-  static constexpr int RCP = V + 2 * BLK * LD;  // 128 floats follow the 16-bit tiles
-  static constexpr size_t BYTES = (size_t)RCP * 2 + 128 * 4;
+// 16-bit pair of two fp32 values, and the pair of the residuals (x - hi).
+template <int DT>
+__device__ __forceinline__ void qt_split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack2<DT>(x0, x1);
+  lo = pack2<DT>(x0 - h2f<DT>((uint16_t)(hi & 0xFFFF)), x1 - h2f<DT>((uint16_t)(hi >> 16)));
+}
+
+// Stores 32 consecutive 16-bit values (columns c0..c0+31, c0 % 32 == 0) of
+// row r of a tile.
+__device__ __forceinline__ void qt_store32(uint8_t* tile, int r, int c0, const uint32_t (&w)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(tile + qt_elem(r, c0 + 8 * q)) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
+// Shared-memory control block of the attention kernels (kQtShBytes):
+// barriers [0, 128), the lane quarters' pair barriers [128, 160), the
+// tensor-memory base and the abort flag, the UE4M3 reciprocals [256, 768),
+// the pair exchange [1024, 2048).
+struct QtShared {
+  uint64_t* bars;
+  uint64_t* xbar;
+  uint32_t* tmem;
+  volatile int* abort;
+  float* rcp;
+  float* xch;
 };
 
-// ------------------------------------------------------------- forward --
-// grid (ceil(maxlen / 128) * H, nseq), 256 threads, the tile index the
-// slowest: causal grids start the longest rows of every head first.  Warp w
-// owns query rows 16w..16w+15 of the tile; the eight warps share the
-// double-buffered K and V tiles.
-//
-// One pass over the key tiles with a running maximum m (log2 units): the
-// FP4 image of P on a key tile does not depend on lse, because
-// P / sigma = 2688 exp(S - max_tile S); the tile's sigma =
-// exp(max_tile S - lse) / 2688 enters as exp2(mt - m) / 2688 x (the rescale
-// of the running sums to the final m and the division by l), the same
-// bookkeeping as O' = sum exp2(s - m) V / l.
-template <int DT, int D, int BLK>
-__global__ void __launch_bounds__(256) qat_fwd_kernel(QatParams p) {
-  using L = QatFwdSmem<D, BLK>;
-  constexpr int LD = L::LD, NT = BLK / 8, ND = D / 8, ROWS = kQatFwdRows;
-  extern __shared__ __align__(16) uint16_t qsm[];
-  uint16_t* sQ = qsm + L::Q;
-  int64_t st;
-  int len;
-  p.si.get(blockIdx.y, st, len);
-  const int tiles = (len + ROWS - 1) / ROWS;
-  const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
-  if (ti >= tiles) return;
-  const int q0 = (p.causal ? tiles - 1 - ti : ti) * ROWS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;
-  const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
-  const int kend = p.causal ? min(len, q0 + ROWS) : len;
-  const int ntiles = (kend + BLK - 1) / BLK;
-
-  auto issue = [&](int kt) {
-    const int buf = kt & 1;
-    stage_rows_async<D, BLK, LD>(qsm + L::K + buf * BLK * LD, p.ki, st, len, kt * BLK, p.Hkv, hk);
-    stage_rows_async<D, BLK, LD>(qsm + L::V + buf * BLK * LD, p.vi, st, len, kt * BLK, p.Hkv, hk);
-  };
-  float* s_rcp = reinterpret_cast<float*>(qsm + L::RCP);
-  qat_rcp_table(s_rcp);  // visible after the first barrier of the loop
-  stage_rows_async<D, ROWS, LD>(sQ, p.qi, st, len, q0, p.H, h);
-  issue(0);
-  cp_async_commit();
-
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
-  float o[ND][4], oh[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[n][e] = oh[n][e] = 0.0f;
-  for (int kt = 0; kt < ntiles; ++kt) {
-    const uint16_t* sK = qsm + L::K + (kt & 1) * BLK * LD;
-    const uint16_t* sV = qsm + L::V + (kt & 1) * BLK * LD;
-    if (kt + 1 < ntiles) {
-      issue(kt + 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int j0 = kt * BLK;
-    float s[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t a[4];
-      frag_a<LD>(a, sQ, 16 * warp, 16 * kk, g, tq);
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        uint32_t b0, b1;
-        frag_b<LD>(b0, b1, sK, 8 * n, 16 * kk, g, tq);
-        mma16816<DT>(s[n], a, b0, b1);
-      }
-    }
-    // scores in log2 units, masked; tile row maxima; running maxima
-    float mt[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = j0 + 8 * n + 2 * tq + (e & 1), i = row[e >> 1];
-        const bool ok = j < len && (!p.causal || j <= i);
-        s[n][e] = ok ? s[n][e] * c2 : -INFINITY;
-        mt[e >> 1] = fmaxf(mt[e >> 1], s[n][e]);
-      }
-    float fct[2], inv2688 = 1.0f / kTensorScaleDiv;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mt[r] = quad_max(mt[r]);
-      const float mn = fmaxf(m[r], mt[r]);
-      const float alpha = (m[r] == -INFINITY || mn == -INFINITY) ? 0.0f : exp2f(m[r] - mn);
-      m[r] = mn;
-      l[r] *= alpha;
-#pragma unroll
-      for (int n = 0; n < ND; ++n) {
-        o[n][2 * r] *= alpha;
-        o[n][2 * r + 1] *= alpha;
-        oh[n][2 * r] *= alpha;
-        oh[n][2 * r + 1] *= alpha;
-      }
-      // sigma of this tile relative to the running maximum
-      fct[r] = mt[r] == -INFINITY ? 0.0f : exp2f(mt[r] - mn) * inv2688;
-    }
-    // a row without a visible key in the tile has s = -inf throughout:
-    // finite references keep its exponentials at 0
-    const float mr[2] = {m[0] == -INFINITY ? 0.0f : m[0], m[1] == -INFINITY ? 0.0f : m[1]};
-    const float mtr[2] = {mt[0] == -INFINITY ? 0.0f : mt[0], mt[1] == -INFINITY ? 0.0f : mt[1]};
-#pragma unroll
-    for (int b = 0; b < NT / 2; ++b) {
-      float qv[2][4], pe[2][4];  // P^ / (tile factor) and exp2(s - m), C layout
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float s0 = s[2 * b + u][2 * r], s1 = s[2 * b + u][2 * r + 1];
-          pe[u][2 * r] = exp2f(s0 - mr[r]);
-          pe[u][2 * r + 1] = exp2f(s1 - mr[r]);
-          l[r] += pe[u][2 * r] + pe[u][2 * r + 1];
-          // P / sigma of the oracle's reading: 2688 exp(S - max_tile S)
-          qv[u][2 * r] = kTensorScaleDiv * exp2f(s0 - mtr[r]);
-          qv[u][2 * r + 1] = kTensorScaleDiv * exp2f(s1 - mtr[r]);
-        }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const PBlock pb(quad_max(fmaxf(fmaxf(qv[0][2 * r], qv[0][2 * r + 1]),
-                                       fmaxf(qv[1][2 * r], qv[1][2 * r + 1]))),
-                        s_rcp);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float y0, y1;
-          pb.apply(qv[u][2 * r], qv[u][2 * r + 1], y0, y1);
-          qv[u][2 * r] = __fmul_rn(y0, fct[r]);
-          qv[u][2 * r + 1] = __fmul_rn(y1, fct[r]);
-        }
-      }
-      // O' carries P in two parts: it sets D = rowsum(dO o O') of the
-      // backward, whose error reaches dQ multiplied by the keys' means
-      uint32_t aq[4], ph[4], pl[4];
-      c_to_a<DT>(aq, qv[0], qv[1]);
-      c_to_a_split<DT>(ph, pl, pe[0], pe[1]);
-#pragma unroll
-      for (int n = 0; n < ND; n += 2) {
-        uint32_t bb[4];
-        frag_b_t2<LD>(bb, sV, 16 * b, 8 * n, lane);
-        mma16816<DT>(oh[n], ph, bb[0], bb[1]);
-        mma16816<DT>(oh[n + 1], ph, bb[2], bb[3]);
-        mma16816<DT>(o[n], aq, bb[0], bb[1]);
-        mma16816<DT>(o[n + 1], aq, bb[2], bb[3]);
-        mma16816<DT>(oh[n], pl, bb[0], bb[1]);
-        mma16816<DT>(oh[n + 1], pl, bb[2], bb[3]);
-      }
-    }
-    __syncthreads();  // every read of this buffer done before it is refilled
+// many_mask: the barriers every row-owning thread arrives on (count 256);
+// the others complete on one arrival or an MMA commit.
+__device__ __forceinline__ QtShared qt_setup(uint8_t* sh, int nbar, uint32_t many_mask) {
+  QtShared s;
+  s.bars = reinterpret_cast<uint64_t*>(sh);
+  s.xbar = reinterpret_cast<uint64_t*>(sh + 128);
+  s.tmem = reinterpret_cast<uint32_t*>(sh + 160);
+  s.abort = reinterpret_cast<volatile int*>(sh + 164);
+  s.rcp = reinterpret_cast<float*>(sh + 256);
+  s.xch = reinterpret_cast<float*>(sh + 1024);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbar; ++i)
+      mbar_init(&s.bars[i], ((many_mask >> i) & 1u) ? kQtWarps * 32 : 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.xbar[i], 64);
+    *s.abort = 0;
+    fence_mbar_init();
   }
-  const float gv = p.g[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float t = l[r];
-    t += __shfl_xor_sync(0xffffffffu, t, 1);
-    t += __shfl_xor_sync(0xffffffffu, t, 2);
-    if (row[r] >= len) continue;
-    if (tq == 0) p.lse[(int64_t)h * p.total + st + row[r]] = (m[r] + log2f(t)) * kQatLn2;
-    const float sc_out = gv / t;
-    const int64_t base = ((st + row[r]) * p.H + h) * D;
-#pragma unroll
-    for (int n = 0; n < ND; ++n) {
-      const int c = 8 * n + 2 * tq;
-      *reinterpret_cast<uint32_t*>(p.out + base + c) =
-          qpack2<DT>(o[n][2 * r] * sc_out, o[n][2 * r + 1] * sc_out);
-      *reinterpret_cast<float2*>(p.out_hp + base + c) =
-          make_float2(oh[n][2 * r] * sc_out, oh[n][2 * r + 1] * sc_out);
-    }
+  qat_rcp_table(s.rcp);
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kQtMma) {
+    tmem_alloc(s.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return s;
+}
+
+__device__ __forceinline__ void qt_teardown(const QtShared& s) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kQtMma) {
+    tc_fence_after();
+    tmem_dealloc(*s.tmem, 512);
   }
 }
 
-// D = rowsum(dO o O') per (token, head); one warp per row.
-template <int DT, int D>
-__global__ void __launch_bounds__(256) qat_rowdot_kernel(const uint16_t* __restrict__ dout,
-                                                         const float* __restrict__ out_hp,
-                                                         int64_t total, int H,
-                                                         float* __restrict__ dsum) {
-  const int lane = threadIdx.x & 31;
-  const int64_t nrows = total * H;
-  for (int64_t rr = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; rr < nrows;
-       rr += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    float acc = 0.0f;
-#pragma unroll
-    for (int c = lane; c < D; c += 32) acc = fmaf(h2f<DT>(dout[rr * D + c]), out_hp[rr * D + c], acc);
-#pragma unroll
-    for (int m2 = 16; m2 >= 1; m2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m2);
-    if (lane == 0) dsum[(rr % H) * total + rr / H] = acc;
-  }
+// Bounded wait a copy or MMA role makes at its end for the last phase it
+// armed: no copy or MMA outlives the CTA.
+__device__ __forceinline__ void qt_drain(uint64_t* bar, uint32_t parity) {
+  int flag = 0;
+  volatile int* never = &flag;
+  mbar_wait(bar, parity, never, 200000000ull);
 }
 
-template <int D, int BLK>
-struct QatKvSmem {
-  static constexpr int LD = D + 8, NW = BLK / 16;
-  static constexpr int K = 0;
-  static constexpr int V = K + BLK * LD;
-  static constexpr int Q = V + BLK * LD;             // two buffers of [64][LD] each:
-  static constexpr int DO = Q + 2 * kQatChunk * LD;  // the chunk in use and the next one
-  static constexpr int END16 = DO + 2 * kQatChunk * LD;  // 16-bit elements; fp32 arrays follow
-  // fp32: lse (log2 units) [2][64], D [2][64], column maxima [NW][64], the
-  // columns' 2688 / max and max / 2688 [2][64], UE4M3 reciprocals [128]
-  static constexpr size_t BYTES =
-      (size_t)END16 * 2 + (size_t)(6 + NW) * kQatChunk * 4 + 128 * 4;
-};
-
-// ------------------------------------------------- backward: dK and dV --
-// grid (ceil(maxlen / BLK) * Hkv, nseq), BLK / 16 warps, the key tile the
-// slowest (causal grids start the tiles with the most queries first); warp w
-// owns keys 16w..16w+15 of the tile (one 16-key block of the P
-// quantisation).
-template <int DT, int D, int BLK>
-__global__ void __launch_bounds__(BLK * 2) qat_bwd_kv_kernel(QatParams p) {
-  using L = QatKvSmem<D, BLK>;
-  constexpr int LD = L::LD, NW = L::NW, QC = kQatChunk, NQ = QC / 8, ND = D / 8;
-  extern __shared__ __align__(16) uint16_t qsm[];
-  uint16_t* sK = qsm + L::K;
-  uint16_t* sV = qsm + L::V;
-  float* s_lse2b = reinterpret_cast<float*>(qsm + L::END16);  // [2][QC]
-  float* s_Db = s_lse2b + 2 * QC;                               // [2][QC]
-  float* s_cmax = s_Db + 2 * QC;                                // [NW][QC]
-  float* s_cinv = s_cmax + NW * QC;                             // [QC]
-  float* s_csig = s_cinv + QC;                                  // [QC]
-  float* s_rcp = s_csig + QC;                                   // [128]
-  int64_t st;
-  int len;
-  p.si.get(blockIdx.y, st, len);
-  const int j0 = (int)blockIdx.x / p.Hkv * BLK, hk = (int)blockIdx.x % p.Hkv, grp = p.H / p.Hkv;
-  if (j0 >= len) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
-  const int key[2] = {j0 + 16 * warp + g, j0 + 16 * warp + g + 8};
-  // query chunks: every head of the group, from the first chunk that sees a
-  // key of this tile; chunk it + 1 is fetched while chunk it is computed
-  const int qstart = p.causal ? j0 / QC * QC : 0;
-  const int nch = (len - qstart + QC - 1) / QC;
-  const int n_it = grp * nch;
-  auto issue = [&](int it) {
-    const int buf = it & 1, h = hk * grp + it / nch, qc0 = qstart + (it % nch) * QC;
-    stage_rows_async<D, QC, LD>(qsm + L::Q + buf * QC * LD, p.qi, st, len, qc0, p.H, h);
-    stage_rows_async<D, QC, LD>(qsm + L::DO + buf * QC * LD, p.dout, st, len, qc0, p.H, h);
-    for (int i = threadIdx.x; i < QC; i += blockDim.x) {
-      const bool ok = qc0 + i < len;
-      s_lse2b[buf * QC + i] = ok ? p.lse[(int64_t)h * p.total + st + qc0 + i] * kQatLog2e : 0.0f;
-      s_Db[buf * QC + i] = ok ? p.dsum[(int64_t)h * p.total + st + qc0 + i] : 0.0f;
-    }
-  };
-
-  qat_rcp_table(s_rcp);  // visible after the first barrier of the loop
-  stage_rows_async<D, BLK, LD>(sK, p.ki, st, len, j0, p.Hkv, hk);
-  stage_rows_async<D, BLK, LD>(sV, p.vi, st, len, j0, p.Hkv, hk);
-  issue(0);
-  cp_async_commit();
-  float dk[ND][4], dv[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.0f;
-
-  for (int it = 0; it < n_it; ++it) {
-    if (it + 1 < n_it) {
-      issue(it + 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    {
-      const int buf = it & 1, qc0 = qstart + (it % nch) * QC;
-      const uint16_t* sQ = qsm + L::Q + buf * QC * LD;
-      const uint16_t* sdO = qsm + L::DO + buf * QC * LD;
-      const float* s_lse2 = s_lse2b + buf * QC;
-      const float* s_D = s_Db + buf * QC;
-      // S^T (keys x queries) and P^T
-      float s[NQ][4];
-#pragma unroll
-      for (int n = 0; n < NQ; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4];
-        frag_a<LD>(a, sK, 16 * warp, 16 * kk, g, tq);
-#pragma unroll
-        for (int n = 0; n < NQ; ++n) {
-          uint32_t b0, b1;
-          frag_b<LD>(b0, b1, sQ, 8 * n, 16 * kk, g, tq);
-          mma16816<DT>(s[n], a, b0, b1);
-        }
-      }
-#pragma unroll
-      for (int n = 0; n < NQ; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int il = 8 * n + 2 * tq + (e & 1), i = qc0 + il, j = key[e >> 1];
-          const bool ok = j < len && i < len && (!p.causal || j <= i);
-          s[n][e] = ok ? exp2f(s[n][e] * c2 - s_lse2[il]) : 0.0f;
-        }
-      // per query: max of P over the key tile (all warps)
-#pragma unroll
-      for (int n = 0; n < NQ; ++n)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v = fmaxf(s[n][c], s[n][c + 2]);
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-          if (g == 0) s_cmax[warp * QC + 8 * n + 2 * tq + c] = v;
-        }
-      __syncthreads();
-      // per query column, once: the max over the key tile and its factors
-      for (int c = threadIdx.x; c < QC; c += blockDim.x) {
-        float cm = 0.0f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) cm = fmaxf(cm, s_cmax[w * QC + c]);
-        s_cinv[c] = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
-        s_csig[c] = __fdiv_rn(cm, kTensorScaleDiv);
-      }
-      __syncthreads();
-      // dV += (P^)^T dO, one 16-query k-step at a time
-#pragma unroll
-      for (int b = 0; b < NQ / 2; ++b) {
-        float qv[2][4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int il = 8 * (2 * b + u) + 2 * tq + c;
-            const float inv = s_cinv[il], sig = s_csig[il];
-            const float x0 = __fmul_rn(s[2 * b + u][c], inv), x1 = __fmul_rn(s[2 * b + u][c + 2], inv);
-            float am = fmaxf(x0, x1);
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
-            const PBlock pb(am, s_rcp);
-            float y0, y1;
-            pb.apply(x0, x1, y0, y1);
-            qv[u][c] = __fmul_rn(y0, sig);
-            qv[u][c + 2] = __fmul_rn(y1, sig);
-          }
-        uint32_t a[4];
-        c_to_a<DT>(a, qv[0], qv[1]);
-#pragma unroll
-        for (int n = 0; n < ND; n += 2) {
-          uint32_t bb[4];
-          frag_b_t2<LD>(bb, sdO, 16 * b, 8 * n, lane);
-          mma16816<DT>(dv[n], a, bb[0], bb[1]);
-          mma16816<DT>(dv[n + 1], a, bb[2], bb[3]);
-        }
-      }
-      // dP^T = V^ dO^T, dS^T = P^T o (dP^T - D)
-      float dp[NQ][4];
-#pragma unroll
-      for (int n = 0; n < NQ; ++n) dp[n][0] = dp[n][1] = dp[n][2] = dp[n][3] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4];
-        frag_a<LD>(a, sV, 16 * warp, 16 * kk, g, tq);
-#pragma unroll
-        for (int n = 0; n < NQ; ++n) {
-          uint32_t b0, b1;
-          frag_b<LD>(b0, b1, sdO, 8 * n, 16 * kk, g, tq);
-          mma16816<DT>(dp[n], a, b0, b1);
-        }
-      }
-#pragma unroll
-      for (int n = 0; n < NQ; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int il = 8 * n + 2 * tq + (e & 1);
-          dp[n][e] = s[n][e] * (dp[n][e] * gv - s_D[il]);
-        }
-      // dK += dS^T Q^
-#pragma unroll
-      for (int b = 0; b < NQ / 2; ++b) {
-        uint32_t ah[4], al[4];
-        c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
-#pragma unroll
-        for (int n = 0; n < ND; n += 2) {
-          uint32_t bb[4];
-          frag_b_t2<LD>(bb, sQ, 16 * b, 8 * n, lane);
-          mma16816<DT>(dk[n], ah, bb[0], bb[1]);
-          mma16816<DT>(dk[n + 1], ah, bb[2], bb[3]);
-          mma16816<DT>(dk[n], al, bb[0], bb[1]);
-          mma16816<DT>(dk[n + 1], al, bb[2], bb[3]);
-        }
-      }
-    }
-    __syncthreads();  // every read of this buffer done before it is refilled
-  }
-  const float kscale = p.g[0] * p.sc;
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    if (key[r] >= len) continue;
-    const int64_t base = ((st + key[r]) * p.Hkv + hk) * D;
-#pragma unroll
-    for (int n = 0; n < ND; ++n) {
-      const int c = 8 * n + 2 * tq;
-      *reinterpret_cast<float2*>(p.dk + base + c) =
-          make_float2(dk[n][2 * r] * kscale, dk[n][2 * r + 1] * kscale);
-      *reinterpret_cast<float2*>(p.dv + base + c) = make_float2(dv[n][2 * r], dv[n][2 * r + 1]);
-    }
-  }
+// One value per row exchanged between the two warps of a lane quarter
+// (phase `phase` of the quarter's pair barrier): returns the partner's.
+__device__ __forceinline__ bool qt_pair_swap(const QtShared& s, int quarter, int half, int r,
+                                             uint32_t phase, float mine, float& other) {
+  s.xch[half * 128 + r] = mine;
+  mbar_arrive(&s.xbar[quarter]);
+  const bool ok = warp_wait(&s.xbar[quarter], phase & 1, s.abort);
+  other = s.xch[(half ^ 1) * 128 + r];
+  return ok;
 }
 
+// Largest raw score of 32 columns over the visible keys (key0 + i < klim);
+// -inf when none is visible.  tcgen05.ld is warp-wide: called by all lanes.
+__device__ __forceinline__ float qt_chunk_max(uint32_t taddr, int key0, int klim) {
+  float a[32];
+  tmem_ld32(taddr, a);
+  tmem_ld_wait();
+  float mx = -INFINITY;
+  if (__all_sync(0xffffffffu, key0 + 32 <= klim)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, a[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, key0 + i < klim ? a[i] : -INFINITY);
+  }
+  return mx;
+}
+
+__device__ __forceinline__ uint8_t* qt_smem_base() {
+  extern __shared__ uint8_t qt_raw[];
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qt_raw) + 1023) &
+                                    ~(uintptr_t)1023);
+}
+
+// ============================================================ forward ==
 template <int D>
-struct QatQSmem {
-  static constexpr int LD = D + 8;
-  static constexpr int Q = 0;
-  static constexpr int DO = Q + kQatRows * LD;
-  static constexpr int K = DO + kQatRows * LD;  // two buffers each: the key chunk
-  static constexpr int V = K + 2 * kQatChunk * LD;  // in use and the next one
-  static constexpr size_t BYTES = (size_t)(V + 2 * kQatChunk * LD) * 2;
+struct QtFwdLayout {
+  static constexpr uint32_t T = qt_tile_bytes(D);
+  static constexpr uint32_t Q = 0, K = T, V = 3 * T, P = 4 * T;  // K: 2 stages
+  static constexpr uint32_t PH = P + kQtPTile, PL = PH + kQtPTile, SH = PL + kQtPTile;
+  static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
+  static constexpr uint32_t T_S = 0, T_O = 256, T_OH = 256 + D;  // S: 2 slots
+  static_assert(T_OH + D <= 512, "tensor memory budget");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-// ------------------------------------------------------ backward: dQ --
-// grid (ceil(maxlen / 64) * H, nseq), 128 threads, the tile index the
-// slowest (causal grids start the longest rows first); warp w owns query
-// rows 16w..16w+15; keys in chunks of 64.
-template <int DT, int D>
-__global__ void __launch_bounds__(128) qat_bwd_q_kernel(QatParams p) {
-  using L = QatQSmem<D>;
-  constexpr int LD = L::LD, KC = kQatChunk, NK = KC / 8, ND = D / 8;
-  extern __shared__ __align__(16) uint16_t qsm[];
-  uint16_t* sQ = qsm + L::Q;
-  uint16_t* sdO = qsm + L::DO;
+enum : int {
+  FQ = 0, FKF = 1 /* 1,2 */, FKE = 3 /* 3,4 */, FVF = 5, FVE = 6, FSF = 7 /* 7,8 */,
+  FSE = 9 /* 9,10 */, FPF = 11, FPE = 12, FDONE = 13, FN = 14
+};
+constexpr uint32_t kFwdMany = (1u << FSE) | (1u << (FSE + 1)) | (1u << FPF);
+
+// grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads; causal grids
+// start the query tiles with the most keys.  Steps u < nt are pass A over
+// key tile u, steps nt <= u < 2 nt pass B over key tile u - nt.
+template <int DT, int D, int BLK>
+__global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams p) {
+  using L = QtFwdLayout<D>;
+  uint8_t* sm = qt_smem_base();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = blockIdx.y;
   int64_t st;
   int len;
-  p.si.get(blockIdx.y, st, len);
-  const int tiles = (len + kQatRows - 1) / kQatRows;
+  p.si.get(seq, st, len);
+  const int ntq = (len + 127) / 128;
   const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
-  if (ti >= tiles) return;
-  const int q0 = (p.causal ? tiles - 1 - ti : ti) * kQatRows;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
-  const int row[2] = {q0 + 16 * warp + g, q0 + 16 * warp + g + 8};
-  float lse2[2], dsum[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const bool ok = row[r] < len;
-    lse2[r] = ok ? p.lse[(int64_t)h * p.total + st + row[r]] * kQatLog2e : 0.0f;
-    dsum[r] = ok ? p.dsum[(int64_t)h * p.total + st + row[r]] : 0.0f;
-  }
-  float dq[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.0f;
-  const int kend = p.causal ? min(len, q0 + kQatRows) : len;
-  const int n_it = (kend + KC - 1) / KC;
-  // key chunk it + 1 is fetched while chunk it is computed
-  auto issue = [&](int it) {
-    const int buf = it & 1;
-    stage_rows_async<D, KC, LD>(qsm + L::K + buf * KC * LD, p.ki, st, len, it * KC, p.Hkv, hk);
-    stage_rows_async<D, KC, LD>(qsm + L::V + buf * KC * LD, p.vi, st, len, it * KC, p.Hkv, hk);
-  };
-  stage_rows_async<D, kQatRows, LD>(sQ, p.qi, st, len, q0, p.H, h);
-  stage_rows_async<D, kQatRows, LD>(sdO, p.dout, st, len, q0, p.H, h);
-  issue(0);
-  cp_async_commit();
-  for (int it = 0; it < n_it; ++it) {
-    const int k0 = it * KC;
-    const uint16_t* sK = qsm + L::K + (it & 1) * KC * LD;
-    const uint16_t* sV = qsm + L::V + (it & 1) * KC * LD;
-    if (it + 1 < n_it) {
-      issue(it + 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  if (ti >= ntq) return;
+  const int qt = p.causal ? ntq - 1 - ti : ti;
+  const int q0 = qt * 128;
+  const int kend = p.causal ? min(len, q0 + 128) : len;
+  const int nt = (kend + 127) / 128, nsteps = 2 * nt;
+  const QtShared S = qt_setup(sm + L::SH, FN, kFwdMany);
+  uint64_t* bars = S.bars;
+  const uint32_t tmem = *S.tmem;
+
+  if (warp == kQtProducer) {
+    if (lane == 0) {
+      const uint8_t* kbase = p.kt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
+      const uint8_t* vbase = p.vt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
+      mbar_arrive_expect_tx(&bars[FQ], L::T);
+      bulk_g2s(sm + L::Q, p.qt + qat_slot(h, p.nslot, st, seq, qt) * L::T, L::T, &bars[FQ]);
+      int lastk[2] = {-1, -1}, lastv = -1;
+      for (int u = 0; u < nsteps && !*S.abort; ++u) {
+        const int j = u < nt ? u : u - nt, sl = u & 1;
+        if (u >= 2 && !mbar_wait(&bars[FKE + sl], ((u >> 1) - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[FKF + sl], L::T);
+        bulk_g2s(sm + L::K + sl * L::T, kbase + (int64_t)j * L::T, L::T, &bars[FKF + sl]);
+        lastk[sl] = u;
+        if (u >= nt) {
+          if (j >= 1 && !mbar_wait(&bars[FVE], (j - 1) & 1, S.abort)) break;
+          mbar_arrive_expect_tx(&bars[FVF], L::T);
+          bulk_g2s(sm + L::V, vbase + (int64_t)j * L::T, L::T, &bars[FVF]);
+          lastv = j;
+        }
+      }
+      qt_drain(&bars[FQ], 0);
+      for (int sl = 0; sl < 2; ++sl)
+        if (lastk[sl] >= 0) qt_drain(&bars[FKF + sl], (lastk[sl] >> 1) & 1);
+      if (lastv >= 0) qt_drain(&bars[FVF], lastv & 1);
     }
-    __syncthreads();
-    float s[NK][4], dp[NK][4];
+  } else if (warp == kQtMma) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(DT, 128, 128);
+      constexpr uint32_t idPV = idesc_f16(DT, 128, D) | kIdescBmn;
+      const uint32_t base = smem_u32(sm);
+      auto issue_s = [&](int u) -> bool {
+        const int sl = u & 1;
+        if (!mbar_wait(&bars[FKF + sl], (u >> 1) & 1, S.abort)) return false;
+        if (u >= 2 && !mbar_wait(&bars[FSE + sl], ((u >> 1) - 1) & 1, S.abort)) return false;
+        tc_fence_after();
 #pragma unroll
-    for (int n = 0; n < NK; ++n)
+        for (int s = 0; s < D / 16; ++s)
+          mma_f16(tmem + L::T_S + sl * 128, qt_desc_k(base + L::Q, s),
+                  qt_desc_k(base + L::K + sl * L::T, s), idS, s > 0);
+        tc_commit(&bars[FSF + sl]);
+        tc_commit(&bars[FKE + sl]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars[FQ], 0, S.abort) && issue_s(0);
+      for (int u = 0; u < nsteps && ok; ++u) {
+        // the next tile's scores go ahead of this tile's products
+        if (u + 1 < nsteps && !issue_s(u + 1)) break;
+        if (u < nt) continue;
+        const int j = u - nt;
+        if (!mbar_wait(&bars[FPF], j & 1, S.abort) || !mbar_wait(&bars[FVF], j & 1, S.abort)) break;
+        tc_fence_after();
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.0f;
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t bv = qt_desc_mn(base + L::V, s);
+          mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
+          mma_f16(tmem + L::T_OH, qt_desc_k(base + L::PH, s), bv, idPV, j > 0 || s > 0);
+          mma_f16(tmem + L::T_OH, qt_desc_k(base + L::PL, s), bv, idPV, 1);
+        }
+        tc_commit(&bars[FPE]);
+        tc_commit(&bars[FVE]);
+      }
+      tc_commit(&bars[FDONE]);
+      qt_drain(&bars[FDONE], 0);
+    }
+  } else {
+    // row r of the tile; this warp's columns 64 half .. 64 half + 63
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane, row = q0 + r;
+    const bool row_ok = row < len;
+    const int klim = row_ok ? (p.causal ? row + 1 : len) : 0;  // visible keys: key < klim
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;  // raw score -> log2 units
+    bool ok = true;
+    // pass A: the row maximum over this warp's columns, then the pair's
+    float mraw = -INFINITY;
+    for (int u = 0; u < nt && ok; ++u) {
+      const int sl = u & 1;
+      if (!warp_wait(&bars[FSF + sl], (u >> 1) & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = 64 * half + 32 * cc;
+        mraw = fmaxf(mraw, qt_chunk_max(tl + L::T_S + sl * 128 + col, u * 128 + col, klim));
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[FSE + sl]);
+    }
+    float other = -INFINITY;
+    if (ok) ok = qt_pair_swap(S, quarter, half, r, 0, mraw, other);
+    const float m = fmaxf(mraw, other) * c2;  // rounding is monotone: max of the scaled scores
+    const float mref = m == -INFINITY ? 0.0f : m;
+    // pass B: P against the final maximum, P^ against each BLK-key
+    // sub-tile's own maximum
+    float lsum = 0.0f;
+    uint8_t* tP = sm + L::P;
+    uint8_t* tH = sm + L::PH;
+    uint8_t* tL = sm + L::PL;
+    for (int u = nt; u < nsteps && ok; ++u) {
+      const int sl = u & 1, j = u - nt, kb = j * 128;
+      const uint32_t ts = tl + L::T_S + sl * 128;
+      if (!warp_wait(&bars[FSF + sl], (u >> 1) & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+      float mt_raw = -INFINITY;
+      if constexpr (BLK == 128) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) mt_raw = fmaxf(mt_raw, qt_chunk_max(ts + 32 * c, kb + 32 * c, klim));
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = 64 * half + 32 * cc;
+          mt_raw = fmaxf(mt_raw, qt_chunk_max(ts + col, kb + col, klim));
+        }
+      }
+      const bool live = mt_raw != -INFINITY;
+      const float mt = mt_raw * c2;
+      const float mtr = live ? mt : 0.0f;
+      const float fct = live ? ex2_ftz(mt - mref) * (1.0f / kTensorScaleDiv) : 0.0f;
+      // the P tiles are free once the products of the previous tile are done
+      if (j >= 1 && !warp_wait(&bars[FPE], (j - 1) & 1, S.abort)) { ok = false; break; }
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = 64 * half + 32 * cc, key0 = kb + col;
+        float a[32];
+        tmem_ld32(ts + col, a);
+        tmem_ld_wait();
+        if (cc == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[FSE + sl]);
+        }
+        uint32_t wq[16], wh[16], wl[16];
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t aq[4], ad[4];
-      frag_a<LD>(aq, sQ, 16 * warp, 16 * kk, g, tq);
-      frag_a<LD>(ad, sdO, 16 * warp, 16 * kk, g, tq);
+        for (int b = 0; b < 2; ++b) {
+          float qv[16], pe[16];
+          float am = 0.0f;
 #pragma unroll
-      for (int n = 0; n < NK; ++n) {
-        uint32_t b0, b1;
-        frag_b<LD>(b0, b1, sK, 8 * n, 16 * kk, g, tq);
-        mma16816<DT>(s[n], aq, b0, b1);
-        frag_b<LD>(b0, b1, sV, 8 * n, 16 * kk, g, tq);
-        mma16816<DT>(dp[n], ad, b0, b1);
+          for (int i = 0; i < 16; ++i) {
+            const int e = 16 * b + i;
+            const bool vis = key0 + e < klim;
+            const float s = a[e] * c2;
+            pe[i] = vis ? ex2_ftz(s - mref) : 0.0f;
+            // P / sigma of the tile: 2688 exp(S - max_tile S)
+            qv[i] = vis ? kTensorScaleDiv * ex2_ftz(s - mtr) : 0.0f;
+            lsum += pe[i];
+            am = fmaxf(am, qv[i]);
+          }
+          const PBlock pb(am, S.rcp);
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            float y0, y1;
+            pb.apply(qv[i], qv[i + 1], y0, y1);
+            wq[8 * b + i / 2] = pack2<DT>(__fmul_rn(y0, fct), __fmul_rn(y1, fct));
+            qt_split2<DT>(pe[i], pe[i + 1], wh[8 * b + i / 2], wl[8 * b + i / 2]);
+          }
+        }
+        qt_store32(tP, r, col, wq);
+        qt_store32(tH, r, col, wh);
+        qt_store32(tL, r, col, wl);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[FPF]);
+    }
+    // epilogue: O = P^ V^ g_V / l, O' = P V^ g_V / l, lse; the row sum l
+    // from both halves (after the last products, so the exchange slots are
+    // free)
+    if (ok) ok = warp_wait(&bars[FPE], (nt - 1) & 1, S.abort);
+    float lo = 0.0f;
+    if (ok) ok = qt_pair_swap(S, quarter, half, r, 1, lsum, lo);
+    if (ok) {
+      tc_fence_after();
+      const float l = half == 0 ? lsum + lo : lo + lsum;
+      const float sc_out = l > 0.0f ? p.g[2] / l : 0.0f;
+      const int64_t base = ((st + (row_ok ? row : 0)) * p.H + h) * D;
+#pragma unroll 1
+      for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
+        float o[32], oh[32];
+        tmem_ld32(tl + L::T_O + c, o);
+        tmem_ld32(tl + L::T_OH + c, oh);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 w;
+            w.x = pack2<DT>(o[i] * sc_out, o[i + 1] * sc_out);
+            w.y = pack2<DT>(o[i + 2] * sc_out, o[i + 3] * sc_out);
+            w.z = pack2<DT>(o[i + 4] * sc_out, o[i + 5] * sc_out);
+            w.w = pack2<DT>(o[i + 6] * sc_out, o[i + 7] * sc_out);
+            *reinterpret_cast<uint4*>(p.out + base + c + i) = w;
+            *reinterpret_cast<float4*>(p.out_hp + base + c + i) =
+                make_float4(oh[i] * sc_out, oh[i + 1] * sc_out, oh[i + 2] * sc_out,
+                            oh[i + 3] * sc_out);
+            *reinterpret_cast<float4*>(p.out_hp + base + c + i + 4) =
+                make_float4(oh[i + 4] * sc_out, oh[i + 5] * sc_out, oh[i + 6] * sc_out,
+                            oh[i + 7] * sc_out);
+          }
+        }
+      }
+      if (row_ok && half == 0)
+        p.lse[(int64_t)h * p.total + st + row] = l > 0.0f ? (m + log2f(l)) * kQatLn2 : -INFINITY;
+    }
+  }
+  qt_teardown(S);
+}
+
+// ======================================================= backward: dQ ==
+template <int D>
+struct QtQLayout {
+  static constexpr uint32_t T = qt_tile_bytes(D);
+  static constexpr uint32_t Q = 0, DO = T, K = 2 * T, V = 4 * T;  // K: 2 stages, V: 1
+  static constexpr uint32_t DSH = 5 * T, DSL = DSH + kQtPTile, SH = DSL + kQtPTile;
+  static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  static_assert(T_DQ + D <= 512, "tensor memory budget");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+enum : int {
+  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSE = 8, QPF = 9,
+  QPE = 10, QDONE = 11, QN = 12
+};
+constexpr uint32_t kQMany = (1u << QSE) | (1u << QPF);
+
+// grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads.
+template <int DT, int D>
+__global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParams p) {
+  using L = QtQLayout<D>;
+  uint8_t* sm = qt_smem_base();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = blockIdx.y;
+  int64_t st;
+  int len;
+  p.si.get(seq, st, len);
+  const int ntq = (len + 127) / 128;
+  const int ti = (int)blockIdx.x / p.H, h = (int)blockIdx.x % p.H, hk = h / (p.H / p.Hkv);
+  if (ti >= ntq) return;
+  const int qt = p.causal ? ntq - 1 - ti : ti;
+  const int q0 = qt * 128;
+  const int kend = p.causal ? min(len, q0 + 128) : len;
+  const int nt = (kend + 127) / 128;
+  const QtShared S = qt_setup(sm + L::SH, QN, kQMany);
+  uint64_t* bars = S.bars;
+  const uint32_t tmem = *S.tmem;
+
+  if (warp == kQtProducer) {
+    if (lane == 0) {
+      const int64_t qs = qat_slot(h, p.nslot, st, seq, qt);
+      const uint8_t* kbase = p.kt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
+      const uint8_t* vbase = p.vt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
+      mbar_arrive_expect_tx(&bars[QQ], 2 * L::T);
+      bulk_g2s(sm + L::Q, p.qt + qs * L::T, L::T, &bars[QQ]);
+      bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[QQ]);
+      int lastk[2] = {-1, -1}, lastv = -1;
+      for (int j = 0; j < nt && !*S.abort; ++j) {
+        const int sl = j & 1;
+        if (j >= 2 && !mbar_wait(&bars[QKE + sl], ((j >> 1) - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[QKF + sl], L::T);
+        bulk_g2s(sm + L::K + sl * L::T, kbase + (int64_t)j * L::T, L::T, &bars[QKF + sl]);
+        lastk[sl] = j;
+        if (j >= 1 && !mbar_wait(&bars[QVE], (j - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[QVF], L::T);
+        bulk_g2s(sm + L::V, vbase + (int64_t)j * L::T, L::T, &bars[QVF]);
+        lastv = j;
+      }
+      qt_drain(&bars[QQ], 0);
+      for (int sl = 0; sl < 2; ++sl)
+        if (lastk[sl] >= 0) qt_drain(&bars[QKF + sl], (lastk[sl] >> 1) & 1);
+      if (lastv >= 0) qt_drain(&bars[QVF], lastv & 1);
+    }
+  } else if (warp == kQtMma) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(DT, 128, 128);
+      constexpr uint32_t idDQ = idesc_f16(DT, 128, D) | kIdescBmn;
+      const uint32_t base = smem_u32(sm);
+      // S = Q^ K^T and dP = dO V^T of key tile j
+      auto issue_s = [&](int j) -> bool {
+        const int sl = j & 1;
+        if (!mbar_wait(&bars[QKF + sl], (j >> 1) & 1, S.abort)) return false;
+        if (!mbar_wait(&bars[QVF], j & 1, S.abort)) return false;
+        if (j >= 1 && !mbar_wait(&bars[QSE], (j - 1) & 1, S.abort)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + sl * L::T, s),
+                  idS, s > 0);
+          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
+                  s > 0);
+        }
+        tc_commit(&bars[QSF]);
+        tc_commit(&bars[QVE]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0);
+      for (int j = 0; j < nt && ok; ++j) {
+        if (j + 1 < nt && !issue_s(j + 1)) break;
+        if (!mbar_wait(&bars[QPF], j & 1, S.abort)) break;
+        tc_fence_after();
+        const uint32_t kt = base + L::K + (j & 1) * L::T;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t bk = qt_desc_mn(kt, s);
+          mma_f16(tmem + L::T_DQ, qt_desc_k(base + L::DSH, s), bk, idDQ, j > 0 || s > 0);
+          mma_f16(tmem + L::T_DQ, qt_desc_k(base + L::DSL, s), bk, idDQ, 1);
+        }
+        tc_commit(&bars[QPE]);
+        tc_commit(&bars[QKE + (j & 1)]);
+      }
+      tc_commit(&bars[QDONE]);
+      qt_drain(&bars[QDONE], 0);
+    }
+  } else {
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane, row = q0 + r;
+    const bool row_ok = row < len;
+    const int klim = row_ok ? (p.causal ? row + 1 : len) : 0;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
+    const float nlse2 = row_ok ? -p.lse[(int64_t)h * p.total + st + row] * kQatLog2e : 0.0f;
+    const float dsum = row_ok ? p.dsum[(int64_t)h * p.total + st + row] : 0.0f;
+    uint8_t* tH = sm + L::DSH;
+    uint8_t* tL = sm + L::DSL;
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      if (!warp_wait(&bars[QSF], j & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+      // the dS tiles are free once the products of the previous tile are done
+      if (j >= 1 && !warp_wait(&bars[QPE], (j - 1) & 1, S.abort)) { ok = false; break; }
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = 64 * half + 32 * cc, key0 = j * 128 + col;
+        float a[32], dp[32];
+        tmem_ld32(tl + L::T_S + col, a);
+        tmem_ld32(tl + L::T_DP + col, dp);
+        tmem_ld_wait();
+        if (cc == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[QSE]);
+        }
+        uint32_t wh[16], wl[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float pr = key0 + i + e < klim ? ex2_ftz(fmaf(a[i + e], c2, nlse2)) : 0.0f;
+            ds[e] = pr * (dp[i + e] * gv - dsum);
+          }
+          qt_split2<DT>(ds[0], ds[1], wh[i / 2], wl[i / 2]);
+        }
+        qt_store32(tH, r, col, wh);
+        qt_store32(tL, r, col, wl);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[QPF]);
+    }
+    if (ok && warp_wait(&bars[QPE], (nt - 1) & 1, S.abort)) {
+      tc_fence_after();
+      const float qscale = p.g[1] * p.sc;
+      const int64_t base = ((st + (row_ok ? row : 0)) * p.H + h) * D;
+#pragma unroll 1
+      for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
+        float gq[32];
+        tmem_ld32(tl + L::T_DQ + c, gq);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(p.dq + base + c + i) =
+                make_float4(gq[i] * qscale, gq[i + 1] * qscale, gq[i + 2] * qscale,
+                            gq[i + 3] * qscale);
+        }
       }
     }
-#pragma unroll
-    for (int n = 0; n < NK; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = k0 + 8 * n + 2 * tq + (e & 1), r = e >> 1, i = row[r];
-        const bool ok = j < len && i < len && (!p.causal || j <= i);
-        const float pr = ok ? exp2f(s[n][e] * c2 - lse2[r]) : 0.0f;
-        dp[n][e] = pr * (dp[n][e] * gv - dsum[r]);
+  }
+  qt_teardown(S);
+}
+
+// =================================================== backward: dK, dV ==
+template <int D>
+struct QtKvLayout {
+  static constexpr uint32_t T = qt_tile_bytes(D);
+  static constexpr uint32_t K = 0, V = T, Q = 2 * T, DO = 3 * T;
+  static constexpr uint32_t P = 4 * T, DSH = P + kQtPTile, DSL = DSH + kQtPTile;
+  static constexpr uint32_t SH = DSL + kQtPTile;
+  static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static_assert(T_DK + D <= 512, "tensor memory budget");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+enum : int { KKV = 0, KQF = 1, KQE = 2, KSF = 3, KSE = 4, KPF = 5, KPE = 6, KDONE = 7, KN = 8 };
+constexpr uint32_t kKvMany = (1u << KSE) | (1u << KPF);
+
+// grid (ceil(maxlen / 128) * Hkv, nseq), kQtThreads threads: key tile
+// blockIdx.x / Hkv (causal grids: the tiles with the most queries first).
+// Iteration it takes query chunk c0 + it % nch of query head
+// hk * grp + it / nch.
+template <int DT, int D, int BLK>
+__global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatParams p) {
+  using L = QtKvLayout<D>;
+  uint8_t* sm = qt_smem_base();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = blockIdx.y;
+  int64_t st;
+  int len;
+  p.si.get(seq, st, len);
+  const int kt = (int)blockIdx.x / p.Hkv, hk = (int)blockIdx.x % p.Hkv, grp = p.H / p.Hkv;
+  const int j0 = kt * 128;
+  if (j0 >= len) return;
+  const int c0 = p.causal ? kt : 0;  // first query chunk that sees a key of the tile
+  const int nch = (len + 127) / 128 - c0;
+  const int n_it = grp * nch;
+  const QtShared S = qt_setup(sm + L::SH, KN, kKvMany);
+  uint64_t* bars = S.bars;
+  const uint32_t tmem = *S.tmem;
+
+  if (warp == kQtProducer) {
+    if (lane == 0) {
+      const int64_t ks = qat_slot(hk, p.nslot, st, seq, kt);
+      mbar_arrive_expect_tx(&bars[KKV], 2 * L::T);
+      bulk_g2s(sm + L::K, p.kt + ks * L::T, L::T, &bars[KKV]);
+      bulk_g2s(sm + L::V, p.vt + ks * L::T, L::T, &bars[KKV]);
+      int last = -1;
+      for (int it = 0; it < n_it && !*S.abort; ++it) {
+        const int64_t qs = qat_slot(hk * grp + it / nch, p.nslot, st, seq, c0 + it % nch);
+        if (it >= 1 && !mbar_wait(&bars[KQE], (it - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[KQF], 2 * L::T);
+        bulk_g2s(sm + L::Q, p.qt + qs * L::T, L::T, &bars[KQF]);
+        bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[KQF]);
+        last = it;
       }
+      qt_drain(&bars[KKV], 0);
+      if (last >= 0) qt_drain(&bars[KQF], last & 1);
+    }
+  } else if (warp == kQtMma) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(DT, 128, 128);
+      constexpr uint32_t idG = idesc_f16(DT, 128, D) | kIdescAmn | kIdescBmn;
+      const uint32_t base = smem_u32(sm);
+      bool ok = mbar_wait(&bars[KKV], 0, S.abort);
+      for (int it = 0; it < n_it && ok; ++it) {
+        if (!mbar_wait(&bars[KQF], it & 1, S.abort)) break;
+        if (it >= 1 && !mbar_wait(&bars[KSE], (it - 1) & 1, S.abort)) break;
+        tc_fence_after();
 #pragma unroll
-    for (int b = 0; b < NK / 2; ++b) {
-      uint32_t ah[4], al[4];
-      c_to_a_split<DT>(ah, al, dp[2 * b], dp[2 * b + 1]);
+        for (int s = 0; s < D / 16; ++s) {
+          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K, s), idS, s > 0);
+          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
+                  s > 0);
+        }
+        tc_commit(&bars[KSF]);
+        if (!mbar_wait(&bars[KPF], it & 1, S.abort)) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q^: M = the 128 keys, K = the 128 queries
 #pragma unroll
-      for (int n = 0; n < ND; n += 2) {
-        uint32_t bb[4];
-        frag_b_t2<LD>(bb, sK, 16 * b, 8 * n, lane);
-        mma16816<DT>(dq[n], ah, bb[0], bb[1]);
-        mma16816<DT>(dq[n + 1], ah, bb[2], bb[3]);
-        mma16816<DT>(dq[n], al, bb[0], bb[1]);
-        mma16816<DT>(dq[n + 1], al, bb[2], bb[3]);
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t bq = qt_desc_mn(base + L::Q, s);
+          mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
+                  it > 0 || s > 0);
+          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSH, s), bq, idG, it > 0 || s > 0);
+          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSL, s), bq, idG, 1);
+        }
+        tc_commit(&bars[KPE]);
+        tc_commit(&bars[KQE]);
+      }
+      tc_commit(&bars[KDONE]);
+      qt_drain(&bars[KDONE], 0);
+    }
+  } else {
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
+    uint8_t* tP = sm + L::P;
+    uint8_t* tH = sm + L::DSH;
+    uint8_t* tL = sm + L::DSL;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int hq = hk * grp + it / nch, row = (c0 + it % nch) * 128 + r;
+      const bool row_ok = row < len;
+      const int klim = row_ok ? (p.causal ? row + 1 : len) : 0;
+      const float nlse2 = row_ok ? -p.lse[(int64_t)hq * p.total + st + row] * kQatLog2e : 0.0f;
+      const float dsum = row_ok ? p.dsum[(int64_t)hq * p.total + st + row] : 0.0f;
+      if (!warp_wait(&bars[KSF], it & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+      // sigma of this warp's BLK-key sub-tile: the largest P there / 2688
+      float cm_raw = -INFINITY;
+      if constexpr (BLK == 128) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c)
+          cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + 32 * c, j0 + 32 * c, klim));
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = 64 * half + 32 * cc;
+          cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + col, j0 + col, klim));
+        }
+      }
+      const float cm = cm_raw == -INFINITY ? 0.0f : ex2_ftz(fmaf(cm_raw, c2, nlse2));
+      const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
+      const float sig = __fdiv_rn(cm, kTensorScaleDiv);
+      // the tiles are free once the products of the previous chunk are done
+      if (it >= 1 && !warp_wait(&bars[KPE], (it - 1) & 1, S.abort)) { ok = false; break; }
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = 64 * half + 32 * cc, key0 = j0 + col;
+        float a[32], dp[32];
+        tmem_ld32(tl + L::T_S + col, a);
+        tmem_ld32(tl + L::T_DP + col, dp);
+        tmem_ld_wait();
+        if (cc == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[KSE]);
+        }
+        uint32_t wq[16], wh[16], wl[16];
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float pr[16], x[16];
+          float am = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = 16 * b + i;
+            pr[i] = key0 + e < klim ? ex2_ftz(fmaf(a[e], c2, nlse2)) : 0.0f;
+            x[i] = __fmul_rn(pr[i], inv);
+            am = fmaxf(am, x[i]);
+          }
+          const PBlock pb(am, S.rcp);
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            float y0, y1;
+            pb.apply(x[i], x[i + 1], y0, y1);
+            wq[8 * b + i / 2] = pack2<DT>(__fmul_rn(y0, sig), __fmul_rn(y1, sig));
+            const int e = 16 * b + i;
+            const float d0 = pr[i] * (dp[e] * gv - dsum), d1 = pr[i + 1] * (dp[e + 1] * gv - dsum);
+            qt_split2<DT>(d0, d1, wh[8 * b + i / 2], wl[8 * b + i / 2]);
+          }
+        }
+        qt_store32(tP, r, col, wq);
+        qt_store32(tH, r, col, wh);
+        qt_store32(tL, r, col, wl);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[KPF]);
+    }
+    // epilogue: lane r of the dV and dK accumulators is key j0 + r
+    if (ok && warp_wait(&bars[KPE], (n_it - 1) & 1, S.abort)) {
+      tc_fence_after();
+      const int key = j0 + r;
+      const bool key_ok = key < len;
+      const float kscale = p.g[0] * p.sc;
+      const int64_t base = ((st + (key_ok ? key : 0)) * p.Hkv + hk) * D;
+#pragma unroll 1
+      for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
+        float gdv[32], gdk[32];
+        tmem_ld32(tl + L::T_DV + c, gdv);
+        tmem_ld32(tl + L::T_DK + c, gdk);
+        tmem_ld_wait();
+        if (key_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            *reinterpret_cast<float4*>(p.dv + base + c + i) =
+                make_float4(gdv[i], gdv[i + 1], gdv[i + 2], gdv[i + 3]);
+            *reinterpret_cast<float4*>(p.dk + base + c + i) =
+                make_float4(gdk[i] * kscale, gdk[i + 1] * kscale, gdk[i + 2] * kscale,
+                            gdk[i + 3] * kscale);
+          }
+        }
       }
     }
-    __syncthreads();  // every read of this buffer done before it is refilled
   }
-  const float qscale = p.g[1] * p.sc;
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    if (row[r] >= len) continue;
-    const int64_t base = ((st + row[r]) * p.H + h) * D;
-#pragma unroll
-    for (int n = 0; n < ND; ++n)
-      *reinterpret_cast<float2*>(p.dq + base + 8 * n + 2 * tq) =
-          make_float2(dq[n][2 * r] * qscale, dq[n][2 * r + 1] * qscale);
-  }
+  qt_teardown(S);
 }
 
 }  // namespace thrift

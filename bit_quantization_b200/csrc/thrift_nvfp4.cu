@@ -632,21 +632,26 @@ __global__ void wait_timeout_kernel(int mode, uint64_t limit_ns) {
 // ---------------------------------------------------------- Attn-QAT glue --
 
 struct QatWs {
-  uint16_t* qi;
-  uint16_t* ki;
-  uint16_t* vi;
+  uint8_t* qt;   // fake-quantised tiles of Q [H][nslot], K, V [Hkv][nslot]
+  uint8_t* kt;
+  uint8_t* vt;
+  uint8_t* dot;  // dO tiles [H][nslot]
+  int64_t nslot;
   uint32_t* amax;  // [4]
   float* g;        // [4]
   float* dsum;     // [H, total]
   size_t bytes;
 };
 
-QatWs carve_qat(void* base, int64_t total, int H, int Hkv, int d) {
+QatWs carve_qat(void* base, int64_t total, int nseq, int H, int Hkv, int d) {
   Carve c(base);
   QatWs w;
-  w.qi = c.take<uint16_t>((size_t)total * H * d * 2);
-  w.ki = c.take<uint16_t>((size_t)total * Hkv * d * 2);
-  w.vi = c.take<uint16_t>((size_t)total * Hkv * d * 2);
+  w.nslot = qat_nslot(total, nseq);
+  const size_t T = qt_tile_bytes(d);
+  w.qt = c.take<uint8_t>((size_t)w.nslot * H * T);
+  w.kt = c.take<uint8_t>((size_t)w.nslot * Hkv * T);
+  w.vt = c.take<uint8_t>((size_t)w.nslot * Hkv * T);
+  w.dot = c.take<uint8_t>((size_t)w.nslot * H * T);
   w.amax = c.take<uint32_t>(16);
   w.g = c.take<float>(16);
   w.dsum = c.take<float>((size_t)total * H * 4);
@@ -654,8 +659,22 @@ QatWs carve_qat(void* base, int64_t total, int H, int Hkv, int d) {
   return w;
 }
 
+template <int DT, bool SS, int D>
+void qat_fq_tiles(const void* q, const void* k, const void* v, SeqInfo si, int nseq, int maxlen,
+                  int H, int Hkv, const QatWs& w, cudaStream_t st) {
+  const unsigned nt = (unsigned)ceil_div(maxlen, 128);
+  const auto* qp = static_cast<const uint16_t*>(q);
+  const auto* kp = static_cast<const uint16_t*>(k);
+  const auto* vp = static_cast<const uint16_t*>(v);
+  qat_fq_tile_kernel<DT, SS, D, false><<<dim3(nt, H, nseq), kThreads, 0, st>>>(
+      qp, si, H, w.nslot, w.amax, w.g, w.qt);
+  qat_fq_tile_kernel<DT, SS, D, false><<<dim3(nt, Hkv, nseq), kThreads, 0, st>>>(
+      kp, si, Hkv, w.nslot, w.amax + 1, w.g + 1, w.kt);
+  qat_fq_tile_kernel<DT, SS, D, true><<<dim3(nt, Hkv, nseq), kThreads, 0, st>>>(
+      vp, si, Hkv, w.nslot, w.amax + 2, w.g + 2, w.vt);
+}
 
-// Fake-quantised images of Q, K, V and their tensor scales.
+// Fake-quantised tiles of Q, K, V and their tensor scales.
 template <int DT>
 thrift_status qat_images(const void* q, const void* k, const void* v, SeqInfo si, int nseq,
                          int64_t total, int maxlen, int H, int Hkv, int d, int ss, const QatWs& w,
@@ -664,20 +683,12 @@ thrift_status qat_images(const void* q, const void* k, const void* v, SeqInfo si
   launch_amax<DT>(q, total * H * d / 16, 0, w.amax + 0, st);
   launch_amax<DT>(k, total * Hkv * d / 16, 0, w.amax + 1, st);
   launch_amax<DT>(v, total * Hkv * d / 16, 0, w.amax + 2, st);
-  const auto* qp = static_cast<const uint16_t*>(q);
-  const auto* kp = static_cast<const uint16_t*>(k);
-  const auto* vp = static_cast<const uint16_t*>(v);
-  const int64_t nq = total * H * d / 16, nk = total * Hkv * d / 16;
-  if (ss) {
-    qat_fq_rows_kernel<DT, true><<<grid_for(nq), kThreads, 0, st>>>(qp, nq, w.amax, w.g, w.qi);
-    qat_fq_rows_kernel<DT, true><<<grid_for(nk), kThreads, 0, st>>>(kp, nk, w.amax + 1, w.g + 1, w.ki);
-    qat_fq_v_kernel<DT, true><<<dim3((unsigned)ceil_div(maxlen, 16), nseq), kThreads, 0, st>>>(
-        vp, si, Hkv * d, w.amax + 2, w.g + 2, w.vi);
+  if (d == 128) {
+    if (ss) qat_fq_tiles<DT, true, 128>(q, k, v, si, nseq, maxlen, H, Hkv, w, st);
+    else qat_fq_tiles<DT, false, 128>(q, k, v, si, nseq, maxlen, H, Hkv, w, st);
   } else {
-    qat_fq_rows_kernel<DT, false><<<grid_for(nq), kThreads, 0, st>>>(qp, nq, w.amax, w.g, w.qi);
-    qat_fq_rows_kernel<DT, false><<<grid_for(nk), kThreads, 0, st>>>(kp, nk, w.amax + 1, w.g + 1, w.ki);
-    qat_fq_v_kernel<DT, false><<<dim3((unsigned)ceil_div(maxlen, 16), nseq), kThreads, 0, st>>>(
-        vp, si, Hkv * d, w.amax + 2, w.g + 2, w.vi);
+    if (ss) qat_fq_tiles<DT, true, 64>(q, k, v, si, nseq, maxlen, H, Hkv, w, st);
+    else qat_fq_tiles<DT, false, 64>(q, k, v, si, nseq, maxlen, H, Hkv, w, st);
   }
   return launch_status();
 }
@@ -685,32 +696,32 @@ thrift_status qat_images(const void* q, const void* k, const void* v, SeqInfo si
 template <int DT, int D, int BLK>
 thrift_status qat_fwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
   static DeviceSet attr;
-  const size_t smem = QatFwdSmem<D, BLK>::BYTES;
+  const size_t smem = QtFwdLayout<D>::SMEM_ALLOC;
   if (!smem_attr(qat_fwd_kernel<DT, D, BLK>, smem, attr)) return THRIFT_ERR_CUDA;
-  const dim3 grid((unsigned)(ceil_div(maxlen, kQatFwdRows) * p.H), nseq);
+  const dim3 grid((unsigned)(ceil_div(maxlen, 128) * p.H), nseq);
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
-  qat_fwd_kernel<DT, D, BLK><<<grid, 256, smem, st>>>(p);
+  qat_fwd_kernel<DT, D, BLK><<<grid, kQtThreads, smem, st>>>(p);
   const thrift_status s = launch_status();
   if (ev) cudaEventRecord(ev[1], st);
   return s;
 }
 
 template <int DT, int D, int BLK>
-thrift_status qat_bwd_launch(const QatParams& p, int nseq, int maxlen, cudaStream_t st) {
+thrift_status qat_bwd_launch(const QatParams& p, const void* dout, int nseq, int maxlen,
+                             cudaStream_t st) {
   static DeviceSet attr_kv, attr_q;
-  const size_t skv = QatKvSmem<D, BLK>::BYTES, sq = QatQSmem<D>::BYTES;
+  const size_t skv = QtKvLayout<D>::SMEM_ALLOC, sq = QtQLayout<D>::SMEM_ALLOC;
   if (!smem_attr(qat_bwd_kv_kernel<DT, D, BLK>, skv, attr_kv)) return THRIFT_ERR_CUDA;
   if (!smem_attr(qat_bwd_q_kernel<DT, D>, sq, attr_q)) return THRIFT_ERR_CUDA;
-  const int64_t rows = p.total * p.H;
-  qat_rowdot_kernel<DT, D><<<grid_for(rows * 32), kThreads, 0, st>>>(p.dout, p.out_hp, p.total,
-                                                                    p.H, const_cast<float*>(p.dsum));
+  const unsigned nt = (unsigned)ceil_div(maxlen, 128);
+  qat_rowdot_tile_kernel<DT, D><<<dim3(nt, p.H, nseq), kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(dout), p.out_hp, p.si, p.H, p.total, p.nslot,
+      const_cast<float*>(p.dsum), const_cast<uint8_t*>(p.dot));
   cudaEvent_t* ev = g_timer.enabled ? g_timer.next_pair() : nullptr;
   if (ev) cudaEventRecord(ev[0], st);
-  qat_bwd_kv_kernel<DT, D, BLK><<<dim3((unsigned)(ceil_div(maxlen, BLK) * p.Hkv), nseq), BLK * 2,
-                                  skv, st>>>(p);
-  qat_bwd_q_kernel<DT, D><<<dim3((unsigned)(ceil_div(maxlen, kQatRows) * p.H), nseq), 128, sq,
-                            st>>>(p);
+  qat_bwd_kv_kernel<DT, D, BLK><<<dim3(nt * p.Hkv, nseq), kQtThreads, skv, st>>>(p);
+  qat_bwd_q_kernel<DT, D><<<dim3(nt * p.H, nseq), kQtThreads, sq, st>>>(p);
   const thrift_status s = launch_status();
   if (ev) cudaEventRecord(ev[1], st);
   return s;
@@ -726,12 +737,12 @@ thrift_status qat_fwd_dispatch(const QatParams& p, int nseq, int maxlen, int d, 
 }
 
 template <int DT>
-thrift_status qat_bwd_dispatch(const QatParams& p, int nseq, int maxlen, int d, int blk,
-                               cudaStream_t st) {
-  if (d == 128 && blk == 128) return qat_bwd_launch<DT, 128, 128>(p, nseq, maxlen, st);
-  if (d == 128 && blk == 64) return qat_bwd_launch<DT, 128, 64>(p, nseq, maxlen, st);
-  if (d == 64 && blk == 128) return qat_bwd_launch<DT, 64, 128>(p, nseq, maxlen, st);
-  return qat_bwd_launch<DT, 64, 64>(p, nseq, maxlen, st);
+thrift_status qat_bwd_dispatch(const QatParams& p, const void* dout, int nseq, int maxlen, int d,
+                               int blk, cudaStream_t st) {
+  if (d == 128 && blk == 128) return qat_bwd_launch<DT, 128, 128>(p, dout, nseq, maxlen, st);
+  if (d == 128 && blk == 64) return qat_bwd_launch<DT, 128, 64>(p, dout, nseq, maxlen, st);
+  if (d == 64 && blk == 128) return qat_bwd_launch<DT, 64, 128>(p, dout, nseq, maxlen, st);
+  return qat_bwd_launch<DT, 64, 64>(p, dout, nseq, maxlen, st);
 }
 
 thrift_status check_qat_args(const void* q, const void* k, const void* v, int dt,
@@ -744,7 +755,7 @@ thrift_status check_qat_args(const void* q, const void* k, const void* v, int dt
   if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
   if (blk != 64 && blk != 128) return THRIFT_ERR_UNSUPPORTED;
   if (H > 65535 || nseq > 65535) return THRIFT_ERR_UNSUPPORTED;
-  if (ws_bytes < carve_qat(nullptr, total, H, Hkv, d).bytes) return THRIFT_ERR_ARG;
+  if (ws_bytes < carve_qat(nullptr, total, nseq, H, Hkv, d).bytes) return THRIFT_ERR_ARG;
   return THRIFT_OK;
 }
 
@@ -1163,9 +1174,9 @@ thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, i
 
 // ------------------------------------------------------------ Attn-QAT --
 
-size_t thrift_qat_workspace_size(int64_t total, int H, int Hkv, int d) {
-  if (total <= 0 || H <= 0 || Hkv <= 0 || (d != 64 && d != 128)) return 0;
-  return carve_qat(nullptr, total, H, Hkv, d).bytes;
+size_t thrift_qat_workspace_size(int64_t total, int nseq, int H, int Hkv, int d) {
+  if (total <= 0 || nseq <= 0 || H <= 0 || Hkv <= 0 || (d != 64 && d != 128)) return 0;
+  return carve_qat(nullptr, total, nseq, H, Hkv, d).bytes;
 }
 
 thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v, thrift_dtype dt,
@@ -1178,12 +1189,13 @@ thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v,
   if (s != THRIFT_OK) return s;
   if (!out || !out_hp || !lse || !aligned16(out) || !aligned16(out_hp)) return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const QatWs w = carve_qat(workspace, total, H, Hkv, d);
+  const QatWs w = carve_qat(workspace, total, nseq, H, Hkv, d);
   const SeqInfo si{cu_seqlens, 0};
   QatParams p{};
-  p.qi = w.qi;
-  p.ki = w.ki;
-  p.vi = w.vi;
+  p.qt = w.qt;
+  p.kt = w.kt;
+  p.vt = w.vt;
+  p.nslot = w.nslot;
   p.g = w.g;
   p.si = si;
   p.H = H;
@@ -1215,13 +1227,14 @@ thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v,
   if (!aligned16(dout) || !aligned16(out_hp) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return THRIFT_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const QatWs w = carve_qat(workspace, total, H, Hkv, d);
+  const QatWs w = carve_qat(workspace, total, nseq, H, Hkv, d);
   const SeqInfo si{cu_seqlens, 0};
   QatParams p{};
-  p.qi = w.qi;
-  p.ki = w.ki;
-  p.vi = w.vi;
-  p.dout = static_cast<const uint16_t*>(dout);
+  p.qt = w.qt;
+  p.kt = w.kt;
+  p.vt = w.vt;
+  p.dot = w.dot;
+  p.nslot = w.nslot;
   p.g = w.g;
   p.si = si;
   p.H = H;
@@ -1238,11 +1251,11 @@ thrift_status thrift_qat_bwd_varlen(const void* q, const void* k, const void* v,
   if (dt == THRIFT_BF16) {
     if (!reuse_images)
       s = qat_images<1>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-    return s != THRIFT_OK ? s : qat_bwd_dispatch<1>(p, nseq, max_seqlen, d, blk, st);
+    return s != THRIFT_OK ? s : qat_bwd_dispatch<1>(p, dout, nseq, max_seqlen, d, blk, st);
   }
   if (!reuse_images)
     s = qat_images<0>(q, k, v, si, nseq, total, max_seqlen, H, Hkv, d, use_scalesearch, w, st);
-  return s != THRIFT_OK ? s : qat_bwd_dispatch<0>(p, nseq, max_seqlen, d, blk, st);
+  return s != THRIFT_OK ? s : qat_bwd_dispatch<0>(p, dout, nseq, max_seqlen, d, blk, st);
 }
 
 }  // extern "C"

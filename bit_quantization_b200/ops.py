@@ -106,7 +106,7 @@ def lib():
         L.thrift_attn_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, sz, P, P, f32,
                                          i32, i32, i32, P, P, P, sz, P]
         L.thrift_qat_workspace_size.restype = sz
-        L.thrift_qat_workspace_size.argtypes = [i64, i32, i32, i32]
+        L.thrift_qat_workspace_size.argtypes = [i64, i32, i32, i32, i32]
         L.thrift_qat_fwd_varlen.restype = i32
         L.thrift_qat_fwd_varlen.argtypes = [P, P, P, i32, P, i32, i64, i32, i32, i32, i32, i32,
                                             i32, i32, P, P, P, P, sz, P]
@@ -588,8 +588,10 @@ def thrift_attn_decode(q, cache: DoubleKVCache, topk_frac=0.0, sink_blocks=0, re
 
 # --------------------------------------------------------------- Attn-QAT --
 
-def qat_workspace_size(total, H, Hkv, d=128) -> int:
-    return int(lib().thrift_qat_workspace_size(int(total), H, Hkv, d))
+def qat_workspace_size(total, H, Hkv, d=128, nseq=1) -> int:
+    """Bytes of the Attn-QAT workspace for ``nseq`` packed sequences of
+    ``total`` tokens."""
+    return int(lib().thrift_qat_workspace_size(int(total), int(nseq), H, Hkv, d))
 
 
 def _qat_pack(q, k, v, cu_seqlens, max_seqlen):
@@ -625,7 +627,7 @@ def thrift_qat_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, blk=128, causal=Tr
     out = torch.empty_like(qp)
     out_hp = torch.empty(qp.shape, dtype=torch.float32, device=q.device)
     lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
-    need = qat_workspace_size(total, H, Hkv, d)
+    need = qat_workspace_size(total, H, Hkv, d, cu.numel() - 1)
     if need == 0:
         raise ThriftError("thrift_qat_fwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)
@@ -666,7 +668,7 @@ def thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu_seqlens=None, max_seqlen=None,
     dq = torch.empty(qp.shape, dtype=torch.float32, device=q.device)
     dk = torch.empty(kp.shape, dtype=torch.float32, device=q.device)
     dv = torch.empty(kp.shape, dtype=torch.float32, device=q.device)
-    need = qat_workspace_size(total, H, Hkv, d)
+    need = qat_workspace_size(total, H, Hkv, d, cu.numel() - 1)
     if need == 0:
         raise ThriftError("thrift_qat_bwd: unsupported shape")
     ws = workspace if workspace is not None else _ws.get(need, q.device)

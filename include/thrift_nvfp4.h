@@ -365,17 +365,20 @@ thrift_status thrift_attn_decode(const void* q, thrift_dtype dt, int B, int H, i
  * type (O), out_hp fp32 [total, H, d] (O'), lse fp32 [H, total] (natural
  * log); dq fp32 [total, H, d], dk, dv fp32 [total, Hkv, d].
  *
- * Workspace: thrift_qat_workspace_size(total, H, Hkv, d) bytes of device
- * memory, 16-byte aligned; it holds the fake-quantised images (each element
- * E2M1 value x UE4M3 block scale, exact in the input type), the tensor
- * scales and D.  thrift_qat_bwd_varlen with reuse_images != 0 takes the
+ * Workspace: thrift_qat_workspace_size(total, nseq, H, Hkv, d) bytes of
+ * device memory, 16-byte aligned; it holds the fake-quantised images of Q,
+ * K, V (each element E2M1 value x UE4M3 block scale, exact in the input
+ * type) and the dO image as 128-row operand tiles (total / 128 + nseq tiles
+ * per head), the tensor scales and D.  cu_seqlens must describe sequences
+ * that partition [0, total): the tile slots of a sequence are derived from
+ * its start.  thrift_qat_bwd_varlen with reuse_images != 0 takes the
  * images and scales from the workspace as a thrift_qat_fwd_varlen call on
  * the same q, k, v, flags and workspace left them; with 0 it recomputes them.
  *
  * Errors: THRIFT_ERR_ARG for null or misaligned pointers, bad shapes or a
  * short workspace (returned before any launch); THRIFT_ERR_CUDA if a launch
  * fails.  Asynchronous on `stream`. */
-size_t thrift_qat_workspace_size(int64_t total, int H, int Hkv, int d);
+size_t thrift_qat_workspace_size(int64_t total, int nseq, int H, int Hkv, int d);
 thrift_status thrift_qat_fwd_varlen(const void* q, const void* k, const void* v, thrift_dtype dt,
                                     const int32_t* cu_seqlens, int nseq, int64_t total,
                                     int max_seqlen, int H, int Hkv, int d, int blk, int causal,

@@ -139,11 +139,14 @@ def test_qat_entry_points_check_arguments_before_launch(L):
     any launch (no device needed)."""
     P = C.c_void_p
     dummy, ws, big = P(4096), P(8192), 1 << 40
-    size = L.thrift_qat_workspace_size(1000, 8, 2, 128)
-    # three images in the input type, 2 x 16-byte scalars, D in fp32 (1024-byte slices)
-    assert size >= 1000 * (8 + 2 + 2) * 128 * 2 + 1000 * 8 * 4
-    assert L.thrift_qat_workspace_size(1000, 8, 2, 96) == 0
-    assert L.thrift_qat_workspace_size(0, 8, 2, 128) == 0
+    size = L.thrift_qat_workspace_size(1000, 2, 8, 2, 128)
+    # 128-row tiles of Q, K, V and dO (1000 // 128 + 2 slots a head), 2 x
+    # 16-byte scalars, D in fp32 (1024-byte slices)
+    assert size >= (1000 // 128 + 2) * (8 + 2 + 2 + 8) * 128 * 128 * 2 + 1000 * 8 * 4
+    assert L.thrift_qat_workspace_size(1000, 3, 8, 2, 128) > size
+    assert L.thrift_qat_workspace_size(1000, 2, 8, 2, 96) == 0
+    assert L.thrift_qat_workspace_size(0, 2, 8, 2, 128) == 0
+    assert L.thrift_qat_workspace_size(1000, 0, 8, 2, 128) == 0
 
     def fwd(d=128, blk=128, H=8, Hkv=2, q=dummy, cu=dummy, wsb=big, out=dummy):
         return L.thrift_qat_fwd_varlen(q, dummy, dummy, 1, cu, 2, 1000, 600, H, Hkv, d, blk, 1, 0,

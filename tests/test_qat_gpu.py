@@ -41,8 +41,8 @@ def _run_gpu(inp, w, reuse=False):
     q, k, v, dout = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
     cu = inp["cu_seqlens"].cuda()
     maxlen = max(inp["lengths"])
-    ws = torch.empty(ops.qat_workspace_size(q.shape[0], w.H, w.Hkv, w.d), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(ops.qat_workspace_size(q.shape[0], w.H, w.Hkv, w.d, cu.numel() - 1),
+                     dtype=torch.uint8, device="cuda")
     out, out_hp, lse = ops.thrift_qat_fwd(q, k, v, cu, maxlen, blk=w.blk, causal=w.causal,
                                           use_scalesearch=w.use_scalesearch, workspace=ws)
     dq, dk, dv = ops.thrift_qat_bwd(q, k, v, dout, out_hp, lse, cu, maxlen, blk=w.blk,
