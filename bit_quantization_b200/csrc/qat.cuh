@@ -59,6 +59,7 @@ namespace thrift {
 
 constexpr float kQatLog2e = 1.4426950408889634f;
 constexpr float kQatLn2 = 0.6931471805599453f;
+constexpr float kLog2TensorScaleDiv = 11.392317422778761f;  // log2(2688)
 
 constexpr int kQtWarps = 8;             // row-owning warps, two per lane quarter
 constexpr int kQtProducer = kQtWarps;   // warp 8
@@ -66,6 +67,7 @@ constexpr int kQtMma = kQtWarps + 1;    // warp 9
 constexpr int kQtThreads = 32 * (kQtWarps + 2);
 constexpr uint32_t kQtPTile = 128u * 128u * 2u;  // [128][128] 16-bit
 constexpr uint32_t kQtShBytes = 2048;            // barriers, flags, tables
+constexpr int kQtRing = 4;                       // K/V tile slots of the forward
 
 __host__ __device__ constexpr uint32_t qt_tile_bytes(int d) { return 128u * (uint32_t)d * 2u; }
 __host__ __device__ constexpr int64_t qat_nslot(int64_t total, int nseq) {
@@ -247,10 +249,14 @@ struct PBlock {
     dec = ue4m3_decode(sp);
     rr = rcp[sp];
   }
-  __device__ __forceinline__ void apply(float x0, float x1, float& q0, float& q1) const {
+  // The 16-bit pair of the FP4 values of x0, x1 times t (t = sigma): the
+  // code values times (block scale x t), 0 for a zero block.
+  template <int DT>
+  __device__ __forceinline__ uint32_t scaled(float x0, float x1, float t) const {
+    float q0, q1;
     e2m1x2_roundtrip(__fmul_rn(x0, rr), __fmul_rn(x1, rr), q0, q1);
-    q0 = zero ? 0.0f : __fmul_rn(q0, dec);
-    q1 = zero ? 0.0f : __fmul_rn(q1, dec);
+    const float f = zero ? 0.0f : dec * t;
+    return pack2<DT>(q0 * f, q1 * f);
   }
 };
 
@@ -277,8 +283,14 @@ __device__ __forceinline__ void qt_store32(uint8_t* tile, int r, int c0, const u
         make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
+// Stores 16 consecutive 16-bit values (columns c0..c0+15, c0 % 16 == 0).
+__device__ __forceinline__ void qt_store16(uint8_t* tile, int r, int c0, const uint32_t (&w)[8]) {
+  *reinterpret_cast<uint4*>(tile + qt_elem(r, c0)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(tile + qt_elem(r, c0 + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 // Shared-memory control block of the attention kernels (kQtShBytes):
-// barriers [0, 128), the lane quarters' pair barriers [128, 160), the
+// barriers [0, 192), the lane quarters' pair barriers [192, 224), the
 // tensor-memory base and the abort flag, the UE4M3 reciprocals [256, 768),
 // the pair exchange [1024, 2048).
 struct QtShared {
@@ -290,19 +302,21 @@ struct QtShared {
   float* xch;
 };
 
-// many_mask: the barriers every row-owning thread arrives on (count 256);
-// the others complete on one arrival or an MMA commit.
-__device__ __forceinline__ QtShared qt_setup(uint8_t* sh, int nbar, uint32_t many_mask) {
+// m256: the barriers every row-owning thread arrives on (count 256); m128:
+// those one half of them (four warps) arrives on; the others complete on one
+// arrival or an MMA commit.
+__device__ __forceinline__ QtShared qt_setup(uint8_t* sh, int nbar, uint32_t m256,
+                                             uint32_t m128) {
   QtShared s;
   s.bars = reinterpret_cast<uint64_t*>(sh);
-  s.xbar = reinterpret_cast<uint64_t*>(sh + 128);
-  s.tmem = reinterpret_cast<uint32_t*>(sh + 160);
-  s.abort = reinterpret_cast<volatile int*>(sh + 164);
+  s.xbar = reinterpret_cast<uint64_t*>(sh + 192);
+  s.tmem = reinterpret_cast<uint32_t*>(sh + 224);
+  s.abort = reinterpret_cast<volatile int*>(sh + 228);
   s.rcp = reinterpret_cast<float*>(sh + 256);
   s.xch = reinterpret_cast<float*>(sh + 1024);
   if (threadIdx.x == 0) {
     for (int i = 0; i < nbar; ++i)
-      mbar_init(&s.bars[i], ((many_mask >> i) & 1u) ? kQtWarps * 32 : 1);
+      mbar_init(&s.bars[i], ((m256 >> i) & 1u) ? 256 : (((m128 >> i) & 1u) ? 128 : 1));
     for (int i = 0; i < 4; ++i) mbar_init(&s.xbar[i], 64);
     *s.abort = 0;
     fence_mbar_init();
@@ -347,20 +361,39 @@ __device__ __forceinline__ bool qt_pair_swap(const QtShared& s, int quarter, int
   return ok;
 }
 
-// Largest raw score of 32 columns over the visible keys (key0 + i < klim);
-// -inf when none is visible.  tcgen05.ld is warp-wide: called by all lanes.
+// Raw scores of keys key0..key0+31 with the invisible ones (key >= klim)
+// set to -inf; the compare runs only where a lane of the warp needs it.
+__device__ __forceinline__ void qt_mask32(float (&a)[32], int key0, int klim) {
+  if (!__all_sync(0xffffffffu, key0 + 32 <= klim)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = key0 + i < klim ? a[i] : -INFINITY;
+  }
+}
+
+// Largest raw score of 32 columns over the visible keys; -inf when none is
+// visible.  tcgen05.ld is warp-wide: called by all lanes.
 __device__ __forceinline__ float qt_chunk_max(uint32_t taddr, int key0, int klim) {
   float a[32];
   tmem_ld32(taddr, a);
   tmem_ld_wait();
-  float mx = -INFINITY;
-  if (__all_sync(0xffffffffu, key0 + 32 <= klim)) {
+  qt_mask32(a, key0, klim);
+  float mx = a[0];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, a[i]);
-  } else {
+  for (int i = 1; i < 32; ++i) mx = fmaxf(mx, a[i]);
+  return mx;
+}
+
+// Largest raw score of 64 columns (two loads, one wait).
+__device__ __forceinline__ float qt_max64(uint32_t taddr, int key0, int klim) {
+  float a[32], b[32];
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld_wait();
+  qt_mask32(a, key0, klim);
+  qt_mask32(b, key0 + 32, klim);
+  float mx = fmaxf(a[0], b[0]);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, key0 + i < klim ? a[i] : -INFINITY);
-  }
+  for (int i = 1; i < 32; ++i) mx = fmaxf(mx, fmaxf(a[i], b[i]));
   return mx;
 }
 
@@ -374,19 +407,56 @@ __device__ __forceinline__ uint8_t* qt_smem_base() {
 template <int D>
 struct QtFwdLayout {
   static constexpr uint32_t T = qt_tile_bytes(D);
-  static constexpr uint32_t Q = 0, K = T, V = 3 * T, P = 4 * T;  // K: 2 stages
-  static constexpr uint32_t PH = P + kQtPTile, PL = PH + kQtPTile, SH = PL + kQtPTile;
+  static constexpr uint32_t Q = 0, RING = T, P = (1 + kQtRing) * T;  // RING: K or V tiles
+  static constexpr uint32_t SH = P + kQtPTile;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
-  static constexpr uint32_t T_S = 0, T_O = 256, T_OH = 256 + D;  // S: 2 slots
-  static_assert(T_OH + D <= 512, "tensor memory budget");
+  // S slot 0; slot 1 (pass A only) is the columns O and O' take in pass B;
+  // P hi and lo (the A operand of O' += P V^, two 16-bit values a column)
+  static constexpr uint32_t T_S = 0, T_S1 = 128, T_O = 128, T_OH = 128 + D;
+  static constexpr uint32_t T_PH = 384, T_PL = 448;
+  static_assert(T_OH + D <= T_PH, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// The K and V tiles of a forward CTA pass through one ring of kQtRing slots
+// in the order the MMAs read them: K(0..nt-1) for pass A, then K(0), and for
+// each key tile j: K(j+1) (when j+1 < nt), V(j).  Item i sits in slot
+// i % kQtRing; V(j+1) loads during the products of tile j at the latest.
+__device__ __forceinline__ int qt_ring_item(int i, int nt, bool& is_v) {
+  is_v = false;
+  if (i < nt) return i;
+  if (i == nt) return 0;
+  const int q = i - nt - 1;
+  if (q == 2 * (nt - 1)) {
+    is_v = true;
+    return nt - 1;
+  }
+  is_v = (q & 1) != 0;
+  return is_v ? (q >> 1) : (q >> 1) + 1;
+}
+// Ring index of the K tile of step u and of V(j).
+__device__ __forceinline__ int qt_ring_k(int u, int nt) {
+  return u <= nt ? u : nt + 2 * (u - nt) - 1;
+}
+__device__ __forceinline__ int qt_ring_v(int j, int nt) {
+  return j == nt - 1 ? 3 * nt - 1 : nt + 2 * j + 2;
+}
+
+// RF + s / RE + s: ring slot s loaded / free; FSF + t / FSE + t: S slot t
+// written / read; FPF + h / FPE + h: key half h (keys 64h..64h+63) of P^
+// and of P's two parts written / consumed by the products.
 enum : int {
-  FQ = 0, FKF = 1 /* 1,2 */, FKE = 3 /* 3,4 */, FVF = 5, FVE = 6, FSF = 7 /* 7,8 */,
-  FSE = 9 /* 9,10 */, FPF = 11, FPE = 12, FDONE = 13, FN = 14
+  FQ = 0, RF = 1 /* 1..4 */, RE = 5 /* 5..8 */, FSF = 9 /* 9,10 */,
+  FSE = 11 /* 11,12 */, FPF = 13 /* 13,14 */, FPE = 15 /* 15,16 */, FDONE = 17, FN = 18
 };
-constexpr uint32_t kFwdMany = (1u << FSE) | (1u << (FSE + 1)) | (1u << FPF);
+// S slot of step u and how many earlier steps used it: pass A alternates
+// the two slots, pass B uses slot 0 only.
+__device__ __forceinline__ int qt_s_slot(int u, int nt) { return u < nt ? (u & 1) : 0; }
+__device__ __forceinline__ int qt_s_use(int u, int nt) {
+  return u < nt ? (u >> 1) : ((nt + 1) >> 1) + (u - nt);
+}
+constexpr uint32_t kFwd256 = (1u << FSE) | (1u << (FSE + 1));
+constexpr uint32_t kFwd128 = (1u << FPF) | (1u << (FPF + 1));
 
 // grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads; causal grids
 // start the query tiles with the most keys.  Steps u < nt are pass A over
@@ -407,7 +477,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
   const int q0 = qt * 128;
   const int kend = p.causal ? min(len, q0 + 128) : len;
   const int nt = (kend + 127) / 128, nsteps = 2 * nt;
-  const QtShared S = qt_setup(sm + L::SH, FN, kFwdMany);
+  const QtShared S = qt_setup(sm + L::SH, FN, kFwd256, kFwd128);
   uint64_t* bars = S.bars;
   const uint32_t tmem = *S.tmem;
 
@@ -417,24 +487,23 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
       const uint8_t* vbase = p.vt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
       mbar_arrive_expect_tx(&bars[FQ], L::T);
       bulk_g2s(sm + L::Q, p.qt + qat_slot(h, p.nslot, st, seq, qt) * L::T, L::T, &bars[FQ]);
-      int lastk[2] = {-1, -1}, lastv = -1;
-      for (int u = 0; u < nsteps && !*S.abort; ++u) {
-        const int j = u < nt ? u : u - nt, sl = u & 1;
-        if (u >= 2 && !mbar_wait(&bars[FKE + sl], ((u >> 1) - 1) & 1, S.abort)) break;
-        mbar_arrive_expect_tx(&bars[FKF + sl], L::T);
-        bulk_g2s(sm + L::K + sl * L::T, kbase + (int64_t)j * L::T, L::T, &bars[FKF + sl]);
-        lastk[sl] = u;
-        if (u >= nt) {
-          if (j >= 1 && !mbar_wait(&bars[FVE], (j - 1) & 1, S.abort)) break;
-          mbar_arrive_expect_tx(&bars[FVF], L::T);
-          bulk_g2s(sm + L::V, vbase + (int64_t)j * L::T, L::T, &bars[FVF]);
-          lastv = j;
-        }
+      const int nitems = 3 * nt;
+      int last[kQtRing];
+#pragma unroll
+      for (int sl = 0; sl < kQtRing; ++sl) last[sl] = -1;
+      for (int i = 0; i < nitems && !*S.abort; ++i) {
+        const int sl = i % kQtRing;
+        if (i >= kQtRing && !mbar_wait(&bars[RE + sl], (i / kQtRing - 1) & 1, S.abort)) break;
+        bool is_v;
+        const int t = qt_ring_item(i, nt, is_v);
+        mbar_arrive_expect_tx(&bars[RF + sl], L::T);
+        bulk_g2s(sm + L::RING + sl * L::T, (is_v ? vbase : kbase) + (int64_t)t * L::T, L::T,
+                 &bars[RF + sl]);
+        last[sl] = i;
       }
       qt_drain(&bars[FQ], 0);
-      for (int sl = 0; sl < 2; ++sl)
-        if (lastk[sl] >= 0) qt_drain(&bars[FKF + sl], (lastk[sl] >> 1) & 1);
-      if (lastv >= 0) qt_drain(&bars[FVF], lastv & 1);
+      for (int sl = 0; sl < kQtRing; ++sl)
+        if (last[sl] >= 0) qt_drain(&bars[RF + sl], (last[sl] / kQtRing) & 1);
     }
   } else if (warp == kQtMma) {
     if (lane == 0) {
@@ -442,16 +511,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
       constexpr uint32_t idPV = idesc_f16(DT, 128, D) | kIdescBmn;
       const uint32_t base = smem_u32(sm);
       auto issue_s = [&](int u) -> bool {
-        const int sl = u & 1;
-        if (!mbar_wait(&bars[FKF + sl], (u >> 1) & 1, S.abort)) return false;
-        if (u >= 2 && !mbar_wait(&bars[FSE + sl], ((u >> 1) - 1) & 1, S.abort)) return false;
+        const int sl = qt_s_slot(u, nt), use = qt_s_use(u, nt);
+        const int i = qt_ring_k(u, nt), rs = i % kQtRing;
+        if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) return false;
+        // the previous scores in this slot have been read
+        if (use >= 1 && !mbar_wait(&bars[FSE + sl], (use - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S + sl * 128, qt_desc_k(base + L::Q, s),
-                  qt_desc_k(base + L::K + sl * L::T, s), idS, s > 0);
+          mma_f16(tmem + (sl ? L::T_S1 : L::T_S), qt_desc_k(base + L::Q, s),
+                  qt_desc_k(base + L::RING + rs * L::T, s), idS, s > 0);
         tc_commit(&bars[FSF + sl]);
-        tc_commit(&bars[FKE + sl]);
+        tc_commit(&bars[RE + rs]);
         return true;
       };
       bool ok = mbar_wait(&bars[FQ], 0, S.abort) && issue_s(0);
@@ -459,18 +530,26 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
         // the next tile's scores go ahead of this tile's products
         if (u + 1 < nsteps && !issue_s(u + 1)) break;
         if (u < nt) continue;
-        const int j = u - nt;
-        if (!mbar_wait(&bars[FPF], j & 1, S.abort) || !mbar_wait(&bars[FVF], j & 1, S.abort)) break;
-        tc_fence_after();
+        const int j = u - nt, i = qt_ring_v(j, nt), rs = i % kQtRing;
+        if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) break;
+        const uint32_t vt = base + L::RING + rs * L::T;
+        bool fine = true;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint64_t bv = qt_desc_mn(base + L::V, s);
-          mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
-          mma_f16(tmem + L::T_OH, qt_desc_k(base + L::PH, s), bv, idPV, j > 0 || s > 0);
-          mma_f16(tmem + L::T_OH, qt_desc_k(base + L::PL, s), bv, idPV, 1);
+        for (int hf = 0; hf < 2 && fine; ++hf) {
+          // the products of a key half start once its warps have written it
+          if (!mbar_wait(&bars[FPF + hf], j & 1, S.abort)) { fine = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int s = 4 * hf; s < 4 * hf + 4; ++s) {
+            const uint64_t bv = qt_desc_mn(vt, s);
+            mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
+            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PH + 8 * s, bv, idPV, j > 0 || s > 0);
+            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PL + 8 * s, bv, idPV, 1);
+          }
+          tc_commit(&bars[FPE + hf]);
         }
-        tc_commit(&bars[FPE]);
-        tc_commit(&bars[FVE]);
+        if (!fine) break;
+        tc_commit(&bars[RE + rs]);
       }
       tc_commit(&bars[FDONE]);
       qt_drain(&bars[FDONE], 0);
@@ -487,14 +566,11 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
     // pass A: the row maximum over this warp's columns, then the pair's
     float mraw = -INFINITY;
     for (int u = 0; u < nt && ok; ++u) {
-      const int sl = u & 1;
-      if (!warp_wait(&bars[FSF + sl], (u >> 1) & 1, S.abort)) { ok = false; break; }
+      const int sl = qt_s_slot(u, nt);
+      if (!warp_wait(&bars[FSF + sl], qt_s_use(u, nt) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int col = 64 * half + 32 * cc;
-        mraw = fmaxf(mraw, qt_chunk_max(tl + L::T_S + sl * 128 + col, u * 128 + col, klim));
-      }
+      mraw = fmaxf(mraw, qt_max64(tl + (sl ? L::T_S1 : L::T_S) + 64 * half, u * 128 + 64 * half,
+                                  klim));
       tc_fence_before();
       mbar_arrive(&bars[FSE + sl]);
     }
@@ -506,76 +582,72 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
     // sub-tile's own maximum
     float lsum = 0.0f;
     uint8_t* tP = sm + L::P;
-    uint8_t* tH = sm + L::PH;
-    uint8_t* tL = sm + L::PL;
     for (int u = nt; u < nsteps && ok; ++u) {
-      const int sl = u & 1, j = u - nt, kb = j * 128;
-      const uint32_t ts = tl + L::T_S + sl * 128;
-      if (!warp_wait(&bars[FSF + sl], (u >> 1) & 1, S.abort)) { ok = false; break; }
+      const int sl = 0, j = u - nt, kb = j * 128, c0 = 64 * half;
+      const uint32_t ts = tl + L::T_S;
+      if (!warp_wait(&bars[FSF + sl], qt_s_use(u, nt) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
       float mt_raw = -INFINITY;
-      if constexpr (BLK == 128) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) mt_raw = fmaxf(mt_raw, qt_chunk_max(ts + 32 * c, kb + 32 * c, klim));
-      } else {
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col = 64 * half + 32 * cc;
-          mt_raw = fmaxf(mt_raw, qt_chunk_max(ts + col, kb + col, klim));
-        }
-      }
+      // a 128-key sub-tile takes the partner's columns into its maximum too
+      if constexpr (BLK == 128) mt_raw = qt_max64(ts + (c0 ^ 64), kb + (c0 ^ 64), klim);
+      float a[2][32];
+      tmem_ld32(ts + c0, a[0]);
+      tmem_ld32(ts + c0 + 32, a[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[FSE + sl]);
+      qt_mask32(a[0], kb + c0, klim);
+      qt_mask32(a[1], kb + c0 + 32, klim);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) mt_raw = fmaxf(mt_raw, fmaxf(a[0][i], a[1][i]));
       const bool live = mt_raw != -INFINITY;
-      const float mt = mt_raw * c2;
-      const float mtr = live ? mt : 0.0f;
-      const float fct = live ? ex2_ftz(mt - mref) * (1.0f / kTensorScaleDiv) : 0.0f;
-      // the P tiles are free once the products of the previous tile are done
-      if (j >= 1 && !warp_wait(&bars[FPE], (j - 1) & 1, S.abort)) { ok = false; break; }
-#pragma unroll 1
+      // P / sigma of the sub-tile = 2688 exp(S - max_tile S) = 2^(s c2 + off);
+      // P = that times fct = 2^(mt - m) / 2688 (the sub-tile's sigma relative
+      // to the row's)
+      const float off = live ? kLog2TensorScaleDiv - mt_raw * c2 : 0.0f;
+      const float fct = live ? ex2_ftz(mt_raw * c2 - mref) * (1.0f / kTensorScaleDiv) : 0.0f;
+      // P^ and the two parts of P in registers first: they are written (P^ to
+      // shared memory, P to tensor memory) once the products of the previous
+      // tile have read their predecessors
+      uint32_t wq[2][16], wh[2][16], wl[2][16];
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int col = 64 * half + 32 * cc, key0 = kb + col;
-        float a[32];
-        tmem_ld32(ts + col, a);
-        tmem_ld_wait();
-        if (cc == 1) {
-          tc_fence_before();
-          mbar_arrive(&bars[FSE + sl]);
-        }
-        uint32_t wq[16], wh[16], wl[16];
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          float qv[16], pe[16];
+          float qv[16];
           float am = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int e = 16 * b + i;
-            const bool vis = key0 + e < klim;
-            const float s = a[e] * c2;
-            pe[i] = vis ? ex2_ftz(s - mref) : 0.0f;
-            // P / sigma of the tile: 2688 exp(S - max_tile S)
-            qv[i] = vis ? kTensorScaleDiv * ex2_ftz(s - mtr) : 0.0f;
-            lsum += pe[i];
+            qv[i] = ex2_ftz(fmaf(a[cc][16 * b + i], c2, off));
             am = fmaxf(am, qv[i]);
           }
           const PBlock pb(am, S.rcp);
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            float y0, y1;
-            pb.apply(qv[i], qv[i + 1], y0, y1);
-            wq[8 * b + i / 2] = pack2<DT>(__fmul_rn(y0, fct), __fmul_rn(y1, fct));
-            qt_split2<DT>(pe[i], pe[i + 1], wh[8 * b + i / 2], wl[8 * b + i / 2]);
+            wq[cc][8 * b + i / 2] = pb.scaled<DT>(qv[i], qv[i + 1], fct);
+            const float p0 = qv[i] * fct, p1 = qv[i + 1] * fct;
+            lsum += p0 + p1;
+            qt_split2<DT>(p0, p1, wh[cc][8 * b + i / 2], wl[cc][8 * b + i / 2]);
           }
         }
-        qt_store32(tP, r, col, wq);
-        qt_store32(tH, r, col, wh);
-        qt_store32(tL, r, col, wl);
+      }
+      if (j >= 1 && !warp_wait(&bars[FPE + half], (j - 1) & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        qt_store32(tP, r, c0 + 32 * cc, wq[cc]);
+        tmem_st16u(tl + L::T_PH + 32 * half + 16 * cc, wh[cc]);
+        tmem_st16u(tl + L::T_PL + 32 * half + 16 * cc, wl[cc]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars[FPF]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[FPF + half]);
     }
     // epilogue: O = P^ V^ g_V / l, O' = P V^ g_V / l, lse; the row sum l
-    // from both halves (after the last products, so the exchange slots are
-    // free)
-    if (ok) ok = warp_wait(&bars[FPE], (nt - 1) & 1, S.abort);
+    // from both halves (after the last products, when every warp is past
+    // the first exchange)
+    if (ok) ok = warp_wait(&bars[FDONE], 0, S.abort);
     float lo = 0.0f;
     if (ok) ok = qt_pair_swap(S, quarter, half, r, 1, lsum, lo);
     if (ok) {
@@ -619,18 +691,22 @@ template <int D>
 struct QtQLayout {
   static constexpr uint32_t T = qt_tile_bytes(D);
   static constexpr uint32_t Q = 0, DO = T, K = 2 * T, V = 4 * T;  // K: 2 stages, V: 1
-  static constexpr uint32_t DSH = 5 * T, DSL = DSH + kQtPTile, SH = DSL + kQtPTile;
+  static constexpr uint32_t SH = 5 * T;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
-  static_assert(T_DQ + D <= 512, "tensor memory budget");
+  // dS hi and lo: the A operand of dQ += dS K^ in tensor memory (64 columns
+  // each, two 16-bit values a column)
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DSH = 384, T_DSL = 448;
+  static_assert(T_DQ + D <= T_DSH, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// QPF + h / QPE + h: key half h of the dS tiles written / consumed.
 enum : int {
-  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSE = 8, QPF = 9,
-  QPE = 10, QDONE = 11, QN = 12
+  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSE = 8,
+  QPF = 9 /* 9,10 */, QPE = 11 /* 11,12 */, QDONE = 13, QN = 14
 };
-constexpr uint32_t kQMany = (1u << QSE) | (1u << QPF);
+constexpr uint32_t kQ256 = 1u << QSE;
+constexpr uint32_t kQ128 = (1u << QPF) | (1u << (QPF + 1));
 
 // grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads.
 template <int DT, int D>
@@ -649,7 +725,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
   const int q0 = qt * 128;
   const int kend = p.causal ? min(len, q0 + 128) : len;
   const int nt = (kend + 127) / 128;
-  const QtShared S = qt_setup(sm + L::SH, QN, kQMany);
+  const QtShared S = qt_setup(sm + L::SH, QN, kQ256, kQ128);
   uint64_t* bars = S.bars;
   const uint32_t tmem = *S.tmem;
 
@@ -704,16 +780,21 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
       bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0);
       for (int j = 0; j < nt && ok; ++j) {
         if (j + 1 < nt && !issue_s(j + 1)) break;
-        if (!mbar_wait(&bars[QPF], j & 1, S.abort)) break;
-        tc_fence_after();
         const uint32_t kt = base + L::K + (j & 1) * L::T;
+        bool fine = true;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint64_t bk = qt_desc_mn(kt, s);
-          mma_f16(tmem + L::T_DQ, qt_desc_k(base + L::DSH, s), bk, idDQ, j > 0 || s > 0);
-          mma_f16(tmem + L::T_DQ, qt_desc_k(base + L::DSL, s), bk, idDQ, 1);
+        for (int hf = 0; hf < 2 && fine; ++hf) {
+          if (!mbar_wait(&bars[QPF + hf], j & 1, S.abort)) { fine = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int s = 4 * hf; s < 4 * hf + 4; ++s) {
+            const uint64_t bk = qt_desc_mn(kt, s);
+            mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSH + 8 * s, bk, idDQ, j > 0 || s > 0);
+            mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSL + 8 * s, bk, idDQ, 1);
+          }
+          tc_commit(&bars[QPE + hf]);
         }
-        tc_commit(&bars[QPE]);
+        if (!fine) break;
         tc_commit(&bars[QKE + (j & 1)]);
       }
       tc_commit(&bars[QDONE]);
@@ -728,15 +809,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
     const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
     const float nlse2 = row_ok ? -p.lse[(int64_t)h * p.total + st + row] * kQatLog2e : 0.0f;
     const float dsum = row_ok ? p.dsum[(int64_t)h * p.total + st + row] : 0.0f;
-    uint8_t* tH = sm + L::DSH;
-    uint8_t* tL = sm + L::DSL;
     bool ok = true;
     for (int j = 0; j < nt && ok; ++j) {
       if (!warp_wait(&bars[QSF], j & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-      // the dS tiles are free once the products of the previous tile are done
-      if (j >= 1 && !warp_wait(&bars[QPE], (j - 1) & 1, S.abort)) { ok = false; break; }
-#pragma unroll 1
+      // dS of this warp's 64 keys in registers first: they go to tensor
+      // memory once the products of the previous tile have read it
+      uint32_t wh[2][16], wl[2][16];
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int col = 64 * half + 32 * cc, key0 = j * 128 + col;
         float a[32], dp[32];
@@ -747,24 +827,26 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
           tc_fence_before();
           mbar_arrive(&bars[QSE]);
         }
-        uint32_t wh[16], wl[16];
+        qt_mask32(a, key0, klim);
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float pr = key0 + i + e < klim ? ex2_ftz(fmaf(a[i + e], c2, nlse2)) : 0.0f;
-            ds[e] = pr * (dp[i + e] * gv - dsum);
-          }
-          qt_split2<DT>(ds[0], ds[1], wh[i / 2], wl[i / 2]);
+          const float d0 = ex2_ftz(fmaf(a[i], c2, nlse2)) * fmaf(dp[i], gv, -dsum);
+          const float d1 = ex2_ftz(fmaf(a[i + 1], c2, nlse2)) * fmaf(dp[i + 1], gv, -dsum);
+          qt_split2<DT>(d0, d1, wh[cc][i / 2], wl[cc][i / 2]);
         }
-        qt_store32(tH, r, col, wh);
-        qt_store32(tL, r, col, wl);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[QPF]);
+      if (j >= 1 && !warp_wait(&bars[QPE + half], (j - 1) & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        tmem_st16u(tl + L::T_DSH + 32 * half + 16 * cc, wh[cc]);
+        tmem_st16u(tl + L::T_DSL + 32 * half + 16 * cc, wl[cc]);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[QPF + half]);
     }
-    if (ok && warp_wait(&bars[QPE], (nt - 1) & 1, S.abort)) {
+    if (ok && warp_wait(&bars[QDONE], 0, S.abort)) {
       tc_fence_after();
       const float qscale = p.g[1] * p.sc;
       const int64_t base = ((st + (row_ok ? row : 0)) * p.H + h) * D;
@@ -799,13 +881,20 @@ struct QtKvLayout {
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-enum : int { KKV = 0, KQF = 1, KQE = 2, KSF = 3, KSE = 4, KPF = 5, KPE = 6, KDONE = 7, KN = 8 };
-constexpr uint32_t kKvMany = (1u << KSE) | (1u << KPF);
+// KQF / KOF: the Q / dO chunk loaded; KQE / KOE: the Q / dO chunk free
+// (its last product done); KSF / KDF: S / dP in tensor memory.
+enum : int {
+  KKV = 0, KQF = 1, KOF = 2, KQE = 3, KOE = 4, KSF = 5, KDF = 6, KSE = 7, KPF = 8, KPE = 9,
+  KDONE = 10, KN = 11
+};
+constexpr uint32_t kKv256 = (1u << KSE) | (1u << KPF);
 
 // grid (ceil(maxlen / 128) * Hkv, nseq), kQtThreads threads: key tile
 // blockIdx.x / Hkv (causal grids: the tiles with the most queries first).
 // Iteration it takes query chunk c0 + it % nch of query head
-// hk * grp + it / nch.
+// hk * grp + it / nch.  The products of a chunk run dK (dS^T Q^) before dV
+// (P^T dO), so the next Q chunk loads while dV runs, and the next dO chunk
+// while S and the maxima of the next chunk are computed.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatParams p) {
   using L = QtKvLayout<D>;
@@ -821,7 +910,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
   const int c0 = p.causal ? kt : 0;  // first query chunk that sees a key of the tile
   const int nch = (len + 127) / 128 - c0;
   const int n_it = grp * nch;
-  const QtShared S = qt_setup(sm + L::SH, KN, kKvMany);
+  const QtShared S = qt_setup(sm + L::SH, KN, kKv256, 0);
   uint64_t* bars = S.bars;
   const uint32_t tmem = *S.tmem;
 
@@ -831,17 +920,21 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       mbar_arrive_expect_tx(&bars[KKV], 2 * L::T);
       bulk_g2s(sm + L::K, p.kt + ks * L::T, L::T, &bars[KKV]);
       bulk_g2s(sm + L::V, p.vt + ks * L::T, L::T, &bars[KKV]);
-      int last = -1;
+      int lastq = -1, lasto = -1;
       for (int it = 0; it < n_it && !*S.abort; ++it) {
         const int64_t qs = qat_slot(hk * grp + it / nch, p.nslot, st, seq, c0 + it % nch);
         if (it >= 1 && !mbar_wait(&bars[KQE], (it - 1) & 1, S.abort)) break;
-        mbar_arrive_expect_tx(&bars[KQF], 2 * L::T);
+        mbar_arrive_expect_tx(&bars[KQF], L::T);
         bulk_g2s(sm + L::Q, p.qt + qs * L::T, L::T, &bars[KQF]);
-        bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[KQF]);
-        last = it;
+        lastq = it;
+        if (it >= 1 && !mbar_wait(&bars[KOE], (it - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[KOF], L::T);
+        bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[KOF]);
+        lasto = it;
       }
       qt_drain(&bars[KKV], 0);
-      if (last >= 0) qt_drain(&bars[KQF], last & 1);
+      if (lastq >= 0) qt_drain(&bars[KQF], lastq & 1);
+      if (lasto >= 0) qt_drain(&bars[KOF], lasto & 1);
     }
   } else if (warp == kQtMma) {
     if (lane == 0) {
@@ -854,67 +947,79 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
         if (it >= 1 && !mbar_wait(&bars[KSE], (it - 1) & 1, S.abort)) break;
         tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
+        for (int s = 0; s < D / 16; ++s)
           mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K, s), idS, s > 0);
+        tc_commit(&bars[KSF]);
+        if (!mbar_wait(&bars[KOF], it & 1, S.abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
           mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
                   s > 0);
-        }
-        tc_commit(&bars[KSF]);
+        tc_commit(&bars[KDF]);
         if (!mbar_wait(&bars[KPF], it & 1, S.abort)) break;
         tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q^: M = the 128 keys, K = the 128 queries
+        // dK += dS^T Q^, dV += P^T dO: M = the 128 keys, K = the 128 queries
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const uint64_t bq = qt_desc_mn(base + L::Q, s);
-          mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
-                  it > 0 || s > 0);
           mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSH, s), bq, idG, it > 0 || s > 0);
           mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSL, s), bq, idG, 1);
         }
-        tc_commit(&bars[KPE]);
         tc_commit(&bars[KQE]);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
+                  it > 0 || s > 0);
+        tc_commit(&bars[KOE]);
+        tc_commit(&bars[KPE]);
       }
       tc_commit(&bars[KDONE]);
       qt_drain(&bars[KDONE], 0);
     }
   } else {
     const int quarter = warp & 3, half = warp >> 2;
-    const int r = quarter * 32 + lane;
+    const int r = quarter * 32 + lane, cb = 64 * half;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
     uint8_t* tP = sm + L::P;
     uint8_t* tH = sm + L::DSH;
     uint8_t* tL = sm + L::DSL;
+    // -lse (log2 units) and D of this thread's query row in iteration it
+    auto row_stats = [&](int it, float& nl, float& dsv) {
+      const int hq = hk * grp + it / nch, row = (c0 + it % nch) * 128 + r;
+      const bool ok_row = row < len;
+      nl = ok_row ? -p.lse[(int64_t)hq * p.total + st + row] * kQatLog2e : 0.0f;
+      dsv = ok_row ? p.dsum[(int64_t)hq * p.total + st + row] : 0.0f;
+    };
+    float nl_next, ds_next;
+    row_stats(0, nl_next, ds_next);
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
-      const int hq = hk * grp + it / nch, row = (c0 + it % nch) * 128 + r;
-      const bool row_ok = row < len;
-      const int klim = row_ok ? (p.causal ? row + 1 : len) : 0;
-      const float nlse2 = row_ok ? -p.lse[(int64_t)hq * p.total + st + row] * kQatLog2e : 0.0f;
-      const float dsum = row_ok ? p.dsum[(int64_t)hq * p.total + st + row] : 0.0f;
+      const int row = (c0 + it % nch) * 128 + r;
+      const int klim = row < len ? (p.causal ? row + 1 : len) : 0;
+      const float nlse2 = nl_next, dsum = ds_next;
+      if (it + 1 < n_it) row_stats(it + 1, nl_next, ds_next);  // in flight meanwhile
       if (!warp_wait(&bars[KSF], it & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
       // sigma of this warp's BLK-key sub-tile: the largest P there / 2688
-      float cm_raw = -INFINITY;
+      float cm_raw = qt_max64(tl + L::T_S + cb, j0 + cb, klim);
       if constexpr (BLK == 128) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c)
-          cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + 32 * c, j0 + 32 * c, klim));
-      } else {
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col = 64 * half + 32 * cc;
-          cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + col, j0 + col, klim));
-        }
+        for (int c = 0; c < 2; ++c)
+          cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + (cb ^ 64) + 32 * c,
+                                              j0 + (cb ^ 64) + 32 * c, klim));
       }
       const float cm = cm_raw == -INFINITY ? 0.0f : ex2_ftz(fmaf(cm_raw, c2, nlse2));
       const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
       const float sig = __fdiv_rn(cm, kTensorScaleDiv);
+      if (!warp_wait(&bars[KDF], it & 1, S.abort)) { ok = false; break; }
       // the tiles are free once the products of the previous chunk are done
       if (it >= 1 && !warp_wait(&bars[KPE], (it - 1) & 1, S.abort)) { ok = false; break; }
+      tc_fence_after();
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
-        const int col = 64 * half + 32 * cc, key0 = j0 + col;
+        const int col = cb + 32 * cc, key0 = j0 + col;
         float a[32], dp[32];
         tmem_ld32(tl + L::T_S + col, a);
         tmem_ld32(tl + L::T_DP + col, dp);
@@ -923,38 +1028,37 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
           tc_fence_before();
           mbar_arrive(&bars[KSE]);
         }
-        uint32_t wq[16], wh[16], wl[16];
+        qt_mask32(a, key0, klim);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
           float pr[16], x[16];
           float am = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int e = 16 * b + i;
-            pr[i] = key0 + e < klim ? ex2_ftz(fmaf(a[e], c2, nlse2)) : 0.0f;
-            x[i] = __fmul_rn(pr[i], inv);
+            pr[i] = ex2_ftz(fmaf(a[16 * b + i], c2, nlse2));
+            x[i] = pr[i] * inv;
             am = fmaxf(am, x[i]);
           }
           const PBlock pb(am, S.rcp);
+          uint32_t wq[8], wh[8], wl[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            float y0, y1;
-            pb.apply(x[i], x[i + 1], y0, y1);
-            wq[8 * b + i / 2] = pack2<DT>(__fmul_rn(y0, sig), __fmul_rn(y1, sig));
+            wq[i / 2] = pb.scaled<DT>(x[i], x[i + 1], sig);
             const int e = 16 * b + i;
-            const float d0 = pr[i] * (dp[e] * gv - dsum), d1 = pr[i + 1] * (dp[e + 1] * gv - dsum);
-            qt_split2<DT>(d0, d1, wh[8 * b + i / 2], wl[8 * b + i / 2]);
+            const float d0 = pr[i] * fmaf(dp[e], gv, -dsum);
+            const float d1 = pr[i + 1] * fmaf(dp[e + 1], gv, -dsum);
+            qt_split2<DT>(d0, d1, wh[i / 2], wl[i / 2]);
           }
+          qt_store16(tP, r, col + 16 * b, wq);
+          qt_store16(tH, r, col + 16 * b, wh);
+          qt_store16(tL, r, col + 16 * b, wl);
         }
-        qt_store32(tP, r, col, wq);
-        qt_store32(tH, r, col, wh);
-        qt_store32(tL, r, col, wl);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[KPF]);
     }
     // epilogue: lane r of the dV and dK accumulators is key j0 + r
-    if (ok && warp_wait(&bars[KPE], (n_it - 1) & 1, S.abort)) {
+    if (ok && warp_wait(&bars[KDONE], 0, S.abort)) {
       tc_fence_after();
       const int key = j0 + r;
       const bool key_ok = key < len;
