@@ -40,10 +40,11 @@
 //                           tokens) -> fake-quantised tiles, one 128-row
 //                           tile per CTA staged in shared memory
 //   qat_rowdot_tile_kernel  D = rowsum(dO o O') and the dO tiles
-//   qat_fwd_kernel          per 128 query rows: pass A over the key tiles
-//                           for the row maxima (S only), pass B for P, P^,
-//                           O = P^ V^ and O' = P V^ against the final
-//                           maxima (no rescaling of the accumulators), lse
+//   qat_fwd_kernel          per 128 query rows, one pass over the key
+//                           tiles: S, P and P^, O += P^ V^ and O' += P V^
+//                           against a per-row reference maximum that moves
+//                           (rescaling O and O') only when a tile passes it
+//                           by more than 2^8, lse
 //   qat_bwd_q_kernel        per 128 query rows: S, dP, dS; dQ += dS K^
 //   qat_bwd_kv_kernel       per 128-key tile over the 128-row query chunks
 //                           of its query heads: S, dP, P, P^, dS;
@@ -51,7 +52,10 @@
 // The three attention kernels have ten warps: warps 0-7 own the rows (two
 // per tensor-memory lane quarter, each taking half of the 128 columns of
 // a score tile), warp 8 moves tiles with bulk copies, warp 9 issues the MMAs
-// from one thread.  Every wait is bounded.
+// from one thread.  Every wait is bounded.  Where the A operand of a product
+// has the query rows on its M side (P of O' in the forward, dS of dQ), the
+// rows write it to tensor memory and the MMA reads it from there: no
+// shared-memory round trip.
 #pragma once
 #include "attn.cuh"
 
@@ -243,8 +247,12 @@ __global__ void __launch_bounds__(256) qat_rowdot_tile_kernel(
 struct PBlock {
   float dec, rr;
   bool zero;
-  __device__ __forceinline__ PBlock(float amax, const float* rcp) {
-    const uint32_t sp = ue4m3(__fdiv_rn(amax, 6.0f));
+  // by_mul: amax / 6 as amax times the fp32 value of 1/6 (a multiply
+  // instead of a division; it can differ from the quotient by one fp32 ulp,
+  // which moves the UE4M3 byte only when amax / 6 lies that close to a
+  // rounding boundary of the byte)
+  __device__ __forceinline__ PBlock(float amax, const float* rcp, bool by_mul = false) {
+    const uint32_t sp = ue4m3(by_mul ? amax * (1.0f / 6.0f) : __fdiv_rn(amax, 6.0f));
     zero = sp == 0;
     dec = ue4m3_decode(sp);
     rr = rcp[sp];
@@ -410,23 +418,20 @@ struct QtFwdLayout {
   static constexpr uint32_t Q = 0, RING = T, P = (1 + kQtRing) * T;  // RING: K or V tiles
   static constexpr uint32_t SH = P + kQtPTile;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
-  // S slot 0; slot 1 (pass A only) is the columns O and O' take in pass B;
-  // P hi and lo (the A operand of O' += P V^, two 16-bit values a column)
-  static constexpr uint32_t T_S = 0, T_S1 = 128, T_O = 128, T_OH = 128 + D;
-  static constexpr uint32_t T_PH = 384, T_PL = 448;
+  // S; O and O'; P hi and lo (the A operand of O' += P V^, two 16-bit
+  // values a column)
+  static constexpr uint32_t T_S = 0, T_O = 128, T_OH = 128 + D, T_PH = 384, T_PL = 448;
   static_assert(T_OH + D <= T_PH, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 // The K and V tiles of a forward CTA pass through one ring of kQtRing slots
-// in the order the MMAs read them: K(0..nt-1) for pass A, then K(0), and for
-// each key tile j: K(j+1) (when j+1 < nt), V(j).  Item i sits in slot
-// i % kQtRing; V(j+1) loads during the products of tile j at the latest.
+// in the order the MMAs read them: K(0), then for each key tile j: K(j+1)
+// (when j+1 < nt), V(j).  Item i sits in slot i % kQtRing.
 __device__ __forceinline__ int qt_ring_item(int i, int nt, bool& is_v) {
   is_v = false;
-  if (i < nt) return i;
-  if (i == nt) return 0;
-  const int q = i - nt - 1;
+  if (i == 0) return 0;
+  const int q = i - 1;
   if (q == 2 * (nt - 1)) {
     is_v = true;
     return nt - 1;
@@ -434,33 +439,29 @@ __device__ __forceinline__ int qt_ring_item(int i, int nt, bool& is_v) {
   is_v = (q & 1) != 0;
   return is_v ? (q >> 1) : (q >> 1) + 1;
 }
-// Ring index of the K tile of step u and of V(j).
-__device__ __forceinline__ int qt_ring_k(int u, int nt) {
-  return u <= nt ? u : nt + 2 * (u - nt) - 1;
-}
+// Ring index of K(j) and of V(j).
+__device__ __forceinline__ int qt_ring_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int qt_ring_v(int j, int nt) {
-  return j == nt - 1 ? 3 * nt - 1 : nt + 2 * j + 2;
+  return j == nt - 1 ? 2 * nt - 1 : 2 * j + 2;
 }
 
-// RF + s / RE + s: ring slot s loaded / free; FSF + t / FSE + t: S slot t
-// written / read; FPF + h / FPE + h: key half h (keys 64h..64h+63) of P^
-// and of P's two parts written / consumed by the products.
+// RF + s / RE + s: ring slot s loaded / free; FSF / FSE: S written / read;
+// FPF: P^ (shared memory) and P's two parts (tensor memory) written, with O
+// and O' rescaled; FPE: the products of a key tile done.
 enum : int {
-  FQ = 0, RF = 1 /* 1..4 */, RE = 5 /* 5..8 */, FSF = 9 /* 9,10 */,
-  FSE = 11 /* 11,12 */, FPF = 13 /* 13,14 */, FPE = 15 /* 15,16 */, FDONE = 17, FN = 18
+  FQ = 0, RF = 1 /* 1..4 */, RE = 5 /* 5..8 */, FSF = 9, FSE = 10, FPF = 11, FPE = 12,
+  FDONE = 13, FN = 14
 };
-// S slot of step u and how many earlier steps used it: pass A alternates
-// the two slots, pass B uses slot 0 only.
-__device__ __forceinline__ int qt_s_slot(int u, int nt) { return u < nt ? (u & 1) : 0; }
-__device__ __forceinline__ int qt_s_use(int u, int nt) {
-  return u < nt ? (u >> 1) : ((nt + 1) >> 1) + (u - nt);
-}
-constexpr uint32_t kFwd256 = (1u << FSE) | (1u << (FSE + 1));
-constexpr uint32_t kFwd128 = (1u << FPF) | (1u << (FPF + 1));
+constexpr uint32_t kFwd256 = (1u << FSE) | (1u << FPF);
+// A row's reference maximum (log2 units) moves only when a key tile's
+// maximum exceeds it by more than this: P and l stay below 2^8 times their
+// values against the exact running maximum, and O, O' are rescaled rarely.
+constexpr float kQtRescale = 8.0f;
 
 // grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads; causal grids
-// start the query tiles with the most keys.  Steps u < nt are pass A over
-// key tile u, steps nt <= u < 2 nt pass B over key tile u - nt.
+// start the query tiles with the most keys.  One pass over the key tiles:
+// S(j+1) is computed while the rows turn S(j) into P^ and P, then O += P^ V^
+// and O' += P V^ against each row's reference maximum.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams p) {
   using L = QtFwdLayout<D>;
@@ -476,8 +477,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
   const int qt = p.causal ? ntq - 1 - ti : ti;
   const int q0 = qt * 128;
   const int kend = p.causal ? min(len, q0 + 128) : len;
-  const int nt = (kend + 127) / 128, nsteps = 2 * nt;
-  const QtShared S = qt_setup(sm + L::SH, FN, kFwd256, kFwd128);
+  const int nt = (kend + 127) / 128;
+  const QtShared S = qt_setup(sm + L::SH, FN, kFwd256, 0);
   uint64_t* bars = S.bars;
   const uint32_t tmem = *S.tmem;
 
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
       const uint8_t* vbase = p.vt + qat_slot(hk, p.nslot, st, seq, 0) * L::T;
       mbar_arrive_expect_tx(&bars[FQ], L::T);
       bulk_g2s(sm + L::Q, p.qt + qat_slot(h, p.nslot, st, seq, qt) * L::T, L::T, &bars[FQ]);
-      const int nitems = 3 * nt;
+      const int nitems = 2 * nt;
       int last[kQtRing];
 #pragma unroll
       for (int sl = 0; sl < kQtRing; ++sl) last[sl] = -1;
@@ -510,45 +511,37 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idPV = idesc_f16(DT, 128, D) | kIdescBmn;
       const uint32_t base = smem_u32(sm);
-      auto issue_s = [&](int u) -> bool {
-        const int sl = qt_s_slot(u, nt), use = qt_s_use(u, nt);
-        const int i = qt_ring_k(u, nt), rs = i % kQtRing;
+      auto issue_s = [&](int j) -> bool {
+        const int i = qt_ring_k(j), rs = i % kQtRing;
         if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) return false;
-        // the previous scores in this slot have been read
-        if (use >= 1 && !mbar_wait(&bars[FSE + sl], (use - 1) & 1, S.abort)) return false;
+        // the rows have read the previous scores
+        if (j >= 1 && !mbar_wait(&bars[FSE], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + (sl ? L::T_S1 : L::T_S), qt_desc_k(base + L::Q, s),
+          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s),
                   qt_desc_k(base + L::RING + rs * L::T, s), idS, s > 0);
-        tc_commit(&bars[FSF + sl]);
+        tc_commit(&bars[FSF]);
         tc_commit(&bars[RE + rs]);
         return true;
       };
       bool ok = mbar_wait(&bars[FQ], 0, S.abort) && issue_s(0);
-      for (int u = 0; u < nsteps && ok; ++u) {
+      for (int j = 0; j < nt && ok; ++j) {
         // the next tile's scores go ahead of this tile's products
-        if (u + 1 < nsteps && !issue_s(u + 1)) break;
-        if (u < nt) continue;
-        const int j = u - nt, i = qt_ring_v(j, nt), rs = i % kQtRing;
+        if (j + 1 < nt && !issue_s(j + 1)) break;
+        const int i = qt_ring_v(j, nt), rs = i % kQtRing;
         if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) break;
+        if (!mbar_wait(&bars[FPF], j & 1, S.abort)) break;
+        tc_fence_after();
         const uint32_t vt = base + L::RING + rs * L::T;
-        bool fine = true;
 #pragma unroll
-        for (int hf = 0; hf < 2 && fine; ++hf) {
-          // the products of a key half start once its warps have written it
-          if (!mbar_wait(&bars[FPF + hf], j & 1, S.abort)) { fine = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int s = 4 * hf; s < 4 * hf + 4; ++s) {
-            const uint64_t bv = qt_desc_mn(vt, s);
-            mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
-            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PH + 8 * s, bv, idPV, j > 0 || s > 0);
-            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PL + 8 * s, bv, idPV, 1);
-          }
-          tc_commit(&bars[FPE + hf]);
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t bv = qt_desc_mn(vt, s);
+          mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
+          mma_f16_ta(tmem + L::T_OH, tmem + L::T_PH + 8 * s, bv, idPV, j > 0 || s > 0);
+          mma_f16_ta(tmem + L::T_OH, tmem + L::T_PL + 8 * s, bv, idPV, 1);
         }
-        if (!fine) break;
+        tc_commit(&bars[FPE]);
         tc_commit(&bars[RE + rs]);
       }
       tc_commit(&bars[FDONE]);
@@ -562,53 +555,49 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
     const int klim = row_ok ? (p.causal ? row + 1 : len) : 0;  // visible keys: key < klim
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e;  // raw score -> log2 units
-    bool ok = true;
-    // pass A: the row maximum over this warp's columns, then the pair's
-    float mraw = -INFINITY;
-    for (int u = 0; u < nt && ok; ++u) {
-      const int sl = qt_s_slot(u, nt);
-      if (!warp_wait(&bars[FSF + sl], qt_s_use(u, nt) & 1, S.abort)) { ok = false; break; }
-      tc_fence_after();
-      mraw = fmaxf(mraw, qt_max64(tl + (sl ? L::T_S1 : L::T_S) + 64 * half, u * 128 + 64 * half,
-                                  klim));
-      tc_fence_before();
-      mbar_arrive(&bars[FSE + sl]);
-    }
-    float other = -INFINITY;
-    if (ok) ok = qt_pair_swap(S, quarter, half, r, 0, mraw, other);
-    const float m = fmaxf(mraw, other) * c2;  // rounding is monotone: max of the scaled scores
-    const float mref = m == -INFINITY ? 0.0f : m;
-    // pass B: P against the final maximum, P^ against each BLK-key
-    // sub-tile's own maximum
-    float lsum = 0.0f;
+    const int c0 = 64 * half;
     uint8_t* tP = sm + L::P;
-    for (int u = nt; u < nsteps && ok; ++u) {
-      const int sl = 0, j = u - nt, kb = j * 128, c0 = 64 * half;
+    bool ok = true;
+    // mref: the row's reference maximum (log2 units, -inf before the first
+    // visible key); lsum: this warp's share of l = sum 2^(s - mref)
+    float mref = -INFINITY, lsum = 0.0f;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int kb = j * 128;
       const uint32_t ts = tl + L::T_S;
-      if (!warp_wait(&bars[FSF + sl], qt_s_use(u, nt) & 1, S.abort)) { ok = false; break; }
+      if (!warp_wait(&bars[FSF], j & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-      float mt_raw = -INFINITY;
-      // a 128-key sub-tile takes the partner's columns into its maximum too
-      if constexpr (BLK == 128) mt_raw = qt_max64(ts + (c0 ^ 64), kb + (c0 ^ 64), klim);
+      // the tile's row maximum from both halves' columns (the two warps of a
+      // row compute the same value), this half's maximum for a 64-key sigma
+      const float mpart = qt_max64(ts + (c0 ^ 64), kb + (c0 ^ 64), klim);
       float a[2][32];
       tmem_ld32(ts + c0, a[0]);
       tmem_ld32(ts + c0 + 32, a[1]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars[FSE + sl]);
+      mbar_arrive(&bars[FSE]);
       qt_mask32(a[0], kb + c0, klim);
       qt_mask32(a[1], kb + c0 + 32, klim);
+      float mown = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mt_raw = fmaxf(mt_raw, fmaxf(a[0][i], a[1][i]));
-      const bool live = mt_raw != -INFINITY;
-      // P / sigma of the sub-tile = 2688 exp(S - max_tile S) = 2^(s c2 + off);
-      // P = that times fct = 2^(mt - m) / 2688 (the sub-tile's sigma relative
-      // to the row's)
-      const float off = live ? kLog2TensorScaleDiv - mt_raw * c2 : 0.0f;
-      const float fct = live ? ex2_ftz(mt_raw * c2 - mref) * (1.0f / kTensorScaleDiv) : 0.0f;
-      // P^ and the two parts of P in registers first: they are written (P^ to
-      // shared memory, P to tensor memory) once the products of the previous
-      // tile have read their predecessors
+      for (int i = 0; i < 32; ++i) mown = fmaxf(mown, fmaxf(a[0][i], a[1][i]));
+      const float mtile = half == 0 ? fmaxf(mown, mpart) : fmaxf(mpart, mown);
+      const float msig_raw = BLK == 128 ? mtile : mown;
+      // a new reference when the tile's maximum passes the old one by more
+      // than kQtRescale: O, O' and l are multiplied by alpha = 2^(old - new)
+      float alpha = 1.0f;
+      if (mtile != -INFINITY && mtile * c2 > mref + kQtRescale) {
+        alpha = mref == -INFINITY ? 0.0f : ex2_ftz(mref - mtile * c2);
+        mref = mtile * c2;
+      }
+      lsum *= alpha;
+      const bool live = msig_raw != -INFINITY;
+      // P / sigma of the sub-tile = 2688 exp(S - max_sub S) = 2^(s c2 + off);
+      // P = that times fct = 2^(max_sub - mref) / 2688
+      const float off = live ? kLog2TensorScaleDiv - msig_raw * c2 : 0.0f;
+      const float fct = live ? ex2_ftz(msig_raw * c2 - mref) * (1.0f / kTensorScaleDiv) : 0.0f;
+      // P^ and the two parts of P in registers first; they are written (P^
+      // to shared memory, P to tensor memory) once the products of the
+      // previous tile are done
       uint32_t wq[2][16], wh[2][16], wl[2][16];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -631,8 +620,26 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
           }
         }
       }
-      if (j >= 1 && !warp_wait(&bars[FPE + half], (j - 1) & 1, S.abort)) { ok = false; break; }
+      if (j >= 1 && !warp_wait(&bars[FPE], (j - 1) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        // this warp's columns of O and O' against the new reference
+#pragma unroll 1
+        for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 16) {
+          float o[16], oh[16];
+          tmem_ld16(tl + L::T_O + c, o);
+          tmem_ld16(tl + L::T_OH + c, oh);
+          tmem_ld_wait();
+          uint32_t uo[16], uh[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            uo[i] = __float_as_uint(o[i] * alpha);
+            uh[i] = __float_as_uint(oh[i] * alpha);
+          }
+          tmem_st16u(tl + L::T_O + c, uo);
+          tmem_st16u(tl + L::T_OH + c, uh);
+        }
+      }
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         qt_store32(tP, r, c0 + 32 * cc, wq[cc]);
@@ -642,14 +649,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[FPF + half]);
+      mbar_arrive(&bars[FPF]);
     }
+    const float m = mref;
     // epilogue: O = P^ V^ g_V / l, O' = P V^ g_V / l, lse; the row sum l
-    // from both halves (after the last products, when every warp is past
-    // the first exchange)
+    // from both halves
     if (ok) ok = warp_wait(&bars[FDONE], 0, S.abort);
     float lo = 0.0f;
-    if (ok) ok = qt_pair_swap(S, quarter, half, r, 1, lsum, lo);
+    if (ok) ok = qt_pair_swap(S, quarter, half, r, 0, lsum, lo);
     if (ok) {
       tc_fence_after();
       const float l = half == 0 ? lsum + lo : lo + lsum;
@@ -1039,7 +1046,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
             x[i] = pr[i] * inv;
             am = fmaxf(am, x[i]);
           }
-          const PBlock pb(am, S.rcp);
+          const PBlock pb(am, S.rcp, true);
           uint32_t wq[8], wh[8], wl[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {

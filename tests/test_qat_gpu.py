@@ -86,6 +86,34 @@ def test_qat_matches_oracle(name):
     _compare(_run_gpu(inp, w), _run_oracle(inp, w))
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_rising_scores_move_the_reference_maximum(causal):
+    """Scores that grow by about 6 (natural units) per 128-key tile: every
+    key tile's row maximum passes the previous one by more than 2^8, so the
+    forward rescales O and O' at nearly every tile; results still match the
+    oracle."""
+    H, Hkv, d, N = 2, 1, 128, 640
+    gen = torch.Generator().manual_seed(21)
+    u = torch.randn(d, generator=gen)
+    u = u / u.norm() * d ** 0.5
+    a = (6.0 / d ** 0.5) ** 0.5
+    t = torch.arange(N, dtype=torch.float32)[:, None, None] / 128.0
+    q = a * u + 0.2 * torch.randn((N, H, d), generator=gen)
+    k = a * t * u + 0.2 * torch.randn((N, Hkv, d), generator=gen)
+    v = torch.randn((N, Hkv, d), generator=gen)
+    dout = torch.randn((N, H, d), generator=gen)
+    inp = {"q": q.to(torch.bfloat16), "k": k.to(torch.bfloat16), "v": v.to(torch.bfloat16),
+           "dout": dout.to(torch.bfloat16), "cu_seqlens": torch.tensor([0, N], dtype=torch.int32),
+           "lengths": [N]}
+    w = synth.QatWorkload("rising", 1, H, Hkv, N, d, torch.bfloat16, causal, 128, False, seed=21)
+    got, want = _run_gpu(inp, w), _run_oracle(inp, w)
+    # the scores really do climb by more than 8 (log2) from tile to tile
+    s = (q[:, 0].double() @ k[:, 0].double().T) / d ** 0.5
+    tile_max = torch.stack([s[:, j:j + 128].max() for j in range(0, N, 128)])
+    assert float((tile_max[1:] - tile_max[:-1]).min()) * 1.4427 > 8.0
+    _compare(got, want)
+
+
 def test_reused_images_give_the_same_gradients():
     dt, H, Hkv, d, blk, causal, ss, lengths = CASES["bf16_gqa_causal_varlen"]
     w = synth.QatWorkload("reuse", 1, H, Hkv, max(lengths), d, dt, causal, blk, True, seed=5)
