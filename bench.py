@@ -83,23 +83,25 @@ def _src_sha(name):
 
 
 # DRAM traffic of one attention launch measured by ncu (read + write bytes)
-# for the attention source with this hash; reported only while the source is
-# unchanged since the capture.
-ATTN_TRAFFIC = {"src_sha16": "abe4ba02cd17350b", "workload": "b2h32n8192d128_bf16_noncausal_top10",
-                "bytes": 395558144 + 121920256}
+# per workload, for the attention source with this hash; reported only while
+# the source is unchanged since the capture.
+ATTN_TRAFFIC = {"src_sha16": "abe4ba02cd17350b",
+                "bytes": {"b2h32n8192d128_bf16_noncausal_top10": 395558144 + 121920256,
+                          "b1h32hkv8n32768d128_bf16_causal_had_ss_top5": 499836672}}
 
 
 def attn_traffic(w):
-    if _src_sha("attn.cuh") == ATTN_TRAFFIC["src_sha16"] and w.name == ATTN_TRAFFIC["workload"]:
-        return ATTN_TRAFFIC["bytes"]
+    if _src_sha("attn.cuh") == ATTN_TRAFFIC["src_sha16"]:
+        return ATTN_TRAFFIC["bytes"].get(w.name)
     return None
 
 
 # DRAM traffic per step of the three Attn-QAT attention kernels (forward,
 # key-tile and query-tile backward) from the ncu launch list of the QAT source
-# with this hash; reported only while the source is unchanged.
-QAT_TRAFFIC = {"src_sha16": "932e539dcdf5cdaa", "workload": "qat_b1h32hkv8n4096d128_bf16_causal",
-               "bytes": int((99.2 + 90.2 + 111.9) * 1e6)}
+# with this hash (per-launch means over five steps); reported only while the
+# source is unchanged.
+QAT_TRAFFIC = {"src_sha16": "7e38716da3938b80", "workload": "qat_b1h32hkv8n4096d128_bf16_causal",
+               "bytes": int((96.6 + 90.8 + 107.9) * 1e6)}
 
 
 def qat_traffic(w):
@@ -668,10 +670,10 @@ def qat_line(ops, dev, peaks, peak_src, args, steps=20, warmup=3):
                          "peak_note": f"{src} bf16 burst (the kernels run 16-bit MMAs; the "
                                       f"timed region is tens of milliseconds)",
                          "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
-                         "executed_mma_flops": 14 * 2 * pairs * w.d,
-                         "note": "7 algorithmic products; the kernels execute 14 (the forward "
-                                 "computes S in both of its passes, each gradient kernel S and "
-                                 "dP again; dS and the P of O' enter as two 16-bit parts)"},
+                         "executed_mma_flops": 13 * 2 * pairs * w.d,
+                         "note": "7 algorithmic products; the kernels execute 13 (each "
+                                 "gradient kernel computes S and dP again; dS and the P of O' "
+                                 "enter as two 16-bit parts)"},
             "kernels_per_step": QAT_KERNELS_PER_STEP, "steps": steps}
     if not args.no_cpu_baseline:
         # the oracle on a causal prefix of kv head 0 with its query heads: a
