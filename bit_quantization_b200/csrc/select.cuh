@@ -240,8 +240,20 @@ __device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, F
       kcache[i] = valid(i) ? order_key(score(i)) : 0ull;
   }
   auto key_of = [&](int64_t i) { return kcache ? kcache[i] : order_key(score(i)); };
+  // keys of kU consecutive strides per thread, loaded before any is used (an
+  // invalid or out-of-range entry reads as 0 with ok = false)
+  constexpr int kU = 4;
+  auto load_keys = [&](int64_t base, uint64_t (&key)[kU], bool (&ok)[kU]) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = base + (int64_t)u * blockDim.x + threadIdx.x;
+      ok[u] = i < n && valid(i);
+      key[u] = ok[u] ? key_of(i) : 0ull;
+    }
+  };
   uint64_t prefix = 0, pmask = 0;
   int64_t rem = k;
+  bool whole_bucket = false;  // the threshold bucket is taken whole
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
@@ -249,16 +261,18 @@ __device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, F
     // keys sharing a digit in a warp add to its bin once (the leading
     // digits of nearby scores coincide, and same-address shared atomics
     // serialise)
-    for (int64_t base = 0; base < n; base += blockDim.x) {
-      const int64_t i = base + threadIdx.x;
-      int digit = -1;
-      if (i < n && valid(i)) {
-        const uint64_t key = key_of(i);
-        if ((key & pmask) == prefix) digit = (int)((key >> shift) & 255);
+    for (int64_t base = 0; base < n; base += (int64_t)kU * blockDim.x) {
+      uint64_t key[kU];
+      bool ok[kU];
+      load_keys(base, key, ok);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int digit =
+            (ok[u] && (key[u] & pmask) == prefix) ? (int)((key[u] >> shift) & 255) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, digit);
+        if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
+          atomicAdd(&sh.hist[digit], __popc(same));
       }
-      const unsigned same = __match_any_sync(0xffffffffu, digit);
-      if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
-        atomicAdd(&sh.hist[digit], __popc(same));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -274,11 +288,27 @@ __device__ void radix_topk(int64_t n, int64_t k, int64_t n_valid, Valid valid, F
     prefix = sh.prefix;
     rem = sh.remaining;
     pmask |= (uint64_t)255 << shift;
-    if (sh.done) break;  // uniform: every thread read the same word
+    whole_bucket = sh.done != 0;
+    __syncthreads();  // sh.done is rewritten by the next pass
+    if (whole_bucket) break;  // uniform: every thread read the same word
   }
   // compare on the decided bits only (all of them unless the select stopped
   // early, when every key of the threshold bucket is taken)
   const uint64_t T = prefix;
+  if (whole_bucket) {
+    // every key at the threshold is taken: no order among them to keep
+    for (int64_t base = 0; base < n; base += (int64_t)kU * blockDim.x) {
+      uint64_t key[kU];
+      bool ok[kU];
+      load_keys(base, key, ok);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x + threadIdx.x;
+        if (i < n) out[i] = (ok[u] && ((key[u] & pmask) >= T || fixed(i))) ? 1 : 0;
+      }
+    }
+    return;
+  }
   const int64_t take_eq = rem;
   int64_t taken = 0;
   for (int64_t base = 0; base < n; base += blockDim.x) {
