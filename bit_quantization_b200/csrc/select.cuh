@@ -8,6 +8,8 @@
 // the valid pairs (causal: j <= i); ties between equal scores go to the lower
 // linear index i * nB + j.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "quant_kernels.cuh"
 
 namespace thrift {
@@ -369,6 +371,189 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double* __rest
 inline size_t topk_smem(int nB) {
   const int64_t np = (int64_t)nB * nB;
   return np <= kTopkCache ? (size_t)np * 8 : 0;
+}
+
+// ---------------------------------------------- top-k over a CTA cluster --
+// The same exact selection as radix_topk with the n entries split into
+// kTopkCluster contiguous index ranges, one per CTA of a cluster; each CTA
+// caches its range's keys in shared memory when they fit.  Per pass every
+// CTA counts its range, rank 0 adds the histograms (distributed shared
+// memory) and decides the digit, and every CTA reads the decision back.
+// Ties at the threshold keep ascending index order across the ranges: each
+// CTA's count of threshold keys, summed over the lower ranks, starts its
+// scan.  All CTAs of the cluster call it with the same n, k, n_valid.
+constexpr int kTopkCluster = 4;
+constexpr int kTopkClusterCacheBytes = 192 * 1024;
+
+struct TopkClusterShared {
+  int hist[256];
+  int warp_sums[32];
+  int total;
+  int done;
+  uint64_t prefix;
+  int64_t remaining;
+  unsigned long long eq_count;  // this CTA's keys at the threshold
+};
+
+template <class Valid, class Fixed, class Score>
+__device__ void radix_topk_cluster(int64_t n, int64_t k, int64_t n_valid, Valid valid,
+                                   Fixed fixed, Score score, uint64_t* kcache,
+                                   TopkClusterShared& sh, uint8_t* __restrict__ out) {
+  namespace cgx = cooperative_groups;
+  cgx::cluster_group cl = cgx::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int64_t per = (n + kTopkCluster - 1) / kTopkCluster;
+  const int64_t lo = min(n, (int64_t)rank * per), hi = min(n, lo + per);
+  if (k == 0 || k == n_valid) {
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x)
+      out[i] = (valid(i) && (k != 0 || fixed(i))) ? 1 : 0;
+    return;
+  }
+  if (kcache) {
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x)
+      kcache[i - lo] = valid(i) ? order_key(score(i)) : 0ull;
+    __syncthreads();
+  }
+  auto key_of = [&](int64_t i) { return kcache ? kcache[i - lo] : order_key(score(i)); };
+  constexpr int kU = 4;
+  auto load_keys = [&](int64_t base, uint64_t (&key)[kU], bool (&ok)[kU]) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = base + (int64_t)u * blockDim.x + threadIdx.x;
+      ok[u] = i < hi && valid(i);
+      key[u] = ok[u] ? key_of(i) : 0ull;
+    }
+  };
+  TopkClusterShared* s0 = cl.map_shared_rank(&sh, 0);
+  uint64_t prefix = 0, pmask = 0;
+  int64_t rem = k;
+  bool whole_bucket = false;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
+    __syncthreads();
+    for (int64_t base = lo; base < hi; base += (int64_t)kU * blockDim.x) {
+      uint64_t key[kU];
+      bool ok[kU];
+      load_keys(base, key, ok);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int digit =
+            (ok[u] && (key[u] & pmask) == prefix) ? (int)((key[u] >> shift) & 255) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, digit);
+        if (digit >= 0 && (threadIdx.x & 31) == __ffs(same) - 1)
+          atomicAdd(&sh.hist[digit], __popc(same));
+      }
+    }
+    cl.sync();  // every range counted
+    if (rank == 0) {
+      for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+        int t = sh.hist[b];
+#pragma unroll
+        for (int r = 1; r < kTopkCluster; ++r) t += cl.map_shared_rank(sh.hist, r)[b];
+        sh.hist[b] = t;
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        int64_t above;
+        const int sel = select_digit(sh.hist, rem, &above);
+        if (threadIdx.x == 0) {
+          sh.remaining = rem - above;
+          sh.prefix = prefix | ((uint64_t)sel << shift);
+          sh.done = (int64_t)sh.hist[sel] == rem - above;
+        }
+      }
+    }
+    cl.sync();  // the decision is published
+    prefix = s0->prefix;
+    rem = s0->remaining;
+    whole_bucket = s0->done != 0;
+    pmask |= (uint64_t)255 << shift;
+    cl.sync();  // read before rank 0 decides again (or leaves)
+    if (whole_bucket) break;  // uniform across the cluster
+  }
+  const uint64_t T = prefix;
+  if (whole_bucket) {
+    for (int64_t base = lo; base < hi; base += (int64_t)kU * blockDim.x) {
+      uint64_t key[kU];
+      bool ok[kU];
+      load_keys(base, key, ok);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x + threadIdx.x;
+        if (i < hi) out[i] = (ok[u] && ((key[u] & pmask) >= T || fixed(i))) ? 1 : 0;
+      }
+    }
+    return;
+  }
+  // ties: this range's threshold keys, then the lower ranks' counts
+  if (threadIdx.x == 0) sh.eq_count = 0;
+  __syncthreads();
+  {
+    unsigned long long cnt = 0;
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x)
+      if (valid(i) && (key_of(i) & pmask) == T) ++cnt;
+    if (cnt) atomicAdd(&sh.eq_count, cnt);
+  }
+  cl.sync();
+  int64_t taken = 0;
+  for (int r = 0; r < rank; ++r) taken += (int64_t)cl.map_shared_rank(&sh, r)->eq_count;
+  const int64_t take_eq = rem;
+  for (int64_t base = lo; base < hi; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    uint64_t key = 0;
+    bool ok = false;
+    if (i < hi && valid(i)) {
+      key = key_of(i) & pmask;
+      ok = true;
+    }
+    const int eq = (ok && key == T) ? 1 : 0;
+    const int before = block_exclusive_scan(eq, sh.warp_sums, &sh.total);
+    if (i < hi) out[i] = (ok && (key > T || (eq && taken + before < take_eq) || fixed(i))) ? 1 : 0;
+    taken += sh.total;
+    __syncthreads();
+  }
+  cl.sync();  // no CTA leaves while another may still read its counts
+}
+
+// topk_kernel's work over a cluster of kTopkCluster CTAs per (sequence,
+// head): grid nseq * H * kTopkCluster; dynamic shared memory holds a range's
+// keys when topk_cluster_smem(nB) is nonzero.
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
+    topk_cluster_kernel(const double* __restrict__ scores, SeqInfo seqs, int H, int blk, int nB,
+                        int causal, float frac, int sink, int recent,
+                        uint8_t* __restrict__ mask, int use_cache) {
+  __shared__ TopkClusterShared sh;
+  extern __shared__ uint64_t kcache[];
+  const int head = blockIdx.x / kTopkCluster;
+  const int seq = head / H, h = head % H;
+  int64_t start;
+  int len;
+  seqs.get(seq, start, len);
+  const int nb = (int)ceil_div(len, blk);
+  const int64_t npairs = (int64_t)nB * nB;
+  const double* sc = scores + ((int64_t)seq * H + h) * npairs;
+  uint8_t* mk = mask + ((int64_t)seq * H + h) * npairs;
+  const int64_t n_valid = causal ? (int64_t)nb * (nb + 1) / 2 : (int64_t)nb * nb;
+  const int64_t k = topk_count_dev(frac, n_valid);
+  auto valid = [&](int64_t lin) {
+    const int l = (int)lin, i = l / nB, j = l - i * nB;
+    return i < nb && j < nb && (!causal || j <= i);
+  };
+  auto fixed = [&](int64_t lin) {
+    const int l = (int)lin, i = l / nB, j = l - i * nB;
+    return j < sink || (causal ? (j > i - recent) : (j >= nb - recent));
+  };
+  auto score = [&](int64_t lin) { return sc[lin]; };
+  radix_topk_cluster(npairs, k, n_valid, valid, fixed, score, use_cache ? kcache : nullptr, sh,
+                     mk);
+}
+
+// Shared memory of a range's key cache (0: the keys are read from global
+// memory in every pass).
+inline size_t topk_cluster_smem(int nB) {
+  const int64_t per = ((int64_t)nB * nB + kTopkCluster - 1) / kTopkCluster;
+  return per * 8 <= kTopkClusterCacheBytes ? (size_t)per * 8 : 0;
 }
 
 }  // namespace thrift

@@ -202,6 +202,27 @@ thrift_status launch_quantize(const void* x, int64_t nb, int G, bool ss, uint32_
   return THRIFT_ERR_UNSUPPORTED;
 }
 
+// ---------------------------------------------------------- selection --
+
+// The top-k pairs of every (sequence, head): one CTA each when its keys fit
+// the CTA's shared-memory cache, else a cluster of kTopkCluster CTAs that
+// split the keys (same selection, bit for bit).
+thrift_status launch_topk(const double* scores, SeqInfo si, int nseq, int H, int blk, int nB,
+                          int causal, float frac, int sink, int recent, uint8_t* mask,
+                          cudaStream_t st) {
+  if ((int64_t)nB * nB <= kTopkCache) {
+    topk_kernel<<<nseq * H, kTopkThreads, topk_smem(nB), st>>>(scores, si, H, blk, nB, causal,
+                                                               frac, sink, recent, mask);
+    return launch_status();
+  }
+  static DeviceSet attr;
+  const size_t smem = topk_cluster_smem(nB);
+  if (!smem_attr(topk_cluster_kernel, kTopkClusterCacheBytes, attr)) return THRIFT_ERR_CUDA;
+  topk_cluster_kernel<<<nseq * H * kTopkCluster, kTopkThreads, smem, st>>>(
+      scores, si, H, blk, nB, causal, frac, sink, recent, mask, smem > 0 ? 1 : 0);
+  return launch_status();
+}
+
 // ----------------------------------------------------- attention layout --
 
 struct AttnWs {
@@ -389,9 +410,9 @@ thrift_status attn_impl(const void* q, const void* k, const void* v, SeqInfo si,
   // selection
   pair_scores_kernel<<<pair_scores_grid(nseq, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       w.means_q, w.means_k, si, nseq, H, Hkv, d, blk, nB, causal, w.scores);
-  topk_kernel<<<nseq * H, kTopkThreads, topk_smem(nB), st>>>(w.scores, si, H, blk, nB, causal,
-                                                             frac, sink, recent, w.mask);
-  if (launch_status() != THRIFT_OK) return THRIFT_ERR_CUDA;
+  if (launch_topk(w.scores, si, nseq, H, blk, nB, causal, frac, sink, recent, w.mask, st) !=
+      THRIFT_OK)
+    return THRIFT_ERR_CUDA;
 
   AttnParams p;
   p.q4 = w.q4; p.k4 = w.k4; p.v4 = w.v4; p.q16 = w.q16; p.k16 = w.k16; p.v16 = w.v16;
@@ -947,9 +968,8 @@ thrift_status block_mean_topk(const void* q, const void* k, thrift_dtype dt, int
   }
   pair_scores_kernel<<<pair_scores_grid(B, H, nB), kThreads, pair_scores_smem(nB), st>>>(
       mq, mk, si, B, H, Hkv, d, blk, nB, causal, sc);
-  topk_kernel<<<B * H, kTopkThreads, topk_smem(nB), st>>>(sc, si, H, blk, nB, causal, topk_frac,
-                                                          sink_blocks, recent_blocks, mask);
-  return launch_status();
+  return launch_topk(sc, si, B, H, blk, nB, causal, topk_frac, sink_blocks, recent_blocks, mask,
+                     st);
 }
 
 thrift_status block_mean_topk_noalloc(const void* q, const void* k, thrift_dtype dt, int B,
