@@ -315,16 +315,15 @@ def config_of(w, lengths=None):
     return c
 
 
-# Issue slots per element of the ScaleSearch-on quantiser, counted from the
-# source (quant_block16 and block_err): per candidate and 16-block about 110
-# instructions (UE4M3 decode 5, scale product 1, correctly rounded reciprocal
-# ~10, 16 products, 8 E2M1 round trips of 4 converts, 16 differences, 16
-# sequential fmaf, the fp64 error and compare ~9, loop ~5) for 9 candidates,
-# plus ~70 for max scaling and the final codes and ~16 for the loads:
-# (9 x 110 + 86) / 16 = 67 per element.
-QUANT_SS_ISSUE_PER_ELEM = 67.0
-QUANT_SS_ISSUE_NOTE = ("issue slots per element counted from the source (9 candidates x ~110 "
-                       "instructions per 16-block + ~86 for max scaling, codes and loads)")
+# Issue slots per element of the ScaleSearch-on quantiser, from a one-launch
+# ncu capture of quant_rows_kernel<fp16, no rotation, ScaleSearch> on the
+# quantiser workload: 21.09 M warp instructions for 524 288 16-element blocks
+# (one block per thread) = 1287 per block = 80.4 per element.  A count from the
+# source (9 candidates x ~110 instructions + ~86) gives 67; the measured count
+# is the denominator.
+QUANT_SS_ISSUE_PER_ELEM = 80.4
+QUANT_SS_ISSUE_NOTE = ("issue slots per element measured by ncu (smsp__inst_executed.sum of "
+                       "one launch x 32 lanes / elements; ~1290 per 16-block)")
 
 
 def quantizer_line(dev, peaks, with_oracle=True):
