@@ -30,10 +30,12 @@
 // (t < ceil(len / 128)) of its head; nslot = total / 128 + nseq bounds them.
 // The fake-quantised elements (E2M1 value x UE4M3 block scale) are exact in
 // the 16-bit input type; the tensor scales multiply the fp32 accumulators.
-// P^ enters the products rounded to the 16-bit type, P (of O') and dS as
-// two 16-bit parts, hi = round(x) and lo = round(x - hi): rows of dS sum to
-// zero, and one rounding would leave a residue that the products with K^ or
-// Q^ (whose channel means can be large) magnify.
+// P^ enters the products rounded to the 16-bit type, P (of O') and the dS
+// of dQ as two 16-bit parts, hi = round(x) and lo = round(x - hi).  Rows of
+// dS sum to zero, so in dQ = dS K^ (a contraction over the keys) K^'s
+// channel means cancel in exact arithmetic and would multiply the residue of
+// a single rounding; dK = dS^T Q^ contracts over the queries, where dS has no
+// such structure, and takes dS rounded once.
 //
 // Kernels.
 //   qat_fq_tile_kernel      Q, K (blocks along d) or V (blocks along the
@@ -880,8 +882,8 @@ template <int D>
 struct QtKvLayout {
   static constexpr uint32_t T = qt_tile_bytes(D);
   static constexpr uint32_t K = 0, V = T, Q = 2 * T, DO = 3 * T;
-  static constexpr uint32_t P = 4 * T, DSH = P + kQtPTile, DSL = DSH + kQtPTile;
-  static constexpr uint32_t SH = DSL + kQtPTile;
+  static constexpr uint32_t P = 4 * T, DS = P + kQtPTile;
+  static constexpr uint32_t SH = DS + kQtPTile;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
   static_assert(T_DK + D <= 512, "tensor memory budget");
@@ -970,8 +972,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const uint64_t bq = qt_desc_mn(base + L::Q, s);
-          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSH, s), bq, idG, it > 0 || s > 0);
-          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DSL, s), bq, idG, 1);
+          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), bq, idG, it > 0 || s > 0);
         }
         tc_commit(&bars[KQE]);
 #pragma unroll
@@ -990,8 +991,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float c2 = p.g[0] * p.g[1] * p.sc * kQatLog2e, gv = p.g[2];
     uint8_t* tP = sm + L::P;
-    uint8_t* tH = sm + L::DSH;
-    uint8_t* tL = sm + L::DSL;
+    uint8_t* tD = sm + L::DS;
     // -lse (log2 units) and D of this thread's query row in iteration it
     auto row_stats = [&](int it, float& nl, float& dsv) {
       const int hq = hk * grp + it / nch, row = (c0 + it % nch) * 128 + r;
@@ -1047,18 +1047,17 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
             am = fmaxf(am, x[i]);
           }
           const PBlock pb(am, S.rcp, true);
-          uint32_t wq[8], wh[8], wl[8];
+          uint32_t wq[8], wd[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
             wq[i / 2] = pb.scaled<DT>(x[i], x[i + 1], sig);
             const int e = 16 * b + i;
             const float d0 = pr[i] * fmaf(dp[e], gv, -dsum);
             const float d1 = pr[i + 1] * fmaf(dp[e + 1], gv, -dsum);
-            qt_split2<DT>(d0, d1, wh[i / 2], wl[i / 2]);
+            wd[i / 2] = pack2<DT>(d0, d1);
           }
           qt_store16(tP, r, col + 16 * b, wq);
-          qt_store16(tH, r, col + 16 * b, wh);
-          qt_store16(tL, r, col + 16 * b, wl);
+          qt_store16(tD, r, col + 16 * b, wd);
         }
       }
       fence_proxy_async_smem();
