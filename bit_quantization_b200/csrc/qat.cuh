@@ -881,8 +881,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
 template <int D>
 struct QtKvLayout {
   static constexpr uint32_t T = qt_tile_bytes(D);
-  static constexpr uint32_t K = 0, V = T, Q = 2 * T, DO = 3 * T;
-  static constexpr uint32_t P = 4 * T, DS = P + kQtPTile;
+  static constexpr uint32_t K = 0, V = T, Q = 2 * T, DO = 4 * T;  // Q: 2 slots
+  static constexpr uint32_t P = 5 * T, DS = P + kQtPTile;
   static constexpr uint32_t SH = DS + kQtPTile;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
@@ -890,20 +890,23 @@ struct QtKvLayout {
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-// KQF / KOF: the Q / dO chunk loaded; KQE / KOE: the Q / dO chunk free
-// (its last product done); KSF / KDF: S / dP in tensor memory.
+// KQF + s / KQE + s: Q slot s loaded / free (its chunk's dK done); KOF /
+// KOE: the dO chunk loaded / free (its dV done); KSF / KSR: S computed /
+// read by the rows; KDF / KDR: dP computed / read; KPF: P^ and dS written;
+// KPE: the chunk's products done.
 enum : int {
-  KKV = 0, KQF = 1, KOF = 2, KQE = 3, KOE = 4, KSF = 5, KDF = 6, KSE = 7, KPF = 8, KPE = 9,
-  KDONE = 10, KN = 11
+  KKV = 0, KQF = 1 /* 1,2 */, KQE = 3 /* 3,4 */, KOF = 5, KOE = 6, KSF = 7, KSR = 8, KDF = 9,
+  KDR = 10, KPF = 11, KPE = 12, KDONE = 13, KN = 14
 };
-constexpr uint32_t kKv256 = (1u << KSE) | (1u << KPF);
+constexpr uint32_t kKv256 = (1u << KSR) | (1u << KDR) | (1u << KPF);
 
 // grid (ceil(maxlen / 128) * Hkv, nseq), kQtThreads threads: key tile
 // blockIdx.x / Hkv (causal grids: the tiles with the most queries first).
 // Iteration it takes query chunk c0 + it % nch of query head
-// hk * grp + it / nch.  The products of a chunk run dK (dS^T Q^) before dV
-// (P^T dO), so the next Q chunk loads while dV runs, and the next dO chunk
-// while S and the maxima of the next chunk are computed.
+// hk * grp + it / nch.  The rows read S(it) into registers first, so S of
+// the next chunk (its Q in the second slot) runs while they work; the
+// products of a chunk run dV (P^T dO) before dK (dS^T Q^), so the next dO
+// chunk loads during dK.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatParams p) {
   using L = QtKvLayout<D>;
@@ -929,20 +932,22 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       mbar_arrive_expect_tx(&bars[KKV], 2 * L::T);
       bulk_g2s(sm + L::K, p.kt + ks * L::T, L::T, &bars[KKV]);
       bulk_g2s(sm + L::V, p.vt + ks * L::T, L::T, &bars[KKV]);
-      int lastq = -1, lasto = -1;
+      int lastq[2] = {-1, -1}, lasto = -1;
       for (int it = 0; it < n_it && !*S.abort; ++it) {
         const int64_t qs = qat_slot(hk * grp + it / nch, p.nslot, st, seq, c0 + it % nch);
-        if (it >= 1 && !mbar_wait(&bars[KQE], (it - 1) & 1, S.abort)) break;
-        mbar_arrive_expect_tx(&bars[KQF], L::T);
-        bulk_g2s(sm + L::Q, p.qt + qs * L::T, L::T, &bars[KQF]);
-        lastq = it;
+        const int sl = it & 1;
+        if (it >= 2 && !mbar_wait(&bars[KQE + sl], ((it >> 1) - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[KQF + sl], L::T);
+        bulk_g2s(sm + L::Q + sl * L::T, p.qt + qs * L::T, L::T, &bars[KQF + sl]);
+        lastq[sl] = it;
         if (it >= 1 && !mbar_wait(&bars[KOE], (it - 1) & 1, S.abort)) break;
         mbar_arrive_expect_tx(&bars[KOF], L::T);
         bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[KOF]);
         lasto = it;
       }
       qt_drain(&bars[KKV], 0);
-      if (lastq >= 0) qt_drain(&bars[KQF], lastq & 1);
+      for (int sl = 0; sl < 2; ++sl)
+        if (lastq[sl] >= 0) qt_drain(&bars[KQF + sl], (lastq[sl] >> 1) & 1);
       if (lasto >= 0) qt_drain(&bars[KOF], lasto & 1);
     }
   } else if (warp == kQtMma) {
@@ -950,36 +955,46 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idG = idesc_f16(DT, 128, D) | kIdescAmn | kIdescBmn;
       const uint32_t base = smem_u32(sm);
-      bool ok = mbar_wait(&bars[KKV], 0, S.abort);
-      for (int it = 0; it < n_it && ok; ++it) {
-        if (!mbar_wait(&bars[KQF], it & 1, S.abort)) break;
-        if (it >= 1 && !mbar_wait(&bars[KSE], (it - 1) & 1, S.abort)) break;
+      // S(it) = Q^ K^T into the S columns (the rows have read S(it - 1))
+      auto issue_s = [&](int it) -> bool {
+        const int sl = it & 1;
+        if (!mbar_wait(&bars[KQF + sl], (it >> 1) & 1, S.abort)) return false;
+        if (it >= 1 && !mbar_wait(&bars[KSR], (it - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K, s), idS, s > 0);
+          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q + sl * L::T, s),
+                  qt_desc_k(base + L::K, s), idS, s > 0);
         tc_commit(&bars[KSF]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars[KKV], 0, S.abort) && issue_s(0);
+      for (int it = 0; it < n_it && ok; ++it) {
+        // dP(it) = dO V^T (the rows have read dP(it - 1))
         if (!mbar_wait(&bars[KOF], it & 1, S.abort)) break;
+        if (it >= 1 && !mbar_wait(&bars[KDR], (it - 1) & 1, S.abort)) break;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
           mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
                   s > 0);
         tc_commit(&bars[KDF]);
+        // the next chunk's scores while the rows work on this one
+        if (it + 1 < n_it && !issue_s(it + 1)) break;
         if (!mbar_wait(&bars[KPF], it & 1, S.abort)) break;
         tc_fence_after();
-        // dK += dS^T Q^, dV += P^T dO: M = the 128 keys, K = the 128 queries
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint64_t bq = qt_desc_mn(base + L::Q, s);
-          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), bq, idG, it > 0 || s > 0);
-        }
-        tc_commit(&bars[KQE]);
+        // dV += P^T dO, dK += dS^T Q^: M = the 128 keys, K = the 128 queries
+        const uint32_t qt = base + L::Q + (it & 1) * L::T;
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
                   it > 0 || s > 0);
         tc_commit(&bars[KOE]);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), qt_desc_mn(qt, s), idG,
+                  it > 0 || s > 0);
+        tc_commit(&bars[KQE + (it & 1)]);
         tc_commit(&bars[KPE]);
       }
       tc_commit(&bars[KDONE]);
@@ -1009,14 +1024,26 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       if (it + 1 < n_it) row_stats(it + 1, nl_next, ds_next);  // in flight meanwhile
       if (!warp_wait(&bars[KSF], it & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-      // sigma of this warp's BLK-key sub-tile: the largest P there / 2688
-      float cm_raw = qt_max64(tl + L::T_S + cb, j0 + cb, klim);
+      // this warp's 64 scores into registers, and with them (and, for a
+      // 128-key sigma, the partner's columns) the largest visible one
+      float a[2][32];
+      tmem_ld32(tl + L::T_S + cb, a[0]);
+      tmem_ld32(tl + L::T_S + cb + 32, a[1]);
+      tmem_ld_wait();
+      qt_mask32(a[0], j0 + cb, klim);
+      qt_mask32(a[1], j0 + cb + 32, klim);
+      float cm_raw = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) cm_raw = fmaxf(cm_raw, fmaxf(a[0][i], a[1][i]));
       if constexpr (BLK == 128) {
 #pragma unroll 1
         for (int c = 0; c < 2; ++c)
           cm_raw = fmaxf(cm_raw, qt_chunk_max(tl + L::T_S + (cb ^ 64) + 32 * c,
                                               j0 + (cb ^ 64) + 32 * c, klim));
       }
+      tc_fence_before();
+      mbar_arrive(&bars[KSR]);  // the next chunk's S may overwrite these columns
+      // sigma of this warp's BLK-key sub-tile: the largest P there / 2688
       const float cm = cm_raw == -INFINITY ? 0.0f : ex2_ftz(fmaf(cm_raw, c2, nlse2));
       const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
       const float sig = __fdiv_rn(cm, kTensorScaleDiv);
@@ -1024,25 +1051,23 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       // the tiles are free once the products of the previous chunk are done
       if (it >= 1 && !warp_wait(&bars[KPE], (it - 1) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int col = cb + 32 * cc, key0 = j0 + col;
-        float a[32], dp[32];
-        tmem_ld32(tl + L::T_S + col, a);
+        const int col = cb + 32 * cc;
+        float dp[32];
         tmem_ld32(tl + L::T_DP + col, dp);
         tmem_ld_wait();
         if (cc == 1) {
           tc_fence_before();
-          mbar_arrive(&bars[KSE]);
+          mbar_arrive(&bars[KDR]);
         }
-        qt_mask32(a, key0, klim);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
           float pr[16], x[16];
           float am = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            pr[i] = ex2_ftz(fmaf(a[16 * b + i], c2, nlse2));
+            pr[i] = ex2_ftz(fmaf(a[cc][16 * b + i], c2, nlse2));
             x[i] = pr[i] * inv;
             am = fmaxf(am, x[i]);
           }
@@ -1052,9 +1077,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
           for (int i = 0; i < 16; i += 2) {
             wq[i / 2] = pb.scaled<DT>(x[i], x[i + 1], sig);
             const int e = 16 * b + i;
-            const float d0 = pr[i] * fmaf(dp[e], gv, -dsum);
-            const float d1 = pr[i + 1] * fmaf(dp[e + 1], gv, -dsum);
-            wd[i / 2] = pack2<DT>(d0, d1);
+            wd[i / 2] = pack2<DT>(pr[i] * fmaf(dp[e], gv, -dsum),
+                                  pr[i + 1] * fmaf(dp[e + 1], gv, -dsum));
           }
           qt_store16(tP, r, col + 16 * b, wq);
           qt_store16(tD, r, col + 16 * b, wd);
