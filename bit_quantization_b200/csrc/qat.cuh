@@ -709,12 +709,13 @@ struct QtQLayout {
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-// QPF + h / QPE + h: key half h of the dS tiles written / consumed.
+// QSF / QSR: S computed / read by the rows; QDF / QDR: dP computed / read;
+// QPF + h / QPE + h: key half h of dS written / consumed.
 enum : int {
-  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSE = 8,
-  QPF = 9 /* 9,10 */, QPE = 11 /* 11,12 */, QDONE = 13, QN = 14
+  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSR = 8,
+  QDF = 9, QDR = 10, QPF = 11 /* 11,12 */, QPE = 13 /* 13,14 */, QDONE = 15, QN = 16
 };
-constexpr uint32_t kQ256 = 1u << QSE;
+constexpr uint32_t kQ256 = (1u << QSR) | (1u << QDR);
 constexpr uint32_t kQ128 = (1u << QPF) | (1u << (QPF + 1));
 
 // grid (ceil(maxlen / 128) * H, nseq), kQtThreads threads.
@@ -768,27 +769,35 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idDQ = idesc_f16(DT, 128, D) | kIdescBmn;
       const uint32_t base = smem_u32(sm);
-      // S = Q^ K^T and dP = dO V^T of key tile j
+      // S = Q^ K^T of key tile j once the rows have read S(j - 1)
       auto issue_s = [&](int j) -> bool {
         const int sl = j & 1;
         if (!mbar_wait(&bars[QKF + sl], (j >> 1) & 1, S.abort)) return false;
-        if (!mbar_wait(&bars[QVF], j & 1, S.abort)) return false;
-        if (j >= 1 && !mbar_wait(&bars[QSE], (j - 1) & 1, S.abort)) return false;
+        if (j >= 1 && !mbar_wait(&bars[QSR], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
+        for (int s = 0; s < D / 16; ++s)
           mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + sl * L::T, s),
                   idS, s > 0);
+        tc_commit(&bars[QSF]);
+        return true;
+      };
+      // dP = dO V^T of key tile j once the rows have read dP(j - 1)
+      auto issue_dp = [&](int j) -> bool {
+        if (!mbar_wait(&bars[QVF], j & 1, S.abort)) return false;
+        if (j >= 1 && !mbar_wait(&bars[QDR], (j - 1) & 1, S.abort)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
           mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
                   s > 0);
-        }
-        tc_commit(&bars[QSF]);
+        tc_commit(&bars[QDF]);
         tc_commit(&bars[QVE]);
         return true;
       };
-      bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0);
+      bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0) && issue_dp(0);
       for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt && !issue_s(j + 1)) break;
+        if (j + 1 < nt && !(issue_s(j + 1) && issue_dp(j + 1))) break;
         const uint32_t kt = base + L::K + (j & 1) * L::T;
         bool fine = true;
 #pragma unroll
@@ -822,34 +831,39 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
     for (int j = 0; j < nt && ok; ++j) {
       if (!warp_wait(&bars[QSF], j & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
-      // dS of this warp's 64 keys in registers first: they go to tensor
-      // memory once the products of the previous tile have read it
-      uint32_t wh[2][16], wl[2][16];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int col = 64 * half + 32 * cc, key0 = j * 128 + col;
-        float a[32], dp[32];
-        tmem_ld32(tl + L::T_S + col, a);
-        tmem_ld32(tl + L::T_DP + col, dp);
-        tmem_ld_wait();
-        if (cc == 1) {
-          tc_fence_before();
-          mbar_arrive(&bars[QSE]);
-        }
-        qt_mask32(a, key0, klim);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float d0 = ex2_ftz(fmaf(a[i], c2, nlse2)) * fmaf(dp[i], gv, -dsum);
-          const float d1 = ex2_ftz(fmaf(a[i + 1], c2, nlse2)) * fmaf(dp[i + 1], gv, -dsum);
-          qt_split2<DT>(d0, d1, wh[cc][i / 2], wl[cc][i / 2]);
-        }
-      }
+      // this warp's 64 scores into registers, released at once (S of the
+      // next tile may overwrite them); then dP chunk by chunk
+      float a[2][32];
+      tmem_ld32(tl + L::T_S + 64 * half, a[0]);
+      tmem_ld32(tl + L::T_S + 64 * half + 32, a[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[QSR]);
+      qt_mask32(a[0], j * 128 + 64 * half, klim);
+      qt_mask32(a[1], j * 128 + 64 * half + 32, klim);
+      if (!warp_wait(&bars[QDF], j & 1, S.abort)) { ok = false; break; }
+      // this half's dS columns are free once the products of the previous
+      // tile have read them
       if (j >= 1 && !warp_wait(&bars[QPE + half], (j - 1) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        tmem_st16u(tl + L::T_DSH + 32 * half + 16 * cc, wh[cc]);
-        tmem_st16u(tl + L::T_DSL + 32 * half + 16 * cc, wl[cc]);
+        float dp[32];
+        tmem_ld32(tl + L::T_DP + 64 * half + 32 * cc, dp);
+        tmem_ld_wait();
+        if (cc == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars[QDR]);
+        }
+        uint32_t wh[16], wl[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float d0 = ex2_ftz(fmaf(a[cc][i], c2, nlse2)) * fmaf(dp[i], gv, -dsum);
+          const float d1 = ex2_ftz(fmaf(a[cc][i + 1], c2, nlse2)) * fmaf(dp[i + 1], gv, -dsum);
+          qt_split2<DT>(d0, d1, wh[i / 2], wl[i / 2]);
+        }
+        tmem_st16u(tl + L::T_DSH + 32 * half + 16 * cc, wh);
+        tmem_st16u(tl + L::T_DSL + 32 * half + 16 * cc, wl);
       }
       tmem_st_wait();
       tc_fence_before();
