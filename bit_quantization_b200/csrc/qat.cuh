@@ -699,8 +699,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
 template <int D>
 struct QtQLayout {
   static constexpr uint32_t T = qt_tile_bytes(D);
-  static constexpr uint32_t Q = 0, DO = T, K = 2 * T, V = 4 * T;  // K: 2 stages, V: 1
-  static constexpr uint32_t SH = 5 * T;
+  static constexpr uint32_t Q = 0, DO = T, K = 2 * T, V = 5 * T;  // K: 3 slots, V: 2
+  static constexpr uint32_t SH = 7 * T;
   static constexpr uint32_t SMEM_ALLOC = SH + kQtShBytes + 1024;
   // dS hi and lo: the A operand of dQ += dS K^ in tensor memory (64 columns
   // each, two 16-bit values a column)
@@ -712,8 +712,9 @@ struct QtQLayout {
 // QSF / QSR: S computed / read by the rows; QDF / QDR: dP computed / read;
 // QPF + h / QPE + h: key half h of dS written / consumed.
 enum : int {
-  QQ = 0, QKF = 1 /* 1,2 */, QKE = 3 /* 3,4 */, QVF = 5, QVE = 6, QSF = 7, QSR = 8,
-  QDF = 9, QDR = 10, QPF = 11 /* 11,12 */, QPE = 13 /* 13,14 */, QDONE = 15, QN = 16
+  QQ = 0, QKF = 1 /* 1..3 */, QKE = 4 /* 4..6 */, QVF = 7 /* 7,8 */, QVE = 9 /* 9,10 */,
+  QSF = 11, QSR = 12, QDF = 13, QDR = 14, QPF = 15 /* 15,16 */, QPE = 17 /* 17,18 */,
+  QDONE = 19, QN = 20
 };
 constexpr uint32_t kQ256 = (1u << QSR) | (1u << QDR);
 constexpr uint32_t kQ128 = (1u << QPF) | (1u << (QPF + 1));
@@ -747,22 +748,23 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
       mbar_arrive_expect_tx(&bars[QQ], 2 * L::T);
       bulk_g2s(sm + L::Q, p.qt + qs * L::T, L::T, &bars[QQ]);
       bulk_g2s(sm + L::DO, p.dot + qs * L::T, L::T, &bars[QQ]);
-      int lastk[2] = {-1, -1}, lastv = -1;
+      int lastk[3] = {-1, -1, -1}, lastv[2] = {-1, -1};
       for (int j = 0; j < nt && !*S.abort; ++j) {
-        const int sl = j & 1;
-        if (j >= 2 && !mbar_wait(&bars[QKE + sl], ((j >> 1) - 1) & 1, S.abort)) break;
-        mbar_arrive_expect_tx(&bars[QKF + sl], L::T);
-        bulk_g2s(sm + L::K + sl * L::T, kbase + (int64_t)j * L::T, L::T, &bars[QKF + sl]);
-        lastk[sl] = j;
-        if (j >= 1 && !mbar_wait(&bars[QVE], (j - 1) & 1, S.abort)) break;
-        mbar_arrive_expect_tx(&bars[QVF], L::T);
-        bulk_g2s(sm + L::V, vbase + (int64_t)j * L::T, L::T, &bars[QVF]);
-        lastv = j;
+        const int ks = j % 3, vs = j & 1;
+        if (j >= 3 && !mbar_wait(&bars[QKE + ks], (j / 3 - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[QKF + ks], L::T);
+        bulk_g2s(sm + L::K + ks * L::T, kbase + (int64_t)j * L::T, L::T, &bars[QKF + ks]);
+        lastk[ks] = j;
+        if (j >= 2 && !mbar_wait(&bars[QVE + vs], ((j >> 1) - 1) & 1, S.abort)) break;
+        mbar_arrive_expect_tx(&bars[QVF + vs], L::T);
+        bulk_g2s(sm + L::V + vs * L::T, vbase + (int64_t)j * L::T, L::T, &bars[QVF + vs]);
+        lastv[vs] = j;
       }
       qt_drain(&bars[QQ], 0);
+      for (int sl = 0; sl < 3; ++sl)
+        if (lastk[sl] >= 0) qt_drain(&bars[QKF + sl], (lastk[sl] / 3) & 1);
       for (int sl = 0; sl < 2; ++sl)
-        if (lastk[sl] >= 0) qt_drain(&bars[QKF + sl], (lastk[sl] >> 1) & 1);
-      if (lastv >= 0) qt_drain(&bars[QVF], lastv & 1);
+        if (lastv[sl] >= 0) qt_drain(&bars[QVF + sl], (lastv[sl] >> 1) & 1);
     }
   } else if (warp == kQtMma) {
     if (lane == 0) {
@@ -771,34 +773,35 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
       const uint32_t base = smem_u32(sm);
       // S = Q^ K^T of key tile j once the rows have read S(j - 1)
       auto issue_s = [&](int j) -> bool {
-        const int sl = j & 1;
-        if (!mbar_wait(&bars[QKF + sl], (j >> 1) & 1, S.abort)) return false;
+        const int ks = j % 3;
+        if (!mbar_wait(&bars[QKF + ks], (j / 3) & 1, S.abort)) return false;
         if (j >= 1 && !mbar_wait(&bars[QSR], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + sl * L::T, s),
+          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + ks * L::T, s),
                   idS, s > 0);
         tc_commit(&bars[QSF]);
         return true;
       };
       // dP = dO V^T of key tile j once the rows have read dP(j - 1)
       auto issue_dp = [&](int j) -> bool {
-        if (!mbar_wait(&bars[QVF], j & 1, S.abort)) return false;
+        const int vs = j & 1;
+        if (!mbar_wait(&bars[QVF + vs], (j >> 1) & 1, S.abort)) return false;
         if (j >= 1 && !mbar_wait(&bars[QDR], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
-                  s > 0);
+          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V + vs * L::T, s),
+                  idS, s > 0);
         tc_commit(&bars[QDF]);
-        tc_commit(&bars[QVE]);
+        tc_commit(&bars[QVE + vs]);
         return true;
       };
       bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0) && issue_dp(0);
       for (int j = 0; j < nt && ok; ++j) {
         if (j + 1 < nt && !(issue_s(j + 1) && issue_dp(j + 1))) break;
-        const uint32_t kt = base + L::K + (j & 1) * L::T;
+        const uint32_t kt = base + L::K + (j % 3) * L::T;
         bool fine = true;
 #pragma unroll
         for (int hf = 0; hf < 2 && fine; ++hf) {
@@ -813,7 +816,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
           tc_commit(&bars[QPE + hf]);
         }
         if (!fine) break;
-        tc_commit(&bars[QKE + (j & 1)]);
+        tc_commit(&bars[QKE + j % 3]);
       }
       tc_commit(&bars[QDONE]);
       qt_drain(&bars[QDONE], 0);
