@@ -908,22 +908,23 @@ struct QtKvLayout {
 };
 
 // KQF + s / KQE + s: Q slot s loaded / free (its chunk's dK done); KOF /
-// KOE: the dO chunk loaded / free (its dV done); KSF / KSR: S computed /
-// read by the rows; KDF / KDR: dP computed / read; KPF: P^ and dS written;
-// KPE: the chunk's products done.
+// KOE: the dO chunk and the P^ tile loaded / free (the chunk's dV done);
+// KSF / KSR: S computed / read by the rows; KDF / KDR: dP computed / read;
+// KPPF: P^ written; KDSF: dS written; KPE: the chunk's dK done.
 enum : int {
   KKV = 0, KQF = 1 /* 1,2 */, KQE = 3 /* 3,4 */, KOF = 5, KOE = 6, KSF = 7, KSR = 8, KDF = 9,
-  KDR = 10, KPF = 11, KPE = 12, KDONE = 13, KN = 14
+  KDR = 10, KPPF = 11, KDSF = 12, KPE = 13, KDONE = 14, KN = 15
 };
-constexpr uint32_t kKv256 = (1u << KSR) | (1u << KDR) | (1u << KPF);
+constexpr uint32_t kKv256 = (1u << KSR) | (1u << KDR) | (1u << KPPF) | (1u << KDSF);
 
 // grid (ceil(maxlen / 128) * Hkv, nseq), kQtThreads threads: key tile
 // blockIdx.x / Hkv (causal grids: the tiles with the most queries first).
 // Iteration it takes query chunk c0 + it % nch of query head
 // hk * grp + it / nch.  The rows read S(it) into registers first, so S of
-// the next chunk (its Q in the second slot) runs while they work; the
-// products of a chunk run dV (P^T dO) before dK (dS^T Q^), so the next dO
-// chunk loads during dK.
+// the next chunk (its Q in the second slot) runs while they work; they form
+// P and P^ from S alone and publish P^, so dV (P^T dO) runs while they wait
+// for dP and form dS; dK (dS^T Q^) follows, and the next dO chunk loads from
+// the end of dV on.
 template <int DT, int D, int BLK>
 __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatParams p) {
   using L = QtKvLayout<D>;
@@ -998,15 +999,17 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
         tc_commit(&bars[KDF]);
         // the next chunk's scores while the rows work on this one
         if (it + 1 < n_it && !issue_s(it + 1)) break;
-        if (!mbar_wait(&bars[KPF], it & 1, S.abort)) break;
-        tc_fence_after();
         // dV += P^T dO, dK += dS^T Q^: M = the 128 keys, K = the 128 queries
+        if (!mbar_wait(&bars[KPPF], it & 1, S.abort)) break;
+        tc_fence_after();
         const uint32_t qt = base + L::Q + (it & 1) * L::T;
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
                   it > 0 || s > 0);
         tc_commit(&bars[KOE]);
+        if (!mbar_wait(&bars[KDSF], it & 1, S.abort)) break;
+        tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), qt_desc_mn(qt, s), idG,
@@ -1064,8 +1067,35 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       const float cm = cm_raw == -INFINITY ? 0.0f : ex2_ftz(fmaf(cm_raw, c2, nlse2));
       const float inv = cm > 0.0f ? __fdiv_rn(kTensorScaleDiv, cm) : 0.0f;
       const float sig = __fdiv_rn(cm, kTensorScaleDiv);
+      // P (kept in place of S) and P^, written once dV of the previous chunk
+      // has read the P^ tile
+      if (it >= 1 && !warp_wait(&bars[KOE], (it - 1) & 1, S.abort)) { ok = false; break; }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = cb + 32 * cc;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float x[16];
+          float am = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float pr = ex2_ftz(fmaf(a[cc][16 * b + i], c2, nlse2));
+            a[cc][16 * b + i] = pr;
+            x[i] = pr * inv;
+            am = fmaxf(am, x[i]);
+          }
+          const PBlock pb(am, S.rcp, true);
+          uint32_t wq[8];
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) wq[i / 2] = pb.scaled<DT>(x[i], x[i + 1], sig);
+          qt_store16(tP, r, col + 16 * b, wq);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[KPPF]);
+      // dS = P o (dP g_V - D), written once dK of the previous chunk has read
+      // the dS tile
       if (!warp_wait(&bars[KDF], it & 1, S.abort)) { ok = false; break; }
-      // the tiles are free once the products of the previous chunk are done
       if (it >= 1 && !warp_wait(&bars[KPE], (it - 1) & 1, S.abort)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
@@ -1080,29 +1110,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
         }
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          float pr[16], x[16];
-          float am = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            pr[i] = ex2_ftz(fmaf(a[cc][16 * b + i], c2, nlse2));
-            x[i] = pr[i] * inv;
-            am = fmaxf(am, x[i]);
-          }
-          const PBlock pb(am, S.rcp, true);
-          uint32_t wq[8], wd[8];
+          uint32_t wd[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            wq[i / 2] = pb.scaled<DT>(x[i], x[i + 1], sig);
             const int e = 16 * b + i;
-            wd[i / 2] = pack2<DT>(pr[i] * fmaf(dp[e], gv, -dsum),
-                                  pr[i + 1] * fmaf(dp[e + 1], gv, -dsum));
+            wd[i / 2] = pack2<DT>(a[cc][e] * fmaf(dp[e], gv, -dsum),
+                                  a[cc][e + 1] * fmaf(dp[e + 1], gv, -dsum));
           }
-          qt_store16(tP, r, col + 16 * b, wq);
           qt_store16(tD, r, col + 16 * b, wd);
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars[KPF]);
+      mbar_arrive(&bars[KDSF]);
     }
     // epilogue: lane r of the dV and dK accumulators is key j0 + r
     if (ok && warp_wait(&bars[KDONE], 0, S.abort)) {
