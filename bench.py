@@ -382,7 +382,7 @@ def quantizer_line(dev, peaks, with_oracle=True):
         del g
     res["workload"] = synth.QUANT.name
     res["algorithmic_bytes"] = algo
-    res["kernels_per_call"] = 1
+    res["kernels_per_call"] = {"scale_given": 1, "scale_computed": 2}
     res["timing"] = "CUDA graph of 120 calls, 12 rotating inputs (201 MB > L2)"
     if with_oracle:
         import oracle
