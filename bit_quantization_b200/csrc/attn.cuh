@@ -369,13 +369,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     }
   } else if (warp == kMmaWarp || warp == kPvWarp) {
     // ---------------------------------------------------- MMA issuers --
-    // One elected lane issues QK^T for every tile in order (warp kMmaWarp),
-    // another PV (warp kPvWarp), so scores for the next tiles never queue
-    // behind a PV that waits for its P tile or for the correction step.
-    // QK^T(t) reads the K half of its stage before PV(t) is issued (PV(t)
-    // follows P(t), which follows the scores of tile t), so the PV side's
-    // commit alone frees the stage.
-    if (lane == 0) {
+    // One warp issues QK^T for every tile in order (warp kMmaWarp), another
+    // PV (warp kPvWarp), so scores for the next tiles never queue behind a PV
+    // that waits for its P tile or for the correction step.  The whole warp
+    // runs the loop and its waits, so the operand descriptors are uniform
+    // across it; one elected lane issues the tensor instructions and their
+    // commits.  QK^T(t) reads the K half of its stage before PV(t) is issued
+    // (PV(t) follows P(t), which follows the scores of tile t), so the PV
+    // side's commit alone frees the stage.
+    {
       constexpr uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
       constexpr uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
       constexpr uint32_t swz_d = swz_mode_for_pitch(D / 2), swz_b = swz_mode_for_pitch(BLK / 2);
@@ -418,27 +420,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             pin64(cpk[s]);
             pin64(db[s]);
           }
-          if (!mbar_wait(full, par, s_abort)) { ok = false; break; }
+          if (!warp_wait(full, par, s_abort)) { ok = false; break; }
           if (!f16 && !q4_ready) {
-            if (!mbar_wait(&bars[B_Q4], 0, s_abort)) { ok = false; break; }
+            if (!warp_wait(&bars[B_Q4], 0, s_abort)) { ok = false; break; }
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-            for (int s = 0; s < D / 64; ++s)
-              tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
-                               d_sf + ((L::OFF4_Q + 128 * (D / 2) + 512 * s) >> 4));
+              for (int s = 0; s < D / 64; ++s)
+                tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
+                                 d_sf + ((L::OFF4_Q + 128 * (D / 2) + 512 * s) >> 4));
+            }
+            __syncwarp();
             q4_ready = true;
           }
           if (f16 && !q16_ready) {
-            if (!mbar_wait(&bars[B_Q16], 0, s_abort)) { ok = false; break; }
+            if (!warp_wait(&bars[B_Q16], 0, s_abort)) { ok = false; break; }
             q16_ready = true;
           }
           // the S buffer of tile t-2 has been read
-          if (t >= 2 && !mbar_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) {
+          if (t >= 2 && !warp_wait(&bars[B_SE + st], ((t >> 1) - 1) & 1, s_abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (!f16) {
+          if (elect_one()) {
+            if (!f16) {
 #pragma unroll
             for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
 #pragma unroll
@@ -450,8 +456,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             for (int s = 0; s < D / 16; ++s)
               mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
                       d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
+            }
+            tc_commit(&bars[B_SF + st]);
           }
-          tc_commit(&bars[B_SF + st]);
+          __syncwarp();
           advance(t);
         }
       } else {
@@ -483,10 +491,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             pin64(da[s]);
             pin64(db[s]);
           }
-          if (!mbar_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
-          if (!mbar_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
+          if (!warp_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
+          if (!warp_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
           tc_fence_after();
-          if (!f16) {
+          if (elect_one()) {
+            if (!f16) {
 #pragma unroll
             for (int s = 0; s < BLK / 64; ++s) {
               tc_cp_32x128b_x4(psf + 4 * s, cpp[s]);
@@ -501,14 +510,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
               mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
                       d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
                       t > 0 || s > 0);
+            }
+            tc_commit(&bars[B_OD + st]);
+            tc_commit(empty);
           }
-          tc_commit(&bars[B_OD + st]);
-          tc_commit(empty);
+          __syncwarp();
           advance(t);
         }
       }
       // every MMA of both issuers has completed before the CTA ends
-      tc_commit(&bars[B_DONE]);
+      if (elect_one()) tc_commit(&bars[B_DONE]);
+      __syncwarp();
       int dummy = 0;
       volatile int* never = &dummy;
       mbar_wait(&bars[B_DONE], 0, never, 200000000ull);

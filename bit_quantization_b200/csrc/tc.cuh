@@ -102,6 +102,16 @@ __device__ __forceinline__ bool spin_until_geq(const unsigned* word, unsigned ta
 // lets the next kernel of the stream that was launched with that attribute
 // be scheduled before this grid completes (it then waits in its own
 // pdl_wait for what it must not overtake).
+// Elects one lane of the converged warp (elect.sync over all 32 lanes):
+// true in that lane only, the same lane for every call of a converged warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
