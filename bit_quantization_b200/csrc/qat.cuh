@@ -509,44 +509,56 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_fwd_kernel(const QatParams 
         if (last[sl] >= 0) qt_drain(&bars[RF + sl], (last[sl] / kQtRing) & 1);
     }
   } else if (warp == kQtMma) {
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop and waits (uniform operand
+    // descriptors); the elected lane issues every MMA and commit.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idPV = idesc_f16(DT, 128, D) | kIdescBmn;
       const uint32_t base = smem_u32(sm);
       auto issue_s = [&](int j) -> bool {
         const int i = qt_ring_k(j), rs = i % kQtRing;
-        if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) return false;
+        if (!warp_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) return false;
         // the rows have read the previous scores
-        if (j >= 1 && !mbar_wait(&bars[FSE], (j - 1) & 1, S.abort)) return false;
+        if (j >= 1 && !warp_wait(&bars[FSE], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s),
-                  qt_desc_k(base + L::RING + rs * L::T, s), idS, s > 0);
-        tc_commit(&bars[FSF]);
-        tc_commit(&bars[RE + rs]);
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s),
+                    qt_desc_k(base + L::RING + rs * L::T, s), idS, s > 0);
+          tc_commit(&bars[FSF]);
+          tc_commit(&bars[RE + rs]);
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait(&bars[FQ], 0, S.abort) && issue_s(0);
+      bool ok = warp_wait(&bars[FQ], 0, S.abort) && issue_s(0);
       for (int j = 0; j < nt && ok; ++j) {
         // the next tile's scores go ahead of this tile's products
         if (j + 1 < nt && !issue_s(j + 1)) break;
         const int i = qt_ring_v(j, nt), rs = i % kQtRing;
-        if (!mbar_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) break;
-        if (!mbar_wait(&bars[FPF], j & 1, S.abort)) break;
+        if (!warp_wait(&bars[RF + rs], (i / kQtRing) & 1, S.abort)) break;
+        if (!warp_wait(&bars[FPF], j & 1, S.abort)) break;
         tc_fence_after();
         const uint32_t vt = base + L::RING + rs * L::T;
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint64_t bv = qt_desc_mn(vt, s);
-          mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
-          mma_f16_ta(tmem + L::T_OH, tmem + L::T_PH + 8 * s, bv, idPV, j > 0 || s > 0);
-          mma_f16_ta(tmem + L::T_OH, tmem + L::T_PL + 8 * s, bv, idPV, 1);
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t bv = qt_desc_mn(vt, s);
+            mma_f16(tmem + L::T_O, qt_desc_k(base + L::P, s), bv, idPV, j > 0 || s > 0);
+            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PH + 8 * s, bv, idPV, j > 0 || s > 0);
+            mma_f16_ta(tmem + L::T_OH, tmem + L::T_PL + 8 * s, bv, idPV, 1);
+          }
+          tc_commit(&bars[FPE]);
+          tc_commit(&bars[RE + rs]);
         }
-        tc_commit(&bars[FPE]);
-        tc_commit(&bars[RE + rs]);
+        __syncwarp();
       }
-      tc_commit(&bars[FDONE]);
+      if (leader) {
+        tc_commit(&bars[FDONE]);
+      }
+      __syncwarp();
       qt_drain(&bars[FDONE], 0);
     }
   } else {
@@ -767,58 +779,76 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_q_kernel(const QatParam
         if (lastv[sl] >= 0) qt_drain(&bars[QVF + sl], (lastv[sl] >> 1) & 1);
     }
   } else if (warp == kQtMma) {
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop and waits (uniform operand
+    // descriptors); the elected lane issues every MMA and commit.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idDQ = idesc_f16(DT, 128, D) | kIdescBmn;
       const uint32_t base = smem_u32(sm);
       // S = Q^ K^T of key tile j once the rows have read S(j - 1)
       auto issue_s = [&](int j) -> bool {
         const int ks = j % 3;
-        if (!mbar_wait(&bars[QKF + ks], (j / 3) & 1, S.abort)) return false;
-        if (j >= 1 && !mbar_wait(&bars[QSR], (j - 1) & 1, S.abort)) return false;
+        if (!warp_wait(&bars[QKF + ks], (j / 3) & 1, S.abort)) return false;
+        if (j >= 1 && !warp_wait(&bars[QSR], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + ks * L::T, s),
-                  idS, s > 0);
-        tc_commit(&bars[QSF]);
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q, s), qt_desc_k(base + L::K + ks * L::T, s),
+                    idS, s > 0);
+          tc_commit(&bars[QSF]);
+        }
+        __syncwarp();
         return true;
       };
       // dP = dO V^T of key tile j once the rows have read dP(j - 1)
       auto issue_dp = [&](int j) -> bool {
         const int vs = j & 1;
-        if (!mbar_wait(&bars[QVF + vs], (j >> 1) & 1, S.abort)) return false;
-        if (j >= 1 && !mbar_wait(&bars[QDR], (j - 1) & 1, S.abort)) return false;
+        if (!warp_wait(&bars[QVF + vs], (j >> 1) & 1, S.abort)) return false;
+        if (j >= 1 && !warp_wait(&bars[QDR], (j - 1) & 1, S.abort)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V + vs * L::T, s),
-                  idS, s > 0);
-        tc_commit(&bars[QDF]);
-        tc_commit(&bars[QVE + vs]);
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V + vs * L::T, s),
+                    idS, s > 0);
+          tc_commit(&bars[QDF]);
+          tc_commit(&bars[QVE + vs]);
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait(&bars[QQ], 0, S.abort) && issue_s(0) && issue_dp(0);
+      bool ok = warp_wait(&bars[QQ], 0, S.abort) && issue_s(0) && issue_dp(0);
       for (int j = 0; j < nt && ok; ++j) {
         if (j + 1 < nt && !(issue_s(j + 1) && issue_dp(j + 1))) break;
         const uint32_t kt = base + L::K + (j % 3) * L::T;
         bool fine = true;
 #pragma unroll
         for (int hf = 0; hf < 2 && fine; ++hf) {
-          if (!mbar_wait(&bars[QPF + hf], j & 1, S.abort)) { fine = false; break; }
+          if (!warp_wait(&bars[QPF + hf], j & 1, S.abort)) { fine = false; break; }
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int s = 4 * hf; s < 4 * hf + 4; ++s) {
-            const uint64_t bk = qt_desc_mn(kt, s);
-            mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSH + 8 * s, bk, idDQ, j > 0 || s > 0);
-            mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSL + 8 * s, bk, idDQ, 1);
+            for (int s = 4 * hf; s < 4 * hf + 4; ++s) {
+              const uint64_t bk = qt_desc_mn(kt, s);
+              mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSH + 8 * s, bk, idDQ, j > 0 || s > 0);
+              mma_f16_ta(tmem + L::T_DQ, tmem + L::T_DSL + 8 * s, bk, idDQ, 1);
+            }
+            tc_commit(&bars[QPE + hf]);
           }
-          tc_commit(&bars[QPE + hf]);
+          __syncwarp();
         }
         if (!fine) break;
-        tc_commit(&bars[QKE + j % 3]);
+        if (leader) {
+          tc_commit(&bars[QKE + j % 3]);
+        }
+        __syncwarp();
       }
-      tc_commit(&bars[QDONE]);
+      if (leader) {
+        tc_commit(&bars[QDONE]);
+      }
+      __syncwarp();
       qt_drain(&bars[QDONE], 0);
     }
   } else {
@@ -969,55 +999,73 @@ __global__ void __launch_bounds__(kQtThreads, 1) qat_bwd_kv_kernel(const QatPara
       if (lasto >= 0) qt_drain(&bars[KOF], lasto & 1);
     }
   } else if (warp == kQtMma) {
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop and waits (uniform operand
+    // descriptors); the elected lane issues every MMA and commit.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_f16(DT, 128, 128);
       constexpr uint32_t idG = idesc_f16(DT, 128, D) | kIdescAmn | kIdescBmn;
       const uint32_t base = smem_u32(sm);
       // S(it) = Q^ K^T into the S columns (the rows have read S(it - 1))
       auto issue_s = [&](int it) -> bool {
         const int sl = it & 1;
-        if (!mbar_wait(&bars[KQF + sl], (it >> 1) & 1, S.abort)) return false;
-        if (it >= 1 && !mbar_wait(&bars[KSR], (it - 1) & 1, S.abort)) return false;
+        if (!warp_wait(&bars[KQF + sl], (it >> 1) & 1, S.abort)) return false;
+        if (it >= 1 && !warp_wait(&bars[KSR], (it - 1) & 1, S.abort)) return false;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q + sl * L::T, s),
-                  qt_desc_k(base + L::K, s), idS, s > 0);
-        tc_commit(&bars[KSF]);
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(tmem + L::T_S, qt_desc_k(base + L::Q + sl * L::T, s),
+                    qt_desc_k(base + L::K, s), idS, s > 0);
+          tc_commit(&bars[KSF]);
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait(&bars[KKV], 0, S.abort) && issue_s(0);
+      bool ok = warp_wait(&bars[KKV], 0, S.abort) && issue_s(0);
       for (int it = 0; it < n_it && ok; ++it) {
         // dP(it) = dO V^T (the rows have read dP(it - 1))
-        if (!mbar_wait(&bars[KOF], it & 1, S.abort)) break;
-        if (it >= 1 && !mbar_wait(&bars[KDR], (it - 1) & 1, S.abort)) break;
+        if (!warp_wait(&bars[KOF], it & 1, S.abort)) break;
+        if (it >= 1 && !warp_wait(&bars[KDR], (it - 1) & 1, S.abort)) break;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
-                  s > 0);
-        tc_commit(&bars[KDF]);
+          for (int s = 0; s < D / 16; ++s)
+            mma_f16(tmem + L::T_DP, qt_desc_k(base + L::DO, s), qt_desc_k(base + L::V, s), idS,
+                    s > 0);
+          tc_commit(&bars[KDF]);
+        }
+        __syncwarp();
         // the next chunk's scores while the rows work on this one
         if (it + 1 < n_it && !issue_s(it + 1)) break;
         // dV += P^T dO, dK += dS^T Q^: M = the 128 keys, K = the 128 queries
-        if (!mbar_wait(&bars[KPPF], it & 1, S.abort)) break;
+        if (!warp_wait(&bars[KPPF], it & 1, S.abort)) break;
         tc_fence_after();
         const uint32_t qt = base + L::Q + (it & 1) * L::T;
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
-                  it > 0 || s > 0);
-        tc_commit(&bars[KOE]);
-        if (!mbar_wait(&bars[KDSF], it & 1, S.abort)) break;
+          for (int s = 0; s < 8; ++s)
+            mma_f16(tmem + L::T_DV, qt_desc_mn(base + L::P, s), qt_desc_mn(base + L::DO, s), idG,
+                    it > 0 || s > 0);
+          tc_commit(&bars[KOE]);
+        }
+        __syncwarp();
+        if (!warp_wait(&bars[KDSF], it & 1, S.abort)) break;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), qt_desc_mn(qt, s), idG,
-                  it > 0 || s > 0);
-        tc_commit(&bars[KQE + (it & 1)]);
-        tc_commit(&bars[KPE]);
+          for (int s = 0; s < 8; ++s)
+            mma_f16(tmem + L::T_DK, qt_desc_mn(base + L::DS, s), qt_desc_mn(qt, s), idG,
+                    it > 0 || s > 0);
+          tc_commit(&bars[KQE + (it & 1)]);
+          tc_commit(&bars[KPE]);
+        }
+        __syncwarp();
       }
-      tc_commit(&bars[KDONE]);
+      if (leader) {
+        tc_commit(&bars[KDONE]);
+      }
+      __syncwarp();
       qt_drain(&bars[KDONE], 0);
     }
   } else {
