@@ -21,8 +21,10 @@
 //               memory) between PV(t-1) and PV(t), then divides by the row
 //               sum and writes the output and LSE;
 //   warp 20     producer: bulk copies of the pre-quantised tile images;
-//   warp 21     tensor-memory owner and QK^T issuer (one elected lane);
-//   warp 22     PV issuer (one elected lane).
+//   warp 21     tensor-memory owner and QK^T issuer;
+//   warp 22     PV issuer (each issuer warp runs its loop and waits with
+//               all lanes, one elected lane issuing the tensor
+//               instructions and commits).
 // The MMA accumulates every PV straight into O, so the softmax warps never
 // wait on a PV product.
 // Tensor memory (512 columns): S double buffer [2][BLK], O [D], then the

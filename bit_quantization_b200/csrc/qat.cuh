@@ -54,8 +54,9 @@
 // The three attention kernels have ten warps: warps 0-7 own the rows (two
 // per tensor-memory lane quarter, each taking half of the 128 columns of
 // a score tile), warp 8 moves tiles with bulk copies, warp 9 issues the MMAs
-// from one thread.  Every wait is bounded.  Where the A operand of a product
-// has the query rows on its M side (P of O' in the forward, dS of dQ), the
+// (the whole warp runs the loop and its waits, one elected lane issues).
+// Every wait is bounded.  Where the A operand of a product has the query
+// rows on its M side (P of O' in the forward, dS of dQ), the
 // rows write it to tensor memory and the MMA reads it from there: no
 // shared-memory round trip.
 #pragma once
