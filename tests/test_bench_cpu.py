@@ -52,3 +52,31 @@ def test_recorded_traffic_only_for_its_workload():
     t = b.qat_traffic(synth.C_QAT4K)
     # either the source is the one the counters were taken on, or nothing
     assert t is None or t == b.QAT_TRAFFIC["bytes"]
+
+
+def test_tensor_roofline_splits_the_ideal_time_by_precision():
+    b = _bench()
+    peaks = {"bf16_tflops": 1000.0}
+    # pure NVFP4: the ideal is F / (4 x the bf16 rate)
+    r = b.tensor_roofline(4e12, 0.0, 2.0, peaks, "measured")
+    assert abs(r["achieved"] - 2000.0) < 1e-9
+    assert abs(r["peak"] - 4000.0) < 1e-9
+    assert abs(r["frac"] - 0.5) < 1e-12
+    # mixed: t_ideal = 3e12 / 4e15 + 1e12 / 1e15 = 1.75 ms; the kernel took 3.5 ms
+    r = b.tensor_roofline(3e12, 1e12, 3.5, peaks, "measured")
+    assert abs(r["frac"] - 0.5) < 1e-12
+    assert abs(r["peak"] - 4e12 / 1.75e-3 / 1e12) < 1e-9
+    # the fraction against the nominal dense peaks uses their own ideal time
+    t_nom = 3e12 / (b.NOMINAL_FP4_TFLOPS * 1e12) + 1e12 / (b.NOMINAL_BF16_TFLOPS * 1e12)
+    assert abs(r["frac_of_nominal"] - t_nom / 3.5e-3) < 1e-12
+
+
+def test_alu_roofline_counts_score_elements():
+    b = _bench()
+    d, n_sm, mhz = 128, 148, 2000.0
+    flops = 4 * d * 1e9  # 1e9 score elements
+    r = b.alu_roofline(flops, d, 1.0, mhz, n_sm)
+    assert abs(r["achieved"] - 1000.0) < 1e-9  # Gelem/s
+    peak = b.XU_OPS_PER_CLK_PER_SM * n_sm * mhz * 1e6 / b.XU_OPS_PER_ELEMENT / 1e9
+    assert abs(r["peak"] - peak) < 1e-9
+    assert abs(r["tflops_equivalent_peak"] - peak * 1e9 * 4 * d / 1e12) < 1e-6
