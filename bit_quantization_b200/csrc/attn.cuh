@@ -448,16 +448,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           if (elect_one()) {
             if (!f16) {
 #pragma unroll
-            for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
+              for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
 #pragma unroll
-            for (int s = 0; s < D / 64; ++s)
-              mma_nvf4(dS, d_q4 + 2 * s, db[s], id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s,
-                       s > 0);
-          } else {
+              for (int s = 0; s < D / 64; ++s)
+                mma_nvf4(dS, d_q4 + 2 * s, db[s], id_qk4, tmem + L::T_QSF + 4 * s, ksf + 4 * s,
+                         s > 0);
+            } else {
 #pragma unroll
-            for (int s = 0; s < D / 16; ++s)
-              mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
-                      d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
+              for (int s = 0; s < D / 16; ++s)
+                mma_f16(dS, d_q16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                        d_k16 + so + ((s / 4) * BLK * 128 >> 4) + 2 * (s % 4), id_qk16, s > 0);
             }
             tc_commit(&bars[B_SF + st]);
           }
@@ -499,19 +499,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           if (elect_one()) {
             if (!f16) {
 #pragma unroll
-            for (int s = 0; s < BLK / 64; ++s) {
-              tc_cp_32x128b_x4(psf + 4 * s, cpp[s]);
-              tc_cp_32x128b_x4(vsf + 4 * s, cpv[s]);
-            }
+              for (int s = 0; s < BLK / 64; ++s) {
+                tc_cp_32x128b_x4(psf + 4 * s, cpp[s]);
+                tc_cp_32x128b_x4(vsf + 4 * s, cpv[s]);
+              }
 #pragma unroll
-            for (int s = 0; s < BLK / 64; ++s)
-              mma_nvf4(dO, da[s], db[s], id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
-          } else {
+              for (int s = 0; s < BLK / 64; ++s)
+                mma_nvf4(dO, da[s], db[s], id_pv4, psf + 4 * s, vsf + 4 * s, t > 0 || s > 0);
+            } else {
 #pragma unroll
-            for (int s = 0; s < BLK / 16; ++s)
-              mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
-                      d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
-                      t > 0 || s > 0);
+              for (int s = 0; s < BLK / 16; ++s)
+                mma_f16(dO, d_p16 + ((s / 4) * 128 * 128 >> 4) + 2 * (s % 4),
+                        d_v16 + so + ((s / 4) * D * 128 >> 4) + 2 * (s % 4), id_pv16,
+                        t > 0 || s > 0);
             }
             tc_commit(&bars[B_OD + st]);
             tc_commit(empty);
