@@ -378,8 +378,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
     // across it; one elected lane issues the tensor instructions and their
     // commits.  QK^T(t) reads the K half of its stage before PV(t) is issued
     // (PV(t) follows P(t), which follows the scores of tile t), so the PV
-    // side's commit alone frees the stage.
+    // side's commit alone frees the stage.  The lane is elected once, so
+    // every tensor instruction of the warp and the commits that track them
+    // come from the same thread.
     {
+      const bool leader = elect_one();
       constexpr uint32_t id_qk4 = idesc_nvf4(128, BLK), id_pv4 = idesc_nvf4(128, D);
       constexpr uint32_t id_qk16 = idesc_f16(DT, 128, BLK), id_pv16 = idesc_f16(DT, 128, D);
       constexpr uint32_t swz_d = swz_mode_for_pitch(D / 2), swz_b = swz_mode_for_pitch(BLK / 2);
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           if (!f16 && !q4_ready) {
             if (!warp_wait(&bars[B_Q4], 0, s_abort)) { ok = false; break; }
             tc_fence_after();
-            if (elect_one()) {
+            if (leader) {
 #pragma unroll
               for (int s = 0; s < D / 64; ++s)
                 tc_cp_32x128b_x4(tmem + L::T_QSF + 4 * s,
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
             break;
           }
           tc_fence_after();
-          if (elect_one()) {
+          if (leader) {
             if (!f16) {
 #pragma unroll
               for (int s = 0; s < D / 64; ++s) tc_cp_32x128b_x4(ksf + 4 * s, cpk[s]);
@@ -496,7 +499,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
           if (!warp_wait(&bars[B_PF + st], (t >> 1) & 1, s_abort)) { ok = false; break; }
           if (!warp_wait(&bars[B_CF], t & 1, s_abort)) { ok = false; break; }  // O rescaled
           tc_fence_after();
-          if (elect_one()) {
+          if (leader) {
             if (!f16) {
 #pragma unroll
               for (int s = 0; s < BLK / 64; ++s) {
@@ -521,7 +524,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const AttnPar
         }
       }
       // every MMA of both issuers has completed before the CTA ends
-      if (elect_one()) tc_commit(&bars[B_DONE]);
+      if (leader) tc_commit(&bars[B_DONE]);
       __syncwarp();
       int dummy = 0;
       volatile int* never = &dummy;

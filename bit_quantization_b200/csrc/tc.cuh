@@ -103,7 +103,9 @@ __device__ __forceinline__ bool spin_until_geq(const unsigned* word, unsigned ta
 // be scheduled before this grid completes (it then waits in its own
 // pdl_wait for what it must not overtake).
 // Elects one lane of the converged warp (elect.sync over all 32 lanes):
-// true in that lane only, the same lane for every call of a converged warp.
+// true in that lane only.  Callers elect once and keep the result, so that
+// the tensor instructions of a warp and the commits tracking them come from
+// one thread.
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;
   asm volatile(
