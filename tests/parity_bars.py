@@ -1,7 +1,7 @@
 """The attention parity bar shared by the GPU tests (prefill and decode).
 
-Bar (the benchmark spec: max-abs 1e-2, cosine >= 0.9999 against the oracle's
-emulation of the same quantisation and tiling), element by element against
+Bar (max-abs 1e-2 and cosine >= 0.9999 against the oracle's emulation of
+the same quantisation and tiling), element by element against
 the oracle's fp64 result before its final rounding:
 
     |got - want| <= 1e-2 + half an ulp of the 16-bit output type at want
