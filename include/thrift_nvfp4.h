@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
   THRIFT_OK = 0,
   THRIFT_ERR_ARG = -1,          /* bad pointer, size or flag */
-  THRIFT_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle */
+  THRIFT_ERR_UNSUPPORTED = -2,  /* valid request the library does not handle */
   THRIFT_ERR_CUDA = -3,         /* a CUDA runtime call failed */
   THRIFT_ERR_TIMEOUT = -4,      /* a device-side wait gave up */
   THRIFT_ERR_SCRATCH = -5       /* problem too large for a fixed scratch area */
